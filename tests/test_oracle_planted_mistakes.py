@@ -1,0 +1,105 @@
+"""Each test plants one plausible mistake in the oracle (on the CPU, through
+monkeypatch) and checks that one of the pins catches it. This guards the
+pins themselves: a pin that passes on a broken oracle would pin nothing."""
+import numpy as np
+import pytest
+
+import oracle.eaas as eaas
+import oracle.layer as layer_mod
+import oracle.sh as sh_mod
+import test_oracle_eaas_layer as T
+import test_oracle_sh_cg_wigner as S
+
+
+def _fails(fn, *a):
+    with pytest.raises(AssertionError):
+        fn(*a)
+
+
+def test_z_axis_layer_message_is_so2_map_of_gated_neighbour():
+    # Two atoms on the z axis: node 0's only neighbour sits at +z, so the
+    # edge frame is the identity and out_0 = SO2_W(g_v * x_1) exactly.
+    rng = np.random.default_rng(21)
+    L, C, H = 3, 2, 2
+    pos = np.array([[0, 0, 0], [0, 0, 1.7]], np.float32)
+    x = rng.normal(size=(2, (L + 1) ** 2, C))
+    flat = T._rand_so2(rng, L, C)
+    Wrad = rng.normal(size=(16, (L + 1) * C + H))
+    lay = layer_mod.DenseLayer(L, C, H, 16, 3.0, np.eye(C), np.eye(C), Wrad, flat)
+    rp = np.array([0, 1, 2], np.int32)
+    col = np.array([1, 0], np.int32)
+    out = lay(pos, None, rp, col, x)
+    g = layer_mod.radial_basis(np.array([float(np.float32(1.7))]), 3.0, 16) @ Wrad
+    lk = np.concatenate([np.full(2 * l + 1, l) for l in range(L + 1)])
+    h = g[0, :(L + 1) * C].reshape(L + 1, C)[lk] * x[1]
+    A, B = eaas.unpack_so2(flat, L, C)
+    from so2_form import so2_apply
+    np.testing.assert_allclose(out[0], so2_apply(h, A, B, L, C), atol=1e-12)
+
+
+def test_catches_transposed_channel_weight(monkeypatch):
+    orig = layer_mod.dense_messages
+
+    def bad(h, Y, w):
+        return orig(h, Y, {p: W.T for p, W in w.items()})
+    monkeypatch.setattr(layer_mod, "dense_messages", bad)
+    monkeypatch.setattr(T, "dense_messages", bad)
+    _fails(T.test_eq13_so2_form_equals_dense_cg_contraction, 2, 4)
+
+
+def test_catches_sign_error_in_odd_parity_block(monkeypatch):
+    orig = eaas._systems
+
+    def bad(l1, l3):
+        e, o, Me, Mo = orig(l1, l3)
+        return e, o, Me, -Mo
+    monkeypatch.setattr(eaas, "_systems", bad)
+    _fails(T.test_eq13_so2_form_equals_dense_cg_contraction, 2, 4)
+
+
+def test_catches_dropped_path(monkeypatch):
+    orig = layer_mod.dense_messages
+
+    def bad(h, Y, w):
+        return orig(h, Y, {p: W for p, W in w.items() if p != (2, 1, 1)})
+    monkeypatch.setattr(T, "dense_messages", bad)
+    _fails(T.test_eq13_so2_form_equals_dense_cg_contraction, 2, 4)
+
+
+def test_catches_wrong_sign_convention_of_sine_harmonics(monkeypatch):
+    orig = sh_mod.real_sh
+
+    def bad(lmax, vec):
+        Y = orig(lmax, vec).copy()
+        for l in range(1, lmax + 1):
+            Y[..., l * l:l * l + l] *= -1
+        return Y
+    monkeypatch.setattr(S, "real_sh", bad)
+    _fails(S.test_sh_textbook_closed_forms_l_le_2)
+
+
+def test_catches_reversed_edge_direction(monkeypatch):
+    orig = layer_mod.edge_vectors
+    monkeypatch.setattr(layer_mod, "edge_vectors", lambda pos, box, i, j: -orig(pos, box, i, j))
+    _fails(test_z_axis_layer_message_is_so2_map_of_gated_neighbour)
+
+
+def test_catches_scrambled_output_index(monkeypatch):
+    orig = layer_mod.DenseLayer.edge_terms
+
+    def bad(self, pos, box, x, i, j):
+        g_a, v = orig(self, pos, box, x, i, j)
+        return g_a, v[:, ::-1, :].copy()
+    monkeypatch.setattr(layer_mod.DenseLayer, "edge_terms", bad)
+    _fails(test_z_axis_layer_message_is_so2_map_of_gated_neighbour)
+
+
+def test_catches_swapped_query_and_key(monkeypatch):
+    orig_init = layer_mod.DenseLayer.__init__
+
+    def bad(self, *a, **k):
+        orig_init(self, *a, **k)
+        self.Wq, self.Wk = self.Wk.copy(), self.Wq.copy()
+    monkeypatch.setattr(layer_mod.DenseLayer, "__init__", bad)
+    monkeypatch.setattr(T, "DenseLayer", layer_mod.DenseLayer)
+    _fails(T.test_layer_L0_reduces_to_scalar_graph_attention)
