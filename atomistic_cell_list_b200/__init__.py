@@ -1,0 +1,198 @@
+"""Python binding of libe2f.so: a GPU cell-list neighbour build and the
+on-the-fly equivariant attention forward of E2Former-V2, written for B200
+(sm_100a).
+
+This module only marshals arguments: every step of the computation runs in
+the library's CUDA kernels. PyTorch supplies device memory and the current
+stream. Functions carry the C entry points' names (see include/e2f.h); the
+library must be built (``python -m atomistic_cell_list_b200.build``) and a
+CUDA device must be present, otherwise the calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libe2f.so")
+HEADER = os.path.join(os.path.dirname(_HERE), "include", "e2f.h")
+
+E2F_OK = 0
+STATUS_NAMES = {0: "E2F_OK", 1: "E2F_ERR_INVALID_ARG", 2: "E2F_ERR_UNSUPPORTED", 3: "E2F_ERR_CAPACITY",
+                4: "E2F_ERR_ALIGNMENT", 5: "E2F_ERR_TIMEOUT", 6: "E2F_ERR_CUDA", 7: "E2F_ERR_NONFINITE"}
+E2F_F32, E2F_BF16 = 0, 1
+
+
+class E2FError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {STATUS_NAMES.get(code, code)} ({status_string(code)})")
+
+
+class e2f_attn_cfg(ctypes.Structure):
+    _fields_ = [("L", ctypes.c_int), ("C", ctypes.c_int), ("H", ctypes.c_int), ("n_rbf", ctypes.c_int),
+                ("cutoff", ctypes.c_float), ("feat_dtype", ctypes.c_int)]
+
+
+_lib = None
+_vp, _i64, _sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t
+
+_SIGS = {
+    "e2f_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "e2f_neighbors_workspace_size": (_sz, [_i64, _vp, ctypes.c_float, ctypes.c_int32]),
+    "e2f_build_neighbors": (ctypes.c_int, [_vp, _i64, _vp, ctypes.c_float, _vp, ctypes.c_int32, _vp, _vp, _i64,
+                                           ctypes.POINTER(_i64), _vp, _sz, _vp]),
+    "e2f_attention_workspace_size": (_sz, [_i64, _i64, ctypes.POINTER(e2f_attn_cfg)]),
+    "e2f_onfly_attention": (ctypes.c_int, [ctypes.POINTER(e2f_attn_cfg), _vp, _i64, _vp, _vp, _vp, _i64, _vp, _vp,
+                                           _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "e2f_attention_status": (ctypes.c_int, [_vp, _sz, _vp]),
+    "e2f_edge_wigner_blocks": (ctypes.c_int, [_vp, _i64, ctypes.c_int, _vp, _vp, _vp]),
+    "e2f_launch_count": (_i64, []),
+}
+
+
+def lib() -> ctypes.CDLL:
+    """Load libe2f.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with `python -m atomistic_cell_list_b200.build`")
+        h = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            f = getattr(h, name)
+            f.restype, f.argtypes = res, args
+        _lib = h
+    return _lib
+
+
+def header_symbols(path: str = HEADER) -> list[str]:
+    """Names of the functions include/e2f.h declares."""
+    src = open(path).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(e2f_[a-z0-9_]+)\s*\(", src)))
+
+
+def status_string(code: int) -> str:
+    return lib().e2f_status_string(int(code)).decode()
+
+
+def e2f_status_string(code: int) -> str:
+    return status_string(code)
+
+
+def _check(code: int, where: str):
+    if code != E2F_OK:
+        raise E2FError(code, where)
+
+
+def _stream(stream=None) -> int:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return int(s.cuda_stream)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _box_arg(box):
+    if box is None:
+        return None, None
+    arr = (ctypes.c_float * 3)(*[float(v) for v in box])
+    return ctypes.cast(arr, ctypes.c_void_p), arr
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("tensors must be contiguous CUDA tensors")
+
+
+def e2f_neighbors_workspace_size(n_atoms: int, box, cutoff: float, n_graphs: int = 1) -> int:
+    b, keep = _box_arg(box)
+    return int(lib().e2f_neighbors_workspace_size(int(n_atoms), b, float(cutoff), int(n_graphs)))
+
+
+def e2f_build_neighbors(pos: torch.Tensor, box, cutoff: float, graph_ptr: torch.Tensor | None = None,
+                        col_capacity: int | None = None, stream=None):
+    """CSR neighbour list (row_ptr int32 [N+1], col int32 [E]) by the GPU cell list."""
+    _need_cuda(pos, graph_ptr)
+    assert pos.dtype == torch.float32 and pos.dim() == 2 and pos.shape[1] == 3
+    n = pos.shape[0]
+    n_graphs = 1 if graph_ptr is None else graph_ptr.numel() - 1
+    dev = pos.device
+    ws_bytes = e2f_neighbors_workspace_size(n, box, cutoff, n_graphs)
+    ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
+    row_ptr = torch.empty(n + 1, dtype=torch.int32, device=dev)
+    cap = int(col_capacity) if col_capacity is not None else max(1024, 128 * n)
+    b, keep = _box_arg(box)
+    for _ in range(2):
+        col = torch.empty(max(cap, 1), dtype=torch.int32, device=dev)
+        npairs = ctypes.c_int64(0)
+        code = lib().e2f_build_neighbors(_ptr(pos), n, b, float(cutoff), _ptr(graph_ptr), n_graphs,
+                                         _ptr(row_ptr), _ptr(col), cap, ctypes.byref(npairs), _ptr(ws), ws_bytes,
+                                         _stream(stream))
+        if code == 3:  # capacity: grow to the exact size and retry
+            cap = int(npairs.value)
+            continue
+        _check(code, "e2f_build_neighbors")
+        return row_ptr, col[: npairs.value]
+    raise E2FError(3, "e2f_build_neighbors")
+
+
+def make_cfg(L: int, C: int, H: int, n_rbf: int, cutoff: float, dtype: str) -> e2f_attn_cfg:
+    return e2f_attn_cfg(L, C, H, n_rbf, float(cutoff), E2F_BF16 if dtype == "bf16" else E2F_F32)
+
+
+def e2f_attention_workspace_size(n_atoms: int, n_pairs: int, cfg: e2f_attn_cfg) -> int:
+    return int(lib().e2f_attention_workspace_size(int(n_atoms), int(n_pairs), ctypes.byref(cfg)))
+
+
+def e2f_onfly_attention(cfg: e2f_attn_cfg, pos, box, row_ptr, col, x, W_q, W_k, W_rad, W_so2,
+                        out: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+                        stream=None, check: bool = True) -> torch.Tensor:
+    """out[N, (L+1)^2, C] fp32 = on-the-fly equivariant attention (see include/e2f.h)."""
+    _need_cuda(pos, row_ptr, col, x, W_q, W_k, W_rad, W_so2, out, workspace)
+    n = pos.shape[0]
+    K = (cfg.L + 1) ** 2
+    if out is None:
+        out = torch.empty((n, K, cfg.C), dtype=torch.float32, device=pos.device)
+    ws_bytes = e2f_attention_workspace_size(n, col.numel(), cfg)
+    if workspace is None or workspace.numel() < ws_bytes:
+        workspace = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=pos.device)
+    b, keep = _box_arg(box)
+    s = _stream(stream)
+    code = lib().e2f_onfly_attention(ctypes.byref(cfg), _ptr(pos), n, b, _ptr(row_ptr), _ptr(col), col.numel(),
+                                     _ptr(x), _ptr(W_q), _ptr(W_k), _ptr(W_rad), _ptr(W_so2), _ptr(out),
+                                     _ptr(workspace), workspace.numel(), s)
+    _check(code, "e2f_onfly_attention")
+    if check:
+        _check(lib().e2f_attention_status(_ptr(workspace), workspace.numel(), s), "e2f_onfly_attention (device)")
+    return out
+
+
+def e2f_attention_status(workspace: torch.Tensor, stream=None) -> int:
+    return int(lib().e2f_attention_status(_ptr(workspace), workspace.numel(), _stream(stream)))
+
+
+def e2f_edge_wigner_blocks(r: torch.Tensor, L: int, with_frames: bool = False, stream=None):
+    _need_cuda(r)
+    n = r.shape[0]
+    S = sum((2 * l + 1) ** 2 for l in range(L + 1))
+    out = torch.empty((n, S), dtype=torch.float32, device=r.device)
+    fr = torch.empty((n, 3, 3), dtype=torch.float32, device=r.device) if with_frames else None
+    _check(lib().e2f_edge_wigner_blocks(_ptr(r), n, int(L), _ptr(out), _ptr(fr), _stream(stream)),
+           "e2f_edge_wigner_blocks")
+    return (out, fr) if with_frames else out
+
+
+def e2f_launch_count() -> int:
+    return int(lib().e2f_launch_count())
+
+
+# short aliases
+build_neighbors = e2f_build_neighbors
+onfly_attention = e2f_onfly_attention
+edge_wigner_blocks = e2f_edge_wigner_blocks

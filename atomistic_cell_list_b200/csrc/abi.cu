@@ -1,0 +1,135 @@
+// C-ABI entry points of libe2f.so for the attention path (argument checks,
+// workspace layout, dispatch). The neighbour build lives in neighbors.cu.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <atomic>
+#include <cmath>
+
+#include "attention.cuh"
+#include "common.cuh"
+
+namespace e2f {
+static std::atomic<long long> g_launches{0};
+void count_launch(int n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+}  // namespace e2f
+
+using namespace e2f;
+
+namespace {
+
+struct AttnWs {
+    size_t o_status, o_q, o_k, o_wt, bytes;
+};
+
+AttnWs attn_layout(int64_t n_atoms, const e2f_attn_cfg& c) {
+    AttnWs w{};
+    size_t o = 0;
+    auto take = [&](size_t b) { size_t r = o; o = align_up(o + b, 256); return r; };
+    w.o_status = take(256);
+    w.o_q = take(4 * (size_t)n_atoms * c.C);
+    w.o_k = take(4 * (size_t)n_atoms * c.C);
+    w.o_wt = take(4 * so2_total(c.L, c.C));
+    w.bytes = o;
+    return w;
+}
+
+e2f_status check_cfg(const e2f_attn_cfg* c) {
+    if (!c) return E2F_ERR_INVALID_ARG;
+    if (c->L < 0 || c->C <= 0 || c->H <= 0 || !(c->cutoff > 0.f) || !std::isfinite(c->cutoff))
+        return E2F_ERR_INVALID_ARG;
+    if (c->feat_dtype != E2F_F32 && c->feat_dtype != E2F_BF16) return E2F_ERR_UNSUPPORTED;
+    if (c->L > kMaxL || c->C % 16 != 0 || c->C > 256 || c->C % c->H != 0 || c->n_rbf < 2 || c->n_rbf > 32)
+        return E2F_ERR_UNSUPPORTED;
+    return E2F_OK;
+}
+
+}  // namespace
+
+extern "C" const char* e2f_status_string(e2f_status s) {
+    switch (s) {
+        case E2F_OK: return "ok";
+        case E2F_ERR_INVALID_ARG: return "invalid argument";
+        case E2F_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+        case E2F_ERR_CAPACITY: return "output capacity too small";
+        case E2F_ERR_ALIGNMENT: return "misaligned pointer";
+        case E2F_ERR_TIMEOUT: return "device-side wait timed out";
+        case E2F_ERR_CUDA: return "CUDA error";
+        case E2F_ERR_NONFINITE: return "non-finite position";
+    }
+    return "unknown status";
+}
+
+extern "C" size_t e2f_attention_workspace_size(int64_t n_atoms, int64_t n_pairs, const e2f_attn_cfg* cfg) {
+    (void)n_pairs;
+    if (check_cfg(cfg) != E2F_OK || n_atoms < 0) return 0;
+    return attn_layout(n_atoms, *cfg).bytes;
+}
+
+extern "C" e2f_status e2f_onfly_attention(const e2f_attn_cfg* cfg, const float* pos, int64_t n_atoms,
+                                          const float* box_host, const int32_t* row_ptr, const int32_t* col,
+                                          int64_t n_pairs, const void* x, const float* W_q, const float* W_k,
+                                          const float* W_rad, const void* W_so2, float* out, void* workspace,
+                                          size_t ws_bytes, void* stream_) {
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    e2f_status st = check_cfg(cfg);
+    if (st != E2F_OK) return st;
+    if (n_atoms < 0 || n_atoms > INT32_MAX || n_pairs < 0 || n_pairs > INT32_MAX) return E2F_ERR_INVALID_ARG;
+    if (n_atoms == 0) return E2F_OK;
+    if (!pos || !row_ptr || (n_pairs > 0 && !col) || !x || !W_q || !W_k || !W_rad || !W_so2 || !out || !workspace)
+        return E2F_ERR_INVALID_ARG;
+    if (box_host) {
+        for (int a = 0; a < 3; ++a)
+            if (!(box_host[a] > 0.f) || !std::isfinite(box_host[a]) || cfg->cutoff > 0.5f * box_host[a])
+                return E2F_ERR_INVALID_ARG;
+    }
+    if (reinterpret_cast<uintptr_t>(workspace) % 256 || reinterpret_cast<uintptr_t>(x) % 16 ||
+        reinterpret_cast<uintptr_t>(W_so2) % 16 || reinterpret_cast<uintptr_t>(out) % 16)
+        return E2F_ERR_ALIGNMENT;
+    AttnWs L = attn_layout(n_atoms, *cfg);
+    if (ws_bytes < L.bytes) return E2F_ERR_INVALID_ARG;
+    char* ws = static_cast<char*>(workspace);
+
+    AttnArgs a{};
+    a.L = cfg->L; a.C = cfg->C; a.H = cfg->H; a.n_rbf = cfg->n_rbf; a.cutoff = cfg->cutoff;
+    a.bf16 = cfg->feat_dtype == E2F_BF16;
+    a.n_atoms = (int)n_atoms; a.n_pairs = n_pairs;
+    a.box.periodic = box_host != nullptr;
+    if (box_host) {
+        a.box.len = make_float3(box_host[0], box_host[1], box_host[2]);
+        a.box.inv = make_float3(1.0f / box_host[0], 1.0f / box_host[1], 1.0f / box_host[2]);
+    } else {
+        a.box.len = a.box.inv = make_float3(0.f, 0.f, 0.f);
+    }
+    a.pos = pos; a.row_ptr = row_ptr; a.col = col; a.x = x;
+    a.Wq = W_q; a.Wk = W_k; a.Wrad = W_rad; a.Wso2 = W_so2; a.out = out;
+    a.status = reinterpret_cast<int*>(ws + L.o_status);
+    a.q = reinterpret_cast<float*>(ws + L.o_q);
+    a.k = reinterpret_cast<float*>(ws + L.o_k);
+    a.Wt = reinterpret_cast<float*>(ws + L.o_wt);
+    E2F_CUDA_TRY(cudaMemsetAsync(a.status, 0, sizeof(int), stream));
+    E2F_CUDA_TRY(run_attention_simt(a, stream));
+    return E2F_OK;
+}
+
+extern "C" e2f_status e2f_attention_status(void* workspace, size_t ws_bytes, void* stream_) {
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    if (!workspace || ws_bytes < 256) return E2F_ERR_INVALID_ARG;
+    int v = 0;
+    E2F_CUDA_TRY(cudaMemcpyAsync(&v, workspace, sizeof(int), cudaMemcpyDeviceToHost, stream));
+    E2F_CUDA_TRY(cudaMemsetAsync(workspace, 0, sizeof(int), stream));
+    E2F_CUDA_TRY(cudaStreamSynchronize(stream));
+    E2F_CUDA_TRY(cudaGetLastError());
+    return v == 0 ? E2F_OK : static_cast<e2f_status>(v);
+}
+
+extern "C" e2f_status e2f_edge_wigner_blocks(const float* r, int64_t n_edges, int L, float* out, float* frames,
+                                             void* stream_) {
+    if (L < 0 || L > kMaxL || n_edges < 0) return L > kMaxL ? E2F_ERR_UNSUPPORTED : E2F_ERR_INVALID_ARG;
+    if (n_edges == 0) return E2F_OK;
+    if (!r || !out) return E2F_ERR_INVALID_ARG;
+    E2F_CUDA_TRY(run_edge_wigner(r, n_edges, L, out, frames, static_cast<cudaStream_t>(stream_)));
+    return E2F_OK;
+}
+
+extern "C" int64_t e2f_launch_count(void) { return (int64_t)g_launches.load(); }

@@ -1,0 +1,57 @@
+// Internal interface between the C-ABI entry points and the attention kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <algorithm>
+
+#include "common.cuh"
+
+namespace e2f {
+
+// Packed SO(2) weight blocks: A(0) of side (L+1)C, then A(m), B(m) of side
+// (L+1-m)C for m = 1..L. which = 0 selects A(m), 1 selects B(m).
+__host__ __device__ inline size_t so2_offset(int L, int C, int m, int which) {
+    size_t n0 = (size_t)(L + 1) * C;
+    size_t off = n0 * n0;
+    if (m == 0) return 0;
+    for (int k = 1; k < m; ++k) {
+        size_t n = (size_t)(L + 1 - k) * C;
+        off += 2 * n * n;
+    }
+    size_t n = (size_t)(L + 1 - m) * C;
+    return off + (which ? n * n : 0);
+}
+
+__host__ __device__ inline size_t so2_total(int L, int C) {
+    return so2_offset(L, C, L + 1, 0);
+}
+
+struct AttnArgs {
+    int L, C, H, n_rbf;
+    float cutoff;
+    bool bf16;
+    int n_atoms;
+    int64_t n_pairs;
+    Box box;
+    const float* pos;
+    const int32_t* row_ptr;
+    const int32_t* col;
+    const void* x;
+    const float* Wq;
+    const float* Wk;
+    const float* Wrad;
+    const void* Wso2;
+    float* out;
+    // workspace pieces
+    int* status;
+    float* q;
+    float* k;
+    float* Wt;
+};
+
+cudaError_t run_attention_simt(const AttnArgs& a, cudaStream_t s);
+cudaError_t run_edge_wigner(const float* r, int64_t n, int L, float* out, float* frames, cudaStream_t s);
+
+}  // namespace e2f

@@ -1,0 +1,394 @@
+// Cell-list neighbour build for libe2f (see include/e2f.h).
+//
+// Pipeline (one stream, one host synchronisation to read E):
+//   1 prep      per atom: finite check, graph id, cell -> bucket, rank in
+//               bucket (atomic count)
+//   2 scan      bucket counts -> bucket starts
+//   3 scatter   atoms sorted by bucket: float4 (x, y, z, graph id), index
+//   4 count     one warp per atom scans its 27 neighbouring buckets with
+//               the exact fp32 predicate -> degree
+//   5 scan      degrees -> row_ptr; E and error flags copied to the host
+//   6 fill      same scan, neighbours gathered in shared memory, bitonic
+//               sorted, written ascending
+// Periodic boxes use a direct grid of n_c^3 cells per graph (cells at least
+// cutoff*(1+1e-3) wide); open boundaries hash (graph, cell) into 2^k
+// buckets and drop repeated buckets from the 27-cell stencil, so a
+// collision only adds candidates that the predicate then rejects.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <algorithm>
+#include <cmath>
+
+#include "common.cuh"
+#include "scan.cuh"
+
+namespace e2f {
+namespace {
+
+constexpr int kSortCap = 1024;   // rows up to this many neighbours sort in shared memory
+constexpr int kWarpsPerBlock = 4;
+constexpr float kCellSlack = 1.0e-3f;
+
+enum : int { kFlagNonFinite = 1, kFlagBadGraph = 2 };
+
+struct Grid {
+    Box box;
+    int nc[3];           // periodic: cells per axis
+    float cell;          // open: cell side
+    uint32_t n_buckets;  // periodic: n_graphs * nc^3; open: power of two
+    uint32_t mask;       // open: n_buckets - 1
+    int offs[3][3];      // periodic stencil offsets per axis (deduplicated)
+    int noff[3];
+};
+
+__device__ __forceinline__ bool pair_within(float4 a, float4 b, const Grid& g, float rc2) {
+    // the exact sequence of IEEE round-to-nearest operations (no FMA)
+    float dx = __fsub_rn(b.x, a.x), dy = __fsub_rn(b.y, a.y), dz = __fsub_rn(b.z, a.z);
+    if (g.box.periodic) {
+        dx = __fsub_rn(dx, __fmul_rn(g.box.len.x, rintf(__fmul_rn(dx, g.box.inv.x))));
+        dy = __fsub_rn(dy, __fmul_rn(g.box.len.y, rintf(__fmul_rn(dy, g.box.inv.y))));
+        dz = __fsub_rn(dz, __fmul_rn(g.box.len.z, rintf(__fmul_rn(dz, g.box.inv.z))));
+    }
+    float d2 = __fadd_rn(__fadd_rn(__fmul_rn(dx, dx), __fmul_rn(dy, dy)), __fmul_rn(dz, dz));
+    return d2 < rc2;
+}
+
+__device__ __forceinline__ void cell_of(float x, float y, float z, const Grid& g, long long c[3]) {
+    // fp64 so that the cell of a point never moves by more than the slack
+    const double p[3] = {x, y, z};
+    if (g.box.periodic) {
+        const double len[3] = {g.box.len.x, g.box.len.y, g.box.len.z};
+#pragma unroll
+        for (int a = 0; a < 3; ++a) {
+            double w = p[a] - len[a] * floor(p[a] / len[a]);   // wrapped into [0, len]
+            long long k = (long long)(w * (double(g.nc[a]) / len[a]));
+            c[a] = k < 0 ? 0 : (k >= g.nc[a] ? g.nc[a] - 1 : k);
+        }
+    } else {
+#pragma unroll
+        for (int a = 0; a < 3; ++a) c[a] = (long long)floor(p[a] / double(g.cell));
+    }
+}
+
+__device__ __forceinline__ uint32_t bucket_of(const long long c[3], int gid, const Grid& g) {
+    if (g.box.periodic) {
+        long long idx = (((long long)gid * g.nc[2] + c[2]) * g.nc[1] + c[1]) * g.nc[0] + c[0];
+        return (uint32_t)idx;
+    }
+    uint64_t h = (uint64_t)c[0] * 0x9E3779B97F4A7C15ull;
+    h ^= (uint64_t)c[1] * 0xC2B2AE3D27D4EB4Full + (h >> 29);
+    h ^= (uint64_t)c[2] * 0x165667B19E3779F9ull + (h >> 32);
+    h ^= (uint64_t)(uint32_t)gid * 0x27D4EB2F165667C5ull + (h >> 31);
+    h ^= h >> 33;
+    return (uint32_t)h & g.mask;
+}
+
+// the (up to) 27 distinct buckets around cell c; returns how many
+__device__ __forceinline__ int stencil_buckets(const long long c[3], int gid, const Grid& g, uint32_t out[27]) {
+    int n = 0;
+    if (g.box.periodic) {
+        for (int iz = 0; iz < g.noff[2]; ++iz)
+            for (int iy = 0; iy < g.noff[1]; ++iy)
+                for (int ix = 0; ix < g.noff[0]; ++ix) {
+                    long long cc[3] = {c[0] + g.offs[0][ix], c[1] + g.offs[1][iy], c[2] + g.offs[2][iz]};
+                    for (int a = 0; a < 3; ++a) cc[a] = (cc[a] % g.nc[a] + g.nc[a]) % g.nc[a];
+                    out[n++] = bucket_of(cc, gid, g);
+                }
+        return n;
+    }
+    for (int dz = -1; dz <= 1; ++dz)
+        for (int dy = -1; dy <= 1; ++dy)
+            for (int dx = -1; dx <= 1; ++dx) {
+                long long cc[3] = {c[0] + dx, c[1] + dy, c[2] + dz};
+                uint32_t b = bucket_of(cc, gid, g);
+                bool dup = false;
+                for (int k = 0; k < n; ++k) dup |= (out[k] == b);
+                if (!dup) out[n++] = b;
+            }
+    return n;
+}
+
+__device__ __forceinline__ int graph_id(const int32_t* gp, int n_graphs, int i) {
+    if (!gp) return 0;
+    int lo = 0, hi = n_graphs - 1;  // last g with gp[g] <= i
+    while (lo < hi) {
+        int mid = (lo + hi + 1) >> 1;
+        if (__ldg(gp + mid) <= i) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+}
+
+__global__ void k_check_graphs(const int32_t* gp, int n_graphs, int n_atoms, int* flags) {
+    int g = blockIdx.x * blockDim.x + threadIdx.x;
+    if (g > n_graphs) return;
+    int v = gp[g];
+    bool bad = (g == 0 && v != 0) || (g == n_graphs && v != n_atoms) || v < 0 || v > n_atoms ||
+               (g < n_graphs && gp[g + 1] < v);
+    if (bad) atomicOr(flags, kFlagBadGraph);
+}
+
+__global__ void k_prep(const float* __restrict__ pos, int n, const int32_t* gp, int n_graphs, Grid g,
+                       uint32_t* key, uint32_t* rank, uint32_t* count, int* flags) {
+    int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= n) return;
+    float x = pos[3 * i], y = pos[3 * i + 1], z = pos[3 * i + 2];
+    uint32_t b = 0;
+    if (!(isfinite(x) && isfinite(y) && isfinite(z))) {
+        atomicOr(flags, kFlagNonFinite);
+    } else {
+        long long c[3];
+        cell_of(x, y, z, g, c);
+        b = bucket_of(c, graph_id(gp, n_graphs, i), g);
+    }
+    key[i] = b;
+    rank[i] = atomicAdd(count + b, 1u);
+}
+
+__global__ void k_scatter(const float* __restrict__ pos, int n, const int32_t* gp, int n_graphs,
+                          const uint32_t* key, const uint32_t* rank, const uint32_t* start,
+                          float4* sorted_pos, int32_t* sorted_idx) {
+    int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= n) return;
+    uint32_t s = start[key[i]] + rank[i];
+    sorted_pos[s] = make_float4(pos[3 * i], pos[3 * i + 1], pos[3 * i + 2],
+                                __int_as_float(graph_id(gp, n_graphs, i)));
+    sorted_idx[s] = i;
+}
+
+// One warp per atom. MODE 0: count neighbours into deg[i]. MODE 1: write the
+// row ascending at col[row_ptr[i] ...].
+template <int MODE>
+__global__ void __launch_bounds__(32 * kWarpsPerBlock)
+k_pairs(const float* __restrict__ pos, int n, const int32_t* gp, int n_graphs, Grid g, float rc2,
+        const uint32_t* __restrict__ start, const float4* __restrict__ sorted_pos,
+        const int32_t* __restrict__ sorted_idx, int32_t* deg, const int32_t* __restrict__ row_ptr,
+        int32_t* col) {
+    __shared__ int32_t buf[kWarpsPerBlock][kSortCap];
+    const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+    const int i = blockIdx.x * kWarpsPerBlock + wib;
+    if (i >= n) return;
+    const int gid = graph_id(gp, n_graphs, i);
+    const float4 me = make_float4(pos[3 * i], pos[3 * i + 1], pos[3 * i + 2], __int_as_float(gid));
+    long long c[3];
+    cell_of(me.x, me.y, me.z, g, c);
+    uint32_t bk[27];
+    const int nb = stencil_buckets(c, gid, g, bk);
+
+    int total = 0;
+    int row0 = 0, rlen = 0;
+    if (MODE == 1) { row0 = row_ptr[i]; rlen = row_ptr[i + 1] - row0; }
+    const bool in_smem = (MODE == 1) && rlen <= kSortCap;
+    for (int b = 0; b < nb; ++b) {
+        const uint32_t s0 = start[bk[b]], s1 = start[bk[b] + 1];
+        for (uint32_t s = s0; s < s1; s += 32) {
+            bool hit = false;
+            int j = -1;
+            if (s + lane < s1) {
+                float4 o = sorted_pos[s + lane];
+                j = sorted_idx[s + lane];
+                hit = (j != i) && (__float_as_int(o.w) == gid) && pair_within(me, o, g, rc2);
+            }
+            unsigned m = __ballot_sync(0xffffffffu, hit);
+            if (MODE == 1 && hit) {
+                int slot = total + __popc(m & ((1u << lane) - 1u));
+                if (slot < rlen) {  // equal counts in both passes; guard anyway
+                    if (in_smem) buf[wib][slot] = j; else col[row0 + slot] = j;
+                }
+            }
+            total += __popc(m);
+        }
+    }
+    if (MODE == 0) {
+        if (lane == 0) deg[i] = total;
+        return;
+    }
+    __syncwarp();
+    if (in_smem) {
+        int P = 1;
+        while (P < rlen) P <<= 1;
+        for (int t = rlen + lane; t < P; t += 32) buf[wib][t] = 0x7fffffff;
+        __syncwarp();
+        for (int k = 2; k <= P; k <<= 1)
+            for (int jj = k >> 1; jj > 0; jj >>= 1) {
+                for (int t = lane; t < P; t += 32) {
+                    int u = t ^ jj;
+                    if (u > t) {
+                        int a = buf[wib][t], bb = buf[wib][u];
+                        bool up = (t & k) == 0;
+                        if ((a > bb) == up) { buf[wib][t] = bb; buf[wib][u] = a; }
+                    }
+                }
+                __syncwarp();
+            }
+        for (int t = lane; t < rlen; t += 32) col[row0 + t] = buf[wib][t];
+        return;
+    }
+    // very dense row: odd-even transposition sort in place (global memory)
+    int32_t* r = col + row0;
+    for (int phase = 0; phase < rlen; ++phase) {
+        for (int t = 2 * lane + (phase & 1); t + 1 < rlen; t += 64) {
+            int a = r[t], bb = r[t + 1];
+            if (a > bb) { r[t] = bb; r[t + 1] = a; }
+        }
+        __syncwarp();
+        __threadfence_block();
+    }
+}
+
+bool make_grid(const float* box_host, float cutoff, int n_graphs, int64_t n_atoms, Grid& g) {
+    g.box.periodic = box_host != nullptr;
+    if (g.box.periodic) {
+        g.box.len = make_float3(box_host[0], box_host[1], box_host[2]);
+        g.box.inv = make_float3(1.0f / box_host[0], 1.0f / box_host[1], 1.0f / box_host[2]);
+        long long total = std::max(1, n_graphs);
+        for (int a = 0; a < 3; ++a) {
+            int nc = (int)std::floor(double(box_host[a]) / (double(cutoff) * (1.0 + kCellSlack)));
+            g.nc[a] = std::max(1, std::min(nc, 1024));
+        }
+        // keep the grid at most 2^26 buckets: coarsen the largest axis
+        while (total * g.nc[0] * g.nc[1] * g.nc[2] > (1ll << 26)) {
+            int a = (g.nc[0] >= g.nc[1] && g.nc[0] >= g.nc[2]) ? 0 : (g.nc[1] >= g.nc[2] ? 1 : 2);
+            g.nc[a] = std::max(1, g.nc[a] / 2);
+        }
+        for (int a = 0; a < 3; ++a) {
+            if (g.nc[a] >= 3) { g.offs[a][0] = -1; g.offs[a][1] = 0; g.offs[a][2] = 1; g.noff[a] = 3; }
+            else if (g.nc[a] == 2) { g.offs[a][0] = 0; g.offs[a][1] = 1; g.noff[a] = 2; }
+            else { g.offs[a][0] = 0; g.noff[a] = 1; }
+        }
+        g.n_buckets = (uint32_t)(total * g.nc[0] * g.nc[1] * g.nc[2]);
+        g.mask = 0;
+        g.cell = 0.f;
+    } else {
+        g.box.len = g.box.inv = make_float3(0.f, 0.f, 0.f);
+        g.cell = cutoff * (1.0f + kCellSlack);
+        uint32_t nb = 64;
+        while ((int64_t)nb < 2 * n_atoms && nb < (1u << 28)) nb <<= 1;
+        g.n_buckets = nb;
+        g.mask = nb - 1;
+        for (int a = 0; a < 3; ++a) { g.nc[a] = 0; g.noff[a] = 0; }
+    }
+    return true;
+}
+
+struct NbrWs {
+    int* flags;
+    uint32_t* key;
+    uint32_t* rank;
+    uint32_t* count;     // n_buckets + 1
+    float4* sorted_pos;
+    int32_t* sorted_idx;
+    int32_t* deg;        // n + 1
+    void* scan_tmp;
+    size_t bytes;
+};
+
+NbrWs carve(void* base, int64_t n, uint32_t n_buckets) {
+    NbrWs w{};
+    size_t o = 0;
+    auto take = [&](size_t b) { size_t r = o; o = align_up(o + b, 256); return r; };
+    char* p = static_cast<char*>(base);
+    size_t o_flags = take(256);
+    size_t o_key = take(4 * (size_t)n), o_rank = take(4 * (size_t)n);
+    size_t o_count = take(4 * ((size_t)n_buckets + 1));
+    size_t o_spos = take(16 * (size_t)n), o_sidx = take(4 * (size_t)n);
+    size_t o_deg = take(4 * ((size_t)n + 1));
+    size_t tmp = std::max(scan_tmp_bytes((size_t)n_buckets + 1), scan_tmp_bytes((size_t)n + 1));
+    size_t o_tmp = take(tmp);
+    w.bytes = o;
+    if (p) {
+        w.flags = (int*)(p + o_flags);
+        w.key = (uint32_t*)(p + o_key);
+        w.rank = (uint32_t*)(p + o_rank);
+        w.count = (uint32_t*)(p + o_count);
+        w.sorted_pos = (float4*)(p + o_spos);
+        w.sorted_idx = (int32_t*)(p + o_sidx);
+        w.deg = (int32_t*)(p + o_deg);
+        w.scan_tmp = p + o_tmp;
+    }
+    return w;
+}
+
+}  // namespace
+}  // namespace e2f
+
+using namespace e2f;
+
+extern "C" size_t e2f_neighbors_workspace_size(int64_t n_atoms, const float* box_host, float cutoff,
+                                               int32_t n_graphs) {
+    if (n_atoms < 0 || !(cutoff > 0.f)) return 0;
+    Grid g;
+    make_grid(box_host, cutoff, std::max(1, (int)n_graphs), n_atoms, g);
+    return carve(nullptr, n_atoms, g.n_buckets).bytes;
+}
+
+extern "C" e2f_status e2f_build_neighbors(const float* pos, int64_t n_atoms, const float* box_host,
+                                          float cutoff, const int32_t* graph_ptr, int32_t n_graphs,
+                                          int32_t* row_ptr, int32_t* col, int64_t col_capacity,
+                                          int64_t* n_pairs_host, void* workspace, size_t ws_bytes,
+                                          void* stream_) {
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    if (!n_pairs_host || !row_ptr || n_atoms < 0 || n_atoms > INT32_MAX - 1 || !(cutoff > 0.f) ||
+        !std::isfinite(cutoff) || col_capacity < 0)
+        return E2F_ERR_INVALID_ARG;
+    if (n_atoms > 0 && (!pos || !workspace)) return E2F_ERR_INVALID_ARG;
+    if (graph_ptr && n_graphs < 1) return E2F_ERR_INVALID_ARG;
+    if (col_capacity > 0 && !col) return E2F_ERR_INVALID_ARG;
+    if (box_host) {
+        for (int a = 0; a < 3; ++a)
+            if (!(box_host[a] > 0.f) || !std::isfinite(box_host[a]) || cutoff > 0.5f * box_host[a])
+                return E2F_ERR_INVALID_ARG;
+    }
+    if (reinterpret_cast<uintptr_t>(workspace) % 256 != 0) return E2F_ERR_ALIGNMENT;
+    const int ng = graph_ptr ? n_graphs : 1;
+    const int n = (int)n_atoms;
+    if (n == 0) {
+        E2F_CUDA_TRY(cudaMemsetAsync(row_ptr, 0, sizeof(int32_t), stream));
+        E2F_CUDA_TRY(cudaStreamSynchronize(stream));
+        *n_pairs_host = 0;
+        return E2F_OK;
+    }
+    Grid g;
+    make_grid(box_host, cutoff, ng, n_atoms, g);
+    NbrWs w = carve(workspace, n_atoms, g.n_buckets);
+    if (ws_bytes < w.bytes) return E2F_ERR_INVALID_ARG;
+    const float rc2 = cutoff * cutoff;  // fp32 product, as in the predicate
+
+    E2F_CUDA_TRY(cudaMemsetAsync(w.flags, 0, 256, stream));
+    E2F_CUDA_TRY(cudaMemsetAsync(w.count, 0, 4 * ((size_t)g.n_buckets + 1), stream));
+    if (graph_ptr) {
+        count_launch();
+        k_check_graphs<<<(ng + 1 + 255) / 256, 256, 0, stream>>>(graph_ptr, ng, n, w.flags);
+    }
+    const int tb = 256, nbk = (n + tb - 1) / tb;
+    count_launch();
+    k_prep<<<nbk, tb, 0, stream>>>(pos, n, graph_ptr, ng, g, w.key, w.rank, w.count, w.flags);
+    E2F_CUDA_TRY(exclusive_scan_u32(w.count, w.count, (size_t)g.n_buckets + 1, w.scan_tmp, stream));
+    count_launch();
+    k_scatter<<<nbk, tb, 0, stream>>>(pos, n, graph_ptr, ng, w.key, w.rank, w.count, w.sorted_pos,
+                                       w.sorted_idx);
+    const int wb = (n + kWarpsPerBlock - 1) / kWarpsPerBlock;
+    count_launch();
+    k_pairs<0><<<wb, 32 * kWarpsPerBlock, 0, stream>>>(pos, n, graph_ptr, ng, g, rc2, w.count,
+                                                       w.sorted_pos, w.sorted_idx, w.deg, nullptr, nullptr);
+    E2F_CUDA_TRY(cudaMemsetAsync(w.deg + n, 0, sizeof(int32_t), stream));
+    E2F_CUDA_TRY(exclusive_scan_u32(reinterpret_cast<uint32_t*>(w.deg), reinterpret_cast<uint32_t*>(row_ptr),
+                                    (size_t)n + 1, w.scan_tmp, stream));
+    int host[2] = {0, 0};
+    E2F_CUDA_TRY(cudaMemcpyAsync(&host[0], row_ptr + n, sizeof(int32_t), cudaMemcpyDeviceToHost, stream));
+    E2F_CUDA_TRY(cudaMemcpyAsync(&host[1], w.flags, sizeof(int32_t), cudaMemcpyDeviceToHost, stream));
+    E2F_CUDA_TRY(cudaStreamSynchronize(stream));
+    E2F_CUDA_TRY(cudaGetLastError());
+    if (host[1] & kFlagBadGraph) return E2F_ERR_INVALID_ARG;
+    if (host[1] & kFlagNonFinite) return E2F_ERR_NONFINITE;
+    const int64_t E = (uint32_t)host[0];
+    *n_pairs_host = E;
+    if (E > col_capacity) return E2F_ERR_CAPACITY;
+    if (E > 0) {
+        count_launch();
+        k_pairs<1><<<wb, 32 * kWarpsPerBlock, 0, stream>>>(pos, n, graph_ptr, ng, g, rc2, w.count,
+                                                           w.sorted_pos, w.sorted_idx, nullptr, row_ptr, col);
+        E2F_CUDA_TRY(cudaGetLastError());
+    }
+    return E2F_OK;
+}

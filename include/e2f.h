@@ -1,0 +1,182 @@
+/*
+ * e2f.h - C ABI of libe2f.so: a GPU cell-list neighbour build and the
+ * node-centric on-the-fly equivariant attention forward pass of E2Former-V2
+ * ("E2Former-V2: On-the-Fly Equivariant Attention with Linear Activation
+ * Memory", arXiv 2601.16622; summarised on gist.science, Technical Summary
+ * sections 2.1 and 2.2, and in the abstract on fugumt.com).
+ *
+ * Conventions shared by every entry point
+ *   - Device pointers point to memory of the current CUDA device; host
+ *     pointers are read (or written) before the call returns.
+ *   - The caller owns every buffer. The library allocates no device memory
+ *     of its own; it works inside the caller's workspace. Per device it keeps
+ *     only lazily set kernel attributes.
+ *   - Work is enqueued on `stream` (0 = legacy default stream) in stream
+ *     order. Calls that return a host value (n_pairs_host) synchronise it.
+ *   - Argument checks happen before any launch; a failed check launches
+ *     nothing and leaves every output untouched. Unsupported shapes return
+ *     E2F_ERR_UNSUPPORTED. There is no CPU fallback.
+ *   - Irreducible features use the flat index k(l, m) = l*l + l + m,
+ *     m = -l..l, with real spherical harmonics ordered so that degree 1 is
+ *     proportional to (y, z, x); the channel index is innermost.
+ */
+#ifndef E2F_H
+#define E2F_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    E2F_OK = 0,
+    E2F_ERR_INVALID_ARG = 1,  /* null pointer, negative size, bad range      */
+    E2F_ERR_UNSUPPORTED = 2,  /* shape or dtype this build does not handle   */
+    E2F_ERR_CAPACITY = 3,     /* output buffer too small (see n_pairs_host)  */
+    E2F_ERR_ALIGNMENT = 4,    /* pointer not aligned as documented           */
+    E2F_ERR_TIMEOUT = 5,      /* a bounded device-side wait ran out          */
+    E2F_ERR_CUDA = 6,         /* a CUDA runtime call or launch failed        */
+    E2F_ERR_NONFINITE = 7     /* NaN/Inf in positions                        */
+} e2f_status;
+
+typedef enum { E2F_F32 = 0, E2F_BF16 = 1 } e2f_dtype;
+
+/* Layer shape. L = highest degree (0..4); C = channels (multiple of 16,
+ * 16..256); H = attention heads (divides C); n_rbf = radial basis size
+ * (2..32); cutoff in the positions' length unit; feat_dtype = storage type of
+ * x and W_so2 (E2F_F32 or E2F_BF16). Arithmetic accumulates in fp32. */
+typedef struct {
+    int L;
+    int C;
+    int H;
+    int n_rbf;
+    float cutoff;
+    e2f_dtype feat_dtype;
+} e2f_attn_cfg;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* e2f_status_string(e2f_status s);
+
+/* ------------------------------------------------------------------------
+ * Neighbour list (cell list).
+ *
+ * The pages iterate over "j in N(i)" (gist.science Technical Summary 2.2)
+ * without saying how N(i) is found. This builds it with a linked-cell grid:
+ * j is a neighbour of i iff j != i, both lie in the same graph, and the
+ * minimum-image distance passes this exact fp32 test (round-to-nearest, no
+ * fused multiply-add):
+ *     dx = x_j - x_i;  periodic: dx -= box * rint(dx * (1/box))   per axis
+ *     d2 = (dx*dx + dy*dy) + dz*dz;   keep d2 < cutoff*cutoff
+ * Output is CSR: row_ptr[N+1], col[E]; rows in atom order, columns
+ * ascending within a row, self excluded, every pair listed in both
+ * directions.
+ *
+ *   pos        device, float [N*3] (x, y, z per atom), finite. Periodic
+ *              positions may lie outside the box; the image is implied.
+ *   n_atoms    N >= 0 (N = 0 gives row_ptr = {0} and E = 0).
+ *   box_host   host, float[3] orthorhombic box lengths, or NULL for open
+ *              boundaries. Requires cutoff <= min(box)/2.
+ *   cutoff     > 0.
+ *   graph_ptr  device, int32 [n_graphs+1], non-decreasing from 0 to N; or
+ *              NULL (all atoms form one graph; n_graphs ignored).
+ *   row_ptr    device, int32 [N+1], written.
+ *   col        device, int32 [col_capacity], written (first E entries).
+ *   n_pairs_host  host, written with E on success and on E2F_ERR_CAPACITY
+ *              (then row_ptr holds the offsets and col is not written;
+ *              grow col and call again). On E2F_ERR_NONFINITE or a bad
+ *              graph_ptr (E2F_ERR_INVALID_ARG) row_ptr is unspecified.
+ *   workspace  device, >= e2f_neighbors_workspace_size(...) bytes,
+ *              256-byte aligned. Contents need no initialisation.
+ * Synchronises `stream` (E is returned to the host). E must fit in int32.
+ * ---------------------------------------------------------------------- */
+size_t e2f_neighbors_workspace_size(int64_t n_atoms, const float* box_host,
+                                    float cutoff, int32_t n_graphs);
+
+e2f_status e2f_build_neighbors(const float* pos, int64_t n_atoms,
+                               const float* box_host, float cutoff,
+                               const int32_t* graph_ptr, int32_t n_graphs,
+                               int32_t* row_ptr, int32_t* col,
+                               int64_t col_capacity, int64_t* n_pairs_host,
+                               void* workspace, size_t ws_bytes,
+                               void* stream);
+
+/* ------------------------------------------------------------------------
+ * On-the-fly equivariant attention, forward (gist.science Technical
+ * Summary 2.1 EAAS: Lemma 4.1 and the re-indexing rule Eq. 13; 2.2:
+ * node-centric factorisation Eq. 6, streaming reduction over j in N(i),
+ * online softmax, no N x K x H x D tensor in HBM).
+ *
+ * For each node i and neighbour j (r = mic(x_j - x_i), d = |r|):
+ *   rho_k(d) = u(d) exp(-((d - k rc/(n_rbf-1)) / (rc/(n_rbf-1)))^2),
+ *              u(d) = (cos(pi d/rc) + 1)/2;   [g_v | g_a] = rho W_rad
+ *   h        = g_v[l, c] * x_j[l, m, c]
+ *   v_ij     = D(R)^T SO2(D(R) h),  R r = |r| z,  D = real Wigner-D blocks
+ *              (Y_l(R v) = D^l(R) Y_l(v)); SO2 per |m| block:
+ *              o[l3,+m] = sum_l1 A(m)[l3,l1] h[l1,+m] - B(m)[l3,l1] h[l1,-m]
+ *              o[l3,-m] = sum_l1 B(m)[l3,l1] h[l1,+m] + A(m)[l3,l1] h[l1,-m]
+ *   a_ij^h   = g_a^h <q_i^h, k_j^h> / sqrt(C/H),  q = W_q x[l=0], k = W_k x[l=0]
+ *   out_i[l,m,c] = sum_j softmax_j(a_ij^{h(c)}) v_ij[l,m,c],  h(c) = c/(C/H);
+ *   out_i = 0 when N(i) is empty.
+ *
+ *   cfg        host; shape and dtype (see e2f_attn_cfg).
+ *   pos        device, float [N*3]; box_host as for the neighbour build.
+ *   row_ptr, col  device CSR as produced by e2f_build_neighbors (any CSR
+ *              with rows in atom order is accepted; col entries in [0, N)).
+ *   n_pairs    E = row_ptr[N].
+ *   x          device, [N, (L+1)^2, C] of feat_dtype, 16-byte aligned.
+ *   W_q, W_k   device, float [C, C] row-major: q[c] = sum_c' W_q[c,c'] x[0,c'].
+ *   W_rad      device, float [n_rbf, (L+1)C + H] row-major; column l*C + c
+ *              is g_v[l, c], column (L+1)C + h is g_a^h.
+ *   W_so2      device, feat_dtype, packed: A(0), then A(m), B(m) for
+ *              m = 1..L; block m is a row-major square matrix of side
+ *              (L+1-m)C indexed [(l3, c_out), (l1, c_in)], l3, l1 = m..L.
+ *              85*C*C values at L = 4. 16-byte aligned.
+ *   out        device, float [N, (L+1)^2, C], written.
+ *   workspace  device, >= e2f_attention_workspace_size(...) bytes, 256-byte
+ *              aligned, contents need no initialisation. Holds the
+ *              repacked weights, per-node Q/K and softmax statistics and a
+ *              device status word; it must not be shared by calls in flight.
+ * Asynchronous: returns after enqueueing. Device-side failures (a bounded
+ * wait that ran out) are recorded in the workspace status word; read it
+ * with e2f_attention_status.
+ * ---------------------------------------------------------------------- */
+size_t e2f_attention_workspace_size(int64_t n_atoms, int64_t n_pairs,
+                                    const e2f_attn_cfg* cfg);
+
+e2f_status e2f_onfly_attention(const e2f_attn_cfg* cfg, const float* pos,
+                               int64_t n_atoms, const float* box_host,
+                               const int32_t* row_ptr, const int32_t* col,
+                               int64_t n_pairs, const void* x,
+                               const float* W_q, const float* W_k,
+                               const float* W_rad, const void* W_so2,
+                               float* out, void* workspace, size_t ws_bytes,
+                               void* stream);
+
+/* Synchronises `stream` and returns the device status recorded by the last
+ * e2f_onfly_attention call on this workspace (E2F_OK or E2F_ERR_TIMEOUT);
+ * each call clears the word when it starts. */
+e2f_status e2f_attention_status(void* workspace, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Edge-frame Wigner-D blocks, exposed for testing the rotation step alone
+ * (gist.science Technical Summary 2.1, "SO(3) -> SO(2) change of basis").
+ * For each unit-free direction r[e] (device, float [E*3], non-zero) writes
+ * the blocks D^l(R_e), l = 0..L, R_e the rotation the attention kernels use
+ * (R_e r = |r| z), row-major and concatenated: out[e*S + off(l) + a*(2l+1) + b]
+ * with off(l) = sum_{l'<l} (2l'+1)^2, S = off(L+1). Also writes R_e itself
+ * to frames[e*9 ...] (row-major) when frames is not NULL. Asynchronous.
+ * ---------------------------------------------------------------------- */
+e2f_status e2f_edge_wigner_blocks(const float* r, int64_t n_edges, int L,
+                                  float* out, float* frames, void* stream);
+
+/* Number of kernels this library has launched in this process (all
+ * devices, all entry points); lets a caller count launches in a region. */
+int64_t e2f_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* E2F_H */

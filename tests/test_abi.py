@@ -1,0 +1,85 @@
+"""CPU checks of the C-ABI boundary: the library loads, exports every symbol
+include/e2f.h declares, and rejects bad arguments before touching a GPU."""
+import ctypes
+
+import pytest
+
+import atomistic_cell_list_b200 as e2f
+
+
+def test_library_exports_every_declared_symbol():
+    h = e2f.lib()
+    syms = e2f.header_symbols()
+    assert {"e2f_build_neighbors", "e2f_onfly_attention", "e2f_neighbors_workspace_size",
+            "e2f_attention_workspace_size", "e2f_status_string"} <= set(syms)
+    for s in syms:
+        assert hasattr(h, s), s
+
+
+def test_status_strings():
+    for code in range(8):
+        assert e2f.status_string(code) and e2f.status_string(code) != "unknown status"
+    assert e2f.status_string(99) == "unknown status"
+
+
+def test_workspace_queries_are_host_only():
+    cfg = e2f.make_cfg(4, 128, 8, 16, 6.0, "bf16")
+    assert e2f.e2f_attention_workspace_size(30000, 2_700_000, cfg) > 0
+    assert e2f.e2f_neighbors_workspace_size(30000, [66.9, 66.9, 66.9], 6.0) > 0
+    assert e2f.e2f_neighbors_workspace_size(10000, None, 5.0, 256) > 0
+    bad = e2f.make_cfg(5, 128, 8, 16, 6.0, "bf16")
+    assert e2f.e2f_attention_workspace_size(10, 10, bad) == 0
+
+
+def _attn(cfg, **kw):
+    a = dict(pos=1, n=4, box=None, rp=1, col=1, npairs=4, x=16, wq=1, wk=1, wr=1, ws=16, out=16, wsp=256,
+             wsb=1 << 20)
+    a.update(kw)
+    v = lambda p: None if p is None else ctypes.c_void_p(p)
+    return e2f.lib().e2f_onfly_attention(ctypes.byref(cfg), v(a["pos"]), a["n"], a["box"], v(a["rp"]), v(a["col"]),
+                                         a["npairs"], v(a["x"]), v(a["wq"]), v(a["wk"]), v(a["wr"]), v(a["ws"]),
+                                         v(a["out"]), v(a["wsp"]), a["wsb"], None)
+
+
+@pytest.mark.parametrize("L,C,H,nr,code", [(5, 128, 8, 16, 2), (4, 120, 8, 16, 2), (4, 128, 3, 16, 2),
+                                           (4, 512, 8, 16, 2), (4, 128, 8, 1, 2), (4, 128, 8, 64, 2),
+                                           (-1, 128, 8, 16, 1), (4, 0, 8, 16, 1)])
+def test_attention_rejects_unsupported_shapes(L, C, H, nr, code):
+    cfg = e2f.e2f_attn_cfg(L, C, H, nr, 6.0, e2f.E2F_BF16)
+    assert _attn(cfg) == code
+
+
+def test_attention_argument_checks():
+    cfg = e2f.make_cfg(2, 16, 1, 16, 5.0, "f32")
+    assert _attn(cfg, pos=None) == 1
+    assert _attn(cfg, npairs=-1) == 1
+    assert _attn(cfg, x=8) == 4            # x not 16-byte aligned
+    assert _attn(cfg, wsp=128) == 4        # workspace not 256-byte aligned
+    assert _attn(cfg, wsb=16) == 1         # workspace too small
+    box = (ctypes.c_float * 3)(8.0, 8.0, 8.0)
+    assert _attn(cfg, box=ctypes.cast(box, ctypes.c_void_p)) == 1   # cutoff > box/2
+    bad_dtype = e2f.e2f_attn_cfg(2, 16, 1, 16, 5.0, 7)
+    assert _attn(bad_dtype) == 2
+    assert _attn(cfg, n=0) == 0            # nothing to do
+
+
+def test_neighbor_argument_checks():
+    f = e2f.lib().e2f_build_neighbors
+    n = ctypes.c_int64(0)
+    vp = ctypes.c_void_p
+    assert f(vp(16), 4, None, 5.0, None, 1, vp(16), vp(16), 10, None, vp(256), 1 << 20, None) == 1
+    assert f(vp(16), 4, None, -1.0, None, 1, vp(16), vp(16), 10, ctypes.byref(n), vp(256), 1 << 20, None) == 1
+    assert f(vp(16), -4, None, 5.0, None, 1, vp(16), vp(16), 10, ctypes.byref(n), vp(256), 1 << 20, None) == 1
+    box = (ctypes.c_float * 3)(9.0, 20.0, 20.0)
+    assert f(vp(16), 4, ctypes.cast(box, vp), 5.0, None, 1, vp(16), vp(16), 10, ctypes.byref(n), vp(256), 1 << 20,
+             None) == 1
+    assert f(vp(16), 4, None, 5.0, None, 1, vp(16), vp(16), 10, ctypes.byref(n), vp(128), 1 << 20, None) == 4
+    assert f(vp(16), 4, None, 5.0, vp(16), 0, vp(16), vp(16), 10, ctypes.byref(n), vp(256), 1 << 20, None) == 1
+    assert f(vp(16), 4, None, 5.0, None, 1, vp(16), vp(16), 10, ctypes.byref(n), vp(256), 16, None) == 1
+
+
+def test_wigner_entry_checks():
+    f = e2f.lib().e2f_edge_wigner_blocks
+    assert f(ctypes.c_void_p(16), 4, 5, ctypes.c_void_p(16), None, None) == 2
+    assert f(None, 4, 2, ctypes.c_void_p(16), None, None) == 1
+    assert f(None, 0, 2, None, None, None) == 0
