@@ -51,6 +51,7 @@ _SIGS = {
     "e2f_attention_status": (ctypes.c_int, [_vp, _sz, _vp]),
     "e2f_edge_wigner_blocks": (ctypes.c_int, [_vp, _i64, ctypes.c_int, _vp, _vp, _vp]),
     "e2f_launch_count": (_i64, []),
+    "e2f_attention_uses_tensor_cores": (ctypes.c_int, [ctypes.POINTER(e2f_attn_cfg)]),
 }
 
 
@@ -186,6 +187,10 @@ def e2f_edge_wigner_blocks(r: torch.Tensor, L: int, with_frames: bool = False, s
     _check(lib().e2f_edge_wigner_blocks(_ptr(r), n, int(L), _ptr(out), _ptr(fr), _stream(stream)),
            "e2f_edge_wigner_blocks")
     return (out, fr) if with_frames else out
+
+
+def e2f_attention_uses_tensor_cores(cfg: e2f_attn_cfg) -> bool:
+    return bool(lib().e2f_attention_uses_tensor_cores(ctypes.byref(cfg)))
 
 
 def e2f_launch_count() -> int:

@@ -7,6 +7,7 @@
 #include <cmath>
 
 #include "attention.cuh"
+#include "attention_tc.cuh"
 #include "common.cuh"
 
 namespace e2f {
@@ -19,7 +20,8 @@ using namespace e2f;
 namespace {
 
 struct AttnWs {
-    size_t o_status, o_q, o_k, o_wt, bytes;
+    size_t o_status, o_q, o_k, o_wt, o_tc, bytes;
+    bool tc;
 };
 
 AttnWs attn_layout(int64_t n_atoms, const e2f_attn_cfg& c) {
@@ -29,7 +31,9 @@ AttnWs attn_layout(int64_t n_atoms, const e2f_attn_cfg& c) {
     w.o_status = take(256);
     w.o_q = take(4 * (size_t)n_atoms * c.C);
     w.o_k = take(4 * (size_t)n_atoms * c.C);
-    w.o_wt = take(4 * so2_total(c.L, c.C));
+    w.tc = tc_supported(c.L, c.C, c.H, c.n_rbf, c.feat_dtype == E2F_BF16);
+    w.o_wt = w.tc ? 0 : take(4 * so2_total(c.L, c.C));
+    w.o_tc = w.tc ? take(tc_workspace_bytes(n_atoms, c.L, c.C, c.H)) : 0;
     w.bytes = o;
     return w;
 }
@@ -84,7 +88,8 @@ extern "C" e2f_status e2f_onfly_attention(const e2f_attn_cfg* cfg, const float* 
                 return E2F_ERR_INVALID_ARG;
     }
     if (reinterpret_cast<uintptr_t>(workspace) % 256 || reinterpret_cast<uintptr_t>(x) % 16 ||
-        reinterpret_cast<uintptr_t>(W_so2) % 16 || reinterpret_cast<uintptr_t>(out) % 16)
+        reinterpret_cast<uintptr_t>(W_so2) % 16 || reinterpret_cast<uintptr_t>(out) % 16 ||
+        reinterpret_cast<uintptr_t>(W_rad) % 16)
         return E2F_ERR_ALIGNMENT;
     AttnWs L = attn_layout(n_atoms, *cfg);
     if (ws_bytes < L.bytes) return E2F_ERR_INVALID_ARG;
@@ -106,9 +111,13 @@ extern "C" e2f_status e2f_onfly_attention(const e2f_attn_cfg* cfg, const float* 
     a.status = reinterpret_cast<int*>(ws + L.o_status);
     a.q = reinterpret_cast<float*>(ws + L.o_q);
     a.k = reinterpret_cast<float*>(ws + L.o_k);
-    a.Wt = reinterpret_cast<float*>(ws + L.o_wt);
+    a.Wt = L.tc ? nullptr : reinterpret_cast<float*>(ws + L.o_wt);
     E2F_CUDA_TRY(cudaMemsetAsync(a.status, 0, sizeof(int), stream));
-    E2F_CUDA_TRY(run_attention_simt(a, stream));
+    if (L.tc) {
+        E2F_CUDA_TRY(run_attention_tc(a, ws + L.o_tc, stream));
+    } else {
+        E2F_CUDA_TRY(run_attention_simt(a, stream));
+    }
     return E2F_OK;
 }
 
@@ -133,3 +142,8 @@ extern "C" e2f_status e2f_edge_wigner_blocks(const float* r, int64_t n_edges, in
 }
 
 extern "C" int64_t e2f_launch_count(void) { return (int64_t)g_launches.load(); }
+
+extern "C" int e2f_attention_uses_tensor_cores(const e2f_attn_cfg* cfg) {
+    if (check_cfg(cfg) != E2F_OK) return 0;
+    return tc_supported(cfg->L, cfg->C, cfg->H, cfg->n_rbf, cfg->feat_dtype == E2F_BF16) ? 1 : 0;
+}

@@ -1,0 +1,71 @@
+// Parameters of the tcgen05 attention path (see attention_tc.cu).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace e2f {
+
+constexpr int kMaxHeads = 16;   // tensor-core path: H <= 16
+constexpr int kMaxRbf = 32;
+constexpr int kMaxCtas = 160;   // persistent CTAs (one per SM; B200 has 148)
+
+struct StatsParams {
+    int n_atoms, C, H, n_rbf, G;
+    float cutoff;
+    Box box;
+    const float* pos;
+    const int32_t* row_ptr;
+    const int32_t* col;
+    const float* q;
+    const float* k;
+    const float* Wrad;
+    float* lse;
+};
+
+namespace tc {
+
+constexpr int kMaxGroups = 32;
+
+// One MMA group: up to two 128-row accumulators fed by one K loop.
+//   mu >= 1: o+ (TMEM cols 0-127) and o- (128-255) for rows [row0, row0+128)
+//            of A(mu)/B(mu) (tensor maps wa/wb); features x+ at xoff0, x- at xoff1
+//   mu == 0: rows row0 and row0b (-1: none) of A(0) (map wa); features at xoff0
+struct TcGroup {
+    int mu, row0, row0b, klen, xoff0, xoff1, wa, wb;
+};
+
+struct TcParams {
+    int C, H, n_rbf, G;
+    float cutoff;
+    Box box;
+    const float* pos;
+    const int32_t* row_ptr;
+    const int32_t* col;
+    const __nv_bfloat16* x;
+    const float* q;
+    const float* k;
+    const float* lse;
+    const float* Wrad;
+    const int32_t* part;
+    __nv_bfloat16* xs;
+    float* out;
+    int* status;
+    int n_groups;
+    TcGroup groups[kMaxGroups];
+};
+
+struct TcMaps {
+    CUtensorMap w[2 * kMaxL + 1];  // A(0), A(1), B(1), ..., A(L), B(L)
+    CUtensorMap xs;                // rotated-feature scratch
+};
+
+}  // namespace tc
+
+bool tc_supported(int L, int C, int H, int n_rbf, bool bf16);
+size_t tc_workspace_bytes(int64_t n_atoms, int L, int C, int H);
+
+}  // namespace e2f

@@ -286,7 +286,7 @@ def run_ours(args):
     peaks, peak_src = measured_peaks()
     F = so2_flops_per_edge(w.L, w.C)
     tflops = E * F / (ms_att * 1e-3) / 1e12
-    path = os.environ.get("E2F_REPORT_PATH", "simt")
+    path = "tensor" if e2f.e2f_attention_uses_tensor_cores(cfg) else "simt"
     if path == "simt":
         clk_max = float(peaks.get("sm_max_mhz", 1965.0))
         peak = 148 * 128 * 2 * clk_max * 1e6 / 1e12
@@ -298,7 +298,8 @@ def run_ours(args):
         peak = float(peaks["bf16_tflops"])
         roof = {"bound": "tensor", "achieved": tflops, "peak": peak, "unit": "TFLOP/s", "frac": tflops / peak,
                 "traffic": None, "peak_note": f"bf16 dense, {peak_src}"}
-    roof["kernel"] = "e2f_onfly_attention (all its launches)"
+    roof["kernel"] = ("k_attn_tc (tcgen05) + its O(N) pre-passes" if path == "tensor"
+                      else "k_attn_simt (fp32 CUDA cores) + its O(N) pre-passes")
     roof["traffic_note"] = "see profiles/ (ncu)"
 
     line = {"metric": METRIC, "value": world * E / (ms_step * 1e-3), "unit": "pairs/s", "n_gpus": world,

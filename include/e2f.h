@@ -128,7 +128,7 @@ e2f_status e2f_build_neighbors(const float* pos, int64_t n_atoms,
  *   x          device, [N, (L+1)^2, C] of feat_dtype, 16-byte aligned.
  *   W_q, W_k   device, float [C, C] row-major: q[c] = sum_c' W_q[c,c'] x[0,c'].
  *   W_rad      device, float [n_rbf, (L+1)C + H] row-major; column l*C + c
- *              is g_v[l, c], column (L+1)C + h is g_a^h.
+ *              is g_v[l, c], column (L+1)C + h is g_a^h. 16-byte aligned.
  *   W_so2      device, feat_dtype, packed: A(0), then A(m), B(m) for
  *              m = 1..L; block m is a row-major square matrix of side
  *              (L+1-m)C indexed [(l3, c_out), (l1, c_in)], l3, l1 = m..L.
@@ -138,6 +138,9 @@ e2f_status e2f_build_neighbors(const float* pos, int64_t n_atoms,
  *              aligned, contents need no initialisation. Holds the
  *              repacked weights, per-node Q/K and softmax statistics and a
  *              device status word; it must not be shared by calls in flight.
+ * Launch shape: the tensor-core kernel runs one persistent CTA per SM; the
+ * environment variable E2F_TC_MAX_CTAS (read at each call) caps that count,
+ * which lets tests give each CTA many tiles on small systems.
  * Asynchronous: returns after enqueueing. Device-side failures (a bounded
  * wait that ran out) are recorded in the workspace status word; read it
  * with e2f_attention_status.
@@ -153,6 +156,11 @@ e2f_status e2f_onfly_attention(const e2f_attn_cfg* cfg, const float* pos,
                                const float* W_rad, const void* W_so2,
                                float* out, void* workspace, size_t ws_bytes,
                                void* stream);
+
+/* 1 when e2f_onfly_attention runs this shape on the tcgen05 tensor-core
+ * kernel (bf16 features, L >= 1, C a multiple of 128 up to 256, H <= 16 and
+ * a multiple of 4), 0 when it runs the fp32 CUDA-core kernel. */
+int e2f_attention_uses_tensor_cores(const e2f_attn_cfg* cfg);
 
 /* Synchronises `stream` and returns the device status recorded by the last
  * e2f_onfly_attention call on this workspace (E2F_OK or E2F_ERR_TIMEOUT);

@@ -32,7 +32,7 @@ def test_workspace_queries_are_host_only():
 
 
 def _attn(cfg, **kw):
-    a = dict(pos=1, n=4, box=None, rp=1, col=1, npairs=4, x=16, wq=1, wk=1, wr=1, ws=16, out=16, wsp=256,
+    a = dict(pos=1, n=4, box=None, rp=1, col=1, npairs=4, x=16, wq=1, wk=1, wr=16, ws=16, out=16, wsp=256,
              wsb=1 << 20)
     a.update(kw)
     v = lambda p: None if p is None else ctypes.c_void_p(p)
@@ -83,3 +83,14 @@ def test_wigner_entry_checks():
     assert f(ctypes.c_void_p(16), 4, 5, ctypes.c_void_p(16), None, None) == 2
     assert f(None, 4, 2, ctypes.c_void_p(16), None, None) == 1
     assert f(None, 0, 2, None, None, None) == 0
+
+
+def test_tensor_core_dispatch_rule():
+    uses = lambda *a: e2f.e2f_attention_uses_tensor_cores(e2f.make_cfg(*a))
+    assert uses(4, 128, 8, 16, 6.0, "bf16")
+    assert uses(2, 256, 16, 16, 6.0, "bf16")
+    assert not uses(4, 128, 8, 16, 6.0, "f32")      # fp32 features: CUDA-core kernel
+    assert not uses(4, 64, 8, 16, 5.0, "bf16")      # C not a multiple of 128
+    assert not uses(2, 16, 1, 16, 5.0, "bf16")
+    assert not uses(0, 128, 8, 16, 5.0, "bf16")
+    assert not uses(4, 128, 2, 16, 5.0, "bf16")     # H not a multiple of 4
