@@ -52,6 +52,8 @@ _SIGS = {
     "e2f_edge_wigner_blocks": (ctypes.c_int, [_vp, _i64, ctypes.c_int, _vp, _vp, _vp]),
     "e2f_launch_count": (_i64, []),
     "e2f_attention_uses_tensor_cores": (ctypes.c_int, [ctypes.POINTER(e2f_attn_cfg)]),
+    "e2f_attention_debug_timers": (ctypes.c_int, [_vp, _sz, _i64, ctypes.POINTER(e2f_attn_cfg),
+                                                  ctypes.POINTER(_i64), ctypes.c_int, _vp]),
 }
 
 
@@ -191,6 +193,16 @@ def e2f_edge_wigner_blocks(r: torch.Tensor, L: int, with_frames: bool = False, s
 
 def e2f_attention_uses_tensor_cores(cfg: e2f_attn_cfg) -> bool:
     return bool(lib().e2f_attention_uses_tensor_cores(ctypes.byref(cfg)))
+
+
+def e2f_attention_debug_timers(workspace: torch.Tensor, n_atoms: int, cfg: e2f_attn_cfg, n_ctas: int = 160,
+                               stream=None):
+    """Per-CTA role cycle counters of the last tensor-core call (E2F_TC_TIMERS=1)."""
+    import numpy as np
+    buf = (_i64 * (16 * n_ctas))()
+    _check(lib().e2f_attention_debug_timers(_ptr(workspace), workspace.numel(), int(n_atoms), ctypes.byref(cfg), buf,
+                                            16 * n_ctas, _stream(stream)), "e2f_attention_debug_timers")
+    return np.frombuffer(buf, dtype=np.int64).reshape(n_ctas, 16).copy()
 
 
 def e2f_launch_count() -> int:

@@ -3,6 +3,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 
@@ -146,4 +147,18 @@ extern "C" int64_t e2f_launch_count(void) { return (int64_t)g_launches.load(); }
 extern "C" int e2f_attention_uses_tensor_cores(const e2f_attn_cfg* cfg) {
     if (check_cfg(cfg) != E2F_OK) return 0;
     return tc_supported(cfg->L, cfg->C, cfg->H, cfg->n_rbf, cfg->feat_dtype == E2F_BF16) ? 1 : 0;
+}
+
+extern "C" e2f_status e2f_attention_debug_timers(void* workspace, size_t ws_bytes, int64_t n_atoms,
+                                                const e2f_attn_cfg* cfg, int64_t* host_out, int n_values,
+                                                void* stream_) {
+    if (!workspace || !host_out || !cfg || n_values < 0) return E2F_ERR_INVALID_ARG;
+    AttnWs L = attn_layout(n_atoms, *cfg);
+    if (!L.tc || ws_bytes < L.bytes) return E2F_ERR_UNSUPPORTED;
+    const size_t n = std::min((size_t)n_values, kTcDebugBytes / 8);
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    E2F_CUDA_TRY(cudaMemcpyAsync(host_out, static_cast<char*>(workspace) + L.o_tc, n * 8, cudaMemcpyDeviceToHost,
+                                 stream));
+    E2F_CUDA_TRY(cudaStreamSynchronize(stream));
+    return E2F_OK;
 }

@@ -114,6 +114,15 @@ __device__ __forceinline__ bool wait(uint64_t* b, uint32_t parity, volatile int*
     }
 }
 
+// Same, adding the cycles spent waiting to `acc` (per-role wait counters).
+__device__ __forceinline__ bool wait_t(uint64_t* b, uint32_t parity, volatile int* abort_flag, int* status,
+                                       long long& acc) {
+    const long long c0 = clock64();
+    const bool r = wait(b, parity, abort_flag, status);
+    acc += clock64() - c0;
+    return r;
+}
+
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
     asm volatile(
         "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
@@ -178,10 +187,10 @@ __device__ __forceinline__ uint64_t sdesc_sw64(uint32_t saddr) {
     return d;
 }
 
-// kind::f16 instruction descriptor: D fp32, A and B bf16, both K-major,
-// M = 128, N = 128, optional negation of A.
-__host__ __device__ constexpr uint32_t idesc_bf16(bool neg_a) {
-    return (1u << 4) | (1u << 7) | (1u << 10) | ((neg_a ? 1u : 0u) << 13) | ((128u >> 3) << 17) |
+// kind::f16 instruction descriptor: D fp32, A and B fp16 (format 0), both
+// K-major, M = 128, N = 128, optional negation of A.
+__host__ __device__ constexpr uint32_t idesc_f16(bool neg_a) {
+    return (1u << 4) | (0u << 7) | (0u << 10) | ((neg_a ? 1u : 0u) << 13) | ((128u >> 3) << 17) |
            ((128u >> 4) << 24);
 }
 
@@ -216,7 +225,7 @@ __global__ void __launch_bounds__(256) k_softmax_stats(StatsParams P) {
         float3 r = edge_vec(P.pos, i, j, P.box);
         const float d = sqrtf(r.x * r.x + r.y * r.y + r.z * r.z);
         float rho[kMaxRbf];
-        for (int kb = 0; kb < P.n_rbf; ++kb) rho[kb] = rbf(d, kb, P.cutoff, P.n_rbf);
+        rbf_all(d, P.cutoff, P.n_rbf, rho);
 #pragma unroll
         for (int h = 0; h < kMaxHeads; ++h) {
             if (h < H) {
@@ -296,6 +305,90 @@ __global__ void __launch_bounds__(256) k_qk_tiled(const __nv_bfloat16* __restric
 }
 
 // ----------------------------------------------------------------------------
+// fp16 operand preparation. The tensor cores take fp16 (3 more mantissa bits
+// than bf16). Features are scaled by an exact power of two s so that
+// |s x| <= 1; the gate bound n_rbf * max|W_rad| then keeps every rotated,
+// gated value far inside the fp16 range (checked). The output is linear in x
+// through the value path, so multiplying the softmax weights by 1/s restores
+// it exactly.
+// ----------------------------------------------------------------------------
+__global__ void k_amax(const __nv_bfloat16* __restrict__ x, size_t n, const float* __restrict__ w, size_t nw,
+                       unsigned* amax) {
+    float mx = 0.f, mw = 0.f;
+    const size_t stride = (size_t)gridDim.x * blockDim.x;
+    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n / 8; i += stride) {
+        const uint4 u = reinterpret_cast<const uint4*>(x)[i];
+        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const float2 f = __bfloat1622float2(h[q]);
+            mx = fmaxf(mx, fmaxf(fabsf(f.x), fabsf(f.y)));
+        }
+    }
+    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < nw; i += stride) mw = fmaxf(mw, fabsf(w[i]));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        mw = fmaxf(mw, __shfl_xor_sync(0xffffffffu, mw, o));
+    }
+    if ((threadIdx.x & 31) == 0) {  // non-negative floats order like their bit patterns
+        atomicMax(amax, __float_as_uint(mx));
+        atomicMax(amax + 1, __float_as_uint(mw));
+    }
+}
+
+__global__ void k_make_scale(const unsigned* amax, int n_rbf, float* scale, int* status) {
+    const float mx = __uint_as_float(amax[0]), mw = __uint_as_float(amax[1]);
+    int e = 0;
+    if (mx > 0.f && isfinite(mx)) e = ilogbf(mx) + 1;  // s x in (-1, 1)
+    e = max(-60, min(60, e));
+    scale[0] = ldexpf(1.f, -e);
+    scale[1] = ldexpf(1.f, e);
+    // |rotated gated value| <= sqrt(2l+1) |s x| |g| <= 3 n_rbf max|W_rad|
+    if (!(isfinite(mx) && isfinite(mw)) || 3.f * n_rbf * mw > 16384.f) atomicExch(status, (int)E2F_ERR_UNSUPPORTED);
+}
+
+__global__ void k_x_to_f16(const __nv_bfloat16* __restrict__ x, size_t n, const float* __restrict__ scale,
+                           __half* __restrict__ out) {
+    const float s = scale[0];
+    const size_t stride = (size_t)gridDim.x * blockDim.x;
+    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n / 8; i += stride) {
+        const uint4 u = reinterpret_cast<const uint4*>(x)[i];
+        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+        uint4 v;
+        __half2* o = reinterpret_cast<__half2*>(&v);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const float2 f = __bfloat1622float2(h[q]);
+            o[q] = __floats2half2_rn(f.x * s, f.y * s);
+        }
+        reinterpret_cast<uint4*>(out)[i] = v;
+    }
+}
+
+__global__ void k_w_to_f16(const __nv_bfloat16* __restrict__ w, size_t n, __half* __restrict__ out) {
+    const size_t stride = (size_t)gridDim.x * blockDim.x;
+    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride)
+        out[i] = __float2half_rn(__bfloat162float(w[i]));
+}
+
+// value-gate weights transposed to [(L+1)C][16] fp16 (radial index innermost)
+__global__ void k_wrad_t(const float* __restrict__ Wrad, int n_rbf, int G, int Gv, __half* __restrict__ whT) {
+    const int t = blockIdx.x * blockDim.x + threadIdx.x;
+    if (t >= Gv * kTcMaxRbf) return;
+    const int n = t / kTcMaxRbf, k = t % kTcMaxRbf;
+    whT[t] = __float2half_rn(k < n_rbf ? Wrad[(size_t)k * G + n] : 0.f);
+}
+
+__device__ __forceinline__ void mma_16816(float* d, const uint32_t* a, const uint32_t* b) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+// ----------------------------------------------------------------------------
 // main kernel
 // ----------------------------------------------------------------------------
 constexpr int kTileE = 128;
@@ -304,21 +397,44 @@ constexpr int kNS = 3;                        // ring stages
 constexpr int kSlot = kTileE * kKS * 2;       // 8 KB per operand tile
 constexpr int kStage = 4 * kSlot;
 constexpr int kThreads = 320;
+constexpr int kChunk = 16;                    // epilogue: edges per TMEM load
+constexpr int kStageD = 20480;                // epilogue Wigner staging buffer (bytes)
 
-template <int L>
-struct Smem {
-    static constexpr int WS = wig_size(L);
-    static constexpr int WSP = (WS + 7) & ~7;                 // padded stride (halves)
-    static constexpr size_t ring = 0;
-    static constexpr size_t dbuf = ring + (size_t)kNS * kStage;
-    static constexpr size_t pbuf = dbuf + 2ull * kTileE * WSP * 2;
-    static constexpr size_t nid = pbuf + 2ull * kTileE * kMaxHeads * 4;
-    static constexpr size_t jn = nid + 2ull * kTileE * 4;
-    static constexpr size_t rho = jn + 2ull * kTileE * 4;
-    static constexpr size_t bars = rho + (size_t)kTileE * kMaxRbf * 4;
-    static constexpr int n_bars = 2 * kNS + 9;
-    static constexpr size_t misc = bars + n_bars * 8;
-    static constexpr size_t total = misc + 64;
+// Wigner blocks of an edge in "pair" form: for each degree l and each
+// |m| = mu <= l the 2l+1 pairs (D^l[+mu][n], D^l[-mu][n]) (padded to 2l+2).
+// A pair rotates into both x~[+mu] and x~[-mu] (producer) and rotates o+ and
+// o- back (epilogue). Pairs of block (l, mu) start at dpair_off(l, mu).
+__host__ __device__ constexpr int dpair_block(int l) { return (l + 1) * (2 * l + 2); }
+__host__ __device__ constexpr int dpair_off(int l, int mu) {
+    int o = 0;
+    for (int k = 0; k < l; ++k) o += dpair_block(k);
+    return o + mu * (2 * l + 2);
+}
+__host__ __device__ constexpr int dpairs(int L) { return dpair_off(L + 1, 0); }  // 110 at L = 4
+// Global scratch, per tile buffer, block-major: block (l, mu) holds 128 edges
+// x (2l+2) float2, so the epilogue fetches one group's slice in one bulk copy.
+__host__ __device__ constexpr size_t dglob_floats() { return 2ull * kTileE * dpairs(kMaxL); }
+__host__ __device__ constexpr size_t dglob_block(int l, int mu) { return 2ull * kTileE * dpair_off(l, mu); }
+
+// Shared memory layout (bytes), shared by host (size) and device (offsets).
+struct SmemLayout {
+    size_t ring, dstage, dph, pbuf, nid, jn, segm, rpw, rho, bars, misc, total;
+    __host__ __device__ SmemLayout(int L, int H, int n_rbf) {
+        size_t o = 0;
+        ring = o;   o += (size_t)kNS * kStage;
+        dstage = o; o += 2ull * kStageD;
+        dph = o;    o += (size_t)kTileE * dpairs(L) * 4;
+        pbuf = o;   o += 2ull * kTileE * H * 4;
+        nid = o;    o += 2ull * kTileE * 4;
+        jn = o;     o += 2ull * kTileE * 4;
+        segm = o;   o += 2ull * (kTileE / kChunk) * 4;
+        rpw = o;    o += (size_t)kTileE * 4;
+        rho = o;    o += (size_t)kTileE * kTcMaxRbf * 2;
+        o = (o + 7) & ~size_t(7);
+        bars = o;   o += (2 * kNS + 11) * 8;
+        misc = o;   o += 64;
+        total = o;
+    }
 };
 
 __device__ __forceinline__ int kpos(int l1, int m, int L, int C) {
@@ -331,102 +447,232 @@ __device__ __forceinline__ int kpos(int l1, int m, int L, int C) {
     return off + (m > 0 ? 0 : nm) + (l1 - mu) * C;
 }
 
-template <int L, int L3>
-__device__ __forceinline__ void epi_flush(float* out, int node, int c, int C, const float* acc) {
-    constexpr int K = n_sh(L);
-    float* o = out + ((size_t)node * K + L3 * L3) * C + c;
-#pragma unroll
-    for (int n = 0; n < 2 * L3 + 1; ++n) o[(size_t)n * C] += acc[n];
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     smem_u32(dst)),
+                 "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
 }
 
-// One accumulator pair (o+, o-) of block |m| = mu >= 1, or a single
-// accumulator (m = 0, pair = false). Thread = output feature (L3, c).
-template <int L, int L3>
-__device__ __forceinline__ void epi_group(uint32_t tacc, bool pair, int mu, int c, int h, int H, const __half* Db,
-                                          const float* pb, const int* nb, float* out, int C) {
-    constexpr int WSP = Smem<L>::WSP;
-    constexpr int W3 = 2 * L3 + 1;
-    float acc[W3];
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr)
+        : "memory");
 #pragma unroll
-    for (int n = 0; n < W3; ++n) acc[n] = 0.f;
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void tmem_ld_16x256(uint32_t taddr, uint32_t* r) {
+    asm volatile("tcgen05.ld.sync.aligned.16x256b.x1.b32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(taddr)
+                 : "memory");
+}
+
+__device__ __forceinline__ uint32_t pack_h2(float a, float b) {
+    __half2 h = __floats2half2_rn(a, b);
+    return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// Epilogue of one accumulator pair (o+ at tacc, o- at tacc + 128) or one
+// accumulator (SIGNS = 1) holding output rows (l3, channel) for the tile's
+// 128 edges, on mma.sync: per 16-edge chunk and 8 channels,
+//     acc[m'][c] += sum_e D_e[+mu][m'] y+[e][c] + D_e[-mu][m'] y-[e][c],
+//     y[e][c] = p_e^{head(c)} o[c][e],
+// i.e. the rotate-back D^T of the |m| = mu rows weighted by the softmax and
+// summed over the node's edges. A = Wigner rows (m' padded to 16, from the
+// staged pairs), B = p * o straight from tcgen05.ld.16x256b (whose thread
+// layout is the mma B/D fragment layout), D = fp32 accumulators. Node sums
+// go to out with fire-and-forget reductions at segment ends: one thread owns
+// each (node, l3, m', c) element, so the additions happen in program order.
+// Warp w covers channels cbase..cbase+31 (TMEM lanes 32w..32w+31).
+template <int SIGNS>
+__device__ __noinline__ void epi_mma(uint32_t tacc, int l3, int cbase, int H, int dh, int K, int C,
+                                     const float2* __restrict__ Ds, const float* __restrict__ pb,
+                                     const int* __restrict__ nb, const uint32_t* __restrict__ segm,
+                                     float* __restrict__ out) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
+    const int W3 = 2 * l3 + 1, DS = 2 * l3 + 2;
+    float acc[2][2][4];  // [lane half][n-tile lo/hi][fragment]
+#pragma unroll
+    for (int a = 0; a < 2; ++a)
+#pragma unroll
+        for (int b2 = 0; b2 < 2; ++b2)
+#pragma unroll
+            for (int r = 0; r < 4; ++r) acc[a][b2][r] = 0.f;
     int cur = -1;
-    const int rp = (L3 + mu) * W3, rm = (L3 - mu) * W3;
+    // heads of the B columns this thread loads: channel cbase + 16*hh + 8*lh + g
+    int hd[2][2];
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+        for (int lh = 0; lh < 2; ++lh) hd[hh][lh] = (cbase + 16 * hh + 8 * lh + g) / dh;
+
+    auto flush = [&]() {
+        if (cur < 0) return;
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+            for (int lh = 0; lh < 2; ++lh)
+#pragma unroll
+                for (int r = 0; r < 4; ++r) {
+                    const int mp = g + ((r >> 1) << 3);
+                    if (mp < W3) {
+                        const int c = cbase + 16 * hh + 8 * lh + 2 * q + (r & 1);
+                        atomicAdd(out + ((size_t)cur * K + l3 * l3 + mp) * C + c, acc[hh][lh][r]);
+                    }
+                    acc[hh][lh][r] = 0.f;
+                }
+    };
+
 #pragma unroll 1
-    for (int ch = 0; ch < kTileE / 32; ++ch) {
-        float vp[32], vm[32];
-        tmem_ld32(tacc + ch * 32, vp);
-        if (pair) tmem_ld32(tacc + 128 + ch * 32, vm);
+    for (int ch = 0; ch < kTileE / 16; ++ch) {
+        const int e0 = ch * 16;
+        // o values: [sign][lane half][edge half][4]: (c_lo,e), (c_lo,e+1), (c_hi,e), (c_hi,e+1)
+        uint32_t ov[SIGNS][2][2][4];
+#pragma unroll
+        for (int s2 = 0; s2 < SIGNS; ++s2)
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+                for (int eh = 0; eh < 2; ++eh)
+                    tmem_ld_16x256(tacc + s2 * 128 + ((uint32_t)(16 * hh) << 16) + e0 + 8 * eh, ov[s2][hh][eh]);
         tmem_wait_ld();
-#pragma unroll
-        for (int q = 0; q < 32; ++q) {
-            const int e = ch * 32 + q;
-            const int node = nb[e];
-            if (node != cur) {
-                if (cur >= 0) epi_flush<L, L3>(out, cur, c, C, acc);
-#pragma unroll
-                for (int n = 0; n < W3; ++n) acc[n] = 0.f;
-                cur = node;
-            }
-            if (node < 0) continue;
-            const float p = pb[e * kMaxHeads + h];
-            const __half* D = Db + (size_t)e * WSP + wig_off(L3);
-            const float yp = p * vp[q];
-            if (pair) {
-                const float ym = p * vm[q];
-#pragma unroll
-                for (int n = 0; n < W3; ++n)
-                    acc[n] = fmaf(__half2float(D[rp + n]), yp, fmaf(__half2float(D[rm + n]), ym, acc[n]));
-            } else {
-#pragma unroll
-                for (int n = 0; n < W3; ++n) acc[n] = fmaf(__half2float(D[rp + n]), yp, acc[n]);
+        // this thread's four edges: e0 + 2q, +1, e0 + 8 + 2q, +1
+        const int ea = e0 + 2 * q, eb = e0 + 8 + 2 * q;
+        // Wigner A fragments per sign: rows m' = g (a0, a2) and g + 8 (a1, a3)
+        uint32_t af[SIGNS][4];
+        {
+            const bool r0 = g < W3, r1 = g + 8 < W3;
+            const float2 z = make_float2(0.f, 0.f);
+            const float2 d00 = r0 ? Ds[ea * DS + g] : z, d01 = r0 ? Ds[(ea + 1) * DS + g] : z;
+            const float2 d10 = r1 ? Ds[ea * DS + g + 8] : z, d11 = r1 ? Ds[(ea + 1) * DS + g + 8] : z;
+            const float2 d20 = r0 ? Ds[eb * DS + g] : z, d21 = r0 ? Ds[(eb + 1) * DS + g] : z;
+            const float2 d30 = r1 ? Ds[eb * DS + g + 8] : z, d31 = r1 ? Ds[(eb + 1) * DS + g + 8] : z;
+            af[0][0] = pack_h2(d00.x, d01.x); af[0][1] = pack_h2(d10.x, d11.x);
+            af[0][2] = pack_h2(d20.x, d21.x); af[0][3] = pack_h2(d30.x, d31.x);
+            if (SIGNS == 2) {
+                af[SIGNS - 1][0] = pack_h2(d00.y, d01.y); af[SIGNS - 1][1] = pack_h2(d10.y, d11.y);
+                af[SIGNS - 1][2] = pack_h2(d20.y, d21.y); af[SIGNS - 1][3] = pack_h2(d30.y, d31.y);
             }
         }
+        // softmax weights of the four edges for the B columns' heads
+        float pw[2][2][4];
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+            for (int lh = 0; lh < 2; ++lh) {
+                const int h = hd[hh][lh];
+                pw[hh][lh][0] = pb[ea * H + h];
+                pw[hh][lh][1] = pb[(ea + 1) * H + h];
+                pw[hh][lh][2] = pb[eb * H + h];
+                pw[hh][lh][3] = pb[(eb + 1) * H + h];
+            }
+        // segments of this chunk: bit k = edge e0 + k starts a node
+        uint32_t bits = segm[ch];
+        int lo = 0;
+        if (bits & 1u) {
+            flush();
+            cur = nb[e0];
+        }
+        bits &= ~1u;
+        while (true) {
+            const int hi = bits ? __ffs(bits) - 1 : 16;
+            // edge masks of this thread's four edges for [lo, hi)
+            const float m0 = (2 * q >= lo && 2 * q < hi) ? 1.f : 0.f;
+            const float m1 = (2 * q + 1 >= lo && 2 * q + 1 < hi) ? 1.f : 0.f;
+            const float m2 = (8 + 2 * q >= lo && 8 + 2 * q < hi) ? 1.f : 0.f;
+            const float m3 = (9 + 2 * q >= lo && 9 + 2 * q < hi) ? 1.f : 0.f;
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+                for (int lh = 0; lh < 2; ++lh) {
+                    const float* pwv = pw[hh][lh];
+#pragma unroll
+                    for (int s2 = 0; s2 < SIGNS; ++s2) {
+                        const uint32_t* va = ov[s2][hh][0];
+                        const uint32_t* vb = ov[s2][hh][1];
+                        uint32_t bf[2];
+                        bf[0] = pack_h2(pwv[0] * m0 * __uint_as_float(va[2 * lh]),
+                                        pwv[1] * m1 * __uint_as_float(va[2 * lh + 1]));
+                        bf[1] = pack_h2(pwv[2] * m2 * __uint_as_float(vb[2 * lh]),
+                                        pwv[3] * m3 * __uint_as_float(vb[2 * lh + 1]));
+                        mma_16816(acc[hh][lh], af[s2], bf);
+                    }
+                }
+            if (hi == 16) break;
+            flush();
+            cur = nb[e0 + hi];
+            lo = hi;
+            bits &= bits - 1;
+        }
     }
-    if (cur >= 0) epi_flush<L, L3>(out, cur, c, C, acc);
-    (void)H;
+    flush();
 }
 
-template <int L>
-__device__ __forceinline__ void epi_dispatch(int l3, uint32_t tacc, bool pair, int mu, int c, int h, int H,
-                                             const __half* Db, const float* pb, const int* nb, float* out, int C) {
-    switch (l3) {
-        case 0: epi_group<L, 0>(tacc, pair, mu, c, h, H, Db, pb, nb, out, C); break;
-        case 1: if constexpr (L >= 1) epi_group<L, 1>(tacc, pair, mu, c, h, H, Db, pb, nb, out, C); break;
-        case 2: if constexpr (L >= 2) epi_group<L, 2>(tacc, pair, mu, c, h, H, Db, pb, nb, out, C); break;
-        case 3: if constexpr (L >= 3) epi_group<L, 3>(tacc, pair, mu, c, h, H, Db, pb, nb, out, C); break;
-        case 4: if constexpr (L >= 4) epi_group<L, 4>(tacc, pair, mu, c, h, H, Db, pb, nb, out, C); break;
-        default: break;
+// Wigner slice(s) a group's epilogue needs, by block (l, mu): returns bytes
+// queued on `bar` into staging buffer `dst`.
+__device__ __forceinline__ uint32_t stage_group_pairs(const TcGroup& g, int C, const float* Dglob, uint8_t* dst,
+                                                      uint64_t* bar) {
+    if (g.mu > 0) {
+        const int l3 = g.mu + g.row0 / C;
+        const uint32_t bytes = (uint32_t)kTileE * (2 * l3 + 2) * 8;
+        mbar_arrive_tx(bar, bytes);
+        bulk_load(dst, Dglob + dglob_block(l3, g.mu), bytes, bar);
+        return bytes;
     }
+    const int la = g.row0 / C;
+    const uint32_t ba = (uint32_t)kTileE * (2 * la + 2) * 8;
+    uint32_t bb = 0;
+    int lb = -1;
+    if (g.row0b >= 0) {
+        lb = g.row0b / C;
+        bb = (uint32_t)kTileE * (2 * lb + 2) * 8;
+    }
+    mbar_arrive_tx(bar, ba + bb);
+    bulk_load(dst, Dglob + dglob_block(la, 0), ba, bar);
+    if (lb >= 0) bulk_load(dst + ba, Dglob + dglob_block(lb, 0), bb, bar);
+    return ba + bb;
 }
 
 template <int L>
 __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__ TcParams P,
                                                          const __grid_constant__ TcMaps T) {
-    using S = Smem<L>;
     constexpr int K = n_sh(L);
-    constexpr int WS = S::WS, WSP = S::WSP;
+    constexpr int WS = wig_size(L);
+    constexpr int NPAIR = dpairs(L);
+    const int C = P.C, H = P.H, dh = C / H, G = P.G, NR = P.n_rbf;
+    const SmemLayout S(L, H, NR);
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // operand tiles need 1024-byte alignment in the shared window
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    uint8_t* ring = smem + S::ring;
-    __half* dbuf = reinterpret_cast<__half*>(smem + S::dbuf);
-    float* pbuf = reinterpret_cast<float*>(smem + S::pbuf);
-    int* nid = reinterpret_cast<int*>(smem + S::nid);
-    int* jn = reinterpret_cast<int*>(smem + S::jn);
-    float* rho = reinterpret_cast<float*>(smem + S::rho);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::bars);
+    uint8_t* ring = smem + S.ring;
+    uint8_t* dstage = smem + S.dstage;
+    __half2* dph = reinterpret_cast<__half2*>(smem + S.dph);
+    float* pbuf = reinterpret_cast<float*>(smem + S.pbuf);
+    int* nid = reinterpret_cast<int*>(smem + S.nid);
+    int* jn = reinterpret_cast<int*>(smem + S.jn);
+    uint32_t* segm = reinterpret_cast<uint32_t*>(smem + S.segm);
+    int* rpw = reinterpret_cast<int*>(smem + S.rpw);
+    __half* rho = reinterpret_cast<__half*>(smem + S.rho);  // [128][16] radial basis, fp16
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S.bars);
     uint64_t* full = bars;
     uint64_t* empty = bars + kNS;
     uint64_t* tfull = bars + 2 * kNS;
     uint64_t* tempty = tfull + 2;
     uint64_t* xready = tempty + 2;
     uint64_t* xfree = xready + 2;
-    uint64_t* fin = xfree + 2;
-    uint32_t* tmem_sm = reinterpret_cast<uint32_t*>(smem + S::misc);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + S::misc + 8);
+    uint64_t* dbar = xfree + 2;   // epilogue Wigner staging, per buffer
+    uint64_t* fin = dbar + 2;
+    uint32_t* tmem_sm = reinterpret_cast<uint32_t*>(smem + S.misc);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + S.misc + 8);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int C = P.C, H = P.H, dh = C / H, G = P.G;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kNS; ++s) { mbar_init(full + s, 1); mbar_init(empty + s, 1); }
@@ -435,6 +681,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
             mbar_init(tempty + b, 128);
             mbar_init(xready + b, 128);
             mbar_init(xfree + b, 128);
+            mbar_init(dbar + b, 1);
         }
         mbar_init(fin, 1);
         *abort_flag = 0;
@@ -458,27 +705,64 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
         // ---------------- producer ----------------
         const int p = threadIdx.x - 128;
         const float inv_sqrt_dh = rsqrtf((float)dh);
+        const float inv_s = P.scale[1];
         const int CG = C / 8;
+        const int Gv = (L + 1) * C;
+        __half* gs = P.gscr + (size_t)blockIdx.x * kTileE * Gv;
+        int nbase = n_begin;
         const size_t KT = (size_t)K * C;
+        long long w_free = 0, c_p1 = 0, c_p2 = 0;
+        const long long c_start = clock64();
         for (int t = 0; t < ntiles; ++t) {
             const int b = t & 1;
-            const bool okw = (t < 2) || wait(xfree + b, ((t - 2) >> 1) & 1, abort_flag, P.status);
+            const bool okw = (t < 2) || wait_t(xfree + b, ((t - 2) >> 1) & 1, abort_flag, P.status, w_free);
             if (!bar_and(1, 128, okw)) break;
+            const long long c_a = clock64();
             const int e0 = e_begin + t * kTileE;
             const int ne = min(kTileE, e_end - e0);
-            __half* Db = dbuf + (size_t)b * kTileE * WSP;
-            // P1: one edge per thread
+            // window of row_ptr after the node of the tile's first edge
             {
-                __half* Dp = Db + (size_t)p * WSP;
+                int nb0;
+                if (t == 0) {
+                    int lo = n_begin, hi = n_end - 1;
+                    while (lo < hi) {
+                        int mid = (lo + hi + 1) >> 1;
+                        if (P.row_ptr[mid] <= e0) lo = mid; else hi = mid - 1;
+                    }
+                    nb0 = lo;
+                } else {
+                    nb0 = nid[(b ^ 1) * kTileE + kTileE - 1];  // node of edge e0 - 1
+                }
+                nbase = nb0;
+                const int n = nbase + 1 + p;
+                rpw[p] = (n <= n_end) ? P.row_ptr[n] : 0x7fffffff;
+            }
+            asm volatile("bar.sync 1, 128;" ::: "memory");
+            float* Dg = P.dscr + (size_t)(blockIdx.x * 2 + b) * dglob_floats();
+            // P1: one edge per thread: frame, Wigner pairs (shared f16 copy for
+            // the rotation below, global fp32 copy for the epilogue), softmax weight
+            {
+                __half2* Dh = dph + (size_t)p * NPAIR;
                 if (p < ne) {
                     const int e = e0 + p;
                     const int j = P.col[e];
-                    int lo = n_begin, hi = n_end - 1;  // node i: last n with row_ptr[n] <= e
-                    while (lo < hi) {
-                        int mid = (lo + hi + 1) >> 1;
-                        if (P.row_ptr[mid] <= e) lo = mid; else hi = mid - 1;
+                    // node i: last n with row_ptr[n] <= e = nbase + #{k: rpw[k] <= e}
+                    int i;
+                    if (e < rpw[kTileE - 1]) {
+                        int lo = 0, hi = kTileE;  // first k with rpw[k] > e
+                        while (lo < hi) {
+                            const int mid = (lo + hi) >> 1;
+                            if (rpw[mid] <= e) lo = mid + 1; else hi = mid;
+                        }
+                        i = nbase + lo;
+                    } else {  // more than 128 nodes in reach (runs of empty rows): global search
+                        int lo = nbase, hi = n_end - 1;
+                        while (lo < hi) {
+                            int mid = (lo + hi + 1) >> 1;
+                            if (P.row_ptr[mid] <= e) lo = mid; else hi = mid - 1;
+                        }
+                        i = lo;
                     }
-                    const int i = lo;
                     float3 r = edge_vec(P.pos, i, j, P.box);
                     const float d = sqrtf(r.x * r.x + r.y * r.y + r.z * r.z);
                     float R[3][3];
@@ -486,33 +770,99 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
                     float D[WS];
                     wigner_blocks<L>(R, D);
 #pragma unroll
-                    for (int a = 0; a < WS; ++a) Dp[a] = __float2half_rn(D[a]);
-                    float rr[kMaxRbf];
-                    for (int kb = 0; kb < P.n_rbf; ++kb) {
-                        rr[kb] = rbf(d, kb, P.cutoff, P.n_rbf);
-                        rho[p * kMaxRbf + kb] = rr[kb];
+                    for (int l = 0; l <= L; ++l) {
+                        const int w = 2 * l + 1;
+                        const float* Dl = D + wig_off(l);
+#pragma unroll
+                        for (int mu = 0; mu <= l; ++mu) {
+                            float4* gq = reinterpret_cast<float4*>(Dg + dglob_block(l, mu) + (size_t)p * 2 * (2 * l + 2));
+#pragma unroll
+                            for (int n = 0; n < w; n += 2) {
+                                const float a0 = Dl[(l + mu) * w + n], b0 = Dl[(l - mu) * w + n];
+                                const float a1 = (n + 1 < w) ? Dl[(l + mu) * w + n + 1] : 0.f;
+                                const float b1 = (n + 1 < w) ? Dl[(l - mu) * w + n + 1] : 0.f;
+                                gq[n / 2] = make_float4(a0, b0, a1, b1);
+                                Dh[dpair_off(l, mu) + n] = __floats2half2_rn(a0, b0);
+                                Dh[dpair_off(l, mu) + n + 1] = __floats2half2_rn(a1, b1);
+                            }
+                        }
+                    }
+                    float rr[kTcMaxRbf];
+                    rbf_all(d, P.cutoff, NR, rr);
+                    for (int kb = 0; kb < kTcMaxRbf; ++kb) {
+                        if (kb >= NR) rr[kb] = 0.f;
+                        rho[p * kTcMaxRbf + kb] = __float2half_rn(rr[kb]);
                     }
                     for (int h = 0; h < H; ++h) {
-                        float a = edge_logit(rr, P.n_rbf, P.Wrad, G, G - H + h, P.q + (size_t)i * C + h * dh,
+                        float a = edge_logit(rr, NR, P.Wrad, G, G - H + h, P.q + (size_t)i * C + h * dh,
                                              P.k + (size_t)j * C + h * dh, dh, inv_sqrt_dh);
-                        pbuf[(b * kTileE + p) * kMaxHeads + h] = expf(a - P.lse[(size_t)i * H + h]);
+                        pbuf[(b * kTileE + p) * H + h] = expf(a - P.lse[(size_t)i * H + h]) * inv_s;
                     }
                     nid[b * kTileE + p] = i;
                     jn[b * kTileE + p] = j;
                 } else {
-                    for (int a = 0; a < WS; ++a) Dp[a] = __float2half_rn(0.f);
-                    for (int kb = 0; kb < P.n_rbf; ++kb) rho[p * kMaxRbf + kb] = 0.f;
-                    for (int h = 0; h < H; ++h) pbuf[(b * kTileE + p) * kMaxHeads + h] = 0.f;
+#pragma unroll
+                    for (int l = 0; l <= L; ++l)
+#pragma unroll
+                        for (int mu = 0; mu <= l; ++mu) {
+                            float4* gq = reinterpret_cast<float4*>(Dg + dglob_block(l, mu) + (size_t)p * 2 * (2 * l + 2));
+                            for (int n = 0; n < 2 * l + 1; n += 2) gq[n / 2] = make_float4(0.f, 0.f, 0.f, 0.f);
+                        }
+                    for (int a = 0; a < NPAIR; ++a) Dh[a] = __floats2half2_rn(0.f, 0.f);
+                    for (int kb = 0; kb < kTcMaxRbf; ++kb) rho[p * kTcMaxRbf + kb] = __float2half_rn(0.f);
+                    for (int h = 0; h < H; ++h) pbuf[(b * kTileE + p) * H + h] = 0.f;
                     nid[b * kTileE + p] = -1;
                     jn[b * kTileE + p] = 0;
                 }
             }
             asm volatile("bar.sync 1, 128;" ::: "memory");
-            // P2: rotated, gated features -> scratch row (e), all |m| blocks
-            __nv_bfloat16* xrow0 = P.xs + ((size_t)(blockIdx.x * 2 + b) * kTileE) * KT;
+            if (p < kTileE / kChunk) {  // segment starts per 16-edge chunk
+                uint32_t m = 0;
+                for (int q = 0; q < kChunk; ++q) {
+                    const int e = p * kChunk + q;
+                    if (e == 0 || nid[b * kTileE + e] != nid[b * kTileE + e - 1]) m |= 1u << q;
+                }
+                segm[b * (kTileE / kChunk) + p] = m;
+            }
+            // P1.5: value gate g[e][n] = rho[e] . W_rad[:, n] for the tile (128 x (L+1)C), one k=16
+            // mma.sync per 16 edges x 8 columns; warp pw takes edge blocks 2pw and 2pw+1
+            {
+                const int pw = warp - 4, g8 = lane >> 2, t4 = lane & 3;
+                uint32_t af[2][4];
+#pragma unroll
+                for (int mb = 0; mb < 2; ++mb) {
+                    const int r0 = (2 * pw + mb) * 16 + g8;
+                    const __half* rr0 = rho + r0 * kTcMaxRbf + 2 * t4;
+                    af[mb][0] = *reinterpret_cast<const uint32_t*>(rr0);
+                    af[mb][1] = *reinterpret_cast<const uint32_t*>(rr0 + 8 * kTcMaxRbf);
+                    af[mb][2] = *reinterpret_cast<const uint32_t*>(rr0 + 8);
+                    af[mb][3] = *reinterpret_cast<const uint32_t*>(rr0 + 8 * kTcMaxRbf + 8);
+                }
+#pragma unroll 4
+                for (int n0 = 0; n0 < Gv; n0 += 8) {
+                    const __half* wb = P.whT + (size_t)(n0 + g8) * kTcMaxRbf + 2 * t4;
+                    uint32_t bf[2];
+                    bf[0] = __ldg(reinterpret_cast<const unsigned int*>(wb));
+                    bf[1] = __ldg(reinterpret_cast<const unsigned int*>(wb + 8));
+#pragma unroll
+                    for (int mb = 0; mb < 2; ++mb) {
+                        float acc4[4] = {0.f, 0.f, 0.f, 0.f};
+                        mma_16816(acc4, af[mb], bf);
+                        const int e = (2 * pw + mb) * 16 + g8;
+                        *reinterpret_cast<__half2*>(gs + (size_t)e * Gv + n0 + 2 * t4) = __floats2half2_rn(acc4[0], acc4[1]);
+                        *reinterpret_cast<__half2*>(gs + (size_t)(e + 8) * Gv + n0 + 2 * t4) =
+                            __floats2half2_rn(acc4[2], acc4[3]);
+                    }
+                }
+            }
+            asm volatile("bar.sync 1, 128;" ::: "memory");
+            const long long c_b = clock64();
+            c_p1 += c_b - c_a;
+            // P2: rotated, gated features -> scratch row (e), all |m| blocks (fp16, packed math)
+            __half* xrow0 = P.xs + ((size_t)(blockIdx.x * 2 + b) * kTileE) * KT;
             for (int it = p; it < kTileE * CG; it += 128) {
                 const int e = it / CG, c0 = (it % CG) * 8;
-                __nv_bfloat16* xrow = xrow0 + (size_t)e * KT;
+                __half* xrow = xrow0 + (size_t)e * KT;
                 if (e >= ne) {
                     const uint4 z = make_uint4(0, 0, 0, 0);
 #pragma unroll
@@ -523,65 +873,64 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
                     continue;
                 }
                 const int j = jn[b * kTileE + e];
-                const float* rr = rho + e * kMaxRbf;
-                const __half* De = Db + (size_t)e * WSP;
+                const __half2* De = dph + (size_t)e * NPAIR;
+                // all (L+1)^2 rows of x_j for these 8 channels in flight at once
+                uint4 raw[K];
+                const __half* xj = P.x + (size_t)j * K * C + c0;
+#pragma unroll
+                for (int n = 0; n < K; ++n) raw[n] = __ldg(reinterpret_cast<const uint4*>(xj + (size_t)n * C));
+                uint4 gr[L + 1];
+#pragma unroll
+                for (int l1 = 0; l1 <= L; ++l1) gr[l1] = *reinterpret_cast<const uint4*>(gs + (size_t)e * Gv + l1 * C + c0);
 #pragma unroll
                 for (int l1 = 0; l1 <= L; ++l1) {
-                    float g[8];
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) g[q] = 0.f;
-                    for (int kb = 0; kb < P.n_rbf; ++kb) {
-                        const float4* wr = reinterpret_cast<const float4*>(P.Wrad + (size_t)kb * G + l1 * C + c0);
-                        const float4 w0 = __ldg(wr), w1 = __ldg(wr + 1);
-                        const float rk = rr[kb];
-                        g[0] = fmaf(rk, w0.x, g[0]); g[1] = fmaf(rk, w0.y, g[1]);
-                        g[2] = fmaf(rk, w0.z, g[2]); g[3] = fmaf(rk, w0.w, g[3]);
-                        g[4] = fmaf(rk, w1.x, g[4]); g[5] = fmaf(rk, w1.y, g[5]);
-                        g[6] = fmaf(rk, w1.z, g[6]); g[7] = fmaf(rk, w1.w, g[7]);
-                    }
+                    constexpr int kMaxW = 2 * kMaxL + 1;
                     const int w = 2 * l1 + 1;
-                    float xv[9][8];
+                    const __half2* g2 = reinterpret_cast<const __half2*>(&gr[l1]);
+                    __half2 xs2[kMaxW][4];
 #pragma unroll
-                    for (int n = 0; n < 9; ++n) {
+                    for (int n = 0; n < kMaxW; ++n) {
                         if (n < w) {
-                            const uint4 u = __ldg(reinterpret_cast<const uint4*>(
-                                P.x + ((size_t)j * K + l1 * l1 + n) * C + c0));
-                            const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+                            const __half2* h2 = reinterpret_cast<const __half2*>(&raw[l1 * l1 + n]);
 #pragma unroll
-                            for (int q = 0; q < 4; ++q) {
-                                float2 f = __bfloat1622float2(h2[q]);
-                                xv[n][2 * q] = f.x;
-                                xv[n][2 * q + 1] = f.y;
-                            }
+                            for (int q = 0; q < 4; ++q) xs2[n][q] = __hmul2(h2[q], g2[q]);
                         }
                     }
-                    const __half* Dl = De + wig_off(l1);
 #pragma unroll
-                    for (int m = 0; m < 9; ++m) {
-                        if (m < w) {
-                            float o[8];
+                    for (int mu = 0; mu <= kMaxL; ++mu) {
+                        if (mu <= l1) {
+                            const __half2* Dq = De + dpair_off(l1, mu);
+                            __half2 op[4], om[4];
 #pragma unroll
-                            for (int q = 0; q < 8; ++q) o[q] = 0.f;
+                            for (int q = 0; q < 4; ++q) { op[q] = __float2half2_rn(0.f); om[q] = op[q]; }
 #pragma unroll
-                            for (int n = 0; n < 9; ++n) {
+                            for (int n = 0; n < kMaxW; ++n) {
                                 if (n < w) {
-                                    const float dm = __half2float(Dl[m * w + n]);
+                                    const __half2 pr = Dq[n];
+                                    const __half2 dp = __low2half2(pr), dm = __high2half2(pr);
 #pragma unroll
-                                    for (int q = 0; q < 8; ++q) o[q] = fmaf(dm, xv[n][q], o[q]);
+                                    for (int q = 0; q < 4; ++q) {
+                                        op[q] = __hfma2(dp, xs2[n][q], op[q]);
+                                        om[q] = __hfma2(dm, xs2[n][q], om[q]);
+                                    }
                                 }
                             }
-                            uint4 u;
-                            __nv_bfloat162* h2 = reinterpret_cast<__nv_bfloat162*>(&u);
-#pragma unroll
-                            for (int q = 0; q < 4; ++q)
-                                h2[q] = __floats2bfloat162_rn(o[2 * q] * g[2 * q], o[2 * q + 1] * g[2 * q + 1]);
-                            *reinterpret_cast<uint4*>(xrow + kpos(l1, m - l1, L, C) + c0) = u;
+                            *reinterpret_cast<uint4*>(xrow + kpos(l1, mu, L, C) + c0) = *reinterpret_cast<uint4*>(op);
+                            if (mu > 0)
+                                *reinterpret_cast<uint4*>(xrow + kpos(l1, -mu, L, C) + c0) =
+                                    *reinterpret_cast<uint4*>(om);
                         }
                     }
                 }
             }
+            // generic-proxy stores (features, Wigner pairs) -> visible to TMA / bulk copies
             asm volatile("fence.proxy.async.global;" ::: "memory");
             mbar_arrive(xready + b);
+            c_p2 += clock64() - c_b;
+        }
+        if (P.dbg && p == 0) {
+            long long* d = P.dbg + blockIdx.x * 16;
+            d[0] = w_free; d[1] = clock64() - c_start; d[11] = c_p1; d[12] = c_p2;
         }
     } else if (warp == 8) {
         // ---------------- TMA ----------------
@@ -591,14 +940,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
             bool ok = true;
             int pending[kNS];
             for (int s2 = 0; s2 < kNS; ++s2) pending[s2] = -1;
+            long long w_x = 0, w_e = 0;
+            const long long c_start = clock64();
             for (int t = 0; t < ntiles && ok; ++t) {
                 const int b = t & 1;
-                if (!wait(xready + b, (t >> 1) & 1, abort_flag, P.status)) { ok = false; break; }
+                if (!wait_t(xready + b, (t >> 1) & 1, abort_flag, P.status, w_x)) { ok = false; break; }
                 const int rowT = (blockIdx.x * 2 + b) * kTileE;
                 for (int gi = 0; gi < ng && ok; ++gi) {
                     const TcGroup g = P.groups[gi];
                     for (int kk = 0; kk < g.klen; kk += kKS) {
-                        if (!wait(empty + stage, ph ^ 1, abort_flag, P.status)) { ok = false; break; }
+                        if (!wait_t(empty + stage, ph ^ 1, abort_flag, P.status, w_e)) { ok = false; break; }
                         uint8_t* st = ring + (size_t)stage * kStage;
                         const int ntile = g.mu > 0 ? 4 : (g.row0b >= 0 ? 3 : 2);
                         mbar_arrive_tx(full + stage, ntile * kSlot);
@@ -617,6 +968,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
                     }
                 }
             }
+            if (P.dbg) {
+                long long* d = P.dbg + blockIdx.x * 16;
+                d[2] = w_x; d[3] = w_e; d[4] = clock64() - c_start;
+            }
             // every issued load lands (bounded wait) before the CTA can leave
             for (int s2 = 0; s2 < kNS; ++s2) {
                 if (pending[s2] < 0) continue;
@@ -633,17 +988,19 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
             uint32_t ph = 0;
             long long gcount = 0;
             bool ok = true;
-            constexpr uint32_t ID = idesc_bf16(false), IDN = idesc_bf16(true);
+            long long w_t = 0, w_f = 0;
+            const long long c_start = clock64();
+            constexpr uint32_t ID = idesc_f16(false), IDN = idesc_f16(true);
             for (int t = 0; t < ntiles && ok; ++t) {
                 for (int gi = 0; gi < ng && ok; ++gi, ++gcount) {
                     const TcGroup g = P.groups[gi];
                     const int slot = (int)(gcount & 1);
                     const uint32_t use = (uint32_t)(gcount >> 1);
-                    if (!wait(tempty + slot, (use & 1) ^ 1, abort_flag, P.status)) { ok = false; break; }
+                    if (!wait_t(tempty + slot, (use & 1) ^ 1, abort_flag, P.status, w_t)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t d0 = tmem + slot * 256, d1 = d0 + 128;
                     for (int kk = 0; kk < g.klen; kk += kKS) {
-                        if (!wait(full + stage, ph, abort_flag, P.status)) { ok = false; break; }
+                        if (!wait_t(full + stage, ph, abort_flag, P.status, w_f)) { ok = false; break; }
                         tc_fence_after();
                         const uint32_t sa = smem_u32(ring + (size_t)stage * kStage);
 #pragma unroll
@@ -669,6 +1026,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
                     if (ok) umma_commit(tfull + slot);
                 }
             }
+            if (P.dbg) {
+                long long* d = P.dbg + blockIdx.x * 16;
+                d[5] = w_t; d[6] = w_f; d[7] = clock64() - c_start;
+            }
             // every issued MMA completes (bounded wait) before TMEM is released
             umma_commit(fin);
             const uint64_t t0 = gtimer();
@@ -678,45 +1039,80 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
         __syncwarp();
     } else {
         // ---------------- epilogue (warps 0-3, thread = TMEM lane) ----------------
+        // Every decision to stop goes through bar_and, so the 128 threads leave
+        // together and no thread is left at a named barrier.
         const int r = threadIdx.x;
         long long gcount = 0;
         bool ok = true;
-        for (int t = 0; t < ntiles && ok; ++t) {
+        long long w_x = 0, w_t = 0;
+        long long staged[2] = {-1, -1};  // last group index staged into each buffer (thread 0)
+        const long long c_start = clock64();
+        for (int t = 0; t < ntiles; ++t) {
             const int b = t & 1;
-            if (!wait(xready + b, (t >> 1) & 1, abort_flag, P.status)) { ok = false; break; }
-            const __half* Db = dbuf + (size_t)b * kTileE * WSP;
-            const float* pb = pbuf + (size_t)b * kTileE * kMaxHeads;
+            const bool okx = wait_t(xready + b, (t >> 1) & 1, abort_flag, P.status, w_x);
+            if (!bar_and(2, 128, ok && okx)) { ok = false; break; }
+            const float* Dg = P.dscr + (size_t)(blockIdx.x * 2 + b) * dglob_floats();
+            const float* pb = pbuf + (size_t)b * kTileE * H;
             const int* nb = nid + b * kTileE;
+            const uint32_t* sg = segm + b * (kTileE / kChunk);
+            if (r == 0) {
+                stage_group_pairs(P.groups[0], C, Dg, dstage + (gcount & 1) * kStageD, dbar + (gcount & 1));
+                staged[gcount & 1] = gcount;
+            }
             for (int gi = 0; gi < ng; ++gi, ++gcount) {
+                // all threads are done with group gcount-1, so its staging buffer can be refilled
+                if (!bar_and(2, 128, ok)) { ok = false; break; }
+                if (r == 0 && gi + 1 < ng) {
+                    stage_group_pairs(P.groups[gi + 1], C, Dg, dstage + ((gcount + 1) & 1) * kStageD,
+                                      dbar + ((gcount + 1) & 1));
+                    staged[(gcount + 1) & 1] = gcount + 1;
+                }
                 const TcGroup g = P.groups[gi];
                 const int slot = (int)(gcount & 1);
                 const uint32_t use = (uint32_t)(gcount >> 1);
-                if (!wait(tfull + slot, use & 1, abort_flag, P.status)) { ok = false; break; }
-                tc_fence_after();
-                const uint32_t tacc = tmem + ((uint32_t)(warp * 32) << 16) + slot * 256;
-                if (g.mu > 0) {
-                    const int row = g.row0 + r;
-                    const int l3 = g.mu + row / C, c = row % C;
-                    epi_dispatch<L>(l3, tacc, true, g.mu, c, c / dh, H, Db, pb, nb, P.out, C);
-                } else {
-                    const int ra = g.row0 + r;
-                    epi_dispatch<L>(ra / C, tacc, false, 0, ra % C, (ra % C) / dh, H, Db, pb, nb, P.out, C);
-                    if (g.row0b >= 0) {
-                        const int rb = g.row0b + r;
-                        epi_dispatch<L>(rb / C, tacc + 128, false, 0, rb % C, (rb % C) / dh, H, Db, pb, nb, P.out,
-                                        C);
+                const bool okd = wait_t(dbar + slot, use & 1, abort_flag, P.status, w_t);
+                const bool okt = okd && wait_t(tfull + slot, use & 1, abort_flag, P.status, w_t);
+                if (okt) {
+                    tc_fence_after();
+                    const uint32_t tacc = tmem + ((uint32_t)(warp * 32) << 16) + slot * 256;
+                    const float2* Ds = reinterpret_cast<const float2*>(dstage + slot * kStageD);
+                    const uint32_t twarp = tmem + ((uint32_t)(warp * 32) << 16) + slot * 256;
+                    if (g.mu > 0) {
+                        const int row = g.row0 + warp * 32;  // rows of this warp: one l3, 32 channels
+                        epi_mma<2>(twarp, g.mu + row / C, row % C, H, dh, K, C, Ds, pb, nb, sg, P.out);
+                    } else {
+                        const int ra = g.row0 + warp * 32, la = ra / C;
+                        epi_mma<1>(twarp, la, ra % C, H, dh, K, C, Ds, pb, nb, sg, P.out);
+                        if (g.row0b >= 0) {
+                            const int rb = g.row0b + warp * 32;
+                            epi_mma<1>(twarp + 128, rb / C, rb % C, H, dh, K, C, Ds + kTileE * (2 * la + 2), pb,
+                                       nb, sg, P.out);
+                        }
                     }
+                    tc_fence_before();
+                } else {
+                    ok = false;
                 }
-                tc_fence_before();
                 mbar_arrive(tempty + slot);
             }
-            if (ok) mbar_arrive(xfree + b);
+            if (!bar_and(2, 128, ok)) { ok = false; break; }
+            mbar_arrive(xfree + b);
+        }
+        if (P.dbg && r == 0) {
+            long long* d = P.dbg + blockIdx.x * 16;
+            d[8] = w_x; d[9] = w_t; d[10] = clock64() - c_start; d[13] = ntiles;
+        }
+        // a staging copy that was issued but never waited for lands before exit
+        if (r == 0) {
+            for (int s2 = 0; s2 < 2; ++s2) {
+                if (staged[s2] < 0) continue;
+                const uint64_t t0 = gtimer();
+                while (!mbar_try(dbar + s2, (uint32_t)((staged[s2] >> 1) & 1)) && gtimer() - t0 < kWaitNs) {
+                }
+            }
         }
     }
 
-    // MMA completion before TMEM release: the epilogue consumed every group it
-    // waited for; on a normal exit all MMAs are complete. On abort, wait
-    // (bounded) for the last commits to land.
     tc_fence_before();
     __syncthreads();
     if (warp == 8) {
@@ -755,7 +1151,7 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows) {
     cuuint64_t strides[1] = {cols * 2};
     cuuint32_t box[2] = {(cuuint32_t)tc::kKS, 128};
     cuuint32_t es[2] = {1, 1};
-    return f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+    return f(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -764,20 +1160,36 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows) {
 
 bool tc_supported(int L, int C, int H, int n_rbf, bool bf16) {
     return bf16 && L >= 1 && L <= kMaxL && C % 128 == 0 && C <= 256 && H <= kMaxHeads && H % 4 == 0 &&
-           n_rbf <= kMaxRbf;
+           n_rbf <= kTcMaxRbf && tc::SmemLayout(L, H, n_rbf).total + 1024 <= 232448;
 }
 
-size_t tc_workspace_bytes(int64_t n_atoms, int L, int C, int H) {
-    size_t b = 0;
-    b += align_up(4 * (size_t)n_atoms * H, 256);                                       // lse
-    b += align_up(4 * (size_t)(kMaxCtas + 1), 256);                                    // partition
-    b += align_up((size_t)kMaxCtas * 2 * tc::kTileE * n_sh(L) * C * 2, 256);           // feature scratch
-    return b;
-}
+namespace {
+struct TcWs {
+    size_t dbg, lse, part, xs, dscr, x16, w16, whT, gscr, words, total;
+    TcWs(int64_t n_atoms, int L, int C, int H) {
+        const int K = n_sh(L), Gv = (L + 1) * C;
+        size_t o = 0;
+        auto take = [&](size_t b) { size_t r = o; o = align_up(o + b, 256); return r; };
+        dbg = take(kTcDebugBytes);
+        lse = take(4 * (size_t)n_atoms * H);
+        part = take(4 * (size_t)(kMaxCtas + 1));
+        xs = take((size_t)kMaxCtas * 2 * tc::kTileE * K * C * 2);
+        dscr = take((size_t)kMaxCtas * 2 * tc::dglob_floats() * 4);
+        x16 = take((size_t)n_atoms * K * C * 2);
+        w16 = take(so2_total(L, C) * 2);
+        whT = take((size_t)Gv * kTcMaxRbf * 2);
+        gscr = take((size_t)kMaxCtas * tc::kTileE * Gv * 2);
+        words = take(256);
+        total = o;
+    }
+};
+}  // namespace
+
+size_t tc_workspace_bytes(int64_t n_atoms, int L, int C, int H) { return TcWs(n_atoms, L, C, H).total; }
 
 template <int L>
 static cudaError_t launch_tc(const tc::TcParams& P, const tc::TcMaps& T, int grid, cudaStream_t s) {
-    const size_t smem = tc::Smem<L>::total + 1024;
+    const size_t smem = tc::SmemLayout(L, P.H, P.n_rbf).total + 1024;
     cudaError_t e = cudaFuncSetAttribute(tc::k_attn_tc<L>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     count_launch();
@@ -798,12 +1210,35 @@ cudaError_t run_attention_tc(const AttnArgs& a, void* tc_ws, cudaStream_t s) {
         if (v > 0 && v < cap) cap = v;
     }
     const int grid = std::max(1, std::min(sms, cap));
+    const TcWs Wl(N, L, C, H);
     char* w = static_cast<char*>(tc_ws);
-    float* lse = reinterpret_cast<float*>(w);
-    w += align_up(4 * (size_t)N * H, 256);
-    int32_t* part = reinterpret_cast<int32_t*>(w);
-    w += align_up(4 * (size_t)(kMaxCtas + 1), 256);
-    __nv_bfloat16* xs = reinterpret_cast<__nv_bfloat16*>(w);
+    long long* dbg = reinterpret_cast<long long*>(w + Wl.dbg);
+    float* lse = reinterpret_cast<float*>(w + Wl.lse);
+    int32_t* part = reinterpret_cast<int32_t*>(w + Wl.part);
+    __half* xs = reinterpret_cast<__half*>(w + Wl.xs);
+    float* dscr = reinterpret_cast<float*>(w + Wl.dscr);
+    __half* x16 = reinterpret_cast<__half*>(w + Wl.x16);
+    __half* w16 = reinterpret_cast<__half*>(w + Wl.w16);
+    __half* whT = reinterpret_cast<__half*>(w + Wl.whT);
+    __half* gscr = reinterpret_cast<__half*>(w + Wl.gscr);
+    unsigned* amax = reinterpret_cast<unsigned*>(w + Wl.words);
+    float* scale = reinterpret_cast<float*>(w + Wl.words + 16);
+    const int G = (L + 1) * C + H, Gv = (L + 1) * C;
+
+    // fp16 operands: feature scale, scaled features, weights
+    e = cudaMemsetAsync(amax, 0, 16, s);
+    if (e != cudaSuccess) return e;
+    const size_t nx = (size_t)N * K * C;
+    count_launch();
+    tc::k_amax<<<592, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(a.x), nx, a.Wrad, (size_t)a.n_rbf * G, amax);
+    count_launch();
+    tc::k_make_scale<<<1, 1, 0, s>>>(amax, a.n_rbf, scale, a.status);
+    count_launch();
+    tc::k_x_to_f16<<<1184, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(a.x), nx, scale, x16);
+    count_launch();
+    tc::k_w_to_f16<<<592, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(a.Wso2), so2_total(L, C), w16);
+    count_launch();
+    tc::k_wrad_t<<<(Gv * kTcMaxRbf + 255) / 256, 256, 0, s>>>(a.Wrad, a.n_rbf, G, Gv, whT);
 
     // pre-passes: Q/K, softmax statistics, partition, zeroed output
     const size_t qk_smem = (32 * C + tc::kQkRows * (C + 1)) * 4;
@@ -825,9 +1260,17 @@ cudaError_t run_attention_tc(const AttnArgs& a, void* tc_ws, cudaStream_t s) {
 
     tc::TcParams P{};
     P.C = C; P.H = H; P.n_rbf = a.n_rbf; P.G = (L + 1) * C + H; P.cutoff = a.cutoff; P.box = a.box;
-    P.pos = a.pos; P.row_ptr = a.row_ptr; P.col = a.col; P.x = static_cast<const __nv_bfloat16*>(a.x);
-    P.q = a.q; P.k = a.k; P.lse = lse; P.Wrad = a.Wrad; P.part = part; P.xs = xs; P.out = a.out;
+    P.pos = a.pos; P.row_ptr = a.row_ptr; P.col = a.col; P.x = x16; P.whT = whT; P.gscr = gscr; P.scale = scale;
+    P.q = a.q; P.k = a.k; P.lse = lse; P.Wrad = a.Wrad; P.part = part; P.xs = xs; P.dscr = dscr; P.out = a.out;
     P.status = a.status;
+    P.dbg = nullptr;
+    if (const char* env = getenv("E2F_TC_TIMERS")) {
+        if (atoi(env) > 0) {
+            P.dbg = dbg;
+            e = cudaMemsetAsync(dbg, 0, kTcDebugBytes, s);
+            if (e != cudaSuccess) return e;
+        }
+    }
     // groups: m = 0 feature blocks in pairs; then (o+, o-) pairs per block for m >= 1
     int ng = 0;
     const int n0 = (L + 1) * C;
@@ -851,7 +1294,7 @@ cudaError_t run_attention_tc(const AttnArgs& a, void* tc_ws, cudaStream_t s) {
     P.n_groups = ng;
 
     tc::TcMaps T;
-    const __nv_bfloat16* W = static_cast<const __nv_bfloat16*>(a.Wso2);
+    const __half* W = w16;
     if (!make_map(&T.w[0], W + so2_offset(L, C, 0, 0), n0, n0)) return cudaErrorInvalidValue;
     for (int mu = 1; mu <= L; ++mu) {
         const int nm = (L + 1 - mu) * C;

@@ -3,6 +3,7 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <stdint.h>
 
 #include "common.cuh"
@@ -11,7 +12,9 @@ namespace e2f {
 
 constexpr int kMaxHeads = 16;   // tensor-core path: H <= 16
 constexpr int kMaxRbf = 32;
+constexpr int kTcMaxRbf = 16;   // tensor-core path: the radial gate is one k=16 mma
 constexpr int kMaxCtas = 160;   // persistent CTAs (one per SM; B200 has 148)
+constexpr size_t kTcDebugBytes = (size_t)kMaxCtas * 16 * 8;  // per-CTA role timers
 
 struct StatsParams {
     int n_atoms, C, H, n_rbf, G;
@@ -45,15 +48,20 @@ struct TcParams {
     const float* pos;
     const int32_t* row_ptr;
     const int32_t* col;
-    const __nv_bfloat16* x;
+    const __half* x;       // features in fp16, scaled by scale[0] (an exact power of two)
+    const __half* whT;     // value-gate weights, fp16, [(L+1)C][16] (radial index innermost, zero padded)
+    __half* gscr;          // per-CTA value-gate scratch [n_ctas][128][(L+1)C]
+    const float* scale;    // [0] feature scale s, [1] 1/s
     const float* q;
     const float* k;
     const float* lse;
     const float* Wrad;
     const int32_t* part;
-    __nv_bfloat16* xs;
+    __half* xs;
+    float* dscr;     // per-CTA Wigner pair blocks [n_ctas * 2 * 128][kDStride]
     float* out;
     int* status;
+    long long* dbg;  // per-CTA role cycle counters, or null
     int n_groups;
     TcGroup groups[kMaxGroups];
 };

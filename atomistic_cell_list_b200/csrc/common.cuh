@@ -60,11 +60,21 @@ __device__ __forceinline__ void edge_frame(float x, float y, float z, float R[3]
 // ---------------------------------------------------------------------------
 namespace ir {
 
-template <int l>
-struct Coef {  // u, v, w of the recursion for degree l, row m, column n
-    __device__ static __forceinline__ float den(int n) {
-        return (n > -l && n < l) ? float((l + n) * (l - n)) : float((2 * l) * (2 * l - 1));
-    }
+// square root evaluated by the compiler (Newton's method in double)
+constexpr double csqrt_iter(double x, double cur, double prev) {
+    return cur == prev ? cur : csqrt_iter(x, 0.5 * (cur + x / cur), cur);
+}
+constexpr double csqrt(double x) { return x > 0.0 ? csqrt_iter(x, x > 1.0 ? x : 1.0, 0.0) : 0.0; }
+
+// u, v, w of the recursion for degree l, row m, column n (compile time)
+template <int l, int m, int n>
+struct Coef {
+    static constexpr int am = m < 0 ? -m : m;
+    static constexpr double den = (n > -l && n < l) ? double((l + n) * (l - n)) : double((2 * l) * (2 * l - 1));
+    static constexpr double d0 = (m == 0) ? 1.0 : 0.0;
+    static constexpr float u = float(csqrt(double((l + m) * (l - m)) / den));
+    static constexpr float v = float(0.5 * csqrt((1.0 + d0) * double((l + am - 1) * (l + am)) / den) * (1.0 - 2.0 * d0));
+    static constexpr float w = float(-0.5 * csqrt(double((l - am - 1) * (l - am)) / den) * (1.0 - d0));
 };
 
 template <int l>
@@ -78,39 +88,46 @@ __device__ __forceinline__ float Pterm(int i, int a, int b, const float* R1, con
     return r1(i, 0) * dp(a, b);
 }
 
+template <int l, int m, int n>
+__device__ __forceinline__ void entry(const float* R1, const float* Dp, float* Dl) {
+    using K = Coef<l, m, n>;
+    constexpr int am = K::am;
+    float acc = 0.f;
+    if constexpr (am < l) acc += K::u * Pterm<l>(0, m, n, R1, Dp);
+    float V;
+    if constexpr (m == 0) {
+        V = Pterm<l>(1, 1, n, R1, Dp) + Pterm<l>(-1, -1, n, R1, Dp);
+    } else if constexpr (m > 0) {
+        V = Pterm<l>(1, m - 1, n, R1, Dp) * (m == 1 ? 1.41421356237309515f : 1.f);
+        if constexpr (m != 1) V -= Pterm<l>(-1, -m + 1, n, R1, Dp);
+    } else {
+        V = Pterm<l>(-1, -m - 1, n, R1, Dp) * (m == -1 ? 1.41421356237309515f : 1.f);
+        if constexpr (m != -1) V += Pterm<l>(1, m + 1, n, R1, Dp);
+    }
+    acc += K::v * V;
+    if constexpr (m != 0 && am < l - 1) {
+        const float W = (m > 0) ? Pterm<l>(1, m + 1, n, R1, Dp) + Pterm<l>(-1, -m - 1, n, R1, Dp)
+                                : Pterm<l>(1, m - 1, n, R1, Dp) - Pterm<l>(-1, -m + 1, n, R1, Dp);
+        acc += K::w * W;
+    }
+    Dl[(m + l) * (2 * l + 1) + (n + l)] = acc;
+}
+
+template <int l, int m, int n>
+__device__ __forceinline__ void row(const float* R1, const float* Dp, float* Dl) {
+    entry<l, m, n>(R1, Dp, Dl);
+    if constexpr (n < l) row<l, m, n + 1>(R1, Dp, Dl);
+}
+
+template <int l, int m>
+__device__ __forceinline__ void rows(const float* R1, const float* Dp, float* Dl) {
+    row<l, m, -l>(R1, Dp, Dl);
+    if constexpr (m < l) rows<l, m + 1>(R1, Dp, Dl);
+}
+
 template <int l>
 __device__ __forceinline__ void step(const float* R1, const float* Dp, float* Dl) {
-#pragma unroll
-    for (int m = -l; m <= l; ++m) {
-#pragma unroll
-        for (int n = -l; n <= l; ++n) {
-            const float den = Coef<l>::den(n);
-            const int am = m < 0 ? -m : m;
-            const float d0 = (m == 0) ? 1.f : 0.f;
-            const float u = sqrtf(float((l + m) * (l - m)) / den);
-            const float v = 0.5f * sqrtf((1.f + d0) * float((l + am - 1) * (l + am)) / den) * (1.f - 2.f * d0);
-            const float wc = -0.5f * sqrtf(float((l - am - 1) * (l - am)) / den) * (1.f - d0);
-            float acc = 0.f;
-            if (am < l) acc += u * Pterm<l>(0, m, n, R1, Dp);
-            float V;
-            if (m == 0) {
-                V = Pterm<l>(1, 1, n, R1, Dp) + Pterm<l>(-1, -1, n, R1, Dp);
-            } else if (m > 0) {
-                V = Pterm<l>(1, m - 1, n, R1, Dp) * (m == 1 ? 1.41421356237309515f : 1.f);
-                if (m != 1) V -= Pterm<l>(-1, -m + 1, n, R1, Dp);
-            } else {
-                V = Pterm<l>(-1, -m - 1, n, R1, Dp) * (m == -1 ? 1.41421356237309515f : 1.f);
-                if (m != -1) V += Pterm<l>(1, m + 1, n, R1, Dp);
-            }
-            acc += v * V;
-            if (m != 0 && am < l - 1) {
-                float W = (m > 0) ? Pterm<l>(1, m + 1, n, R1, Dp) + Pterm<l>(-1, -m - 1, n, R1, Dp)
-                                  : Pterm<l>(1, m - 1, n, R1, Dp) - Pterm<l>(-1, -m + 1, n, R1, Dp);
-                acc += wc * W;
-            }
-            Dl[(m + l) * (2 * l + 1) + (n + l)] = acc;
-        }
-    }
+    rows<l, -l>(R1, Dp, Dl);
 }
 
 }  // namespace ir
@@ -159,6 +176,16 @@ __device__ __forceinline__ float rbf(float d, int k, float cutoff, int n_rbf) {
     const float t = (d - float(k) * step) / step;
     const float u = 0.5f * (cosf(3.14159265358979323846f * d / cutoff) + 1.f);
     return u * expf(-t * t);
+}
+
+// all n_rbf basis values of one distance (the envelope evaluated once)
+__device__ __forceinline__ void rbf_all(float d, float cutoff, int n_rbf, float* out) {
+    const float step = cutoff / float(n_rbf - 1);
+    const float u = 0.5f * (cosf(3.14159265358979323846f * d / cutoff) + 1.f);
+    for (int k = 0; k < n_rbf; ++k) {
+        const float t = (d - float(k) * step) / step;
+        out[k] = u * expf(-t * t);
+    }
 }
 
 }  // namespace e2f
