@@ -45,6 +45,8 @@ _SIGS = {
     "e2f_neighbors_workspace_size": (_sz, [_i64, _vp, ctypes.c_float, ctypes.c_int32]),
     "e2f_build_neighbors": (ctypes.c_int, [_vp, _i64, _vp, ctypes.c_float, _vp, ctypes.c_int32, _vp, _vp, _i64,
                                            ctypes.POINTER(_i64), _vp, _sz, _vp]),
+    "e2f_build_neighbors_noalloc": (ctypes.c_int, [_vp, _i64, _vp, ctypes.c_float, _vp, ctypes.c_int32, _vp, _vp,
+                                                   _i64, ctypes.POINTER(_i64), _vp]),
     "e2f_attention_workspace_size": (_sz, [_i64, _i64, ctypes.POINTER(e2f_attn_cfg)]),
     "e2f_onfly_attention": (ctypes.c_int, [ctypes.POINTER(e2f_attn_cfg), _vp, _i64, _vp, _vp, _vp, _i64, _vp, _vp,
                                            _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
@@ -143,6 +145,41 @@ def e2f_build_neighbors(pos: torch.Tensor, box, cutoff: float, graph_ptr: torch.
         _check(code, "e2f_build_neighbors")
         return row_ptr, col[: npairs.value]
     raise E2FError(3, "e2f_build_neighbors")
+
+
+NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
+
+
+def e2f_build_neighbors_noalloc(pos: torch.Tensor, box, cutoff: float, graph_ptr: torch.Tensor | None = None,
+                                row_ptr: torch.Tensor | None = None, col: torch.Tensor | None = None,
+                                stream=None):
+    """CSR neighbour list built in the library's static scratch (no workspace).
+
+    row_ptr / col may be passed in (int32, [N+1] and [capacity]); the call
+    then writes them and returns (row_ptr, col[:E]). With col=None a buffer
+    of 128 N entries is made here, grown once on E2F_ERR_CAPACITY.
+    """
+    _need_cuda(pos, graph_ptr, row_ptr, col)
+    assert pos.dtype == torch.float32 and pos.dim() == 2 and pos.shape[1] == 3
+    n = pos.shape[0]
+    n_graphs = 1 if graph_ptr is None else graph_ptr.numel() - 1
+    if row_ptr is None:
+        row_ptr = torch.empty(n + 1, dtype=torch.int32, device=pos.device)
+    given = col is not None
+    if col is None:
+        col = torch.empty(max(1024, 128 * n), dtype=torch.int32, device=pos.device)
+    b, keep = _box_arg(box)
+    for _ in range(2):
+        npairs = ctypes.c_int64(0)
+        code = lib().e2f_build_neighbors_noalloc(_ptr(pos), n, b, float(cutoff), _ptr(graph_ptr), n_graphs,
+                                                 _ptr(row_ptr), _ptr(col), col.numel(), ctypes.byref(npairs),
+                                                 _stream(stream))
+        if code == 3 and not given:
+            col = torch.empty(int(npairs.value), dtype=torch.int32, device=pos.device)
+            continue
+        _check(code, "e2f_build_neighbors_noalloc")
+        return row_ptr, col[: npairs.value]
+    raise E2FError(3, "e2f_build_neighbors_noalloc")
 
 
 def make_cfg(L: int, C: int, H: int, n_rbf: int, cutoff: float, dtype: str) -> e2f_attn_cfg:

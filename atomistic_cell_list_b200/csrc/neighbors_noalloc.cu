@@ -1,0 +1,65 @@
+// Neighbour build with its scratch in a fixed device array of this library.
+//
+// Some callers cannot allocate device memory at the moment they need a
+// neighbour list: a host program embedded in another runtime whose caching
+// allocator already owns nearly all of HBM, or a caller with a latency bound
+// that cannot take the device-wide synchronisation of cudaMalloc/cudaFree.
+// This entry point serves them: it runs the same kernels as
+// e2f_build_neighbors, with the scratch taken from a static __device__
+// array instead of a caller workspace, and it allocates nothing itself (no
+// cudaMalloc, no allocating library).
+#include <mutex>
+
+#include "common.cuh"
+
+namespace e2f {
+namespace {
+
+static_assert(E2F_NOALLOC_SCRATCH_BYTES % 256 == 0, "scratch size must keep 256-byte granules");
+
+// Module memory: placed when the module is loaded, one copy per device.
+__device__ __align__(256) unsigned char g_nbr_scratch[E2F_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mu;
+void* g_scratch_ptr[kMaxDevices] = {};
+
+// Device address of this device's copy of the scratch; looked up once per
+// device, with that device current (the lookup may load the module).
+cudaError_t scratch_for_current_device(void** out) {
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    if (!g_scratch_ptr[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_nbr_scratch);
+        if (e != cudaSuccess) return e;
+        g_scratch_ptr[dev] = p;
+    }
+    *out = g_scratch_ptr[dev];
+    return cudaSuccess;
+}
+
+}  // namespace
+}  // namespace e2f
+
+using namespace e2f;
+
+extern "C" e2f_status e2f_build_neighbors_noalloc(const float* pos, int64_t n_atoms, const float* box_host,
+                                                  float cutoff, const int32_t* graph_ptr, int32_t n_graphs,
+                                                  int32_t* row_ptr, int32_t* col, int64_t col_capacity,
+                                                  int64_t* n_pairs_host, void* stream) {
+    if (n_atoms < 0 || !(cutoff > 0.f)) return E2F_ERR_INVALID_ARG;
+    // problems whose scratch would not fit are refused before anything runs
+    const size_t need = e2f_neighbors_workspace_size(n_atoms, box_host, cutoff, graph_ptr ? n_graphs : 1);
+    if (need > (size_t)E2F_NOALLOC_SCRATCH_BYTES) return E2F_ERR_UNSUPPORTED;
+    void* scratch = nullptr;
+    if (scratch_for_current_device(&scratch) != cudaSuccess || !scratch) return E2F_ERR_CUDA;
+    // e2f_build_neighbors clears, on `stream`, every scratch word that must
+    // start at zero (the flag word, the bucket counts, the degree sentinel)
+    // before its first kernel, so what an earlier call left there is harmless.
+    return e2f_build_neighbors(pos, n_atoms, box_host, cutoff, graph_ptr, n_graphs, row_ptr, col, col_capacity,
+                               n_pairs_host, scratch, (size_t)E2F_NOALLOC_SCRATCH_BYTES, stream);
+}

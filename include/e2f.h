@@ -10,7 +10,8 @@
  *     pointers are read (or written) before the call returns.
  *   - The caller owns every buffer. The library allocates no device memory
  *     of its own; it works inside the caller's workspace. Per device it keeps
- *     only lazily set kernel attributes.
+ *     only lazily set kernel attributes and the static scratch array of
+ *     e2f_build_neighbors_noalloc (module memory).
  *   - Work is enqueued on `stream` (0 = legacy default stream) in stream
  *     order. Calls that return a host value (n_pairs_host) synchronise it.
  *   - Argument checks happen before any launch; a failed check launches
@@ -101,6 +102,36 @@ e2f_status e2f_build_neighbors(const float* pos, int64_t n_atoms,
                                int64_t col_capacity, int64_t* n_pairs_host,
                                void* workspace, size_t ws_bytes,
                                void* stream);
+
+/* ------------------------------------------------------------------------
+ * Neighbour list without a caller workspace. The pages have no counterpart
+ * of this call: it exists for callers that cannot allocate device memory
+ * when they need the list (an allocator of another runtime owns the heap,
+ * or cudaMalloc's device-wide synchronisation is not acceptable).
+ *
+ * Same arguments, outputs, checks and results as e2f_build_neighbors, minus
+ * workspace/ws_bytes: the scratch is a static device array of this library
+ * of E2F_NOALLOC_SCRATCH_BYTES (16 MiB) per device, enough for about 390k
+ * atoms with open boundaries or 500k in a periodic box at a 6 A cutoff.
+ * The call allocates no device memory.
+ *   Returns E2F_ERR_UNSUPPORTED, before any launch, when
+ *   e2f_neighbors_workspace_size(...) exceeds E2F_NOALLOC_SCRATCH_BYTES;
+ *   E2F_ERR_CUDA if the scratch address cannot be looked up.
+ * The scratch is shared: calls that overlap on one device (other threads,
+ * other streams, or a call enqueued while an earlier one's kernels still
+ * run) race on it and give undefined results; serialise them. The first
+ * call on each device looks up the array's device address (which may load
+ * the module): make it with that device current and before any stream
+ * capture starts on it. Like e2f_build_neighbors it synchronises `stream`.
+ * ---------------------------------------------------------------------- */
+#define E2F_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
+
+e2f_status e2f_build_neighbors_noalloc(const float* pos, int64_t n_atoms,
+                                       const float* box_host, float cutoff,
+                                       const int32_t* graph_ptr,
+                                       int32_t n_graphs, int32_t* row_ptr,
+                                       int32_t* col, int64_t col_capacity,
+                                       int64_t* n_pairs_host, void* stream);
 
 /* ------------------------------------------------------------------------
  * On-the-fly equivariant attention, forward (gist.science Technical
