@@ -232,14 +232,18 @@ def e2f_attention_uses_tensor_cores(cfg: e2f_attn_cfg) -> bool:
     return bool(lib().e2f_attention_uses_tensor_cores(ctypes.byref(cfg)))
 
 
+DEBUG_SLOTS = 32
+
+
 def e2f_attention_debug_timers(workspace: torch.Tensor, n_atoms: int, cfg: e2f_attn_cfg, n_ctas: int = 160,
                                stream=None):
     """Per-CTA role cycle counters of the last tensor-core call (E2F_TC_TIMERS=1)."""
     import numpy as np
-    buf = (_i64 * (16 * n_ctas))()
+    n = DEBUG_SLOTS * n_ctas
+    buf = (_i64 * n)()
     _check(lib().e2f_attention_debug_timers(_ptr(workspace), workspace.numel(), int(n_atoms), ctypes.byref(cfg), buf,
-                                            16 * n_ctas, _stream(stream)), "e2f_attention_debug_timers")
-    return np.frombuffer(buf, dtype=np.int64).reshape(n_ctas, 16).copy()
+                                            n, _stream(stream)), "e2f_attention_debug_timers")
+    return np.frombuffer(buf, dtype=np.int64).reshape(n_ctas, DEBUG_SLOTS).copy()
 
 
 def e2f_launch_count() -> int:

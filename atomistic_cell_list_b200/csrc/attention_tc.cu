@@ -208,51 +208,58 @@ __device__ __forceinline__ float edge_logit(const float* rho, int n_rbf, const f
 }
 
 // Softmax statistics per node and head, lse = m + log(sum exp(a - m)), by an
-// online max/sum over the node's edges (one warp per node).
+// online max/sum over the node's edges. One warp per node; lane = (edge slot
+// es, head h) with 32 / H edge slots, so a head's q and logit-gate column
+// stay in registers and the key row of an edge is read as float4 by its H
+// lanes. The logit is evaluated in the same order as in the main kernel.
 __global__ void __launch_bounds__(256) k_softmax_stats(StatsParams P) {
     const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
     if (warp >= P.n_atoms) return;
     const int i = warp;
-    const int H = P.H, C = P.C, dh = C / H, G = P.G;
+    const int H = P.H, C = P.C, dh = C / H, G = P.G, Gv = G - H;
+    const int h = lane % H, es = lane / H, EP = 32 / H;
     const float inv = rsqrtf((float)dh);
-    float m[kMaxHeads], s[kMaxHeads];
+    float wcol[kTcMaxRbf];
 #pragma unroll
-    for (int h = 0; h < kMaxHeads; ++h) { m[h] = -INFINITY; s[h] = 0.f; }
+    for (int kb = 0; kb < kTcMaxRbf; ++kb) wcol[kb] = kb < P.n_rbf ? P.Wrad[(size_t)kb * G + Gv + h] : 0.f;
+    const float4* q4 = reinterpret_cast<const float4*>(P.q + (size_t)i * C + h * dh);
+    const int d4 = dh / 4;
+    float m = -INFINITY, s = 0.f;
     const int e0 = P.row_ptr[i], e1 = P.row_ptr[i + 1];
-    for (int e = e0 + lane; e < e1; e += 32) {
+    for (int e = e0 + es; e < e1; e += EP) {
         const int j = P.col[e];
-        float3 r = edge_vec(P.pos, i, j, P.box);
+        const float3 r = edge_vec(P.pos, i, j, P.box);
         const float d = sqrtf(r.x * r.x + r.y * r.y + r.z * r.z);
-        float rho[kMaxRbf];
-        rbf_all(d, P.cutoff, P.n_rbf, rho);
+        float rr[kTcMaxRbf];
+        rbf_all<kTcMaxRbf>(d, P.cutoff, P.n_rbf, rr);
+        float ga = 0.f;
 #pragma unroll
-        for (int h = 0; h < kMaxHeads; ++h) {
-            if (h < H) {
-                float a = edge_logit(rho, P.n_rbf, P.Wrad, G, G - H + h, P.q + (size_t)i * C + h * dh,
-                                     P.k + (size_t)j * C + h * dh, dh, inv);
-                float mn = fmaxf(m[h], a);
-                s[h] = s[h] * expf(m[h] - mn) + expf(a - mn);
-                m[h] = mn;
-            }
+        for (int kb = 0; kb < kTcMaxRbf; ++kb) ga = fmaf(rr[kb], wcol[kb], ga);
+        const float4* k4 = reinterpret_cast<const float4*>(P.k + (size_t)j * C + h * dh);
+        float dot = 0.f;
+        for (int c4 = 0; c4 < d4; ++c4) {
+            const float4 qa = __ldg(q4 + c4), kv = __ldg(k4 + c4);
+            dot = fmaf(qa.x, kv.x, dot);
+            dot = fmaf(qa.y, kv.y, dot);
+            dot = fmaf(qa.z, kv.z, dot);
+            dot = fmaf(qa.w, kv.w, dot);
         }
+        const float a = ga * dot * inv;
+        const float mn = fmaxf(m, a);
+        s = s * expf(m - mn) + expf(a - mn);
+        m = mn;
     }
-#pragma unroll
-    for (int h = 0; h < kMaxHeads; ++h) {
-        if (h < H) {
-            float mh = m[h], sh = s[h];
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                float mo = __shfl_xor_sync(0xffffffffu, mh, o), so = __shfl_xor_sync(0xffffffffu, sh, o);
-                float mn = fmaxf(mh, mo);
-                float sa = (mh == -INFINITY) ? 0.f : sh * expf(mh - mn);
-                float sb = (mo == -INFINITY) ? 0.f : so * expf(mo - mn);
-                mh = mn;
-                sh = sa + sb;
-            }
-            if (lane == 0) P.lse[(size_t)i * H + h] = (e1 > e0) ? mh + logf(sh) : 0.f;
-        }
+    // combine the edge slots of each head
+    for (int o = H; o < 32; o <<= 1) {
+        const float mo = __shfl_xor_sync(0xffffffffu, m, o), so = __shfl_xor_sync(0xffffffffu, s, o);
+        const float mn = fmaxf(m, mo);
+        const float sa = (m == -INFINITY) ? 0.f : s * expf(m - mn);
+        const float sb = (mo == -INFINITY) ? 0.f : so * expf(mo - mn);
+        m = mn;
+        s = sa + sb;
     }
+    if (es == 0) P.lse[(size_t)i * H + h] = (e1 > e0) ? m + logf(s) : 0.f;
 }
 
 // Node range per CTA: part[k] = first node whose edges start at or after
@@ -396,43 +403,71 @@ constexpr int kKS = 32;                       // K per ring stage
 constexpr int kNS = 3;                        // ring stages
 constexpr int kSlot = kTileE * kKS * 2;       // 8 KB per operand tile
 constexpr int kStage = 4 * kSlot;
-constexpr int kThreads = 320;
+constexpr int kThreads = 512;
+// Warp roles (16 warps, 65536 / 512 = 128 registers per thread):
+//   0-3, 8-11  epilogue (warp w: TMEM lane quadrant w % 4, lane half w / 8)
+//   4-7        producer
+//   12         TMA, 13 MMA, 14-15 idle
+constexpr int kEpiThreads = 256;
 constexpr int kChunk = 16;                    // epilogue: edges per TMEM load
-constexpr int kStageD = 20480;                // epilogue Wigner staging buffer (bytes)
 
 // Wigner blocks of an edge in "pair" form: for each degree l and each
-// |m| = mu <= l the 2l+1 pairs (D^l[+mu][n], D^l[-mu][n]) (padded to 2l+2).
-// A pair rotates into both x~[+mu] and x~[-mu] (producer) and rotates o+ and
-// o- back (epilogue). Pairs of block (l, mu) start at dpair_off(l, mu).
-__host__ __device__ constexpr int dpair_block(int l) { return (l + 1) * (2 * l + 2); }
-__host__ __device__ constexpr int dpair_off(int l, int mu) {
+// |m| = mu <= l the 2l+1 pairs (D^l[+mu][n], D^l[-mu][n]) as fp16x2, padded
+// to npair(l) = a multiple of 4 pairs so that a block is read with 16-byte
+// loads. A pair rotates into both x~[+mu] and x~[-mu] (producer) and rotates
+// o+ and o- back (epilogue). Block (l, mu) of an edge starts at pair dpo(l, mu).
+__host__ __device__ constexpr int npair(int l) { return (2 * l + 4) & ~3; }
+__host__ __device__ constexpr int dpo(int l, int mu) {
     int o = 0;
-    for (int k = 0; k < l; ++k) o += dpair_block(k);
-    return o + mu * (2 * l + 2);
+    for (int k = 0; k < l; ++k) o += (k + 1) * npair(k);
+    return o + mu * npair(l);
 }
-__host__ __device__ constexpr int dpairs(int L) { return dpair_off(L + 1, 0); }  // 110 at L = 4
-// Global scratch, per tile buffer, block-major: block (l, mu) holds 128 edges
-// x (2l+2) float2, so the epilogue fetches one group's slice in one bulk copy.
-__host__ __device__ constexpr size_t dglob_floats() { return 2ull * kTileE * dpairs(kMaxL); }
-__host__ __device__ constexpr size_t dglob_block(int l, int mu) { return 2ull * kTileE * dpair_off(l, mu); }
+__host__ __device__ constexpr int dptotal(int L) { return dpo(L + 1, 0); }  // 128 at L = 4
+// shared copy (producer): [edge][dptotal + 4] pairs; the 4 spare pairs move
+// consecutive edges 4 banks apart
+__host__ __device__ constexpr int dph_stride(int L) { return dptotal(L) + 4; }
+// global copy (epilogue), per tile buffer, block-major: block (l, mu) holds
+// 128 edges x npair(l) pairs, so a group's slice is one bulk copy
+__host__ __device__ constexpr size_t dglob_pairs() { return (size_t)kTileE * dptotal(kMaxL); }
+__host__ __device__ constexpr size_t dglob_block(int l, int mu) { return (size_t)kTileE * dpo(l, mu); }
+static_assert(npair(0) == 4 && npair(1) == 4 && npair(2) == 8 && npair(3) == 8 && npair(4) == 12, "pairs");
+static_assert(dptotal(4) == 128, "pair layout");
+
+// Bytes of Wigner pairs one group's epilogue stages: npair(l) pairs of 4
+// bytes per edge for each feature block the group covers (m = 0 groups cover
+// two 128-row blocks, possibly of different degrees).
+__host__ __device__ inline size_t stage_bytes(int L, int C) {
+    size_t mx = (size_t)kTileE * 4 * npair(L);  // an |m| >= 1 group of degree L
+    const int n0 = (L + 1) * C;
+    for (int r0 = 0; r0 < n0; r0 += 256) {
+        const int la = r0 / C, lb = (r0 + 128 < n0) ? (r0 + 128) / C : -1;
+        size_t b = (size_t)kTileE * 4 * npair(la);
+        if (lb >= 0) b += (size_t)kTileE * 4 * npair(lb);
+        mx = b > mx ? b : mx;
+    }
+    return mx;
+}
 
 // Shared memory layout (bytes), shared by host (size) and device (offsets).
 struct SmemLayout {
-    size_t ring, dstage, dph, pbuf, nid, jn, segm, rpw, rho, bars, misc, total;
-    __host__ __device__ SmemLayout(int L, int H, int n_rbf) {
+    size_t ring, dstage, dstride, dph, pch, nid, jn, segm, rpw, rho, wga, bars, misc, dsub, total;
+    __host__ __device__ SmemLayout(int L, int C, int H, int n_rbf) {
         size_t o = 0;
         ring = o;   o += (size_t)kNS * kStage;
-        dstage = o; o += 2ull * kStageD;
-        dph = o;    o += (size_t)kTileE * dpairs(L) * 4;
-        pbuf = o;   o += 2ull * kTileE * H * 4;
+        dstride = (stage_bytes(L, C) + 127) & ~size_t(127);
+        dstage = o; o += 2 * dstride;
+        dph = o;    o += (size_t)kTileE * dph_stride(L) * 4;
+        pch = o;    o += 2ull * kTileE * (C / 8) * 4;
         nid = o;    o += 2ull * kTileE * 4;
         jn = o;     o += 2ull * kTileE * 4;
         segm = o;   o += 2ull * (kTileE / kChunk) * 4;
         rpw = o;    o += (size_t)kTileE * 4;
         rho = o;    o += (size_t)kTileE * kTcMaxRbf * 2;
+        wga = o;    o += (size_t)kTcMaxRbf * kMaxHeads * 4;
         o = (o + 7) & ~size_t(7);
-        bars = o;   o += (2 * kNS + 11) * 8;
+        bars = o;   o += (2 * kNS + 15) * 8;
         misc = o;   o += 64;
+        dsub = o;   o += 16 * 8;
         total = o;
     }
 };
@@ -485,94 +520,81 @@ __device__ __forceinline__ uint32_t pack_h2(float a, float b) {
 //     acc[m'][c] += sum_e D_e[+mu][m'] y+[e][c] + D_e[-mu][m'] y-[e][c],
 //     y[e][c] = p_e^{head(c)} o[c][e],
 // i.e. the rotate-back D^T of the |m| = mu rows weighted by the softmax and
-// summed over the node's edges. A = Wigner rows (m' padded to 16, from the
-// staged pairs), B = p * o straight from tcgen05.ld.16x256b (whose thread
-// layout is the mma B/D fragment layout), D = fp32 accumulators. Node sums
-// go to out with fire-and-forget reductions at segment ends: one thread owns
-// each (node, l3, m', c) element, so the additions happen in program order.
-// Warp w covers channels cbase..cbase+31 (TMEM lanes 32w..32w+31).
+// summed over the node's edges. A = Wigner rows (m' padded to 16, built from
+// the staged fp16 pairs), B = p * o straight from tcgen05.ld.16x256b (whose
+// thread layout is the mma B/D fragment layout), D = fp32 accumulators.
+// Node sums go to out with fire-and-forget reductions at segment ends: one
+// thread owns each (node, l3, m', c) element, so the additions happen in
+// program order. The warp covers 16 TMEM lanes (channels cbase..cbase+15);
+// the two warps of a lane quadrant take one half each.
 template <int SIGNS>
-__device__ __noinline__ void epi_mma(uint32_t tacc, int l3, int cbase, int H, int dh, int K, int C,
-                                     const float2* __restrict__ Ds, const float* __restrict__ pb,
+__device__ __noinline__ void epi_mma(uint32_t tacc, int l3, int cbase, int K, int C,
+                                     const __half2* __restrict__ Ds, const float* __restrict__ pch,
                                      const int* __restrict__ nb, const uint32_t* __restrict__ segm,
                                      float* __restrict__ out) {
     const int lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
-    const int W3 = 2 * l3 + 1, DS = 2 * l3 + 2;
-    float acc[2][2][4];  // [lane half][n-tile lo/hi][fragment]
+    const int W3 = 2 * l3 + 1, NP = npair(l3), C8 = C / 8;
+    float acc[2][4];  // [n-tile lo/hi][fragment]
 #pragma unroll
-    for (int a = 0; a < 2; ++a)
+    for (int b2 = 0; b2 < 2; ++b2)
 #pragma unroll
-        for (int b2 = 0; b2 < 2; ++b2)
-#pragma unroll
-            for (int r = 0; r < 4; ++r) acc[a][b2][r] = 0.f;
+        for (int r = 0; r < 4; ++r) acc[b2][r] = 0.f;
     int cur = -1;
-    // heads of the B columns this thread loads: channel cbase + 16*hh + 8*lh + g
-    int hd[2][2];
-#pragma unroll
-    for (int hh = 0; hh < 2; ++hh)
-#pragma unroll
-        for (int lh = 0; lh < 2; ++lh) hd[hh][lh] = (cbase + 16 * hh + 8 * lh + g) / dh;
+    const float* pc = pch + cbase / 8;  // 8-channel groups cbase/8 (lh = 0) and +1 (lh = 1)
 
     auto flush = [&]() {
         if (cur < 0) return;
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh)
+        for (int lh = 0; lh < 2; ++lh)
 #pragma unroll
-            for (int lh = 0; lh < 2; ++lh)
-#pragma unroll
-                for (int r = 0; r < 4; ++r) {
-                    const int mp = g + ((r >> 1) << 3);
-                    if (mp < W3) {
-                        const int c = cbase + 16 * hh + 8 * lh + 2 * q + (r & 1);
-                        atomicAdd(out + ((size_t)cur * K + l3 * l3 + mp) * C + c, acc[hh][lh][r]);
-                    }
-                    acc[hh][lh][r] = 0.f;
+            for (int r = 0; r < 4; ++r) {
+                const int mp = g + ((r >> 1) << 3);
+                if (mp < W3) {
+                    const int c = cbase + 8 * lh + 2 * q + (r & 1);
+                    atomicAdd(out + ((size_t)cur * K + l3 * l3 + mp) * C + c, acc[lh][r]);
                 }
+                acc[lh][r] = 0.f;
+            }
     };
 
 #pragma unroll 1
     for (int ch = 0; ch < kTileE / 16; ++ch) {
         const int e0 = ch * 16;
-        // o values: [sign][lane half][edge half][4]: (c_lo,e), (c_lo,e+1), (c_hi,e), (c_hi,e+1)
-        uint32_t ov[SIGNS][2][2][4];
+        // o values: [sign][edge half][4]: (c_lo,e), (c_lo,e+1), (c_hi,e), (c_hi,e+1)
+        uint32_t ov[SIGNS][2][4];
 #pragma unroll
         for (int s2 = 0; s2 < SIGNS; ++s2)
 #pragma unroll
-            for (int hh = 0; hh < 2; ++hh)
-#pragma unroll
-                for (int eh = 0; eh < 2; ++eh)
-                    tmem_ld_16x256(tacc + s2 * 128 + ((uint32_t)(16 * hh) << 16) + e0 + 8 * eh, ov[s2][hh][eh]);
-        tmem_wait_ld();
+            for (int eh = 0; eh < 2; ++eh) tmem_ld_16x256(tacc + s2 * 128 + e0 + 8 * eh, ov[s2][eh]);
         // this thread's four edges: e0 + 2q, +1, e0 + 8 + 2q, +1
         const int ea = e0 + 2 * q, eb = e0 + 8 + 2 * q;
         // Wigner A fragments per sign: rows m' = g (a0, a2) and g + 8 (a1, a3)
         uint32_t af[SIGNS][4];
         {
             const bool r0 = g < W3, r1 = g + 8 < W3;
-            const float2 z = make_float2(0.f, 0.f);
-            const float2 d00 = r0 ? Ds[ea * DS + g] : z, d01 = r0 ? Ds[(ea + 1) * DS + g] : z;
-            const float2 d10 = r1 ? Ds[ea * DS + g + 8] : z, d11 = r1 ? Ds[(ea + 1) * DS + g + 8] : z;
-            const float2 d20 = r0 ? Ds[eb * DS + g] : z, d21 = r0 ? Ds[(eb + 1) * DS + g] : z;
-            const float2 d30 = r1 ? Ds[eb * DS + g + 8] : z, d31 = r1 ? Ds[(eb + 1) * DS + g + 8] : z;
-            af[0][0] = pack_h2(d00.x, d01.x); af[0][1] = pack_h2(d10.x, d11.x);
-            af[0][2] = pack_h2(d20.x, d21.x); af[0][3] = pack_h2(d30.x, d31.x);
+            const __half2 z = __float2half2_rn(0.f);
+            const __half2 p00 = r0 ? Ds[ea * NP + g] : z, p01 = r0 ? Ds[(ea + 1) * NP + g] : z;
+            const __half2 p10 = r1 ? Ds[ea * NP + g + 8] : z, p11 = r1 ? Ds[(ea + 1) * NP + g + 8] : z;
+            const __half2 p20 = r0 ? Ds[eb * NP + g] : z, p21 = r0 ? Ds[(eb + 1) * NP + g] : z;
+            const __half2 p30 = r1 ? Ds[eb * NP + g + 8] : z, p31 = r1 ? Ds[(eb + 1) * NP + g + 8] : z;
+            const __half2 lo[4] = {__lows2half2(p00, p01), __lows2half2(p10, p11), __lows2half2(p20, p21),
+                                   __lows2half2(p30, p31)};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) af[0][k] = *reinterpret_cast<const uint32_t*>(&lo[k]);
             if (SIGNS == 2) {
-                af[SIGNS - 1][0] = pack_h2(d00.y, d01.y); af[SIGNS - 1][1] = pack_h2(d10.y, d11.y);
-                af[SIGNS - 1][2] = pack_h2(d20.y, d21.y); af[SIGNS - 1][3] = pack_h2(d30.y, d31.y);
+                const __half2 hi[4] = {__highs2half2(p00, p01), __highs2half2(p10, p11), __highs2half2(p20, p21),
+                                       __highs2half2(p30, p31)};
+#pragma unroll
+                for (int k = 0; k < 4; ++k) af[SIGNS - 1][k] = *reinterpret_cast<const uint32_t*>(&hi[k]);
             }
         }
-        // softmax weights of the four edges for the B columns' heads
-        float pw[2][2][4];
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh)
-#pragma unroll
-            for (int lh = 0; lh < 2; ++lh) {
-                const int h = hd[hh][lh];
-                pw[hh][lh][0] = pb[ea * H + h];
-                pw[hh][lh][1] = pb[(ea + 1) * H + h];
-                pw[hh][lh][2] = pb[eb * H + h];
-                pw[hh][lh][3] = pb[(eb + 1) * H + h];
-            }
+        // softmax weights of the four edges for the two 8-channel groups
+        const float2 w0 = *reinterpret_cast<const float2*>(pc + ea * C8);
+        const float2 w1 = *reinterpret_cast<const float2*>(pc + (ea + 1) * C8);
+        const float2 w2 = *reinterpret_cast<const float2*>(pc + eb * C8);
+        const float2 w3 = *reinterpret_cast<const float2*>(pc + (eb + 1) * C8);
+        const float pw[2][4] = {{w0.x, w1.x, w2.x, w3.x}, {w0.y, w1.y, w2.y, w3.y}};
+        tmem_wait_ld();
         // segments of this chunk: bit k = edge e0 + k starts a node
         uint32_t bits = segm[ch];
         int lo = 0;
@@ -589,22 +611,20 @@ __device__ __noinline__ void epi_mma(uint32_t tacc, int l3, int cbase, int H, in
             const float m2 = (8 + 2 * q >= lo && 8 + 2 * q < hi) ? 1.f : 0.f;
             const float m3 = (9 + 2 * q >= lo && 9 + 2 * q < hi) ? 1.f : 0.f;
 #pragma unroll
-            for (int hh = 0; hh < 2; ++hh)
+            for (int lh = 0; lh < 2; ++lh) {
+                const float* pwv = pw[lh];
 #pragma unroll
-                for (int lh = 0; lh < 2; ++lh) {
-                    const float* pwv = pw[hh][lh];
-#pragma unroll
-                    for (int s2 = 0; s2 < SIGNS; ++s2) {
-                        const uint32_t* va = ov[s2][hh][0];
-                        const uint32_t* vb = ov[s2][hh][1];
-                        uint32_t bf[2];
-                        bf[0] = pack_h2(pwv[0] * m0 * __uint_as_float(va[2 * lh]),
-                                        pwv[1] * m1 * __uint_as_float(va[2 * lh + 1]));
-                        bf[1] = pack_h2(pwv[2] * m2 * __uint_as_float(vb[2 * lh]),
-                                        pwv[3] * m3 * __uint_as_float(vb[2 * lh + 1]));
-                        mma_16816(acc[hh][lh], af[s2], bf);
-                    }
+                for (int s2 = 0; s2 < SIGNS; ++s2) {
+                    const uint32_t* va = ov[s2][0];
+                    const uint32_t* vb = ov[s2][1];
+                    uint32_t bf[2];
+                    bf[0] = pack_h2(pwv[0] * m0 * __uint_as_float(va[2 * lh]),
+                                    pwv[1] * m1 * __uint_as_float(va[2 * lh + 1]));
+                    bf[1] = pack_h2(pwv[2] * m2 * __uint_as_float(vb[2 * lh]),
+                                    pwv[3] * m3 * __uint_as_float(vb[2 * lh + 1]));
+                    mma_16816(acc[lh], af[s2], bf);
                 }
+            }
             if (hi == 16) break;
             flush();
             cur = nb[e0 + hi];
@@ -617,22 +637,22 @@ __device__ __noinline__ void epi_mma(uint32_t tacc, int l3, int cbase, int H, in
 
 // Wigner slice(s) a group's epilogue needs, by block (l, mu): returns bytes
 // queued on `bar` into staging buffer `dst`.
-__device__ __forceinline__ uint32_t stage_group_pairs(const TcGroup& g, int C, const float* Dglob, uint8_t* dst,
+__device__ __forceinline__ uint32_t stage_group_pairs(const TcGroup& g, int C, const __half2* Dglob, uint8_t* dst,
                                                       uint64_t* bar) {
     if (g.mu > 0) {
         const int l3 = g.mu + g.row0 / C;
-        const uint32_t bytes = (uint32_t)kTileE * (2 * l3 + 2) * 8;
+        const uint32_t bytes = (uint32_t)kTileE * npair(l3) * 4;
         mbar_arrive_tx(bar, bytes);
         bulk_load(dst, Dglob + dglob_block(l3, g.mu), bytes, bar);
         return bytes;
     }
     const int la = g.row0 / C;
-    const uint32_t ba = (uint32_t)kTileE * (2 * la + 2) * 8;
+    const uint32_t ba = (uint32_t)kTileE * npair(la) * 4;
     uint32_t bb = 0;
     int lb = -1;
     if (g.row0b >= 0) {
         lb = g.row0b / C;
-        bb = (uint32_t)kTileE * (2 * lb + 2) * 8;
+        bb = (uint32_t)kTileE * npair(lb) * 4;
     }
     mbar_arrive_tx(bar, ba + bb);
     bulk_load(dst, Dglob + dglob_block(la, 0), ba, bar);
@@ -645,21 +665,21 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
                                                          const __grid_constant__ TcMaps T) {
     constexpr int K = n_sh(L);
     constexpr int WS = wig_size(L);
-    constexpr int NPAIR = dpairs(L);
+    constexpr int DPS = dph_stride(L);
     const int C = P.C, H = P.H, dh = C / H, G = P.G, NR = P.n_rbf;
-    const SmemLayout S(L, H, NR);
+    const SmemLayout S(L, C, H, NR);
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // operand tiles need 1024-byte alignment in the shared window
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint8_t* ring = smem + S.ring;
     uint8_t* dstage = smem + S.dstage;
     __half2* dph = reinterpret_cast<__half2*>(smem + S.dph);
-    float* pbuf = reinterpret_cast<float*>(smem + S.pbuf);
+    float* pch = reinterpret_cast<float*>(smem + S.pch);  // [2][128][C/8] softmax weight per 8 channels
     int* nid = reinterpret_cast<int*>(smem + S.nid);
     int* jn = reinterpret_cast<int*>(smem + S.jn);
     uint32_t* segm = reinterpret_cast<uint32_t*>(smem + S.segm);
     int* rpw = reinterpret_cast<int*>(smem + S.rpw);
-    __half* rho = reinterpret_cast<__half*>(smem + S.rho);  // [128][16] radial basis, fp16
+    __half* rho = reinterpret_cast<__half*>(smem + S.rho);  // [128][16] radial basis, fp16 (gate warps)
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S.bars);
     uint64_t* full = bars;
     uint64_t* empty = bars + kNS;
@@ -669,8 +689,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
     uint64_t* xfree = xready + 2;
     uint64_t* dbar = xfree + 2;   // epilogue Wigner staging, per buffer
     uint64_t* fin = dbar + 2;
+    uint64_t* gfull = fin + 1;    // value gate of a tile buffer written (gate warps -> producer)
+    uint64_t* gempty = gfull + 2; // value gate of a tile buffer consumed (producer -> gate warps)
     uint32_t* tmem_sm = reinterpret_cast<uint32_t*>(smem + S.misc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + S.misc + 8);
+    long long* dsub = reinterpret_cast<long long*>(smem + S.dsub);  // sub-step cycle sums (timers on)
+    float* wga = reinterpret_cast<float*>(smem + S.wga);            // [16][H] logit-gate weights
+    const bool dbgon = P.dbg != nullptr;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -678,16 +703,21 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
         for (int s = 0; s < kNS; ++s) { mbar_init(full + s, 1); mbar_init(empty + s, 1); }
         for (int b = 0; b < 2; ++b) {
             mbar_init(tfull + b, 1);
-            mbar_init(tempty + b, 128);
+            mbar_init(tempty + b, kEpiThreads);
             mbar_init(xready + b, 128);
-            mbar_init(xfree + b, 128);
+            mbar_init(xfree + b, kEpiThreads);
             mbar_init(dbar + b, 1);
         }
         mbar_init(fin, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(gfull + b, 64);
+            mbar_init(gempty + b, 128);
+        }
         *abort_flag = 0;
+        for (int k = 0; k < 16; ++k) dsub[k] = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    if (warp == 8) {
+    if (warp == 12) {
         tmem_alloc(tmem_sm, 512);
         tmem_relinquish();
     }
@@ -695,6 +725,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_sm;
+
 
     const int n_begin = P.part[blockIdx.x], n_end = P.part[blockIdx.x + 1];
     const int e_begin = P.row_ptr[n_begin], e_end = P.row_ptr[n_end];
@@ -708,8 +739,22 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
         const float inv_s = P.scale[1];
         const int CG = C / 8;
         const int Gv = (L + 1) * C;
-        __half* gs = P.gscr + (size_t)blockIdx.x * kTileE * Gv;
+        const int C8 = C / 8;
+        for (int t2 = p; t2 < kTcMaxRbf * H; t2 += 128) {
+            const int kb = t2 / H, h = t2 % H;
+            wga[t2] = kb < NR ? P.Wrad[(size_t)kb * G + Gv + h] : 0.f;
+        }
+        asm volatile("bar.sync 1, 128;" ::: "memory");
         int nbase = n_begin;
+        long long tlast = 0;
+#define E2F_TICK(k)                                                   \
+    do {                                                              \
+        if (dbgon && p == 0) {                                        \
+            const long long now_ = clock64();                         \
+            dsub[k] += now_ - tlast;                                  \
+            tlast = now_;                                             \
+        }                                                             \
+    } while (0)
         const size_t KT = (size_t)K * C;
         long long w_free = 0, c_p1 = 0, c_p2 = 0;
         const long long c_start = clock64();
@@ -738,11 +783,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
                 rpw[p] = (n <= n_end) ? P.row_ptr[n] : 0x7fffffff;
             }
             asm volatile("bar.sync 1, 128;" ::: "memory");
-            float* Dg = P.dscr + (size_t)(blockIdx.x * 2 + b) * dglob_floats();
-            // P1: one edge per thread: frame, Wigner pairs (shared f16 copy for
-            // the rotation below, global fp32 copy for the epilogue), softmax weight
+            tlast = c_a;
+            E2F_TICK(0);
+            __half2* Dg = P.dscr + (size_t)(blockIdx.x * 2 + b) * dglob_pairs();
+            // P1: one edge per thread: frame, Wigner pairs (fp16x2; shared copy for
+            // the rotation below, global copy for the epilogue), softmax weights
             {
-                __half2* Dh = dph + (size_t)p * NPAIR;
+                __half2* Dh = dph + (size_t)p * DPS;
                 if (p < ne) {
                     const int e = e0 + p;
                     const int j = P.col[e];
@@ -765,57 +812,83 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
                     }
                     float3 r = edge_vec(P.pos, i, j, P.box);
                     const float d = sqrtf(r.x * r.x + r.y * r.y + r.z * r.z);
+                    E2F_TICK(1);
                     float R[3][3];
                     edge_frame(r.x / d, r.y / d, r.z / d, R);
                     float D[WS];
                     wigner_blocks<L>(R, D);
+                    E2F_TICK(2);
 #pragma unroll
                     for (int l = 0; l <= L; ++l) {
                         const int w = 2 * l + 1;
                         const float* Dl = D + wig_off(l);
 #pragma unroll
                         for (int mu = 0; mu <= l; ++mu) {
-                            float4* gq = reinterpret_cast<float4*>(Dg + dglob_block(l, mu) + (size_t)p * 2 * (2 * l + 2));
+                            uint4* sq = reinterpret_cast<uint4*>(Dh + dpo(l, mu));
+                            uint4* gq = reinterpret_cast<uint4*>(Dg + dglob_block(l, mu) + (size_t)p * npair(l));
 #pragma unroll
-                            for (int n = 0; n < w; n += 2) {
-                                const float a0 = Dl[(l + mu) * w + n], b0 = Dl[(l - mu) * w + n];
-                                const float a1 = (n + 1 < w) ? Dl[(l + mu) * w + n + 1] : 0.f;
-                                const float b1 = (n + 1 < w) ? Dl[(l - mu) * w + n + 1] : 0.f;
-                                gq[n / 2] = make_float4(a0, b0, a1, b1);
-                                Dh[dpair_off(l, mu) + n] = __floats2half2_rn(a0, b0);
-                                Dh[dpair_off(l, mu) + n + 1] = __floats2half2_rn(a1, b1);
+                            for (int n4 = 0; n4 < npair(l); n4 += 4) {
+                                uint32_t wv[4];
+#pragma unroll
+                                for (int t4 = 0; t4 < 4; ++t4) {
+                                    const int n = n4 + t4;
+                                    const float a0 = n < w ? Dl[(l + mu) * w + n] : 0.f;
+                                    const float b0 = n < w ? Dl[(l - mu) * w + n] : 0.f;
+                                    wv[t4] = pack_h2(a0, b0);
+                                }
+                                const uint4 u = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+                                sq[n4 / 4] = u;
+                                gq[n4 / 4] = u;
                             }
                         }
                     }
+                    E2F_TICK(3);
                     float rr[kTcMaxRbf];
-                    rbf_all(d, P.cutoff, NR, rr);
-                    for (int kb = 0; kb < kTcMaxRbf; ++kb) {
-                        if (kb >= NR) rr[kb] = 0.f;
-                        rho[p * kTcMaxRbf + kb] = __float2half_rn(rr[kb]);
-                    }
-                    for (int h = 0; h < H; ++h) {
-                        float a = edge_logit(rr, NR, P.Wrad, G, G - H + h, P.q + (size_t)i * C + h * dh,
-                                             P.k + (size_t)j * C + h * dh, dh, inv_sqrt_dh);
-                        pbuf[(b * kTileE + p) * H + h] = expf(a - P.lse[(size_t)i * H + h]) * inv_s;
+                    rbf_all<kTcMaxRbf>(d, P.cutoff, NR, rr);
+                    E2F_TICK(4);
+                    {
+                        const float4* q4 = reinterpret_cast<const float4*>(P.q + (size_t)i * C);
+                        const float4* k4 = reinterpret_cast<const float4*>(P.k + (size_t)j * C);
+                        const int d4 = dh / 4;
+#pragma unroll 2
+                        for (int h = 0; h < H; ++h) {
+                            float ga = 0.f;
+#pragma unroll
+                            for (int kb = 0; kb < kTcMaxRbf; ++kb) ga = fmaf(rr[kb], wga[kb * H + h], ga);
+                            float dot = 0.f;
+                            for (int c4 = 0; c4 < d4; ++c4) {
+                                const float4 qa = __ldg(q4 + h * d4 + c4), kv = __ldg(k4 + h * d4 + c4);
+                                dot = fmaf(qa.x, kv.x, dot);
+                                dot = fmaf(qa.y, kv.y, dot);
+                                dot = fmaf(qa.z, kv.z, dot);
+                                dot = fmaf(qa.w, kv.w, dot);
+                            }
+                            const float a = ga * dot * inv_sqrt_dh;
+                            const float pw = expf(a - P.lse[(size_t)i * H + h]) * inv_s;
+                            for (int k8 = h * (dh / 8); k8 < (h + 1) * (dh / 8); ++k8)
+                                pch[(b * kTileE + p) * C8 + k8] = pw;
+                        }
                     }
                     nid[b * kTileE + p] = i;
                     jn[b * kTileE + p] = j;
+                    E2F_TICK(5);
                 } else {
+                    const uint4 z = make_uint4(0, 0, 0, 0);
 #pragma unroll
                     for (int l = 0; l <= L; ++l)
 #pragma unroll
                         for (int mu = 0; mu <= l; ++mu) {
-                            float4* gq = reinterpret_cast<float4*>(Dg + dglob_block(l, mu) + (size_t)p * 2 * (2 * l + 2));
-                            for (int n = 0; n < 2 * l + 1; n += 2) gq[n / 2] = make_float4(0.f, 0.f, 0.f, 0.f);
+                            uint4* gq = reinterpret_cast<uint4*>(Dg + dglob_block(l, mu) + (size_t)p * npair(l));
+                            for (int n4 = 0; n4 < npair(l); n4 += 4) gq[n4 / 4] = z;
                         }
-                    for (int a = 0; a < NPAIR; ++a) Dh[a] = __floats2half2_rn(0.f, 0.f);
-                    for (int kb = 0; kb < kTcMaxRbf; ++kb) rho[p * kTcMaxRbf + kb] = __float2half_rn(0.f);
-                    for (int h = 0; h < H; ++h) pbuf[(b * kTileE + p) * H + h] = 0.f;
+                    for (int a = 0; a < DPS; a += 4) *reinterpret_cast<uint4*>(Dh + a) = z;
+                    for (int k8 = 0; k8 < C8; ++k8) pch[(b * kTileE + p) * C8 + k8] = 0.f;
                     nid[b * kTileE + p] = -1;
                     jn[b * kTileE + p] = 0;
                 }
             }
             asm volatile("bar.sync 1, 128;" ::: "memory");
+            E2F_TICK(6);
             if (p < kTileE / kChunk) {  // segment starts per 16-edge chunk
                 uint32_t m = 0;
                 for (int q = 0; q < kChunk; ++q) {
@@ -824,41 +897,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
                 }
                 segm[b * (kTileE / kChunk) + p] = m;
             }
-            // P1.5: value gate g[e][n] = rho[e] . W_rad[:, n] for the tile (128 x (L+1)C), one k=16
-            // mma.sync per 16 edges x 8 columns; warp pw takes edge blocks 2pw and 2pw+1
-            {
-                const int pw = warp - 4, g8 = lane >> 2, t4 = lane & 3;
-                uint32_t af[2][4];
-#pragma unroll
-                for (int mb = 0; mb < 2; ++mb) {
-                    const int r0 = (2 * pw + mb) * 16 + g8;
-                    const __half* rr0 = rho + r0 * kTcMaxRbf + 2 * t4;
-                    af[mb][0] = *reinterpret_cast<const uint32_t*>(rr0);
-                    af[mb][1] = *reinterpret_cast<const uint32_t*>(rr0 + 8 * kTcMaxRbf);
-                    af[mb][2] = *reinterpret_cast<const uint32_t*>(rr0 + 8);
-                    af[mb][3] = *reinterpret_cast<const uint32_t*>(rr0 + 8 * kTcMaxRbf + 8);
-                }
-#pragma unroll 4
-                for (int n0 = 0; n0 < Gv; n0 += 8) {
-                    const __half* wb = P.whT + (size_t)(n0 + g8) * kTcMaxRbf + 2 * t4;
-                    uint32_t bf[2];
-                    bf[0] = __ldg(reinterpret_cast<const unsigned int*>(wb));
-                    bf[1] = __ldg(reinterpret_cast<const unsigned int*>(wb + 8));
-#pragma unroll
-                    for (int mb = 0; mb < 2; ++mb) {
-                        float acc4[4] = {0.f, 0.f, 0.f, 0.f};
-                        mma_16816(acc4, af[mb], bf);
-                        const int e = (2 * pw + mb) * 16 + g8;
-                        *reinterpret_cast<__half2*>(gs + (size_t)e * Gv + n0 + 2 * t4) = __floats2half2_rn(acc4[0], acc4[1]);
-                        *reinterpret_cast<__half2*>(gs + (size_t)(e + 8) * Gv + n0 + 2 * t4) =
-                            __floats2half2_rn(acc4[2], acc4[3]);
-                    }
-                }
-            }
             asm volatile("bar.sync 1, 128;" ::: "memory");
+            E2F_TICK(7);
             const long long c_b = clock64();
             c_p1 += c_b - c_a;
             // P2: rotated, gated features -> scratch row (e), all |m| blocks (fp16, packed math)
+            {
+                const bool okg = wait_t(gfull + b, (t >> 1) & 1, abort_flag, P.status, w_free);
+                if (!bar_and(1, 128, okg)) break;
+            }
+            const __half* gs = P.gscr + ((size_t)blockIdx.x * 2 + b) * kTileE * Gv;
             __half* xrow0 = P.xs + ((size_t)(blockIdx.x * 2 + b) * kTileE) * KT;
             for (int it = p; it < kTileE * CG; it += 128) {
                 const int e = it / CG, c0 = (it % CG) * 8;
@@ -873,7 +921,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
                     continue;
                 }
                 const int j = jn[b * kTileE + e];
-                const __half2* De = dph + (size_t)e * NPAIR;
+                const __half2* De = dph + (size_t)e * DPS;
                 // all (L+1)^2 rows of x_j for these 8 channels in flight at once
                 uint4 raw[K];
                 const __half* xj = P.x + (size_t)j * K * C + c0;
@@ -899,7 +947,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
 #pragma unroll
                     for (int mu = 0; mu <= kMaxL; ++mu) {
                         if (mu <= l1) {
-                            const __half2* Dq = De + dpair_off(l1, mu);
+                            const __half2* Dq = De + dpo(l1, mu);
                             __half2 op[4], om[4];
 #pragma unroll
                             for (int q = 0; q < 4; ++q) { op[q] = __float2half2_rn(0.f); om[q] = op[q]; }
@@ -923,16 +971,19 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
                     }
                 }
             }
+            mbar_arrive(gempty + b);  // this tile's value gates have been read
             // generic-proxy stores (features, Wigner pairs) -> visible to TMA / bulk copies
             asm volatile("fence.proxy.async.global;" ::: "memory");
             mbar_arrive(xready + b);
             c_p2 += clock64() - c_b;
         }
         if (P.dbg && p == 0) {
-            long long* d = P.dbg + blockIdx.x * 16;
+            long long* d = P.dbg + blockIdx.x * kDbgSlots;
             d[0] = w_free; d[1] = clock64() - c_start; d[11] = c_p1; d[12] = c_p2;
+            for (int k = 0; k < 8; ++k) d[14 + k] = dsub[k];
         }
-    } else if (warp == 8) {
+#undef E2F_TICK
+    } else if (warp == 12) {
         // ---------------- TMA ----------------
         if (lane == 0) {
             int stage = 0;
@@ -969,7 +1020,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
                 }
             }
             if (P.dbg) {
-                long long* d = P.dbg + blockIdx.x * 16;
+                long long* d = P.dbg + blockIdx.x * kDbgSlots;
                 d[2] = w_x; d[3] = w_e; d[4] = clock64() - c_start;
             }
             // every issued load lands (bounded wait) before the CTA can leave
@@ -981,7 +1032,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
             }
         }
         __syncwarp();
-    } else if (warp == 9) {
+    } else if (warp == 13) {
         // ---------------- MMA ----------------
         if (lane == 0) {
             int stage = 0;
@@ -1027,7 +1078,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
                 }
             }
             if (P.dbg) {
-                long long* d = P.dbg + blockIdx.x * 16;
+                long long* d = P.dbg + blockIdx.x * kDbgSlots;
                 d[5] = w_t; d[6] = w_f; d[7] = clock64() - c_start;
             }
             // every issued MMA completes (bounded wait) before TMEM is released
@@ -1037,8 +1088,79 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
             }
         }
         __syncwarp();
-    } else {
-        // ---------------- epilogue (warps 0-3, thread = TMEM lane) ----------------
+    } else if (warp >= 14) {
+        // ---------------- value gate (warps 14-15), up to two tiles ahead ----------------
+        // g[e][n] = rho(d_e) . W_rad[:, n] for the tile's 128 edges and n < (L+1)C, into a
+        // per-CTA global buffer per tile parity that the producer's rotation reads.
+        const int gp = threadIdx.x - 448, gw = warp - 14, g8 = lane >> 2, t4 = lane & 3;
+        const int Gv = (L + 1) * C;
+        long long w_g = 0;
+        const long long c_start = clock64();
+        for (int t = 0; t < ntiles; ++t) {
+            const int b = t & 1;
+            const bool okw = (t < 2) || wait_t(gempty + b, ((t - 2) >> 1) & 1, abort_flag, P.status, w_g);
+            if (!bar_and(3, 64, okw)) break;
+            const int e0 = e_begin + t * kTileE;
+            const int ne = min(kTileE, e_end - e0);
+            for (int k = gp; k < kTileE; k += 64) {  // radial basis of the tile's edges
+                float rr[kTcMaxRbf];
+                if (k < ne) {
+                    const int e = e0 + k, j = P.col[e];
+                    int lo = n_begin, hi = n_end - 1;  // node i: last n with row_ptr[n] <= e
+                    while (lo < hi) {
+                        const int mid = (lo + hi + 1) >> 1;
+                        if (P.row_ptr[mid] <= e) lo = mid; else hi = mid - 1;
+                    }
+                    const float3 r = edge_vec(P.pos, lo, j, P.box);
+                    const float d = sqrtf(r.x * r.x + r.y * r.y + r.z * r.z);
+                    rbf_all<kTcMaxRbf>(d, P.cutoff, NR, rr);
+                } else {
+#pragma unroll
+                    for (int kb = 0; kb < kTcMaxRbf; ++kb) rr[kb] = 0.f;
+                }
+                uint32_t hw[kTcMaxRbf / 2];
+#pragma unroll
+                for (int kb = 0; kb < kTcMaxRbf / 2; ++kb) hw[kb] = pack_h2(rr[2 * kb], rr[2 * kb + 1]);
+                uint4* rq = reinterpret_cast<uint4*>(rho + k * kTcMaxRbf);
+                rq[0] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+                rq[1] = make_uint4(hw[4], hw[5], hw[6], hw[7]);
+            }
+            asm volatile("bar.sync 3, 64;" ::: "memory");
+            // one k = 16 mma.sync per 16 edges x 8 columns; warp gw takes edge blocks 4 gw .. 4 gw + 3
+            __half* gs = P.gscr + ((size_t)blockIdx.x * 2 + b) * kTileE * Gv;
+            uint32_t af[4][4];
+#pragma unroll
+            for (int mb = 0; mb < 4; ++mb) {
+                const __half* rr0 = rho + ((4 * gw + mb) * 16 + g8) * kTcMaxRbf + 2 * t4;
+                af[mb][0] = *reinterpret_cast<const uint32_t*>(rr0);
+                af[mb][1] = *reinterpret_cast<const uint32_t*>(rr0 + 8 * kTcMaxRbf);
+                af[mb][2] = *reinterpret_cast<const uint32_t*>(rr0 + 8);
+                af[mb][3] = *reinterpret_cast<const uint32_t*>(rr0 + 8 * kTcMaxRbf + 8);
+            }
+#pragma unroll 2
+            for (int n0 = 0; n0 < Gv; n0 += 8) {
+                const __half* wb = P.whT + (size_t)(n0 + g8) * kTcMaxRbf + 2 * t4;
+                uint32_t bf[2];
+                bf[0] = __ldg(reinterpret_cast<const unsigned int*>(wb));
+                bf[1] = __ldg(reinterpret_cast<const unsigned int*>(wb + 8));
+#pragma unroll
+                for (int mb = 0; mb < 4; ++mb) {
+                    float acc4[4] = {0.f, 0.f, 0.f, 0.f};
+                    mma_16816(acc4, af[mb], bf);
+                    const int e = (4 * gw + mb) * 16 + g8;
+                    *reinterpret_cast<__half2*>(gs + (size_t)e * Gv + n0 + 2 * t4) = __floats2half2_rn(acc4[0], acc4[1]);
+                    *reinterpret_cast<__half2*>(gs + (size_t)(e + 8) * Gv + n0 + 2 * t4) =
+                        __floats2half2_rn(acc4[2], acc4[3]);
+                }
+            }
+            mbar_arrive(gfull + b);  // releases the stores above to the producer (CTA scope)
+        }
+        if (P.dbg && gp == 0) {
+            long long* d = P.dbg + blockIdx.x * kDbgSlots;
+            d[23] = w_g; d[24] = clock64() - c_start;
+        }
+    } else if (warp < 12) {
+        // ---------------- epilogue (warps 0-3 and 8-11) ----------------
         // Every decision to stop goes through bar_and, so the 128 threads leave
         // together and no thread is left at a named barrier.
         const int r = threadIdx.x;
@@ -1050,20 +1172,20 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
         for (int t = 0; t < ntiles; ++t) {
             const int b = t & 1;
             const bool okx = wait_t(xready + b, (t >> 1) & 1, abort_flag, P.status, w_x);
-            if (!bar_and(2, 128, ok && okx)) { ok = false; break; }
-            const float* Dg = P.dscr + (size_t)(blockIdx.x * 2 + b) * dglob_floats();
-            const float* pb = pbuf + (size_t)b * kTileE * H;
+            if (!bar_and(2, kEpiThreads, ok && okx)) { ok = false; break; }
+            const __half2* Dg = P.dscr + (size_t)(blockIdx.x * 2 + b) * dglob_pairs();
+            const float* pb = pch + (size_t)b * kTileE * (C / 8);
             const int* nb = nid + b * kTileE;
             const uint32_t* sg = segm + b * (kTileE / kChunk);
             if (r == 0) {
-                stage_group_pairs(P.groups[0], C, Dg, dstage + (gcount & 1) * kStageD, dbar + (gcount & 1));
+                stage_group_pairs(P.groups[0], C, Dg, dstage + (gcount & 1) * S.dstride, dbar + (gcount & 1));
                 staged[gcount & 1] = gcount;
             }
             for (int gi = 0; gi < ng; ++gi, ++gcount) {
                 // all threads are done with group gcount-1, so its staging buffer can be refilled
-                if (!bar_and(2, 128, ok)) { ok = false; break; }
+                if (!bar_and(2, kEpiThreads, ok)) { ok = false; break; }
                 if (r == 0 && gi + 1 < ng) {
-                    stage_group_pairs(P.groups[gi + 1], C, Dg, dstage + ((gcount + 1) & 1) * kStageD,
+                    stage_group_pairs(P.groups[gi + 1], C, Dg, dstage + ((gcount + 1) & 1) * S.dstride,
                                       dbar + ((gcount + 1) & 1));
                     staged[(gcount + 1) & 1] = gcount + 1;
                 }
@@ -1073,34 +1195,35 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
                 const bool okd = wait_t(dbar + slot, use & 1, abort_flag, P.status, w_t);
                 const bool okt = okd && wait_t(tfull + slot, use & 1, abort_flag, P.status, w_t);
                 if (okt) {
+                    const long long c_e0 = clock64();
                     tc_fence_after();
-                    const uint32_t tacc = tmem + ((uint32_t)(warp * 32) << 16) + slot * 256;
-                    const float2* Ds = reinterpret_cast<const float2*>(dstage + slot * kStageD);
-                    const uint32_t twarp = tmem + ((uint32_t)(warp * 32) << 16) + slot * 256;
+                    const __half2* Ds = reinterpret_cast<const __half2*>(dstage + slot * S.dstride);
+                    const int lrow = (warp & 3) * 32 + (warp >> 3) * 16;  // this warp's 16 TMEM lanes
+                    const uint32_t twarp = tmem + ((uint32_t)lrow << 16) + slot * 256;
                     if (g.mu > 0) {
-                        const int row = g.row0 + warp * 32;  // rows of this warp: one l3, 32 channels
-                        epi_mma<2>(twarp, g.mu + row / C, row % C, H, dh, K, C, Ds, pb, nb, sg, P.out);
+                        const int row = g.row0 + lrow;  // rows of this warp: one l3, 16 channels
+                        epi_mma<2>(twarp, g.mu + row / C, row % C, K, C, Ds, pb, nb, sg, P.out);
                     } else {
-                        const int ra = g.row0 + warp * 32, la = ra / C;
-                        epi_mma<1>(twarp, la, ra % C, H, dh, K, C, Ds, pb, nb, sg, P.out);
+                        const int ra = g.row0 + lrow, la = ra / C;
+                        epi_mma<1>(twarp, la, ra % C, K, C, Ds, pb, nb, sg, P.out);
                         if (g.row0b >= 0) {
-                            const int rb = g.row0b + warp * 32;
-                            epi_mma<1>(twarp + 128, rb / C, rb % C, H, dh, K, C, Ds + kTileE * (2 * la + 2), pb,
-                                       nb, sg, P.out);
+                            const int rb = g.row0b + lrow;
+                            epi_mma<1>(twarp + 128, rb / C, rb % C, K, C, Ds + kTileE * npair(la), pb, nb, sg, P.out);
                         }
                     }
                     tc_fence_before();
+                    if (dbgon && r == 0) dsub[8] += clock64() - c_e0;
                 } else {
                     ok = false;
                 }
                 mbar_arrive(tempty + slot);
             }
-            if (!bar_and(2, 128, ok)) { ok = false; break; }
+            if (!bar_and(2, kEpiThreads, ok)) { ok = false; break; }
             mbar_arrive(xfree + b);
         }
         if (P.dbg && r == 0) {
-            long long* d = P.dbg + blockIdx.x * 16;
-            d[8] = w_x; d[9] = w_t; d[10] = clock64() - c_start; d[13] = ntiles;
+            long long* d = P.dbg + blockIdx.x * kDbgSlots;
+            d[8] = w_x; d[9] = w_t; d[10] = clock64() - c_start; d[13] = ntiles; d[22] = dsub[8];
         }
         // a staging copy that was issued but never waited for lands before exit
         if (r == 0) {
@@ -1115,7 +1238,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 8) {
+    if (warp == 12) {
         tc_fence_after();
         tmem_dealloc(tmem, 512);
     }
@@ -1160,7 +1283,8 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows) {
 
 bool tc_supported(int L, int C, int H, int n_rbf, bool bf16) {
     return bf16 && L >= 1 && L <= kMaxL && C % 128 == 0 && C <= 256 && H <= kMaxHeads && H % 4 == 0 &&
-           n_rbf <= kTcMaxRbf && tc::SmemLayout(L, H, n_rbf).total + 1024 <= 232448;
+           C % H == 0 && (C / H) % 8 == 0 &&
+           n_rbf <= kTcMaxRbf && tc::SmemLayout(L, C, H, n_rbf).total + 1024 <= 232448;
 }
 
 namespace {
@@ -1174,11 +1298,11 @@ struct TcWs {
         lse = take(4 * (size_t)n_atoms * H);
         part = take(4 * (size_t)(kMaxCtas + 1));
         xs = take((size_t)kMaxCtas * 2 * tc::kTileE * K * C * 2);
-        dscr = take((size_t)kMaxCtas * 2 * tc::dglob_floats() * 4);
+        dscr = take((size_t)kMaxCtas * 2 * tc::dglob_pairs() * 4);
         x16 = take((size_t)n_atoms * K * C * 2);
         w16 = take(so2_total(L, C) * 2);
         whT = take((size_t)Gv * kTcMaxRbf * 2);
-        gscr = take((size_t)kMaxCtas * tc::kTileE * Gv * 2);
+        gscr = take((size_t)kMaxCtas * 2 * tc::kTileE * Gv * 2);  // two tile buffers per CTA
         words = take(256);
         total = o;
     }
@@ -1189,7 +1313,7 @@ size_t tc_workspace_bytes(int64_t n_atoms, int L, int C, int H) { return TcWs(n_
 
 template <int L>
 static cudaError_t launch_tc(const tc::TcParams& P, const tc::TcMaps& T, int grid, cudaStream_t s) {
-    const size_t smem = tc::SmemLayout(L, P.H, P.n_rbf).total + 1024;
+    const size_t smem = tc::SmemLayout(L, P.C, P.H, P.n_rbf).total + 1024;
     cudaError_t e = cudaFuncSetAttribute(tc::k_attn_tc<L>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     count_launch();
@@ -1216,7 +1340,7 @@ cudaError_t run_attention_tc(const AttnArgs& a, void* tc_ws, cudaStream_t s) {
     float* lse = reinterpret_cast<float*>(w + Wl.lse);
     int32_t* part = reinterpret_cast<int32_t*>(w + Wl.part);
     __half* xs = reinterpret_cast<__half*>(w + Wl.xs);
-    float* dscr = reinterpret_cast<float*>(w + Wl.dscr);
+    __half2* dscr = reinterpret_cast<__half2*>(w + Wl.dscr);
     __half* x16 = reinterpret_cast<__half*>(w + Wl.x16);
     __half* w16 = reinterpret_cast<__half*>(w + Wl.w16);
     __half* whT = reinterpret_cast<__half*>(w + Wl.whT);

@@ -14,7 +14,8 @@ constexpr int kMaxHeads = 16;   // tensor-core path: H <= 16
 constexpr int kMaxRbf = 32;
 constexpr int kTcMaxRbf = 16;   // tensor-core path: the radial gate is one k=16 mma
 constexpr int kMaxCtas = 160;   // persistent CTAs (one per SM; B200 has 148)
-constexpr size_t kTcDebugBytes = (size_t)kMaxCtas * 16 * 8;  // per-CTA role timers
+constexpr int kDbgSlots = 32;                                         // counters per CTA
+constexpr size_t kTcDebugBytes = (size_t)kMaxCtas * kDbgSlots * 8;  // per-CTA role timers
 
 struct StatsParams {
     int n_atoms, C, H, n_rbf, G;
@@ -50,7 +51,7 @@ struct TcParams {
     const int32_t* col;
     const __half* x;       // features in fp16, scaled by scale[0] (an exact power of two)
     const __half* whT;     // value-gate weights, fp16, [(L+1)C][16] (radial index innermost, zero padded)
-    __half* gscr;          // per-CTA value-gate scratch [n_ctas][128][(L+1)C]
+    __half* gscr;          // per-CTA value-gate scratch [n_ctas][2 tile buffers][128][(L+1)C]
     const float* scale;    // [0] feature scale s, [1] 1/s
     const float* q;
     const float* k;
@@ -58,7 +59,7 @@ struct TcParams {
     const float* Wrad;
     const int32_t* part;
     __half* xs;
-    float* dscr;     // per-CTA Wigner pair blocks [n_ctas * 2 * 128][kDStride]
+    __half2* dscr;   // per-CTA Wigner pair blocks (fp16x2), two tile buffers per CTA
     float* out;
     int* status;
     long long* dbg;  // per-CTA role cycle counters, or null

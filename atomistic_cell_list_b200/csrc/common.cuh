@@ -178,13 +178,16 @@ __device__ __forceinline__ float rbf(float d, int k, float cutoff, int n_rbf) {
     return u * expf(-t * t);
 }
 
-// all n_rbf basis values of one distance (the envelope evaluated once)
+// all n_rbf basis values of one distance (the envelope evaluated once);
+// out[k] = 0 for n_rbf <= k < NMAX (unrolled: out stays in registers)
+template <int NMAX>
 __device__ __forceinline__ void rbf_all(float d, float cutoff, int n_rbf, float* out) {
     const float step = cutoff / float(n_rbf - 1);
     const float u = 0.5f * (cosf(3.14159265358979323846f * d / cutoff) + 1.f);
-    for (int k = 0; k < n_rbf; ++k) {
+#pragma unroll
+    for (int k = 0; k < NMAX; ++k) {
         const float t = (d - float(k) * step) / step;
-        out[k] = u * expf(-t * t);
+        out[k] = k < n_rbf ? u * expf(-t * t) : 0.f;
     }
 }
 

@@ -195,13 +195,16 @@ int e2f_attention_uses_tensor_cores(const e2f_attn_cfg* cfg);
 
 /* Diagnostics of the tensor-core kernel. When the environment variable
  * E2F_TC_TIMERS=1 is set at call time, each persistent CTA records clock64
- * cycle counts of its warp roles into the workspace: per CTA 16 int64 values,
+ * cycle counts of its warp roles into the workspace: per CTA 32 int64 values,
  * [0] producer wait for a free tile buffer, [1] producer total, [2] TMA wait
  * for features, [3] TMA wait for a free ring stage, [4] TMA total, [5] MMA
  * wait for a free TMEM group, [6] MMA wait for a full stage, [7] MMA total,
  * [8] epilogue wait for tile data, [9] epilogue wait for accumulators,
  * [10] epilogue total, [11] producer per-edge setup, [12] producer feature
- * rotation, [13] tiles. Copies the first n_values counters to host_out
+ * rotation, [13] tiles, [14..21] sub-steps of the per-edge setup (one
+ * thread's view: node search, geometry, Wigner blocks, their stores, radial
+ * basis, logits, barrier, value gate), [22] epilogue rotate-back; the rest
+ * is zero. Copies the first n_values counters to host_out
  * (synchronises `stream`). No counterpart in the paper: a profiling aid. */
 e2f_status e2f_attention_debug_timers(void* workspace, size_t ws_bytes, int64_t n_atoms,
                                       const e2f_attn_cfg* cfg, int64_t* host_out, int n_values,
