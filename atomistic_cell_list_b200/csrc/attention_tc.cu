@@ -450,7 +450,7 @@ __host__ __device__ inline size_t stage_bytes(int L, int C) {
 
 // Shared memory layout (bytes), shared by host (size) and device (offsets).
 struct SmemLayout {
-    size_t ring, dstage, dstride, dph, pch, nid, jn, segm, rpw, rho, wga, bars, misc, dsub, total;
+    size_t ring, dstage, dstride, dph, pch, nid, jn, segm, rpw, rho, rrs, wga, bars, misc, dsub, total;
     __host__ __device__ SmemLayout(int L, int C, int H, int n_rbf) {
         size_t o = 0;
         ring = o;   o += (size_t)kNS * kStage;
@@ -463,6 +463,7 @@ struct SmemLayout {
         segm = o;   o += 2ull * (kTileE / kChunk) * 4;
         rpw = o;    o += (size_t)kTileE * 4;
         rho = o;    o += (size_t)kTileE * kTcMaxRbf * 2;
+        rrs = o;    o += (size_t)kTileE * kTcMaxRbf * 4;
         wga = o;    o += (size_t)kTcMaxRbf * kMaxHeads * 4;
         o = (o + 7) & ~size_t(7);
         bars = o;   o += (2 * kNS + 15) * 8;
@@ -680,6 +681,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
     uint32_t* segm = reinterpret_cast<uint32_t*>(smem + S.segm);
     int* rpw = reinterpret_cast<int*>(smem + S.rpw);
     __half* rho = reinterpret_cast<__half*>(smem + S.rho);  // [128][16] radial basis, fp16 (gate warps)
+    float* rrs = reinterpret_cast<float*>(smem + S.rrs);    // [128][16] radial basis, fp32 (logits)
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S.bars);
     uint64_t* full = bars;
     uint64_t* empty = bars + kNS;
@@ -845,33 +847,20 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
                     E2F_TICK(3);
                     float rr[kTcMaxRbf];
                     rbf_all<kTcMaxRbf>(d, P.cutoff, NR, rr);
-                    E2F_TICK(4);
                     {
-                        const float4* q4 = reinterpret_cast<const float4*>(P.q + (size_t)i * C);
-                        const float4* k4 = reinterpret_cast<const float4*>(P.k + (size_t)j * C);
-                        const int d4 = dh / 4;
-#pragma unroll 2
-                        for (int h = 0; h < H; ++h) {
-                            float ga = 0.f;
+                        float4* rq = reinterpret_cast<float4*>(rrs + p * kTcMaxRbf);
 #pragma unroll
-                            for (int kb = 0; kb < kTcMaxRbf; ++kb) ga = fmaf(rr[kb], wga[kb * H + h], ga);
-                            float dot = 0.f;
-                            for (int c4 = 0; c4 < d4; ++c4) {
-                                const float4 qa = __ldg(q4 + h * d4 + c4), kv = __ldg(k4 + h * d4 + c4);
-                                dot = fmaf(qa.x, kv.x, dot);
-                                dot = fmaf(qa.y, kv.y, dot);
-                                dot = fmaf(qa.z, kv.z, dot);
-                                dot = fmaf(qa.w, kv.w, dot);
-                            }
-                            const float a = ga * dot * inv_sqrt_dh;
-                            const float pw = expf(a - P.lse[(size_t)i * H + h]) * inv_s;
-                            for (int k8 = h * (dh / 8); k8 < (h + 1) * (dh / 8); ++k8)
-                                pch[(b * kTileE + p) * C8 + k8] = pw;
-                        }
+                        for (int k4 = 0; k4 < kTcMaxRbf / 4; ++k4)
+                            rq[k4] = make_float4(rr[4 * k4], rr[4 * k4 + 1], rr[4 * k4 + 2], rr[4 * k4 + 3]);
                     }
+                    // the neighbour's feature row is read by the rotation below: start it towards L2
+                    if (p < 16)
+                        asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(P.x + (size_t)j * KT),
+                                     "r"((uint32_t)(KT * 2))
+                                     : "memory");
+                    E2F_TICK(4);
                     nid[b * kTileE + p] = i;
                     jn[b * kTileE + p] = j;
-                    E2F_TICK(5);
                 } else {
                     const uint4 z = make_uint4(0, 0, 0, 0);
 #pragma unroll
@@ -889,6 +878,43 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
             }
             asm volatile("bar.sync 1, 128;" ::: "memory");
             E2F_TICK(6);
+            // logits and softmax weights, one (edge, head) pair per thread and step: the
+            // thread's head h = p % H is fixed (H divides 128), the H lanes of an edge read
+            // its key row as consecutive float4
+            {
+                const int h = p % H, d4 = dh / 4;
+                float wh[kTcMaxRbf];
+#pragma unroll
+                for (int kb = 0; kb < kTcMaxRbf; ++kb) wh[kb] = wga[kb * H + h];
+#pragma unroll 2
+                for (int e = p / H; e < ne; e += kTileE / H) {
+                    const int i = nid[b * kTileE + e], j = jn[b * kTileE + e];
+                    const float4* rq = reinterpret_cast<const float4*>(rrs + e * kTcMaxRbf);
+                    float ga = 0.f;
+#pragma unroll
+                    for (int k4 = 0; k4 < kTcMaxRbf / 4; ++k4) {
+                        const float4 r4 = rq[k4];
+                        ga = fmaf(r4.x, wh[4 * k4], ga);
+                        ga = fmaf(r4.y, wh[4 * k4 + 1], ga);
+                        ga = fmaf(r4.z, wh[4 * k4 + 2], ga);
+                        ga = fmaf(r4.w, wh[4 * k4 + 3], ga);
+                    }
+                    const float4* q4 = reinterpret_cast<const float4*>(P.q + (size_t)i * C + h * dh);
+                    const float4* k4 = reinterpret_cast<const float4*>(P.k + (size_t)j * C + h * dh);
+                    float dot = 0.f;
+                    for (int c4 = 0; c4 < d4; ++c4) {
+                        const float4 qa = __ldg(q4 + c4), kv = __ldg(k4 + c4);
+                        dot = fmaf(qa.x, kv.x, dot);
+                        dot = fmaf(qa.y, kv.y, dot);
+                        dot = fmaf(qa.z, kv.z, dot);
+                        dot = fmaf(qa.w, kv.w, dot);
+                    }
+                    const float a = ga * dot * inv_sqrt_dh;
+                    const float pw = expf(a - P.lse[(size_t)i * H + h]) * inv_s;
+                    for (int k8 = h * (dh / 8); k8 < (h + 1) * (dh / 8); ++k8) pch[(b * kTileE + e) * C8 + k8] = pw;
+                }
+            }
+            E2F_TICK(5);
             if (p < kTileE / kChunk) {  // segment starts per 16-edge chunk
                 uint32_t m = 0;
                 for (int q = 0; q < kChunk; ++q) {
@@ -921,6 +947,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
                     continue;
                 }
                 const int j = jn[b * kTileE + e];
+                if (c0 == 0 && e + 16 < ne)  // neighbour row of the edge two rounds ahead
+                    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(
+                                     P.x + (size_t)jn[b * kTileE + e + 16] * KT),
+                                 "r"((uint32_t)(KT * 2))
+                                 : "memory");
                 const __half2* De = dph + (size_t)e * DPS;
                 // all (L+1)^2 rows of x_j for these 8 channels in flight at once
                 uint4 raw[K];
