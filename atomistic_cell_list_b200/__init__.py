@@ -54,6 +54,7 @@ _SIGS = {
     "e2f_edge_wigner_blocks": (ctypes.c_int, [_vp, _i64, ctypes.c_int, _vp, _vp, _vp]),
     "e2f_launch_count": (_i64, []),
     "e2f_attention_uses_tensor_cores": (ctypes.c_int, [ctypes.POINTER(e2f_attn_cfg)]),
+    "e2f_attention_set_kernel_events": (None, [_vp, _vp]),
     "e2f_attention_debug_timers": (ctypes.c_int, [_vp, _sz, _i64, ctypes.POINTER(e2f_attn_cfg),
                                                   ctypes.POINTER(_i64), ctypes.c_int, _vp]),
 }
@@ -244,6 +245,13 @@ def e2f_attention_debug_timers(workspace: torch.Tensor, n_atoms: int, cfg: e2f_a
     _check(lib().e2f_attention_debug_timers(_ptr(workspace), workspace.numel(), int(n_atoms), ctypes.byref(cfg), buf,
                                             n, _stream(stream)), "e2f_attention_debug_timers")
     return np.frombuffer(buf, dtype=np.int64).reshape(n_ctas, DEBUG_SLOTS).copy()
+
+
+def e2f_attention_set_kernel_events(start=None, stop=None):
+    """Record torch.cuda.Event pair around the next calls' main kernel (None, None: off)."""
+    a = None if start is None else ctypes.c_void_p(start.cuda_event)
+    b = None if stop is None else ctypes.c_void_p(stop.cuda_event)
+    lib().e2f_attention_set_kernel_events(a, b)
 
 
 def e2f_launch_count() -> int:

@@ -149,6 +149,10 @@ extern "C" int e2f_attention_uses_tensor_cores(const e2f_attn_cfg* cfg) {
     return tc_supported(cfg->L, cfg->C, cfg->H, cfg->n_rbf, cfg->feat_dtype == E2F_BF16) ? 1 : 0;
 }
 
+extern "C" void e2f_attention_set_kernel_events(void* start_event, void* stop_event) {
+    set_tc_kernel_events(start_event, stop_event);
+}
+
 extern "C" e2f_status e2f_attention_debug_timers(void* workspace, size_t ws_bytes, int64_t n_atoms,
                                                 const e2f_attn_cfg* cfg, int64_t* host_out, int n_values,
                                                 void* stream_) {

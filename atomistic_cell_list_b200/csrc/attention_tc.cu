@@ -1342,6 +1342,17 @@ struct TcWs {
 
 size_t tc_workspace_bytes(int64_t n_atoms, int L, int C, int H) { return TcWs(n_atoms, L, C, H).total; }
 
+namespace {
+// caller events recorded around the main kernel (profiling aid; see
+// e2f_attention_set_kernel_events)
+cudaEvent_t g_kernel_ev[2] = {nullptr, nullptr};
+}  // namespace
+
+void set_tc_kernel_events(void* start, void* stop) {
+    g_kernel_ev[0] = static_cast<cudaEvent_t>(start);
+    g_kernel_ev[1] = static_cast<cudaEvent_t>(stop);
+}
+
 template <int L>
 static cudaError_t launch_tc(const tc::TcParams& P, const tc::TcMaps& T, int grid, cudaStream_t s) {
     const size_t smem = tc::SmemLayout(L, P.C, P.H, P.n_rbf).total + 1024;
@@ -1458,6 +1469,19 @@ cudaError_t run_attention_tc(const AttnArgs& a, void* tc_ws, cudaStream_t s) {
     }
     if (!make_map(&T.xs, xs, (uint64_t)K * C, (uint64_t)grid * 2 * tc::kTileE)) return cudaErrorInvalidValue;
 
+    if (g_kernel_ev[0] && g_kernel_ev[1]) {
+        e = cudaEventRecord(g_kernel_ev[0], s);
+        if (e != cudaSuccess) return e;
+        switch (L) {
+            case 1: e = launch_tc<1>(P, T, grid, s); break;
+            case 2: e = launch_tc<2>(P, T, grid, s); break;
+            case 3: e = launch_tc<3>(P, T, grid, s); break;
+            case 4: e = launch_tc<4>(P, T, grid, s); break;
+            default: return cudaErrorInvalidValue;
+        }
+        if (e != cudaSuccess) return e;
+        return cudaEventRecord(g_kernel_ev[1], s);
+    }
     switch (L) {
         case 1: return launch_tc<1>(P, T, grid, s);
         case 2: return launch_tc<2>(P, T, grid, s);

@@ -47,6 +47,31 @@ def measured_peaks():
         "fallback"
 
 
+# DRAM traffic of one k_attn_tc launch on the 30000-atom workload, from the ncu
+# capture summarised in profiles/k_attn_tc_chain_water_30k.md. Valid only for
+# the kernel source it was taken on (sha256 of the files below); otherwise the
+# bench reports traffic null.
+KERNEL_TRAFFIC = {
+    "sources": ["atomistic_cell_list_b200/csrc/attention_tc.cu", "atomistic_cell_list_b200/csrc/attention_tc.cuh",
+                "atomistic_cell_list_b200/csrc/common.cuh"],
+    "sha256": "df05443b1baac352ef2328a7359e68eb460a2a17bb364565968c705552fb7ee6",
+    "dram_read_bytes": 46.28e9,
+    "dram_write_bytes": 24.20e9,
+}
+
+
+def kernel_traffic():
+    import hashlib
+    if KERNEL_TRAFFIC["sha256"] is None:
+        return None
+    h = hashlib.sha256()
+    for f in KERNEL_TRAFFIC["sources"]:
+        h.update(open(os.path.join(ROOT, f), "rb").read())
+    if h.hexdigest() != KERNEL_TRAFFIC["sha256"]:
+        return None
+    return KERNEL_TRAFFIC["dram_read_bytes"] + KERNEL_TRAFFIC["dram_write_bytes"]
+
+
 def workload_desc(w):
     return {"workload": f"cfg{w.cfg_id}: {w.name}, cutoff {w.cutoff} A, L={w.L} C={w.C} H={w.H}, "
                         f"{w.dtype} features",
@@ -234,6 +259,11 @@ def run_ours(args):
     assert e2f.e2f_attention_status(ws) == 0
 
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    # events around the main attention kernel alone (recorded by the library on this stream)
+    kev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    for pair in kev:
+        for e_ in pair:
+            e_.record(stream)  # materialise the CUDA events before handing them over
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
@@ -244,9 +274,11 @@ def run_ours(args):
             ev[s][0].record(stream)
             rp_, col_ = step()
             ev[s][1].record(stream)
+            e2f.e2f_attention_set_kernel_events(kev[s][0], kev[s][1])
             attn(rp_, col_)
             ev[s][2].record(stream)
         torch.cuda.synchronize(dev)
+    e2f.e2f_attention_set_kernel_events(None, None)
     launches = e2f.e2f_launch_count() - n0 - 0
     if world > 1:
         dist.barrier()
@@ -255,12 +287,15 @@ def run_ours(args):
     t_step = [ev[s][0].elapsed_time(ev[s][2]) for s in range(args.steps)]
     t_nbr = [ev[s][0].elapsed_time(ev[s][1]) for s in range(args.steps)]
     t_att = [ev[s][1].elapsed_time(ev[s][2]) for s in range(args.steps)]
-    tot = torch.tensor([sum(t_step), sum(t_att), sum(t_nbr)], dtype=torch.float64, device=dev)
+    use_tc = e2f.e2f_attention_uses_tensor_cores(cfg)
+    t_ker = [kev[s][0].elapsed_time(kev[s][1]) for s in range(args.steps)] if use_tc else t_att
+    tot = torch.tensor([sum(t_step), sum(t_att), sum(t_nbr), sum(t_ker)], dtype=torch.float64, device=dev)
     if world > 1:
         dist.all_reduce(tot, op=dist.ReduceOp.MAX)
     ms_step = float(tot[0]) / args.steps
     ms_att = float(tot[1]) / args.steps
     ms_nbr = float(tot[2]) / args.steps
+    ms_ker = float(tot[3]) / args.steps
 
     # end to end through the public API with pinned host buffers
     pinned = {k: v.pin_memory() for k, v in h_inputs.items()}
@@ -285,22 +320,27 @@ def run_ours(args):
 
     peaks, peak_src = measured_peaks()
     F = so2_flops_per_edge(w.L, w.C)
-    tflops = E * F / (ms_att * 1e-3) / 1e12
-    path = "tensor" if e2f.e2f_attention_uses_tensor_cores(cfg) else "simt"
+    tflops = E * F / (ms_att * 1e-3) / 1e12          # whole attention call (with its O(N) pre-passes)
+    tflops_ker = E * F / (ms_ker * 1e-3) / 1e12      # the main kernel alone
+    path = "tensor" if use_tc else "simt"
     if path == "simt":
         clk_max = float(peaks.get("sm_max_mhz", 1965.0))
         peak = 148 * 128 * 2 * clk_max * 1e6 / 1e12
-        roof = {"bound": "alu", "achieved": tflops, "peak": peak, "unit": "TFLOP/s", "frac": tflops / peak,
+        roof = {"bound": "alu", "achieved": tflops_ker, "peak": peak, "unit": "TFLOP/s", "frac": tflops_ker / peak,
                 "traffic": None,
                 "peak_note": f"fp32 FMA pipe: 148 SMs x 128 lanes x 2 FLOP x {clk_max:.0f} MHz (derived, "
                              f"{peak_src} clock)"}
     else:
         peak = float(peaks["bf16_tflops"])
-        roof = {"bound": "tensor", "achieved": tflops, "peak": peak, "unit": "TFLOP/s", "frac": tflops / peak,
-                "traffic": None, "peak_note": f"bf16 dense, {peak_src}"}
-    roof["kernel"] = ("k_attn_tc (tcgen05) + its O(N) pre-passes" if path == "tensor"
-                      else "k_attn_simt (fp32 CUDA cores) + its O(N) pre-passes")
-    roof["traffic_note"] = "see profiles/ (ncu)"
+        sus = float(peaks.get("bf16_tflops_sustained", peak))
+        roof = {"bound": "tensor", "achieved": tflops_ker, "peak": peak, "unit": "TFLOP/s", "frac": tflops_ker / peak,
+                "traffic": kernel_traffic(), "peak_note": f"bf16 dense burst, {peak_src}",
+                "peak_sustained": sus, "frac_sustained": tflops_ker / sus}
+    roof["kernel"] = "k_attn_tc (tcgen05)" if path == "tensor" else "k_attn_simt (fp32 CUDA cores)"
+    roof["ms_per_launch"] = ms_ker
+    roof["units_per_launch"] = f"{E} edges x {F} SO(2) FLOP"
+    roof["traffic_note"] = ("dram read+write bytes per launch from ncu (profiles/k_attn_tc_chain_water_30k.md); "
+                            "null when the kernel source differs from the profiled one")
 
     line = {"metric": METRIC, "value": world * E / (ms_step * 1e-3), "unit": "pairs/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
@@ -308,12 +348,17 @@ def run_ours(args):
             "data": "synthetic",
             "config": {**workload_desc(w), "n_pairs": E, "parallelism": f"replicas x{world}",
                        "l2": "flushed (256 MB write) between timed steps"},
-            "tflops": tflops, "ms_attention": ms_att, "ms_neighbors": ms_nbr,
+            "tflops": tflops, "tflops_kernel": tflops_ker, "ms_attention": ms_att, "ms_attention_kernel": ms_ker,
+            "ms_neighbors": ms_nbr,
             "neighbor_pairs_per_s": E / (ms_nbr * 1e-3), "attention_pairs_per_s": E / (ms_att * 1e-3),
             "roofline": roof,
             "e2e": {"value": world * E / (ms_e2e * 1e-3), "unit": "pairs/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e},
             "gpu_launches": int(launches),
+            "activation_memory": {"workspace_bytes": int(ws.numel()), "edge_tensor_bytes": 0,
+                                  "csr_bytes": 4 * (w.n_atoms + 1) + 4 * E,
+                                  "note": "the library's only scratch is the caller's workspace: O(N) + O(SMs), "
+                                          "no per-edge float tensor"},
             "clocks": clk.summary()}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = oracle_rate(args.config, float(os.environ.get("E2F_CPU_BUDGET_S", "15")))

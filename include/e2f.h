@@ -193,6 +193,15 @@ e2f_status e2f_onfly_attention(const e2f_attn_cfg* cfg, const float* pos,
  * a multiple of 4), 0 when it runs the fp32 CUDA-core kernel. */
 int e2f_attention_uses_tensor_cores(const e2f_attn_cfg* cfg);
 
+/* Profiling aid (no counterpart in the pages). start_event and stop_event
+ * are cudaEvent_t handles created by the caller. While both are non-NULL,
+ * every e2f_onfly_attention call that runs the tensor-core kernel records
+ * start_event on its stream just before that kernel and stop_event just
+ * after, so cudaEventElapsedTime gives the main kernel alone (without the
+ * O(N) pre-passes). NULL, NULL turns it off. One process-wide setting: not
+ * for concurrent calls from several threads. */
+void e2f_attention_set_kernel_events(void* start_event, void* stop_event);
+
 /* Diagnostics of the tensor-core kernel. When the environment variable
  * E2F_TC_TIMERS=1 is set at call time, each persistent CTA records clock64
  * cycle counts of its warp roles into the workspace: per CTA 32 int64 values,
