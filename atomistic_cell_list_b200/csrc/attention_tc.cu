@@ -10,27 +10,29 @@
 //   o+[f, e] = sum_k A(m)[f, k] h+[e, k] - B(m)[f, k] h-[e, k]
 //   o-[f, e] = sum_k B(m)[f, k] h+[e, k] + A(m)[f, k] h-[e, k]
 //
-// A and B are read by TMA straight from the caller's packed weights (the
-// A operand, K-major); h = the tile's rotated, gated neighbour features (the
+// A and B are read by TMA from fp16 copies of the packed weights (the A
+// operand, K-major); h = the tile's rotated, gated neighbour features (the
 // B operand, K-major). One A/B weight tile serves two MMAs (the -B product
-// uses the instruction's negate bit), so each weight byte is read once per
-// 128 edges. A group = up to two accumulators (o+ and o- of the same
-// features, or two feature blocks of m = 0) = 256 TMEM columns; two groups
-// in flight let the epilogue drain one while the MMA fills the other.
+// uses the instruction's negate bit). A group = up to two accumulators (o+
+// and o- of the same features, or two feature blocks of m = 0) = 256 TMEM
+// columns; two groups in flight let the epilogue drain one while the MMA
+// fills the other.
 //
-// Warp roles (320 threads):
-//   0-3  epilogue: tcgen05.ld of the accumulators; per thread one output
-//        feature (l3, c) for all 128 edges: p * D^l3(R)^T restricted to the
-//        group's |m| rows (the rotate-back, one block at a time), summed
-//        over each node's edges in registers, added to out[node] (a CTA owns
-//        its nodes, so the read-modify-write is race-free and deterministic)
-//   4-7  producer: per edge the frame, Wigner blocks, radial gate, softmax
-//        weight p = exp(a - lse) (statistics from a scalar pre-pass: the
-//        logits do not depend on the value path, Eq. 6); then the rotated,
-//        gated features for all |m| written once per tile to a per-CTA
-//        global scratch (bf16, K-major rows) for TMA to stream
-//   8    TMA loads of weight and feature tiles into a 3-stage ring
-//   9    tcgen05.mma issue (one thread), commits to the ring and TMEM barriers
+// Warp roles (512 threads, 128 registers each):
+//   0-3, 8-11  epilogue: tcgen05.ld 16x256b fragments of the accumulators;
+//              rotate-back p * D^l3(R)^T restricted to the group's |m| rows
+//              on mma.sync, summed over each node's edges, added to
+//              out[node] (one owner thread per element: fixed order)
+//   4-7        producer: per edge the node, frame, Wigner blocks (fp16 pairs,
+//              shared and global copies); per (edge, head) the softmax weight
+//              p = exp(a - lse) (statistics from an O(N) pre-pass); per
+//              (edge, 8 channels) the gathered, gated, rotated features,
+//              written once per tile to a per-CTA global scratch row for TMA
+//   12         TMA loads of weight and feature tiles into a 3-stage ring
+//   13         tcgen05.mma issue (one thread), commits to the ring and TMEM
+//              barriers
+//   14-15      value gates rho(d) W_rad of a tile (mma.sync), up to two tiles
+//              ahead of the producer, into a double-buffered global scratch
 // Every mbarrier wait is bounded by the global timer; on expiry the kernel
 // records E2F_ERR_TIMEOUT, drains what it issued and returns.
 #include <cuda.h>

@@ -54,7 +54,7 @@ def measured_peaks():
 KERNEL_TRAFFIC = {
     "sources": ["atomistic_cell_list_b200/csrc/attention_tc.cu", "atomistic_cell_list_b200/csrc/attention_tc.cuh",
                 "atomistic_cell_list_b200/csrc/common.cuh"],
-    "sha256": "df05443b1baac352ef2328a7359e68eb460a2a17bb364565968c705552fb7ee6",
+    "sha256": "168b6447e503b6b20cf0aa4bc3d26628fcb802eaacd3773d92d9e08af21ab7f0",
     "dram_read_bytes": 46.28e9,
     "dram_write_bytes": 24.20e9,
 }
