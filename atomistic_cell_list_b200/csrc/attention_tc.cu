@@ -133,6 +133,39 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
         : "memory");
 }
 
+// same, with an L2 cache policy (createpolicy) for the source lines
+__device__ __forceinline__ void tma_load_2d_hint(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar,
+                                                 uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint "
+        "[%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar)), "l"(policy)
+        : "memory");
+}
+__device__ __forceinline__ uint64_t policy_evict_last() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+__device__ __forceinline__ uint64_t policy_evict_first() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+// 16-byte global store / streaming load with an L2 cache policy
+__device__ __forceinline__ void st_hint(void* ptr, uint4 v, uint64_t policy) {
+    asm volatile("st.global.L2::cache_hint.v4.b32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(ptr), "r"(v.x), "r"(v.y),
+                 "r"(v.z), "r"(v.w), "l"(policy)
+                 : "memory");
+}
+__device__ __forceinline__ uint4 ld_hint(const void* ptr, uint64_t policy) {
+    uint4 v;
+    asm volatile("ld.global.nc.L2::cache_hint.v4.b32 {%0, %1, %2, %3}, [%4], %5;"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(ptr), "l"(policy));
+    return v;
+}
+
 __device__ __forceinline__ void tmem_alloc(uint32_t* dst, uint32_t ncols) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst)), "r"(ncols)
                  : "memory");
@@ -760,6 +793,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
         }                                                             \
     } while (0)
         const size_t KT = (size_t)K * C;
+        // L2 policies: the feature scratch is re-read by TMA (keep), neighbour rows stream (evict first)
+        const uint64_t pol_last = policy_evict_last(), pol_first = policy_evict_first();
         long long w_free = 0, c_p1 = 0, c_p2 = 0;
         const long long c_start = clock64();
         for (int t = 0; t < ntiles; ++t) {
@@ -959,7 +994,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
                 uint4 raw[K];
                 const __half* xj = P.x + (size_t)j * K * C + c0;
 #pragma unroll
-                for (int n = 0; n < K; ++n) raw[n] = __ldg(reinterpret_cast<const uint4*>(xj + (size_t)n * C));
+                for (int n = 0; n < K; ++n) raw[n] = ld_hint(xj + (size_t)n * C, pol_first);
                 uint4 gr[L + 1];
 #pragma unroll
                 for (int l1 = 0; l1 <= L; ++l1) gr[l1] = *reinterpret_cast<const uint4*>(gs + (size_t)e * Gv + l1 * C + c0);
@@ -996,10 +1031,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
                                     }
                                 }
                             }
-                            *reinterpret_cast<uint4*>(xrow + kpos(l1, mu, L, C) + c0) = *reinterpret_cast<uint4*>(op);
+                            st_hint(xrow + kpos(l1, mu, L, C) + c0, *reinterpret_cast<uint4*>(op), pol_last);
                             if (mu > 0)
-                                *reinterpret_cast<uint4*>(xrow + kpos(l1, -mu, L, C) + c0) =
-                                    *reinterpret_cast<uint4*>(om);
+                                st_hint(xrow + kpos(l1, -mu, L, C) + c0, *reinterpret_cast<uint4*>(om), pol_last);
                         }
                     }
                 }
@@ -1019,6 +1053,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
     } else if (warp == 12) {
         // ---------------- TMA ----------------
         if (lane == 0) {
+            const uint64_t pol_xs = policy_evict_last();
             int stage = 0;
             uint32_t ph = 0;
             bool ok = true;
@@ -1040,12 +1075,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
                         if (g.mu > 0) {
                             tma_load_2d(st, &T.w[g.wa], kk, g.row0, full + stage);
                             tma_load_2d(st + kSlot, &T.w[g.wb], kk, g.row0, full + stage);
-                            tma_load_2d(st + 2 * kSlot, &T.xs, g.xoff0 + kk, rowT, full + stage);
-                            tma_load_2d(st + 3 * kSlot, &T.xs, g.xoff1 + kk, rowT, full + stage);
+                            tma_load_2d_hint(st + 2 * kSlot, &T.xs, g.xoff0 + kk, rowT, full + stage, pol_xs);
+                            tma_load_2d_hint(st + 3 * kSlot, &T.xs, g.xoff1 + kk, rowT, full + stage, pol_xs);
                         } else {
                             tma_load_2d(st, &T.w[g.wa], kk, g.row0, full + stage);
                             if (g.row0b >= 0) tma_load_2d(st + kSlot, &T.w[g.wa], kk, g.row0b, full + stage);
-                            tma_load_2d(st + 2 * kSlot, &T.xs, g.xoff0 + kk, rowT, full + stage);
+                            tma_load_2d_hint(st + 2 * kSlot, &T.xs, g.xoff0 + kk, rowT, full + stage, pol_xs);
                         }
                         pending[stage] = (int)ph;
                         if (++stage == kNS) { stage = 0; ph ^= 1; }
