@@ -54,9 +54,9 @@ def measured_peaks():
 KERNEL_TRAFFIC = {
     "sources": ["atomistic_cell_list_b200/csrc/attention_tc.cu", "atomistic_cell_list_b200/csrc/attention_tc.cuh",
                 "atomistic_cell_list_b200/csrc/common.cuh"],
-    "sha256": "168b6447e503b6b20cf0aa4bc3d26628fcb802eaacd3773d92d9e08af21ab7f0",
-    "dram_read_bytes": 46.28e9,
-    "dram_write_bytes": 24.20e9,
+    "sha256": "c85f48ca0483b3f824f810b3856a60cf85903877b6e886b32e92bdee2f29e4dc",
+    "dram_read_bytes": 44.33e9,
+    "dram_write_bytes": 24.02e9,
 }
 
 
