@@ -369,19 +369,96 @@ def run_ours(args):
     return 0
 
 
+def run_naive(args):
+    """Edge-materialising PyTorch baseline (naive_baseline.py) beside this
+    library on the same workload: time, SO(2) TFLOP/s and peak activation
+    memory of both (context for the pages' node-centric vs edge-centric
+    comparison; not the product path)."""
+    import torch
+
+    import atomistic_cell_list_b200 as e2f
+    import workloads as W
+    from naive_baseline import naive_attention
+
+    if int(os.environ.get("RANK", "0")) != 0:
+        return 0
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    cfg_id = args.config
+    w = W.load_workload(cfg_id)
+    xs, _ = W.make_features(cfg_id, w.n_atoms, w.L, w.C, w.dtype)
+    wt = W.make_weights(cfg_id, w.L, w.C, w.H, w.n_rbf, w.dtype)
+
+    def dt(a):
+        if a.dtype == np.uint16:
+            return torch.from_numpy(a.view(np.int16).copy()).view(torch.bfloat16).to(dev)
+        return torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+
+    pos, x = dt(w.pos), dt(xs).reshape(w.n_atoms, w.K, w.C)
+    Wq, Wk, Wrad, Wso2 = dt(wt.Wq), dt(wt.Wk), dt(wt.Wrad), dt(wt.Wso2)
+    box = None if w.box is None else [float(b) for b in w.box]
+    gptr = None if w.graph_ptr is None else torch.from_numpy(w.graph_ptr).to(dev)
+    cfg = e2f.make_cfg(w.L, w.C, w.H, w.n_rbf, w.cutoff, w.dtype)
+    rp, col = e2f.e2f_build_neighbors(pos, box, w.cutoff, gptr)
+    E = int(col.numel())
+    out_bytes = w.n_atoms * w.K * w.C * 4
+
+    def measure(fn):
+        res = None
+        for _ in range(max(1, args.warmup)):
+            res = fn()
+        torch.cuda.synchronize(dev)
+        del res
+        torch.cuda.empty_cache()
+        torch.cuda.reset_peak_memory_stats(dev)
+        base = torch.cuda.memory_allocated(dev)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ts = []
+        for _ in range(args.steps):
+            a.record()
+            res = fn()
+            b.record()
+            torch.cuda.synchronize(dev)
+            ts.append(a.elapsed_time(b))
+            del res
+        peak = torch.cuda.max_memory_allocated(dev) - base
+        return statistics.median(ts), peak
+
+    F = so2_flops_per_edge(w.L, w.C)
+    ours_ms, ours_peak = measure(lambda: e2f.e2f_onfly_attention(cfg, pos, box, rp, col, x, Wq, Wk, Wrad, Wso2))
+    line = {"impl": "naive", "metric": "edge-materialising PyTorch baseline vs this library, same workload",
+            "config": {**workload_desc(w), "n_pairs": E}, "unit": "ms", "data": "synthetic",
+            "ours": {"ms": ours_ms, "tflops": E * F / (ours_ms * 1e-3) / 1e12,
+                     "peak_activation_bytes": int(ours_peak - out_bytes)}}
+    try:
+        naive_ms, naive_peak = measure(lambda: naive_attention(cfg, pos, box, rp, col, x, Wq, Wk, Wrad, Wso2))
+        line["naive"] = {"ms": naive_ms, "tflops": E * F / (naive_ms * 1e-3) / 1e12,
+                         "peak_activation_bytes": int(naive_peak - out_bytes)}
+        line["speedup"] = naive_ms / ours_ms
+        line["memory_ratio"] = (naive_peak - out_bytes) / max(1, ours_peak - out_bytes)
+    except torch.cuda.OutOfMemoryError as exc:  # E x K x C tensors do not fit
+        line["naive"] = {"oom": str(exc).splitlines()[0][:160]}
+    line["note"] = ("peak_activation_bytes = max_memory_allocated during the call minus inputs, weights, CSR and "
+                    "the fp32 output; this library's is its workspace")
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--config", type=int, default=4)
-    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--impl", choices=["ours", "reference", "naive"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":
         return run_reference(args)
+    if args.impl == "naive":
+        return run_naive(args)
     return run_ours(args)
 
 
