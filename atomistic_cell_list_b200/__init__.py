@@ -34,7 +34,7 @@ class E2FError(RuntimeError):
 
 class e2f_attn_cfg(ctypes.Structure):
     _fields_ = [("L", ctypes.c_int), ("C", ctypes.c_int), ("H", ctypes.c_int), ("n_rbf", ctypes.c_int),
-                ("cutoff", ctypes.c_float), ("feat_dtype", ctypes.c_int)]
+                ("cutoff", ctypes.c_float), ("feat_dtype", ctypes.c_int), ("m_max", ctypes.c_int)]
 
 
 _lib = None
@@ -183,8 +183,9 @@ def e2f_build_neighbors_noalloc(pos: torch.Tensor, box, cutoff: float, graph_ptr
     raise E2FError(3, "e2f_build_neighbors_noalloc")
 
 
-def make_cfg(L: int, C: int, H: int, n_rbf: int, cutoff: float, dtype: str) -> e2f_attn_cfg:
-    return e2f_attn_cfg(L, C, H, n_rbf, float(cutoff), E2F_BF16 if dtype == "bf16" else E2F_F32)
+def make_cfg(L: int, C: int, H: int, n_rbf: int, cutoff: float, dtype: str, m_max: int = -1) -> e2f_attn_cfg:
+    """m_max: SO(2) truncation order (-1 = full layer; W_so2 then holds blocks m <= m_max only)."""
+    return e2f_attn_cfg(L, C, H, n_rbf, float(cutoff), E2F_BF16 if dtype == "bf16" else E2F_F32, int(m_max))
 
 
 def e2f_attention_workspace_size(n_atoms: int, n_pairs: int, cfg: e2f_attn_cfg) -> int:

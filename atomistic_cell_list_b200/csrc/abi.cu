@@ -33,7 +33,7 @@ AttnWs attn_layout(int64_t n_atoms, const e2f_attn_cfg& c) {
     w.o_q = take(4 * (size_t)n_atoms * c.C);
     w.o_k = take(4 * (size_t)n_atoms * c.C);
     w.tc = tc_supported(c.L, c.C, c.H, c.n_rbf, c.feat_dtype == E2F_BF16);
-    w.o_wt = w.tc ? 0 : take(4 * so2_total(c.L, c.C));
+    w.o_wt = w.tc ? 0 : take(4 * so2_total(c.L, c.C, effective_mmax(c.L, c.m_max)));
     w.o_tc = w.tc ? take(tc_workspace_bytes(n_atoms, c.L, c.C, c.H)) : 0;
     w.bytes = o;
     return w;
@@ -44,6 +44,7 @@ e2f_status check_cfg(const e2f_attn_cfg* c) {
     if (c->L < 0 || c->C <= 0 || c->H <= 0 || !(c->cutoff > 0.f) || !std::isfinite(c->cutoff))
         return E2F_ERR_INVALID_ARG;
     if (c->feat_dtype != E2F_F32 && c->feat_dtype != E2F_BF16) return E2F_ERR_UNSUPPORTED;
+    if (c->m_max < -1) return E2F_ERR_INVALID_ARG;
     if (c->L > kMaxL || c->C % 16 != 0 || c->C > 256 || c->C % c->H != 0 || c->n_rbf < 2 || c->n_rbf > 32)
         return E2F_ERR_UNSUPPORTED;
     return E2F_OK;
@@ -98,6 +99,7 @@ extern "C" e2f_status e2f_onfly_attention(const e2f_attn_cfg* cfg, const float* 
 
     AttnArgs a{};
     a.L = cfg->L; a.C = cfg->C; a.H = cfg->H; a.n_rbf = cfg->n_rbf; a.cutoff = cfg->cutoff;
+    a.M = effective_mmax(cfg->L, cfg->m_max);
     a.bf16 = cfg->feat_dtype == E2F_BF16;
     a.n_atoms = (int)n_atoms; a.n_pairs = n_pairs;
     a.box.periodic = box_host != nullptr;

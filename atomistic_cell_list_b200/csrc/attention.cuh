@@ -24,12 +24,18 @@ __host__ __device__ inline size_t so2_offset(int L, int C, int m, int which) {
     return off + (which ? n * n : 0);
 }
 
-__host__ __device__ inline size_t so2_total(int L, int C) {
-    return so2_offset(L, C, L + 1, 0);
+// values in the packed weights of a layer whose maps stop at |m| = M
+__host__ __device__ inline size_t so2_total(int L, int C, int M) {
+    return so2_offset(L, C, M + 1, 0);
 }
+__host__ __device__ inline size_t so2_total(int L, int C) { return so2_total(L, C, L); }
+
+// effective truncation order of a configuration
+inline int effective_mmax(int L, int m_max) { return (m_max < 0 || m_max > L) ? L : m_max; }
 
 struct AttnArgs {
     int L, C, H, n_rbf;
+    int M;  // SO(2) maps for |m| <= M
     float cutoff;
     bool bf16;
     int n_atoms;

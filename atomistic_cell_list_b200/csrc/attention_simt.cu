@@ -48,8 +48,8 @@ __global__ void k_qk_project(const T* __restrict__ x, int n_atoms, int K, int C,
 // Packed SO(2) blocks (row-major [(l3,c_out),(l1,c_in)]) -> fp32, each block
 // transposed so that consecutive output rows are consecutive in memory.
 template <typename T>
-__global__ void k_repack_so2_f32(const T* __restrict__ w, int L, int C, float* out) {
-    const size_t total = so2_total(L, C);
+__global__ void k_repack_so2_f32(const T* __restrict__ w, int L, int C, int M, float* out) {
+    const size_t total = so2_total(L, C, M);
     for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += (size_t)gridDim.x * blockDim.x) {
         size_t off = 0;
         int n = (L + 1) * C;
@@ -68,6 +68,7 @@ __global__ void k_repack_so2_f32(const T* __restrict__ w, int L, int C, float* o
 
 struct SimtParams {
     int n_atoms, C, H, n_rbf;
+    int M;  // SO(2) maps for |m| <= M
     float cutoff;
     Box box;
     const float* pos;
@@ -177,7 +178,7 @@ __global__ void __launch_bounds__(256) k_attn_simt(SimtParams P) {
 
         // 4 per |m| block
 #pragma unroll 1
-        for (int m = 0; m <= L; ++m) {
+        for (int m = 0; m <= P.M; ++m) {  // |m| > M: no message (truncated layer)
             const int nm = (L + 1 - m) * C;         // rows (and columns) of A(m)
             // 4a rotated, gated block input: hs[(s, l1-m, c)][e]
             for (int t = tid; t < te * nm; t += nt) {
@@ -293,18 +294,19 @@ cudaError_t run_attention_simt(const AttnArgs& a, cudaStream_t s) {
         k_qk_project<__nv_bfloat16><<<a.n_atoms, 128, C * 4, s>>>(static_cast<const __nv_bfloat16*>(a.x), a.n_atoms,
                                                                   K, C, a.Wq, a.Wk, a.q, a.k);
         count_launch();
-        k_repack_so2_f32<__nv_bfloat16><<<1184, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(a.Wso2), a.L, C, a.Wt);
+        k_repack_so2_f32<__nv_bfloat16><<<1184, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(a.Wso2), a.L, C, a.M,
+                                                             a.Wt);
     } else {
         count_launch();
         k_qk_project<float><<<a.n_atoms, 128, C * 4, s>>>(static_cast<const float*>(a.x), a.n_atoms, K, C, a.Wq,
                                                           a.Wk, a.q, a.k);
         count_launch();
-        k_repack_so2_f32<float><<<1184, 256, 0, s>>>(static_cast<const float*>(a.Wso2), a.L, C, a.Wt);
+        k_repack_so2_f32<float><<<1184, 256, 0, s>>>(static_cast<const float*>(a.Wso2), a.L, C, a.M, a.Wt);
     }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     SimtParams P;
-    P.n_atoms = a.n_atoms; P.C = C; P.H = a.H; P.n_rbf = a.n_rbf; P.cutoff = a.cutoff; P.box = a.box;
+    P.n_atoms = a.n_atoms; P.C = C; P.H = a.H; P.n_rbf = a.n_rbf; P.M = a.M; P.cutoff = a.cutoff; P.box = a.box;
     P.pos = a.pos; P.row_ptr = a.row_ptr; P.col = a.col; P.x = a.x; P.q = a.q; P.k = a.k;
     P.Wrad = a.Wrad; P.Wt = a.Wt; P.out = a.out;
     int te = 16;

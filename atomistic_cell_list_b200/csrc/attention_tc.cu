@@ -1439,7 +1439,7 @@ cudaError_t run_attention_tc(const AttnArgs& a, void* tc_ws, cudaStream_t s) {
     count_launch();
     tc::k_x_to_f16<<<1184, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(a.x), nx, scale, x16);
     count_launch();
-    tc::k_w_to_f16<<<592, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(a.Wso2), so2_total(L, C), w16);
+    tc::k_w_to_f16<<<592, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(a.Wso2), so2_total(L, C, a.M), w16);
     count_launch();
     tc::k_wrad_t<<<(Gv * kTcMaxRbf + 255) / 256, 256, 0, s>>>(a.Wrad, a.n_rbf, G, Gv, whT);
 
@@ -1462,7 +1462,7 @@ cudaError_t run_attention_tc(const AttnArgs& a, void* tc_ws, cudaStream_t s) {
     if (e != cudaSuccess) return e;
 
     tc::TcParams P{};
-    P.C = C; P.H = H; P.n_rbf = a.n_rbf; P.G = (L + 1) * C + H; P.cutoff = a.cutoff; P.box = a.box;
+    P.C = C; P.H = H; P.n_rbf = a.n_rbf; P.G = (L + 1) * C + H; P.M = a.M; P.cutoff = a.cutoff; P.box = a.box;
     P.pos = a.pos; P.row_ptr = a.row_ptr; P.col = a.col; P.x = x16; P.whT = whT; P.gscr = gscr; P.scale = scale;
     P.q = a.q; P.k = a.k; P.lse = lse; P.Wrad = a.Wrad; P.part = part; P.xs = xs; P.dscr = dscr; P.out = a.out;
     P.status = a.status;
@@ -1484,7 +1484,7 @@ cudaError_t run_attention_tc(const AttnArgs& a, void* tc_ws, cudaStream_t s) {
         P.groups[ng++] = g;
     }
     int koff = n0;
-    for (int mu = 1; mu <= L; ++mu) {
+    for (int mu = 1; mu <= a.M; ++mu) {  // |m| > M: no message (truncated layer)
         const int nm = (L + 1 - mu) * C;
         for (int r0 = 0; r0 < nm; r0 += 128) {
             tc::TcGroup g{};
@@ -1499,7 +1499,7 @@ cudaError_t run_attention_tc(const AttnArgs& a, void* tc_ws, cudaStream_t s) {
     tc::TcMaps T;
     const __half* W = w16;
     if (!make_map(&T.w[0], W + so2_offset(L, C, 0, 0), n0, n0)) return cudaErrorInvalidValue;
-    for (int mu = 1; mu <= L; ++mu) {
+    for (int mu = 1; mu <= a.M; ++mu) {
         const int nm = (L + 1 - mu) * C;
         if (!make_map(&T.w[2 * mu - 1], W + so2_offset(L, C, mu, 0), nm, nm)) return cudaErrorInvalidValue;
         if (!make_map(&T.w[2 * mu], W + so2_offset(L, C, mu, 1), nm, nm)) return cudaErrorInvalidValue;

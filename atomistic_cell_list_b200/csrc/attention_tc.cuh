@@ -44,6 +44,7 @@ struct TcGroup {
 
 struct TcParams {
     int C, H, n_rbf, G;
+    int M;  // SO(2) maps for |m| <= M
     float cutoff;
     Box box;
     const float* pos;

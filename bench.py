@@ -33,9 +33,10 @@ import numpy as np  # noqa: E402
 METRIC = "neighbor pairs/s + achieved TFLOPS, fused equivariant attn fwd, 1×B200"
 
 
-def so2_flops_per_edge(L: int, C: int) -> int:
-    """Algorithmic SO(2) FLOPs per edge: 2((L+1)C)^2 + sum_m 8((L+1-m)C)^2."""
-    return 2 * ((L + 1) * C) ** 2 + sum(8 * ((L + 1 - m) * C) ** 2 for m in range(1, L + 1))
+def so2_flops_per_edge(L: int, C: int, M: int | None = None) -> int:
+    """Algorithmic SO(2) FLOPs per edge: 2((L+1)C)^2 + sum_{m=1..M} 8((L+1-m)C)^2 (M = L: full layer)."""
+    M = L if M is None or M < 0 or M > L else M
+    return 2 * ((L + 1) * C) ** 2 + sum(8 * ((L + 1 - m) * C) ** 2 for m in range(1, M + 1))
 
 
 def measured_peaks():
@@ -228,12 +229,14 @@ def run_ours(args):
             return torch.from_numpy(a.view(np.int16).copy()).view(torch.bfloat16)
         return torch.from_numpy(np.ascontiguousarray(a))
 
+    M = w.L if args.m_max < 0 or args.m_max > w.L else args.m_max
+    n_so2 = sum(W.so2_block_sizes(w.L, w.C)[:2 * M + 1])  # truncated layer: blocks m <= M
     h_inputs = {"pos": host(w.pos), "x": host(xs).reshape(w.n_atoms, w.K, w.C), "Wq": host(wt.Wq),
-                "Wk": host(wt.Wk), "Wrad": host(wt.Wrad), "Wso2": host(wt.Wso2)}
+                "Wk": host(wt.Wk), "Wrad": host(wt.Wrad), "Wso2": host(np.ascontiguousarray(wt.Wso2[:n_so2]))}
     d = {k: v.to(dev) for k, v in h_inputs.items()}
     box = None if w.box is None else [float(b) for b in w.box]
     gptr = None if w.graph_ptr is None else torch.from_numpy(w.graph_ptr).to(dev)
-    cfg = e2f.make_cfg(w.L, w.C, w.H, w.n_rbf, w.cutoff, w.dtype)
+    cfg = e2f.make_cfg(w.L, w.C, w.H, w.n_rbf, w.cutoff, w.dtype, m_max=M)
     stream = torch.cuda.current_stream(dev)
 
     # buffers reused by every step
@@ -319,7 +322,7 @@ def run_ours(args):
     ms_e2e = float(t_e2e[0]) / args.steps
 
     peaks, peak_src = measured_peaks()
-    F = so2_flops_per_edge(w.L, w.C)
+    F = so2_flops_per_edge(w.L, w.C, M)
     tflops = E * F / (ms_att * 1e-3) / 1e12          # whole attention call (with its O(N) pre-passes)
     tflops_ker = E * F / (ms_ker * 1e-3) / 1e12      # the main kernel alone
     path = "tensor" if use_tc else "simt"
@@ -346,7 +349,7 @@ def run_ours(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32" if path == "simt" else "bf16",
             "data": "synthetic",
-            "config": {**workload_desc(w), "n_pairs": E, "parallelism": f"replicas x{world}",
+            "config": {**workload_desc(w), "n_pairs": E, "m_max": M, "parallelism": f"replicas x{world}",
                        "l2": "flushed (256 MB write) between timed steps"},
             "tflops": tflops, "tflops_kernel": tflops_ker, "ms_attention": ms_att, "ms_attention_kernel": ms_ker,
             "ms_neighbors": ms_nbr,
@@ -452,6 +455,7 @@ def main():
     ap.add_argument("--config", type=int, default=4)
     ap.add_argument("--impl", choices=["ours", "reference", "naive"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--m-max", type=int, default=-1, help="SO(2) truncation order (-1: full layer)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

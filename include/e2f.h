@@ -55,6 +55,11 @@ typedef struct {
     int n_rbf;
     float cutoff;
     e2f_dtype feat_dtype;
+    /* SO(2) truncation: the maps act on |m| <= M only, M = m_max (0 <= m_max
+     * < L), or M = L when m_max < 0 or m_max >= L (the full layer). Rows with
+     * |m| > M get no message (as if A(m), B(m) were zero); W_so2 holds the
+     * blocks m <= M only. */
+    int m_max;
 } e2f_attn_cfg;
 
 /* Human-readable name of a status code (static string, never NULL). */
@@ -161,9 +166,10 @@ e2f_status e2f_build_neighbors_noalloc(const float* pos, int64_t n_atoms,
  *   W_rad      device, float [n_rbf, (L+1)C + H] row-major; column l*C + c
  *              is g_v[l, c], column (L+1)C + h is g_a^h. 16-byte aligned.
  *   W_so2      device, feat_dtype, packed: A(0), then A(m), B(m) for
- *              m = 1..L; block m is a row-major square matrix of side
- *              (L+1-m)C indexed [(l3, c_out), (l1, c_in)], l3, l1 = m..L.
- *              85*C*C values at L = 4. 16-byte aligned.
+ *              m = 1..M (M = L unless cfg->m_max truncates); block m is a
+ *              row-major square matrix of side (L+1-m)C indexed
+ *              [(l3, c_out), (l1, c_in)], l3, l1 = m..L. 85*C*C values at
+ *              L = 4 (full). 16-byte aligned.
  *   out        device, float [N, (L+1)^2, C], written.
  *   workspace  device, >= e2f_attention_workspace_size(...) bytes, 256-byte
  *              aligned, contents need no initialisation. Holds the

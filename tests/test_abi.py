@@ -29,6 +29,11 @@ def test_workspace_queries_are_host_only():
     assert e2f.e2f_neighbors_workspace_size(10000, None, 5.0, 256) > 0
     bad = e2f.make_cfg(5, 128, 8, 16, 6.0, "bf16")
     assert e2f.e2f_attention_workspace_size(10, 10, bad) == 0
+    assert e2f.e2f_attention_workspace_size(10, 10, e2f.make_cfg(2, 16, 1, 16, 5.0, "f32", m_max=-2)) == 0
+    # the fp32 path keeps a repacked copy of the SO(2) weights: a truncated layer needs less
+    full = e2f.e2f_attention_workspace_size(64, 1000, e2f.make_cfg(2, 16, 1, 16, 5.0, "f32"))
+    trunc = e2f.e2f_attention_workspace_size(64, 1000, e2f.make_cfg(2, 16, 1, 16, 5.0, "f32", m_max=0))
+    assert 0 < trunc < full
 
 
 def _attn(cfg, **kw):
