@@ -232,16 +232,6 @@ __host__ __device__ constexpr uint32_t idesc_f16(bool neg_a) {
 // ----------------------------------------------------------------------------
 // pre-passes
 // ----------------------------------------------------------------------------
-// Logit of edge (i <- j) for head h (Eq. 6 reading): g_a^h <q_i^h, k_j^h>/sqrt(d).
-__device__ __forceinline__ float edge_logit(const float* rho, int n_rbf, const float* Wrad, int G, int gcol,
-                                            const float* qi, const float* kj, int dh, float inv_sqrt_dh) {
-    float ga = 0.f;
-    for (int kb = 0; kb < n_rbf; ++kb) ga = fmaf(rho[kb], Wrad[(size_t)kb * G + gcol], ga);
-    float dot = 0.f;
-    for (int c = 0; c < dh; ++c) dot = fmaf(qi[c], kj[c], dot);
-    return ga * dot * inv_sqrt_dh;
-}
-
 // Softmax statistics per node and head, lse = m + log(sum exp(a - m)), by an
 // online max/sum over the node's edges. One warp per node; lane = (edge slot
 // es, head h) with 32 / H edge slots, so a head's q and logit-gate column
