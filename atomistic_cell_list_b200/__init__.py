@@ -51,6 +51,9 @@ _SIGS = {
     "e2f_onfly_attention": (ctypes.c_int, [ctypes.POINTER(e2f_attn_cfg), _vp, _i64, _vp, _vp, _vp, _i64, _vp, _vp,
                                            _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "e2f_attention_status": (ctypes.c_int, [_vp, _sz, _vp]),
+    "e2f_attention_cells_workspace_size": (_sz, [_i64, _vp, ctypes.POINTER(e2f_attn_cfg)]),
+    "e2f_onfly_attention_cells": (ctypes.c_int, [ctypes.POINTER(e2f_attn_cfg), _vp, _i64, _vp, _vp, _vp, _vp, _vp,
+                                                 _vp, _vp, _vp, _sz, _vp]),
     "e2f_edge_wigner_blocks": (ctypes.c_int, [_vp, _i64, ctypes.c_int, _vp, _vp, _vp]),
     "e2f_launch_count": (_i64, []),
     "e2f_attention_uses_tensor_cores": (ctypes.c_int, [ctypes.POINTER(e2f_attn_cfg)]),
@@ -212,6 +215,36 @@ def e2f_onfly_attention(cfg: e2f_attn_cfg, pos, box, row_ptr, col, x, W_q, W_k, 
     _check(code, "e2f_onfly_attention")
     if check:
         _check(lib().e2f_attention_status(_ptr(workspace), workspace.numel(), s), "e2f_onfly_attention (device)")
+    return out
+
+
+def e2f_attention_cells_workspace_size(n_atoms: int, box, cfg: e2f_attn_cfg) -> int:
+    b, keep = _box_arg(box)
+    return int(lib().e2f_attention_cells_workspace_size(int(n_atoms), b, ctypes.byref(cfg)))
+
+
+def e2f_onfly_attention_cells(cfg: e2f_attn_cfg, pos, box, x, W_q, W_k, W_rad, W_so2,
+                              out: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+                              stream=None, check: bool = True) -> torch.Tensor:
+    """The attention with the cell-list traversal fused in: no neighbour list (see include/e2f.h)."""
+    _need_cuda(pos, x, W_q, W_k, W_rad, W_so2, out, workspace)
+    n = pos.shape[0]
+    if out is None:
+        out = torch.empty((n, (cfg.L + 1) ** 2, cfg.C), dtype=torch.float32, device=pos.device)
+    ws_bytes = e2f_attention_cells_workspace_size(n, box, cfg)
+    if ws_bytes == 0:
+        raise E2FError(2, "e2f_onfly_attention_cells")
+    if workspace is None or workspace.numel() < ws_bytes:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=pos.device)
+    b, keep = _box_arg(box)
+    s = _stream(stream)
+    code = lib().e2f_onfly_attention_cells(ctypes.byref(cfg), _ptr(pos), n, b, _ptr(x), _ptr(W_q), _ptr(W_k),
+                                           _ptr(W_rad), _ptr(W_so2), _ptr(out), _ptr(workspace),
+                                           workspace.numel(), s)
+    _check(code, "e2f_onfly_attention_cells")
+    if check:
+        _check(lib().e2f_attention_status(_ptr(workspace), workspace.numel(), s),
+               "e2f_onfly_attention_cells (device)")
     return out
 
 

@@ -58,7 +58,9 @@ struct AttnArgs {
 };
 
 cudaError_t run_attention_simt(const AttnArgs& a, cudaStream_t s);
-cudaError_t run_attention_tc(const AttnArgs& a, void* tc_ws, cudaStream_t s);
+struct CellLists;
+// cl != nullptr: fused traversal (a.row_ptr = per-slot offsets in cell order, a.col unused)
+cudaError_t run_attention_tc(const AttnArgs& a, void* tc_ws, cudaStream_t s, const CellLists* cl = nullptr);
 void set_tc_kernel_events(void* start, void* stop);
 cudaError_t run_edge_wigner(const float* r, int64_t n, int L, float* out, float* frames, cudaStream_t s);
 

@@ -46,6 +46,7 @@
 
 #include "attention.cuh"
 #include "attention_tc.cuh"
+#include "cell_grid.cuh"
 #include "common.cuh"
 
 namespace e2f {
@@ -287,6 +288,72 @@ __global__ void __launch_bounds__(256) k_softmax_stats(StatsParams P) {
     if (es == 0) P.lse[(size_t)i * H + h] = (e1 > e0) ? m + logf(s) : 0.f;
 }
 
+// The same statistics with the neighbours enumerated from the cell lists
+// (fused traversal): one warp per node slot in cell order, one lane per
+// neighbour found, logits evaluated as in the main kernel.
+__global__ void __launch_bounds__(256) k_softmax_stats_cells(StatsParams P, CellView cv) {
+    const int s = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (s >= P.n_atoms) return;
+    const int H = P.H, C = P.C, dh = C / H, G = P.G, Gv = G - H;
+    const float inv = rsqrtf((float)dh);
+    const int i = cv.sidx[s];
+    float m[kMaxHeads], sm[kMaxHeads];
+#pragma unroll
+    for (int h = 0; h < kMaxHeads; ++h) { m[h] = -INFINITY; sm[h] = 0.f; }
+    const int cnt = warp_neighbors(cv, cv.spos[s], i, [&](int, int j) {
+        const float3 r = edge_vec(P.pos, i, j, P.box);
+        const float d = sqrtf(r.x * r.x + r.y * r.y + r.z * r.z);
+        float rr[kTcMaxRbf];
+        rbf_all<kTcMaxRbf>(d, P.cutoff, P.n_rbf, rr);
+        for (int h = 0; h < H; ++h) {
+            float ga = 0.f;
+#pragma unroll
+            for (int kb = 0; kb < kTcMaxRbf; ++kb)
+                ga = fmaf(rr[kb], kb < P.n_rbf ? __ldg(P.Wrad + (size_t)kb * G + Gv + h) : 0.f, ga);
+            const float4* q4 = reinterpret_cast<const float4*>(P.q + (size_t)i * C + h * dh);
+            const float4* k4 = reinterpret_cast<const float4*>(P.k + (size_t)j * C + h * dh);
+            float dot = 0.f;
+            for (int c4 = 0; c4 < dh / 4; ++c4) {
+                const float4 qa = __ldg(q4 + c4), kv = __ldg(k4 + c4);
+                dot = fmaf(qa.x, kv.x, dot);
+                dot = fmaf(qa.y, kv.y, dot);
+                dot = fmaf(qa.z, kv.z, dot);
+                dot = fmaf(qa.w, kv.w, dot);
+            }
+            const float a = ga * dot * inv;
+#pragma unroll
+            for (int hh = 0; hh < kMaxHeads; ++hh) {
+                if (hh == h) {
+                    const float mn = fmaxf(m[hh], a);
+                    sm[hh] = sm[hh] * expf(m[hh] - mn) + expf(a - mn);
+                    m[hh] = mn;
+                }
+            }
+        }
+    });
+#pragma unroll
+    for (int h = 0; h < kMaxHeads; ++h) {
+        if (h < H) {
+            float mh = m[h], shh = sm[h];
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                const float mo = __shfl_xor_sync(0xffffffffu, mh, o), so = __shfl_xor_sync(0xffffffffu, shh, o);
+                const float mn = fmaxf(mh, mo);
+                const float sa = (mh == -INFINITY) ? 0.f : shh * expf(mh - mn);
+                const float sb = (mo == -INFINITY) ? 0.f : so * expf(mo - mn);
+                mh = mn;
+                shh = sa + sb;
+            }
+            if (lane == 0) P.lse[(size_t)i * H + h] = (cnt > 0) ? mh + logf(shh) : 0.f;
+        }
+    }
+}
+
+__global__ void k_flags_to_status(const int* flags, int* status) {
+    if (*flags & kFlagNonFinite) atomicExch(status, (int)E2F_ERR_NONFINITE);
+}
+
 // Node range per CTA: part[k] = first node whose edges start at or after
 // k * E / n_ctas (so a node never spans two CTAs).
 __global__ void k_partition(const int32_t* row_ptr, int n_atoms, int n_ctas, int32_t* part) {
@@ -492,7 +559,7 @@ struct SmemLayout {
         wga = o;    o += (size_t)kTcMaxRbf * kMaxHeads * 4;
         o = (o + 7) & ~size_t(7);
         bars = o;   o += (2 * kNS + 15) * 8;
-        misc = o;   o += 64;
+        misc = o;   o += 64 + 4 * kTileE * 4;  // TMEM base, abort flag, last slot; gate (i, j) lists
         dsub = o;   o += 16 * 8;
         total = o;
     }
@@ -720,6 +787,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
     uint64_t* gempty = gfull + 2; // value gate of a tile buffer consumed (producer -> gate warps)
     uint32_t* tmem_sm = reinterpret_cast<uint32_t*>(smem + S.misc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + S.misc + 8);
+    int* last_slot = reinterpret_cast<int*>(smem + S.misc + 16);  // producer: node slot of the last edge
+    int* gij = reinterpret_cast<int*>(smem + S.misc + 64);        // gate warps: [2][128] (i, j) per edge
     long long* dsub = reinterpret_cast<long long*>(smem + S.dsub);  // sub-step cycle sums (timers on)
     float* wga = reinterpret_cast<float*>(smem + S.wga);            // [16][H] logit-gate weights
     const bool dbgon = P.dbg != nullptr;
@@ -805,13 +874,43 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
                     }
                     nb0 = lo;
                 } else {
-                    nb0 = nid[(b ^ 1) * kTileE + kTileE - 1];  // node of edge e0 - 1
+                    nb0 = *last_slot;  // node slot of edge e0 - 1
                 }
                 nbase = nb0;
                 const int n = nbase + 1 + p;
                 rpw[p] = (n <= n_end) ? P.row_ptr[n] : 0x7fffffff;
             }
             asm volatile("bar.sync 1, 128;" ::: "memory");
+            if (P.cells) {
+                // fused traversal: the neighbours of the tile's nodes, enumerated from the
+                // cell lists (one warp per node slot, stencil order) into jn
+                const int e_last = e0 + ne - 1;
+                int s_last;
+                if (e_last < rpw[kTileE - 1]) {
+                    int lo = 0, hi = kTileE;
+                    while (lo < hi) {
+                        const int mid = (lo + hi) >> 1;
+                        if (rpw[mid] <= e_last) lo = mid + 1; else hi = mid;
+                    }
+                    s_last = nbase + lo;
+                } else {
+                    int lo = nbase, hi = n_end - 1;
+                    while (lo < hi) {
+                        int mid = (lo + hi + 1) >> 1;
+                        if (P.row_ptr[mid] <= e_last) lo = mid; else hi = mid - 1;
+                    }
+                    s_last = lo;
+                }
+                int* jt = jn + b * kTileE;
+                for (int sl = nbase + (warp - 4); sl <= s_last; sl += 4) {
+                    const int base = P.row_ptr[sl];
+                    warp_neighbors(P.cv, P.cv.spos[sl], P.cv.sidx[sl], [&](int k, int j) {
+                        const int e = base + k;
+                        if (e >= e0 && e < e0 + ne) jt[e - e0] = j;
+                    });
+                }
+                asm volatile("bar.sync 1, 128;" ::: "memory");
+            }
             tlast = c_a;
             E2F_TICK(0);
             __half2* Dg = P.dscr + (size_t)(blockIdx.x * 2 + b) * dglob_pairs();
@@ -821,8 +920,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
                 __half2* Dh = dph + (size_t)p * DPS;
                 if (p < ne) {
                     const int e = e0 + p;
-                    const int j = P.col[e];
-                    // node i: last n with row_ptr[n] <= e = nbase + #{k: rpw[k] <= e}
+                    const int j = P.cells ? jn[b * kTileE + p] : P.col[e];
+                    // node slot: last n with row_ptr[n] <= e = nbase + #{k: rpw[k] <= e}
                     int i;
                     if (e < rpw[kTileE - 1]) {
                         int lo = 0, hi = kTileE;  // first k with rpw[k] > e
@@ -839,6 +938,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
                         }
                         i = lo;
                     }
+                    if (p == kTileE - 1) *last_slot = i;
+                    if (P.cells) i = P.cv.sidx[i];  // slot -> atom
                     float3 r = edge_vec(P.pos, i, j, P.box);
                     const float d = sqrtf(r.x * r.x + r.y * r.y + r.z * r.z);
                     E2F_TICK(1);
@@ -1160,14 +1261,45 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
             if (!bar_and(3, 64, okw)) break;
             const int e0 = e_begin + t * kTileE;
             const int ne = min(kTileE, e_end - e0);
-            for (int k = gp; k < kTileE; k += 64) {  // radial basis of the tile's edges
-                float rr[kTcMaxRbf];
-                if (k < ne) {
-                    const int e = e0 + k, j = P.col[e];
-                    int lo = n_begin, hi = n_end - 1;  // node i: last n with row_ptr[n] <= e
+            int* gi = gij + b * 2 * kTileE;
+            if (P.cells) {  // fused traversal: (atom, neighbour) of each edge from the cell lists
+                auto slot_of = [&](int e) {
+                    int lo = n_begin, hi = n_end - 1;
                     while (lo < hi) {
                         const int mid = (lo + hi + 1) >> 1;
                         if (P.row_ptr[mid] <= e) lo = mid; else hi = mid - 1;
+                    }
+                    return lo;
+                };
+                const int s_first = slot_of(e0), s_last = slot_of(e0 + ne - 1);
+                for (int sl = s_first + (warp - 14); sl <= s_last; sl += 2) {
+                    const int base = P.row_ptr[sl], ia = P.cv.sidx[sl];
+                    warp_neighbors(P.cv, P.cv.spos[sl], ia, [&](int k, int j) {
+                        const int e = base + k;
+                        if (e >= e0 && e < e0 + ne) {
+                            gi[e - e0] = ia;
+                            gi[kTileE + e - e0] = j;
+                        }
+                    });
+                }
+                asm volatile("bar.sync 3, 64;" ::: "memory");
+            }
+            for (int k = gp; k < kTileE; k += 64) {  // radial basis of the tile's edges
+                float rr[kTcMaxRbf];
+                if (k < ne) {
+                    const int e = e0 + k;
+                    int lo, j;
+                    if (P.cells) {
+                        lo = gi[k];
+                        j = gi[kTileE + k];
+                    } else {
+                        j = P.col[e];
+                        lo = n_begin;
+                        int hi = n_end - 1;  // node i: last n with row_ptr[n] <= e
+                        while (lo < hi) {
+                            const int mid = (lo + hi + 1) >> 1;
+                            if (P.row_ptr[mid] <= e) lo = mid; else hi = mid - 1;
+                        }
                     }
                     const float3 r = edge_vec(P.pos, lo, j, P.box);
                     const float d = sqrtf(r.x * r.x + r.y * r.y + r.z * r.z);
@@ -1390,7 +1522,7 @@ static cudaError_t launch_tc(const tc::TcParams& P, const tc::TcMaps& T, int gri
     return cudaGetLastError();
 }
 
-cudaError_t run_attention_tc(const AttnArgs& a, void* tc_ws, cudaStream_t s) {
+cudaError_t run_attention_tc(const AttnArgs& a, void* tc_ws, cudaStream_t s, const CellLists* cl) {
     const int L = a.L, C = a.C, H = a.H, K = n_sh(L), N = a.n_atoms;
     int dev = 0, sms = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -1445,7 +1577,13 @@ cudaError_t run_attention_tc(const AttnArgs& a, void* tc_ws, cudaStream_t s) {
     sp.box = a.box; sp.pos = a.pos; sp.row_ptr = a.row_ptr; sp.col = a.col; sp.q = a.q; sp.k = a.k;
     sp.Wrad = a.Wrad; sp.lse = lse;
     count_launch();
-    tc::k_softmax_stats<<<(N + 7) / 8, 256, 0, s>>>(sp);
+    if (cl) {
+        tc::k_softmax_stats_cells<<<(N + 7) / 8, 256, 0, s>>>(sp, cl->view);
+        count_launch();
+        tc::k_flags_to_status<<<1, 1, 0, s>>>(cl->flags, a.status);
+    } else {
+        tc::k_softmax_stats<<<(N + 7) / 8, 256, 0, s>>>(sp);
+    }
     count_launch();
     tc::k_partition<<<(grid + 1 + 127) / 128, 128, 0, s>>>(a.row_ptr, N, grid, part);
     e = cudaMemsetAsync(a.out, 0, (size_t)N * K * C * 4, s);
@@ -1456,6 +1594,8 @@ cudaError_t run_attention_tc(const AttnArgs& a, void* tc_ws, cudaStream_t s) {
     P.pos = a.pos; P.row_ptr = a.row_ptr; P.col = a.col; P.x = x16; P.whT = whT; P.gscr = gscr; P.scale = scale;
     P.q = a.q; P.k = a.k; P.lse = lse; P.Wrad = a.Wrad; P.part = part; P.xs = xs; P.dscr = dscr; P.out = a.out;
     P.status = a.status;
+    P.cells = cl ? 1 : 0;
+    if (cl) P.cv = cl->view;
     P.dbg = nullptr;
     if (const char* env = getenv("E2F_TC_TIMERS")) {
         if (atoi(env) > 0) {

@@ -6,6 +6,7 @@
 #include <cuda_fp16.h>
 #include <stdint.h>
 
+#include "cell_grid.cuh"
 #include "common.cuh"
 
 namespace e2f {
@@ -44,7 +45,9 @@ struct TcGroup {
 
 struct TcParams {
     int C, H, n_rbf, G;
-    int M;  // SO(2) maps for |m| <= M
+    int M;      // SO(2) maps for |m| <= M
+    int cells;  // fused traversal: row_ptr is per node slot in cell order, neighbours from cv
+    CellView cv;
     float cutoff;
     Box box;
     const float* pos;

@@ -1,0 +1,187 @@
+// Cell grid shared by the neighbour build and the fused-traversal attention:
+// the exact fp32 pair predicate, the cell of a point, the bucket of a cell
+// and the 27-cell stencil (see include/e2f.h, neighbour list).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <algorithm>
+#include <cmath>
+
+#include "common.cuh"
+
+namespace e2f {
+
+constexpr float kCellSlack = 1.0e-3f;
+
+enum : int { kFlagNonFinite = 1, kFlagBadGraph = 2 };
+
+struct Grid {
+    Box box;
+    int nc[3];           // periodic: cells per axis
+    float cell;          // open: cell side
+    uint32_t n_buckets;  // periodic: n_graphs * nc^3; open: power of two
+    uint32_t mask;       // open: n_buckets - 1
+    int offs[3][3];      // periodic stencil offsets per axis (deduplicated)
+    int noff[3];
+};
+
+__device__ __forceinline__ bool pair_within(float4 a, float4 b, const Grid& g, float rc2) {
+    // the exact sequence of IEEE round-to-nearest operations (no FMA)
+    float dx = __fsub_rn(b.x, a.x), dy = __fsub_rn(b.y, a.y), dz = __fsub_rn(b.z, a.z);
+    if (g.box.periodic) {
+        dx = __fsub_rn(dx, __fmul_rn(g.box.len.x, rintf(__fmul_rn(dx, g.box.inv.x))));
+        dy = __fsub_rn(dy, __fmul_rn(g.box.len.y, rintf(__fmul_rn(dy, g.box.inv.y))));
+        dz = __fsub_rn(dz, __fmul_rn(g.box.len.z, rintf(__fmul_rn(dz, g.box.inv.z))));
+    }
+    float d2 = __fadd_rn(__fadd_rn(__fmul_rn(dx, dx), __fmul_rn(dy, dy)), __fmul_rn(dz, dz));
+    return d2 < rc2;
+}
+
+__device__ __forceinline__ void cell_of(float x, float y, float z, const Grid& g, long long c[3]) {
+    // fp64 so that the cell of a point never moves by more than the slack
+    const double p[3] = {x, y, z};
+    if (g.box.periodic) {
+        const double len[3] = {g.box.len.x, g.box.len.y, g.box.len.z};
+#pragma unroll
+        for (int a = 0; a < 3; ++a) {
+            double w = p[a] - len[a] * floor(p[a] / len[a]);   // wrapped into [0, len]
+            long long k = (long long)(w * (double(g.nc[a]) / len[a]));
+            c[a] = k < 0 ? 0 : (k >= g.nc[a] ? g.nc[a] - 1 : k);
+        }
+    } else {
+#pragma unroll
+        for (int a = 0; a < 3; ++a) c[a] = (long long)floor(p[a] / double(g.cell));
+    }
+}
+
+__device__ __forceinline__ uint32_t bucket_of(const long long c[3], int gid, const Grid& g) {
+    if (g.box.periodic) {
+        long long idx = (((long long)gid * g.nc[2] + c[2]) * g.nc[1] + c[1]) * g.nc[0] + c[0];
+        return (uint32_t)idx;
+    }
+    uint64_t h = (uint64_t)c[0] * 0x9E3779B97F4A7C15ull;
+    h ^= (uint64_t)c[1] * 0xC2B2AE3D27D4EB4Full + (h >> 29);
+    h ^= (uint64_t)c[2] * 0x165667B19E3779F9ull + (h >> 32);
+    h ^= (uint64_t)(uint32_t)gid * 0x27D4EB2F165667C5ull + (h >> 31);
+    h ^= h >> 33;
+    return (uint32_t)h & g.mask;
+}
+
+// the (up to) 27 distinct buckets around cell c; returns how many
+__device__ __forceinline__ int stencil_buckets(const long long c[3], int gid, const Grid& g, uint32_t out[27]) {
+    int n = 0;
+    if (g.box.periodic) {
+        for (int iz = 0; iz < g.noff[2]; ++iz)
+            for (int iy = 0; iy < g.noff[1]; ++iy)
+                for (int ix = 0; ix < g.noff[0]; ++ix) {
+                    long long cc[3] = {c[0] + g.offs[0][ix], c[1] + g.offs[1][iy], c[2] + g.offs[2][iz]};
+                    for (int a = 0; a < 3; ++a) cc[a] = (cc[a] % g.nc[a] + g.nc[a]) % g.nc[a];
+                    out[n++] = bucket_of(cc, gid, g);
+                }
+        return n;
+    }
+    for (int dz = -1; dz <= 1; ++dz)
+        for (int dy = -1; dy <= 1; ++dy)
+            for (int dx = -1; dx <= 1; ++dx) {
+                long long cc[3] = {c[0] + dx, c[1] + dy, c[2] + dz};
+                uint32_t b = bucket_of(cc, gid, g);
+                bool dup = false;
+                for (int k = 0; k < n; ++k) dup |= (out[k] == b);
+                if (!dup) out[n++] = b;
+            }
+    return n;
+}
+
+
+// Read-only view of a periodic cell list (one graph) for kernels that
+// enumerate neighbours on the fly: atoms sorted by bucket (float4 x, y, z,
+// graph id), their indices, bucket starts (n_buckets + 1).
+struct CellView {
+    Grid g;
+    float rc2;
+    const float4* spos;
+    const int32_t* sidx;
+    const uint32_t* start;
+};
+
+// One warp: enumerates the neighbours j of atom i (at me) in stencil order,
+// bucket by bucket, atoms of a bucket in their stored order; calls
+// f(k, j) on the lane that holds the k-th neighbour. Returns the count
+// (the same on every lane). The predicate is the neighbour build's.
+template <typename F>
+__device__ __forceinline__ int warp_neighbors(const CellView& cv, float4 me, int i, F&& f) {
+    const int lane = threadIdx.x & 31;
+    long long c[3];
+    cell_of(me.x, me.y, me.z, cv.g, c);
+    uint32_t bk[27];
+    const int nb = stencil_buckets(c, 0, cv.g, bk);
+    int total = 0;
+    for (int b = 0; b < nb; ++b) {
+        const uint32_t s0 = cv.start[bk[b]], s1 = cv.start[bk[b] + 1];
+        for (uint32_t s = s0; s < s1; s += 32) {
+            bool hit = false;
+            int j = -1;
+            if (s + lane < s1) {
+                const float4 o = cv.spos[s + lane];
+                j = cv.sidx[s + lane];
+                hit = (j != i) && pair_within(me, o, cv.g, cv.rc2);
+            }
+            const unsigned m = __ballot_sync(0xffffffffu, hit);
+            if (hit) f(total + __popc(m & ((1u << lane) - 1u)), j);
+            total += __popc(m);
+        }
+    }
+    return total;
+}
+
+// Cell lists of one periodic system for the fused attention (built by
+// build_cell_lists in neighbors.cu): the view, the per-node edge offsets in
+// bucket order (rp[N+1]) and an error flag word.
+struct CellLists {
+    CellView view;
+    const int32_t* rp;
+    int* flags;
+};
+size_t cell_lists_bytes(int64_t n_atoms, const float* box_host, float cutoff);
+cudaError_t build_cell_lists(const float* pos, int n_atoms, const float* box_host, float cutoff, void* ws,
+                             CellLists* out, cudaStream_t s);
+
+inline bool make_grid(const float* box_host, float cutoff, int n_graphs, int64_t n_atoms, Grid& g) {
+    g.box.periodic = box_host != nullptr;
+    if (g.box.periodic) {
+        g.box.len = make_float3(box_host[0], box_host[1], box_host[2]);
+        g.box.inv = make_float3(1.0f / box_host[0], 1.0f / box_host[1], 1.0f / box_host[2]);
+        long long total = std::max(1, n_graphs);
+        for (int a = 0; a < 3; ++a) {
+            int nc = (int)std::floor(double(box_host[a]) / (double(cutoff) * (1.0 + kCellSlack)));
+            g.nc[a] = std::max(1, std::min(nc, 1024));
+        }
+        // keep the grid at most 2^26 buckets: coarsen the largest axis
+        while (total * g.nc[0] * g.nc[1] * g.nc[2] > (1ll << 26)) {
+            int a = (g.nc[0] >= g.nc[1] && g.nc[0] >= g.nc[2]) ? 0 : (g.nc[1] >= g.nc[2] ? 1 : 2);
+            g.nc[a] = std::max(1, g.nc[a] / 2);
+        }
+        for (int a = 0; a < 3; ++a) {
+            if (g.nc[a] >= 3) { g.offs[a][0] = -1; g.offs[a][1] = 0; g.offs[a][2] = 1; g.noff[a] = 3; }
+            else if (g.nc[a] == 2) { g.offs[a][0] = 0; g.offs[a][1] = 1; g.noff[a] = 2; }
+            else { g.offs[a][0] = 0; g.noff[a] = 1; }
+        }
+        g.n_buckets = (uint32_t)(total * g.nc[0] * g.nc[1] * g.nc[2]);
+        g.mask = 0;
+        g.cell = 0.f;
+    } else {
+        g.box.len = g.box.inv = make_float3(0.f, 0.f, 0.f);
+        g.cell = cutoff * (1.0f + kCellSlack);
+        uint32_t nb = 64;
+        while ((int64_t)nb < 2 * n_atoms && nb < (1u << 28)) nb <<= 1;
+        g.n_buckets = nb;
+        g.mask = nb - 1;
+        for (int a = 0; a < 3; ++a) { g.nc[a] = 0; g.noff[a] = 0; }
+    }
+    return true;
+}
+
+
+}  // namespace e2f

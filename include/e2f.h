@@ -225,6 +225,36 @@ e2f_status e2f_attention_debug_timers(void* workspace, size_t ws_bytes, int64_t 
                                       const e2f_attn_cfg* cfg, int64_t* host_out, int n_values,
                                       void* stream);
 
+/* ------------------------------------------------------------------------
+ * On-the-fly equivariant attention with the cell-list traversal fused in
+ * (no neighbour list in memory): the same layer as e2f_onfly_attention,
+ * but the kernels find each node's neighbours themselves from a cell list
+ * of the positions (the neighbour build's grid, buckets ordered by atom
+ * index), so no E-sized array (col) is written or read. Only O(N) data is
+ * kept: the cell lists and per-node edge offsets. Nodes are processed in
+ * cell order. The neighbour set is the exact fp32 predicate of
+ * e2f_build_neighbors (cutoff = cfg->cutoff); the order of the edges of a
+ * node differs from the CSR call, so sums may differ in the last bits.
+ *
+ * Periodic boxes (box_host non-NULL, cutoff <= min(box)/2) and the
+ * tensor-core configurations (e2f_attention_uses_tensor_cores) only;
+ * otherwise E2F_ERR_UNSUPPORTED. One system (no graph batching).
+ * Arguments as for e2f_onfly_attention without row_ptr, col, n_pairs;
+ * workspace >= e2f_attention_cells_workspace_size(...) bytes, 256-byte
+ * aligned. Asynchronous (no host synchronisation); non-finite positions
+ * are reported through e2f_attention_status as E2F_ERR_NONFINITE.
+ * ---------------------------------------------------------------------- */
+size_t e2f_attention_cells_workspace_size(int64_t n_atoms, const float* box_host,
+                                          const e2f_attn_cfg* cfg);
+
+e2f_status e2f_onfly_attention_cells(const e2f_attn_cfg* cfg, const float* pos,
+                                     int64_t n_atoms, const float* box_host,
+                                     const void* x, const float* W_q,
+                                     const float* W_k, const float* W_rad,
+                                     const void* W_so2, float* out,
+                                     void* workspace, size_t ws_bytes,
+                                     void* stream);
+
 /* Synchronises `stream` and returns the device status recorded by the last
  * e2f_onfly_attention call on this workspace (E2F_OK or E2F_ERR_TIMEOUT);
  * each call clears the word when it starts. */

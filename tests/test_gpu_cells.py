@@ -1,0 +1,51 @@
+"""Attention with the cell-list traversal fused in (no neighbour list in
+memory): the same layer as the CSR call on the same neighbour sets, checked
+against the CSR call, the oracle, and itself (repeatability)."""
+import numpy as np
+import pytest
+import torch
+
+import atomistic_cell_list_b200 as e2f
+from gpu_util import TOL, DeviceInputs, oracle_csr, rel_err_per_degree
+
+pytestmark = pytest.mark.gpu
+
+
+def _both(cfg_id):
+    d = DeviceInputs(cfg_id)
+    w = d.w
+    cfg = e2f.make_cfg(w.L, w.C, w.H, w.n_rbf, w.cutoff, w.dtype)
+    rp, col = e2f.e2f_build_neighbors(d.pos, d.box, w.cutoff, d.graph_ptr)
+    csr = e2f.e2f_onfly_attention(cfg, d.pos, d.box, rp, col, d.x, d.Wq, d.Wk, d.Wrad, d.Wso2)
+    fused = e2f.e2f_onfly_attention_cells(cfg, d.pos, d.box, d.x, d.Wq, d.Wk, d.Wrad, d.Wso2)
+    return d, cfg, csr, fused
+
+
+@pytest.mark.parametrize("cfg_id", [3, 4])
+def test_fused_traversal_matches_the_csr_call(cfg_id):
+    d, cfg, csr, fused = _both(cfg_id)
+    # same edges and per-edge arithmetic; the edges of a node come in another order, so
+    # the per-node sums (about 90 terms of both signs) round differently in fp32
+    assert rel_err_per_degree(fused.cpu().numpy(), csr.cpu().numpy(), d.w.L) <= 1e-3
+
+
+def test_fused_traversal_matches_the_oracle_and_repeats():
+    d, cfg, csr, fused = _both(3)
+    w = d.w
+    nodes = np.random.default_rng(11).choice(w.n_atoms, 24, replace=False)
+    rp0, col0 = oracle_csr(3)
+    ref = d.oracle()(w.pos, w.box, rp0, col0, d.x_f64, nodes=nodes)
+    assert rel_err_per_degree(fused.cpu().numpy()[nodes].astype(np.float64), ref, w.L) <= TOL[w.dtype]
+    again = e2f.e2f_onfly_attention_cells(cfg, d.pos, d.box, d.x, d.Wq, d.Wk, d.Wrad, d.Wso2)
+    assert torch.equal(again, fused)
+
+
+def test_fused_traversal_scope():
+    d = DeviceInputs(3)
+    w = d.w
+    cfg = e2f.make_cfg(w.L, w.C, w.H, w.n_rbf, w.cutoff, w.dtype)
+    assert e2f.e2f_attention_cells_workspace_size(w.n_atoms, None, cfg) == 0  # periodic boxes only
+    f32 = e2f.make_cfg(w.L, w.C, w.H, w.n_rbf, w.cutoff, "f32")
+    with pytest.raises(e2f.E2FError) as ei:
+        e2f.e2f_onfly_attention_cells(f32, d.pos, d.box, d.x, d.Wq, d.Wk, d.Wrad, d.Wso2)
+    assert ei.value.code == 2
