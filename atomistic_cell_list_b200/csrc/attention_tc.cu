@@ -289,32 +289,47 @@ __global__ void __launch_bounds__(256) k_softmax_stats(StatsParams P) {
 }
 
 // The same statistics with the neighbours enumerated from the cell lists
-// (fused traversal): one warp per node slot in cell order, one lane per
-// neighbour found, logits evaluated as in the main kernel.
+// (fused traversal): one warp per node slot in cell order. The warp collects
+// the node's neighbours in shared memory, kStatsCap at a time (a denser node
+// enumerates again for the next window), then evaluates them with the lane
+// layout and per-edge arithmetic of k_softmax_stats.
+constexpr int kStatsCap = 256;
 __global__ void __launch_bounds__(256) k_softmax_stats_cells(StatsParams P, CellView cv) {
+    __shared__ int jbuf[8][kStatsCap];
     const int s = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
     if (s >= P.n_atoms) return;
+    int* jb = jbuf[threadIdx.x >> 5];
     const int H = P.H, C = P.C, dh = C / H, G = P.G, Gv = G - H;
+    const int h = lane % H, es = lane / H, EP = 32 / H;
     const float inv = rsqrtf((float)dh);
-    const int i = cv.sidx[s];
-    float m[kMaxHeads], sm[kMaxHeads];
+    float wcol[kTcMaxRbf];
 #pragma unroll
-    for (int h = 0; h < kMaxHeads; ++h) { m[h] = -INFINITY; sm[h] = 0.f; }
-    const int cnt = warp_neighbors(cv, cv.spos[s], i, [&](int, int j) {
-        const float3 r = edge_vec(P.pos, i, j, P.box);
-        const float d = sqrtf(r.x * r.x + r.y * r.y + r.z * r.z);
-        float rr[kTcMaxRbf];
-        rbf_all<kTcMaxRbf>(d, P.cutoff, P.n_rbf, rr);
-        for (int h = 0; h < H; ++h) {
+    for (int kb = 0; kb < kTcMaxRbf; ++kb) wcol[kb] = kb < P.n_rbf ? P.Wrad[(size_t)kb * G + Gv + h] : 0.f;
+    const int i = cv.sidx[s];
+    const float4 me = cv.spos[s];
+    const float4* q4 = reinterpret_cast<const float4*>(P.q + (size_t)i * C + h * dh);
+    const int d4 = dh / 4;
+    float m = -INFINITY, sum = 0.f;
+    int cnt = 0;
+    for (int w0 = 0;; w0 += kStatsCap) {
+        cnt = warp_neighbors(cv, me, i, [&](int k, int j) {
+            if (k >= w0 && k < w0 + kStatsCap) jb[k - w0] = j;
+        });
+        __syncwarp();
+        const int n_here = min(cnt - w0, kStatsCap);
+        for (int k = es; k < n_here; k += EP) {
+            const int j = jb[k];
+            const float3 r = edge_vec(P.pos, i, j, P.box);
+            const float d = sqrtf(r.x * r.x + r.y * r.y + r.z * r.z);
+            float rr[kTcMaxRbf];
+            rbf_all<kTcMaxRbf>(d, P.cutoff, P.n_rbf, rr);
             float ga = 0.f;
 #pragma unroll
-            for (int kb = 0; kb < kTcMaxRbf; ++kb)
-                ga = fmaf(rr[kb], kb < P.n_rbf ? __ldg(P.Wrad + (size_t)kb * G + Gv + h) : 0.f, ga);
-            const float4* q4 = reinterpret_cast<const float4*>(P.q + (size_t)i * C + h * dh);
+            for (int kb = 0; kb < kTcMaxRbf; ++kb) ga = fmaf(rr[kb], wcol[kb], ga);
             const float4* k4 = reinterpret_cast<const float4*>(P.k + (size_t)j * C + h * dh);
             float dot = 0.f;
-            for (int c4 = 0; c4 < dh / 4; ++c4) {
+            for (int c4 = 0; c4 < d4; ++c4) {
                 const float4 qa = __ldg(q4 + c4), kv = __ldg(k4 + c4);
                 dot = fmaf(qa.x, kv.x, dot);
                 dot = fmaf(qa.y, kv.y, dot);
@@ -322,32 +337,22 @@ __global__ void __launch_bounds__(256) k_softmax_stats_cells(StatsParams P, Cell
                 dot = fmaf(qa.w, kv.w, dot);
             }
             const float a = ga * dot * inv;
-#pragma unroll
-            for (int hh = 0; hh < kMaxHeads; ++hh) {
-                if (hh == h) {
-                    const float mn = fmaxf(m[hh], a);
-                    sm[hh] = sm[hh] * expf(m[hh] - mn) + expf(a - mn);
-                    m[hh] = mn;
-                }
-            }
+            const float mn = fmaxf(m, a);
+            sum = sum * expf(m - mn) + expf(a - mn);
+            m = mn;
         }
-    });
-#pragma unroll
-    for (int h = 0; h < kMaxHeads; ++h) {
-        if (h < H) {
-            float mh = m[h], shh = sm[h];
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                const float mo = __shfl_xor_sync(0xffffffffu, mh, o), so = __shfl_xor_sync(0xffffffffu, shh, o);
-                const float mn = fmaxf(mh, mo);
-                const float sa = (mh == -INFINITY) ? 0.f : shh * expf(mh - mn);
-                const float sb = (mo == -INFINITY) ? 0.f : so * expf(mo - mn);
-                mh = mn;
-                shh = sa + sb;
-            }
-            if (lane == 0) P.lse[(size_t)i * H + h] = (cnt > 0) ? mh + logf(shh) : 0.f;
-        }
+        __syncwarp();
+        if (cnt <= w0 + kStatsCap) break;
     }
+    for (int o = H; o < 32; o <<= 1) {
+        const float mo = __shfl_xor_sync(0xffffffffu, m, o), so = __shfl_xor_sync(0xffffffffu, sum, o);
+        const float mn = fmaxf(m, mo);
+        const float sa = (m == -INFINITY) ? 0.f : sum * expf(m - mn);
+        const float sb = (mo == -INFINITY) ? 0.f : so * expf(mo - mn);
+        m = mn;
+        sum = sa + sb;
+    }
+    if (es == 0) P.lse[(size_t)i * H + h] = (cnt > 0) ? m + logf(sum) : 0.f;
 }
 
 __global__ void k_flags_to_status(const int* flags, int* status) {
@@ -558,7 +563,7 @@ struct SmemLayout {
         rrs = o;    o += (size_t)kTileE * kTcMaxRbf * 4;
         wga = o;    o += (size_t)kTcMaxRbf * kMaxHeads * 4;
         o = (o + 7) & ~size_t(7);
-        bars = o;   o += (2 * kNS + 15) * 8;
+        bars = o;   o += (2 * kNS + 17) * 8;
         misc = o;   o += 64 + 4 * kTileE * 4;  // TMEM base, abort flag, last slot; gate (i, j) lists
         dsub = o;   o += 16 * 8;
         total = o;
@@ -785,6 +790,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
     uint64_t* fin = dbar + 2;
     uint64_t* gfull = fin + 1;    // value gate of a tile buffer written (gate warps -> producer)
     uint64_t* gempty = gfull + 2; // value gate of a tile buffer consumed (producer -> gate warps)
+    uint64_t* jfull = gempty + 2; // fused traversal: (i, j) of a tile buffer listed (gate warps -> producer)
     uint32_t* tmem_sm = reinterpret_cast<uint32_t*>(smem + S.misc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + S.misc + 8);
     int* last_slot = reinterpret_cast<int*>(smem + S.misc + 16);  // producer: node slot of the last edge
@@ -808,6 +814,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
         for (int b = 0; b < 2; ++b) {
             mbar_init(gfull + b, 64);
             mbar_init(gempty + b, 128);
+            mbar_init(jfull + b, 64);
         }
         *abort_flag = 0;
         for (int k = 0; k < 16; ++k) dsub[k] = 0;
@@ -882,34 +889,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
             }
             asm volatile("bar.sync 1, 128;" ::: "memory");
             if (P.cells) {
-                // fused traversal: the neighbours of the tile's nodes, enumerated from the
-                // cell lists (one warp per node slot, stencil order) into jn
-                const int e_last = e0 + ne - 1;
-                int s_last;
-                if (e_last < rpw[kTileE - 1]) {
-                    int lo = 0, hi = kTileE;
-                    while (lo < hi) {
-                        const int mid = (lo + hi) >> 1;
-                        if (rpw[mid] <= e_last) lo = mid + 1; else hi = mid;
-                    }
-                    s_last = nbase + lo;
-                } else {
-                    int lo = nbase, hi = n_end - 1;
-                    while (lo < hi) {
-                        int mid = (lo + hi + 1) >> 1;
-                        if (P.row_ptr[mid] <= e_last) lo = mid; else hi = mid - 1;
-                    }
-                    s_last = lo;
-                }
-                int* jt = jn + b * kTileE;
-                for (int sl = nbase + (warp - 4); sl <= s_last; sl += 4) {
-                    const int base = P.row_ptr[sl];
-                    warp_neighbors(P.cv, P.cv.spos[sl], P.cv.sidx[sl], [&](int k, int j) {
-                        const int e = base + k;
-                        if (e >= e0 && e < e0 + ne) jt[e - e0] = j;
-                    });
-                }
-                asm volatile("bar.sync 1, 128;" ::: "memory");
+                // fused traversal: the gate warps list (atom, neighbour) of the tile's edges in
+                // gij[b]; they refill it only after gempty[b], i.e. after this tile's P2
+                const bool okj = wait_t(jfull + b, (t >> 1) & 1, abort_flag, P.status, w_free);
+                if (!bar_and(1, 128, okj)) break;
             }
             tlast = c_a;
             E2F_TICK(0);
@@ -920,7 +903,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
                 __half2* Dh = dph + (size_t)p * DPS;
                 if (p < ne) {
                     const int e = e0 + p;
-                    const int j = P.cells ? jn[b * kTileE + p] : P.col[e];
+                    const int* gl = gij + b * 2 * kTileE;  // fused traversal: [i x 128][j x 128]
+                    const int j = P.cells ? gl[kTileE + p] : P.col[e];
                     // node slot: last n with row_ptr[n] <= e = nbase + #{k: rpw[k] <= e}
                     int i;
                     if (e < rpw[kTileE - 1]) {
@@ -939,7 +923,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
                         i = lo;
                     }
                     if (p == kTileE - 1) *last_slot = i;
-                    if (P.cells) i = P.cv.sidx[i];  // slot -> atom
+                    if (P.cells) i = gl[p];  // slot -> atom
                     float3 r = edge_vec(P.pos, i, j, P.box);
                     const float d = sqrtf(r.x * r.x + r.y * r.y + r.z * r.z);
                     E2F_TICK(1);
@@ -1283,6 +1267,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
                     });
                 }
                 asm volatile("bar.sync 3, 64;" ::: "memory");
+                mbar_arrive(jfull + b);  // releases the lists to the producer (CTA scope)
             }
             for (int k = gp; k < kTileE; k += 64) {  // radial basis of the tile's edges
                 float rr[kTcMaxRbf];

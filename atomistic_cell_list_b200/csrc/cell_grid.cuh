@@ -69,6 +69,12 @@ __device__ __forceinline__ uint32_t bucket_of(const long long c[3], int gid, con
     return (uint32_t)h & g.mask;
 }
 
+// periodic: cell index c + offset wrapped into [0, nc); c is in [0, nc) and
+// the offset in {-1, 0, 1}, so one add or subtract of nc suffices
+__device__ __forceinline__ long long wrap_cell(long long c, int nc) {
+    return c < 0 ? c + nc : (c >= nc ? c - nc : c);
+}
+
 // the (up to) 27 distinct buckets around cell c; returns how many
 __device__ __forceinline__ int stencil_buckets(const long long c[3], int gid, const Grid& g, uint32_t out[27]) {
     int n = 0;
@@ -76,8 +82,9 @@ __device__ __forceinline__ int stencil_buckets(const long long c[3], int gid, co
         for (int iz = 0; iz < g.noff[2]; ++iz)
             for (int iy = 0; iy < g.noff[1]; ++iy)
                 for (int ix = 0; ix < g.noff[0]; ++ix) {
-                    long long cc[3] = {c[0] + g.offs[0][ix], c[1] + g.offs[1][iy], c[2] + g.offs[2][iz]};
-                    for (int a = 0; a < 3; ++a) cc[a] = (cc[a] % g.nc[a] + g.nc[a]) % g.nc[a];
+                    long long cc[3] = {wrap_cell(c[0] + g.offs[0][ix], g.nc[0]),
+                                       wrap_cell(c[1] + g.offs[1][iy], g.nc[1]),
+                                       wrap_cell(c[2] + g.offs[2][iz], g.nc[2])};
                     out[n++] = bucket_of(cc, gid, g);
                 }
         return n;
@@ -106,30 +113,73 @@ struct CellView {
     const uint32_t* start;
 };
 
+// Periodic stencil entry b (0 <= b < noff[0] noff[1] noff[2]; x fastest, as
+// in stencil_buckets): the bucket of one graph's grid. Offsets are {-1, 0, 1}
+// on an axis of three or more cells, {0, 1} on two cells, {0} on one.
+__device__ __forceinline__ uint32_t stencil_bucket(const long long c[3], const Grid& g, int b) {
+    const int ix = b % g.noff[0], r = b / g.noff[0];
+    const int iy = r % g.noff[1], iz = r / g.noff[1];
+    const long long cx = wrap_cell(c[0] + ix - (g.noff[0] == 3), g.nc[0]);
+    const long long cy = wrap_cell(c[1] + iy - (g.noff[1] == 3), g.nc[1]);
+    const long long cz = wrap_cell(c[2] + iz - (g.noff[2] == 3), g.nc[2]);
+    return (uint32_t)((cz * g.nc[1] + cy) * g.nc[0] + cx);
+}
+
 // One warp: enumerates the neighbours j of atom i (at me) in stencil order,
 // bucket by bucket, atoms of a bucket in their stored order; calls
 // f(k, j) on the lane that holds the k-th neighbour. Returns the count
 // (the same on every lane). The predicate is the neighbour build's.
+// Lane b holds the range of stencil bucket b; a warp scan concatenates the
+// ranges into one candidate sequence t = 0 .. ncand-1 (stencil order kept),
+// and candidate t sits at sorted position base(b) + t for the bucket b with
+// excl(b) <= t < incl(b), found by a binary search over the lanes. Candidates
+// are loaded 4 x 32 at a time before any is tested, so the loads overlap.
 template <typename F>
 __device__ __forceinline__ int warp_neighbors(const CellView& cv, float4 me, int i, F&& f) {
+    constexpr unsigned kAll = 0xffffffffu;
+    constexpr int kU = 4;
     const int lane = threadIdx.x & 31;
     long long c[3];
     cell_of(me.x, me.y, me.z, cv.g, c);
-    uint32_t bk[27];
-    const int nb = stencil_buckets(c, 0, cv.g, bk);
+    const int nb = cv.g.noff[0] * cv.g.noff[1] * cv.g.noff[2];
+    uint32_t st = 0, len = 0;
+    if (lane < nb) {
+        const uint32_t bk = stencil_bucket(c, cv.g, lane);
+        st = cv.start[bk];
+        len = cv.start[bk + 1] - st;
+    }
+    uint32_t incl = len;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t v = __shfl_up_sync(kAll, incl, o);
+        if (lane >= o) incl += v;
+    }
+    const uint32_t ncand = __shfl_sync(kAll, incl, 31);
+    const uint32_t base = st - (incl - len);  // modulo 2^32: base + t is the sorted position
     int total = 0;
-    for (int b = 0; b < nb; ++b) {
-        const uint32_t s0 = cv.start[bk[b]], s1 = cv.start[bk[b] + 1];
-        for (uint32_t s = s0; s < s1; s += 32) {
-            bool hit = false;
-            int j = -1;
-            if (s + lane < s1) {
-                const float4 o = cv.spos[s + lane];
-                j = cv.sidx[s + lane];
-                hit = (j != i) && pair_within(me, o, cv.g, cv.rc2);
+    for (uint32_t t0 = 0; t0 < ncand; t0 += 32 * kU) {
+        float4 o[kU];
+        int jj[kU];
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+            const uint32_t t = t0 + 32 * u + lane;
+            int b = 0;  // number of buckets with incl <= t
+#pragma unroll
+            for (int step = 16; step > 0; step >>= 1)
+                if (__shfl_sync(kAll, incl, b + step - 1) <= t) b += step;
+            const uint32_t sp = __shfl_sync(kAll, base, b) + t;
+            o[u] = me;
+            jj[u] = -1;
+            if (t < ncand) {
+                o[u] = cv.spos[sp];
+                jj[u] = cv.sidx[sp];
             }
-            const unsigned m = __ballot_sync(0xffffffffu, hit);
-            if (hit) f(total + __popc(m & ((1u << lane) - 1u)), j);
+        }
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+            const bool hit = jj[u] >= 0 && jj[u] != i && pair_within(me, o[u], cv.g, cv.rc2);
+            const unsigned m = __ballot_sync(kAll, hit);
+            if (hit) f(total + __popc(m & ((1u << lane) - 1u)), jj[u]);
             total += __popc(m);
         }
     }

@@ -204,6 +204,10 @@ def run_reference(args):
 # --------------------------------------------------------------------------
 # our arm
 # --------------------------------------------------------------------------
+def use_tc_path(e2f, cfg) -> bool:
+    return bool(e2f.e2f_attention_uses_tensor_cores(cfg))
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -300,6 +304,41 @@ def run_ours(args):
     ms_nbr = float(tot[2]) / args.steps
     ms_ker = float(tot[3]) / args.steps
 
+    # the same step with the cell-list traversal fused into the attention (periodic boxes):
+    # no neighbour list is written; the call sorts atoms into cells and enumerates each
+    # node's neighbours inside the kernel
+    fused = None
+    if use_tc_path(e2f, cfg) and box is not None and gptr is None:
+        ws_c = torch.empty(e2f.e2f_attention_cells_workspace_size(w.n_atoms, box, cfg), dtype=torch.uint8,
+                           device=dev)
+        out_c = torch.empty_like(out)
+
+        def fused_step():
+            e2f.e2f_onfly_attention_cells(cfg, d["pos"], box, d["x"], d["Wq"], d["Wk"], d["Wrad"], d["Wso2"],
+                                          out=out_c, workspace=ws_c, check=False)
+        for _ in range(args.warmup):
+            fused_step()
+        torch.cuda.synchronize(dev)
+        assert e2f.e2f_attention_status(ws_c) == 0
+        f_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+        for s in range(args.steps):
+            flush.zero_()
+            f_ev[s][0].record(stream)
+            fused_step()
+            f_ev[s][1].record(stream)
+        torch.cuda.synchronize(dev)
+        status = e2f.e2f_attention_status(ws_c)
+        assert status == 0, e2f.status_string(status)
+        t_f = torch.tensor([sum(e[0].elapsed_time(e[1]) for e in f_ev)], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(t_f, op=dist.ReduceOp.MAX)
+        ms_f = float(t_f[0]) / args.steps
+        fused = {"ms_per_step": ms_f, "value": world * E / (ms_f * 1e-3), "unit": "pairs/s",
+                 "workspace_bytes": int(ws_c.numel()), "neighbor_list_bytes": 0,
+                 "note": "e2f_onfly_attention_cells: cell sort + attention with in-kernel neighbour "
+                         "enumeration, same layer and neighbour sets as the CSR step"}
+        del ws_c, out_c
+
     # end to end through the public API with pinned host buffers
     pinned = {k: v.pin_memory() for k, v in h_inputs.items()}
     h_out = torch.empty(out.shape, dtype=torch.float32).pin_memory()
@@ -358,6 +397,7 @@ def run_ours(args):
             "e2e": {"value": world * E / (ms_e2e * 1e-3), "unit": "pairs/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e},
             "gpu_launches": int(launches),
+            "fused_traversal": fused,
             "activation_memory": {"workspace_bytes": int(ws.numel()), "edge_tensor_bytes": 0,
                                   "csr_bytes": 4 * (w.n_atoms + 1) + 4 * E,
                                   "note": "the library's only scratch is the caller's workspace: O(N) + O(SMs), "

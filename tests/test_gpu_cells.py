@@ -49,3 +49,21 @@ def test_fused_traversal_scope():
     with pytest.raises(e2f.E2FError) as ei:
         e2f.e2f_onfly_attention_cells(f32, d.pos, d.box, d.x, d.Wq, d.Wk, d.Wrad, d.Wso2)
     assert ei.value.code == 2
+
+
+def test_fused_traversal_dense_nodes():
+    # about 570 neighbours per atom: more than a tile (128 edges) and more than the
+    # statistics pass buffers per window (256), on a 3 x 3 x 3 cell grid
+    d = DeviceInputs(3)
+    w = d.w
+    n, side, rc = 4000, 17.0, 5.5
+    pos = torch.from_numpy(np.random.default_rng(5).uniform(0.0, side, (n, 3)).astype(np.float32)).to(d.pos.device)
+    box = [side] * 3
+    x = d.x.repeat(2, 1, 1)[:n].contiguous()
+    cfg = e2f.make_cfg(w.L, w.C, w.H, w.n_rbf, rc, w.dtype)
+    rp, col = e2f.e2f_build_neighbors(pos, box, rc)
+    deg = (rp[1:] - rp[:-1]).cpu().numpy()
+    assert deg.min() > 256 and deg.max() > 512
+    csr = e2f.e2f_onfly_attention(cfg, pos, box, rp, col, x, d.Wq, d.Wk, d.Wrad, d.Wso2)
+    fused = e2f.e2f_onfly_attention_cells(cfg, pos, box, x, d.Wq, d.Wk, d.Wrad, d.Wso2)
+    assert rel_err_per_degree(fused.cpu().numpy(), csr.cpu().numpy(), w.L) <= 1e-3
