@@ -24,4 +24,6 @@ Modules:
   eaas       SO(2) weights <-> dense path weights (Lemma 4.1 + Eq. 13)
   layer      radial basis, gates, logits, two-pass softmax, dense messages
   neighbors  the exact fp32 cutoff predicate, brute force and KD-tree search
+  grad       the same layer in plain PyTorch fp64, differentiated by autograd
+             (gradients for the backward pass)
 """
