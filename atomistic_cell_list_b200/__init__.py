@@ -54,6 +54,10 @@ _SIGS = {
     "e2f_attention_cells_workspace_size": (_sz, [_i64, _vp, ctypes.POINTER(e2f_attn_cfg)]),
     "e2f_onfly_attention_cells": (ctypes.c_int, [ctypes.POINTER(e2f_attn_cfg), _vp, _i64, _vp, _vp, _vp, _vp, _vp,
                                                  _vp, _vp, _vp, _sz, _vp]),
+    "e2f_attention_backward_workspace_size": (_sz, [_i64, _i64, ctypes.POINTER(e2f_attn_cfg)]),
+    "e2f_onfly_attention_backward": (ctypes.c_int, [ctypes.POINTER(e2f_attn_cfg), _vp, _i64, _vp, _vp, _vp, _i64,
+                                                    _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                                    _vp, _sz, _vp]),
     "e2f_edge_wigner_blocks": (ctypes.c_int, [_vp, _i64, ctypes.c_int, _vp, _vp, _vp]),
     "e2f_launch_count": (_i64, []),
     "e2f_attention_uses_tensor_cores": (ctypes.c_int, [ctypes.POINTER(e2f_attn_cfg)]),
@@ -246,6 +250,40 @@ def e2f_onfly_attention_cells(cfg: e2f_attn_cfg, pos, box, x, W_q, W_k, W_rad, W
         _check(lib().e2f_attention_status(_ptr(workspace), workspace.numel(), s),
                "e2f_onfly_attention_cells (device)")
     return out
+
+
+def e2f_attention_backward_workspace_size(n_atoms: int, n_pairs: int, cfg: e2f_attn_cfg) -> int:
+    return int(lib().e2f_attention_backward_workspace_size(int(n_atoms), int(n_pairs), ctypes.byref(cfg)))
+
+
+def e2f_onfly_attention_backward(cfg: e2f_attn_cfg, pos, box, row_ptr, col, x, W_q, W_k, W_rad, W_so2, grad_out,
+                                 want_weights: bool = True, workspace: torch.Tensor | None = None,
+                                 out: dict | None = None, stream=None) -> dict:
+    """Gradients of sum(grad_out * layer(...)) (see include/e2f.h): a dict with
+    pos, x, W_rad and, when want_weights, W_q, W_k, W_so2 (all fp32)."""
+    _need_cuda(pos, row_ptr, col, x, W_q, W_k, W_rad, W_so2, grad_out, workspace)
+    n = pos.shape[0]
+    dev = pos.device
+    f32 = torch.float32
+    g = dict(out) if out is not None else {}
+    g.setdefault("pos", torch.empty((n, 3), dtype=f32, device=dev))
+    g.setdefault("x", torch.empty(x.shape, dtype=f32, device=dev))
+    g.setdefault("W_rad", torch.empty(W_rad.shape, dtype=f32, device=dev))
+    if want_weights:
+        g.setdefault("W_q", torch.empty(W_q.shape, dtype=f32, device=dev))
+        g.setdefault("W_k", torch.empty(W_k.shape, dtype=f32, device=dev))
+        g.setdefault("W_so2", torch.empty(W_so2.shape, dtype=f32, device=dev))
+    ws_bytes = e2f_attention_backward_workspace_size(n, col.numel(), cfg)
+    if workspace is None or workspace.numel() < ws_bytes:
+        workspace = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
+    b, keep = _box_arg(box)
+    code = lib().e2f_onfly_attention_backward(
+        ctypes.byref(cfg), _ptr(pos), n, b, _ptr(row_ptr), _ptr(col), col.numel(), _ptr(x), _ptr(W_q), _ptr(W_k),
+        _ptr(W_rad), _ptr(W_so2), _ptr(grad_out), _ptr(g["pos"]), _ptr(g["x"]), _ptr(g.get("W_q")),
+        _ptr(g.get("W_k")), _ptr(g["W_rad"]), _ptr(g.get("W_so2")), _ptr(workspace), workspace.numel(),
+        _stream(stream))
+    _check(code, "e2f_onfly_attention_backward")
+    return g
 
 
 def e2f_attention_status(workspace: torch.Tensor, stream=None) -> int:

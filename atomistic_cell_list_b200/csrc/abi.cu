@@ -208,6 +208,93 @@ extern "C" void e2f_attention_set_kernel_events(void* start_event, void* stop_ev
     set_tc_kernel_events(start_event, stop_event);
 }
 
+namespace {
+
+struct BwdWs {
+    size_t o_q, o_k, o_wt, o_lse, o_gq, o_gk, o_beta, bytes;
+};
+
+BwdWs bwd_layout(int64_t n_atoms, int64_t n_pairs, const e2f_attn_cfg& c) {
+    BwdWs w{};
+    size_t o = 0;
+    auto take = [&](size_t b) { size_t r = o; o = align_up(o + b, 256); return r; };
+    w.o_q = take(4 * (size_t)n_atoms * c.C);
+    w.o_k = take(4 * (size_t)n_atoms * c.C);
+    w.o_wt = take(4 * so2_total(c.L, c.C, effective_mmax(c.L, c.m_max)));
+    w.o_lse = take(4 * (size_t)n_atoms * c.H);
+    w.o_gq = take(4 * (size_t)n_atoms * c.C);
+    w.o_gk = take(4 * (size_t)n_atoms * c.C);
+    w.o_beta = take(4 * (size_t)n_pairs * c.H);
+    w.bytes = o;
+    return w;
+}
+
+}  // namespace
+
+extern "C" size_t e2f_attention_backward_workspace_size(int64_t n_atoms, int64_t n_pairs, const e2f_attn_cfg* cfg) {
+    if (check_cfg(cfg) != E2F_OK || n_atoms < 0 || n_pairs < 0) return 0;
+    return bwd_layout(n_atoms, n_pairs, *cfg).bytes;
+}
+
+extern "C" e2f_status e2f_onfly_attention_backward(const e2f_attn_cfg* cfg, const float* pos, int64_t n_atoms,
+                                                   const float* box_host, const int32_t* row_ptr,
+                                                   const int32_t* col, int64_t n_pairs, const void* x,
+                                                   const float* W_q, const float* W_k, const float* W_rad,
+                                                   const void* W_so2, const float* grad_out, float* grad_pos,
+                                                   float* grad_x, float* grad_W_q, float* grad_W_k,
+                                                   float* grad_W_rad, float* grad_W_so2, void* workspace,
+                                                   size_t ws_bytes, void* stream_) {
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    e2f_status st = check_cfg(cfg);
+    if (st != E2F_OK) return st;
+    if (!bwd_supported(cfg->L, cfg->C, cfg->H, cfg->n_rbf)) return E2F_ERR_UNSUPPORTED;
+    if (n_atoms < 0 || n_atoms > INT32_MAX || n_pairs < 0 || n_pairs > INT32_MAX) return E2F_ERR_INVALID_ARG;
+    if (n_atoms == 0) return E2F_OK;
+    if (!pos || !row_ptr || (n_pairs > 0 && !col) || !x || !W_q || !W_k || !W_rad || !W_so2 || !grad_out ||
+        !grad_pos || !grad_x || !grad_W_rad || !workspace)
+        return E2F_ERR_INVALID_ARG;
+    if (box_host) {
+        for (int a = 0; a < 3; ++a)
+            if (!(box_host[a] > 0.f) || !std::isfinite(box_host[a]) || cfg->cutoff > 0.5f * box_host[a])
+                return E2F_ERR_INVALID_ARG;
+    }
+    if (reinterpret_cast<uintptr_t>(workspace) % 256 || reinterpret_cast<uintptr_t>(x) % 16 ||
+        reinterpret_cast<uintptr_t>(W_so2) % 16 || reinterpret_cast<uintptr_t>(grad_out) % 16 ||
+        reinterpret_cast<uintptr_t>(grad_x) % 16)
+        return E2F_ERR_ALIGNMENT;
+    const BwdWs L = bwd_layout(n_atoms, n_pairs, *cfg);
+    if (ws_bytes < L.bytes) return E2F_ERR_INVALID_ARG;
+    char* ws = static_cast<char*>(workspace);
+
+    BwdArgs b{};
+    AttnArgs& a = b.fwd;
+    a.L = cfg->L; a.C = cfg->C; a.H = cfg->H; a.n_rbf = cfg->n_rbf; a.cutoff = cfg->cutoff;
+    a.M = effective_mmax(cfg->L, cfg->m_max);
+    a.bf16 = cfg->feat_dtype == E2F_BF16;
+    a.n_atoms = (int)n_atoms; a.n_pairs = n_pairs;
+    a.box.periodic = box_host != nullptr;
+    if (box_host) {
+        a.box.len = make_float3(box_host[0], box_host[1], box_host[2]);
+        a.box.inv = make_float3(1.0f / box_host[0], 1.0f / box_host[1], 1.0f / box_host[2]);
+    } else {
+        a.box.len = a.box.inv = make_float3(0.f, 0.f, 0.f);
+    }
+    a.pos = pos; a.row_ptr = row_ptr; a.col = col; a.x = x;
+    a.Wq = W_q; a.Wk = W_k; a.Wrad = W_rad; a.Wso2 = W_so2;
+    a.q = reinterpret_cast<float*>(ws + L.o_q);
+    a.k = reinterpret_cast<float*>(ws + L.o_k);
+    a.Wt = reinterpret_cast<float*>(ws + L.o_wt);
+    b.grad_out = grad_out;
+    b.lse = reinterpret_cast<float*>(ws + L.o_lse);
+    b.beta = reinterpret_cast<float*>(ws + L.o_beta);
+    b.gq = reinterpret_cast<float*>(ws + L.o_gq);
+    b.gk = reinterpret_cast<float*>(ws + L.o_gk);
+    b.gpos = grad_pos; b.gx = grad_x; b.gWq = grad_W_q; b.gWk = grad_W_k; b.gWrad = grad_W_rad;
+    b.gWso2 = grad_W_so2;
+    E2F_CUDA_TRY(run_attention_bwd(b, stream));
+    return E2F_OK;
+}
+
 extern "C" e2f_status e2f_attention_debug_timers(void* workspace, size_t ws_bytes, int64_t n_atoms,
                                                 const e2f_attn_cfg* cfg, int64_t* host_out, int n_values,
                                                 void* stream_) {

@@ -58,6 +58,30 @@ struct AttnArgs {
 };
 
 cudaError_t run_attention_simt(const AttnArgs& a, cudaStream_t s);
+// q = W_q x[l=0], k = W_k x[l=0]; packed SO(2) weights -> fp32 with each block transposed
+cudaError_t qk_project(const void* x, bool bf16, int n_atoms, int K, int C, const float* Wq, const float* Wk,
+                       float* q, float* k, cudaStream_t s);
+cudaError_t repack_so2_f32(const void* w, bool bf16, int L, int C, int M, float* out, cudaStream_t s);
+
+// Backward pass: the forward's arguments (a.out unused; a.q, a.k, a.Wt are
+// workspace) plus dLoss/dout and the gradient outputs (gWq, gWk, gWso2 may be
+// null: not computed).
+struct BwdArgs {
+    AttnArgs fwd;
+    const float* grad_out;
+    float* lse;
+    float* beta;
+    float* gq;
+    float* gk;
+    float* gpos;
+    float* gx;
+    float* gWq;
+    float* gWk;
+    float* gWrad;
+    float* gWso2;
+};
+bool bwd_supported(int L, int C, int H, int n_rbf);
+cudaError_t run_attention_bwd(const BwdArgs& b, cudaStream_t s);
 struct CellLists;
 // cl != nullptr: fused traversal (a.row_ptr = per-slot offsets in cell order, a.col unused)
 cudaError_t run_attention_tc(const AttnArgs& a, void* tc_ws, cudaStream_t s, const CellLists* cl = nullptr);

@@ -1,0 +1,850 @@
+// Backward of the on-the-fly equivariant attention (fp32 CUDA cores).
+//
+// The pages' conservative variant takes forces as the negative gradient of
+// the energy with respect to the positions (E2Former-V2, gist.science
+// Technical Summary 2.2 and the experiments on molecular dynamics), so the
+// layer's backward pass follows its forward. Given G = dLoss/dout [N, K, C],
+// this file computes dLoss / d(pos, x, W_q, W_k, W_rad, W_so2) in the same
+// recompute style as the forward: per-edge quantities (frame, Wigner blocks,
+// gates, rotated features, SO(2) outputs) are rebuilt on chip and never
+// stored per edge; the only O(E) scratch is one scalar per edge and head.
+//
+// Per edge e = (i <- j) with alpha = softmax weight, X~ = D(g_v . x_j),
+// Y = F(X~) (the SO(2) maps), v = D^T Y, out_i = sum_e alpha v:
+//   beta^h   = sum_{c in h} <D G_i, Y>                 (= <G_i, v> per head)
+//   dY       = alpha D G_i,   dX~ = F^T(dY)
+//   dx_j    += g_v . D^T dX~,  dg_v = sum_m x_j . D^T dX~
+//   dW_so2   = sum_e dY (x) X~   (A and B blocks; a separate tile kernel)
+//   da^h     = alpha^h (beta^h - delta_i^h),  delta_i^h = sum_e alpha beta
+//   logits a = g_a <q_i, k_j>/sqrt(d): dq_i, dk_j, dg_a
+//   gates    [g_v | g_a] = rho(d) W_rad: dW_rad, dd through rho'(d)
+//   direction: for the rotation exp(eps Omega_a) R (Omega_a = e_a x, a = x, y)
+//     dLoss/deps_a = <dD_a (alpha G_i), Y> + <dX~, dD_a (g_v . x_j)>,
+//     with dD_a = d/deps D(exp(eps Omega_a) R); the direction moves by
+//     R^T e_y (a = x) and -R^T e_x (a = y), so the tangential part of
+//     dLoss/dr is (dL/deps_x R^T e_y - dL/deps_y R^T e_x) / d.
+//   dpos_j += dLoss/dr,  dpos_i -= dLoss/dr  (r = mic(pos_j - pos_i)).
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include <algorithm>
+
+#include "attention.cuh"
+#include "common.cuh"
+
+#define E2F_CUDA_TRY_E(expr)                          \
+    do {                                              \
+        const cudaError_t e2f_e_ = (expr);            \
+        if (e2f_e_ != cudaSuccess) return e2f_e_;     \
+    } while (0)
+
+namespace e2f {
+namespace bwd {
+
+constexpr int kNt = 256;     // threads of the node kernel and the weight-gradient kernel
+constexpr int kTe = 8;       // edges per tile of the node kernel
+constexpr int kDwT = 64;     // weight-gradient tile side
+constexpr int kDwE = 32;     // edges per operand sub-chunk of the weight-gradient kernel
+constexpr int kDwChunk = 256;  // edges per geometry chunk (one per thread)
+
+struct BwdParams {
+    int n_atoms, C, H, n_rbf, M;
+    int n_pairs;
+    float cutoff;
+    Box box;
+    const float* pos;
+    const int32_t* row_ptr;
+    const int32_t* col;
+    const void* x;
+    const void* W;     // packed SO(2) weights as given (row-major blocks)
+    const float* Wt;   // the same, fp32, each block transposed
+    const float* Wrad;
+    const float* q;
+    const float* k;
+    const float* G;    // dLoss/dout
+    float* lse;        // [N, H]
+    float* beta;       // [E, H]
+    float* gq;         // [N, C]
+    float* gk;         // [N, C]
+    float* gpos;       // [N, 3]
+    float* gx;         // [N, K, C]
+    float* gWrad;      // [n_rbf, G]
+    float* gW;         // packed like W
+};
+
+// Derivative of the Wigner blocks along dR (R -> R + eps dR): the recursion
+// D^l = step(D^1, D^{l-1}) is bilinear in its two arguments, so
+// dD^l = step(dD^1, D^{l-1}) + step(D^1, dD^{l-1}), with dD^1 = dR in the
+// (y, z, x) order of the degree-1 harmonics.
+template <int L>
+__device__ __forceinline__ void wigner_dblocks(const float* D, const float dR[3][3], float* dD) {
+    dD[0] = 0.f;
+    if constexpr (L >= 1) {
+        const int p[3] = {1, 2, 0};
+#pragma unroll
+        for (int a = 0; a < 3; ++a)
+#pragma unroll
+            for (int b = 0; b < 3; ++b) dD[1 + a * 3 + b] = dR[p[a]][p[b]];
+    }
+    float t[81];
+    if constexpr (L >= 2) {
+        ir::step<2>(dD + 1, D + wig_off(1), dD + wig_off(2));
+        ir::step<2>(D + 1, dD + wig_off(1), t);
+        for (int a = 0; a < 25; ++a) dD[wig_off(2) + a] += t[a];
+    }
+    if constexpr (L >= 3) {
+        ir::step<3>(dD + 1, D + wig_off(2), dD + wig_off(3));
+        ir::step<3>(D + 1, dD + wig_off(2), t);
+        for (int a = 0; a < 49; ++a) dD[wig_off(3) + a] += t[a];
+    }
+    if constexpr (L >= 4) {
+        ir::step<4>(dD + 1, D + wig_off(3), dD + wig_off(4));
+        ir::step<4>(D + 1, dD + wig_off(3), t);
+        for (int a = 0; a < 81; ++a) dD[wig_off(4) + a] += t[a];
+    }
+}
+
+// radial basis value and its derivative in d (the forward's rbf)
+__device__ __forceinline__ void rbf_and_deriv(float d, int k, float cutoff, int n_rbf, float& v, float& dv) {
+    const float step = cutoff / float(n_rbf - 1);
+    const float t = (d - float(k) * step) / step;
+    const float ang = 3.14159265358979323846f * d / cutoff;
+    const float u = 0.5f * (cosf(ang) + 1.f);
+    const float du = -0.5f * (3.14159265358979323846f / cutoff) * sinf(ang);
+    const float ex = expf(-t * t);
+    v = u * ex;
+    dv = du * ex + u * ex * (-2.f * t / step);
+}
+
+// logit of edge (i <- j), head h, and the pieces its gradient needs
+struct Logit {
+    float a, ga, dot;
+};
+__device__ __forceinline__ Logit edge_logit(const BwdParams& P, int i, int j, int h, int Gv, int G, float inv,
+                                            float3* u_out, float* d_out, float* gap_out) {
+    const float3 r = edge_vec(P.pos, i, j, P.box);
+    const float d = sqrtf(r.x * r.x + r.y * r.y + r.z * r.z);
+    float ga = 0.f, gap = 0.f;
+    for (int kb = 0; kb < P.n_rbf; ++kb) {
+        float v, dv;
+        rbf_and_deriv(d, kb, P.cutoff, P.n_rbf, v, dv);
+        const float w = P.Wrad[(size_t)kb * G + Gv + h];
+        ga = fmaf(v, w, ga);
+        gap = fmaf(dv, w, gap);
+    }
+    const int dh = P.C / P.H;
+    const float* qi = P.q + (size_t)i * P.C + h * dh;
+    const float* kj = P.k + (size_t)j * P.C + h * dh;
+    float dot = 0.f;
+    for (int c = 0; c < dh; ++c) dot = fmaf(qi[c], kj[c], dot);
+    if (u_out) *u_out = make_float3(r.x / d, r.y / d, r.z / d);
+    if (d_out) *d_out = d;
+    if (gap_out) *gap_out = gap;
+    return Logit{ga * dot * inv, ga, dot};
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+size_t node_smem_floats(int L, int C, int H, int n_rbf) {
+    const int K = n_sh(L), WS = wig_size(L), Gv = (L + 1) * C, G = Gv + H;
+    const int KH = (L >= 1) ? std::max((L + 1) * C, 2 * L * C) : C;
+    return (size_t)K * C + 3ull * kTe * WS + 2ull * kTe * n_rbf + (size_t)kTe * G + (size_t)kTe * Gv +
+           2ull * kTe * H + 12ull * kTe + 2ull * KH * kTe + (size_t)n_rbf * G + C + 2ull * H + 4 + kTe +
+           2ull * kNt + kTe;
+}
+
+// One CTA per destination node at a time (persistent over nodes): every
+// gradient except dW_so2, dW_q, dW_k and the l = 0 part of dx that flows
+// through q and k.
+template <int L, typename T>
+__global__ void __launch_bounds__(kNt) k_bwd_node(BwdParams P) {
+    constexpr int K = n_sh(L);
+    constexpr int WS = wig_size(L);
+    const int C = P.C, H = P.H, dh = C / H, nr = P.n_rbf, M = P.M;
+    const int Gv = (L + 1) * C, G = Gv + H;
+    const int KH = (L >= 1) ? max((L + 1) * C, 2 * L * C) : C;
+    const T* __restrict__ x = static_cast<const T*>(P.x);
+    const T* __restrict__ W = static_cast<const T*>(P.W);
+
+    extern __shared__ float sm[];
+    float* Gi = sm;                    // [K][C] dLoss/dout_i
+    float* Dm = Gi + K * C;            // [te][WS] Wigner blocks
+    float* Dx = Dm + kTe * WS;         // [te][WS] their derivative along Omega_x
+    float* Dy = Dx + kTe * WS;         // [te][WS] ... along Omega_y
+    float* rho = Dy + kTe * WS;        // [te][nr]
+    float* rhop = rho + kTe * nr;      // [te][nr] d rho / d d
+    float* g = rhop + kTe * nr;        // [te][G] gates
+    float* dgv = g + kTe * G;          // [te][Gv] dLoss/dg_v
+    float* alpha = dgv + kTe * Gv;     // [te][H]
+    float* beta = alpha + kTe * H;     // [te][H]
+    float* geo = beta + kTe * H;       // [te][12]: r^ (3), d, R^T e_y (3), -R^T e_x (3), dL/deps_x, dL/deps_y
+    float* hs = geo + 12 * kTe;        // [KH][te] gated rotated input of the |m| block
+    float* gy = hs + KH * kTe;         // [KH][te] dLoss/dY of the block
+    float* gWr = gy + KH * kTe;        // [nr][G] this CTA's part of dW_rad
+    float* gqi = gWr + nr * G;         // [C]
+    float* lse_s = gqi + C;            // [H]
+    float* dlt = lse_s + H;            // [H] delta_i
+    float* gpi = dlt + H;              // [4] dpos_i
+    float* ddv = gpi + 4;              // [te]
+    float* red = ddv + kTe;            // [2 kNt]
+    int* jn = reinterpret_cast<int*>(red + 2 * kNt);  // [te]
+
+    const int tid = threadIdx.x, nt = blockDim.x, lane = tid & 31, warp = tid >> 5;
+    const float inv = rsqrtf((float)dh);
+    for (int t = tid; t < nr * G; t += nt) gWr[t] = 0.f;
+
+    for (int i = blockIdx.x; i < P.n_atoms; i += gridDim.x) {
+        const int e_begin = P.row_ptr[i], e_end = P.row_ptr[i + 1], deg = e_end - e_begin;
+        __syncthreads();
+        for (int t = tid; t < K * C; t += nt) Gi[t] = P.G[(size_t)i * K * C + t];
+        for (int t = tid; t < C; t += nt) gqi[t] = 0.f;
+        if (tid < H) dlt[tid] = 0.f;
+        if (tid < 4) gpi[tid] = 0.f;
+        // softmax statistics of node i (thread t: head t % H)
+        {
+            const int h = tid % H;
+            float mh = -INFINITY, sh = 0.f;
+            for (int e = tid / H; e < deg; e += nt / H) {
+                const Logit lg = edge_logit(P, i, P.col[e_begin + e], h, Gv, G, inv, nullptr, nullptr, nullptr);
+                const float mn = fmaxf(mh, lg.a);
+                sh = sh * expf(mh - mn) + expf(lg.a - mn);
+                mh = mn;
+            }
+            red[tid] = mh;
+            red[nt + tid] = sh;
+        }
+        __syncthreads();
+        if (tid < H) {
+            float mh = -INFINITY, sh = 0.f;
+            for (int t = tid; t < nt; t += H) {
+                const float mo = red[t], so = red[nt + t];
+                if (mo == -INFINITY) continue;
+                const float mn = fmaxf(mh, mo);
+                sh = ((mh == -INFINITY) ? 0.f : sh * expf(mh - mn)) + so * expf(mo - mn);
+                mh = mn;
+            }
+            lse_s[tid] = (deg > 0) ? mh + logf(sh) : 0.f;
+            P.lse[(size_t)i * H + tid] = lse_s[tid];
+        }
+        __syncthreads();
+
+        for (int e0 = e_begin; e0 < e_end; e0 += kTe) {
+            const int ne = min(kTe, e_end - e0);
+            // geometry, frame, Wigner blocks and their two tangential derivatives
+            if (tid < kTe) {
+                const int e = tid;
+                float* gg = geo + e * 12;
+                if (e < ne) {
+                    const int j = P.col[e0 + e];
+                    jn[e] = j;
+                    const float3 r = edge_vec(P.pos, i, j, P.box);
+                    const float d = sqrtf(r.x * r.x + r.y * r.y + r.z * r.z);
+                    float R[3][3];
+                    edge_frame(r.x / d, r.y / d, r.z / d, R);
+                    wigner_blocks<L>(R, Dm + e * WS);
+                    float dR[3][3];
+#pragma unroll
+                    for (int c = 0; c < 3; ++c) { dR[0][c] = 0.f; dR[1][c] = -R[2][c]; dR[2][c] = R[1][c]; }
+                    wigner_dblocks<L>(Dm + e * WS, dR, Dx + e * WS);
+#pragma unroll
+                    for (int c = 0; c < 3; ++c) { dR[0][c] = R[2][c]; dR[1][c] = 0.f; dR[2][c] = -R[0][c]; }
+                    wigner_dblocks<L>(Dm + e * WS, dR, Dy + e * WS);
+                    for (int kb = 0; kb < nr; ++kb) rbf_and_deriv(d, kb, P.cutoff, nr, rho[e * nr + kb], rhop[e * nr + kb]);
+                    gg[0] = r.x / d; gg[1] = r.y / d; gg[2] = r.z / d; gg[3] = d;
+                    gg[4] = R[1][0]; gg[5] = R[1][1]; gg[6] = R[1][2];
+                    gg[7] = -R[0][0]; gg[8] = -R[0][1]; gg[9] = -R[0][2];
+                } else {
+                    jn[e] = i;
+                    for (int a = 0; a < WS; ++a) { Dm[e * WS + a] = 0.f; Dx[e * WS + a] = 0.f; Dy[e * WS + a] = 0.f; }
+                    for (int kb = 0; kb < nr; ++kb) { rho[e * nr + kb] = 0.f; rhop[e * nr + kb] = 0.f; }
+                    for (int a = 0; a < 10; ++a) gg[a] = 0.f;
+                    gg[3] = 1.f;
+                }
+                gg[10] = 0.f;
+                gg[11] = 0.f;
+            }
+            __syncthreads();
+            for (int t = tid; t < kTe * G; t += nt) {
+                const int e = t / G, c = t % G;
+                float s = 0.f;
+                for (int kb = 0; kb < nr; ++kb) s = fmaf(rho[e * nr + kb], P.Wrad[(size_t)kb * G + c], s);
+                g[t] = s;
+            }
+            for (int t = tid; t < kTe * Gv; t += nt) dgv[t] = 0.f;
+            __syncthreads();
+            for (int t = tid; t < kTe * H; t += nt) {
+                const int e = t / H, h = t % H;
+                float al = 0.f;
+                if (e < ne) {
+                    const float* qi = P.q + (size_t)i * C + h * dh;
+                    const float* kj = P.k + (size_t)jn[e] * C + h * dh;
+                    float dot = 0.f;
+                    for (int c = 0; c < dh; ++c) dot = fmaf(qi[c], kj[c], dot);
+                    al = expf(g[e * G + Gv + h] * dot * inv - lse_s[h]);
+                }
+                alpha[t] = al;
+                beta[t] = 0.f;
+            }
+            __syncthreads();
+
+#pragma unroll 1
+            for (int m = 0; m <= M; ++m) {
+                const int nm = (L + 1 - m) * C;
+                // gated rotated input X~ of the block: hs[(s, l1-m, c)][e]
+                for (int t = tid; t < kTe * nm; t += nt) {
+                    const int e = t / nm, r = t % nm;
+                    const int l1 = m + r / C, c = r % C;
+                    float vp = 0.f, vm = 0.f;
+                    if (e < ne) {
+                        const float* D = Dm + e * WS + wig_off(l1);
+                        const int w = 2 * l1 + 1;
+                        const size_t xb = ((size_t)jn[e] * K + l1 * l1) * C + c;
+                        for (int n = 0; n < w; ++n) {
+                            const float xv = load_feat(x, xb + (size_t)n * C);
+                            vp = fmaf(D[(l1 + m) * w + n], xv, vp);
+                            vm = fmaf(D[(l1 - m) * w + n], xv, vm);
+                        }
+                        const float gv = g[e * G + l1 * C + c];
+                        vp *= gv;
+                        vm *= gv;
+                    }
+                    hs[(size_t)r * kTe + e] = vp;
+                    if (m > 0) hs[(size_t)(nm + r) * kTe + e] = vm;
+                }
+                __syncthreads();
+                // Y = F(X~) row by row; beta, the first direction term, dY = alpha D G_i
+                const float* At = P.Wt + so2_offset(L, C, m, 0);
+                const float* Bt = (m > 0) ? P.Wt + so2_offset(L, C, m, 1) : nullptr;
+                for (int r = tid; r < nm; r += nt) {
+                    const int l3 = m + r / C, c = r % C, h = c / dh;
+                    float op[kTe], om[kTe];
+#pragma unroll
+                    for (int e = 0; e < kTe; ++e) { op[e] = 0.f; om[e] = 0.f; }
+                    for (int kk = 0; kk < nm; ++kk) {
+                        const float a = At[(size_t)kk * nm + r];
+                        const float4* hp = reinterpret_cast<const float4*>(hs + (size_t)kk * kTe);
+                        if (m == 0) {
+#pragma unroll
+                            for (int q4 = 0; q4 < kTe / 4; ++q4) {
+                                const float4 v = hp[q4];
+                                op[4 * q4 + 0] = fmaf(a, v.x, op[4 * q4 + 0]);
+                                op[4 * q4 + 1] = fmaf(a, v.y, op[4 * q4 + 1]);
+                                op[4 * q4 + 2] = fmaf(a, v.z, op[4 * q4 + 2]);
+                                op[4 * q4 + 3] = fmaf(a, v.w, op[4 * q4 + 3]);
+                            }
+                        } else {
+                            const float b = Bt[(size_t)kk * nm + r];
+                            const float4* hmn = reinterpret_cast<const float4*>(hs + (size_t)(nm + kk) * kTe);
+#pragma unroll
+                            for (int q4 = 0; q4 < kTe / 4; ++q4) {
+                                const float4 u = hp[q4], v = hmn[q4];
+                                op[4 * q4 + 0] = fmaf(a, u.x, fmaf(-b, v.x, op[4 * q4 + 0]));
+                                op[4 * q4 + 1] = fmaf(a, u.y, fmaf(-b, v.y, op[4 * q4 + 1]));
+                                op[4 * q4 + 2] = fmaf(a, u.z, fmaf(-b, v.z, op[4 * q4 + 2]));
+                                op[4 * q4 + 3] = fmaf(a, u.w, fmaf(-b, v.w, op[4 * q4 + 3]));
+                                om[4 * q4 + 0] = fmaf(b, u.x, fmaf(a, v.x, om[4 * q4 + 0]));
+                                om[4 * q4 + 1] = fmaf(b, u.y, fmaf(a, v.y, om[4 * q4 + 1]));
+                                om[4 * q4 + 2] = fmaf(b, u.z, fmaf(a, v.z, om[4 * q4 + 2]));
+                                om[4 * q4 + 3] = fmaf(b, u.w, fmaf(a, v.w, om[4 * q4 + 3]));
+                            }
+                        }
+                    }
+                    const int w3 = 2 * l3 + 1;
+                    const float* gi = Gi + (size_t)(l3 * l3) * C + c;
+#pragma unroll
+                    for (int e = 0; e < kTe; ++e) {
+                        float yp = 0.f, ym = 0.f;
+                        if (e < ne) {
+                            const float* D = Dm + e * WS + wig_off(l3);
+                            const float* Ex = Dx + e * WS + wig_off(l3);
+                            const float* Ey = Dy + e * WS + wig_off(l3);
+                            float gp = 0.f, gm = 0.f, xp = 0.f, xm = 0.f, zp = 0.f, zm = 0.f;
+                            for (int n = 0; n < w3; ++n) {
+                                const float gv = gi[(size_t)n * C];
+                                gp = fmaf(D[(l3 + m) * w3 + n], gv, gp);
+                                gm = fmaf(D[(l3 - m) * w3 + n], gv, gm);
+                                xp = fmaf(Ex[(l3 + m) * w3 + n], gv, xp);
+                                xm = fmaf(Ex[(l3 - m) * w3 + n], gv, xm);
+                                zp = fmaf(Ey[(l3 + m) * w3 + n], gv, zp);
+                                zm = fmaf(Ey[(l3 - m) * w3 + n], gv, zm);
+                            }
+                            const float al = alpha[e * H + h];
+                            float bs = gp * op[e], tx = xp * op[e], ty = zp * op[e];
+                            if (m > 0) {
+                                bs = fmaf(gm, om[e], bs);
+                                tx = fmaf(xm, om[e], tx);
+                                ty = fmaf(zm, om[e], ty);
+                            }
+                            atomicAdd(&beta[e * H + h], bs);
+                            atomicAdd(&geo[e * 12 + 10], al * tx);
+                            atomicAdd(&geo[e * 12 + 11], al * ty);
+                            yp = al * gp;
+                            ym = al * gm;
+                        }
+                        gy[(size_t)r * kTe + e] = yp;
+                        if (m > 0) gy[(size_t)(nm + r) * kTe + e] = ym;
+                    }
+                }
+                __syncthreads();
+                // dX~ = F^T(dY) column by column, and what it feeds: dx_j, dg_v, the second direction term
+                const size_t oa = so2_offset(L, C, m, 0), ob = so2_offset(L, C, m, 1);
+                for (int kc = tid; kc < nm; kc += nt) {
+                    const int l1 = m + kc / C, c = kc % C;
+                    float dp[kTe], dq[kTe];
+#pragma unroll
+                    for (int e = 0; e < kTe; ++e) { dp[e] = 0.f; dq[e] = 0.f; }
+                    for (int r = 0; r < nm; ++r) {
+                        const float a = load_feat(W, oa + (size_t)r * nm + kc);
+                        const float4* yp4 = reinterpret_cast<const float4*>(gy + (size_t)r * kTe);
+                        if (m == 0) {
+#pragma unroll
+                            for (int q4 = 0; q4 < kTe / 4; ++q4) {
+                                const float4 v = yp4[q4];
+                                dp[4 * q4 + 0] = fmaf(a, v.x, dp[4 * q4 + 0]);
+                                dp[4 * q4 + 1] = fmaf(a, v.y, dp[4 * q4 + 1]);
+                                dp[4 * q4 + 2] = fmaf(a, v.z, dp[4 * q4 + 2]);
+                                dp[4 * q4 + 3] = fmaf(a, v.w, dp[4 * q4 + 3]);
+                            }
+                        } else {
+                            const float b = load_feat(W, ob + (size_t)r * nm + kc);
+                            const float4* ym4 = reinterpret_cast<const float4*>(gy + (size_t)(nm + r) * kTe);
+#pragma unroll
+                            for (int q4 = 0; q4 < kTe / 4; ++q4) {
+                                const float4 u = yp4[q4], v = ym4[q4];
+                                dp[4 * q4 + 0] = fmaf(a, u.x, fmaf(b, v.x, dp[4 * q4 + 0]));
+                                dp[4 * q4 + 1] = fmaf(a, u.y, fmaf(b, v.y, dp[4 * q4 + 1]));
+                                dp[4 * q4 + 2] = fmaf(a, u.z, fmaf(b, v.z, dp[4 * q4 + 2]));
+                                dp[4 * q4 + 3] = fmaf(a, u.w, fmaf(b, v.w, dp[4 * q4 + 3]));
+                                dq[4 * q4 + 0] = fmaf(-b, u.x, fmaf(a, v.x, dq[4 * q4 + 0]));
+                                dq[4 * q4 + 1] = fmaf(-b, u.y, fmaf(a, v.y, dq[4 * q4 + 1]));
+                                dq[4 * q4 + 2] = fmaf(-b, u.z, fmaf(a, v.z, dq[4 * q4 + 2]));
+                                dq[4 * q4 + 3] = fmaf(-b, u.w, fmaf(a, v.w, dq[4 * q4 + 3]));
+                            }
+                        }
+                    }
+                    const int w1 = 2 * l1 + 1;
+#pragma unroll
+                    for (int e = 0; e < kTe; ++e) {
+                        if (e < ne) {
+                            const float* D = Dm + e * WS + wig_off(l1);
+                            const float* Ex = Dx + e * WS + wig_off(l1);
+                            const float* Ey = Dy + e * WS + wig_off(l1);
+                            const size_t xb = ((size_t)jn[e] * K + l1 * l1) * C + c;
+                            const float gv = g[e * G + l1 * C + c];
+                            float rp = 0.f, rm = 0.f, xp = 0.f, xm = 0.f, zp = 0.f, zm = 0.f;
+                            for (int n = 0; n < w1; ++n) {
+                                const float xv = load_feat(x, xb + (size_t)n * C);
+                                rp = fmaf(D[(l1 + m) * w1 + n], xv, rp);
+                                rm = fmaf(D[(l1 - m) * w1 + n], xv, rm);
+                                xp = fmaf(Ex[(l1 + m) * w1 + n], xv, xp);
+                                xm = fmaf(Ex[(l1 - m) * w1 + n], xv, xm);
+                                zp = fmaf(Ey[(l1 + m) * w1 + n], xv, zp);
+                                zm = fmaf(Ey[(l1 - m) * w1 + n], xv, zm);
+                                float gxv = D[(l1 + m) * w1 + n] * dp[e];
+                                if (m > 0) gxv = fmaf(D[(l1 - m) * w1 + n], dq[e], gxv);
+                                atomicAdd(P.gx + xb + (size_t)n * C, gv * gxv);
+                            }
+                            float dg = dp[e] * rp, tx = dp[e] * xp, ty = dp[e] * zp;
+                            if (m > 0) {
+                                dg = fmaf(dq[e], rm, dg);
+                                tx = fmaf(dq[e], xm, tx);
+                                ty = fmaf(dq[e], zm, ty);
+                            }
+                            dgv[e * Gv + l1 * C + c] += dg;
+                            atomicAdd(&geo[e * 12 + 10], gv * tx);
+                            atomicAdd(&geo[e * 12 + 11], gv * ty);
+                        }
+                    }
+                }
+                __syncthreads();
+            }
+            // value gates -> rho: dLoss/drho_k = sum_c W_rad[k][c] dg_v[c]; dW_rad += rho (x) dg_v
+            for (int pk = warp; pk < kTe * nr; pk += nt / 32) {
+                const int e = pk / nr, kb = pk % nr;
+                float s = 0.f;
+                for (int c = lane; c < Gv; c += 32) s = fmaf(P.Wrad[(size_t)kb * G + c], dgv[e * Gv + c], s);
+                s = warp_sum(s);
+                if (lane == 0) red[pk] = s;
+            }
+            for (int t = tid; t < nr * Gv; t += nt) {
+                const int kb = t / Gv, c = t % Gv;
+                float s = 0.f;
+#pragma unroll
+                for (int e = 0; e < kTe; ++e) s = fmaf(rho[e * nr + kb], dgv[e * Gv + c], s);
+                gWr[(size_t)kb * G + c] += s;
+            }
+            __syncthreads();
+            if (tid < ne) {
+                const int e = tid;
+                const float* gg = geo + e * 12;
+                float dd = 0.f;
+                for (int kb = 0; kb < nr; ++kb) dd = fmaf(rhop[e * nr + kb], red[e * nr + kb], dd);
+                const float id = 1.f / gg[3];
+                const int j = jn[e];
+#pragma unroll
+                for (int c = 0; c < 3; ++c) {
+                    const float dr = dd * gg[c] + (gg[10] * gg[4 + c] + gg[11] * gg[7 + c]) * id;
+                    atomicAdd(P.gpos + 3 * (size_t)j + c, dr);
+                    atomicAdd(gpi + c, -dr);
+                }
+                for (int h = 0; h < H; ++h) {
+                    P.beta[(size_t)(e0 + e) * H + h] = beta[e * H + h];
+                    atomicAdd(dlt + h, alpha[e * H + h] * beta[e * H + h]);
+                }
+            }
+            __syncthreads();
+        }
+        // logit gradient: needs delta_i over all the node's edges
+        {
+            const int h = tid % H;
+            const float* qi = P.q + (size_t)i * C + h * dh;
+            for (int e = tid / H; e < deg; e += nt / H) {
+                const int j = P.col[e_begin + e];
+                float3 u;
+                float d, gap;
+                const Logit lg = edge_logit(P, i, j, h, Gv, G, inv, &u, &d, &gap);
+                const float al = expf(lg.a - lse_s[h]);
+                const float da = al * (P.beta[(size_t)(e_begin + e) * H + h] - dlt[h]);
+                const float dga = da * lg.dot * inv, ds = da * lg.ga * inv;
+                const float* kj = P.k + (size_t)j * C + h * dh;
+                for (int c = 0; c < dh; ++c) {
+                    atomicAdd(gqi + h * dh + c, ds * kj[c]);
+                    atomicAdd(P.gk + (size_t)j * C + h * dh + c, ds * qi[c]);
+                }
+                for (int kb = 0; kb < nr; ++kb) {
+                    float v, dv;
+                    rbf_and_deriv(d, kb, P.cutoff, nr, v, dv);
+                    atomicAdd(gWr + (size_t)kb * G + Gv + h, v * dga);
+                }
+                const float dd = dga * gap;
+                atomicAdd(P.gpos + 3 * (size_t)j + 0, dd * u.x);
+                atomicAdd(P.gpos + 3 * (size_t)j + 1, dd * u.y);
+                atomicAdd(P.gpos + 3 * (size_t)j + 2, dd * u.z);
+                atomicAdd(gpi + 0, -dd * u.x);
+                atomicAdd(gpi + 1, -dd * u.y);
+                atomicAdd(gpi + 2, -dd * u.z);
+            }
+        }
+        __syncthreads();
+        for (int c = tid; c < C; c += nt) P.gq[(size_t)i * C + c] = gqi[c];
+        if (tid < 3) atomicAdd(P.gpos + 3 * (size_t)i + tid, gpi[tid]);
+    }
+    __syncthreads();
+    for (int t = tid; t < nr * G; t += nt) atomicAdd(P.gWrad + t, gWr[t]);
+}
+
+// dW_so2 = sum over edges of dY (x) X~, one 64 x 64 tile of one |m| block per
+// CTA (A and B tiles together for m >= 1):
+//   dA += dY+ X~+^T + dY- X~-^T,   dB += dY- X~+^T - dY+ X~-^T
+// with dY(l3, +-m, c) = alpha^{head c} sum_n D^l3[+-m][n] G_i[l3, n, c] and
+// X~(l1, +-m, c) = g_v[l1, c] sum_n D^l1[+-m][n] x_j[l1, n, c], rebuilt per
+// edge from the geometry (no per-edge storage). Edges are visited in CSR
+// order in chunks of 256 (one thread per edge for the frame and weights).
+__device__ __forceinline__ int drow_off(int m, int l, int s) {
+    // rows (l+m) and (l-m) of D^l for l = m..L, stored per edge back to back
+    const int nrow = (m == 0) ? 1 : 2;
+    int o = 0;
+    for (int k = m; k < l; ++k) o += nrow * (2 * k + 1);
+    return o + s * (2 * l + 1);
+}
+
+size_t dw_smem_floats(int L, int H, int n_rbf) {
+    (void)L;
+    return (size_t)kDwChunk * 50 + (size_t)kDwChunk * n_rbf + (size_t)kDwChunk * H + 2 * kDwChunk +
+           4ull * kDwE * kDwT;
+}
+
+template <int L, typename T>
+__global__ void __launch_bounds__(kNt) k_bwd_dw(BwdParams P) {
+    constexpr int K = n_sh(L);
+    constexpr int WS = wig_size(L);
+    const int C = P.C, H = P.H, dh = C / H, nr = P.n_rbf;
+    const int Gv = (L + 1) * C, G = Gv + H;
+    const T* __restrict__ x = static_cast<const T*>(P.x);
+    // this CTA's tile: blocks m = 0..M in order, tiles of a block row-major
+    int m = 0, nm = (L + 1) * C, side = (nm + kDwT - 1) / kDwT, b = blockIdx.x;
+    while (b >= side * side && m < P.M) {
+        b -= side * side;
+        ++m;
+        nm = (L + 1 - m) * C;
+        side = (nm + kDwT - 1) / kDwT;
+    }
+    const int r0 = (b / side) * kDwT, k0 = (b % side) * kDwT;
+    const int nrow = (m == 0) ? 1 : 2;
+
+    extern __shared__ float sm[];
+    float* drow = sm;                          // [chunk][50]
+    float* rho = drow + kDwChunk * 50;         // [chunk][nr]
+    float* alpha = rho + kDwChunk * nr;        // [chunk][H]
+    int* ei = reinterpret_cast<int*>(alpha + kDwChunk * H);  // [chunk] node i
+    int* ej = ei + kDwChunk;                   // [chunk] neighbour j
+    float* Yop = reinterpret_cast<float*>(ej + kDwChunk);    // [2][kDwE][kDwT] dY rows of the tile
+    float* Xop = Yop + 2 * kDwE * kDwT;        // [2][kDwE][kDwT] X~ columns of the tile
+
+    const int tid = threadIdx.x, ty = tid / 16, tx = tid % 16;
+    const float inv = rsqrtf((float)dh);
+    float accA[4][4], accB[4][4];
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) { accA[a][b] = 0.f; accB[a][b] = 0.f; }
+
+    for (int c0 = 0; c0 < P.n_pairs; c0 += kDwChunk) {
+        const int nc = min(kDwChunk, P.n_pairs - c0);
+        __syncthreads();
+        if (tid < nc) {
+            const int e = c0 + tid;
+            int lo = 0, hi = P.n_atoms - 1;  // node i: last n with row_ptr[n] <= e
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                if (P.row_ptr[mid] <= e) lo = mid; else hi = mid - 1;
+            }
+            const int i = lo, j = P.col[e];
+            ei[tid] = i;
+            ej[tid] = j;
+            const float3 r = edge_vec(P.pos, i, j, P.box);
+            const float d = sqrtf(r.x * r.x + r.y * r.y + r.z * r.z);
+            float R[3][3];
+            edge_frame(r.x / d, r.y / d, r.z / d, R);
+            float D[WS];
+            wigner_blocks<L>(R, D);
+            float* dr = drow + tid * 50;
+            for (int l = m; l <= L; ++l) {
+                const int w = 2 * l + 1;
+                for (int s = 0; s < nrow; ++s) {
+                    const int row = s == 0 ? l + m : l - m;
+                    for (int n = 0; n < w; ++n) dr[drow_off(m, l, s) + n] = D[wig_off(l) + row * w + n];
+                }
+            }
+            for (int kb = 0; kb < nr; ++kb) rho[tid * nr + kb] = rbf(d, kb, P.cutoff, nr);
+            for (int h = 0; h < H; ++h) {
+                float ga = 0.f;
+                for (int kb = 0; kb < nr; ++kb) ga = fmaf(rho[tid * nr + kb], P.Wrad[(size_t)kb * G + Gv + h], ga);
+                const float* qi = P.q + (size_t)i * C + h * dh;
+                const float* kj = P.k + (size_t)j * C + h * dh;
+                float dot = 0.f;
+                for (int c = 0; c < dh; ++c) dot = fmaf(qi[c], kj[c], dot);
+                alpha[tid * H + h] = expf(ga * dot * inv - P.lse[(size_t)i * H + h]);
+            }
+        }
+        __syncthreads();
+        for (int s0 = 0; s0 < nc; s0 += kDwE) {
+            const int ns = min(kDwE, nc - s0);
+            // operands of the sub-chunk: dY rows r0.., X~ columns k0..
+            for (int t = tid; t < 2 * kDwE * kDwT; t += kNt) {
+                const int s = t / (kDwE * kDwT), rem = t % (kDwE * kDwT);
+                const int e = rem / kDwT, q = rem % kDwT;
+                float vy = 0.f, vx = 0.f;
+                if (e < ns && s < nrow) {
+                    const int el = s0 + e;
+                    const int ry = r0 + q, kx = k0 + q;
+                    if (ry < nm) {
+                        const int l3 = m + ry / C, c = ry % C, w = 2 * l3 + 1;
+                        const float* dr = drow + el * 50 + drow_off(m, l3, s);
+                        const float* gi = P.G + ((size_t)ei[el] * K + l3 * l3) * C + c;
+                        float acc = 0.f;
+                        for (int n = 0; n < w; ++n) acc = fmaf(dr[n], gi[(size_t)n * C], acc);
+                        vy = alpha[el * H + c / dh] * acc;
+                    }
+                    if (kx < nm) {
+                        const int l1 = m + kx / C, c = kx % C, w = 2 * l1 + 1;
+                        const float* dr = drow + el * 50 + drow_off(m, l1, s);
+                        const size_t xb = ((size_t)ej[el] * K + l1 * l1) * C + c;
+                        float acc = 0.f;
+                        for (int n = 0; n < w; ++n) acc = fmaf(dr[n], load_feat(x, xb + (size_t)n * C), acc);
+                        float gv = 0.f;
+                        for (int kb = 0; kb < nr; ++kb) gv = fmaf(rho[el * nr + kb], P.Wrad[(size_t)kb * G + l1 * C + c], gv);
+                        vx = gv * acc;
+                    }
+                }
+                Yop[t] = vy;
+                Xop[t] = vx;
+            }
+            __syncthreads();
+            for (int e = 0; e < ns; ++e) {
+                const float4 yp = *reinterpret_cast<const float4*>(Yop + e * kDwT + ty * 4);
+                const float4 xp = *reinterpret_cast<const float4*>(Xop + e * kDwT + tx * 4);
+                const float ypa[4] = {yp.x, yp.y, yp.z, yp.w}, xpa[4] = {xp.x, xp.y, xp.z, xp.w};
+                if (m == 0) {
+#pragma unroll
+                    for (int a = 0; a < 4; ++a)
+#pragma unroll
+                        for (int b = 0; b < 4; ++b) accA[a][b] = fmaf(ypa[a], xpa[b], accA[a][b]);
+                } else {
+                    const float4 ym = *reinterpret_cast<const float4*>(Yop + (kDwE + e) * kDwT + ty * 4);
+                    const float4 xm = *reinterpret_cast<const float4*>(Xop + (kDwE + e) * kDwT + tx * 4);
+                    const float yma[4] = {ym.x, ym.y, ym.z, ym.w}, xma[4] = {xm.x, xm.y, xm.z, xm.w};
+#pragma unroll
+                    for (int a = 0; a < 4; ++a)
+#pragma unroll
+                        for (int b = 0; b < 4; ++b) {
+                            accA[a][b] = fmaf(ypa[a], xpa[b], fmaf(yma[a], xma[b], accA[a][b]));
+                            accB[a][b] = fmaf(yma[a], xpa[b], fmaf(-ypa[a], xma[b], accB[a][b]));
+                        }
+                }
+            }
+            __syncthreads();
+        }
+    }
+    const size_t oa = so2_offset(L, C, m, 0), ob = so2_offset(L, C, m, 1);
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+        const int r = r0 + ty * 4 + a;
+        if (r >= nm) continue;
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+            const int kx = k0 + tx * 4 + b;
+            if (kx >= nm) continue;
+            P.gW[oa + (size_t)r * nm + kx] = accA[a][b];
+            if (m > 0) P.gW[ob + (size_t)r * nm + kx] = accB[a][b];
+        }
+    }
+}
+
+// dW_q = sum_i dq_i (x) x_i[l=0], dW_k likewise (q = W_q x[l=0]); one thread per weight
+template <typename T>
+__global__ void k_bwd_wqk(const T* __restrict__ x, int n, int K, int C, const float* __restrict__ gq,
+                          const float* __restrict__ gk, float* gWq, float* gWk) {
+    const int t = blockIdx.x * blockDim.x + threadIdx.x;
+    if (t >= C * C) return;
+    const int o = t / C, c = t % C;
+    float sq = 0.f, sk = 0.f;
+    for (int i = 0; i < n; ++i) {
+        const float xv = load_feat(x, (size_t)i * K * C + c);
+        sq = fmaf(gq[(size_t)i * C + o], xv, sq);
+        sk = fmaf(gk[(size_t)i * C + o], xv, sk);
+    }
+    if (gWq) gWq[t] = sq;
+    if (gWk) gWk[t] = sk;
+}
+
+// dx[i, l=0, c] += sum_o W_q[o][c] dq_i[o] + W_k[o][c] dk_i[o]
+__global__ void k_bwd_x0(int n, int K, int C, const float* __restrict__ Wq, const float* __restrict__ Wk,
+                         const float* __restrict__ gq, const float* __restrict__ gk, float* gx) {
+    const int t = blockIdx.x * blockDim.x + threadIdx.x;
+    if (t >= n * C) return;
+    const int i = t / C, c = t % C;
+    float s = 0.f;
+    for (int o = 0; o < C; ++o) {
+        s = fmaf(Wq[(size_t)o * C + c], gq[(size_t)i * C + o], s);
+        s = fmaf(Wk[(size_t)o * C + c], gk[(size_t)i * C + o], s);
+    }
+    gx[(size_t)i * K * C + c] += s;
+}
+
+template <int L, typename T>
+cudaError_t launch_node(const BwdParams& P, size_t smem, int grid, cudaStream_t s) {
+    cudaError_t e = cudaFuncSetAttribute(k_bwd_node<L, T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    count_launch();
+    k_bwd_node<L, T><<<grid, kNt, smem, s>>>(P);
+    return cudaGetLastError();
+}
+
+template <int L, typename T>
+cudaError_t launch_dw(const BwdParams& P, int n_tiles, size_t smem, cudaStream_t s) {
+    cudaError_t e = cudaFuncSetAttribute(k_bwd_dw<L, T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    count_launch();
+    k_bwd_dw<L, T><<<n_tiles, kNt, smem, s>>>(P);
+    return cudaGetLastError();
+}
+
+int n_dw_tiles(int L, int C, int M) {
+    int n = 0;
+    for (int m = 0; m <= M; ++m) {
+        const int t = ((L + 1 - m) * C + kDwT - 1) / kDwT;
+        n += t * t;
+    }
+    return n;
+}
+
+}  // namespace bwd
+
+bool bwd_supported(int L, int C, int H, int n_rbf) {
+    if (L < 0 || L > kMaxL || bwd::kNt % H != 0) return false;
+    return bwd::node_smem_floats(L, C, H, n_rbf) * 4 <= 227 * 1024 &&
+           bwd::dw_smem_floats(L, H, n_rbf) * 4 <= 227 * 1024;
+}
+
+cudaError_t run_attention_bwd(const BwdArgs& b, cudaStream_t s) {
+    using namespace bwd;
+    const AttnArgs& a = b.fwd;
+    const int L = a.L, C = a.C, H = a.H, K = n_sh(L), N = a.n_atoms;
+    const int G = (L + 1) * C + H;
+    cudaError_t e;
+    E2F_CUDA_TRY_E(qk_project(a.x, a.bf16, N, K, C, a.Wq, a.Wk, a.q, a.k, s));
+    E2F_CUDA_TRY_E(repack_so2_f32(a.Wso2, a.bf16, L, C, a.M, a.Wt, s));
+    E2F_CUDA_TRY_E(cudaMemsetAsync(b.gpos, 0, 12 * (size_t)N, s));
+    E2F_CUDA_TRY_E(cudaMemsetAsync(b.gx, 0, 4 * (size_t)N * K * C, s));
+    E2F_CUDA_TRY_E(cudaMemsetAsync(b.gk, 0, 4 * (size_t)N * C, s));
+    E2F_CUDA_TRY_E(cudaMemsetAsync(b.gWrad, 0, 4 * (size_t)a.n_rbf * G, s));
+
+    BwdParams P{};
+    P.n_atoms = N; P.C = C; P.H = H; P.n_rbf = a.n_rbf; P.M = a.M; P.n_pairs = (int)a.n_pairs;
+    P.cutoff = a.cutoff; P.box = a.box; P.pos = a.pos; P.row_ptr = a.row_ptr; P.col = a.col; P.x = a.x;
+    P.W = a.Wso2; P.Wt = a.Wt; P.Wrad = a.Wrad; P.q = a.q; P.k = a.k; P.G = b.grad_out;
+    P.lse = b.lse; P.beta = b.beta; P.gq = b.gq; P.gk = b.gk; P.gpos = b.gpos; P.gx = b.gx; P.gWrad = b.gWrad;
+    P.gW = b.gWso2;
+
+    int dev = 0, n_sm = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
+    const size_t smem = node_smem_floats(L, C, H, a.n_rbf) * 4;
+    const int grid = std::max(1, std::min(N, n_sm));
+#define E2F_BWD_NODE(LL)                                                                                     \
+    case LL:                                                                                                 \
+        e = a.bf16 ? launch_node<LL, __nv_bfloat16>(P, smem, grid, s) : launch_node<LL, float>(P, smem, grid, s); \
+        break;
+    switch (L) {
+        E2F_BWD_NODE(0)
+        E2F_BWD_NODE(1)
+        E2F_BWD_NODE(2)
+        E2F_BWD_NODE(3)
+        E2F_BWD_NODE(4)
+        default: return cudaErrorInvalidValue;
+    }
+#undef E2F_BWD_NODE
+    if (e != cudaSuccess) return e;
+    if (b.gWq || b.gWk) {
+        count_launch();
+        if (a.bf16)
+            k_bwd_wqk<__nv_bfloat16><<<(C * C + 255) / 256, 256, 0, s>>>(
+                static_cast<const __nv_bfloat16*>(a.x), N, K, C, b.gq, b.gk, b.gWq, b.gWk);
+        else
+            k_bwd_wqk<float><<<(C * C + 255) / 256, 256, 0, s>>>(static_cast<const float*>(a.x), N, K, C, b.gq,
+                                                                 b.gk, b.gWq, b.gWk);
+        E2F_CUDA_TRY_E(cudaGetLastError());
+    }
+    count_launch();
+    k_bwd_x0<<<(N * C + 255) / 256, 256, 0, s>>>(N, K, C, a.Wq, a.Wk, b.gq, b.gk, b.gx);
+    E2F_CUDA_TRY_E(cudaGetLastError());
+    if (b.gWso2 && a.n_pairs > 0) {
+        const int nt = n_dw_tiles(L, C, a.M);
+        const size_t dsm = dw_smem_floats(L, H, a.n_rbf) * 4;
+#define E2F_BWD_DW(LL)                                                                                         \
+    case LL:                                                                                                   \
+        e = a.bf16 ? launch_dw<LL, __nv_bfloat16>(P, nt, dsm, s) : launch_dw<LL, float>(P, nt, dsm, s); \
+        break;
+        switch (L) {
+            E2F_BWD_DW(0)
+            E2F_BWD_DW(1)
+            E2F_BWD_DW(2)
+            E2F_BWD_DW(3)
+            E2F_BWD_DW(4)
+            default: return cudaErrorInvalidValue;
+        }
+#undef E2F_BWD_DW
+        if (e != cudaSuccess) return e;
+    } else if (b.gWso2) {
+        E2F_CUDA_TRY_E(cudaMemsetAsync(b.gWso2, 0, 4 * so2_total(L, C, a.M), s));
+    }
+    return cudaSuccess;
+}
+
+}  // namespace e2f

@@ -327,6 +327,26 @@ cudaError_t run_attention_simt(const AttnArgs& a, cudaStream_t s) {
 #undef E2F_SIMT_CASE
 }
 
+cudaError_t qk_project(const void* x, bool bf16, int n_atoms, int K, int C, const float* Wq, const float* Wk,
+                       float* q, float* k, cudaStream_t s) {
+    count_launch();
+    if (bf16)
+        k_qk_project<__nv_bfloat16><<<n_atoms, 128, C * 4, s>>>(static_cast<const __nv_bfloat16*>(x), n_atoms, K, C,
+                                                                Wq, Wk, q, k);
+    else
+        k_qk_project<float><<<n_atoms, 128, C * 4, s>>>(static_cast<const float*>(x), n_atoms, K, C, Wq, Wk, q, k);
+    return cudaGetLastError();
+}
+
+cudaError_t repack_so2_f32(const void* w, bool bf16, int L, int C, int M, float* out, cudaStream_t s) {
+    count_launch();
+    if (bf16)
+        k_repack_so2_f32<__nv_bfloat16><<<1184, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(w), L, C, M, out);
+    else
+        k_repack_so2_f32<float><<<1184, 256, 0, s>>>(static_cast<const float*>(w), L, C, M, out);
+    return cudaGetLastError();
+}
+
 // Wigner blocks for a batch of directions (exposed for testing the rotation)
 template <int L>
 __global__ void k_edge_wigner(const float* r, int64_t n, float* out, float* frames) {

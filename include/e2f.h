@@ -255,6 +255,54 @@ e2f_status e2f_onfly_attention_cells(const e2f_attn_cfg* cfg, const float* pos,
                                      void* workspace, size_t ws_bytes,
                                      void* stream);
 
+/* ------------------------------------------------------------------------
+ * Backward of the on-the-fly equivariant attention: the gradients of a
+ * scalar loss with respect to every input of e2f_onfly_attention, given
+ * grad_out = dLoss/dout. The pages' conservative variant takes forces as
+ * the negative position gradient of the energy (gist.science Technical
+ * Summary 2.2; the molecular-dynamics experiments), which this provides
+ * (grad_pos); the weight gradients serve training. The pages print no
+ * backward formulas: the call differentiates exactly the layer documented
+ * above (same neighbour list, periodic image shifts held fixed) and
+ * recomputes every per-edge quantity on chip, as the forward does; the
+ * only O(E) scratch is one float per edge and head.
+ *
+ *   Arguments cfg .. W_so2 as for e2f_onfly_attention (same CSR, which
+ *   need not be symmetric).
+ *   grad_out    device, float [N, (L+1)^2, C].
+ *   grad_pos    device, float [N*3], written.
+ *   grad_x      device, float [N, (L+1)^2, C], written (fp32 for either
+ *               feat_dtype).
+ *   grad_W_q, grad_W_k   device, float [C, C], written; either may be
+ *               NULL (not computed).
+ *   grad_W_rad  device, float [n_rbf, (L+1)C + H], written.
+ *   grad_W_so2  device, float, packed like W_so2 (truncation included),
+ *               written; NULL skips it (its kernel is the costliest part:
+ *               a sweep over all edges per 64 x 64 tile of the SO(2) blocks).
+ *   workspace   device, >= e2f_attention_backward_workspace_size(...)
+ *               bytes, 256-byte aligned.
+ * All arithmetic is fp32 on CUDA cores (a tensor-core backward is not
+ * built). Gradients that sum over edges use fp32 atomics, so their last
+ * bits may differ between runs; grad_W_so2, grad_W_q and grad_W_k are
+ * deterministic. Shapes: those of e2f_onfly_attention with H dividing 256
+ * and the kernels' shared memory within 227 KB (L = 4 allows C <= 128);
+ * otherwise E2F_ERR_UNSUPPORTED. Asynchronous.
+ * ---------------------------------------------------------------------- */
+size_t e2f_attention_backward_workspace_size(int64_t n_atoms, int64_t n_pairs,
+                                             const e2f_attn_cfg* cfg);
+
+e2f_status e2f_onfly_attention_backward(const e2f_attn_cfg* cfg, const float* pos,
+                                        int64_t n_atoms, const float* box_host,
+                                        const int32_t* row_ptr, const int32_t* col,
+                                        int64_t n_pairs, const void* x,
+                                        const float* W_q, const float* W_k,
+                                        const float* W_rad, const void* W_so2,
+                                        const float* grad_out, float* grad_pos,
+                                        float* grad_x, float* grad_W_q,
+                                        float* grad_W_k, float* grad_W_rad,
+                                        float* grad_W_so2, void* workspace,
+                                        size_t ws_bytes, void* stream);
+
 /* Synchronises `stream` and returns the device status recorded by the last
  * e2f_onfly_attention call on this workspace (E2F_OK or E2F_ERR_TIMEOUT);
  * each call clears the word when it starts. */
