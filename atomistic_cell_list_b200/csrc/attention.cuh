@@ -79,8 +79,10 @@ struct BwdArgs {
     float* gWk;
     float* gWrad;
     float* gWso2;
+    float* gWpart;  // bwd_partial_bytes(L, C, M) of scratch for gWso2
 };
 bool bwd_supported(int L, int C, int H, int n_rbf);
+size_t bwd_partial_bytes(int L, int C, int M);
 cudaError_t run_attention_bwd(const BwdArgs& b, cudaStream_t s);
 struct CellLists;
 // cl != nullptr: fused traversal (a.row_ptr = per-slot offsets in cell order, a.col unused)

@@ -47,6 +47,7 @@ constexpr int kTe = 8;       // edges per tile of the node kernel
 constexpr int kDwT = 64;     // weight-gradient tile side
 constexpr int kDwE = 32;     // edges per operand sub-chunk of the weight-gradient kernel
 constexpr int kDwChunk = 256;  // edges per geometry chunk (one per thread)
+constexpr int kDwSplit = 4;    // edge ranges per tile (partial sums added in a fixed order)
 
 struct BwdParams {
     int n_atoms, C, H, n_rbf, M;
@@ -71,6 +72,8 @@ struct BwdParams {
     float* gx;         // [N, K, C]
     float* gWrad;      // [n_rbf, G]
     float* gW;         // packed like W
+    float* gWpart;     // [kDwSplit][so2 total] partial sums of gW
+    int dw_tiles;      // tiles of the SO(2) blocks
 };
 
 // Derivative of the Wigner blocks along dR (R -> R + eps dR): the recursion
@@ -154,7 +157,7 @@ size_t node_smem_floats(int L, int C, int H, int n_rbf) {
     const int K = n_sh(L), WS = wig_size(L), Gv = (L + 1) * C, G = Gv + H;
     const int KH = (L >= 1) ? std::max((L + 1) * C, 2 * L * C) : C;
     return (size_t)K * C + 3ull * kTe * WS + 2ull * kTe * n_rbf + (size_t)kTe * G + (size_t)kTe * Gv +
-           2ull * kTe * H + 12ull * kTe + 2ull * KH * kTe + (size_t)n_rbf * G + C + 2ull * H + 4 + kTe +
+           2ull * kTe * H + 12ull * kTe + 3ull * KH * kTe + (size_t)n_rbf * G + C + 2ull * H + 4 + kTe +
            2ull * kNt + kTe;
 }
 
@@ -162,7 +165,7 @@ size_t node_smem_floats(int L, int C, int H, int n_rbf) {
 // gradient except dW_so2, dW_q, dW_k and the l = 0 part of dx that flows
 // through q and k.
 template <int L, typename T>
-__global__ void __launch_bounds__(kNt) k_bwd_node(BwdParams P) {
+__global__ void __launch_bounds__(kNt, 1) k_bwd_node(BwdParams P) {
     constexpr int K = n_sh(L);
     constexpr int WS = wig_size(L);
     const int C = P.C, H = P.H, dh = C / H, nr = P.n_rbf, M = P.M;
@@ -184,8 +187,9 @@ __global__ void __launch_bounds__(kNt) k_bwd_node(BwdParams P) {
     float* beta = alpha + kTe * H;     // [te][H]
     float* geo = beta + kTe * H;       // [te][12]: r^ (3), d, R^T e_y (3), -R^T e_x (3), dL/deps_x, dL/deps_y
     float* hs = geo + 12 * kTe;        // [KH][te] gated rotated input of the |m| block
-    float* gy = hs + KH * kTe;         // [KH][te] dLoss/dY of the block
-    float* gWr = gy + KH * kTe;        // [nr][G] this CTA's part of dW_rad
+    float* gy = hs + KH * kTe;         // [KH][te] D G_i, then dLoss/dY = alpha D G_i, of the block
+    float* yb = gy + KH * kTe;         // [KH][te] Y = F(X~) of the block
+    float* gWr = yb + KH * kTe;        // [nr][G] this CTA's part of dW_rad
     float* gqi = gWr + nr * G;         // [C]
     float* lse_s = gqi + C;            // [H]
     float* dlt = lse_s + H;            // [H] delta_i
@@ -321,7 +325,7 @@ __global__ void __launch_bounds__(kNt) k_bwd_node(BwdParams P) {
                 const float* At = P.Wt + so2_offset(L, C, m, 0);
                 const float* Bt = (m > 0) ? P.Wt + so2_offset(L, C, m, 1) : nullptr;
                 for (int r = tid; r < nm; r += nt) {
-                    const int l3 = m + r / C, c = r % C, h = c / dh;
+                    const int l3 = m + r / C, c = r % C;
                     float op[kTe], om[kTe];
 #pragma unroll
                     for (int e = 0; e < kTe; ++e) { op[e] = 0.f; om[e] = 0.f; }
@@ -358,41 +362,81 @@ __global__ void __launch_bounds__(kNt) k_bwd_node(BwdParams P) {
                     const float* gi = Gi + (size_t)(l3 * l3) * C + c;
 #pragma unroll
                     for (int e = 0; e < kTe; ++e) {
-                        float yp = 0.f, ym = 0.f;
+                        float gp = 0.f, gm = 0.f;
                         if (e < ne) {
                             const float* D = Dm + e * WS + wig_off(l3);
-                            const float* Ex = Dx + e * WS + wig_off(l3);
-                            const float* Ey = Dy + e * WS + wig_off(l3);
-                            float gp = 0.f, gm = 0.f, xp = 0.f, xm = 0.f, zp = 0.f, zm = 0.f;
                             for (int n = 0; n < w3; ++n) {
                                 const float gv = gi[(size_t)n * C];
                                 gp = fmaf(D[(l3 + m) * w3 + n], gv, gp);
                                 gm = fmaf(D[(l3 - m) * w3 + n], gv, gm);
-                                xp = fmaf(Ex[(l3 + m) * w3 + n], gv, xp);
-                                xm = fmaf(Ex[(l3 - m) * w3 + n], gv, xm);
-                                zp = fmaf(Ey[(l3 + m) * w3 + n], gv, zp);
-                                zm = fmaf(Ey[(l3 - m) * w3 + n], gv, zm);
                             }
-                            const float al = alpha[e * H + h];
-                            float bs = gp * op[e], tx = xp * op[e], ty = zp * op[e];
-                            if (m > 0) {
-                                bs = fmaf(gm, om[e], bs);
-                                tx = fmaf(xm, om[e], tx);
-                                ty = fmaf(zm, om[e], ty);
-                            }
-                            atomicAdd(&beta[e * H + h], bs);
-                            atomicAdd(&geo[e * 12 + 10], al * tx);
-                            atomicAdd(&geo[e * 12 + 11], al * ty);
-                            yp = al * gp;
-                            ym = al * gm;
                         }
-                        gy[(size_t)r * kTe + e] = yp;
-                        if (m > 0) gy[(size_t)(nm + r) * kTe + e] = ym;
+                        gy[(size_t)r * kTe + e] = gp;
+                        yb[(size_t)r * kTe + e] = op[e];
+                        if (m > 0) {
+                            gy[(size_t)(nm + r) * kTe + e] = gm;
+                            yb[(size_t)(nm + r) * kTe + e] = om[e];
+                        }
                     }
+                }
+                __syncthreads();
+                // beta^h = <D G_i, Y> over the head's rows, and the first direction term
+                // alpha <dD_a G_i, Y>: one warp per (edge, head), lanes over the rows
+                const int rows_h = (L + 1 - m) * dh;
+                for (int task = warp; task < ne * H; task += nt / 32) {
+                    const int e = task / H, h = task % H;
+                    const float* Ex = Dx + e * WS;
+                    const float* Ey = Dy + e * WS;
+                    float bs = 0.f, tx = 0.f, ty = 0.f;
+                    for (int q = lane; q < rows_h; q += 32) {
+                        const int l3 = m + q / dh, c = h * dh + q % dh, w3 = 2 * l3 + 1;
+                        const int r = (l3 - m) * C + c;
+                        const float* gi = Gi + (size_t)(l3 * l3) * C + c;
+                        const int op_ = wig_off(l3) + (l3 + m) * w3, om_ = wig_off(l3) + (l3 - m) * w3;
+                        float xp = 0.f, xm = 0.f, zp = 0.f, zm = 0.f;
+                        for (int n = 0; n < w3; ++n) {
+                            const float gv = gi[(size_t)n * C];
+                            xp = fmaf(Ex[op_ + n], gv, xp);
+                            zp = fmaf(Ey[op_ + n], gv, zp);
+                            if (m > 0) {
+                                xm = fmaf(Ex[om_ + n], gv, xm);
+                                zm = fmaf(Ey[om_ + n], gv, zm);
+                            }
+                        }
+                        const float yp = yb[(size_t)r * kTe + e];
+                        bs = fmaf(gy[(size_t)r * kTe + e], yp, bs);
+                        tx = fmaf(xp, yp, tx);
+                        ty = fmaf(zp, yp, ty);
+                        if (m > 0) {
+                            const float ym = yb[(size_t)(nm + r) * kTe + e];
+                            bs = fmaf(gy[(size_t)(nm + r) * kTe + e], ym, bs);
+                            tx = fmaf(xm, ym, tx);
+                            ty = fmaf(zm, ym, ty);
+                        }
+                    }
+                    bs = warp_sum(bs);
+                    tx = warp_sum(tx);
+                    ty = warp_sum(ty);
+                    if (lane == 0) {
+                        const float al = alpha[e * H + h];
+                        beta[e * H + h] += bs;
+                        atomicAdd(&geo[e * 12 + 10], al * tx);
+                        atomicAdd(&geo[e * 12 + 11], al * ty);
+                    }
+                }
+                __syncthreads();
+                // dY = alpha D G_i
+                for (int t = tid; t < (m > 0 ? 2 : 1) * nm * kTe; t += nt) {
+                    const int rr = t / kTe, e = t % kTe;
+                    const int c = (rr % nm) % C;
+                    gy[t] *= alpha[e * H + c / dh];
                 }
                 __syncthreads();
                 // dX~ = F^T(dY) column by column, and what it feeds: dx_j, dg_v, the second direction term
                 const size_t oa = so2_offset(L, C, m, 0), ob = so2_offset(L, C, m, 1);
+                float t2x[kTe], t2y[kTe];
+#pragma unroll
+                for (int e = 0; e < kTe; ++e) { t2x[e] = 0.f; t2y[e] = 0.f; }
                 for (int kc = tid; kc < nm; kc += nt) {
                     const int l1 = m + kc / C, c = kc % C;
                     float dp[kTe], dq[kTe];
@@ -456,9 +500,17 @@ __global__ void __launch_bounds__(kNt) k_bwd_node(BwdParams P) {
                                 ty = fmaf(dq[e], zm, ty);
                             }
                             dgv[e * Gv + l1 * C + c] += dg;
-                            atomicAdd(&geo[e * 12 + 10], gv * tx);
-                            atomicAdd(&geo[e * 12 + 11], gv * ty);
+                            t2x[e] = fmaf(gv, tx, t2x[e]);
+                            t2y[e] = fmaf(gv, ty, t2y[e]);
                         }
+                    }
+                }
+#pragma unroll
+                for (int e = 0; e < kTe; ++e) {
+                    const float sx = warp_sum(t2x[e]), sy = warp_sum(t2y[e]);
+                    if (lane == 0 && e < ne) {
+                        atomicAdd(&geo[e * 12 + 10], sx);
+                        atomicAdd(&geo[e * 12 + 11], sy);
                     }
                 }
                 __syncthreads();
@@ -553,10 +605,12 @@ __device__ __forceinline__ int drow_off(int m, int l, int s) {
     return o + s * (2 * l + 1);
 }
 
+size_t dw_part_floats(int L, int C, int M) { return (size_t)kDwSplit * so2_total(L, C, M); }
+
 size_t dw_smem_floats(int L, int H, int n_rbf) {
     (void)L;
     return (size_t)kDwChunk * 50 + (size_t)kDwChunk * n_rbf + (size_t)kDwChunk * H + 2 * kDwChunk +
-           4ull * kDwE * kDwT;
+           4ull * kDwE * kDwT + (size_t)n_rbf * kDwT;
 }
 
 template <int L, typename T>
@@ -566,8 +620,9 @@ __global__ void __launch_bounds__(kNt) k_bwd_dw(BwdParams P) {
     const int C = P.C, H = P.H, dh = C / H, nr = P.n_rbf;
     const int Gv = (L + 1) * C, G = Gv + H;
     const T* __restrict__ x = static_cast<const T*>(P.x);
-    // this CTA's tile: blocks m = 0..M in order, tiles of a block row-major
-    int m = 0, nm = (L + 1) * C, side = (nm + kDwT - 1) / kDwT, b = blockIdx.x;
+    // this CTA's tile (blocks m = 0..M in order, tiles of a block row-major) and edge range
+    const int split = blockIdx.x / P.dw_tiles;
+    int m = 0, nm = (L + 1) * C, side = (nm + kDwT - 1) / kDwT, b = blockIdx.x % P.dw_tiles;
     while (b >= side * side && m < P.M) {
         b -= side * side;
         ++m;
@@ -585,6 +640,7 @@ __global__ void __launch_bounds__(kNt) k_bwd_dw(BwdParams P) {
     int* ej = ei + kDwChunk;                   // [chunk] neighbour j
     float* Yop = reinterpret_cast<float*>(ej + kDwChunk);    // [2][kDwE][kDwT] dY rows of the tile
     float* Xop = Yop + 2 * kDwE * kDwT;        // [2][kDwE][kDwT] X~ columns of the tile
+    float* wr = Xop + 2 * kDwE * kDwT;         // [nr][kDwT] W_rad columns of the tile's X~ columns
 
     const int tid = threadIdx.x, ty = tid / 16, tx = tid % 16;
     const float inv = rsqrtf((float)dh);
@@ -594,8 +650,14 @@ __global__ void __launch_bounds__(kNt) k_bwd_dw(BwdParams P) {
 #pragma unroll
         for (int b = 0; b < 4; ++b) { accA[a][b] = 0.f; accB[a][b] = 0.f; }
 
-    for (int c0 = 0; c0 < P.n_pairs; c0 += kDwChunk) {
-        const int nc = min(kDwChunk, P.n_pairs - c0);
+    for (int t = tid; t < nr * kDwT; t += kNt) {
+        const int kb = t / kDwT, kx = k0 + t % kDwT;
+        wr[t] = (kx < nm) ? P.Wrad[(size_t)kb * G + (m + kx / C) * C + kx % C] : 0.f;
+    }
+    const int e_lo = (int)((long long)P.n_pairs * split / kDwSplit);
+    const int e_hi = (int)((long long)P.n_pairs * (split + 1) / kDwSplit);
+    for (int c0 = e_lo; c0 < e_hi; c0 += kDwChunk) {
+        const int nc = min(kDwChunk, e_hi - c0);
         __syncthreads();
         if (tid < nc) {
             const int e = c0 + tid;
@@ -658,7 +720,7 @@ __global__ void __launch_bounds__(kNt) k_bwd_dw(BwdParams P) {
                         float acc = 0.f;
                         for (int n = 0; n < w; ++n) acc = fmaf(dr[n], load_feat(x, xb + (size_t)n * C), acc);
                         float gv = 0.f;
-                        for (int kb = 0; kb < nr; ++kb) gv = fmaf(rho[el * nr + kb], P.Wrad[(size_t)kb * G + l1 * C + c], gv);
+                        for (int kb = 0; kb < nr; ++kb) gv = fmaf(rho[el * nr + kb], wr[kb * kDwT + q], gv);
                         vx = gv * acc;
                     }
                 }
@@ -700,9 +762,19 @@ __global__ void __launch_bounds__(kNt) k_bwd_dw(BwdParams P) {
         for (int b = 0; b < 4; ++b) {
             const int kx = k0 + tx * 4 + b;
             if (kx >= nm) continue;
-            P.gW[oa + (size_t)r * nm + kx] = accA[a][b];
-            if (m > 0) P.gW[ob + (size_t)r * nm + kx] = accB[a][b];
+            float* dst = P.gWpart + (size_t)split * so2_total(L, C, P.M);
+            dst[oa + (size_t)r * nm + kx] = accA[a][b];
+            if (m > 0) dst[ob + (size_t)r * nm + kx] = accB[a][b];
         }
+    }
+}
+
+// gW = the edge-range partial sums, added in a fixed order
+__global__ void k_bwd_dw_sum(const float* __restrict__ part, size_t total, float* out) {
+    for (size_t t = (size_t)blockIdx.x * blockDim.x + threadIdx.x; t < total; t += (size_t)gridDim.x * blockDim.x) {
+        float s = part[t];
+        for (int k = 1; k < kDwSplit; ++k) s += part[(size_t)k * total + t];
+        out[t] = s;
     }
 }
 
@@ -766,6 +838,8 @@ int n_dw_tiles(int L, int C, int M) {
 
 }  // namespace bwd
 
+size_t bwd_partial_bytes(int L, int C, int M) { return 4 * bwd::dw_part_floats(L, C, M); }
+
 bool bwd_supported(int L, int C, int H, int n_rbf) {
     if (L < 0 || L > kMaxL || bwd::kNt % H != 0) return false;
     return bwd::node_smem_floats(L, C, H, n_rbf) * 4 <= 227 * 1024 &&
@@ -791,6 +865,8 @@ cudaError_t run_attention_bwd(const BwdArgs& b, cudaStream_t s) {
     P.W = a.Wso2; P.Wt = a.Wt; P.Wrad = a.Wrad; P.q = a.q; P.k = a.k; P.G = b.grad_out;
     P.lse = b.lse; P.beta = b.beta; P.gq = b.gq; P.gk = b.gk; P.gpos = b.gpos; P.gx = b.gx; P.gWrad = b.gWrad;
     P.gW = b.gWso2;
+    P.gWpart = b.gWpart;
+    P.dw_tiles = n_dw_tiles(L, C, a.M);
 
     int dev = 0, n_sm = 148;
     cudaGetDevice(&dev);
@@ -825,7 +901,7 @@ cudaError_t run_attention_bwd(const BwdArgs& b, cudaStream_t s) {
     k_bwd_x0<<<(N * C + 255) / 256, 256, 0, s>>>(N, K, C, a.Wq, a.Wk, b.gq, b.gk, b.gx);
     E2F_CUDA_TRY_E(cudaGetLastError());
     if (b.gWso2 && a.n_pairs > 0) {
-        const int nt = n_dw_tiles(L, C, a.M);
+        const int nt = n_dw_tiles(L, C, a.M) * kDwSplit;
         const size_t dsm = dw_smem_floats(L, H, a.n_rbf) * 4;
 #define E2F_BWD_DW(LL)                                                                                         \
     case LL:                                                                                                   \
@@ -841,6 +917,9 @@ cudaError_t run_attention_bwd(const BwdArgs& b, cudaStream_t s) {
         }
 #undef E2F_BWD_DW
         if (e != cudaSuccess) return e;
+        count_launch();
+        k_bwd_dw_sum<<<592, 256, 0, s>>>(b.gWpart, so2_total(L, C, a.M), b.gWso2);
+        E2F_CUDA_TRY_E(cudaGetLastError());
     } else if (b.gWso2) {
         E2F_CUDA_TRY_E(cudaMemsetAsync(b.gWso2, 0, 4 * so2_total(L, C, a.M), s));
     }

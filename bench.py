@@ -95,7 +95,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except (OSError, FileNotFoundError):
             self.proc = None
         return self
@@ -487,6 +487,78 @@ def run_naive(args):
     return 0
 
 
+def run_backward(args):
+    """The attention's backward (e2f_onfly_attention_backward) on the bench workload: all
+    gradients (positions, features, every weight), and positions + features + W_rad only
+    (what forces need). fp32 CUDA-core kernels: the roofline is the FP32 FMA pipe."""
+    import torch
+
+    import atomistic_cell_list_b200 as e2f
+    import workloads as W
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    w = W.load_workload(args.config)
+    xs, _ = W.make_features(args.config, w.n_atoms, w.L, w.C, w.dtype)
+    wt = W.make_weights(args.config, w.L, w.C, w.H, w.n_rbf, w.dtype)
+
+    def host(a):
+        if a.dtype == np.uint16:
+            return torch.from_numpy(a.view(np.int16).copy()).view(torch.bfloat16)
+        return torch.from_numpy(np.ascontiguousarray(a))
+
+    pos = host(w.pos).to(dev)
+    x = host(xs).reshape(w.n_atoms, w.K, w.C).to(dev)
+    Wq, Wk, Wrad, Wso2 = (host(a).to(dev) for a in (wt.Wq, wt.Wk, wt.Wrad, wt.Wso2))
+    box = None if w.box is None else [float(b) for b in w.box]
+    gptr = None if w.graph_ptr is None else torch.from_numpy(w.graph_ptr).to(dev)
+    cfg = e2f.make_cfg(w.L, w.C, w.H, w.n_rbf, w.cutoff, w.dtype)
+    rp, col = e2f.e2f_build_neighbors(pos, box, w.cutoff, gptr)
+    E = int(col.numel())
+    G = torch.randn((w.n_atoms, w.K, w.C), generator=torch.Generator().manual_seed(1)).to(dev)
+    ws = torch.empty(e2f.e2f_attention_backward_workspace_size(w.n_atoms, E, cfg), dtype=torch.uint8, device=dev)
+    F = so2_flops_per_edge(w.L, w.C)
+    peaks, peak_src = measured_peaks()
+    clk_max = float(peaks.get("sm_max_mhz", 1965.0))
+    fma_peak = 148 * 128 * 2 * clk_max * 1e6 / 1e12
+    res = {}
+    for want in (True, False):
+        outs = e2f.e2f_onfly_attention_backward(cfg, pos, box, rp, col, x, Wq, Wk, Wrad, Wso2, G,
+                                                want_weights=want, workspace=ws)
+        for _ in range(max(0, args.warmup - 1)):
+            e2f.e2f_onfly_attention_backward(cfg, pos, box, rp, col, x, Wq, Wk, Wrad, Wso2, G,
+                                             want_weights=want, workspace=ws, out=outs)
+        torch.cuda.synchronize(dev)
+        ts = []
+        with ClockSampler(0) as clk:
+            for _ in range(args.steps):
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record()
+                e2f.e2f_onfly_attention_backward(cfg, pos, box, rp, col, x, Wq, Wk, Wrad, Wso2, G,
+                                                 want_weights=want, workspace=ws, out=outs)
+                b.record()
+                torch.cuda.synchronize(dev)
+                ts.append(a.elapsed_time(b))
+        ms = statistics.mean(ts)
+        # algorithmic work: the SO(2) maps applied twice per edge (recomputed Y, then the
+        # transposed maps) and, with weights, the weight-gradient contraction (one more F)
+        flops = E * F * (3 if want else 2)
+        res["all" if want else "forces"] = {"ms": ms, "pairs_per_s": E / (ms * 1e-3),
+                                            "tflops": flops / (ms * 1e-3) / 1e12, "clocks": clk.summary()}
+    line = {"metric": "attention backward pairs/s (all gradients), 1xB200", "impl": "ours", "value":
+            res["all"]["pairs_per_s"], "unit": "pairs/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": res["all"]["ms"], "higher_is_better": True, "dtype": "f32", "data": "synthetic",
+            "config": {**workload_desc(w), "n_pairs": E}, "forces_only": res["forces"],
+            "roofline": {"bound": "alu", "achieved": res["all"]["tflops"], "peak": fma_peak, "unit": "TFLOP/s",
+                         "frac": res["all"]["tflops"] / fma_peak, "traffic": None,
+                         "peak_note": f"fp32 FMA pipe: 148 SMs x 128 lanes x 2 FLOP x {clk_max:.0f} MHz "
+                                      f"(derived, {peak_src} clock)",
+                         "units_per_launch": f"{E} edges x 3 x {F} SO(2) FLOP"},
+            "clocks": res["all"]["clocks"]}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -496,9 +568,12 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference", "naive"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--m-max", type=int, default=-1, help="SO(2) truncation order (-1: full layer)")
+    ap.add_argument("--backward", action="store_true", help="time the attention's backward instead")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
+    if args.backward:
+        return run_backward(args)
     if args.impl == "reference":
         return run_reference(args)
     if args.impl == "naive":
