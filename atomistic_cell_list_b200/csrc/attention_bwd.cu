@@ -42,12 +42,14 @@
 namespace e2f {
 namespace bwd {
 
-constexpr int kNt = 256;     // threads of the node kernel and the weight-gradient kernel
+constexpr int kNt = 256;     // threads of the weight-gradient kernel
+constexpr int kNodeNt = 512; // threads of the node kernel (one CTA per SM: 16 warps hide latency)
 constexpr int kTe = 8;       // edges per tile of the node kernel
-constexpr int kDwT = 64;     // weight-gradient tile side
+constexpr int kDwR = 128;    // weight-gradient tile rows
+constexpr int kDwC = 64;     // weight-gradient tile columns
 constexpr int kDwE = 32;     // edges per operand sub-chunk of the weight-gradient kernel
-constexpr int kDwChunk = 256;  // edges per geometry chunk (one per thread)
-constexpr int kDwSplit = 4;    // edge ranges per tile (partial sums added in a fixed order)
+constexpr int kDwChunk = 128;  // edges per geometry chunk (one per thread)
+constexpr int kDwSplit = 8;    // edge ranges per tile (partial sums added in a fixed order)
 
 struct BwdParams {
     int n_atoms, C, H, n_rbf, M;
@@ -158,14 +160,14 @@ size_t node_smem_floats(int L, int C, int H, int n_rbf) {
     const int KH = (L >= 1) ? std::max((L + 1) * C, 2 * L * C) : C;
     return (size_t)K * C + 3ull * kTe * WS + 2ull * kTe * n_rbf + (size_t)kTe * G + (size_t)kTe * Gv +
            2ull * kTe * H + 12ull * kTe + 3ull * KH * kTe + (size_t)n_rbf * G + C + 2ull * H + 4 + kTe +
-           2ull * kNt + kTe;
+           2ull * kNodeNt + kTe;
 }
 
 // One CTA per destination node at a time (persistent over nodes): every
 // gradient except dW_so2, dW_q, dW_k and the l = 0 part of dx that flows
 // through q and k.
 template <int L, typename T>
-__global__ void __launch_bounds__(kNt, 1) k_bwd_node(BwdParams P) {
+__global__ void __launch_bounds__(kNodeNt, 1) k_bwd_node(BwdParams P) {
     constexpr int K = n_sh(L);
     constexpr int WS = wig_size(L);
     const int C = P.C, H = P.H, dh = C / H, nr = P.n_rbf, M = P.M;
@@ -195,8 +197,8 @@ __global__ void __launch_bounds__(kNt, 1) k_bwd_node(BwdParams P) {
     float* dlt = lse_s + H;            // [H] delta_i
     float* gpi = dlt + H;              // [4] dpos_i
     float* ddv = gpi + 4;              // [te]
-    float* red = ddv + kTe;            // [2 kNt]
-    int* jn = reinterpret_cast<int*>(red + 2 * kNt);  // [te]
+    float* red = ddv + kTe;            // [2 kNodeNt]
+    int* jn = reinterpret_cast<int*>(red + 2 * kNodeNt);  // [te]
 
     const int tid = threadIdx.x, nt = blockDim.x, lane = tid & 31, warp = tid >> 5;
     const float inv = rsqrtf((float)dh);
@@ -590,13 +592,15 @@ __global__ void __launch_bounds__(kNt, 1) k_bwd_node(BwdParams P) {
     for (int t = tid; t < nr * G; t += nt) atomicAdd(P.gWrad + t, gWr[t]);
 }
 
-// dW_so2 = sum over edges of dY (x) X~, one 64 x 64 tile of one |m| block per
-// CTA (A and B tiles together for m >= 1):
+// dW_so2 = sum over edges of dY (x) X~, one 128 x 64 tile (rows x columns) of
+// one |m| block per CTA (A and B tiles together for m >= 1), over one of
+// kDwSplit edge ranges:
 //   dA += dY+ X~+^T + dY- X~-^T,   dB += dY- X~+^T - dY+ X~-^T
 // with dY(l3, +-m, c) = alpha^{head c} sum_n D^l3[+-m][n] G_i[l3, n, c] and
 // X~(l1, +-m, c) = g_v[l1, c] sum_n D^l1[+-m][n] x_j[l1, n, c], rebuilt per
 // edge from the geometry (no per-edge storage). Edges are visited in CSR
-// order in chunks of 256 (one thread per edge for the frame and weights).
+// order in chunks of kDwChunk (one thread per edge for the frame and weights),
+// then in sub-chunks of kDwE for the operands.
 __device__ __forceinline__ int drow_off(int m, int l, int s) {
     // rows (l+m) and (l-m) of D^l for l = m..L, stored per edge back to back
     const int nrow = (m == 0) ? 1 : 2;
@@ -610,11 +614,20 @@ size_t dw_part_floats(int L, int C, int M) { return (size_t)kDwSplit * so2_total
 size_t dw_smem_floats(int L, int H, int n_rbf) {
     (void)L;
     return (size_t)kDwChunk * 50 + (size_t)kDwChunk * n_rbf + (size_t)kDwChunk * H + 2 * kDwChunk +
-           4ull * kDwE * kDwT + (size_t)n_rbf * kDwT;
+           2ull * kDwE * kDwR + 2ull * kDwE * kDwC + (size_t)n_rbf * kDwC;
+}
+
+int n_dw_tiles(int L, int C, int M) {
+    int n = 0;
+    for (int m = 0; m <= M; ++m) {
+        const int nm = (L + 1 - m) * C;
+        n += ((nm + kDwR - 1) / kDwR) * ((nm + kDwC - 1) / kDwC);
+    }
+    return n;
 }
 
 template <int L, typename T>
-__global__ void __launch_bounds__(kNt) k_bwd_dw(BwdParams P) {
+__global__ void __launch_bounds__(kNt, 2) k_bwd_dw(BwdParams P) {
     constexpr int K = n_sh(L);
     constexpr int WS = wig_size(L);
     const int C = P.C, H = P.H, dh = C / H, nr = P.n_rbf;
@@ -622,14 +635,16 @@ __global__ void __launch_bounds__(kNt) k_bwd_dw(BwdParams P) {
     const T* __restrict__ x = static_cast<const T*>(P.x);
     // this CTA's tile (blocks m = 0..M in order, tiles of a block row-major) and edge range
     const int split = blockIdx.x / P.dw_tiles;
-    int m = 0, nm = (L + 1) * C, side = (nm + kDwT - 1) / kDwT, b = blockIdx.x % P.dw_tiles;
-    while (b >= side * side && m < P.M) {
-        b -= side * side;
+    int m = 0, nm = (L + 1) * C, b = blockIdx.x % P.dw_tiles;
+    int sr = (nm + kDwR - 1) / kDwR, sc = (nm + kDwC - 1) / kDwC;
+    while (b >= sr * sc && m < P.M) {
+        b -= sr * sc;
         ++m;
         nm = (L + 1 - m) * C;
-        side = (nm + kDwT - 1) / kDwT;
+        sr = (nm + kDwR - 1) / kDwR;
+        sc = (nm + kDwC - 1) / kDwC;
     }
-    const int r0 = (b / side) * kDwT, k0 = (b % side) * kDwT;
+    const int r0 = (b / sc) * kDwR, k0 = (b % sc) * kDwC;
     const int nrow = (m == 0) ? 1 : 2;
 
     extern __shared__ float sm[];
@@ -638,20 +653,20 @@ __global__ void __launch_bounds__(kNt) k_bwd_dw(BwdParams P) {
     float* alpha = rho + kDwChunk * nr;        // [chunk][H]
     int* ei = reinterpret_cast<int*>(alpha + kDwChunk * H);  // [chunk] node i
     int* ej = ei + kDwChunk;                   // [chunk] neighbour j
-    float* Yop = reinterpret_cast<float*>(ej + kDwChunk);    // [2][kDwE][kDwT] dY rows of the tile
-    float* Xop = Yop + 2 * kDwE * kDwT;        // [2][kDwE][kDwT] X~ columns of the tile
-    float* wr = Xop + 2 * kDwE * kDwT;         // [nr][kDwT] W_rad columns of the tile's X~ columns
+    float* Yop = reinterpret_cast<float*>(ej + kDwChunk);    // [2][kDwE][kDwR] dY rows of the tile
+    float* Xop = Yop + 2 * kDwE * kDwR;        // [2][kDwE][kDwC] X~ columns of the tile
+    float* wr = Xop + 2 * kDwE * kDwC;         // [nr][kDwC] W_rad columns of the tile's X~ columns
 
     const int tid = threadIdx.x, ty = tid / 16, tx = tid % 16;
     const float inv = rsqrtf((float)dh);
-    float accA[4][4], accB[4][4];
+    float accA[8][4], accB[8][4];
 #pragma unroll
-    for (int a = 0; a < 4; ++a)
+    for (int a = 0; a < 8; ++a)
 #pragma unroll
-        for (int b = 0; b < 4; ++b) { accA[a][b] = 0.f; accB[a][b] = 0.f; }
+        for (int c = 0; c < 4; ++c) { accA[a][c] = 0.f; accB[a][c] = 0.f; }
 
-    for (int t = tid; t < nr * kDwT; t += kNt) {
-        const int kb = t / kDwT, kx = k0 + t % kDwT;
+    for (int t = tid; t < nr * kDwC; t += kNt) {
+        const int kb = t / kDwC, kx = k0 + t % kDwC;
         wr[t] = (kx < nm) ? P.Wrad[(size_t)kb * G + (m + kx / C) * C + kx % C] : 0.f;
     }
     const int e_lo = (int)((long long)P.n_pairs * split / kDwSplit);
@@ -678,9 +693,9 @@ __global__ void __launch_bounds__(kNt) k_bwd_dw(BwdParams P) {
             float* dr = drow + tid * 50;
             for (int l = m; l <= L; ++l) {
                 const int w = 2 * l + 1;
-                for (int s = 0; s < nrow; ++s) {
-                    const int row = s == 0 ? l + m : l - m;
-                    for (int n = 0; n < w; ++n) dr[drow_off(m, l, s) + n] = D[wig_off(l) + row * w + n];
+                for (int s2 = 0; s2 < nrow; ++s2) {
+                    const int row = s2 == 0 ? l + m : l - m;
+                    for (int n = 0; n < w; ++n) dr[drow_off(m, l, s2) + n] = D[wig_off(l) + row * w + n];
                 }
             }
             for (int kb = 0; kb < nr; ++kb) rho[tid * nr + kb] = rbf(d, kb, P.cutoff, nr);
@@ -698,55 +713,62 @@ __global__ void __launch_bounds__(kNt) k_bwd_dw(BwdParams P) {
         for (int s0 = 0; s0 < nc; s0 += kDwE) {
             const int ns = min(kDwE, nc - s0);
             // operands of the sub-chunk: dY rows r0.., X~ columns k0..
-            for (int t = tid; t < 2 * kDwE * kDwT; t += kNt) {
-                const int s = t / (kDwE * kDwT), rem = t % (kDwE * kDwT);
-                const int e = rem / kDwT, q = rem % kDwT;
-                float vy = 0.f, vx = 0.f;
-                if (e < ns && s < nrow) {
+            for (int t = tid; t < 2 * kDwE * kDwR; t += kNt) {
+                const int s2 = t / (kDwE * kDwR), rem = t % (kDwE * kDwR);
+                const int e = rem / kDwR, q = rem % kDwR, ry = r0 + q;
+                float v = 0.f;
+                if (e < ns && s2 < nrow && ry < nm) {
                     const int el = s0 + e;
-                    const int ry = r0 + q, kx = k0 + q;
-                    if (ry < nm) {
-                        const int l3 = m + ry / C, c = ry % C, w = 2 * l3 + 1;
-                        const float* dr = drow + el * 50 + drow_off(m, l3, s);
-                        const float* gi = P.G + ((size_t)ei[el] * K + l3 * l3) * C + c;
-                        float acc = 0.f;
-                        for (int n = 0; n < w; ++n) acc = fmaf(dr[n], gi[(size_t)n * C], acc);
-                        vy = alpha[el * H + c / dh] * acc;
-                    }
-                    if (kx < nm) {
-                        const int l1 = m + kx / C, c = kx % C, w = 2 * l1 + 1;
-                        const float* dr = drow + el * 50 + drow_off(m, l1, s);
-                        const size_t xb = ((size_t)ej[el] * K + l1 * l1) * C + c;
-                        float acc = 0.f;
-                        for (int n = 0; n < w; ++n) acc = fmaf(dr[n], load_feat(x, xb + (size_t)n * C), acc);
-                        float gv = 0.f;
-                        for (int kb = 0; kb < nr; ++kb) gv = fmaf(rho[el * nr + kb], wr[kb * kDwT + q], gv);
-                        vx = gv * acc;
-                    }
+                    const int l3 = m + ry / C, c = ry % C, w = 2 * l3 + 1;
+                    const float* dr = drow + el * 50 + drow_off(m, l3, s2);
+                    const float* gi = P.G + ((size_t)ei[el] * K + l3 * l3) * C + c;
+                    float acc = 0.f;
+                    for (int n = 0; n < w; ++n) acc = fmaf(dr[n], gi[(size_t)n * C], acc);
+                    v = alpha[el * H + c / dh] * acc;
                 }
-                Yop[t] = vy;
-                Xop[t] = vx;
+                Yop[t] = v;
+            }
+            for (int t = tid; t < 2 * kDwE * kDwC; t += kNt) {
+                const int s2 = t / (kDwE * kDwC), rem = t % (kDwE * kDwC);
+                const int e = rem / kDwC, q = rem % kDwC, kx = k0 + q;
+                float v = 0.f;
+                if (e < ns && s2 < nrow && kx < nm) {
+                    const int el = s0 + e;
+                    const int l1 = m + kx / C, c = kx % C, w = 2 * l1 + 1;
+                    const float* dr = drow + el * 50 + drow_off(m, l1, s2);
+                    const size_t xb = ((size_t)ej[el] * K + l1 * l1) * C + c;
+                    float acc = 0.f;
+                    for (int n = 0; n < w; ++n) acc = fmaf(dr[n], load_feat(x, xb + (size_t)n * C), acc);
+                    float gv = 0.f;
+                    for (int kb = 0; kb < nr; ++kb) gv = fmaf(rho[el * nr + kb], wr[kb * kDwC + q], gv);
+                    v = gv * acc;
+                }
+                Xop[t] = v;
             }
             __syncthreads();
             for (int e = 0; e < ns; ++e) {
-                const float4 yp = *reinterpret_cast<const float4*>(Yop + e * kDwT + ty * 4);
-                const float4 xp = *reinterpret_cast<const float4*>(Xop + e * kDwT + tx * 4);
-                const float ypa[4] = {yp.x, yp.y, yp.z, yp.w}, xpa[4] = {xp.x, xp.y, xp.z, xp.w};
+                const float4 y0 = *reinterpret_cast<const float4*>(Yop + e * kDwR + ty * 8);
+                const float4 y1 = *reinterpret_cast<const float4*>(Yop + e * kDwR + ty * 8 + 4);
+                const float4 xv = *reinterpret_cast<const float4*>(Xop + e * kDwC + tx * 4);
+                const float ypa[8] = {y0.x, y0.y, y0.z, y0.w, y1.x, y1.y, y1.z, y1.w};
+                const float xpa[4] = {xv.x, xv.y, xv.z, xv.w};
                 if (m == 0) {
 #pragma unroll
-                    for (int a = 0; a < 4; ++a)
+                    for (int a = 0; a < 8; ++a)
 #pragma unroll
-                        for (int b = 0; b < 4; ++b) accA[a][b] = fmaf(ypa[a], xpa[b], accA[a][b]);
+                        for (int c = 0; c < 4; ++c) accA[a][c] = fmaf(ypa[a], xpa[c], accA[a][c]);
                 } else {
-                    const float4 ym = *reinterpret_cast<const float4*>(Yop + (kDwE + e) * kDwT + ty * 4);
-                    const float4 xm = *reinterpret_cast<const float4*>(Xop + (kDwE + e) * kDwT + tx * 4);
-                    const float yma[4] = {ym.x, ym.y, ym.z, ym.w}, xma[4] = {xm.x, xm.y, xm.z, xm.w};
+                    const float4 z0 = *reinterpret_cast<const float4*>(Yop + (kDwE + e) * kDwR + ty * 8);
+                    const float4 z1 = *reinterpret_cast<const float4*>(Yop + (kDwE + e) * kDwR + ty * 8 + 4);
+                    const float4 xw = *reinterpret_cast<const float4*>(Xop + (kDwE + e) * kDwC + tx * 4);
+                    const float yma[8] = {z0.x, z0.y, z0.z, z0.w, z1.x, z1.y, z1.z, z1.w};
+                    const float xma[4] = {xw.x, xw.y, xw.z, xw.w};
 #pragma unroll
-                    for (int a = 0; a < 4; ++a)
+                    for (int a = 0; a < 8; ++a)
 #pragma unroll
-                        for (int b = 0; b < 4; ++b) {
-                            accA[a][b] = fmaf(ypa[a], xpa[b], fmaf(yma[a], xma[b], accA[a][b]));
-                            accB[a][b] = fmaf(yma[a], xpa[b], fmaf(-ypa[a], xma[b], accB[a][b]));
+                        for (int c = 0; c < 4; ++c) {
+                            accA[a][c] = fmaf(ypa[a], xpa[c], fmaf(yma[a], xma[c], accA[a][c]));
+                            accB[a][c] = fmaf(yma[a], xpa[c], fmaf(-ypa[a], xma[c], accB[a][c]));
                         }
                 }
             }
@@ -754,17 +776,17 @@ __global__ void __launch_bounds__(kNt) k_bwd_dw(BwdParams P) {
         }
     }
     const size_t oa = so2_offset(L, C, m, 0), ob = so2_offset(L, C, m, 1);
+    float* dst = P.gWpart + (size_t)split * so2_total(L, C, P.M);
 #pragma unroll
-    for (int a = 0; a < 4; ++a) {
-        const int r = r0 + ty * 4 + a;
+    for (int a = 0; a < 8; ++a) {
+        const int r = r0 + ty * 8 + a;
         if (r >= nm) continue;
 #pragma unroll
-        for (int b = 0; b < 4; ++b) {
-            const int kx = k0 + tx * 4 + b;
+        for (int c = 0; c < 4; ++c) {
+            const int kx = k0 + tx * 4 + c;
             if (kx >= nm) continue;
-            float* dst = P.gWpart + (size_t)split * so2_total(L, C, P.M);
-            dst[oa + (size_t)r * nm + kx] = accA[a][b];
-            if (m > 0) dst[ob + (size_t)r * nm + kx] = accB[a][b];
+            dst[oa + (size_t)r * nm + kx] = accA[a][c];
+            if (m > 0) dst[ob + (size_t)r * nm + kx] = accB[a][c];
         }
     }
 }
@@ -814,7 +836,7 @@ cudaError_t launch_node(const BwdParams& P, size_t smem, int grid, cudaStream_t 
     cudaError_t e = cudaFuncSetAttribute(k_bwd_node<L, T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     count_launch();
-    k_bwd_node<L, T><<<grid, kNt, smem, s>>>(P);
+    k_bwd_node<L, T><<<grid, kNodeNt, smem, s>>>(P);
     return cudaGetLastError();
 }
 
@@ -827,21 +849,13 @@ cudaError_t launch_dw(const BwdParams& P, int n_tiles, size_t smem, cudaStream_t
     return cudaGetLastError();
 }
 
-int n_dw_tiles(int L, int C, int M) {
-    int n = 0;
-    for (int m = 0; m <= M; ++m) {
-        const int t = ((L + 1 - m) * C + kDwT - 1) / kDwT;
-        n += t * t;
-    }
-    return n;
-}
 
 }  // namespace bwd
 
 size_t bwd_partial_bytes(int L, int C, int M) { return 4 * bwd::dw_part_floats(L, C, M); }
 
 bool bwd_supported(int L, int C, int H, int n_rbf) {
-    if (L < 0 || L > kMaxL || bwd::kNt % H != 0) return false;
+    if (L < 0 || L > kMaxL || bwd::kNt % H != 0 || bwd::kNodeNt % H != 0) return false;
     return bwd::node_smem_floats(L, C, H, n_rbf) * 4 <= 227 * 1024 &&
            bwd::dw_smem_floats(L, H, n_rbf) * 4 <= 227 * 1024;
 }
