@@ -417,12 +417,18 @@ def run_ours(args):
         roof = {"bound": "tensor", "achieved": tflops_ker, "peak": peak, "unit": "TFLOP/s", "frac": tflops_ker / peak,
                 "traffic": kernel_traffic(), "peak_note": f"bf16 dense burst, {peak_src}",
                 "peak_sustained": sus, "frac_sustained": tflops_ker / sus}
+    hbm = float(peaks.get("hbm_gbs", 6650.0))
+    if roof.get("traffic"):
+        # DRAM bytes per launch (ncu) over the live launch time: the gather phase runs inside this kernel
+        roof["dram_gbs"] = roof["traffic"] / (ms_ker * 1e-3) / 1e9
+        roof["dram_frac_of_hbm"] = roof["dram_gbs"] / hbm
     roof["kernel"] = "k_attn_tc (tcgen05)" if path == "tensor" else "k_attn_simt (fp32 CUDA cores)"
     roof["ms_per_launch"] = ms_ker
     roof["units_per_launch"] = f"{E} edges x {F} SO(2) FLOP"
     roof["traffic_note"] = ("dram read+write bytes per launch from ncu (profiles/k_attn_tc_chain_water_30k.md); "
                             "null when the kernel source differs from the profiled one")
 
+    nbr_bytes = 16 * w.n_atoms + 4 * (w.n_atoms + 1) + 4 * E + 8 * w.n_atoms
     line = {"metric": METRIC, "value": world * E / (ms_step * 1e-3), "unit": "pairs/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32" if path == "simt" else "bf16",
@@ -431,6 +437,11 @@ def run_ours(args):
                        "l2": "flushed (256 MB write) between timed steps"},
             "tflops": tflops, "tflops_kernel": tflops_ker, "ms_attention": ms_att, "ms_attention_kernel": ms_ker,
             "ms_neighbors": ms_nbr,
+            "neighbor_build_hbm": {
+                "algorithmic_bytes": nbr_bytes, "gb_per_s": nbr_bytes / (ms_nbr * 1e-3) / 1e9,
+                "frac_of_hbm": nbr_bytes / (ms_nbr * 1e-3) / 1e9 / hbm,
+                "note": "16N (positions and keys read) + 4(N+1) + 4E (CSR written) + 8N (one pass of the "
+                        "sort); latency-bound at these sizes"},
             "neighbor_pairs_per_s": E / (ms_nbr * 1e-3), "attention_pairs_per_s": E / (ms_att * 1e-3),
             "roofline": roof,
             "e2e": {"value": world * E / (ms_e2e * 1e-3), "unit": "pairs/s", "h2d_bytes_per_step": h2d,
