@@ -310,10 +310,15 @@ __global__ void __launch_bounds__(kNodeNt, 1) k_bwd_node(BwdParams P) {
                         const float* D = Dm + e * WS + wig_off(l1);
                         const int w = 2 * l1 + 1;
                         const size_t xb = ((size_t)jn[e] * K + l1 * l1) * C + c;
-                        for (int n = 0; n < w; ++n) {
-                            const float xv = load_feat(x, xb + (size_t)n * C);
-                            vp = fmaf(D[(l1 + m) * w + n], xv, vp);
-                            vm = fmaf(D[(l1 - m) * w + n], xv, vm);
+                        float xr[2 * L + 1];  // all loads issued before the arithmetic
+#pragma unroll
+                        for (int n = 0; n < 2 * L + 1; ++n) xr[n] = (n < w) ? load_feat(x, xb + (size_t)n * C) : 0.f;
+#pragma unroll
+                        for (int n = 0; n < 2 * L + 1; ++n) {
+                            if (n < w) {
+                                vp = fmaf(D[(l1 + m) * w + n], xr[n], vp);
+                                vm = fmaf(D[(l1 - m) * w + n], xr[n], vm);
+                            }
                         }
                         const float gv = g[e * G + l1 * C + c];
                         vp *= gv;
@@ -483,17 +488,24 @@ __global__ void __launch_bounds__(kNodeNt, 1) k_bwd_node(BwdParams P) {
                             const size_t xb = ((size_t)jn[e] * K + l1 * l1) * C + c;
                             const float gv = g[e * G + l1 * C + c];
                             float rp = 0.f, rm = 0.f, xp = 0.f, xm = 0.f, zp = 0.f, zm = 0.f;
-                            for (int n = 0; n < w1; ++n) {
-                                const float xv = load_feat(x, xb + (size_t)n * C);
-                                rp = fmaf(D[(l1 + m) * w1 + n], xv, rp);
-                                rm = fmaf(D[(l1 - m) * w1 + n], xv, rm);
-                                xp = fmaf(Ex[(l1 + m) * w1 + n], xv, xp);
-                                xm = fmaf(Ex[(l1 - m) * w1 + n], xv, xm);
-                                zp = fmaf(Ey[(l1 + m) * w1 + n], xv, zp);
-                                zm = fmaf(Ey[(l1 - m) * w1 + n], xv, zm);
-                                float gxv = D[(l1 + m) * w1 + n] * dp[e];
-                                if (m > 0) gxv = fmaf(D[(l1 - m) * w1 + n], dq[e], gxv);
-                                atomicAdd(P.gx + xb + (size_t)n * C, gv * gxv);
+                            float xr[2 * L + 1];  // all loads issued before the arithmetic
+#pragma unroll
+                            for (int n = 0; n < 2 * L + 1; ++n)
+                                xr[n] = (n < w1) ? load_feat(x, xb + (size_t)n * C) : 0.f;
+#pragma unroll
+                            for (int n = 0; n < 2 * L + 1; ++n) {
+                                if (n < w1) {
+                                    const float xv = xr[n];
+                                    rp = fmaf(D[(l1 + m) * w1 + n], xv, rp);
+                                    rm = fmaf(D[(l1 - m) * w1 + n], xv, rm);
+                                    xp = fmaf(Ex[(l1 + m) * w1 + n], xv, xp);
+                                    xm = fmaf(Ex[(l1 - m) * w1 + n], xv, xm);
+                                    zp = fmaf(Ey[(l1 + m) * w1 + n], xv, zp);
+                                    zm = fmaf(Ey[(l1 - m) * w1 + n], xv, zm);
+                                    float gxv = D[(l1 + m) * w1 + n] * dp[e];
+                                    if (m > 0) gxv = fmaf(D[(l1 - m) * w1 + n], dq[e], gxv);
+                                    atomicAdd(P.gx + xb + (size_t)n * C, gv * gxv);
+                                }
                             }
                             float dg = dp[e] * rp, tx = dp[e] * xp, ty = dp[e] * zp;
                             if (m > 0) {
@@ -611,10 +623,13 @@ __device__ __forceinline__ int drow_off(int m, int l, int s) {
 
 size_t dw_part_floats(int L, int C, int M) { return (size_t)kDwSplit * so2_total(L, C, M); }
 
-size_t dw_smem_floats(int L, int H, int n_rbf) {
-    (void)L;
-    return (size_t)kDwChunk * 50 + (size_t)kDwChunk * n_rbf + (size_t)kDwChunk * H + 2 * kDwChunk +
-           2ull * kDwE * kDwR + 2ull * kDwE * kDwC + (size_t)n_rbf * kDwC;
+constexpr int kDwStrideH = kDwE + 8;  // fp16 operand row stride (halves): conflict-free fragment loads
+
+size_t dw_smem_bytes(int H, int n_rbf, bool tc) {
+    const size_t common = 4 * ((size_t)kDwChunk * 50 + (size_t)kDwChunk * n_rbf + (size_t)kDwChunk * H +
+                               2 * kDwChunk + (size_t)n_rbf * kDwC);
+    const size_t ops = tc ? 2 * 2ull * (kDwR + kDwC) * kDwStrideH : 4 * 2ull * kDwE * (kDwR + kDwC);
+    return common + ops;
 }
 
 int n_dw_tiles(int L, int C, int M) {
@@ -626,7 +641,20 @@ int n_dw_tiles(int L, int C, int M) {
     return n;
 }
 
-template <int L, typename T>
+// m16n8k16 fp16 x fp16 -> fp32 (A row-major 16 x 16, B col-major 16 x 8)
+__device__ __forceinline__ void mma16816(float* d, const uint32_t* a, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// TC = false: fp32 operands and FMA accumulation (thread tile 8 x 4).
+// TC = true: fp16 operands, tensor-core accumulation in fp32 (warp tile
+// 32 x 32 from m16n8k16 mma.sync); used for bf16 storage, whose inputs
+// already carry 8-bit mantissas.
+template <int L, typename T, bool TC>
 __global__ void __launch_bounds__(kNt, 2) k_bwd_dw(BwdParams P) {
     constexpr int K = n_sh(L);
     constexpr int WS = wig_size(L);
@@ -653,13 +681,20 @@ __global__ void __launch_bounds__(kNt, 2) k_bwd_dw(BwdParams P) {
     float* alpha = rho + kDwChunk * nr;        // [chunk][H]
     int* ei = reinterpret_cast<int*>(alpha + kDwChunk * H);  // [chunk] node i
     int* ej = ei + kDwChunk;                   // [chunk] neighbour j
-    float* Yop = reinterpret_cast<float*>(ej + kDwChunk);    // [2][kDwE][kDwR] dY rows of the tile
-    float* Xop = Yop + 2 * kDwE * kDwR;        // [2][kDwE][kDwC] X~ columns of the tile
-    float* wr = Xop + 2 * kDwE * kDwC;         // [nr][kDwC] W_rad columns of the tile's X~ columns
+    float* wr = reinterpret_cast<float*>(ej + kDwChunk);     // [nr][kDwC] W_rad columns of the tile
+    float* ops = wr + nr * kDwC;
+    // SIMT: Yop [2][kDwE][kDwR], Xop [2][kDwE][kDwC] (fp32, edge-major)
+    // TC:   Ys [2][kDwR][kDwStrideH], Xs [2][kDwC][kDwStrideH] (fp16, edge-minor)
+    float* Yop = ops;
+    float* Xop = Yop + 2 * kDwE * kDwR;
+    __half* Ys = reinterpret_cast<__half*>(ops);
+    __half* Xs = Ys + 2 * kDwR * kDwStrideH;
 
     const int tid = threadIdx.x, ty = tid / 16, tx = tid % 16;
+    const int lane = tid & 31, warp = tid >> 5, g8 = lane >> 2, t4 = lane & 3;
+    const int wrow = (warp >> 1) * 32, wcol = (warp & 1) * 32;
     const float inv = rsqrtf((float)dh);
-    float accA[8][4], accB[8][4];
+    float accA[8][4], accB[8][4];  // SIMT: [row][col]; TC: [m16 tile x 4 + n8 tile][fragment]
 #pragma unroll
     for (int a = 0; a < 8; ++a)
 #pragma unroll
@@ -722,11 +757,17 @@ __global__ void __launch_bounds__(kNt, 2) k_bwd_dw(BwdParams P) {
                     const int l3 = m + ry / C, c = ry % C, w = 2 * l3 + 1;
                     const float* dr = drow + el * 50 + drow_off(m, l3, s2);
                     const float* gi = P.G + ((size_t)ei[el] * K + l3 * l3) * C + c;
+                    float gr[2 * L + 1];  // all loads issued before the arithmetic
+#pragma unroll
+                    for (int n = 0; n < 2 * L + 1; ++n) gr[n] = (n < w) ? gi[(size_t)n * C] : 0.f;
                     float acc = 0.f;
-                    for (int n = 0; n < w; ++n) acc = fmaf(dr[n], gi[(size_t)n * C], acc);
+#pragma unroll
+                    for (int n = 0; n < 2 * L + 1; ++n)
+                        if (n < w) acc = fmaf(dr[n], gr[n], acc);
                     v = alpha[el * H + c / dh] * acc;
                 }
-                Yop[t] = v;
+                if constexpr (TC) Ys[(s2 * kDwR + q) * kDwStrideH + e] = __float2half_rn(v);
+                else Yop[t] = v;
             }
             for (int t = tid; t < 2 * kDwE * kDwC; t += kNt) {
                 const int s2 = t / (kDwE * kDwC), rem = t % (kDwE * kDwC);
@@ -737,39 +778,86 @@ __global__ void __launch_bounds__(kNt, 2) k_bwd_dw(BwdParams P) {
                     const int l1 = m + kx / C, c = kx % C, w = 2 * l1 + 1;
                     const float* dr = drow + el * 50 + drow_off(m, l1, s2);
                     const size_t xb = ((size_t)ej[el] * K + l1 * l1) * C + c;
+                    float xr[2 * L + 1];  // all loads issued before the arithmetic
+#pragma unroll
+                    for (int n = 0; n < 2 * L + 1; ++n) xr[n] = (n < w) ? load_feat(x, xb + (size_t)n * C) : 0.f;
                     float acc = 0.f;
-                    for (int n = 0; n < w; ++n) acc = fmaf(dr[n], load_feat(x, xb + (size_t)n * C), acc);
+#pragma unroll
+                    for (int n = 0; n < 2 * L + 1; ++n)
+                        if (n < w) acc = fmaf(dr[n], xr[n], acc);
                     float gv = 0.f;
                     for (int kb = 0; kb < nr; ++kb) gv = fmaf(rho[el * nr + kb], wr[kb * kDwC + q], gv);
                     v = gv * acc;
                 }
-                Xop[t] = v;
+                if constexpr (TC) Xs[(s2 * kDwC + q) * kDwStrideH + e] = __float2half_rn(v);
+                else Xop[t] = v;
             }
             __syncthreads();
-            for (int e = 0; e < ns; ++e) {
-                const float4 y0 = *reinterpret_cast<const float4*>(Yop + e * kDwR + ty * 8);
-                const float4 y1 = *reinterpret_cast<const float4*>(Yop + e * kDwR + ty * 8 + 4);
-                const float4 xv = *reinterpret_cast<const float4*>(Xop + e * kDwC + tx * 4);
-                const float ypa[8] = {y0.x, y0.y, y0.z, y0.w, y1.x, y1.y, y1.z, y1.w};
-                const float xpa[4] = {xv.x, xv.y, xv.z, xv.w};
-                if (m == 0) {
+            if constexpr (TC) {
+                // warp tile: rows wrow..+31 (two m16), columns wcol..+31 (four n8); K = the sub-chunk's edges
 #pragma unroll
-                    for (int a = 0; a < 8; ++a)
+                for (int kb = 0; kb < kDwE; kb += 16) {
+                    uint32_t ya[2][2][4], xb[2][4][2];  // [sign][m16 | n8][fragment]
 #pragma unroll
-                        for (int c = 0; c < 4; ++c) accA[a][c] = fmaf(ypa[a], xpa[c], accA[a][c]);
-                } else {
-                    const float4 z0 = *reinterpret_cast<const float4*>(Yop + (kDwE + e) * kDwR + ty * 8);
-                    const float4 z1 = *reinterpret_cast<const float4*>(Yop + (kDwE + e) * kDwR + ty * 8 + 4);
-                    const float4 xw = *reinterpret_cast<const float4*>(Xop + (kDwE + e) * kDwC + tx * 4);
-                    const float yma[8] = {z0.x, z0.y, z0.z, z0.w, z1.x, z1.y, z1.z, z1.w};
-                    const float xma[4] = {xw.x, xw.y, xw.z, xw.w};
+                    for (int s2 = 0; s2 < 2; ++s2) {
+                        if (s2 >= nrow) break;
 #pragma unroll
-                    for (int a = 0; a < 8; ++a)
-#pragma unroll
-                        for (int c = 0; c < 4; ++c) {
-                            accA[a][c] = fmaf(ypa[a], xpa[c], fmaf(yma[a], xma[c], accA[a][c]));
-                            accB[a][c] = fmaf(yma[a], xpa[c], fmaf(-ypa[a], xma[c], accB[a][c]));
+                        for (int mi = 0; mi < 2; ++mi) {
+                            const __half* base = Ys + (size_t)(s2 * kDwR + wrow + 16 * mi + g8) * kDwStrideH + kb + 2 * t4;
+                            ya[s2][mi][0] = *reinterpret_cast<const uint32_t*>(base);
+                            ya[s2][mi][1] = *reinterpret_cast<const uint32_t*>(base + 8 * kDwStrideH);
+                            ya[s2][mi][2] = *reinterpret_cast<const uint32_t*>(base + 8);
+                            ya[s2][mi][3] = *reinterpret_cast<const uint32_t*>(base + 8 * kDwStrideH + 8);
                         }
+#pragma unroll
+                        for (int ni = 0; ni < 4; ++ni) {
+                            const __half* base = Xs + (size_t)(s2 * kDwC + wcol + 8 * ni + g8) * kDwStrideH + kb + 2 * t4;
+                            xb[s2][ni][0] = *reinterpret_cast<const uint32_t*>(base);
+                            xb[s2][ni][1] = *reinterpret_cast<const uint32_t*>(base + 8);
+                        }
+                    }
+#pragma unroll
+                    for (int mi = 0; mi < 2; ++mi)
+#pragma unroll
+                        for (int ni = 0; ni < 4; ++ni) {
+                            float* dA = accA[mi * 4 + ni];
+                            mma16816(dA, ya[0][mi], xb[0][ni][0], xb[0][ni][1]);
+                            if (nrow == 2) {
+                                mma16816(dA, ya[1][mi], xb[1][ni][0], xb[1][ni][1]);
+                                float* dB = accB[mi * 4 + ni];
+                                const uint32_t yneg[4] = {ya[0][mi][0] ^ 0x80008000u, ya[0][mi][1] ^ 0x80008000u,
+                                                          ya[0][mi][2] ^ 0x80008000u, ya[0][mi][3] ^ 0x80008000u};
+                                mma16816(dB, ya[1][mi], xb[0][ni][0], xb[0][ni][1]);
+                                mma16816(dB, yneg, xb[1][ni][0], xb[1][ni][1]);
+                            }
+                        }
+                }
+            } else {
+                for (int e = 0; e < ns; ++e) {
+                    const float4 y0 = *reinterpret_cast<const float4*>(Yop + e * kDwR + ty * 8);
+                    const float4 y1 = *reinterpret_cast<const float4*>(Yop + e * kDwR + ty * 8 + 4);
+                    const float4 xv = *reinterpret_cast<const float4*>(Xop + e * kDwC + tx * 4);
+                    const float ypa[8] = {y0.x, y0.y, y0.z, y0.w, y1.x, y1.y, y1.z, y1.w};
+                    const float xpa[4] = {xv.x, xv.y, xv.z, xv.w};
+                    if (m == 0) {
+#pragma unroll
+                        for (int a = 0; a < 8; ++a)
+#pragma unroll
+                            for (int c = 0; c < 4; ++c) accA[a][c] = fmaf(ypa[a], xpa[c], accA[a][c]);
+                    } else {
+                        const float4 z0 = *reinterpret_cast<const float4*>(Yop + (kDwE + e) * kDwR + ty * 8);
+                        const float4 z1 = *reinterpret_cast<const float4*>(Yop + (kDwE + e) * kDwR + ty * 8 + 4);
+                        const float4 xw = *reinterpret_cast<const float4*>(Xop + (kDwE + e) * kDwC + tx * 4);
+                        const float yma[8] = {z0.x, z0.y, z0.z, z0.w, z1.x, z1.y, z1.z, z1.w};
+                        const float xma[4] = {xw.x, xw.y, xw.z, xw.w};
+#pragma unroll
+                        for (int a = 0; a < 8; ++a)
+#pragma unroll
+                            for (int c = 0; c < 4; ++c) {
+                                accA[a][c] = fmaf(ypa[a], xpa[c], fmaf(yma[a], xma[c], accA[a][c]));
+                                accB[a][c] = fmaf(yma[a], xpa[c], fmaf(-ypa[a], xma[c], accB[a][c]));
+                            }
+                    }
                 }
             }
             __syncthreads();
@@ -777,16 +865,31 @@ __global__ void __launch_bounds__(kNt, 2) k_bwd_dw(BwdParams P) {
     }
     const size_t oa = so2_offset(L, C, m, 0), ob = so2_offset(L, C, m, 1);
     float* dst = P.gWpart + (size_t)split * so2_total(L, C, P.M);
+    if constexpr (TC) {
 #pragma unroll
-    for (int a = 0; a < 8; ++a) {
-        const int r = r0 + ty * 8 + a;
-        if (r >= nm) continue;
+        for (int mi = 0; mi < 2; ++mi)
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            const int kx = k0 + tx * 4 + c;
-            if (kx >= nm) continue;
-            dst[oa + (size_t)r * nm + kx] = accA[a][c];
-            if (m > 0) dst[ob + (size_t)r * nm + kx] = accB[a][c];
+            for (int ni = 0; ni < 4; ++ni)
+#pragma unroll
+                for (int f = 0; f < 4; ++f) {
+                    const int r = r0 + wrow + 16 * mi + g8 + (f >= 2 ? 8 : 0);
+                    const int kx = k0 + wcol + 8 * ni + 2 * t4 + (f & 1);
+                    if (r >= nm || kx >= nm) continue;
+                    dst[oa + (size_t)r * nm + kx] = accA[mi * 4 + ni][f];
+                    if (m > 0) dst[ob + (size_t)r * nm + kx] = accB[mi * 4 + ni][f];
+                }
+    } else {
+#pragma unroll
+        for (int a = 0; a < 8; ++a) {
+            const int r = r0 + ty * 8 + a;
+            if (r >= nm) continue;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const int kx = k0 + tx * 4 + c;
+                if (kx >= nm) continue;
+                dst[oa + (size_t)r * nm + kx] = accA[a][c];
+                if (m > 0) dst[ob + (size_t)r * nm + kx] = accB[a][c];
+            }
         }
     }
 }
@@ -840,12 +943,12 @@ cudaError_t launch_node(const BwdParams& P, size_t smem, int grid, cudaStream_t 
     return cudaGetLastError();
 }
 
-template <int L, typename T>
+template <int L, typename T, bool TC>
 cudaError_t launch_dw(const BwdParams& P, int n_tiles, size_t smem, cudaStream_t s) {
-    cudaError_t e = cudaFuncSetAttribute(k_bwd_dw<L, T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = cudaFuncSetAttribute(k_bwd_dw<L, T, TC>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     count_launch();
-    k_bwd_dw<L, T><<<n_tiles, kNt, smem, s>>>(P);
+    k_bwd_dw<L, T, TC><<<n_tiles, kNt, smem, s>>>(P);
     return cudaGetLastError();
 }
 
@@ -856,8 +959,7 @@ size_t bwd_partial_bytes(int L, int C, int M) { return 4 * bwd::dw_part_floats(L
 
 bool bwd_supported(int L, int C, int H, int n_rbf) {
     if (L < 0 || L > kMaxL || bwd::kNt % H != 0 || bwd::kNodeNt % H != 0) return false;
-    return bwd::node_smem_floats(L, C, H, n_rbf) * 4 <= 227 * 1024 &&
-           bwd::dw_smem_floats(L, H, n_rbf) * 4 <= 227 * 1024;
+    return bwd::node_smem_floats(L, C, H, n_rbf) * 4 <= 227 * 1024 && bwd::dw_smem_bytes(H, n_rbf, false) <= 227 * 1024;
 }
 
 cudaError_t run_attention_bwd(const BwdArgs& b, cudaStream_t s) {
@@ -916,10 +1018,10 @@ cudaError_t run_attention_bwd(const BwdArgs& b, cudaStream_t s) {
     E2F_CUDA_TRY_E(cudaGetLastError());
     if (b.gWso2 && a.n_pairs > 0) {
         const int nt = n_dw_tiles(L, C, a.M) * kDwSplit;
-        const size_t dsm = dw_smem_floats(L, H, a.n_rbf) * 4;
+        const size_t dsm = dw_smem_bytes(H, a.n_rbf, a.bf16);
 #define E2F_BWD_DW(LL)                                                                                         \
     case LL:                                                                                                   \
-        e = a.bf16 ? launch_dw<LL, __nv_bfloat16>(P, nt, dsm, s) : launch_dw<LL, float>(P, nt, dsm, s); \
+        e = a.bf16 ? launch_dw<LL, __nv_bfloat16, true>(P, nt, dsm, s) : launch_dw<LL, float, false>(P, nt, dsm, s); \
         break;
         switch (L) {
             E2F_BWD_DW(0)

@@ -80,10 +80,13 @@ def test_backward_matches_the_oracle(L, C, H, n_rbf, dtype, periodic, n, M):
     _, ref = layer_grads(L, C, H, n_rbf, h["cutoff"], h["pos"].astype(np.float64), h["box"], h["rp"], h["col"],
                          h["x64"], h["Wq"], h["Wk"], h["Wrad"], h["w64"], h["G"], M=M)
     names = {"pos": "pos", "x": "x", "W_q": "Wq", "W_k": "Wk", "W_rad": "Wrad", "W_so2": "Wso2"}
-    # fp32 arithmetic throughout (measured 0.4-2e-6 normwise on these cases): 1e-5
+    # fp32 arithmetic (measured 0.3-1.4e-6 normwise on these cases): 1e-5. With bf16 storage
+    # the SO(2) weight gradient's contraction runs on tensor cores with fp16 operands
+    # (relative rounding 2^-11 per operand, fp32 accumulation): 2e-3 for that gradient.
     for k, rk in names.items():
         err = _rel(g[k].cpu().numpy().reshape(ref[rk].shape), ref[rk])
-        assert err <= 1e-5, (k, err)
+        tol = 2e-3 if (k == "W_so2" and dtype == "bf16") else 1e-5
+        assert err <= tol, (k, err)
 
 
 def test_backward_isolated_node_and_position_gradient_only():
