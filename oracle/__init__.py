@@ -13,8 +13,8 @@ Memory" (arXiv 2601.16622), as summarised on the gist.science page,
 Technical Summary section 2 (2.1 EAAS with Lemma 4.1 and the re-indexing
 rule Eq. 13; 2.2 node-centric factorisation Eq. 6, streaming reduction,
 online softmax) and the fugumt abstract page. The pages print no formula;
-every reading taken where they are silent is listed in the design doc and in the
-docstring of the function that implements it.
+every reading taken where they are silent is stated in the docstring of the
+function that implements it.
 
 Modules:
   sh         real spherical harmonics (closed-form Legendre polynomials)
