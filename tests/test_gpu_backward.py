@@ -135,3 +135,36 @@ def test_backward_full_size_properties():
     fd = (loss(d.pos + eps * dirn) - loss(d.pos - eps * dirn)) / (2 * eps)
     an = (gp * dirn.double()).sum().item()
     assert abs(fd - an) <= 2e-2 * abs(an), (fd, an)
+
+
+def test_backward_batched_graphs_sampled():
+    # the 256-graph batch at full size; graphs do not interact, so the position and
+    # feature gradients of the first four graphs equal the oracle's on those graphs alone
+    d = DeviceInputs(2)
+    w = d.w
+    cfg = e2f.make_cfg(w.L, w.C, w.H, w.n_rbf, w.cutoff, w.dtype)
+    rp, col = e2f.e2f_build_neighbors(d.pos, d.box, w.cutoff, d.graph_ptr)
+    G = np.random.default_rng(21).normal(size=(w.n_atoms, w.K, w.C)).astype(np.float32)
+    g = e2f.e2f_onfly_attention_backward(cfg, d.pos, d.box, rp, col, d.x, d.Wq, d.Wk, d.Wrad, d.Wso2,
+                                         torch.from_numpy(G).to(d.pos.device), want_weights=False)
+    gptr = np.asarray(w.graph_ptr)
+    n_sub = int(gptr[4])
+    rp0, col0 = neighbors_bruteforce(w.pos[:n_sub], None, w.cutoff, gptr[:5])
+    wt = d.weights
+    x64 = np.asarray(d.x_f64).reshape(w.n_atoms, w.K, w.C)[:n_sub]
+    _, ref = layer_grads(w.L, w.C, w.H, w.n_rbf, w.cutoff, w.pos[:n_sub].astype(np.float64), None, rp0, col0,
+                         x64, wt.Wq, wt.Wk, wt.Wrad, wt.Wso2_f64, G[:n_sub])
+    assert _rel(g["pos"].cpu().numpy()[:n_sub], ref["pos"]) <= 1e-5
+    assert _rel(g["x"].cpu().numpy()[:n_sub], ref["x"]) <= 1e-5
+
+
+def test_backward_without_edges_is_zero():
+    h, t = _system(9, 8, 2, 16, 2, 8, "f32", False)
+    t["pos"] *= 50.0  # spread the atoms far beyond the cutoff
+    rp = torch.zeros(9, dtype=torch.int32, device=t["pos"].device)
+    col = torch.zeros(0, dtype=torch.int32, device=t["pos"].device)
+    cfg = e2f.make_cfg(2, 16, 2, 8, 5.0, "f32")
+    g = e2f.e2f_onfly_attention_backward(cfg, t["pos"], None, rp, col, t["x"], t["Wq"], t["Wk"], t["Wrad"],
+                                         t["Wso2"], t["G"])
+    for k, v in g.items():
+        assert torch.count_nonzero(v).item() == 0, k
