@@ -211,7 +211,7 @@ extern "C" void e2f_attention_set_kernel_events(void* start_event, void* stop_ev
 namespace {
 
 struct BwdWs {
-    size_t o_q, o_k, o_wt, o_lse, o_gq, o_gk, o_beta, o_part, bytes;
+    size_t o_q, o_k, o_wt, o_lse, o_gq, o_gk, o_beta, o_part, o_w16, bytes;
 };
 
 BwdWs bwd_layout(int64_t n_atoms, int64_t n_pairs, const e2f_attn_cfg& c) {
@@ -226,6 +226,7 @@ BwdWs bwd_layout(int64_t n_atoms, int64_t n_pairs, const e2f_attn_cfg& c) {
     w.o_gk = take(4 * (size_t)n_atoms * c.C);
     w.o_beta = take(4 * (size_t)n_pairs * c.H);
     w.o_part = take(bwd_partial_bytes(c.L, c.C, effective_mmax(c.L, c.m_max)));
+    w.o_w16 = c.feat_dtype == E2F_BF16 ? take(4 * so2_total(c.L, c.C, effective_mmax(c.L, c.m_max))) : 0;
     w.bytes = o;
     return w;
 }
@@ -293,6 +294,7 @@ extern "C" e2f_status e2f_onfly_attention_backward(const e2f_attn_cfg* cfg, cons
     b.gpos = grad_pos; b.gx = grad_x; b.gWq = grad_W_q; b.gWk = grad_W_k; b.gWrad = grad_W_rad;
     b.gWso2 = grad_W_so2;
     b.gWpart = reinterpret_cast<float*>(ws + L.o_part);
+    b.w16 = cfg->feat_dtype == E2F_BF16 ? ws + L.o_w16 : nullptr;
     E2F_CUDA_TRY(run_attention_bwd(b, stream));
     return E2F_OK;
 }

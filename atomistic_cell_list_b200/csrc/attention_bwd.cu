@@ -1,4 +1,7 @@
-// Backward of the on-the-fly equivariant attention (fp32 CUDA cores).
+// Backward of the on-the-fly equivariant attention. fp32 CUDA cores; with
+// bf16 storage the SO(2) maps, their transposes and the weight-gradient
+// contraction run on tensor cores (m16n8k16 mma.sync, fp16 operands, fp32
+// accumulation).
 //
 // The pages' conservative variant takes forces as the negative gradient of
 // the energy with respect to the positions (E2Former-V2, gist.science
@@ -26,9 +29,11 @@
 //   dpos_j += dLoss/dr,  dpos_i -= dLoss/dr  (r = mic(pos_j - pos_i)).
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <stdint.h>
 
 #include <algorithm>
+#include <type_traits>
 
 #include "attention.cuh"
 #include "common.cuh"
@@ -74,6 +79,8 @@ struct BwdParams {
     float* gx;         // [N, K, C]
     float* gWrad;      // [n_rbf, G]
     float* gW;         // packed like W
+    const __half* w16;   // W in fp16, row-major blocks (bf16 storage: tensor-core maps)
+    const __half* wt16;  // the same, each block transposed
     float* gWpart;     // [kDwSplit][so2 total] partial sums of gW
     int dw_tiles;      // tiles of the SO(2) blocks
 };
@@ -149,17 +156,40 @@ __device__ __forceinline__ Logit edge_logit(const BwdParams& P, int i, int j, in
     return Logit{ga * dot * inv, ga, dot};
 }
 
+// m16n8k16 fp16 x fp16 -> fp32 (A row-major 16 x 16, B col-major 16 x 8)
+__device__ __forceinline__ void mma16816(float* d, const uint32_t* a, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// A fragment (16 x 16, row-major source with row stride ld halves) of m16n8k16
+__device__ __forceinline__ void frag_a(const __half* src, int ld, int g8, int t4, uint32_t* a) {
+    const __half* p = src + (size_t)g8 * ld + 2 * t4;
+    a[0] = *reinterpret_cast<const uint32_t*>(p);
+    a[1] = *reinterpret_cast<const uint32_t*>(p + 8 * (size_t)ld);
+    a[2] = *reinterpret_cast<const uint32_t*>(p + 8);
+    a[3] = *reinterpret_cast<const uint32_t*>(p + 8 * (size_t)ld + 8);
+}
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
     return v;
 }
 
-size_t node_smem_floats(int L, int C, int H, int n_rbf) {
+// fp16 operand rows of the tensor-core maps: (L+1)C + 8 halves (conflict-free fragment loads)
+__host__ __device__ inline int node_np(int L, int C) { return (L + 1) * C + 8; }
+
+size_t node_smem_floats(int L, int C, int H, int n_rbf, bool tc) {
+    (void)tc;  // the fp16 operands of the tensor-core maps live in the fp32 X~ region
     const int K = n_sh(L), WS = wig_size(L), Gv = (L + 1) * C, G = Gv + H;
     const int KH = (L >= 1) ? std::max((L + 1) * C, 2 * L * C) : C;
+    const int KHS = std::max(KH, node_np(L, C));  // the X~ region also holds the fp16 operands
     return (size_t)K * C + 3ull * kTe * WS + 2ull * kTe * n_rbf + (size_t)kTe * G + (size_t)kTe * Gv +
-           2ull * kTe * H + 12ull * kTe + 3ull * KH * kTe + (size_t)n_rbf * G + C + 2ull * H + 4 + kTe +
+           2ull * kTe * H + 12ull * kTe + (size_t)(KHS + 2 * KH) * kTe + (size_t)n_rbf * G + C + 2ull * H + 4 + kTe +
            2ull * kNodeNt + kTe;
 }
 
@@ -189,7 +219,7 @@ __global__ void __launch_bounds__(kNodeNt, 1) k_bwd_node(BwdParams P) {
     float* beta = alpha + kTe * H;     // [te][H]
     float* geo = beta + kTe * H;       // [te][12]: r^ (3), d, R^T e_y (3), -R^T e_x (3), dL/deps_x, dL/deps_y
     float* hs = geo + 12 * kTe;        // [KH][te] gated rotated input of the |m| block
-    float* gy = hs + KH * kTe;         // [KH][te] D G_i, then dLoss/dY = alpha D G_i, of the block
+    float* gy = hs + max(KH, node_np(L, C)) * kTe;  // [KH][te] D G_i, then dLoss/dY = alpha D G_i
     float* yb = gy + KH * kTe;         // [KH][te] Y = F(X~) of the block
     float* gWr = yb + KH * kTe;        // [nr][G] this CTA's part of dW_rad
     float* gqi = gWr + nr * G;         // [C]
@@ -199,8 +229,15 @@ __global__ void __launch_bounds__(kNodeNt, 1) k_bwd_node(BwdParams P) {
     float* ddv = gpi + 4;              // [te]
     float* red = ddv + kTe;            // [2 kNodeNt]
     int* jn = reinterpret_cast<int*>(red + 2 * kNodeNt);  // [te]
+    // bf16 storage: the SO(2) maps and their transposes run as m16n8k16 tensor-core products
+    // with fp16 operands, [s][e][np] in the hs region: X~ until the maps are done, then dY
+    constexpr bool TC = std::is_same<T, __nv_bfloat16>::value;
+    const int np = node_np(L, C);
+    __half* hs16 = reinterpret_cast<__half*>(hs);
+    __half* gy16 = hs16;
 
     const int tid = threadIdx.x, nt = blockDim.x, lane = tid & 31, warp = tid >> 5;
+    const int g8 = lane >> 2, t4 = lane & 3, nwarp = nt / 32;
     const float inv = rsqrtf((float)dh);
     for (int t = tid; t < nr * G; t += nt) gWr[t] = 0.f;
 
@@ -324,14 +361,75 @@ __global__ void __launch_bounds__(kNodeNt, 1) k_bwd_node(BwdParams P) {
                         vp *= gv;
                         vm *= gv;
                     }
-                    hs[(size_t)r * kTe + e] = vp;
-                    if (m > 0) hs[(size_t)(nm + r) * kTe + e] = vm;
+                    if constexpr (TC) {
+                        hs16[(size_t)e * np + r] = __float2half_rn(vp);
+                        if (m > 0) hs16[(size_t)(kTe + e) * np + r] = __float2half_rn(vm);
+                    } else {
+                        hs[(size_t)r * kTe + e] = vp;
+                        if (m > 0) hs[(size_t)(nm + r) * kTe + e] = vm;
+                    }
                 }
                 __syncthreads();
                 // Y = F(X~) row by row; beta, the first direction term, dY = alpha D G_i
                 const float* At = P.Wt + so2_offset(L, C, m, 0);
                 const float* Bt = (m > 0) ? P.Wt + so2_offset(L, C, m, 1) : nullptr;
-                for (int r = tid; r < nm; r += nt) {
+                if constexpr (TC) {
+                    // Y+ = A X+ - B X-, Y- = B X+ + A X-: one warp per 16 rows, N = the tile's 8 edges
+                    const __half* Aw = P.w16 + so2_offset(L, C, m, 0);
+                    const __half* Bw = P.w16 + so2_offset(L, C, m, 1);
+                    for (int rb = warp; rb < nm / 16; rb += nwarp) {
+                        float yp[4] = {0.f, 0.f, 0.f, 0.f}, ym[4] = {0.f, 0.f, 0.f, 0.f};
+                        for (int k0 = 0; k0 < nm; k0 += 16) {
+                            uint32_t aa[4];
+                            frag_a(Aw + (size_t)(rb * 16) * nm + k0, nm, g8, t4, aa);
+                            const __half* xp = hs16 + (size_t)g8 * np + k0 + 2 * t4;
+                            const uint32_t xp0 = *reinterpret_cast<const uint32_t*>(xp);
+                            const uint32_t xp1 = *reinterpret_cast<const uint32_t*>(xp + 8);
+                            mma16816(yp, aa, xp0, xp1);
+                            if (m > 0) {
+                                uint32_t ab[4], an[4];
+                                frag_a(Bw + (size_t)(rb * 16) * nm + k0, nm, g8, t4, ab);
+#pragma unroll
+                                for (int q = 0; q < 4; ++q) an[q] = ab[q] ^ 0x80008000u;
+                                const __half* xm = hs16 + (size_t)(kTe + g8) * np + k0 + 2 * t4;
+                                const uint32_t xm0 = *reinterpret_cast<const uint32_t*>(xm);
+                                const uint32_t xm1 = *reinterpret_cast<const uint32_t*>(xm + 8);
+                                mma16816(yp, an, xm0, xm1);
+                                mma16816(ym, ab, xp0, xp1);
+                                mma16816(ym, aa, xm0, xm1);
+                            }
+                        }
+                        const int r = rb * 16 + g8;
+                        yb[(size_t)r * kTe + 2 * t4] = yp[0];
+                        yb[(size_t)r * kTe + 2 * t4 + 1] = yp[1];
+                        yb[(size_t)(r + 8) * kTe + 2 * t4] = yp[2];
+                        yb[(size_t)(r + 8) * kTe + 2 * t4 + 1] = yp[3];
+                        if (m > 0) {
+                            yb[(size_t)(nm + r) * kTe + 2 * t4] = ym[0];
+                            yb[(size_t)(nm + r) * kTe + 2 * t4 + 1] = ym[1];
+                            yb[(size_t)(nm + r + 8) * kTe + 2 * t4] = ym[2];
+                            yb[(size_t)(nm + r + 8) * kTe + 2 * t4 + 1] = ym[3];
+                        }
+                    }
+                    // D G_i rows of the block (unscaled)
+                    for (int t = tid; t < nm * kTe; t += nt) {
+                        const int r = t / kTe, e = t % kTe;
+                        const int l3 = m + r / C, c = r % C, w3 = 2 * l3 + 1;
+                        float gp = 0.f, gm = 0.f;
+                        if (e < ne) {
+                            const float* D = Dm + e * WS + wig_off(l3);
+                            const float* gi = Gi + (size_t)(l3 * l3) * C + c;
+                            for (int n = 0; n < w3; ++n) {
+                                const float gv = gi[(size_t)n * C];
+                                gp = fmaf(D[(l3 + m) * w3 + n], gv, gp);
+                                gm = fmaf(D[(l3 - m) * w3 + n], gv, gm);
+                            }
+                        }
+                        gy[(size_t)r * kTe + e] = gp;
+                        if (m > 0) gy[(size_t)(nm + r) * kTe + e] = gm;
+                    }
+                }
+                for (int r = tid; r < (TC ? 0 : nm); r += nt) {
                     const int l3 = m + r / C, c = r % C;
                     float op[kTe], om[kTe];
 #pragma unroll
@@ -436,9 +534,52 @@ __global__ void __launch_bounds__(kNodeNt, 1) k_bwd_node(BwdParams P) {
                 for (int t = tid; t < (m > 0 ? 2 : 1) * nm * kTe; t += nt) {
                     const int rr = t / kTe, e = t % kTe;
                     const int c = (rr % nm) % C;
-                    gy[t] *= alpha[e * H + c / dh];
+                    const float v = gy[t] * alpha[e * H + c / dh];
+                    gy[t] = v;
+                    if constexpr (TC) gy16[(size_t)((rr / nm) * kTe + e) * np + rr % nm] = __float2half_rn(v);
                 }
                 __syncthreads();
+                if constexpr (TC) {
+                    // dX+ = A^T dY+ + B^T dY-, dX- = -B^T dY+ + A^T dY-: one warp per 16 columns,
+                    // into the Y buffer (Y is no longer needed) as [s][column][edge]
+                    const __half* At16 = P.wt16 + so2_offset(L, C, m, 0);
+                    const __half* Bt16 = P.wt16 + so2_offset(L, C, m, 1);
+                    for (int cb = warp; cb < nm / 16; cb += nwarp) {
+                        float dxp[4] = {0.f, 0.f, 0.f, 0.f}, dxm[4] = {0.f, 0.f, 0.f, 0.f};
+                        for (int r0 = 0; r0 < nm; r0 += 16) {
+                            uint32_t aa[4];
+                            frag_a(At16 + (size_t)(cb * 16) * nm + r0, nm, g8, t4, aa);
+                            const __half* yp = gy16 + (size_t)g8 * np + r0 + 2 * t4;
+                            const uint32_t yp0 = *reinterpret_cast<const uint32_t*>(yp);
+                            const uint32_t yp1 = *reinterpret_cast<const uint32_t*>(yp + 8);
+                            mma16816(dxp, aa, yp0, yp1);
+                            if (m > 0) {
+                                uint32_t ab[4], an[4];
+                                frag_a(Bt16 + (size_t)(cb * 16) * nm + r0, nm, g8, t4, ab);
+#pragma unroll
+                                for (int q = 0; q < 4; ++q) an[q] = ab[q] ^ 0x80008000u;
+                                const __half* ym = gy16 + (size_t)(kTe + g8) * np + r0 + 2 * t4;
+                                const uint32_t ym0 = *reinterpret_cast<const uint32_t*>(ym);
+                                const uint32_t ym1 = *reinterpret_cast<const uint32_t*>(ym + 8);
+                                mma16816(dxp, ab, ym0, ym1);
+                                mma16816(dxm, an, yp0, yp1);
+                                mma16816(dxm, aa, ym0, ym1);
+                            }
+                        }
+                        const int k = cb * 16 + g8;
+                        yb[(size_t)k * kTe + 2 * t4] = dxp[0];
+                        yb[(size_t)k * kTe + 2 * t4 + 1] = dxp[1];
+                        yb[(size_t)(k + 8) * kTe + 2 * t4] = dxp[2];
+                        yb[(size_t)(k + 8) * kTe + 2 * t4 + 1] = dxp[3];
+                        if (m > 0) {
+                            yb[(size_t)(nm + k) * kTe + 2 * t4] = dxm[0];
+                            yb[(size_t)(nm + k) * kTe + 2 * t4 + 1] = dxm[1];
+                            yb[(size_t)(nm + k + 8) * kTe + 2 * t4] = dxm[2];
+                            yb[(size_t)(nm + k + 8) * kTe + 2 * t4 + 1] = dxm[3];
+                        }
+                    }
+                    __syncthreads();
+                }
                 // dX~ = F^T(dY) column by column, and what it feeds: dx_j, dg_v, the second direction term
                 const size_t oa = so2_offset(L, C, m, 0), ob = so2_offset(L, C, m, 1);
                 float t2x[kTe], t2y[kTe];
@@ -448,8 +589,11 @@ __global__ void __launch_bounds__(kNodeNt, 1) k_bwd_node(BwdParams P) {
                     const int l1 = m + kc / C, c = kc % C;
                     float dp[kTe], dq[kTe];
 #pragma unroll
-                    for (int e = 0; e < kTe; ++e) { dp[e] = 0.f; dq[e] = 0.f; }
-                    for (int r = 0; r < nm; ++r) {
+                    for (int e = 0; e < kTe; ++e) {
+                        dp[e] = TC ? yb[(size_t)kc * kTe + e] : 0.f;
+                        dq[e] = (TC && m > 0) ? yb[(size_t)(nm + kc) * kTe + e] : 0.f;
+                    }
+                    for (int r = 0; r < (TC ? 0 : nm); ++r) {
                         const float a = load_feat(W, oa + (size_t)r * nm + kc);
                         const float4* yp4 = reinterpret_cast<const float4*>(gy + (size_t)r * kTe);
                         if (m == 0) {
@@ -639,15 +783,6 @@ int n_dw_tiles(int L, int C, int M) {
         n += ((nm + kDwR - 1) / kDwR) * ((nm + kDwC - 1) / kDwC);
     }
     return n;
-}
-
-// m16n8k16 fp16 x fp16 -> fp32 (A row-major 16 x 16, B col-major 16 x 8)
-__device__ __forceinline__ void mma16816(float* d, const uint32_t* a, uint32_t b0, uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-        "{%0,%1,%2,%3};"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
 // TC = false: fp32 operands and FMA accumulation (thread tile 8 x 4).
@@ -894,6 +1029,26 @@ __global__ void __launch_bounds__(kNt, 2) k_bwd_dw(BwdParams P) {
     }
 }
 
+// Packed SO(2) weights -> fp16, row-major blocks (w16) and each block transposed (wt16)
+template <typename T>
+__global__ void k_bwd_w16(const T* __restrict__ w, int L, int C, int M, __half* w16, __half* wt16) {
+    const size_t total = so2_total(L, C, M);
+    for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += (size_t)gridDim.x * blockDim.x) {
+        size_t off = 0;
+        int n = (L + 1) * C, blk = 0;
+        while (e >= off + (size_t)n * n) {
+            off += (size_t)n * n;
+            ++blk;
+            n = (L + 1 - (blk + 1) / 2) * C;
+        }
+        const size_t loc = e - off;
+        const int r = (int)(loc / n), k = (int)(loc % n);
+        const __half v = __float2half_rn(load_feat(w, e));
+        w16[e] = v;
+        wt16[off + (size_t)k * n + r] = v;
+    }
+}
+
 // gW = the edge-range partial sums, added in a fixed order
 __global__ void k_bwd_dw_sum(const float* __restrict__ part, size_t total, float* out) {
     for (size_t t = (size_t)blockIdx.x * blockDim.x + threadIdx.x; t < total; t += (size_t)gridDim.x * blockDim.x) {
@@ -959,7 +1114,8 @@ size_t bwd_partial_bytes(int L, int C, int M) { return 4 * bwd::dw_part_floats(L
 
 bool bwd_supported(int L, int C, int H, int n_rbf) {
     if (L < 0 || L > kMaxL || bwd::kNt % H != 0 || bwd::kNodeNt % H != 0) return false;
-    return bwd::node_smem_floats(L, C, H, n_rbf) * 4 <= 227 * 1024 && bwd::dw_smem_bytes(H, n_rbf, false) <= 227 * 1024;
+    return bwd::node_smem_floats(L, C, H, n_rbf, true) * 4 <= 227 * 1024 &&
+           bwd::dw_smem_bytes(H, n_rbf, false) <= 227 * 1024;
 }
 
 cudaError_t run_attention_bwd(const BwdArgs& b, cudaStream_t s) {
@@ -987,7 +1143,16 @@ cudaError_t run_attention_bwd(const BwdArgs& b, cudaStream_t s) {
     int dev = 0, n_sm = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
-    const size_t smem = node_smem_floats(L, C, H, a.n_rbf) * 4;
+    const size_t smem = node_smem_floats(L, C, H, a.n_rbf, a.bf16) * 4;
+    if (a.bf16) {
+        P.w16 = static_cast<const __half*>(b.w16);
+        P.wt16 = P.w16 + so2_total(L, C, a.M);
+        count_launch();
+        k_bwd_w16<__nv_bfloat16><<<592, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(a.Wso2), L, C, a.M,
+                                                      static_cast<__half*>(b.w16),
+                                                      static_cast<__half*>(b.w16) + so2_total(L, C, a.M));
+        E2F_CUDA_TRY_E(cudaGetLastError());
+    }
     const int grid = std::max(1, std::min(N, n_sm));
 #define E2F_BWD_NODE(LL)                                                                                     \
     case LL:                                                                                                 \

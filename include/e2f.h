@@ -281,10 +281,13 @@ e2f_status e2f_onfly_attention_cells(const e2f_attn_cfg* cfg, const float* pos,
  *               a sweep over all edges per 64 x 64 tile of the SO(2) blocks).
  *   workspace   device, >= e2f_attention_backward_workspace_size(...)
  *               bytes, 256-byte aligned.
- * All arithmetic is fp32 on CUDA cores (a tensor-core backward is not
- * built). Gradients that sum over edges use fp32 atomics, so their last
- * bits may differ between runs; grad_W_so2, grad_W_q and grad_W_k are
- * deterministic. Shapes: those of e2f_onfly_attention with H dividing 256
+ * Arithmetic: with fp32 storage, fp32 on CUDA cores throughout. With bf16
+ * storage, the SO(2) maps, their transposes and the SO(2) weight-gradient
+ * contraction run on tensor cores (mma.sync) with fp16 operands and fp32
+ * accumulation (about 3e-4 relative error against an exact evaluation);
+ * the rest stays fp32. Gradients that sum over edges use fp32 atomics, so
+ * their last bits may differ between runs; grad_W_so2, grad_W_q and
+ * grad_W_k are deterministic. Shapes: those of e2f_onfly_attention with H dividing 256
  * and the kernels' shared memory within 227 KB (L = 4 allows C <= 128);
  * otherwise E2F_ERR_UNSUPPORTED. Asynchronous.
  * ---------------------------------------------------------------------- */

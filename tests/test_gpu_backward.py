@@ -80,12 +80,13 @@ def test_backward_matches_the_oracle(L, C, H, n_rbf, dtype, periodic, n, M):
     _, ref = layer_grads(L, C, H, n_rbf, h["cutoff"], h["pos"].astype(np.float64), h["box"], h["rp"], h["col"],
                          h["x64"], h["Wq"], h["Wk"], h["Wrad"], h["w64"], h["G"], M=M)
     names = {"pos": "pos", "x": "x", "W_q": "Wq", "W_k": "Wk", "W_rad": "Wrad", "W_so2": "Wso2"}
-    # fp32 arithmetic (measured 0.3-1.4e-6 normwise on these cases): 1e-5. With bf16 storage
-    # the SO(2) weight gradient's contraction runs on tensor cores with fp16 operands
-    # (relative rounding 2^-11 per operand, fp32 accumulation): 2e-3 for that gradient.
+    # fp32 storage: fp32 arithmetic (measured 0.3-1.4e-6 normwise): 1e-5. bf16 storage: the
+    # SO(2) maps, their transposes and the weight-gradient contraction run on tensor cores
+    # with fp16 operands (relative rounding 2^-11 per operand, fp32 accumulation; measured
+    # 1.3-4.2e-4 normwise): 2e-3.
+    tol = 2e-3 if dtype == "bf16" else 1e-5
     for k, rk in names.items():
         err = _rel(g[k].cpu().numpy().reshape(ref[rk].shape), ref[rk])
-        tol = 2e-3 if (k == "W_so2" and dtype == "bf16") else 1e-5
         assert err <= tol, (k, err)
 
 
@@ -154,8 +155,9 @@ def test_backward_batched_graphs_sampled():
     x64 = np.asarray(d.x_f64).reshape(w.n_atoms, w.K, w.C)[:n_sub]
     _, ref = layer_grads(w.L, w.C, w.H, w.n_rbf, w.cutoff, w.pos[:n_sub].astype(np.float64), None, rp0, col0,
                          x64, wt.Wq, wt.Wk, wt.Wrad, wt.Wso2_f64, G[:n_sub])
-    assert _rel(g["pos"].cpu().numpy()[:n_sub], ref["pos"]) <= 1e-5
-    assert _rel(g["x"].cpu().numpy()[:n_sub], ref["x"]) <= 1e-5
+    # bf16 storage: tensor-core maps with fp16 operands (see test_backward_matches_the_oracle)
+    assert _rel(g["pos"].cpu().numpy()[:n_sub], ref["pos"]) <= 2e-3
+    assert _rel(g["x"].cpu().numpy()[:n_sub], ref["x"]) <= 2e-3
 
 
 def test_backward_without_edges_is_zero():
