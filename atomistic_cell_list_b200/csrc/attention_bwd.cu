@@ -839,6 +839,21 @@ __global__ void __launch_bounds__(kNt, 2) k_bwd_dw(BwdParams P) {
         const int kb = t / kDwC, kx = k0 + t % kDwC;
         wr[t] = (kx < nm) ? P.Wrad[(size_t)kb * G + (m + kx / C) * C + kx % C] : 0.f;
     }
+    // this thread's operand roles (fixed for the CTA): dY row (sign y_s, row y_q) and X~ column
+    // (sign x_s, column x_q, edges of parity x_half); offsets into a node's [K][C] row, into
+    // an edge's Wigner rows, the degree's width and the head
+    const int y_s = tid / kDwR, y_q = tid % kDwR, ry = r0 + y_q;
+    const bool y_ok = y_s < nrow && ry < nm;
+    const int y_l = m + (y_ok ? ry / C : 0), y_c = y_ok ? ry % C : 0;
+    const int y_g = y_l * y_l * C + y_c, y_w = 2 * y_l + 1, y_d = y_ok ? drow_off(m, y_l, y_s) : 0;
+    const int y_h = y_c / dh;
+    const int x_role = tid % (2 * kDwC), x_half = tid / (2 * kDwC);
+    const int x_s = x_role / kDwC, x_q = x_role % kDwC, kxx = k0 + x_q;
+    const bool x_ok = x_s < nrow && kxx < nm;
+    const int x_l = m + (x_ok ? kxx / C : 0), x_c = x_ok ? kxx % C : 0;
+    const int x_g = x_l * x_l * C + x_c, x_w = 2 * x_l + 1, x_d = x_ok ? drow_off(m, x_l, x_s) : 0;
+    static_assert(2 * kDwR == kNt && 4 * kDwC == kNt, "operand roles: one dY row per thread, two threads per X~ column");
+
     const int e_lo = (int)((long long)P.n_pairs * split / kDwSplit);
     const int e_hi = (int)((long long)P.n_pairs * (split + 1) / kDwSplit);
     for (int c0 = e_lo; c0 < e_hi; c0 += kDwChunk) {
@@ -882,50 +897,54 @@ __global__ void __launch_bounds__(kNt, 2) k_bwd_dw(BwdParams P) {
         __syncthreads();
         for (int s0 = 0; s0 < nc; s0 += kDwE) {
             const int ns = min(kDwE, nc - s0);
-            // operands of the sub-chunk: dY rows r0.., X~ columns k0..
-            for (int t = tid; t < 2 * kDwE * kDwR; t += kNt) {
-                const int s2 = t / (kDwE * kDwR), rem = t % (kDwE * kDwR);
-                const int e = rem / kDwR, q = rem % kDwR, ry = r0 + q;
-                float v = 0.f;
-                if (e < ns && s2 < nrow && ry < nm) {
-                    const int el = s0 + e;
-                    const int l3 = m + ry / C, c = ry % C, w = 2 * l3 + 1;
-                    const float* dr = drow + el * 50 + drow_off(m, l3, s2);
-                    const float* gi = P.G + ((size_t)ei[el] * K + l3 * l3) * C + c;
-                    float gr[2 * L + 1];  // all loads issued before the arithmetic
+            // operands of the sub-chunk: dY rows r0.. (thread = one (sign, row)), X~ columns
+            // k0.. (thread = one (sign, column) and every other edge); G_i stays in registers
+            // while consecutive edges share their node
+            {
+                int cached = -1;
+                float gr[2 * L + 1];
 #pragma unroll
-                    for (int n = 0; n < 2 * L + 1; ++n) gr[n] = (n < w) ? gi[(size_t)n * C] : 0.f;
-                    float acc = 0.f;
+                for (int n = 0; n < 2 * L + 1; ++n) gr[n] = 0.f;
+                for (int e = 0; e < kDwE; ++e) {
+                    float v = 0.f;
+                    if (e < ns && y_ok) {
+                        const int el = s0 + e, node = ei[el];
+                        if (node != cached) {
+                            const float* gi = P.G + (size_t)node * K * C + y_g;
 #pragma unroll
-                    for (int n = 0; n < 2 * L + 1; ++n)
-                        if (n < w) acc = fmaf(dr[n], gr[n], acc);
-                    v = alpha[el * H + c / dh] * acc;
+                            for (int n = 0; n < 2 * L + 1; ++n) gr[n] = (n < y_w) ? gi[(size_t)n * C] : 0.f;
+                            cached = node;
+                        }
+                        const float* dr = drow + el * 50 + y_d;
+                        float acc = 0.f;
+#pragma unroll
+                        for (int n = 0; n < 2 * L + 1; ++n)
+                            if (n < y_w) acc = fmaf(dr[n], gr[n], acc);
+                        v = alpha[el * H + y_h] * acc;
+                    }
+                    if constexpr (TC) Ys[(y_s * kDwR + y_q) * kDwStrideH + e] = __float2half_rn(v);
+                    else Yop[(y_s * kDwE + e) * kDwR + y_q] = v;
                 }
-                if constexpr (TC) Ys[(s2 * kDwR + q) * kDwStrideH + e] = __float2half_rn(v);
-                else Yop[t] = v;
-            }
-            for (int t = tid; t < 2 * kDwE * kDwC; t += kNt) {
-                const int s2 = t / (kDwE * kDwC), rem = t % (kDwE * kDwC);
-                const int e = rem / kDwC, q = rem % kDwC, kx = k0 + q;
-                float v = 0.f;
-                if (e < ns && s2 < nrow && kx < nm) {
-                    const int el = s0 + e;
-                    const int l1 = m + kx / C, c = kx % C, w = 2 * l1 + 1;
-                    const float* dr = drow + el * 50 + drow_off(m, l1, s2);
-                    const size_t xb = ((size_t)ej[el] * K + l1 * l1) * C + c;
-                    float xr[2 * L + 1];  // all loads issued before the arithmetic
+                for (int e = x_half; e < kDwE; e += 2) {
+                    float v = 0.f;
+                    if (e < ns && x_ok) {
+                        const int el = s0 + e;
+                        const size_t xb = (size_t)ej[el] * K * C + x_g;
+                        float xr[2 * L + 1];  // all loads issued before the arithmetic
 #pragma unroll
-                    for (int n = 0; n < 2 * L + 1; ++n) xr[n] = (n < w) ? load_feat(x, xb + (size_t)n * C) : 0.f;
-                    float acc = 0.f;
+                        for (int n = 0; n < 2 * L + 1; ++n) xr[n] = (n < x_w) ? load_feat(x, xb + (size_t)n * C) : 0.f;
+                        const float* dr = drow + el * 50 + x_d;
+                        float acc = 0.f;
 #pragma unroll
-                    for (int n = 0; n < 2 * L + 1; ++n)
-                        if (n < w) acc = fmaf(dr[n], xr[n], acc);
-                    float gv = 0.f;
-                    for (int kb = 0; kb < nr; ++kb) gv = fmaf(rho[el * nr + kb], wr[kb * kDwC + q], gv);
-                    v = gv * acc;
+                        for (int n = 0; n < 2 * L + 1; ++n)
+                            if (n < x_w) acc = fmaf(dr[n], xr[n], acc);
+                        float gv = 0.f;
+                        for (int kb = 0; kb < nr; ++kb) gv = fmaf(rho[el * nr + kb], wr[kb * kDwC + x_q], gv);
+                        v = gv * acc;
+                    }
+                    if constexpr (TC) Xs[(x_s * kDwC + x_q) * kDwStrideH + e] = __float2half_rn(v);
+                    else Xop[(x_s * kDwE + e) * kDwC + x_q] = v;
                 }
-                if constexpr (TC) Xs[(s2 * kDwC + q) * kDwStrideH + e] = __float2half_rn(v);
-                else Xop[t] = v;
             }
             __syncthreads();
             if constexpr (TC) {
