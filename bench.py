@@ -542,7 +542,9 @@ def run_naive(args):
 def run_backward(args):
     """The attention's backward (e2f_onfly_attention_backward) on the bench workload: all
     gradients (positions, features, every weight), and positions + features + W_rad only
-    (what forces need). fp32 CUDA-core kernels: the roofline is the FP32 FMA pipe."""
+    (what forces need). With bf16 storage the contractions run on tensor cores (mma.sync);
+    the per-edge rebuild of their operands (rotations, gates) on the FP32 pipe bounds the
+    kernels, so the roofline reported is the FP32 FMA pipe's."""
     import torch
 
     import atomistic_cell_list_b200 as e2f
@@ -604,7 +606,8 @@ def run_backward(args):
             "roofline": {"bound": "alu", "achieved": res["all"]["tflops"], "peak": fma_peak, "unit": "TFLOP/s",
                          "frac": res["all"]["tflops"] / fma_peak, "traffic": None,
                          "peak_note": f"fp32 FMA pipe: 148 SMs x 128 lanes x 2 FLOP x {clk_max:.0f} MHz "
-                                      f"(derived, {peak_src} clock)",
+                                      f"(derived, {peak_src} clock); the contractions themselves run on "
+                                      f"tensor cores for bf16 storage",
                          "units_per_launch": f"{E} edges x 3 x {F} SO(2) FLOP"},
             "clocks": res["all"]["clocks"]}
     print(json.dumps(line), flush=True)
