@@ -379,6 +379,7 @@ __global__ void __launch_bounds__(kNodeNt, 1) k_bwd_node(BwdParams P) {
                     const __half* Bw = P.w16 + so2_offset(L, C, m, 1);
                     for (int rb = warp; rb < nm / 16; rb += nwarp) {
                         float yp[4] = {0.f, 0.f, 0.f, 0.f}, ym[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
                         for (int k0 = 0; k0 < nm; k0 += 16) {
                             uint32_t aa[4];
                             frag_a(Aw + (size_t)(rb * 16) * nm + k0, nm, g8, t4, aa);
@@ -546,6 +547,7 @@ __global__ void __launch_bounds__(kNodeNt, 1) k_bwd_node(BwdParams P) {
                     const __half* Bt16 = P.wt16 + so2_offset(L, C, m, 1);
                     for (int cb = warp; cb < nm / 16; cb += nwarp) {
                         float dxp[4] = {0.f, 0.f, 0.f, 0.f}, dxm[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
                         for (int r0 = 0; r0 < nm; r0 += 16) {
                             uint32_t aa[4];
                             frag_a(At16 + (size_t)(cb * 16) * nm + r0, nm, g8, t4, aa);
