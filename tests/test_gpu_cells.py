@@ -6,6 +6,7 @@ import pytest
 import torch
 
 import atomistic_cell_list_b200 as e2f
+import workloads as W
 from gpu_util import TOL, DeviceInputs, oracle_csr, rel_err_per_degree
 
 pytestmark = pytest.mark.gpu
@@ -66,4 +67,18 @@ def test_fused_traversal_dense_nodes():
     assert deg.min() > 256 and deg.max() > 512
     csr = e2f.e2f_onfly_attention(cfg, pos, box, rp, col, x, d.Wq, d.Wk, d.Wrad, d.Wso2)
     fused = e2f.e2f_onfly_attention_cells(cfg, pos, box, x, d.Wq, d.Wk, d.Wrad, d.Wso2)
+    assert rel_err_per_degree(fused.cpu().numpy(), csr.cpu().numpy(), w.L) <= 1e-3
+
+
+def test_fused_traversal_with_truncated_maps():
+    # m_max < L: the fused call and the CSR call apply the same truncated layer
+    d = DeviceInputs(3)
+    w = d.w
+    M = 2
+    cfg = e2f.make_cfg(w.L, w.C, w.H, w.n_rbf, w.cutoff, w.dtype, m_max=M)
+    n_so2 = sum(W.so2_block_sizes(w.L, w.C)[:2 * M + 1])
+    wso2 = d.Wso2[:n_so2].contiguous()
+    rp, col = e2f.e2f_build_neighbors(d.pos, d.box, w.cutoff)
+    csr = e2f.e2f_onfly_attention(cfg, d.pos, d.box, rp, col, d.x, d.Wq, d.Wk, d.Wrad, wso2)
+    fused = e2f.e2f_onfly_attention_cells(cfg, d.pos, d.box, d.x, d.Wq, d.Wk, d.Wrad, wso2)
     assert rel_err_per_degree(fused.cpu().numpy(), csr.cpu().numpy(), w.L) <= 1e-3
