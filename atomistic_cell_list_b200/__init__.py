@@ -258,7 +258,7 @@ def e2f_attention_backward_workspace_size(n_atoms: int, n_pairs: int, cfg: e2f_a
 
 def e2f_onfly_attention_backward(cfg: e2f_attn_cfg, pos, box, row_ptr, col, x, W_q, W_k, W_rad, W_so2, grad_out,
                                  want_weights: bool = True, workspace: torch.Tensor | None = None,
-                                 out: dict | None = None, stream=None) -> dict:
+                                 out: dict | None = None, stream=None, check: bool = True) -> dict:
     """Gradients of sum(grad_out * layer(...)) (see include/e2f.h): a dict with
     pos, x, W_rad and, when want_weights, W_q, W_k, W_so2 (all fp32)."""
     _need_cuda(pos, row_ptr, col, x, W_q, W_k, W_rad, W_so2, grad_out, workspace)
@@ -283,6 +283,9 @@ def e2f_onfly_attention_backward(cfg: e2f_attn_cfg, pos, box, row_ptr, col, x, W
         _ptr(g.get("W_k")), _ptr(g["W_rad"]), _ptr(g.get("W_so2")), _ptr(workspace), workspace.numel(),
         _stream(stream))
     _check(code, "e2f_onfly_attention_backward")
+    if check:
+        _check(lib().e2f_attention_status(_ptr(workspace), workspace.numel(), _stream(stream)),
+               "e2f_onfly_attention_backward (device)")
     return g
 
 

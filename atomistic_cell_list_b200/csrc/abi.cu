@@ -211,13 +211,14 @@ extern "C" void e2f_attention_set_kernel_events(void* start_event, void* stop_ev
 namespace {
 
 struct BwdWs {
-    size_t o_q, o_k, o_wt, o_lse, o_gq, o_gk, o_beta, o_part, o_w16, bytes;
+    size_t o_status, o_q, o_k, o_wt, o_lse, o_gq, o_gk, o_beta, o_part, o_w16, bytes;
 };
 
 BwdWs bwd_layout(int64_t n_atoms, int64_t n_pairs, const e2f_attn_cfg& c) {
     BwdWs w{};
     size_t o = 0;
     auto take = [&](size_t b) { size_t r = o; o = align_up(o + b, 256); return r; };
+    w.o_status = take(256);  // first, as in the forward layout: e2f_attention_status reads it
     w.o_q = take(4 * (size_t)n_atoms * c.C);
     w.o_k = take(4 * (size_t)n_atoms * c.C);
     w.o_wt = take(4 * so2_total(c.L, c.C, effective_mmax(c.L, c.m_max)));
@@ -295,6 +296,8 @@ extern "C" e2f_status e2f_onfly_attention_backward(const e2f_attn_cfg* cfg, cons
     b.gWso2 = grad_W_so2;
     b.gWpart = reinterpret_cast<float*>(ws + L.o_part);
     b.w16 = cfg->feat_dtype == E2F_BF16 ? ws + L.o_w16 : nullptr;
+    b.status = reinterpret_cast<int*>(ws + L.o_status);
+    E2F_CUDA_TRY(cudaMemsetAsync(b.status, 0, sizeof(int), stream));
     E2F_CUDA_TRY(run_attention_bwd(b, stream));
     return E2F_OK;
 }

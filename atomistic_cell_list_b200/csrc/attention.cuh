@@ -81,6 +81,7 @@ struct BwdArgs {
     float* gWso2;
     float* gWpart;  // bwd_partial_bytes(L, C, M) of scratch for gWso2
     void* w16;      // bf16 storage: 4 so2_total(L, C, M) bytes for fp16 copies of W_so2
+    int* status;    // device status word (cleared by the caller)
 };
 bool bwd_supported(int L, int C, int H, int n_rbf);
 size_t bwd_partial_bytes(int L, int C, int M);

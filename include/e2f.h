@@ -280,7 +280,9 @@ e2f_status e2f_onfly_attention_cells(const e2f_attn_cfg* cfg, const float* pos,
  *               written; NULL skips it (its kernel is the costliest part:
  *               a sweep over all edges per 64 x 64 tile of the SO(2) blocks).
  *   workspace   device, >= e2f_attention_backward_workspace_size(...)
- *               bytes, 256-byte aligned.
+ *               bytes, 256-byte aligned. Its status word (a bounded
+ *               device-side wait that ran out: E2F_ERR_TIMEOUT) is read
+ *               with e2f_attention_status, as for the forward.
  * Arithmetic: with fp32 storage, fp32 on CUDA cores throughout. With bf16
  * storage, the SO(2) maps, their transposes and the SO(2) weight-gradient
  * contraction run on tensor cores (mma.sync) with fp16 operands and fp32
