@@ -54,7 +54,8 @@ def measured_peaks():
 # bench reports traffic null.
 KERNEL_TRAFFIC = {
     "sources": ["atomistic_cell_list_b200/csrc/attention_tc.cu", "atomistic_cell_list_b200/csrc/attention_tc.cuh",
-                "atomistic_cell_list_b200/csrc/common.cuh", "atomistic_cell_list_b200/csrc/cell_grid.cuh"],
+                "atomistic_cell_list_b200/csrc/common.cuh", "atomistic_cell_list_b200/csrc/cell_grid.cuh",
+                "atomistic_cell_list_b200/csrc/tcgen05.cuh"],
     "sha256": "6c372fe6c958e5ca70e7bc386a80e6e627d1d932666bea93348cd0b896c52b24",
     "dram_read_bytes": 44.27e9,
     "dram_write_bytes": 24.00e9,
