@@ -56,9 +56,9 @@ KERNEL_TRAFFIC = {
     "sources": ["atomistic_cell_list_b200/csrc/attention_tc.cu", "atomistic_cell_list_b200/csrc/attention_tc.cuh",
                 "atomistic_cell_list_b200/csrc/common.cuh", "atomistic_cell_list_b200/csrc/cell_grid.cuh",
                 "atomistic_cell_list_b200/csrc/tcgen05.cuh"],
-    "sha256": "6c372fe6c958e5ca70e7bc386a80e6e627d1d932666bea93348cd0b896c52b24",
-    "dram_read_bytes": 44.27e9,
-    "dram_write_bytes": 24.00e9,
+    "sha256": "cb5e3b21b5803839972cab0ab0c2f49a533fd3c16690a429eaab198324969eeb",
+    "dram_read_bytes": 44.33e9,
+    "dram_write_bytes": 23.98e9,
 }
 
 
