@@ -167,15 +167,6 @@ __device__ __forceinline__ void mma16816(float* d, const uint32_t* a, uint32_t b
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// A fragment (16 x 16, row-major source with row stride ld halves) of m16n8k16
-__device__ __forceinline__ void frag_a(const __half* src, int ld, int g8, int t4, uint32_t* a) {
-    const __half* p = src + (size_t)g8 * ld + 2 * t4;
-    a[0] = *reinterpret_cast<const uint32_t*>(p);
-    a[1] = *reinterpret_cast<const uint32_t*>(p + 8 * (size_t)ld);
-    a[2] = *reinterpret_cast<const uint32_t*>(p + 8);
-    a[3] = *reinterpret_cast<const uint32_t*>(p + 8 * (size_t)ld + 8);
-}
-
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
@@ -383,15 +374,16 @@ __global__ void __launch_bounds__(kNodeNt, 1) k_bwd_node(BwdParams P) {
                         float yp[4] = {0.f, 0.f, 0.f, 0.f}, ym[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 4
                         for (int k0 = 0; k0 < nm; k0 += 16) {
+                            const size_t fo = (((size_t)rb * (nm >> 4) + (k0 >> 4)) * 32 + lane) * 8;
                             uint32_t aa[4];
-                            frag_a(Aw + (size_t)(rb * 16) * nm + k0, nm, g8, t4, aa);
+                            *reinterpret_cast<uint4*>(aa) = *reinterpret_cast<const uint4*>(Aw + fo);
                             const __half* xp = hs16 + (size_t)g8 * np + k0 + 2 * t4;
                             const uint32_t xp0 = *reinterpret_cast<const uint32_t*>(xp);
                             const uint32_t xp1 = *reinterpret_cast<const uint32_t*>(xp + 8);
                             mma16816(yp, aa, xp0, xp1);
                             if (m > 0) {
                                 uint32_t ab[4], an[4];
-                                frag_a(Bw + (size_t)(rb * 16) * nm + k0, nm, g8, t4, ab);
+                                *reinterpret_cast<uint4*>(ab) = *reinterpret_cast<const uint4*>(Bw + fo);
 #pragma unroll
                                 for (int q = 0; q < 4; ++q) an[q] = ab[q] ^ 0x80008000u;
                                 const __half* xm = hs16 + (size_t)(kTe + g8) * np + k0 + 2 * t4;
@@ -551,15 +543,16 @@ __global__ void __launch_bounds__(kNodeNt, 1) k_bwd_node(BwdParams P) {
                         float dxp[4] = {0.f, 0.f, 0.f, 0.f}, dxm[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 4
                         for (int r0 = 0; r0 < nm; r0 += 16) {
+                            const size_t fo = (((size_t)cb * (nm >> 4) + (r0 >> 4)) * 32 + lane) * 8;
                             uint32_t aa[4];
-                            frag_a(At16 + (size_t)(cb * 16) * nm + r0, nm, g8, t4, aa);
+                            *reinterpret_cast<uint4*>(aa) = *reinterpret_cast<const uint4*>(At16 + fo);
                             const __half* yp = gy16 + (size_t)g8 * np + r0 + 2 * t4;
                             const uint32_t yp0 = *reinterpret_cast<const uint32_t*>(yp);
                             const uint32_t yp1 = *reinterpret_cast<const uint32_t*>(yp + 8);
                             mma16816(dxp, aa, yp0, yp1);
                             if (m > 0) {
                                 uint32_t ab[4], an[4];
-                                frag_a(Bt16 + (size_t)(cb * 16) * nm + r0, nm, g8, t4, ab);
+                                *reinterpret_cast<uint4*>(ab) = *reinterpret_cast<const uint4*>(Bt16 + fo);
 #pragma unroll
                                 for (int q = 0; q < 4; ++q) an[q] = ab[q] ^ 0x80008000u;
                                 const __half* ym = gy16 + (size_t)(kTe + g8) * np + r0 + 2 * t4;
@@ -1313,7 +1306,18 @@ __global__ void __launch_bounds__(kNt, 1) k_bwd_dw_umma(BwdParams P) {
     if (warp == 0) tmem_dealloc(tmem, 512);
 }
 
-// Packed SO(2) weights -> fp16, row-major blocks (w16) and each block transposed (wt16)
+// Position of element (r, k) of an n x n block (n a multiple of 16) in fragment
+// order: 16 x 16 tiles row-major, and within a tile the 8 halves that lane
+// (g, t) of an m16n8k16 A fragment holds, in register order
+// (r g, k 2t..2t+1), (r g+8, k 2t..), (r g, k 2t+8..), (r g+8, k 2t+8..).
+__host__ __device__ inline size_t frag_pos(int r, int k, int n) {
+    const int rb = r >> 4, kb = k >> 4, rr = r & 15, kk = k & 15;
+    const int lane = (rr & 7) * 4 + ((kk & 7) >> 1), q = (rr >> 3) + 2 * (kk >> 3);
+    return (((size_t)rb * (n >> 4) + kb) * 32 + lane) * 8 + q * 2 + (kk & 1);
+}
+
+// Packed SO(2) weights -> fp16 in fragment order: each block (w16) and each
+// block transposed (wt16), so an A fragment is one 16-byte load per lane
 template <typename T>
 __global__ void k_bwd_w16(const T* __restrict__ w, int L, int C, int M, __half* w16, __half* wt16) {
     const size_t total = so2_total(L, C, M);
@@ -1328,8 +1332,8 @@ __global__ void k_bwd_w16(const T* __restrict__ w, int L, int C, int M, __half* 
         const size_t loc = e - off;
         const int r = (int)(loc / n), k = (int)(loc % n);
         const __half v = __float2half_rn(load_feat(w, e));
-        w16[e] = v;
-        wt16[off + (size_t)k * n + r] = v;
+        w16[off + frag_pos(r, k, n)] = v;
+        wt16[off + frag_pos(k, r, n)] = v;
     }
 }
 
