@@ -990,6 +990,15 @@ __global__ void __launch_bounds__(kNt, 2) k_bwd_dw(BwdParams P) {
 // before refilling it.
 // ---------------------------------------------------------------------------
 constexpr int kUR = 128, kUC = 256, kUE = 32, kUChunk = 128;
+constexpr int kURow = 12;   // a Wigner row (2l+1 <= 9 entries) padded to three float4
+constexpr int kUDr = 120;   // floats per edge: rows (l+m), (l-m) for l = m..L, padded
+constexpr int kURbf = 32;   // radial basis per edge, padded (n_rbf <= 32)
+
+// padded Wigner rows of one edge: (l+m) and (l-m) for l = m..L, kURow floats each
+__device__ __forceinline__ int drow_off_p(int m, int l, int s) {
+    const int nrow = (m == 0) ? 1 : 2;
+    return ((l - m) * nrow + s) * kURow;
+}
 
 int n_dw_tiles_umma(int L, int C, int M) {
     int n = 0;
@@ -1001,8 +1010,8 @@ int n_dw_tiles_umma(int L, int C, int M) {
 }
 
 size_t dw_umma_smem_bytes(int H, int n_rbf) {
-    return 4 * ((size_t)kUChunk * 50 + (size_t)kUChunk * n_rbf + (size_t)kUChunk * H + 2 * kUChunk +
-                (size_t)n_rbf * kUC) +
+    (void)n_rbf;
+    return 4 * ((size_t)kUChunk * kUDr + (size_t)kUChunk * kURbf + (size_t)kUChunk * H + 2 * kUChunk) +
            2 * 2 * 2 * (size_t)(kUR + kUC) * kUE  // [buffer][sign] fp16 operands
            + 64;                                  // mbarriers, TMEM address, abort flag
 }
@@ -1046,13 +1055,12 @@ __global__ void __launch_bounds__(kNt, 1) k_bwd_dw_umma(BwdParams P) {
     const int nrow = (m == 0) ? 1 : 2;
 
     extern __shared__ __align__(1024) float sm[];
-    float* drow = sm;                          // [chunk][50]
-    float* rho = drow + kUChunk * 50;          // [chunk][nr]
-    float* alpha = rho + kUChunk * nr;         // [chunk][H]
+    float* drow = sm;                          // [chunk][kUDr] padded Wigner rows
+    float* rho = drow + kUChunk * kUDr;        // [chunk][kURbf] radial basis, zero-padded
+    float* alpha = rho + kUChunk * kURbf;      // [chunk][H]
     int* ei = reinterpret_cast<int*>(alpha + kUChunk * H);
     int* ej = ei + kUChunk;
-    float* wr = reinterpret_cast<float*>(ej + kUChunk);  // [nr][kUC]
-    __half* ops = reinterpret_cast<__half*>(wr + nr * kUC);
+    __half* ops = reinterpret_cast<__half*>(ej + kUChunk);
     // Ys(buf, sign): kUR x kUE halves; Xs(buf, sign): kUC x kUE halves
     auto Ys = [&](int bf, int sg) { return ops + (size_t)(bf * 2 + sg) * kUR * kUE; };
     auto Xs = [&](int bf, int sg) { return ops + (size_t)4 * kUR * kUE + (size_t)(bf * 2 + sg) * kUC * kUE; };
@@ -1073,10 +1081,6 @@ __global__ void __launch_bounds__(kNt, 1) k_bwd_dw_umma(BwdParams P) {
         tmem_alloc(tmem_sm, 512);
         tmem_relinquish();
     }
-    for (int t = tid; t < nr * kUC; t += kNt) {
-        const int kb = t / kUC, kx = k0 + t % kUC;
-        wr[t] = (kx < nm) ? P.Wrad[(size_t)kb * G + (m + kx / C) * C + kx % C] : 0.f;
-    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -1089,13 +1093,17 @@ __global__ void __launch_bounds__(kNt, 1) k_bwd_dw_umma(BwdParams P) {
     const bool y_ok = ry < nm;
     const int y_l = m + (y_ok ? ry / C : 0), y_c = y_ok ? ry % C : 0;
     const int y_g = y_l * y_l * C + y_c, y_w = 2 * y_l + 1;
-    const int y_d0 = y_ok ? drow_off(m, y_l, 0) : 0, y_d1 = (y_ok && m > 0) ? drow_off(m, y_l, 1) : 0;
+    const int y_d0 = y_ok ? drow_off_p(m, y_l, 0) : 0, y_d1 = (y_ok && m > 0) ? drow_off_p(m, y_l, 1) : 0;
     const int y_h = y_c / dh;
     const int x_q = tid, kxx = k0 + x_q;
     const bool x_ok = kxx < nm;
     const int x_l = m + (x_ok ? kxx / C : 0), x_c = x_ok ? kxx % C : 0;
     const int x_g = x_l * x_l * C + x_c, x_w = 2 * x_l + 1;
-    const int x_d0 = x_ok ? drow_off(m, x_l, 0) : 0, x_d1 = (x_ok && m > 0) ? drow_off(m, x_l, 1) : 0;
+    const int x_d0 = x_ok ? drow_off_p(m, x_l, 0) : 0, x_d1 = (x_ok && m > 0) ? drow_off_p(m, x_l, 1) : 0;
+    float wreg[kURbf];  // this column's W_rad entries (value gate), zero beyond n_rbf
+#pragma unroll
+    for (int kb = 0; kb < kURbf; ++kb)
+        wreg[kb] = (x_ok && kb < nr) ? P.Wrad[(size_t)kb * G + x_l * C + x_c] : 0.f;
     static_assert(2 * kUR == kNt && kUC == kNt && kUE % 16 == 0, "operand roles");
 
     const int e_lo = (int)((long long)P.n_pairs * split / kDwSplit);
@@ -1121,18 +1129,19 @@ __global__ void __launch_bounds__(kNt, 1) k_bwd_dw_umma(BwdParams P) {
             edge_frame(r.x / d, r.y / d, r.z / d, R);
             float D[WS];
             wigner_blocks<L>(R, D);
-            float* dr = drow + tid * 50;
+            float* dr = drow + tid * kUDr;
             for (int l = m; l <= L; ++l) {
                 const int w = 2 * l + 1;
                 for (int s2 = 0; s2 < nrow; ++s2) {
                     const int row = s2 == 0 ? l + m : l - m;
-                    for (int n = 0; n < w; ++n) dr[drow_off(m, l, s2) + n] = D[wig_off(l) + row * w + n];
+                    float* o = dr + drow_off_p(m, l, s2);
+                    for (int n = 0; n < kURow; ++n) o[n] = (n < w) ? D[wig_off(l) + row * w + n] : 0.f;
                 }
             }
-            for (int kb = 0; kb < nr; ++kb) rho[tid * nr + kb] = rbf(d, kb, P.cutoff, nr);
+            for (int kb = 0; kb < kURbf; ++kb) rho[tid * kURbf + kb] = (kb < nr) ? rbf(d, kb, P.cutoff, nr) : 0.f;
             for (int h = 0; h < H; ++h) {
                 float ga = 0.f;
-                for (int kb = 0; kb < nr; ++kb) ga = fmaf(rho[tid * nr + kb], P.Wrad[(size_t)kb * G + Gv + h], ga);
+                for (int kb = 0; kb < nr; ++kb) ga = fmaf(rho[tid * kURbf + kb], P.Wrad[(size_t)kb * G + Gv + h], ga);
                 const float* qi = P.q + (size_t)i * C + h * dh;
                 const float* kj = P.k + (size_t)j * C + h * dh;
                 float dot = 0.f;
@@ -1182,14 +1191,20 @@ __global__ void __launch_bounds__(kNt, 1) k_bwd_dw_umma(BwdParams P) {
                                 for (int n = 0; n < 2 * L + 1; ++n) gr[n] = (n < y_w) ? gi[(size_t)n * C] : 0.f;
                                 cached = node;
                             }
-                            const float* dr = drow + el * 50;
+                            float d0[kURow], d1[kURow];
+                            const float4* r0v = reinterpret_cast<const float4*>(drow + el * kUDr + y_d0);
+                            const float4* r1v = reinterpret_cast<const float4*>(drow + el * kUDr + y_d1);
+#pragma unroll
+                            for (int v4 = 0; v4 < kURow / 4; ++v4) {
+                                *reinterpret_cast<float4*>(d0 + 4 * v4) = r0v[v4];
+                                *reinterpret_cast<float4*>(d1 + 4 * v4) = r1v[v4];
+                            }
                             float ap = 0.f, am = 0.f;
 #pragma unroll
-                            for (int n = 0; n < 2 * L + 1; ++n)
-                                if (n < y_w) {
-                                    ap = fmaf(dr[y_d0 + n], gr[n], ap);
-                                    if (nrow == 2) am = fmaf(dr[y_d1 + n], gr[n], am);
-                                }
+                            for (int n = 0; n < 2 * L + 1; ++n) {
+                                ap = fmaf(d0[n], gr[n], ap);
+                                am = fmaf(d1[n], gr[n], am);
+                            }
                             const float al = alpha[el * H + y_h];
                             vp = al * ap;
                             vm = al * am;
@@ -1216,16 +1231,30 @@ __global__ void __launch_bounds__(kNt, 1) k_bwd_dw_umma(BwdParams P) {
 #pragma unroll
                         for (int n = 0; n < 2 * L + 1; ++n)
                             xr[n] = (n < x_w) ? __bfloat162float(x[xb + (size_t)n * C]) : 0.f;
-                        const float* dr = drow + el * 50;
+                        float d0[kURow], d1[kURow];
+                        const float4* r0v = reinterpret_cast<const float4*>(drow + el * kUDr + x_d0);
+                        const float4* r1v = reinterpret_cast<const float4*>(drow + el * kUDr + x_d1);
+#pragma unroll
+                        for (int v4 = 0; v4 < kURow / 4; ++v4) {
+                            *reinterpret_cast<float4*>(d0 + 4 * v4) = r0v[v4];
+                            *reinterpret_cast<float4*>(d1 + 4 * v4) = r1v[v4];
+                        }
                         float ap = 0.f, am = 0.f;
 #pragma unroll
-                        for (int n = 0; n < 2 * L + 1; ++n)
-                            if (n < x_w) {
-                                ap = fmaf(dr[x_d0 + n], xr[n], ap);
-                                if (nrow == 2) am = fmaf(dr[x_d1 + n], xr[n], am);
-                            }
+                        for (int n = 0; n < 2 * L + 1; ++n) {
+                            ap = fmaf(d0[n], xr[n], ap);
+                            am = fmaf(d1[n], xr[n], am);
+                        }
+                        const float4* rv = reinterpret_cast<const float4*>(rho + el * kURbf);
                         float gv = 0.f;
-                        for (int kb = 0; kb < nr; ++kb) gv = fmaf(rho[el * nr + kb], wr[kb * kUC + x_q], gv);
+#pragma unroll
+                        for (int v4 = 0; v4 < kURbf / 4; ++v4) {
+                            const float4 q4 = rv[v4];
+                            gv = fmaf(q4.x, wreg[4 * v4 + 0], gv);
+                            gv = fmaf(q4.y, wreg[4 * v4 + 1], gv);
+                            gv = fmaf(q4.z, wreg[4 * v4 + 2], gv);
+                            gv = fmaf(q4.w, wreg[4 * v4 + 3], gv);
+                        }
                         vp = gv * ap;
                         vm = gv * am;
                     }
