@@ -167,6 +167,15 @@ __device__ __forceinline__ void mma16816(float* d, const uint32_t* a, uint32_t b
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// Wigner blocks in shared memory with every row padded to 12 floats (three
+// float4): row `row` (0..2l) of block l starts at 12 (l^2 + row)
+constexpr int kPRow = 12;
+__host__ __device__ constexpr int wig_padded(int L) { return kPRow * (L + 1) * (L + 1); }
+__device__ __forceinline__ void ld_row(const float* p, float* d) {
+#pragma unroll
+    for (int v = 0; v < kPRow / 4; ++v) *reinterpret_cast<float4*>(d + 4 * v) = reinterpret_cast<const float4*>(p)[v];
+}
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
@@ -181,7 +190,8 @@ size_t node_smem_floats(int L, int C, int H, int n_rbf, bool tc) {
     const int K = n_sh(L), WS = wig_size(L), Gv = (L + 1) * C, G = Gv + H;
     const int KH = (L >= 1) ? std::max((L + 1) * C, 2 * L * C) : C;
     const int KHS = std::max(KH, node_np(L, C));  // the X~ region also holds the fp16 operands
-    return (size_t)K * C + 3ull * kTe * WS + 2ull * kTe * n_rbf + (size_t)kTe * G + (size_t)kTe * Gv +
+    (void)WS;
+    return (size_t)K * C + 3ull * kTe * wig_padded(L) + 2ull * kTe * n_rbf + (size_t)kTe * G + (size_t)kTe * Gv +
            2ull * kTe * H + 12ull * kTe + (size_t)(KHS + 2 * KH) * kTe + (size_t)n_rbf * G + C + 2ull * H + 4 + kTe +
            2ull * kNodeNt + kTe;
 }
@@ -201,10 +211,11 @@ __global__ void __launch_bounds__(kNodeNt, 1) k_bwd_node(BwdParams P) {
 
     extern __shared__ float sm[];
     float* Gi = sm;                    // [K][C] dLoss/dout_i
-    float* Dm = Gi + K * C;            // [te][WS] Wigner blocks
-    float* Dx = Dm + kTe * WS;         // [te][WS] their derivative along Omega_x
-    float* Dy = Dx + kTe * WS;         // [te][WS] ... along Omega_y
-    float* rho = Dy + kTe * WS;        // [te][nr]
+    constexpr int WP = wig_padded(L);
+    float* Dm = Gi + K * C;            // [te][WP] Wigner blocks, rows padded
+    float* Dx = Dm + kTe * WP;         // [te][WP] their derivative along Omega_x
+    float* Dy = Dx + kTe * WP;         // [te][WP] ... along Omega_y
+    float* rho = Dy + kTe * WP;        // [te][nr]
     float* rhop = rho + kTe * nr;      // [te][nr] d rho / d d
     float* g = rhop + kTe * nr;        // [te][G] gates
     float* dgv = g + kTe * G;          // [te][Gv] dLoss/dg_v
@@ -282,21 +293,47 @@ __global__ void __launch_bounds__(kNodeNt, 1) k_bwd_node(BwdParams P) {
                     const float d = sqrtf(r.x * r.x + r.y * r.y + r.z * r.z);
                     float R[3][3];
                     edge_frame(r.x / d, r.y / d, r.z / d, R);
-                    wigner_blocks<L>(R, Dm + e * WS);
+                    // the recursion writes the blocks unpadded at the start of the edge's slots;
+                    // then every entry moves up to its padded place (12 (l^2 + row) + n >=
+                    // wig_off(l) + row (2l+1) + n), highest first, and the padding is zeroed
+                    float* De = Dm + e * WP;
+                    float* Xe = Dx + e * WP;
+                    float* Ye = Dy + e * WP;
+                    wigner_blocks<L>(R, De);
                     float dR[3][3];
 #pragma unroll
                     for (int c = 0; c < 3; ++c) { dR[0][c] = 0.f; dR[1][c] = -R[2][c]; dR[2][c] = R[1][c]; }
-                    wigner_dblocks<L>(Dm + e * WS, dR, Dx + e * WS);
+                    wigner_dblocks<L>(De, dR, Xe);
 #pragma unroll
                     for (int c = 0; c < 3; ++c) { dR[0][c] = R[2][c]; dR[1][c] = 0.f; dR[2][c] = -R[0][c]; }
-                    wigner_dblocks<L>(Dm + e * WS, dR, Dy + e * WS);
+                    wigner_dblocks<L>(De, dR, Ye);
+                    for (int l = L; l >= 0; --l) {
+                        const int w = 2 * l + 1;
+                        for (int row = w - 1; row >= 0; --row)
+                            for (int n = w - 1; n >= 0; --n) {
+                                const int o = kPRow * (l * l + row) + n, q = wig_off(l) + row * w + n;
+                                De[o] = De[q];
+                                Xe[o] = Xe[q];
+                                Ye[o] = Ye[q];
+                            }
+                    }
+                    for (int l = 0; l <= L; ++l) {
+                        const int w = 2 * l + 1;
+                        for (int row = 0; row < w; ++row)
+                            for (int n = w; n < kPRow; ++n) {
+                                const int o = kPRow * (l * l + row) + n;
+                                De[o] = 0.f;
+                                Xe[o] = 0.f;
+                                Ye[o] = 0.f;
+                            }
+                    }
                     for (int kb = 0; kb < nr; ++kb) rbf_and_deriv(d, kb, P.cutoff, nr, rho[e * nr + kb], rhop[e * nr + kb]);
                     gg[0] = r.x / d; gg[1] = r.y / d; gg[2] = r.z / d; gg[3] = d;
                     gg[4] = R[1][0]; gg[5] = R[1][1]; gg[6] = R[1][2];
                     gg[7] = -R[0][0]; gg[8] = -R[0][1]; gg[9] = -R[0][2];
                 } else {
                     jn[e] = i;
-                    for (int a = 0; a < WS; ++a) { Dm[e * WS + a] = 0.f; Dx[e * WS + a] = 0.f; Dy[e * WS + a] = 0.f; }
+                    for (int a = 0; a < WP; ++a) { Dm[e * WP + a] = 0.f; Dx[e * WP + a] = 0.f; Dy[e * WP + a] = 0.f; }
                     for (int kb = 0; kb < nr; ++kb) { rho[e * nr + kb] = 0.f; rhop[e * nr + kb] = 0.f; }
                     for (int a = 0; a < 10; ++a) gg[a] = 0.f;
                     gg[3] = 1.f;
@@ -337,18 +374,18 @@ __global__ void __launch_bounds__(kNodeNt, 1) k_bwd_node(BwdParams P) {
                     const int l1 = m + r / C, c = r % C;
                     float vp = 0.f, vm = 0.f;
                     if (e < ne) {
-                        const float* D = Dm + e * WS + wig_off(l1);
                         const int w = 2 * l1 + 1;
                         const size_t xb = ((size_t)jn[e] * K + l1 * l1) * C + c;
                         float xr[2 * L + 1];  // all loads issued before the arithmetic
 #pragma unroll
                         for (int n = 0; n < 2 * L + 1; ++n) xr[n] = (n < w) ? load_feat(x, xb + (size_t)n * C) : 0.f;
+                        float dp_[kPRow], dm_[kPRow];
+                        ld_row(Dm + e * WP + kPRow * (l1 * l1 + l1 + m), dp_);
+                        ld_row(Dm + e * WP + kPRow * (l1 * l1 + l1 - m), dm_);
 #pragma unroll
                         for (int n = 0; n < 2 * L + 1; ++n) {
-                            if (n < w) {
-                                vp = fmaf(D[(l1 + m) * w + n], xr[n], vp);
-                                vm = fmaf(D[(l1 - m) * w + n], xr[n], vm);
-                            }
+                            vp = fmaf(dp_[n], xr[n], vp);
+                            vm = fmaf(dm_[n], xr[n], vm);
                         }
                         const float gv = g[e * G + l1 * C + c];
                         vp *= gv;
@@ -412,12 +449,15 @@ __global__ void __launch_bounds__(kNodeNt, 1) k_bwd_node(BwdParams P) {
                         const int l3 = m + r / C, c = r % C, w3 = 2 * l3 + 1;
                         float gp = 0.f, gm = 0.f;
                         if (e < ne) {
-                            const float* D = Dm + e * WS + wig_off(l3);
                             const float* gi = Gi + (size_t)(l3 * l3) * C + c;
-                            for (int n = 0; n < w3; ++n) {
-                                const float gv = gi[(size_t)n * C];
-                                gp = fmaf(D[(l3 + m) * w3 + n], gv, gp);
-                                gm = fmaf(D[(l3 - m) * w3 + n], gv, gm);
+                            float dp_[kPRow], dm_[kPRow];
+                            ld_row(Dm + e * WP + kPRow * (l3 * l3 + l3 + m), dp_);
+                            ld_row(Dm + e * WP + kPRow * (l3 * l3 + l3 - m), dm_);
+#pragma unroll
+                            for (int n = 0; n < 2 * L + 1; ++n) {
+                                const float gv = (n < w3) ? gi[(size_t)n * C] : 0.f;
+                                gp = fmaf(dp_[n], gv, gp);
+                                gm = fmaf(dm_[n], gv, gm);
                             }
                         }
                         gy[(size_t)r * kTe + e] = gp;
@@ -464,11 +504,12 @@ __global__ void __launch_bounds__(kNodeNt, 1) k_bwd_node(BwdParams P) {
                     for (int e = 0; e < kTe; ++e) {
                         float gp = 0.f, gm = 0.f;
                         if (e < ne) {
-                            const float* D = Dm + e * WS + wig_off(l3);
+                            const float* Dp_ = Dm + e * WP + kPRow * (l3 * l3 + l3 + m);
+                            const float* Dn_ = Dm + e * WP + kPRow * (l3 * l3 + l3 - m);
                             for (int n = 0; n < w3; ++n) {
                                 const float gv = gi[(size_t)n * C];
-                                gp = fmaf(D[(l3 + m) * w3 + n], gv, gp);
-                                gm = fmaf(D[(l3 - m) * w3 + n], gv, gm);
+                                gp = fmaf(Dp_[n], gv, gp);
+                                gm = fmaf(Dn_[n], gv, gm);
                             }
                         }
                         gy[(size_t)r * kTe + e] = gp;
@@ -485,22 +526,33 @@ __global__ void __launch_bounds__(kNodeNt, 1) k_bwd_node(BwdParams P) {
                 const int rows_h = (L + 1 - m) * dh;
                 for (int task = warp; task < ne * H; task += nt / 32) {
                     const int e = task / H, h = task % H;
-                    const float* Ex = Dx + e * WS;
-                    const float* Ey = Dy + e * WS;
+                    const float* Ex = Dx + e * WP;
+                    const float* Ey = Dy + e * WP;
                     float bs = 0.f, tx = 0.f, ty = 0.f;
                     for (int q = lane; q < rows_h; q += 32) {
                         const int l3 = m + q / dh, c = h * dh + q % dh, w3 = 2 * l3 + 1;
                         const int r = (l3 - m) * C + c;
                         const float* gi = Gi + (size_t)(l3 * l3) * C + c;
-                        const int op_ = wig_off(l3) + (l3 + m) * w3, om_ = wig_off(l3) + (l3 - m) * w3;
+                        const int op_ = kPRow * (l3 * l3 + l3 + m), om_ = kPRow * (l3 * l3 + l3 - m);
+                        float gr_[2 * L + 1];
+#pragma unroll
+                        for (int n = 0; n < 2 * L + 1; ++n) gr_[n] = (n < w3) ? gi[(size_t)n * C] : 0.f;
+                        float ra[kPRow], rb_[kPRow];
                         float xp = 0.f, xm = 0.f, zp = 0.f, zm = 0.f;
-                        for (int n = 0; n < w3; ++n) {
-                            const float gv = gi[(size_t)n * C];
-                            xp = fmaf(Ex[op_ + n], gv, xp);
-                            zp = fmaf(Ey[op_ + n], gv, zp);
-                            if (m > 0) {
-                                xm = fmaf(Ex[om_ + n], gv, xm);
-                                zm = fmaf(Ey[om_ + n], gv, zm);
+                        ld_row(Ex + op_, ra);
+                        ld_row(Ey + op_, rb_);
+#pragma unroll
+                        for (int n = 0; n < 2 * L + 1; ++n) {
+                            xp = fmaf(ra[n], gr_[n], xp);
+                            zp = fmaf(rb_[n], gr_[n], zp);
+                        }
+                        if (m > 0) {
+                            ld_row(Ex + om_, ra);
+                            ld_row(Ey + om_, rb_);
+#pragma unroll
+                            for (int n = 0; n < 2 * L + 1; ++n) {
+                                xm = fmaf(ra[n], gr_[n], xm);
+                                zm = fmaf(rb_[n], gr_[n], zm);
                             }
                         }
                         const float yp = yb[(size_t)r * kTe + e];
@@ -623,9 +675,7 @@ __global__ void __launch_bounds__(kNodeNt, 1) k_bwd_node(BwdParams P) {
 #pragma unroll
                     for (int e = 0; e < kTe; ++e) {
                         if (e < ne) {
-                            const float* D = Dm + e * WS + wig_off(l1);
-                            const float* Ex = Dx + e * WS + wig_off(l1);
-                            const float* Ey = Dy + e * WS + wig_off(l1);
+                            const int pp = e * WP + kPRow * (l1 * l1 + l1 + m), pm = e * WP + kPRow * (l1 * l1 + l1 - m);
                             const size_t xb = ((size_t)jn[e] * K + l1 * l1) * C + c;
                             const float gv = g[e * G + l1 * C + c];
                             float rp = 0.f, rm = 0.f, xp = 0.f, xm = 0.f, zp = 0.f, zm = 0.f;
@@ -633,20 +683,32 @@ __global__ void __launch_bounds__(kNodeNt, 1) k_bwd_node(BwdParams P) {
 #pragma unroll
                             for (int n = 0; n < 2 * L + 1; ++n)
                                 xr[n] = (n < w1) ? load_feat(x, xb + (size_t)n * C) : 0.f;
+                            float ra[kPRow], rb_[kPRow];
+                            ld_row(Dm + pp, ra);
+                            ld_row(Dm + pm, rb_);
 #pragma unroll
                             for (int n = 0; n < 2 * L + 1; ++n) {
+                                rp = fmaf(ra[n], xr[n], rp);
+                                rm = fmaf(rb_[n], xr[n], rm);
                                 if (n < w1) {
-                                    const float xv = xr[n];
-                                    rp = fmaf(D[(l1 + m) * w1 + n], xv, rp);
-                                    rm = fmaf(D[(l1 - m) * w1 + n], xv, rm);
-                                    xp = fmaf(Ex[(l1 + m) * w1 + n], xv, xp);
-                                    xm = fmaf(Ex[(l1 - m) * w1 + n], xv, xm);
-                                    zp = fmaf(Ey[(l1 + m) * w1 + n], xv, zp);
-                                    zm = fmaf(Ey[(l1 - m) * w1 + n], xv, zm);
-                                    float gxv = D[(l1 + m) * w1 + n] * dp[e];
-                                    if (m > 0) gxv = fmaf(D[(l1 - m) * w1 + n], dq[e], gxv);
+                                    float gxv = ra[n] * dp[e];
+                                    if (m > 0) gxv = fmaf(rb_[n], dq[e], gxv);
                                     atomicAdd(P.gx + xb + (size_t)n * C, gv * gxv);
                                 }
+                            }
+                            ld_row(Dx + pp, ra);
+                            ld_row(Dx + pm, rb_);
+#pragma unroll
+                            for (int n = 0; n < 2 * L + 1; ++n) {
+                                xp = fmaf(ra[n], xr[n], xp);
+                                xm = fmaf(rb_[n], xr[n], xm);
+                            }
+                            ld_row(Dy + pp, ra);
+                            ld_row(Dy + pm, rb_);
+#pragma unroll
+                            for (int n = 0; n < 2 * L + 1; ++n) {
+                                zp = fmaf(ra[n], xr[n], zp);
+                                zm = fmaf(rb_[n], xr[n], zm);
                             }
                             float dg = dp[e] * rp, tx = dp[e] * xp, ty = dp[e] * zp;
                             if (m > 0) {
