@@ -99,3 +99,53 @@ def test_tensor_core_dispatch_rule():
     assert not uses(2, 16, 1, 16, 5.0, "bf16")
     assert not uses(0, 128, 8, 16, 5.0, "bf16")
     assert not uses(4, 128, 2, 16, 5.0, "bf16")     # H not a multiple of 4
+
+
+def _bwd(cfg, **kw):
+    a = dict(pos=16, n=4, box=None, rp=16, col=16, npairs=4, x=16, wq=16, wk=16, wr=16, ws=16, gout=16, gpos=16,
+             gx=16, gwq=16, gwk=16, gwr=16, gws=16, wsp=256, wsb=1 << 24)
+    a.update(kw)
+    v = lambda p: None if p is None else ctypes.c_void_p(p)
+    return e2f.lib().e2f_onfly_attention_backward(
+        ctypes.byref(cfg), v(a["pos"]), a["n"], a["box"], v(a["rp"]), v(a["col"]), a["npairs"], v(a["x"]), v(a["wq"]),
+        v(a["wk"]), v(a["wr"]), v(a["ws"]), v(a["gout"]), v(a["gpos"]), v(a["gx"]), v(a["gwq"]), v(a["gwk"]),
+        v(a["gwr"]), v(a["gws"]), v(a["wsp"]), a["wsb"], None)
+
+
+def test_backward_workspace_and_argument_checks():
+    bf = e2f.make_cfg(4, 128, 8, 16, 6.0, "bf16")
+    f32 = e2f.make_cfg(4, 128, 8, 16, 6.0, "f32")
+    # bf16 storage adds fp16 copies of the SO(2) weights; an edge adds one float per head
+    assert e2f.e2f_attention_backward_workspace_size(100, 1000, bf) > e2f.e2f_attention_backward_workspace_size(
+        100, 1000, f32) > 0
+    assert (e2f.e2f_attention_backward_workspace_size(100, 2000, f32) -
+            e2f.e2f_attention_backward_workspace_size(100, 1000, f32)) >= 4 * 8 * 1000
+    assert e2f.e2f_attention_backward_workspace_size(100, 1000, e2f.make_cfg(5, 128, 8, 16, 6.0, "bf16")) == 0
+    cfg = e2f.make_cfg(2, 16, 1, 16, 5.0, "f32")
+    assert _bwd(cfg, gout=None) == 1
+    assert _bwd(cfg, gpos=None) == 1
+    assert _bwd(cfg, gx=8) == 4            # grad_x not 16-byte aligned
+    assert _bwd(cfg, wsp=128) == 4
+    assert _bwd(cfg, wsb=16) == 1
+    assert _bwd(cfg, npairs=-1) == 1
+    assert _bwd(cfg, n=0) == 0
+    assert _bwd(e2f.make_cfg(2, 48, 3, 16, 5.0, "f32")) == 2        # 3 heads: not a divisor of the CTA size
+    assert _bwd(e2f.make_cfg(4, 256, 8, 16, 6.0, "bf16")) == 2      # shared memory beyond 227 KB
+
+
+def test_fused_traversal_argument_checks():
+    cfg = e2f.make_cfg(4, 128, 8, 16, 6.0, "bf16")
+    box = (ctypes.c_float * 3)(30.0, 30.0, 30.0)
+    small = (ctypes.c_float * 3)(10.0, 30.0, 30.0)
+    assert e2f.e2f_attention_cells_workspace_size(3000, box, cfg) > e2f.e2f_attention_workspace_size(3000, 0, cfg)
+    assert e2f.e2f_attention_cells_workspace_size(3000, None, cfg) == 0      # periodic boxes only
+    assert e2f.e2f_attention_cells_workspace_size(3000, small, cfg) == 0     # cutoff above half the box
+    f = e2f.lib().e2f_onfly_attention_cells
+    v = ctypes.c_void_p
+    bx = ctypes.cast(box, v)
+    args = lambda c, b, x=16: (ctypes.byref(c), v(16), 4, b, v(x), v(16), v(16), v(16), v(16), v(16), v(256), 1 << 26,
+                               None)
+    assert f(*args(cfg, None)) == 2                                   # open boundaries
+    assert f(*args(e2f.make_cfg(4, 128, 8, 16, 6.0, "f32"), bx)) == 2  # the tensor-core shapes only
+    assert f(*args(cfg, bx, x=0)) == 1                                # null features
+    assert f(*args(cfg, bx, x=8)) == 4                                # misaligned features
