@@ -127,9 +127,10 @@ extern "C" e2f_status e2f_onfly_attention(const e2f_attn_cfg* cfg, const float* 
 
 extern "C" size_t e2f_attention_cells_workspace_size(int64_t n_atoms, const float* box_host,
                                                      const e2f_attn_cfg* cfg) {
-    if (check_cfg(cfg) != E2F_OK || n_atoms < 0 || !box_host) return 0;
-    for (int a = 0; a < 3; ++a)
-        if (!(box_host[a] > 0.f) || !std::isfinite(box_host[a]) || cfg->cutoff > 0.5f * box_host[a]) return 0;
+    if (check_cfg(cfg) != E2F_OK || n_atoms < 0) return 0;
+    if (box_host)
+        for (int a = 0; a < 3; ++a)
+            if (!(box_host[a] > 0.f) || !std::isfinite(box_host[a]) || cfg->cutoff > 0.5f * box_host[a]) return 0;
     return attn_layout(n_atoms, *cfg).bytes + align_up(cell_lists_bytes(n_atoms, box_host, cfg->cutoff), 256);
 }
 
@@ -141,12 +142,12 @@ extern "C" e2f_status e2f_onfly_attention_cells(const e2f_attn_cfg* cfg, const f
     e2f_status st = check_cfg(cfg);
     if (st != E2F_OK) return st;
     if (n_atoms < 1 || n_atoms > INT32_MAX) return E2F_ERR_INVALID_ARG;
-    if (!box_host) return E2F_ERR_UNSUPPORTED;  // the fused traversal covers periodic boxes
     if (!tc_supported(cfg->L, cfg->C, cfg->H, cfg->n_rbf, cfg->feat_dtype == E2F_BF16)) return E2F_ERR_UNSUPPORTED;
     if (!pos || !x || !W_q || !W_k || !W_rad || !W_so2 || !out || !workspace) return E2F_ERR_INVALID_ARG;
-    for (int a = 0; a < 3; ++a)
-        if (!(box_host[a] > 0.f) || !std::isfinite(box_host[a]) || cfg->cutoff > 0.5f * box_host[a])
-            return E2F_ERR_INVALID_ARG;
+    if (box_host)
+        for (int a = 0; a < 3; ++a)
+            if (!(box_host[a] > 0.f) || !std::isfinite(box_host[a]) || cfg->cutoff > 0.5f * box_host[a])
+                return E2F_ERR_INVALID_ARG;
     if (reinterpret_cast<uintptr_t>(workspace) % 256 || reinterpret_cast<uintptr_t>(x) % 16 ||
         reinterpret_cast<uintptr_t>(W_so2) % 16 || reinterpret_cast<uintptr_t>(out) % 16 ||
         reinterpret_cast<uintptr_t>(W_rad) % 16)
@@ -163,9 +164,13 @@ extern "C" e2f_status e2f_onfly_attention_cells(const e2f_attn_cfg* cfg, const f
     a.M = effective_mmax(cfg->L, cfg->m_max);
     a.bf16 = true;
     a.n_atoms = (int)n_atoms; a.n_pairs = 0;
-    a.box.periodic = 1;
-    a.box.len = make_float3(box_host[0], box_host[1], box_host[2]);
-    a.box.inv = make_float3(1.0f / box_host[0], 1.0f / box_host[1], 1.0f / box_host[2]);
+    a.box.periodic = box_host != nullptr;
+    if (box_host) {
+        a.box.len = make_float3(box_host[0], box_host[1], box_host[2]);
+        a.box.inv = make_float3(1.0f / box_host[0], 1.0f / box_host[1], 1.0f / box_host[2]);
+    } else {
+        a.box.len = a.box.inv = make_float3(0.f, 0.f, 0.f);
+    }
     a.pos = pos; a.row_ptr = cl.rp; a.col = nullptr; a.x = x;
     a.Wq = W_q; a.Wk = W_k; a.Wrad = W_rad; a.Wso2 = W_so2; a.out = out;
     a.status = reinterpret_cast<int*>(ws + L.o_status);

@@ -102,9 +102,10 @@ __device__ __forceinline__ int stencil_buckets(const long long c[3], int gid, co
 }
 
 
-// Read-only view of a periodic cell list (one graph) for kernels that
-// enumerate neighbours on the fly: atoms sorted by bucket (float4 x, y, z,
-// graph id), their indices, bucket starts (n_buckets + 1).
+// Read-only view of a cell list (one graph; periodic grid or, for open
+// boundaries, hashed buckets) for kernels that enumerate neighbours on the
+// fly: atoms sorted by bucket (float4 x, y, z, graph id), their indices,
+// bucket starts (n_buckets + 1).
 struct CellView {
     Grid g;
     float rc2;
@@ -141,10 +142,21 @@ __device__ __forceinline__ int warp_neighbors(const CellView& cv, float4 me, int
     const int lane = threadIdx.x & 31;
     long long c[3];
     cell_of(me.x, me.y, me.z, cv.g, c);
-    const int nb = cv.g.noff[0] * cv.g.noff[1] * cv.g.noff[2];
-    uint32_t st = 0, len = 0;
+    const bool per = cv.g.box.periodic != 0;
+    const int nb = per ? cv.g.noff[0] * cv.g.noff[1] * cv.g.noff[2] : 27;
+    uint32_t bk = 0;
     if (lane < nb) {
-        const uint32_t bk = stencil_bucket(c, cv.g, lane);
+        if (per) {
+            bk = stencil_bucket(c, cv.g, lane);
+        } else {  // open boundaries: the 27 cells around c, x fastest, hashed
+            const long long cc[3] = {c[0] + lane % 3 - 1, c[1] + (lane / 3) % 3 - 1, c[2] + lane / 9 - 1};
+            bk = bucket_of(cc, 0, cv.g);
+        }
+    }
+    // cells that hash to one bucket: only the lowest such lane keeps it
+    const unsigned same = __match_any_sync(kAll, lane < nb ? bk : (0x80000000u | (uint32_t)lane));
+    uint32_t st = 0, len = 0;
+    if (lane < nb && __ffs(same) - 1 == lane) {
         st = cv.start[bk];
         len = cv.start[bk + 1] - st;
     }

@@ -236,9 +236,11 @@ e2f_status e2f_attention_debug_timers(void* workspace, size_t ws_bytes, int64_t 
  * e2f_build_neighbors (cutoff = cfg->cutoff); the order of the edges of a
  * node differs from the CSR call, so sums may differ in the last bits.
  *
- * Periodic boxes (box_host non-NULL, cutoff <= min(box)/2) and the
- * tensor-core configurations (e2f_attention_uses_tensor_cores) only;
- * otherwise E2F_ERR_UNSUPPORTED. One system (no graph batching).
+ * Periodic boxes (box_host non-NULL, cutoff <= min(box)/2) or open
+ * boundaries (box_host NULL: the neighbour build's hashed cells; cells
+ * that hash to one bucket are visited once). The tensor-core
+ * configurations (e2f_attention_uses_tensor_cores) only; otherwise
+ * E2F_ERR_UNSUPPORTED. One system (no graph batching).
  * Arguments as for e2f_onfly_attention without row_ptr, col, n_pairs;
  * workspace >= e2f_attention_cells_workspace_size(...) bytes, 256-byte
  * aligned. Asynchronous (no host synchronisation); non-finite positions

@@ -138,14 +138,13 @@ def test_fused_traversal_argument_checks():
     box = (ctypes.c_float * 3)(30.0, 30.0, 30.0)
     small = (ctypes.c_float * 3)(10.0, 30.0, 30.0)
     assert e2f.e2f_attention_cells_workspace_size(3000, box, cfg) > e2f.e2f_attention_workspace_size(3000, 0, cfg)
-    assert e2f.e2f_attention_cells_workspace_size(3000, None, cfg) == 0      # periodic boxes only
+    assert e2f.e2f_attention_cells_workspace_size(3000, None, cfg) > 0       # open boundaries: hashed cells
     assert e2f.e2f_attention_cells_workspace_size(3000, small, cfg) == 0     # cutoff above half the box
     f = e2f.lib().e2f_onfly_attention_cells
     v = ctypes.c_void_p
     bx = ctypes.cast(box, v)
     args = lambda c, b, x=16: (ctypes.byref(c), v(16), 4, b, v(x), v(16), v(16), v(16), v(16), v(16), v(256), 1 << 26,
                                None)
-    assert f(*args(cfg, None)) == 2                                   # open boundaries
     assert f(*args(e2f.make_cfg(4, 128, 8, 16, 6.0, "f32"), bx)) == 2  # the tensor-core shapes only
     assert f(*args(cfg, bx, x=0)) == 1                                # null features
     assert f(*args(cfg, bx, x=8)) == 4                                # misaligned features

@@ -45,7 +45,6 @@ def test_fused_traversal_scope():
     d = DeviceInputs(3)
     w = d.w
     cfg = e2f.make_cfg(w.L, w.C, w.H, w.n_rbf, w.cutoff, w.dtype)
-    assert e2f.e2f_attention_cells_workspace_size(w.n_atoms, None, cfg) == 0  # periodic boxes only
     f32 = e2f.make_cfg(w.L, w.C, w.H, w.n_rbf, w.cutoff, "f32")
     with pytest.raises(e2f.E2FError) as ei:
         e2f.e2f_onfly_attention_cells(f32, d.pos, d.box, d.x, d.Wq, d.Wk, d.Wrad, d.Wso2)
@@ -82,3 +81,16 @@ def test_fused_traversal_with_truncated_maps():
     csr = e2f.e2f_onfly_attention(cfg, d.pos, d.box, rp, col, d.x, d.Wq, d.Wk, d.Wrad, wso2)
     fused = e2f.e2f_onfly_attention_cells(cfg, d.pos, d.box, d.x, d.Wq, d.Wk, d.Wrad, wso2)
     assert rel_err_per_degree(fused.cpu().numpy(), csr.cpu().numpy(), w.L) <= 1e-3
+
+
+def test_fused_traversal_open_boundaries():
+    # the same atoms without the periodic box: hashed cells, open-boundary predicate
+    d = DeviceInputs(3)
+    w = d.w
+    cfg = e2f.make_cfg(w.L, w.C, w.H, w.n_rbf, w.cutoff, w.dtype)
+    rp, col = e2f.e2f_build_neighbors(d.pos, None, w.cutoff)
+    csr = e2f.e2f_onfly_attention(cfg, d.pos, None, rp, col, d.x, d.Wq, d.Wk, d.Wrad, d.Wso2)
+    fused = e2f.e2f_onfly_attention_cells(cfg, d.pos, None, d.x, d.Wq, d.Wk, d.Wrad, d.Wso2)
+    assert rel_err_per_degree(fused.cpu().numpy(), csr.cpu().numpy(), w.L) <= 1e-3
+    # atoms near the faces have fewer neighbours than in the periodic box
+    assert col.numel() < e2f.e2f_build_neighbors(d.pos, d.box, w.cutoff)[1].numel()
