@@ -75,37 +75,10 @@ __device__ __forceinline__ long long wrap_cell(long long c, int nc) {
     return c < 0 ? c + nc : (c >= nc ? c - nc : c);
 }
 
-// the (up to) 27 distinct buckets around cell c; returns how many
-__device__ __forceinline__ int stencil_buckets(const long long c[3], int gid, const Grid& g, uint32_t out[27]) {
-    int n = 0;
-    if (g.box.periodic) {
-        for (int iz = 0; iz < g.noff[2]; ++iz)
-            for (int iy = 0; iy < g.noff[1]; ++iy)
-                for (int ix = 0; ix < g.noff[0]; ++ix) {
-                    long long cc[3] = {wrap_cell(c[0] + g.offs[0][ix], g.nc[0]),
-                                       wrap_cell(c[1] + g.offs[1][iy], g.nc[1]),
-                                       wrap_cell(c[2] + g.offs[2][iz], g.nc[2])};
-                    out[n++] = bucket_of(cc, gid, g);
-                }
-        return n;
-    }
-    for (int dz = -1; dz <= 1; ++dz)
-        for (int dy = -1; dy <= 1; ++dy)
-            for (int dx = -1; dx <= 1; ++dx) {
-                long long cc[3] = {c[0] + dx, c[1] + dy, c[2] + dz};
-                uint32_t b = bucket_of(cc, gid, g);
-                bool dup = false;
-                for (int k = 0; k < n; ++k) dup |= (out[k] == b);
-                if (!dup) out[n++] = b;
-            }
-    return n;
-}
-
-
-// Read-only view of a cell list (one graph; periodic grid or, for open
-// boundaries, hashed buckets) for kernels that enumerate neighbours on the
-// fly: atoms sorted by bucket (float4 x, y, z, graph id), their indices,
-// bucket starts (n_buckets + 1).
+// Read-only view of a cell list (periodic grid or, for open boundaries,
+// hashed buckets) for kernels that enumerate neighbours: atoms sorted by
+// bucket (float4 x, y, z, graph id), their indices, bucket starts
+// (n_buckets + 1).
 struct CellView {
     Grid g;
     float rc2;
@@ -114,29 +87,30 @@ struct CellView {
     const uint32_t* start;
 };
 
-// Periodic stencil entry b (0 <= b < noff[0] noff[1] noff[2]; x fastest, as
-// in stencil_buckets): the bucket of one graph's grid. Offsets are {-1, 0, 1}
+// Periodic stencil entry b (0 <= b < noff[0] noff[1] noff[2]; z slowest, x
+// fastest): the bucket of graph gid's grid. Offsets are {-1, 0, 1}
 // on an axis of three or more cells, {0, 1} on two cells, {0} on one.
-__device__ __forceinline__ uint32_t stencil_bucket(const long long c[3], const Grid& g, int b) {
+__device__ __forceinline__ uint32_t stencil_bucket(const long long c[3], const Grid& g, int b, int gid = 0) {
     const int ix = b % g.noff[0], r = b / g.noff[0];
     const int iy = r % g.noff[1], iz = r / g.noff[1];
     const long long cx = wrap_cell(c[0] + ix - (g.noff[0] == 3), g.nc[0]);
     const long long cy = wrap_cell(c[1] + iy - (g.noff[1] == 3), g.nc[1]);
     const long long cz = wrap_cell(c[2] + iz - (g.noff[2] == 3), g.nc[2]);
-    return (uint32_t)((cz * g.nc[1] + cy) * g.nc[0] + cx);
+    return (uint32_t)((((long long)gid * g.nc[2] + cz) * g.nc[1] + cy) * g.nc[0] + cx);
 }
 
-// One warp: enumerates the neighbours j of atom i (at me) in stencil order,
-// bucket by bucket, atoms of a bucket in their stored order; calls
-// f(k, j) on the lane that holds the k-th neighbour. Returns the count
-// (the same on every lane). The predicate is the neighbour build's.
+// One warp: enumerates the neighbours j of atom i (at me, in graph gid) in
+// stencil order, bucket by bucket, atoms of a bucket in their stored order;
+// calls f(k, j) on the lane that holds the k-th neighbour. Returns the count
+// (the same on every lane). The predicate is the neighbour build's: j != i,
+// same graph (the w field of the stored positions), fp32 distance test.
 // Lane b holds the range of stencil bucket b; a warp scan concatenates the
 // ranges into one candidate sequence t = 0 .. ncand-1 (stencil order kept),
 // and candidate t sits at sorted position base(b) + t for the bucket b with
 // excl(b) <= t < incl(b), found by a binary search over the lanes. Candidates
 // are loaded 4 x 32 at a time before any is tested, so the loads overlap.
 template <typename F>
-__device__ __forceinline__ int warp_neighbors(const CellView& cv, float4 me, int i, F&& f) {
+__device__ __forceinline__ int warp_neighbors(const CellView& cv, float4 me, int i, F&& f, int gid = 0) {
     constexpr unsigned kAll = 0xffffffffu;
     constexpr int kU = 4;
     const int lane = threadIdx.x & 31;
@@ -147,10 +121,10 @@ __device__ __forceinline__ int warp_neighbors(const CellView& cv, float4 me, int
     uint32_t bk = 0;
     if (lane < nb) {
         if (per) {
-            bk = stencil_bucket(c, cv.g, lane);
+            bk = stencil_bucket(c, cv.g, lane, gid);
         } else {  // open boundaries: the 27 cells around c, x fastest, hashed
             const long long cc[3] = {c[0] + lane % 3 - 1, c[1] + (lane / 3) % 3 - 1, c[2] + lane / 9 - 1};
-            bk = bucket_of(cc, 0, cv.g);
+            bk = bucket_of(cc, gid, cv.g);
         }
     }
     // cells that hash to one bucket: only the lowest such lane keeps it
@@ -189,7 +163,8 @@ __device__ __forceinline__ int warp_neighbors(const CellView& cv, float4 me, int
         }
 #pragma unroll
         for (int u = 0; u < kU; ++u) {
-            const bool hit = jj[u] >= 0 && jj[u] != i && pair_within(me, o[u], cv.g, cv.rc2);
+            const bool hit = jj[u] >= 0 && jj[u] != i && __float_as_int(o[u].w) == gid &&
+                             pair_within(me, o[u], cv.g, cv.rc2);
             const unsigned m = __ballot_sync(kAll, hit);
             if (hit) f(total + __popc(m & ((1u << lane) - 1u)), jj[u]);
             total += __popc(m);

@@ -90,35 +90,18 @@ k_pairs(const float* __restrict__ pos, int n, const int32_t* gp, int n_graphs, G
     if (i >= n) return;
     const int gid = graph_id(gp, n_graphs, i);
     const float4 me = make_float4(pos[3 * i], pos[3 * i + 1], pos[3 * i + 2], __int_as_float(gid));
-    long long c[3];
-    cell_of(me.x, me.y, me.z, g, c);
-    uint32_t bk[27];
-    const int nb = stencil_buckets(c, gid, g, bk);
-
-    int total = 0;
     int row0 = 0, rlen = 0;
     if (MODE == 1) { row0 = row_ptr[i]; rlen = row_ptr[i + 1] - row0; }
     const bool in_smem = (MODE == 1) && rlen <= kSortCap;
-    for (int b = 0; b < nb; ++b) {
-        const uint32_t s0 = start[bk[b]], s1 = start[bk[b] + 1];
-        for (uint32_t s = s0; s < s1; s += 32) {
-            bool hit = false;
-            int j = -1;
-            if (s + lane < s1) {
-                float4 o = sorted_pos[s + lane];
-                j = sorted_idx[s + lane];
-                hit = (j != i) && (__float_as_int(o.w) == gid) && pair_within(me, o, g, rc2);
+    const CellView cv{g, rc2, sorted_pos, sorted_idx, start};
+    const int total = warp_neighbors(
+        cv, me, i,
+        [&](int slot, int j) {
+            if (MODE == 1 && slot < rlen) {  // equal counts in both passes; guard anyway
+                if (in_smem) buf[wib][slot] = j; else col[row0 + slot] = j;
             }
-            unsigned m = __ballot_sync(0xffffffffu, hit);
-            if (MODE == 1 && hit) {
-                int slot = total + __popc(m & ((1u << lane) - 1u));
-                if (slot < rlen) {  // equal counts in both passes; guard anyway
-                    if (in_smem) buf[wib][slot] = j; else col[row0 + slot] = j;
-                }
-            }
-            total += __popc(m);
-        }
-    }
+        },
+        gid);
     if (MODE == 0) {
         if (lane == 0) deg[i] = total;
         return;
