@@ -8,6 +8,7 @@ source or header is newer than them.
 """
 from __future__ import annotations
 
+import concurrent.futures
 import glob
 import os
 import shutil
@@ -41,7 +42,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
     sources = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
     headers = sorted(glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(ROOT, "include", "*.h")))
     hdr_time = _newest(headers)
-    objs = []
+    objs, jobs = [], []
     for src in sources:
         obj = os.path.join(OBJ, os.path.basename(src)[:-3] + ".o")
         objs.append(obj)
@@ -50,7 +51,11 @@ def build(force: bool = False, verbose: bool = False) -> str:
         cmd = [nvcc()] + ARCH + FLAGS + ["-c", src, "-o", obj]
         if verbose:
             print(" ".join(cmd), flush=True)
-        subprocess.run(cmd, check=True)
+        jobs.append(cmd)
+    # translation units compile independently: run them side by side
+    with concurrent.futures.ThreadPoolExecutor(max(1, min(len(jobs), os.cpu_count() or 1))) as ex:
+        for f in [ex.submit(subprocess.run, cmd, check=True) for cmd in jobs]:
+            f.result()
     if force or not os.path.exists(LIB) or os.path.getmtime(LIB) < _newest(objs):
         cmd = [nvcc()] + ARCH + ["-shared", "-o", LIB + ".tmp"] + objs + ["-lcuda"]
         if verbose:
