@@ -61,6 +61,9 @@ def _rel(gpu, ref):
 
 
 CASES = [  # L, C, H, n_rbf, dtype, periodic, n, M
+    (0, 16, 2, 8, "f32", False, 40, None),
+    (1, 32, 2, 8, "f32", True, 40, None),
+    (1, 128, 4, 16, "bf16", True, 40, None),
     (2, 16, 1, 16, "f32", False, 40, None),
     (2, 16, 4, 8, "f32", True, 48, None),
     (4, 128, 8, 16, "bf16", True, 40, None),
