@@ -22,7 +22,8 @@ HEADER = os.path.join(os.path.dirname(_HERE), "include", "e2f.h")
 
 E2F_OK = 0
 STATUS_NAMES = {0: "E2F_OK", 1: "E2F_ERR_INVALID_ARG", 2: "E2F_ERR_UNSUPPORTED", 3: "E2F_ERR_CAPACITY",
-                4: "E2F_ERR_ALIGNMENT", 5: "E2F_ERR_TIMEOUT", 6: "E2F_ERR_CUDA", 7: "E2F_ERR_NONFINITE"}
+                4: "E2F_ERR_ALIGNMENT", 5: "E2F_ERR_TIMEOUT", 6: "E2F_ERR_CUDA", 7: "E2F_ERR_NONFINITE",
+                8: "E2F_ERR_STALE"}
 E2F_F32, E2F_BF16 = 0, 1
 
 
@@ -54,6 +55,9 @@ _SIGS = {
     "e2f_attention_cells_workspace_size": (_sz, [_i64, _vp, ctypes.POINTER(e2f_attn_cfg)]),
     "e2f_onfly_attention_cells": (ctypes.c_int, [ctypes.POINTER(e2f_attn_cfg), _vp, _i64, _vp, _vp, _vp, _vp, _vp,
                                                  _vp, _vp, _vp, _sz, _vp]),
+    "e2f_attention_cells_skin_workspace_size": (_sz, [_i64, _vp, ctypes.POINTER(e2f_attn_cfg), ctypes.c_float]),
+    "e2f_onfly_attention_cells_skin": (ctypes.c_int, [ctypes.POINTER(e2f_attn_cfg), _vp, _i64, _vp, ctypes.c_float,
+                                                      ctypes.c_int, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "e2f_attention_backward_workspace_size": (_sz, [_i64, _i64, ctypes.POINTER(e2f_attn_cfg)]),
     "e2f_onfly_attention_backward": (ctypes.c_int, [ctypes.POINTER(e2f_attn_cfg), _vp, _i64, _vp, _vp, _vp, _i64,
                                                     _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
@@ -249,6 +253,38 @@ def e2f_onfly_attention_cells(cfg: e2f_attn_cfg, pos, box, x, W_q, W_k, W_rad, W
     if check:
         _check(lib().e2f_attention_status(_ptr(workspace), workspace.numel(), s),
                "e2f_onfly_attention_cells (device)")
+    return out
+
+
+def e2f_attention_cells_skin_workspace_size(n_atoms: int, box, cfg: e2f_attn_cfg, skin: float) -> int:
+    b, keep = _box_arg(box)
+    return int(lib().e2f_attention_cells_skin_workspace_size(int(n_atoms), b, ctypes.byref(cfg), float(skin)))
+
+
+def e2f_onfly_attention_cells_skin(cfg: e2f_attn_cfg, pos, box, skin: float, rebuild: bool, x, W_q, W_k, W_rad,
+                                   W_so2, workspace: torch.Tensor, out: torch.Tensor | None = None, stream=None,
+                                   check: bool = True) -> torch.Tensor:
+    """The fused attention with Verlet-skin reuse of the cell lists held in
+    `workspace` (see include/e2f.h). With check, a stale reuse raises
+    E2FError(E2F_ERR_STALE); the caller then calls again with rebuild=True."""
+    _need_cuda(pos, x, W_q, W_k, W_rad, W_so2, out, workspace)
+    n = pos.shape[0]
+    if out is None:
+        out = torch.empty((n, (cfg.L + 1) ** 2, cfg.C), dtype=torch.float32, device=pos.device)
+    ws_bytes = e2f_attention_cells_skin_workspace_size(n, box, cfg, skin)
+    if ws_bytes == 0:
+        raise E2FError(2, "e2f_onfly_attention_cells_skin")
+    if workspace.numel() < ws_bytes:
+        raise E2FError(1, "e2f_onfly_attention_cells_skin: workspace too small")
+    b, keep = _box_arg(box)
+    s = _stream(stream)
+    code = lib().e2f_onfly_attention_cells_skin(ctypes.byref(cfg), _ptr(pos), n, b, float(skin), int(bool(rebuild)),
+                                                _ptr(x), _ptr(W_q), _ptr(W_k), _ptr(W_rad), _ptr(W_so2), _ptr(out),
+                                                _ptr(workspace), workspace.numel(), s)
+    _check(code, "e2f_onfly_attention_cells_skin")
+    if check:
+        _check(lib().e2f_attention_status(_ptr(workspace), workspace.numel(), s),
+               "e2f_onfly_attention_cells_skin (device)")
     return out
 
 

@@ -63,6 +63,7 @@ extern "C" const char* e2f_status_string(e2f_status s) {
         case E2F_ERR_TIMEOUT: return "device-side wait timed out";
         case E2F_ERR_CUDA: return "CUDA error";
         case E2F_ERR_NONFINITE: return "non-finite position";
+        case E2F_ERR_STALE: return "reused cell lists are stale (an atom moved more than skin/2)";
     }
     return "unknown status";
 }
@@ -125,23 +126,29 @@ extern "C" e2f_status e2f_onfly_attention(const e2f_attn_cfg* cfg, const float* 
     return E2F_OK;
 }
 
-extern "C" size_t e2f_attention_cells_workspace_size(int64_t n_atoms, const float* box_host,
-                                                     const e2f_attn_cfg* cfg) {
-    if (check_cfg(cfg) != E2F_OK || n_atoms < 0) return 0;
+extern "C" size_t e2f_attention_cells_skin_workspace_size(int64_t n_atoms, const float* box_host,
+                                                          const e2f_attn_cfg* cfg, float skin) {
+    if (check_cfg(cfg) != E2F_OK || n_atoms < 0 || !(skin >= 0.f) || !std::isfinite(skin)) return 0;
     if (box_host)
         for (int a = 0; a < 3; ++a)
             if (!(box_host[a] > 0.f) || !std::isfinite(box_host[a]) || cfg->cutoff > 0.5f * box_host[a]) return 0;
-    return attn_layout(n_atoms, *cfg).bytes + align_up(cell_lists_bytes(n_atoms, box_host, cfg->cutoff), 256);
+    return attn_layout(n_atoms, *cfg).bytes + align_up(cell_lists_bytes(n_atoms, box_host, cfg->cutoff, skin), 256);
 }
 
-extern "C" e2f_status e2f_onfly_attention_cells(const e2f_attn_cfg* cfg, const float* pos, int64_t n_atoms,
-                                                const float* box_host, const void* x, const float* W_q,
-                                                const float* W_k, const float* W_rad, const void* W_so2,
-                                                float* out, void* workspace, size_t ws_bytes, void* stream_) {
+extern "C" size_t e2f_attention_cells_workspace_size(int64_t n_atoms, const float* box_host,
+                                                     const e2f_attn_cfg* cfg) {
+    return e2f_attention_cells_skin_workspace_size(n_atoms, box_host, cfg, 0.f);
+}
+
+static e2f_status attention_cells(const e2f_attn_cfg* cfg, const float* pos, int64_t n_atoms, const float* box_host,
+                                  float skin, bool rebuild, const void* x, const float* W_q, const float* W_k,
+                                  const float* W_rad, const void* W_so2, float* out, void* workspace,
+                                  size_t ws_bytes, void* stream_) {
     cudaStream_t stream = static_cast<cudaStream_t>(stream_);
     e2f_status st = check_cfg(cfg);
     if (st != E2F_OK) return st;
     if (n_atoms < 1 || n_atoms > INT32_MAX) return E2F_ERR_INVALID_ARG;
+    if (!(skin >= 0.f) || !std::isfinite(skin) || (!rebuild && !(skin > 0.f))) return E2F_ERR_INVALID_ARG;
     if (!tc_supported(cfg->L, cfg->C, cfg->H, cfg->n_rbf, cfg->feat_dtype == E2F_BF16)) return E2F_ERR_UNSUPPORTED;
     if (!pos || !x || !W_q || !W_k || !W_rad || !W_so2 || !out || !workspace) return E2F_ERR_INVALID_ARG;
     if (box_host)
@@ -154,10 +161,14 @@ extern "C" e2f_status e2f_onfly_attention_cells(const e2f_attn_cfg* cfg, const f
         return E2F_ERR_ALIGNMENT;
     AttnWs L = attn_layout(n_atoms, *cfg);
     const size_t cl_off = L.bytes;
-    if (ws_bytes < cl_off + cell_lists_bytes(n_atoms, box_host, cfg->cutoff)) return E2F_ERR_INVALID_ARG;
+    if (ws_bytes < cl_off + cell_lists_bytes(n_atoms, box_host, cfg->cutoff, skin)) return E2F_ERR_INVALID_ARG;
     char* ws = static_cast<char*>(workspace);
     CellLists cl;
-    E2F_CUDA_TRY(build_cell_lists(pos, (int)n_atoms, box_host, cfg->cutoff, ws + cl_off, &cl, stream));
+    if (rebuild) {
+        E2F_CUDA_TRY(build_cell_lists(pos, (int)n_atoms, box_host, cfg->cutoff, ws + cl_off, &cl, stream, skin));
+    } else {
+        E2F_CUDA_TRY(refresh_cell_lists(pos, (int)n_atoms, box_host, cfg->cutoff, skin, ws + cl_off, &cl, stream));
+    }
 
     AttnArgs a{};
     a.L = cfg->L; a.C = cfg->C; a.H = cfg->H; a.n_rbf = cfg->n_rbf; a.cutoff = cfg->cutoff;
@@ -180,6 +191,23 @@ extern "C" e2f_status e2f_onfly_attention_cells(const e2f_attn_cfg* cfg, const f
     E2F_CUDA_TRY(cudaMemsetAsync(a.status, 0, sizeof(int), stream));
     E2F_CUDA_TRY(run_attention_tc(a, ws + L.o_tc, stream, &cl));
     return E2F_OK;
+}
+
+extern "C" e2f_status e2f_onfly_attention_cells(const e2f_attn_cfg* cfg, const float* pos, int64_t n_atoms,
+                                                const float* box_host, const void* x, const float* W_q,
+                                                const float* W_k, const float* W_rad, const void* W_so2,
+                                                float* out, void* workspace, size_t ws_bytes, void* stream) {
+    return attention_cells(cfg, pos, n_atoms, box_host, 0.f, true, x, W_q, W_k, W_rad, W_so2, out, workspace,
+                           ws_bytes, stream);
+}
+
+extern "C" e2f_status e2f_onfly_attention_cells_skin(const e2f_attn_cfg* cfg, const float* pos, int64_t n_atoms,
+                                                     const float* box_host, float skin, int rebuild, const void* x,
+                                                     const float* W_q, const float* W_k, const float* W_rad,
+                                                     const void* W_so2, float* out, void* workspace,
+                                                     size_t ws_bytes, void* stream) {
+    return attention_cells(cfg, pos, n_atoms, box_host, skin, rebuild != 0, x, W_q, W_k, W_rad, W_so2, out,
+                           workspace, ws_bytes, stream);
 }
 
 extern "C" e2f_status e2f_attention_status(void* workspace, size_t ws_bytes, void* stream_) {

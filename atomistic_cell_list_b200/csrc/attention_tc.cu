@@ -155,9 +155,12 @@ __global__ void __launch_bounds__(256) k_softmax_stats_cells(StatsParams P, Cell
     float m = -INFINITY, sum = 0.f;
     int cnt = 0;
     for (int w0 = 0;; w0 += kStatsCap) {
-        cnt = warp_neighbors(cv, me, i, [&](int k, int j) {
-            if (k >= w0 && k < w0 + kStatsCap) jb[k - w0] = j;
-        });
+        cnt = warp_neighbors(
+            cv, me, i,
+            [&](int k, int j) {
+                if (k >= w0 && k < w0 + kStatsCap) jb[k - w0] = j;
+            },
+            0, s);
         __syncwarp();
         const int n_here = min(cnt - w0, kStatsCap);
         for (int k = es; k < n_here; k += EP) {
@@ -198,7 +201,9 @@ __global__ void __launch_bounds__(256) k_softmax_stats_cells(StatsParams P, Cell
 }
 
 __global__ void k_flags_to_status(const int* flags, int* status) {
-    if (*flags & kFlagNonFinite) atomicExch(status, (int)E2F_ERR_NONFINITE);
+    const int f = *flags;
+    if (f & kFlagNonFinite) atomicExch(status, (int)E2F_ERR_NONFINITE);
+    else if (f & kFlagStale) atomicExch(status, (int)E2F_ERR_STALE);
 }
 
 // Node range per CTA: part[k] = first node whose edges start at or after
@@ -1100,13 +1105,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
                 const int s_first = slot_of(e0), s_last = slot_of(e0 + ne - 1);
                 for (int sl = s_first + (warp - 14); sl <= s_last; sl += 2) {
                     const int base = P.row_ptr[sl], ia = P.cv.sidx[sl];
-                    warp_neighbors(P.cv, P.cv.spos[sl], ia, [&](int k, int j) {
-                        const int e = base + k;
-                        if (e >= e0 && e < e0 + ne) {
-                            gi[e - e0] = ia;
-                            gi[kTileE + e - e0] = j;
-                        }
-                    });
+                    warp_neighbors(
+                        P.cv, P.cv.spos[sl], ia,
+                        [&](int k, int j) {
+                            const int e = base + k;
+                            if (e >= e0 && e < e0 + ne) {
+                                gi[e - e0] = ia;
+                                gi[kTileE + e - e0] = j;
+                            }
+                        },
+                        0, sl);
                 }
                 asm volatile("bar.sync 3, 64;" ::: "memory");
                 mbar_arrive(jfull + b);  // releases the lists to the producer (CTA scope)

@@ -15,7 +15,7 @@ namespace e2f {
 
 constexpr float kCellSlack = 1.0e-3f;
 
-enum : int { kFlagNonFinite = 1, kFlagBadGraph = 2 };
+enum : int { kFlagNonFinite = 1, kFlagBadGraph = 2, kFlagStale = 4 };
 
 struct Grid {
     Box box;
@@ -85,6 +85,10 @@ struct CellView {
     const float4* spos;
     const int32_t* sidx;
     const uint32_t* start;
+    // Verlet-skin reuse: the positions the lists were built from (slot order),
+    // else null. The stencil of slot s is then centred on sref[s]'s cell while
+    // the pair test uses the current positions in spos.
+    const float4* sref = nullptr;
 };
 
 // Periodic stencil entry b (0 <= b < noff[0] noff[1] noff[2]; z slowest, x
@@ -109,13 +113,17 @@ __device__ __forceinline__ uint32_t stencil_bucket(const long long c[3], const G
 // and candidate t sits at sorted position base(b) + t for the bucket b with
 // excl(b) <= t < incl(b), found by a binary search over the lanes. Candidates
 // are loaded 4 x 32 at a time before any is tested, so the loads overlap.
+// slot >= 0: i sits at sorted slot `slot`; with build-time positions (cv.sref)
+// the stencil is centred on that slot's build-time cell.
 template <typename F>
-__device__ __forceinline__ int warp_neighbors(const CellView& cv, float4 me, int i, F&& f, int gid = 0) {
+__device__ __forceinline__ int warp_neighbors(const CellView& cv, float4 me, int i, F&& f, int gid = 0,
+                                             int slot = -1) {
     constexpr unsigned kAll = 0xffffffffu;
     constexpr int kU = 4;
     const int lane = threadIdx.x & 31;
+    const float4 ctr = (cv.sref != nullptr && slot >= 0) ? cv.sref[slot] : me;
     long long c[3];
-    cell_of(me.x, me.y, me.z, cv.g, c);
+    cell_of(ctr.x, ctr.y, ctr.z, cv.g, c);
     const bool per = cv.g.box.periodic != 0;
     const int nb = per ? cv.g.noff[0] * cv.g.noff[1] * cv.g.noff[2] : 27;
     uint32_t bk = 0;
@@ -173,17 +181,22 @@ __device__ __forceinline__ int warp_neighbors(const CellView& cv, float4 me, int
     return total;
 }
 
-// Cell lists of one periodic system for the fused attention (built by
-// build_cell_lists in neighbors.cu): the view, the per-node edge offsets in
-// bucket order (rp[N+1]) and an error flag word.
+// Cell lists of one system for the fused attention (built by build_cell_lists
+// in neighbors.cu): the view, the per-node edge offsets in bucket order
+// (rp[N+1]) and an error flag word. With a Verlet skin > 0 the cells are at
+// least cutoff + skin wide and the build-time positions are kept (view.sref);
+// refresh_cell_lists then reuses the sort for new positions that moved less
+// than skin/2 (else kFlagStale), refreshing the positions and the counts.
 struct CellLists {
     CellView view;
     const int32_t* rp;
     int* flags;
 };
-size_t cell_lists_bytes(int64_t n_atoms, const float* box_host, float cutoff);
+size_t cell_lists_bytes(int64_t n_atoms, const float* box_host, float cutoff, float skin = 0.f);
 cudaError_t build_cell_lists(const float* pos, int n_atoms, const float* box_host, float cutoff, void* ws,
-                             CellLists* out, cudaStream_t s);
+                             CellLists* out, cudaStream_t s, float skin = 0.f);
+cudaError_t refresh_cell_lists(const float* pos, int n_atoms, const float* box_host, float cutoff, float skin,
+                               void* ws, CellLists* out, cudaStream_t s);
 
 inline bool make_grid(const float* box_host, float cutoff, int n_graphs, int64_t n_atoms, Grid& g) {
     g.box.periodic = box_host != nullptr;

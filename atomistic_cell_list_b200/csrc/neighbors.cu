@@ -208,24 +208,62 @@ __global__ void k_sort_buckets(const uint32_t* __restrict__ start, uint32_t n_bu
 __global__ void __launch_bounds__(128) k_count_sorted(CellView cv, int n, int32_t* deg) {
     const int s = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     if (s >= n) return;
-    const int cnt = warp_neighbors(cv, cv.spos[s], cv.sidx[s], [](int, int) {});
+    const int cnt = warp_neighbors(cv, cv.spos[s], cv.sidx[s], [](int, int) {}, 0, s);
     if ((threadIdx.x & 31) == 0) deg[s] = cnt;
 }
 
 }  // namespace
 
-size_t cell_lists_bytes(int64_t n_atoms, const float* box_host, float cutoff) {
+// Verlet-skin refresh of one slot: the current position of atom sidx[s]
+// replaces the stored one; a displacement from the build-time position
+// (minimum image) above skin/2, or a non-finite position, is flagged.
+__global__ void k_refresh(const float* __restrict__ pos, int n, Grid g, float half_skin2,
+                          const int32_t* __restrict__ sidx, const float4* __restrict__ sref, float4* spos,
+                          int* flags) {
+    const int s = blockIdx.x * blockDim.x + threadIdx.x;
+    if (s >= n) return;
+    const int i = sidx[s];
+    const float x = pos[3 * i], y = pos[3 * i + 1], z = pos[3 * i + 2];
+    const float4 r = sref[s];
+    if (!(isfinite(x) && isfinite(y) && isfinite(z))) atomicOr(flags, kFlagNonFinite);
+    float dx = x - r.x, dy = y - r.y, dz = z - r.z;
+    if (g.box.periodic) {
+        dx -= g.box.len.x * rintf(dx * g.box.inv.x);
+        dy -= g.box.len.y * rintf(dy * g.box.inv.y);
+        dz -= g.box.len.z * rintf(dz * g.box.inv.z);
+    }
+    if (!(dx * dx + dy * dy + dz * dz <= half_skin2)) atomicOr(flags, kFlagStale);
+    spos[s] = make_float4(x, y, z, r.w);
+}
+
+// Workspace of the cell lists: the neighbour build's arrays, rp[N+1] and,
+// with a skin, the build-time positions in slot order.
+static size_t rp_offset(int64_t n, const Grid& g) { return carve(nullptr, n, g.n_buckets).bytes; }
+static size_t sref_offset(int64_t n, const Grid& g) { return rp_offset(n, g) + align_up(4 * ((size_t)n + 1), 256); }
+
+size_t cell_lists_bytes(int64_t n_atoms, const float* box_host, float cutoff, float skin) {
     Grid g;
-    make_grid(box_host, cutoff, 1, n_atoms, g);
-    return carve(nullptr, n_atoms, g.n_buckets).bytes + align_up(4 * ((size_t)n_atoms + 1), 256);
+    make_grid(box_host, cutoff + skin, 1, n_atoms, g);
+    return sref_offset(n_atoms, g) + (skin > 0.f ? align_up(16 * (size_t)n_atoms, 256) : 0);
+}
+
+// degrees in bucket order, then rp = their exclusive scan
+static cudaError_t count_and_scan(const CellView& cv, int n, const NbrWs& w, int32_t* rp, cudaStream_t s) {
+    count_launch();
+    k_count_sorted<<<(n + 3) / 4, 128, 0, s>>>(cv, n, w.deg);
+    cudaError_t e = cudaMemsetAsync(w.deg + n, 0, sizeof(int32_t), s);
+    if (e != cudaSuccess) return e;
+    return exclusive_scan_u32(reinterpret_cast<uint32_t*>(w.deg), reinterpret_cast<uint32_t*>(rp), (size_t)n + 1,
+                              w.scan_tmp, s);
 }
 
 cudaError_t build_cell_lists(const float* pos, int n, const float* box_host, float cutoff, void* ws,
-                             CellLists* out, cudaStream_t s) {
+                             CellLists* out, cudaStream_t s, float skin) {
     Grid g;
-    make_grid(box_host, cutoff, 1, n, g);
+    make_grid(box_host, cutoff + skin, 1, n, g);
     NbrWs w = carve(ws, n, g.n_buckets);
-    int32_t* rp = reinterpret_cast<int32_t*>(static_cast<char*>(ws) + w.bytes);
+    int32_t* rp = reinterpret_cast<int32_t*>(static_cast<char*>(ws) + rp_offset(n, g));
+    float4* sref = skin > 0.f ? reinterpret_cast<float4*>(static_cast<char*>(ws) + sref_offset(n, g)) : nullptr;
     cudaError_t e = cudaMemsetAsync(w.flags, 0, 256, s);
     if (e == cudaSuccess) e = cudaMemsetAsync(w.count, 0, 4 * ((size_t)g.n_buckets + 1), s);
     if (e != cudaSuccess) return e;
@@ -238,13 +276,34 @@ cudaError_t build_cell_lists(const float* pos, int n, const float* box_host, flo
     k_scatter<<<nbk, tb, 0, s>>>(pos, n, nullptr, 1, w.key, w.rank, w.count, w.sorted_pos, w.sorted_idx);
     count_launch();
     k_sort_buckets<<<(g.n_buckets + 255) / 256, 256, 0, s>>>(w.count, g.n_buckets, w.sorted_pos, w.sorted_idx);
-    CellView cv{g, cutoff * cutoff, w.sorted_pos, w.sorted_idx, w.count};
-    count_launch();
-    k_count_sorted<<<(n + 3) / 4, 128, 0, s>>>(cv, n, w.deg);
-    e = cudaMemsetAsync(w.deg + n, 0, sizeof(int32_t), s);
+    if (sref) {
+        e = cudaMemcpyAsync(sref, w.sorted_pos, 16 * (size_t)n, cudaMemcpyDeviceToDevice, s);
+        if (e != cudaSuccess) return e;
+    }
+    CellView cv{g, cutoff * cutoff, w.sorted_pos, w.sorted_idx, w.count, sref};
+    e = count_and_scan(cv, n, w, rp, s);
     if (e != cudaSuccess) return e;
-    e = exclusive_scan_u32(reinterpret_cast<uint32_t*>(w.deg), reinterpret_cast<uint32_t*>(rp), (size_t)n + 1,
-                           w.scan_tmp, s);
+    out->view = cv;
+    out->rp = rp;
+    out->flags = w.flags;
+    return cudaGetLastError();
+}
+
+cudaError_t refresh_cell_lists(const float* pos, int n, const float* box_host, float cutoff, float skin,
+                               void* ws, CellLists* out, cudaStream_t s) {
+    if (!(skin > 0.f)) return cudaErrorInvalidValue;
+    Grid g;
+    make_grid(box_host, cutoff + skin, 1, n, g);
+    NbrWs w = carve(ws, n, g.n_buckets);
+    int32_t* rp = reinterpret_cast<int32_t*>(static_cast<char*>(ws) + rp_offset(n, g));
+    float4* sref = reinterpret_cast<float4*>(static_cast<char*>(ws) + sref_offset(n, g));
+    cudaError_t e = cudaMemsetAsync(w.flags, 0, 256, s);
+    if (e != cudaSuccess) return e;
+    count_launch();
+    k_refresh<<<(n + 255) / 256, 256, 0, s>>>(pos, n, g, 0.25f * skin * skin, w.sorted_idx, sref, w.sorted_pos,
+                                              w.flags);
+    CellView cv{g, cutoff * cutoff, w.sorted_pos, w.sorted_idx, w.count, sref};
+    e = count_and_scan(cv, n, w, rp, s);
     if (e != cudaSuccess) return e;
     out->view = cv;
     out->rp = rp;

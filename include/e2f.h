@@ -39,7 +39,8 @@ typedef enum {
     E2F_ERR_ALIGNMENT = 4,    /* pointer not aligned as documented           */
     E2F_ERR_TIMEOUT = 5,      /* a bounded device-side wait ran out          */
     E2F_ERR_CUDA = 6,         /* a CUDA runtime call or launch failed        */
-    E2F_ERR_NONFINITE = 7     /* NaN/Inf in positions                        */
+    E2F_ERR_NONFINITE = 7,    /* NaN/Inf in positions                        */
+    E2F_ERR_STALE = 8         /* reused cell lists: an atom moved > skin/2   */
 } e2f_status;
 
 typedef enum { E2F_F32 = 0, E2F_BF16 = 1 } e2f_dtype;
@@ -256,6 +257,50 @@ e2f_status e2f_onfly_attention_cells(const e2f_attn_cfg* cfg, const float* pos,
                                      const void* W_so2, float* out,
                                      void* workspace, size_t ws_bytes,
                                      void* stream);
+
+/* ------------------------------------------------------------------------
+ * The same fused call with Verlet-skin reuse of the cell lists across
+ * molecular-dynamics steps (the layer's conservative variant drives MD,
+ * gist.science Technical Summary 2.2: positions move a little per step, so
+ * the sort of the atoms into cells need not be redone every step).
+ * skin >= 0 (length units of pos).
+ *
+ *   rebuild != 0  sort the atoms into cells at least cutoff + skin wide and
+ *                 keep their positions in the workspace (the reference
+ *                 positions); then the layer as e2f_onfly_attention_cells.
+ *   rebuild == 0  (skin > 0, else E2F_ERR_INVALID_ARG) reuse the sort held
+ *                 in `workspace` from the last rebuild call on it, with the
+ *                 same n_atoms, box, cfg->cutoff and skin (not checked):
+ *                 each atom's slot takes its current position and the
+ *                 neighbours of an atom are searched around its reference
+ *                 cell. Exact while every atom lies within skin/2 of its
+ *                 reference position (minimum image): then every pair within
+ *                 the cutoff now was within cutoff + skin then, so it sits in
+ *                 the 27 cells searched. Otherwise e2f_attention_status
+ *                 reports E2F_ERR_STALE, `out` is unspecified, and the caller
+ *                 repeats the call with rebuild != 0.
+ *
+ * The neighbour set and the pair test are those of e2f_onfly_attention_cells
+ * (cutoff = cfg->cutoff, not cutoff + skin); the edge order differs with the
+ * cell size, so sums may differ in the last bits. skin == 0 with rebuild != 0
+ * is e2f_onfly_attention_cells. workspace >=
+ * e2f_attention_cells_skin_workspace_size(...) bytes (16 bytes per atom
+ * more than without a skin), 256-byte aligned. Asynchronous.
+ * ---------------------------------------------------------------------- */
+size_t e2f_attention_cells_skin_workspace_size(int64_t n_atoms,
+                                               const float* box_host,
+                                               const e2f_attn_cfg* cfg,
+                                               float skin);
+
+e2f_status e2f_onfly_attention_cells_skin(const e2f_attn_cfg* cfg,
+                                          const float* pos, int64_t n_atoms,
+                                          const float* box_host, float skin,
+                                          int rebuild, const void* x,
+                                          const float* W_q, const float* W_k,
+                                          const float* W_rad,
+                                          const void* W_so2, float* out,
+                                          void* workspace, size_t ws_bytes,
+                                          void* stream);
 
 /* ------------------------------------------------------------------------
  * Backward of the on-the-fly equivariant attention: the gradients of a

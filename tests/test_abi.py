@@ -148,3 +148,16 @@ def test_fused_traversal_argument_checks():
     assert f(*args(e2f.make_cfg(4, 128, 8, 16, 6.0, "f32"), bx)) == 2  # the tensor-core shapes only
     assert f(*args(cfg, bx, x=0)) == 1                                # null features
     assert f(*args(cfg, bx, x=8)) == 4                                # misaligned features
+    # Verlet-skin variant: 16 bytes per atom more for the reference positions
+    assert e2f.e2f_attention_cells_skin_workspace_size(3000, box, cfg, 0.0) == \
+        e2f.e2f_attention_cells_workspace_size(3000, box, cfg)
+    assert e2f.e2f_attention_cells_skin_workspace_size(3000, None, cfg, 1.0) >= \
+        e2f.e2f_attention_cells_workspace_size(3000, None, cfg) + 16 * 3000
+    assert e2f.e2f_attention_cells_skin_workspace_size(3000, box, cfg, -1.0) == 0
+    assert e2f.e2f_attention_cells_skin_workspace_size(3000, box, cfg, float("nan")) == 0
+    fs = e2f.lib().e2f_onfly_attention_cells_skin
+    sargs = lambda skin, rebuild: (ctypes.byref(cfg), v(16), 4, bx, skin, rebuild, v(16), v(16), v(16), v(16),
+                                   v(16), v(16), v(256), 1 << 26, None)
+    assert fs(*sargs(0.0, 0)) == 1              # reuse needs a skin
+    assert fs(*sargs(-0.5, 1)) == 1             # negative skin
+    assert fs(*sargs(float("nan"), 1)) == 1

@@ -94,3 +94,99 @@ def test_fused_traversal_open_boundaries():
     assert rel_err_per_degree(fused.cpu().numpy(), csr.cpu().numpy(), w.L) <= 1e-3
     # atoms near the faces have fewer neighbours than in the periodic box
     assert col.numel() < e2f.e2f_build_neighbors(d.pos, d.box, w.cutoff)[1].numel()
+
+
+# ---- Verlet-skin reuse of the cell lists across MD steps ---------------------
+
+SKIN = 1.0
+
+
+def _skin_setup(periodic=True):
+    d = DeviceInputs(3)
+    w = d.w
+    cfg = e2f.make_cfg(w.L, w.C, w.H, w.n_rbf, w.cutoff, w.dtype)
+    box = d.box if periodic else None
+    ws = torch.empty(e2f.e2f_attention_cells_skin_workspace_size(w.n_atoms, box, cfg, SKIN), dtype=torch.uint8,
+                     device=d.pos.device)
+    return d, cfg, box, ws
+
+
+def _skin_call(d, cfg, box, ws, pos, rebuild):
+    return e2f.e2f_onfly_attention_cells_skin(cfg, pos, box, SKIN, rebuild, d.x, d.Wq, d.Wk, d.Wrad, d.Wso2, ws)
+
+
+def _csr_call(d, cfg, box, pos):
+    rp, col = e2f.e2f_build_neighbors(pos, box, d.w.cutoff)
+    return e2f.e2f_onfly_attention(cfg, pos, box, rp, col, d.x, d.Wq, d.Wk, d.Wrad, d.Wso2)
+
+
+def _moved(pos, box, rng, radius):
+    # every atom moved by at most `radius` (uniform direction and length),
+    # wrapped back into the periodic box so that reuse must use the minimum image
+    n = pos.shape[0]
+    u = rng.normal(size=(n, 3))
+    u *= (radius * rng.uniform(0.0, 1.0, (n, 1))) / np.linalg.norm(u, axis=1, keepdims=True)
+    p = pos.cpu().numpy().astype(np.float64) + u
+    if box is not None:
+        p = np.mod(p, np.asarray(box, np.float64))
+    return torch.from_numpy(p.astype(np.float32)).to(pos.device)
+
+
+@pytest.mark.parametrize("periodic", [True, False])
+def test_skin_rebuild_and_reuse_match_the_csr_call(periodic):
+    d, cfg, box, ws = _skin_setup(periodic)
+    out0 = _skin_call(d, cfg, box, ws, d.pos, True)
+    assert rel_err_per_degree(out0.cpu().numpy(), _csr_call(d, cfg, box, d.pos).cpu().numpy(), d.w.L) <= 1e-3
+    rng = np.random.default_rng(21)
+    pos1 = _moved(d.pos, box, rng, 0.49 * SKIN)
+    out1 = _skin_call(d, cfg, box, ws, pos1, False)
+    ref1 = _csr_call(d, cfg, box, pos1)
+    assert rel_err_per_degree(out1.cpu().numpy(), ref1.cpu().numpy(), d.w.L) <= 1e-3
+    # the neighbour sets changed: the layer's output moved by far more than the tolerance
+    assert rel_err_per_degree(out0.cpu().numpy(), ref1.cpu().numpy(), d.w.L) > 1e-2
+
+
+def test_skin_reuse_is_repeatable_and_equals_a_second_reuse():
+    d, cfg, box, ws = _skin_setup()
+    _skin_call(d, cfg, box, ws, d.pos, True)
+    pos1 = _moved(d.pos, box, np.random.default_rng(3), 0.3 * SKIN)
+    a = _skin_call(d, cfg, box, ws, pos1, False)
+    b = _skin_call(d, cfg, box, ws, pos1, False)
+    assert torch.equal(a, b)
+
+
+def test_skin_reuse_flags_a_stale_list_and_recovers():
+    d, cfg, box, ws = _skin_setup()
+    _skin_call(d, cfg, box, ws, d.pos, True)
+    pos1 = d.pos.clone()
+    pos1[17, 0] += 0.51 * SKIN
+    with pytest.raises(e2f.E2FError) as ei:
+        _skin_call(d, cfg, box, ws, pos1, False)
+    assert ei.value.code == 8
+    out = _skin_call(d, cfg, box, ws, pos1, True)
+    assert rel_err_per_degree(out.cpu().numpy(), _csr_call(d, cfg, box, pos1).cpu().numpy(), d.w.L) <= 1e-3
+
+
+def test_skin_md_loop_rebuilds_only_when_needed():
+    # a short trajectory: reuse while every atom stays within skin/2 of its
+    # position at the last rebuild (checked on the host), else rebuild
+    d, cfg, box, ws = _skin_setup()
+    rng = np.random.default_rng(8)
+    vel = rng.normal(size=(d.w.n_atoms, 3)) * 0.06
+    p = d.pos.cpu().numpy().astype(np.float64)
+    ref_pos = p.copy()
+    L_box = np.asarray(box, np.float64)
+    rebuilds = 0
+    for step in range(6):
+        if step:
+            p = np.mod(p + vel, L_box)
+        disp = p - ref_pos
+        disp -= L_box * np.round(disp / L_box)
+        rebuild = step == 0 or np.linalg.norm(disp, axis=1).max() > 0.5 * SKIN
+        if rebuild:
+            ref_pos = p.copy()
+            rebuilds += 1
+        pos = torch.from_numpy(p.astype(np.float32)).to(d.pos.device)
+        out = _skin_call(d, cfg, box, ws, pos, rebuild)
+        assert rel_err_per_degree(out.cpu().numpy(), _csr_call(d, cfg, box, pos).cpu().numpy(), d.w.L) <= 1e-3
+    assert 1 < rebuilds < 6
