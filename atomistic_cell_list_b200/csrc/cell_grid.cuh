@@ -17,14 +17,17 @@ constexpr float kCellSlack = 1.0e-3f;
 
 enum : int { kFlagNonFinite = 1, kFlagBadGraph = 2, kFlagStale = 4 };
 
+// Periodic grids use cells at least half the search radius wide and a
+// stencil of 5 cells per axis (all cells of an axis with fewer than five);
+// open boundaries hash cells at least the search radius wide and search the
+// 3 x 3 x 3 cells around a point.
 struct Grid {
     Box box;
     int nc[3];           // periodic: cells per axis
     float cell;          // open: cell side
     uint32_t n_buckets;  // periodic: n_graphs * nc^3; open: power of two
     uint32_t mask;       // open: n_buckets - 1
-    int offs[3][3];      // periodic stencil offsets per axis (deduplicated)
-    int noff[3];
+    int noff[3];         // periodic: stencil cells per axis (5, or nc below five)
 };
 
 __device__ __forceinline__ bool pair_within(float4 a, float4 b, const Grid& g, float rc2) {
@@ -70,7 +73,8 @@ __device__ __forceinline__ uint32_t bucket_of(const long long c[3], int gid, con
 }
 
 // periodic: cell index c + offset wrapped into [0, nc); c is in [0, nc) and
-// the offset in {-1, 0, 1}, so one add or subtract of nc suffices
+// c + offset lies in (-nc, 2 nc) (offsets -2 .. 2 on axes of five or more
+// cells, 0 .. nc-1 on smaller ones), so one add or subtract of nc suffices
 __device__ __forceinline__ long long wrap_cell(long long c, int nc) {
     return c < 0 ? c + nc : (c >= nc ? c - nc : c);
 }
@@ -91,57 +95,25 @@ struct CellView {
     const float4* sref = nullptr;
 };
 
-// Periodic stencil entry b (0 <= b < noff[0] noff[1] noff[2]; z slowest, x
-// fastest): the bucket of graph gid's grid. Offsets are {-1, 0, 1}
-// on an axis of three or more cells, {0, 1} on two cells, {0} on one.
-__device__ __forceinline__ uint32_t stencil_bucket(const long long c[3], const Grid& g, int b, int gid = 0) {
-    const int ix = b % g.noff[0], r = b / g.noff[0];
-    const int iy = r % g.noff[1], iz = r / g.noff[1];
-    const long long cx = wrap_cell(c[0] + ix - (g.noff[0] == 3), g.nc[0]);
-    const long long cy = wrap_cell(c[1] + iy - (g.noff[1] == 3), g.nc[1]);
-    const long long cz = wrap_cell(c[2] + iz - (g.noff[2] == 3), g.nc[2]);
-    return (uint32_t)((((long long)gid * g.nc[2] + cz) * g.nc[1] + cy) * g.nc[0] + cx);
+// Periodic stencil cell along axis a, entry k (0 <= k < noff[a]): offsets
+// -2 .. 2 on an axis of five or more cells, else every cell of the axis once.
+__device__ __forceinline__ long long stencil_cell(long long c, const Grid& g, int a, int k) {
+    return wrap_cell(c + k - (g.noff[a] == 5 ? 2 : 0), g.nc[a]);
 }
 
-// One warp: enumerates the neighbours j of atom i (at me, in graph gid) in
-// stencil order, bucket by bucket, atoms of a bucket in their stored order;
-// calls f(k, j) on the lane that holds the k-th neighbour. Returns the count
-// (the same on every lane). The predicate is the neighbour build's: j != i,
-// same graph (the w field of the stored positions), fp32 distance test.
-// Lane b holds the range of stencil bucket b; a warp scan concatenates the
-// ranges into one candidate sequence t = 0 .. ncand-1 (stencil order kept),
-// and candidate t sits at sorted position base(b) + t for the bucket b with
-// excl(b) <= t < incl(b), found by a binary search over the lanes. Candidates
-// are loaded 4 x 32 at a time before any is tested, so the loads overlap.
-// slot >= 0: i sits at sorted slot `slot`; with build-time positions (cv.sref)
-// the stencil is centred on that slot's build-time cell.
+// The stencil's candidates: lane l (< 32) holds one range [st, st + len) of
+// sorted positions; a warp scan concatenates the ranges in lane order into
+// one candidate sequence t = 0 .. ncand-1, and candidate t sits at sorted
+// position base(b) + t for the lane b with excl(b) <= t < incl(b), found by a
+// binary search over the lanes. Candidates are loaded 4 x 32 at a time before
+// any is tested, so the loads overlap. Neighbours found are numbered from
+// `total` on; returns the new total (the same on every lane).
 template <typename F>
-__device__ __forceinline__ int warp_neighbors(const CellView& cv, float4 me, int i, F&& f, int gid = 0,
-                                             int slot = -1) {
+__device__ __forceinline__ int scan_candidates(const CellView& cv, float4 me, int i, int gid, uint32_t st,
+                                               uint32_t len, int total, F& f) {
     constexpr unsigned kAll = 0xffffffffu;
     constexpr int kU = 4;
     const int lane = threadIdx.x & 31;
-    const float4 ctr = (cv.sref != nullptr && slot >= 0) ? cv.sref[slot] : me;
-    long long c[3];
-    cell_of(ctr.x, ctr.y, ctr.z, cv.g, c);
-    const bool per = cv.g.box.periodic != 0;
-    const int nb = per ? cv.g.noff[0] * cv.g.noff[1] * cv.g.noff[2] : 27;
-    uint32_t bk = 0;
-    if (lane < nb) {
-        if (per) {
-            bk = stencil_bucket(c, cv.g, lane, gid);
-        } else {  // open boundaries: the 27 cells around c, x fastest, hashed
-            const long long cc[3] = {c[0] + lane % 3 - 1, c[1] + (lane / 3) % 3 - 1, c[2] + lane / 9 - 1};
-            bk = bucket_of(cc, gid, cv.g);
-        }
-    }
-    // cells that hash to one bucket: only the lowest such lane keeps it
-    const unsigned same = __match_any_sync(kAll, lane < nb ? bk : (0x80000000u | (uint32_t)lane));
-    uint32_t st = 0, len = 0;
-    if (lane < nb && __ffs(same) - 1 == lane) {
-        st = cv.start[bk];
-        len = cv.start[bk + 1] - st;
-    }
     uint32_t incl = len;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -150,14 +122,13 @@ __device__ __forceinline__ int warp_neighbors(const CellView& cv, float4 me, int
     }
     const uint32_t ncand = __shfl_sync(kAll, incl, 31);
     const uint32_t base = st - (incl - len);  // modulo 2^32: base + t is the sorted position
-    int total = 0;
     for (uint32_t t0 = 0; t0 < ncand; t0 += 32 * kU) {
         float4 o[kU];
         int jj[kU];
 #pragma unroll
         for (int u = 0; u < kU; ++u) {
             const uint32_t t = t0 + 32 * u + lane;
-            int b = 0;  // number of buckets with incl <= t
+            int b = 0;  // number of lanes with incl <= t
 #pragma unroll
             for (int step = 16; step > 0; step >>= 1)
                 if (__shfl_sync(kAll, incl, b + step - 1) <= t) b += step;
@@ -179,6 +150,67 @@ __device__ __forceinline__ int warp_neighbors(const CellView& cv, float4 me, int
         }
     }
     return total;
+}
+
+// One warp: enumerates the neighbours j of atom i (at me, in graph gid) in
+// stencil order, range by range, atoms of a cell in their stored order;
+// calls f(k, j) on the lane that holds the k-th neighbour. Returns the count
+// (the same on every lane). The predicate is the neighbour build's: j != i,
+// same graph (the w field of the stored positions), fp32 distance test.
+// Periodic grids: the stencil is gathered as rows along x. The cells of a
+// row are consecutive buckets, so lane r holds row r (one (y, z) pair of
+// the stencil) as one range; a row that wraps around the box in x takes a
+// second pass for its wrapped part. Open boundaries: lane b holds hashed
+// bucket b of the 27 (cells that hash to one bucket are visited once).
+// slot >= 0: i sits at sorted slot `slot`; with build-time positions (cv.sref)
+// the stencil is centred on that slot's build-time cell.
+template <typename F>
+__device__ __forceinline__ int warp_neighbors(const CellView& cv, float4 me, int i, F&& f, int gid = 0,
+                                             int slot = -1) {
+    constexpr unsigned kAll = 0xffffffffu;
+    const int lane = threadIdx.x & 31;
+    const float4 ctr = (cv.sref != nullptr && slot >= 0) ? cv.sref[slot] : me;
+    long long c[3];
+    cell_of(ctr.x, ctr.y, ctr.z, cv.g, c);
+    const Grid& g = cv.g;
+    int total = 0;
+    if (g.box.periodic) {
+        const int nrow = g.noff[1] * g.noff[2], nc0 = g.nc[0];
+        const bool all_x = g.noff[0] < 5;
+        const long long x0 = c[0] - 2, x1 = c[0] + 2;
+        const int npass = (!all_x && (x0 < 0 || x1 >= nc0)) ? 2 : 1;
+        for (int p = 0; p < npass; ++p) {
+            uint32_t st = 0, len = 0;
+            if (lane < nrow) {
+                long long lo, hi;
+                if (all_x) { lo = 0; hi = nc0 - 1; }
+                else if (p == 0) { lo = x0 < 0 ? 0 : x0; hi = x1 >= nc0 ? nc0 - 1 : x1; }
+                else if (x0 < 0) { lo = x0 + nc0; hi = nc0 - 1; }
+                else { lo = 0; hi = x1 - nc0; }
+                const long long cy = stencil_cell(c[1], g, 1, lane % g.noff[1]);
+                const long long cz = stencil_cell(c[2], g, 2, lane / g.noff[1]);
+                const long long row = (((long long)gid * g.nc[2] + cz) * g.nc[1] + cy) * nc0;
+                st = cv.start[row + lo];
+                len = cv.start[row + hi + 1] - st;
+            }
+            total = scan_candidates(cv, me, i, gid, st, len, total, f);
+        }
+        return total;
+    }
+    // open boundaries: the 27 cells around c, x fastest, hashed; of cells that
+    // hash to one bucket only the lowest such lane keeps it
+    uint32_t bk = 0;
+    if (lane < 27) {
+        const long long cc[3] = {c[0] + lane % 3 - 1, c[1] + (lane / 3) % 3 - 1, c[2] + lane / 9 - 1};
+        bk = bucket_of(cc, gid, g);
+    }
+    const unsigned same = __match_any_sync(kAll, lane < 27 ? bk : (0x80000000u | (uint32_t)lane));
+    uint32_t st = 0, len = 0;
+    if (lane < 27 && __ffs(same) - 1 == lane) {
+        st = cv.start[bk];
+        len = cv.start[bk + 1] - st;
+    }
+    return scan_candidates(cv, me, i, gid, st, len, total, f);
 }
 
 // Cell lists of one system for the fused attention (built by build_cell_lists
@@ -204,8 +236,8 @@ inline bool make_grid(const float* box_host, float cutoff, int n_graphs, int64_t
         g.box.len = make_float3(box_host[0], box_host[1], box_host[2]);
         g.box.inv = make_float3(1.0f / box_host[0], 1.0f / box_host[1], 1.0f / box_host[2]);
         long long total = std::max(1, n_graphs);
-        for (int a = 0; a < 3; ++a) {
-            int nc = (int)std::floor(double(box_host[a]) / (double(cutoff) * (1.0 + kCellSlack)));
+        for (int a = 0; a < 3; ++a) {  // cells at least half the radius wide
+            int nc = (int)std::floor(double(box_host[a]) / (0.5 * double(cutoff) * (1.0 + kCellSlack)));
             g.nc[a] = std::max(1, std::min(nc, 1024));
         }
         // keep the grid at most 2^26 buckets: coarsen the largest axis
@@ -213,11 +245,7 @@ inline bool make_grid(const float* box_host, float cutoff, int n_graphs, int64_t
             int a = (g.nc[0] >= g.nc[1] && g.nc[0] >= g.nc[2]) ? 0 : (g.nc[1] >= g.nc[2] ? 1 : 2);
             g.nc[a] = std::max(1, g.nc[a] / 2);
         }
-        for (int a = 0; a < 3; ++a) {
-            if (g.nc[a] >= 3) { g.offs[a][0] = -1; g.offs[a][1] = 0; g.offs[a][2] = 1; g.noff[a] = 3; }
-            else if (g.nc[a] == 2) { g.offs[a][0] = 0; g.offs[a][1] = 1; g.noff[a] = 2; }
-            else { g.offs[a][0] = 0; g.noff[a] = 1; }
-        }
+        for (int a = 0; a < 3; ++a) g.noff[a] = std::min(g.nc[a], 5);
         g.n_buckets = (uint32_t)(total * g.nc[0] * g.nc[1] * g.nc[2]);
         g.mask = 0;
         g.cell = 0.f;

@@ -276,7 +276,7 @@ e2f_status e2f_onfly_attention_cells(const e2f_attn_cfg* cfg, const float* pos,
  *                 cell. Exact while every atom lies within skin/2 of its
  *                 reference position (minimum image): then every pair within
  *                 the cutoff now was within cutoff + skin then, so it sits in
- *                 the 27 cells searched. Otherwise e2f_attention_status
+ *                 the stencil searched. Otherwise e2f_attention_status
  *                 reports E2F_ERR_STALE, `out` is unspecified, and the caller
  *                 repeats the call with rebuild != 0.
  *
