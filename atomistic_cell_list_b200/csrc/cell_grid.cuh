@@ -28,6 +28,7 @@ struct Grid {
     uint32_t n_buckets;  // periodic: n_graphs * nc^3; open: power of two
     uint32_t mask;       // open: n_buckets - 1
     int noff[3];         // periodic: stencil cells per axis (5, or nc below five)
+    float reach;         // search radius the grid was made for
 };
 
 __device__ __forceinline__ bool pair_within(float4 a, float4 b, const Grid& g, float rc2) {
@@ -179,19 +180,55 @@ __device__ __forceinline__ int warp_neighbors(const CellView& cv, float4 me, int
         const bool all_x = g.noff[0] < 5;
         const long long x0 = c[0] - 2, x1 = c[0] + 2;
         const int npass = (!all_x && (x0 < 0 || x1 >= nc0)) ? 2 : 1;
+        // Trim the stencil to the cells the search sphere reaches (fp64, radius
+        // padded by 1e-4 relative): a row (y, z offsets) whose y-z distance from
+        // the wrapped centre exceeds the radius is skipped, and a row's x range
+        // is cut to the cells within the remaining half-width. Axes of fewer
+        // than five cells (every cell visited) are not trimmed.
+        long long lo_u = x0, hi_u = x1;
+        bool empty = lane >= nrow;
+        if (!empty) {
+            const double len[3] = {g.box.len.x, g.box.len.y, g.box.len.z};
+            const double p[3] = {ctr.x, ctr.y, ctr.z};
+            double w[3], d2 = 0.0;
+#pragma unroll
+            for (int a = 0; a < 3; ++a) w[a] = p[a] - len[a] * floor(p[a] / len[a]);
+            const int off[3] = {0, lane % g.noff[1], lane / g.noff[1]};
+#pragma unroll
+            for (int a = 1; a < 3; ++a) {
+                if (g.noff[a] == 5) {
+                    const double lc = len[a] / g.nc[a];
+                    const double lo = (double)(c[a] + off[a] - 2) * lc;
+                    const double d = fmax(fmax(lo - w[a], w[a] - (lo + lc)), 0.0);
+                    d2 += d * d;
+                }
+            }
+            const double r = (double)g.reach * (1.0 + 1e-4);
+            const double rem = r * r - d2;
+            if (rem < 0.0) {
+                empty = true;
+            } else if (!all_x) {
+                const double hx = sqrt(rem), lc = len[0] / nc0;
+                const long long a = (long long)floor((w[0] - hx) / lc), b = (long long)floor((w[0] + hx) / lc);
+                lo_u = a > x0 ? a : x0;
+                hi_u = b < x1 ? b : x1;
+            }
+        }
         for (int p = 0; p < npass; ++p) {
             uint32_t st = 0, len = 0;
-            if (lane < nrow) {
+            if (!empty) {
                 long long lo, hi;
                 if (all_x) { lo = 0; hi = nc0 - 1; }
-                else if (p == 0) { lo = x0 < 0 ? 0 : x0; hi = x1 >= nc0 ? nc0 - 1 : x1; }
-                else if (x0 < 0) { lo = x0 + nc0; hi = nc0 - 1; }
-                else { lo = 0; hi = x1 - nc0; }
-                const long long cy = stencil_cell(c[1], g, 1, lane % g.noff[1]);
-                const long long cz = stencil_cell(c[2], g, 2, lane / g.noff[1]);
-                const long long row = (((long long)gid * g.nc[2] + cz) * g.nc[1] + cy) * nc0;
-                st = cv.start[row + lo];
-                len = cv.start[row + hi + 1] - st;
+                else if (p == 0) { lo = lo_u < 0 ? 0 : lo_u; hi = hi_u >= nc0 ? nc0 - 1 : hi_u; }
+                else if (x0 < 0) { lo = lo_u + nc0; hi = nc0 - 1; }
+                else { lo = 0; hi = hi_u - nc0; }
+                if (lo <= hi) {
+                    const long long cy = stencil_cell(c[1], g, 1, lane % g.noff[1]);
+                    const long long cz = stencil_cell(c[2], g, 2, lane / g.noff[1]);
+                    const long long row = (((long long)gid * g.nc[2] + cz) * g.nc[1] + cy) * nc0;
+                    st = cv.start[row + lo];
+                    len = cv.start[row + hi + 1] - st;
+                }
             }
             total = scan_candidates(cv, me, i, gid, st, len, total, f);
         }
@@ -232,6 +269,7 @@ cudaError_t refresh_cell_lists(const float* pos, int n_atoms, const float* box_h
 
 inline bool make_grid(const float* box_host, float cutoff, int n_graphs, int64_t n_atoms, Grid& g) {
     g.box.periodic = box_host != nullptr;
+    g.reach = cutoff;
     if (g.box.periodic) {
         g.box.len = make_float3(box_host[0], box_host[1], box_host[2]);
         g.box.inv = make_float3(1.0f / box_host[0], 1.0f / box_host[1], 1.0f / box_host[2]);
