@@ -6,6 +6,8 @@
 #include <algorithm>
 #include <atomic>
 #include <cmath>
+#include <mutex>
+#include <unordered_map>
 
 #include "attention.cuh"
 #include "cell_grid.cuh"
@@ -140,6 +142,23 @@ extern "C" size_t e2f_attention_cells_workspace_size(int64_t n_atoms, const floa
     return e2f_attention_cells_skin_workspace_size(n_atoms, box_host, cfg, 0.f);
 }
 
+// Verlet-skin reuse: the parameters each workspace's cell lists were last
+// sorted for (host side, keyed by the workspace address). A reuse call must
+// match them; this catches a missing rebuild or a changed system without a
+// device synchronisation.
+struct SkinKey {
+    int64_t n;
+    float box[3], cutoff, skin;
+    size_t cl_off;  // where the lists sit in the workspace (depends on cfg)
+    bool periodic;
+    bool operator==(const SkinKey& o) const {
+        return n == o.n && periodic == o.periodic && cutoff == o.cutoff && skin == o.skin && cl_off == o.cl_off &&
+               (!periodic || (box[0] == o.box[0] && box[1] == o.box[1] && box[2] == o.box[2]));
+    }
+};
+static std::mutex g_skin_mu;
+static std::unordered_map<const void*, SkinKey> g_skin_lists;
+
 static e2f_status attention_cells(const e2f_attn_cfg* cfg, const float* pos, int64_t n_atoms, const float* box_host,
                                   float skin, bool rebuild, const void* x, const float* W_q, const float* W_k,
                                   const float* W_rad, const void* W_so2, float* out, void* workspace,
@@ -163,10 +182,25 @@ static e2f_status attention_cells(const e2f_attn_cfg* cfg, const float* pos, int
     const size_t cl_off = L.bytes;
     if (ws_bytes < cl_off + cell_lists_bytes(n_atoms, box_host, cfg->cutoff, skin)) return E2F_ERR_INVALID_ARG;
     char* ws = static_cast<char*>(workspace);
+    SkinKey key{n_atoms, {0.f, 0.f, 0.f}, cfg->cutoff, skin, cl_off, box_host != nullptr};
+    if (box_host) for (int a = 0; a < 3; ++a) key.box[a] = box_host[a];
     CellLists cl;
     if (rebuild) {
+        {
+            std::lock_guard<std::mutex> lk(g_skin_mu);
+            g_skin_lists.erase(workspace);
+        }
         E2F_CUDA_TRY(build_cell_lists(pos, (int)n_atoms, box_host, cfg->cutoff, ws + cl_off, &cl, stream, skin));
+        if (skin > 0.f) {
+            std::lock_guard<std::mutex> lk(g_skin_mu);
+            g_skin_lists[workspace] = key;
+        }
     } else {
+        {
+            std::lock_guard<std::mutex> lk(g_skin_mu);
+            auto it = g_skin_lists.find(workspace);
+            if (it == g_skin_lists.end() || !(it->second == key)) return E2F_ERR_INVALID_ARG;
+        }
         E2F_CUDA_TRY(refresh_cell_lists(pos, (int)n_atoms, box_host, cfg->cutoff, skin, ws + cl_off, &cl, stream));
     }
 

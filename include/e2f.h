@@ -269,8 +269,15 @@ e2f_status e2f_onfly_attention_cells(const e2f_attn_cfg* cfg, const float* pos,
  *                 keep their positions in the workspace (the reference
  *                 positions); then the layer as e2f_onfly_attention_cells.
  *   rebuild == 0  (skin > 0, else E2F_ERR_INVALID_ARG) reuse the sort held
- *                 in `workspace` from the last rebuild call on it, with the
- *                 same n_atoms, box, cfg->cutoff and skin (not checked):
+ *                 in `workspace` from the last rebuild call on it, which
+ *                 must have had the same n_atoms, box, cfg and skin: the
+ *                 library records these per workspace address at each
+ *                 successful rebuild and returns E2F_ERR_INVALID_ARG, before
+ *                 any launch, when they differ or no rebuild is recorded
+ *                 (host-side check by address: a buffer that is freed and
+ *                 allocated again at the same address is not told apart,
+ *                 so the first call on any new buffer must rebuild; the
+ *                 contents must still be the ones that rebuild wrote):
  *                 each atom's slot takes its current position and the
  *                 neighbours of an atom are searched around its reference
  *                 cell. Exact while every atom lies within skin/2 of its

@@ -159,5 +159,6 @@ def test_fused_traversal_argument_checks():
     sargs = lambda skin, rebuild: (ctypes.byref(cfg), v(16), 4, bx, skin, rebuild, v(16), v(16), v(16), v(16),
                                    v(16), v(16), v(256), 1 << 26, None)
     assert fs(*sargs(0.0, 0)) == 1              # reuse needs a skin
+    assert fs(*sargs(1.0, 0)) == 1              # reuse of a workspace no rebuild was recorded for
     assert fs(*sargs(-0.5, 1)) == 1             # negative skin
     assert fs(*sargs(float("nan"), 1)) == 1

@@ -190,3 +190,25 @@ def test_skin_md_loop_rebuilds_only_when_needed():
         out = _skin_call(d, cfg, box, ws, pos, rebuild)
         assert rel_err_per_degree(out.cpu().numpy(), _csr_call(d, cfg, box, pos).cpu().numpy(), d.w.L) <= 1e-3
     assert 1 < rebuilds < 6
+
+
+def test_skin_reuse_rejects_a_changed_system():
+    # the library records (n, box, cfg, skin) per workspace at each rebuild;
+    # a reuse call with other values is refused before any launch
+    d, cfg, box, ws = _skin_setup()
+    _skin_call(d, cfg, box, ws, d.pos, True)
+    bigger = [1.01 * float(v) for v in box]
+    for args in [(d.pos, bigger), (d.pos[:-10].contiguous(), box)]:
+        with pytest.raises(e2f.E2FError) as ei:
+            e2f.e2f_onfly_attention_cells_skin(cfg, args[0], args[1], SKIN, False, d.x, d.Wq, d.Wk, d.Wrad,
+                                               d.Wso2, ws)
+        assert ei.value.code == 1
+    # a workspace no rebuild was recorded for: 256 bytes into a new block (the
+    # caching allocator's blocks start 512-byte aligned, so a recycled block
+    # address recorded by an earlier rebuild cannot coincide with it)
+    fresh = torch.empty(ws.numel() + 512, dtype=torch.uint8, device=ws.device)[256:256 + ws.numel()]
+    assert fresh.data_ptr() % 512 == 256
+    with pytest.raises(e2f.E2FError) as ei:
+        _skin_call(d, cfg, box, fresh, d.pos, False)
+    assert ei.value.code == 1
+    _skin_call(d, cfg, box, ws, d.pos, False)          # the recorded system still reuses

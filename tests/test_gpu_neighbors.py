@@ -74,7 +74,9 @@ def test_bad_graph_ptr_is_reported():
     assert ei.value.code == 1
 
 
-def test_small_boxes_with_two_or_one_cells_per_axis():
+def test_small_boxes_with_few_cells_per_axis():
+    # 3 to 11 half-width cells per axis: axes of fewer than five cells are
+    # searched whole, larger ones with a stencil that wraps around the box
     rng = np.random.default_rng(3)
     from oracle.neighbors import neighbors_bruteforce
     for side, rc in [(10.0, 5.0), (10.5, 4.0), (7.0, 3.4), (13.0, 4.2)]:
