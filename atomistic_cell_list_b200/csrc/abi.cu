@@ -158,6 +158,7 @@ struct SkinKey {
 };
 static std::mutex g_skin_mu;
 static std::unordered_map<const void*, SkinKey> g_skin_lists;
+constexpr size_t kSkinTableMax = 4096;  // workspaces remembered; beyond it one entry is dropped
 
 static e2f_status attention_cells(const e2f_attn_cfg* cfg, const float* pos, int64_t n_atoms, const float* box_host,
                                   float skin, bool rebuild, const void* x, const float* W_q, const float* W_k,
@@ -193,6 +194,7 @@ static e2f_status attention_cells(const e2f_attn_cfg* cfg, const float* pos, int
         E2F_CUDA_TRY(build_cell_lists(pos, (int)n_atoms, box_host, cfg->cutoff, ws + cl_off, &cl, stream, skin));
         if (skin > 0.f) {
             std::lock_guard<std::mutex> lk(g_skin_mu);
+            if (g_skin_lists.size() >= kSkinTableMax) g_skin_lists.erase(g_skin_lists.begin());
             g_skin_lists[workspace] = key;
         }
     } else {

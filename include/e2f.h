@@ -277,7 +277,9 @@ e2f_status e2f_onfly_attention_cells(const e2f_attn_cfg* cfg, const float* pos,
  *                 (host-side check by address: a buffer that is freed and
  *                 allocated again at the same address is not told apart,
  *                 so the first call on any new buffer must rebuild; the
- *                 contents must still be the ones that rebuild wrote):
+ *                 contents must still be the ones that rebuild wrote; at
+ *                 most 4096 workspaces are remembered, and a reuse call on
+ *                 a forgotten one returns E2F_ERR_INVALID_ARG):
  *                 each atom's slot takes its current position and the
  *                 neighbours of an atom are searched around its reference
  *                 cell. Exact while every atom lies within skin/2 of its
