@@ -34,7 +34,7 @@ extern "C" {
 typedef enum {
     E2F_OK = 0,
     E2F_ERR_INVALID_ARG = 1,  /* null pointer, negative size, bad range      */
-    E2F_ERR_UNSUPPORTED = 2,  /* shape or dtype this build does not handle   */
+    E2F_ERR_UNSUPPORTED = 2,  /* shape or dtype the library does not handle */
     E2F_ERR_CAPACITY = 3,     /* output buffer too small (see n_pairs_host)  */
     E2F_ERR_ALIGNMENT = 4,    /* pointer not aligned as documented           */
     E2F_ERR_TIMEOUT = 5,      /* a bounded device-side wait ran out          */
