@@ -146,6 +146,21 @@ def test_skin_rebuild_and_reuse_match_the_csr_call(periodic):
     assert rel_err_per_degree(out0.cpu().numpy(), ref1.cpu().numpy(), d.w.L) > 1e-2
 
 
+def test_skin_reuse_matches_the_oracle_at_moved_positions():
+    # the oracle's own neighbour list and dense layer at the moved positions
+    from oracle.neighbors import neighbors_bruteforce
+    d, cfg, box, ws = _skin_setup()
+    w = d.w
+    _skin_call(d, cfg, box, ws, d.pos, True)
+    pos1 = _moved(d.pos, box, np.random.default_rng(33), 0.45 * SKIN)
+    out = _skin_call(d, cfg, box, ws, pos1, False)
+    p1 = pos1.cpu().numpy()
+    rp0, col0 = neighbors_bruteforce(p1, w.box, w.cutoff)
+    nodes = np.random.default_rng(12).choice(w.n_atoms, 24, replace=False)
+    ref = d.oracle()(p1, w.box, rp0, col0, d.x_f64, nodes=nodes)
+    assert rel_err_per_degree(out.cpu().numpy()[nodes].astype(np.float64), ref, w.L) <= TOL[w.dtype]
+
+
 def test_skin_reuse_is_repeatable_and_equals_a_second_reuse():
     d, cfg, box, ws = _skin_setup()
     _skin_call(d, cfg, box, ws, d.pos, True)
