@@ -103,3 +103,38 @@ def test_catches_swapped_query_and_key(monkeypatch):
     monkeypatch.setattr(layer_mod.DenseLayer, "__init__", bad)
     monkeypatch.setattr(T, "DenseLayer", layer_mod.DenseLayer)
     _fails(T.test_layer_L0_reduces_to_scalar_graph_attention)
+
+
+# ---- the neighbour and gradient oracles ---------------------------------------
+
+def test_catches_non_strict_cutoff_test(monkeypatch):
+    import oracle.neighbors as nb
+    import test_oracle_neighbors as N
+    orig = nb.predicate_f32
+
+    def bad(pi, pj, box, cutoff):
+        # d2 <= rc^2: keeps a pair exactly at the cutoff
+        return orig(pi, pj, box, float(np.nextafter(np.float32(cutoff), np.float32(np.inf))))
+    monkeypatch.setattr(nb, "predicate_f32", bad)
+    monkeypatch.setattr(N, "predicate_f32", bad)
+    _fails(N.test_exactly_at_cutoff_is_excluded_and_just_inside_is_kept)
+
+
+def test_catches_missing_minimum_image(monkeypatch):
+    import oracle.neighbors as nb
+    import test_oracle_neighbors as N
+    orig = nb.predicate_f32
+    monkeypatch.setattr(nb, "predicate_f32", lambda pi, pj, box, cutoff: orig(pi, pj, None, cutoff))
+    periodic = [c for c in N.parse_cases() if c["box"] is not None]
+    assert periodic
+    _fails(N.test_handmade_fixture, periodic[0])
+
+
+def test_catches_position_gradient_without_the_direction_term(monkeypatch):
+    import oracle.grad as gr
+    import test_oracle_grad as G
+    orig = gr.real_sh_t
+    # the harmonics of the edge direction held constant: forward unchanged,
+    # the position gradient loses the rotation's contribution
+    monkeypatch.setattr(gr, "real_sh_t", lambda lmax, r: orig(lmax, r.detach()))
+    _fails(G.test_gradients_match_finite_differences, 2, 4, 2, 6, False, None)
