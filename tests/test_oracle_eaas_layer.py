@@ -146,6 +146,18 @@ def test_layer_L0_reduces_to_scalar_graph_attention():
         np.testing.assert_allclose(out[i, 0], (al * v).sum(0), atol=1e-12)
 
 
+def test_radial_basis_special_points():
+    # 16 Gaussians at mu_k = k rc/15 of width rc/15 under the cosine envelope:
+    # at d = 0 the envelope is 1 and basis k is exp(-k^2); at d = rc/2 (7.5
+    # widths) the envelope is 1/2; at d = rc it is 0
+    rc = 5.0
+    k = np.arange(16)
+    got = radial_basis(np.array([0.0, rc / 2, rc]), rc, 16)
+    np.testing.assert_allclose(got[0], np.exp(-(k ** 2.0)), rtol=1e-12, atol=0)
+    np.testing.assert_allclose(got[1], 0.5 * np.exp(-((7.5 - k) ** 2.0)), rtol=1e-12, atol=0)
+    np.testing.assert_allclose(got[2], 0.0, atol=1e-16)
+
+
 def test_single_neighbour_gets_full_weight_and_isolated_node_is_zero():
     rng = np.random.default_rng(13)
     L, C, H = 2, 2, 1

@@ -138,3 +138,18 @@ def test_catches_position_gradient_without_the_direction_term(monkeypatch):
     # the position gradient loses the rotation's contribution
     monkeypatch.setattr(gr, "real_sh_t", lambda lmax, r: orig(lmax, r.detach()))
     _fails(G.test_gradients_match_finite_differences, 2, 4, 2, 6, False, None)
+
+
+def test_catches_radial_basis_without_envelope_or_with_wrong_width(monkeypatch):
+    def no_envelope(d, cutoff, n_rbf):
+        mu = np.arange(n_rbf) * (cutoff / (n_rbf - 1))
+        return np.exp(-(((d[:, None] - mu[None, :]) / (cutoff / (n_rbf - 1))) ** 2))
+
+    def wrong_width(d, cutoff, n_rbf):
+        mu = np.arange(n_rbf) * (cutoff / (n_rbf - 1))
+        u = 0.5 * (np.cos(np.pi * d / cutoff) + 1.0)
+        return u[:, None] * np.exp(-(((d[:, None] - mu[None, :]) / (cutoff / n_rbf)) ** 2))
+    for bad in (no_envelope, wrong_width):
+        monkeypatch.setattr(layer_mod, "radial_basis", bad)
+        monkeypatch.setattr(T, "radial_basis", bad)
+        _fails(T.test_radial_basis_special_points)
