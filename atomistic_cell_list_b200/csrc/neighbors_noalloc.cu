@@ -8,8 +8,6 @@
 // e2f_build_neighbors, with the scratch taken from a static __device__
 // array instead of a caller workspace, and it allocates nothing itself (no
 // cudaMalloc, no allocating library).
-#include <mutex>
-
 #include "common.cuh"
 
 namespace e2f {
@@ -17,28 +15,21 @@ namespace {
 
 static_assert(E2F_NOALLOC_SCRATCH_BYTES % 256 == 0, "scratch size must keep 256-byte granules");
 
-// Module memory: placed when the module is loaded, one copy per device.
+// Module memory: placed when the module is loaded, one copy per device
+// context.
 __device__ __align__(256) unsigned char g_nbr_scratch[E2F_NOALLOC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_scratch_mu;
-void* g_scratch_ptr[kMaxDevices] = {};
-
-// Device address of this device's copy of the scratch; looked up once per
-// device, with that device current (the lookup may load the module).
-cudaError_t scratch_for_current_device(void** out) {
-    int dev = -1;
-    cudaError_t e = cudaGetDevice(&dev);
+// Device address of the scratch in the context current on this thread. In
+// host code g_nbr_scratch names a host-side stand-in, so the address is
+// asked for on every call: a symbol's device address belongs to the context
+// the module was loaded in, and a cached one would outlive a device reset
+// or a switch to another context on the same device. The lookup is a host
+// call; the first one in a context may load the module.
+cudaError_t scratch_for_current_context(void** out) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_nbr_scratch);
     if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-    std::lock_guard<std::mutex> lock(g_scratch_mu);
-    if (!g_scratch_ptr[dev]) {
-        void* p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_nbr_scratch);
-        if (e != cudaSuccess) return e;
-        g_scratch_ptr[dev] = p;
-    }
-    *out = g_scratch_ptr[dev];
+    *out = p;
     return cudaSuccess;
 }
 
@@ -56,7 +47,7 @@ extern "C" e2f_status e2f_build_neighbors_noalloc(const float* pos, int64_t n_at
     const size_t need = e2f_neighbors_workspace_size(n_atoms, box_host, cutoff, graph_ptr ? n_graphs : 1);
     if (need > (size_t)E2F_NOALLOC_SCRATCH_BYTES) return E2F_ERR_UNSUPPORTED;
     void* scratch = nullptr;
-    if (scratch_for_current_device(&scratch) != cudaSuccess || !scratch) return E2F_ERR_CUDA;
+    if (scratch_for_current_context(&scratch) != cudaSuccess || !scratch) return E2F_ERR_CUDA;
     // e2f_build_neighbors clears, on `stream`, every scratch word that must
     // start at zero (the flag word, the bucket counts, the degree sentinel)
     // before its first kernel, so what an earlier call left there is harmless.

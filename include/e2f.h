@@ -125,10 +125,15 @@ e2f_status e2f_build_neighbors(const float* pos, int64_t n_atoms,
  *   E2F_ERR_CUDA if the scratch address cannot be looked up.
  * The scratch is shared: calls that overlap on one device (other threads,
  * other streams, or a call enqueued while an earlier one's kernels still
- * run) race on it and give undefined results; serialise them. The first
- * call on each device looks up the array's device address (which may load
- * the module): make it with that device current and before any stream
- * capture starts on it. Like e2f_build_neighbors it synchronises `stream`.
+ * run) race on it and give undefined results; serialise them. Every call
+ * looks up the array's device address in the context current on the
+ * calling thread, so a device reset or another context on the same device
+ * gets its own copy; the first call in a context may load the module, so
+ * make it before any stream capture starts there. The call synchronises
+ * `stream` once, to read the pair count, and returns with the column-fill
+ * kernel still queued on `stream`; that kernel reads the scratch, so the
+ * scratch is free again only once it has run: enqueue the next call on the
+ * same stream, or synchronise `stream` first.
  * ---------------------------------------------------------------------- */
 #define E2F_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
 

@@ -66,3 +66,32 @@ def test_problems_beyond_the_scratch_are_refused_before_any_work():
     assert code == 2 and npairs.value == -7  # E2F_ERR_UNSUPPORTED, nothing written
     code = lib.e2f_build_neighbors_noalloc(None, -1, None, 6.0, None, 1, None, None, 0, ctypes.byref(npairs), None)
     assert code == 1
+
+
+@pytest.mark.gpu
+def test_calls_allocate_no_device_memory():
+    """With its outputs passed in, the call takes no device memory: neither
+    torch's caching allocator nor the device's free memory changes across
+    several calls and a synchronisation. The first calls run before the
+    measurement, because loading the module places its static scratch."""
+    from gpu_util import DeviceInputs
+    d = DeviceInputs(3)
+    ref = e2f.e2f_build_neighbors(d.pos, d.box, d.w.cutoff, d.graph_ptr)
+    n = d.pos.shape[0]
+    rp = torch.empty(n + 1, dtype=torch.int32, device=d.pos.device)
+    col = torch.empty(ref[1].numel() + 16, dtype=torch.int32, device=d.pos.device)
+    for _ in range(2):
+        e2f.e2f_build_neighbors_noalloc(d.pos, d.box, d.w.cutoff, d.graph_ptr, row_ptr=rp, col=col)
+    torch.cuda.synchronize()
+    stats0 = torch.cuda.memory_stats()
+    free0, _ = torch.cuda.mem_get_info()
+    for _ in range(3):
+        got = e2f.e2f_build_neighbors_noalloc(d.pos, d.box, d.w.cutoff, d.graph_ptr, row_ptr=rp, col=col)
+    torch.cuda.synchronize()
+    stats1 = torch.cuda.memory_stats()
+    free1, _ = torch.cuda.mem_get_info()
+    assert free1 == free0
+    for key in ("allocation.all.allocated", "segment.all.allocated", "reserved_bytes.all.current",
+                "allocated_bytes.all.current"):
+        assert stats1.get(key, 0) == stats0.get(key, 0), key
+    _same(got, ref)
