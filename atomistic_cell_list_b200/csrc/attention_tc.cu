@@ -19,20 +19,23 @@
 // fills the other.
 //
 // Warp roles (512 threads, 128 registers each):
-//   0-3, 8-11  epilogue: tcgen05.ld 16x256b fragments of the accumulators;
-//              rotate-back p * D^l3(R)^T restricted to the group's |m| rows
-//              on mma.sync, summed over each node's edges, added to
-//              out[node] (one owner thread per element: fixed order)
+//   0-3        epilogue (warp w: TMEM lanes 32w..32w+31): converts a group's
+//              accumulators in place to fp16 p * o (p = softmax weight of the
+//              edge and the row's head), builds per-node Wigner operand blocks
+//              and drains the rotate-back results D2 = (p o) D into out[node]
+//              (one owner thread per element: fixed order)
 //   4-7        producer: per edge the node, frame, Wigner blocks (fp16 pairs,
 //              shared and global copies); per (edge, head) the softmax weight
 //              p = exp(a - lse) (statistics from an O(N) pre-pass); per
 //              (edge, 8 channels) the gathered, gated, rotated features,
 //              written once per tile to a per-CTA global scratch row for TMA
+//   8, 13      tcgen05.mma issue (one thread each): warp 13 the first
+//              accumulator of a group and the rotate-back MMAs (A operand in
+//              TMEM) of the previous group, warp 8 the second accumulator
 //   12         TMA loads of weight and feature tiles into a 3-stage ring
-//   13         tcgen05.mma issue (one thread), commits to the ring and TMEM
-//              barriers
 //   14-15      value gates rho(d) W_rad of a tile (mma.sync), up to two tiles
 //              ahead of the producer, into a double-buffered global scratch
+//   9-11       idle
 // Every mbarrier wait is bounded by the global timer; on expiry the kernel
 // records E2F_ERR_TIMEOUT, drains what it issued and returns.
 #include <cuda.h>
@@ -348,12 +351,7 @@ constexpr int kNS = 3;                        // ring stages
 constexpr int kSlot = kTileE * kKS * 2;       // 8 KB per operand tile
 constexpr int kStage = 4 * kSlot;
 constexpr int kThreads = 512;
-// Warp roles (16 warps, 65536 / 512 = 128 registers per thread):
-//   0-3, 8-11  epilogue (warp w: TMEM lane quadrant w % 4, lane half w / 8)
-//   4-7        producer
-//   12         TMA, 13 MMA, 14-15 idle
-constexpr int kEpiThreads = 256;
-constexpr int kChunk = 16;                    // epilogue: edges per TMEM load
+constexpr int kEpiThreads = 128;
 
 // Wigner blocks of an edge in "pair" form: for each degree l and each
 // |m| = mu <= l the 2l+1 pairs (D^l[+mu][n], D^l[-mu][n]) as fp16x2, padded
@@ -392,28 +390,37 @@ __host__ __device__ inline size_t stage_bytes(int L, int C) {
     return mx;
 }
 
+// Rotate-back contraction on the tensor cores (see the epilogue): per pass at
+// most kB2Blocks operand blocks of 16 rows (m') x 16 edges, fp16.
+constexpr int kB2Blocks = 30;
+constexpr int kB2Bytes = 512;
+
 // Shared memory layout (bytes), shared by host (size) and device (offsets).
 struct SmemLayout {
-    size_t ring, dstage, dstride, dph, pch, nid, jn, segm, rpw, rho, rrs, wga, bars, misc, dsub, total;
+    size_t ring, dstage, dstride, dph, php, nid, jn, rpw, rho, rrs, wga, b2, slots, req, bars, misc, dsub, total;
     __host__ __device__ SmemLayout(int L, int C, int H, int n_rbf) {
         size_t o = 0;
         ring = o;   o += (size_t)kNS * kStage;
         dstride = (stage_bytes(L, C) + 127) & ~size_t(127);
         dstage = o; o += 2 * dstride;
         dph = o;    o += (size_t)kTileE * dph_stride(L) * 4;
-        pch = o;    o += 2ull * kTileE * (C / 8) * 4;
+        php = o;    o += 2ull * H * kTileE * 4;          // [2][H][128] softmax weight per head and edge
         nid = o;    o += 2ull * kTileE * 4;
         jn = o;     o += 2ull * kTileE * 4;
-        segm = o;   o += 2ull * (kTileE / kChunk) * 4;
         rpw = o;    o += (size_t)kTileE * 4;
         rho = o;    o += (size_t)kTileE * kTcMaxRbf * 2;
         rrs = o;    o += (size_t)kTileE * kTcMaxRbf * 4;
         wga = o;    o += (size_t)kTcMaxRbf * kMaxHeads * 4;
+        o = (o + 1023) & ~size_t(1023);
+        b2 = o;     o += (size_t)kB2Blocks * kB2Bytes;    // rotate-back operand blocks
+        slots = o;  o += (2 * kTileE + 8) * 4;            // node segments of the tile: start, node, count
+        req = o;    o += (kB2Blocks + 4) * 4 + kB2Blocks * 4;  // MMA requests and block parameters
         o = (o + 7) & ~size_t(7);
-        bars = o;   o += (2 * kNS + 17) * 8;
+        bars = o;   o += (2 * kNS + 20) * 8;
         misc = o;   o += 64 + 4 * kTileE * 4;  // TMEM base, abort flag, last slot; gate (i, j) lists
         dsub = o;   o += 16 * 8;
         total = o;
+        (void)n_rbf;
     }
 };
 
@@ -454,131 +461,60 @@ __device__ __forceinline__ void tmem_ld_16x256(uint32_t taddr, uint32_t* r) {
                  : "memory");
 }
 
+// tcgen05.mma kind::f16 with the accumulate flag as an immediate (no predicate setup in the issue loop)
+__device__ __forceinline__ void umma_f(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, int accumulate) {
+    if (accumulate)
+        asm volatile("tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, 1;" ::"r"(d), "l"(a), "l"(b), "r"(idesc)
+                     : "memory");
+    else
+        asm volatile("tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, 0;" ::"r"(d), "l"(a), "l"(b), "r"(idesc)
+                     : "memory");
+}
+
 __device__ __forceinline__ uint32_t pack_h2(float a, float b) {
     __half2 h = __floats2half2_rn(a, b);
     return *reinterpret_cast<uint32_t*>(&h);
 }
 
-// Epilogue of one accumulator pair (o+ at tacc, o- at tacc + 128) or one
-// accumulator (SIGNS = 1) holding output rows (l3, channel) for the tile's
-// 128 edges, on mma.sync: per 16-edge chunk and 8 channels,
-//     acc[m'][c] += sum_e D_e[+mu][m'] y+[e][c] + D_e[-mu][m'] y-[e][c],
-//     y[e][c] = p_e^{head(c)} o[c][e],
-// i.e. the rotate-back D^T of the |m| = mu rows weighted by the softmax and
-// summed over the node's edges. A = Wigner rows (m' padded to 16, built from
-// the staged fp16 pairs), B = p * o straight from tcgen05.ld.16x256b (whose
-// thread layout is the mma B/D fragment layout), D = fp32 accumulators.
-// Node sums go to out with fire-and-forget reductions at segment ends: one
-// thread owns each (node, l3, m', c) element, so the additions happen in
-// program order. The warp covers 16 TMEM lanes (channels cbase..cbase+15);
-// the two warps of a lane quadrant take one half each.
-template <int SIGNS>
-__device__ __noinline__ void epi_mma(uint32_t tacc, int l3, int cbase, int K, int C,
-                                     const __half2* __restrict__ Ds, const float* __restrict__ pch,
-                                     const int* __restrict__ nb, const uint32_t* __restrict__ segm,
-                                     float* __restrict__ out) {
-    const int lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
-    const int W3 = 2 * l3 + 1, NP = npair(l3), C8 = C / 8;
-    float acc[2][4];  // [n-tile lo/hi][fragment]
-#pragma unroll
-    for (int b2 = 0; b2 < 2; ++b2)
-#pragma unroll
-        for (int r = 0; r < 4; ++r) acc[b2][r] = 0.f;
-    int cur = -1;
-    const float* pc = pch + cbase / 8;  // 8-channel groups cbase/8 (lh = 0) and +1 (lh = 1)
-
-    auto flush = [&]() {
-        if (cur < 0) return;
-#pragma unroll
-        for (int lh = 0; lh < 2; ++lh)
-#pragma unroll
-            for (int r = 0; r < 4; ++r) {
-                const int mp = g + ((r >> 1) << 3);
-                if (mp < W3) {
-                    const int c = cbase + 8 * lh + 2 * q + (r & 1);
-                    atomicAdd(out + ((size_t)cur * K + l3 * l3 + mp) * C + c, acc[lh][r]);
-                }
-                acc[lh][r] = 0.f;
-            }
-    };
-
-#pragma unroll 1
-    for (int ch = 0; ch < kTileE / 16; ++ch) {
-        const int e0 = ch * 16;
-        // o values: [sign][edge half][4]: (c_lo,e), (c_lo,e+1), (c_hi,e), (c_hi,e+1)
-        uint32_t ov[SIGNS][2][4];
-#pragma unroll
-        for (int s2 = 0; s2 < SIGNS; ++s2)
-#pragma unroll
-            for (int eh = 0; eh < 2; ++eh) tmem_ld_16x256(tacc + s2 * 128 + e0 + 8 * eh, ov[s2][eh]);
-        // this thread's four edges: e0 + 2q, +1, e0 + 8 + 2q, +1
-        const int ea = e0 + 2 * q, eb = e0 + 8 + 2 * q;
-        // Wigner A fragments per sign: rows m' = g (a0, a2) and g + 8 (a1, a3)
-        uint32_t af[SIGNS][4];
-        {
-            const bool r0 = g < W3, r1 = g + 8 < W3;
-            const __half2 z = __float2half2_rn(0.f);
-            const __half2 p00 = r0 ? Ds[ea * NP + g] : z, p01 = r0 ? Ds[(ea + 1) * NP + g] : z;
-            const __half2 p10 = r1 ? Ds[ea * NP + g + 8] : z, p11 = r1 ? Ds[(ea + 1) * NP + g + 8] : z;
-            const __half2 p20 = r0 ? Ds[eb * NP + g] : z, p21 = r0 ? Ds[(eb + 1) * NP + g] : z;
-            const __half2 p30 = r1 ? Ds[eb * NP + g + 8] : z, p31 = r1 ? Ds[(eb + 1) * NP + g + 8] : z;
-            const __half2 lo[4] = {__lows2half2(p00, p01), __lows2half2(p10, p11), __lows2half2(p20, p21),
-                                   __lows2half2(p30, p31)};
-#pragma unroll
-            for (int k = 0; k < 4; ++k) af[0][k] = *reinterpret_cast<const uint32_t*>(&lo[k]);
-            if (SIGNS == 2) {
-                const __half2 hi[4] = {__highs2half2(p00, p01), __highs2half2(p10, p11), __highs2half2(p20, p21),
-                                       __highs2half2(p30, p31)};
-#pragma unroll
-                for (int k = 0; k < 4; ++k) af[SIGNS - 1][k] = *reinterpret_cast<const uint32_t*>(&hi[k]);
-            }
-        }
-        // softmax weights of the four edges for the two 8-channel groups
-        const float2 w0 = *reinterpret_cast<const float2*>(pc + ea * C8);
-        const float2 w1 = *reinterpret_cast<const float2*>(pc + (ea + 1) * C8);
-        const float2 w2 = *reinterpret_cast<const float2*>(pc + eb * C8);
-        const float2 w3 = *reinterpret_cast<const float2*>(pc + (eb + 1) * C8);
-        const float pw[2][4] = {{w0.x, w1.x, w2.x, w3.x}, {w0.y, w1.y, w2.y, w3.y}};
-        tmem_wait_ld();
-        // segments of this chunk: bit k = edge e0 + k starts a node
-        uint32_t bits = segm[ch];
-        int lo = 0;
-        if (bits & 1u) {
-            flush();
-            cur = nb[e0];
-        }
-        bits &= ~1u;
-        while (true) {
-            const int hi = bits ? __ffs(bits) - 1 : 16;
-            // edge masks of this thread's four edges for [lo, hi)
-            const float m0 = (2 * q >= lo && 2 * q < hi) ? 1.f : 0.f;
-            const float m1 = (2 * q + 1 >= lo && 2 * q + 1 < hi) ? 1.f : 0.f;
-            const float m2 = (8 + 2 * q >= lo && 8 + 2 * q < hi) ? 1.f : 0.f;
-            const float m3 = (9 + 2 * q >= lo && 9 + 2 * q < hi) ? 1.f : 0.f;
-#pragma unroll
-            for (int lh = 0; lh < 2; ++lh) {
-                const float* pwv = pw[lh];
-#pragma unroll
-                for (int s2 = 0; s2 < SIGNS; ++s2) {
-                    const uint32_t* va = ov[s2][0];
-                    const uint32_t* vb = ov[s2][1];
-                    uint32_t bf[2];
-                    bf[0] = pack_h2(pwv[0] * m0 * __uint_as_float(va[2 * lh]),
-                                    pwv[1] * m1 * __uint_as_float(va[2 * lh + 1]));
-                    bf[1] = pack_h2(pwv[2] * m2 * __uint_as_float(vb[2 * lh]),
-                                    pwv[3] * m3 * __uint_as_float(vb[2 * lh + 1]));
-                    mma_16816(acc[lh], af[s2], bf);
-                }
-            }
-            if (hi == 16) break;
-            flush();
-            cur = nb[e0 + hi];
-            lo = hi;
-            bits &= bits - 1;
-        }
-    }
-    flush();
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t* r) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(r[0]),
+                 "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+                 : "memory");
 }
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// Rotate-back operand block: 16 rows (m') x 16 K (edges) fp16, no swizzle,
+// K-major core matrices (8 rows x 16 bytes) 128 bytes apart along K and 256
+// bytes apart along rows. Element (m', k) in halves:
+__device__ __forceinline__ int b2_off(int mp, int k) { return ((mp >> 3) * 2 + (k >> 3)) * 64 + (mp & 7) * 8 + (k & 7); }
+__device__ __forceinline__ uint64_t sdesc_b2(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)(128u >> 4) << 16;   // leading byte offset: next core matrix along K
+    d |= (uint64_t)(256u >> 4) << 32;   // stride byte offset: next 8-row group
+    d |= (uint64_t)1u << 46;            // descriptor version (sm_100)
+    return d;                           // swizzle: none
+}
+// kind::f16, D fp32, A (TMEM) and B fp16, K-major, M = 128, N = 16
+__host__ __device__ constexpr uint32_t idesc_n16() { return (1u << 4) | ((16u >> 3) << 17) | ((128u >> 4) << 24); }
+
+__device__ __forceinline__ void umma_ta(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc, int accumulate) {
+    if (accumulate)
+        asm volatile("tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, 1;" ::"r"(d), "r"(a_tmem), "l"(b),
+                     "r"(idesc)
+                     : "memory");
+    else
+        asm volatile("tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, 0;" ::"r"(d), "r"(a_tmem), "l"(b),
+                     "r"(idesc)
+                     : "memory");
+}
+
+// TMEM column (within an accumulator's 128) of the fp16 operand of edges
+// 16J..16J+15 after the in-place conversion (two fp16 per 32-bit column).
+__device__ __forceinline__ int a2col(int J) { return 8 * J; }
+// Rotate-back result regions (16 columns each) inside a group's 256 columns:
+// the halves of the two accumulators that the conversion has freed.
+__device__ __forceinline__ int d2col(int k) { return 64 + 16 * (k & 3) + 128 * (k >> 2); }
 
 // Wigner slice(s) a group's epilogue needs, by block (l, mu): returns bytes
 // queued on `bar` into staging buffer `dst`.
@@ -619,10 +555,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
     uint8_t* ring = smem + S.ring;
     uint8_t* dstage = smem + S.dstage;
     __half2* dph = reinterpret_cast<__half2*>(smem + S.dph);
-    float* pch = reinterpret_cast<float*>(smem + S.pch);  // [2][128][C/8] softmax weight per 8 channels
+    float* php = reinterpret_cast<float*>(smem + S.php);  // [2][H][128] softmax weight per head and edge
     int* nid = reinterpret_cast<int*>(smem + S.nid);
     int* jn = reinterpret_cast<int*>(smem + S.jn);
-    uint32_t* segm = reinterpret_cast<uint32_t*>(smem + S.segm);
+    uint8_t* b2s = smem + S.b2;                                   // rotate-back operand blocks
+    int* sl_start = reinterpret_cast<int*>(smem + S.slots);       // [129] first edge of each node segment
+    int* sl_node = sl_start + kTileE + 1;                         // [128] its node
+    int* sl_count = sl_node + kTileE;                             // number of segments
+    uint32_t* req = reinterpret_cast<uint32_t*>(smem + S.req);    // [kB2Blocks] MMA requests
+    int* req_n = reinterpret_cast<int*>(req + kB2Blocks);         // request count, TMEM slot
+    uint32_t* req_bp = req + kB2Blocks + 4;                       // [kB2Blocks] block parameters
     int* rpw = reinterpret_cast<int*>(smem + S.rpw);
     __half* rho = reinterpret_cast<__half*>(smem + S.rho);  // [128][16] radial basis, fp16 (gate warps)
     float* rrs = reinterpret_cast<float*>(smem + S.rrs);    // [128][16] radial basis, fp32 (logits)
@@ -634,10 +576,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
     uint64_t* xready = tempty + 2;
     uint64_t* xfree = xready + 2;
     uint64_t* dbar = xfree + 2;   // epilogue Wigner staging, per buffer
-    uint64_t* fin = dbar + 2;
-    uint64_t* gfull = fin + 1;    // value gate of a tile buffer written (gate warps -> producer)
+    uint64_t* fin = dbar + 2;     // [2] final commits of the two MMA warps
+    uint64_t* gfull = fin + 2;    // value gate of a tile buffer written (gate warps -> producer)
     uint64_t* gempty = gfull + 2; // value gate of a tile buffer consumed (producer -> gate warps)
     uint64_t* jfull = gempty + 2; // fused traversal: (i, j) of a tile buffer listed (gate warps -> producer)
+    uint64_t* d2full = jfull + 2; // rotate-back MMAs of a pass complete (tensor core -> epilogue)
+    uint64_t* a2ready = d2full + 1; // rotate-back operands of a group's first pass ready (epilogue -> MMA warp A)
     uint32_t* tmem_sm = reinterpret_cast<uint32_t*>(smem + S.misc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + S.misc + 8);
     int* last_slot = reinterpret_cast<int*>(smem + S.misc + 16);  // producer: node slot of the last edge
@@ -649,15 +593,18 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kNS; ++s) { mbar_init(full + s, 1); mbar_init(empty + s, 1); }
+        for (int s = 0; s < kNS; ++s) { mbar_init(full + s, 1); mbar_init(empty + s, 2); }  // empty: both MMA warps
         for (int b = 0; b < 2; ++b) {
-            mbar_init(tfull + b, 1);
+            mbar_init(tfull + b, 2);  // both MMA warps commit
             mbar_init(tempty + b, kEpiThreads);
             mbar_init(xready + b, 128);
             mbar_init(xfree + b, kEpiThreads);
             mbar_init(dbar + b, 1);
         }
         mbar_init(fin, 1);
+        mbar_init(fin + 1, 1);
+        mbar_init(d2full, 1);
+        mbar_init(a2ready, kEpiThreads);
         for (int b = 0; b < 2; ++b) {
             mbar_init(gfull + b, 64);
             mbar_init(gempty + b, 128);
@@ -689,7 +636,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
         const float inv_s = P.scale[1];
         const int CG = C / 8;
         const int Gv = (L + 1) * C;
-        const int C8 = C / 8;
         for (int t2 = p; t2 < kTcMaxRbf * H; t2 += 128) {
             const int kb = t2 / H, h = t2 % H;
             wga[t2] = kb < NR ? P.Wrad[(size_t)kb * G + Gv + h] : 0.f;
@@ -830,7 +776,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
                             for (int n4 = 0; n4 < npair(l); n4 += 4) gq[n4 / 4] = z;
                         }
                     for (int a = 0; a < DPS; a += 4) *reinterpret_cast<uint4*>(Dh + a) = z;
-                    for (int k8 = 0; k8 < C8; ++k8) pch[(b * kTileE + p) * C8 + k8] = 0.f;
+                    for (int h = 0; h < H; ++h) php[(b * H + h) * kTileE + p] = 0.f;
                     nid[b * kTileE + p] = -1;
                     jn[b * kTileE + p] = 0;
                 }
@@ -870,18 +816,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
                     }
                     const float a = ga * dot * inv_sqrt_dh;
                     const float pw = expf(a - P.lse[(size_t)i * H + h]) * inv_s;
-                    for (int k8 = h * (dh / 8); k8 < (h + 1) * (dh / 8); ++k8) pch[(b * kTileE + e) * C8 + k8] = pw;
+                    php[(b * H + h) * kTileE + e] = pw;
                 }
             }
             E2F_TICK(5);
-            if (p < kTileE / kChunk) {  // segment starts per 16-edge chunk
-                uint32_t m = 0;
-                for (int q = 0; q < kChunk; ++q) {
-                    const int e = p * kChunk + q;
-                    if (e == 0 || nid[b * kTileE + e] != nid[b * kTileE + e - 1]) m |= 1u << q;
-                }
-                segm[b * (kTileE / kChunk) + p] = m;
-            }
             asm volatile("bar.sync 1, 128;" ::: "memory");
             E2F_TICK(7);
             const long long c_b = clock64();
@@ -1022,8 +960,18 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
             }
         }
         __syncwarp();
-    } else if (warp == 13) {
-        // ---------------- MMA ----------------
+    } else if (warp == 13 || warp == 8) {
+        // ---------------- MMA (two issuing warps) ----------------
+        // The issuing thread runs in step with the tensor pipe: whatever it does
+        // between MMAs (barrier polls, commits) leaves the pipe idle. Two warps issue:
+        // A (warp 13) the first accumulator of each group (o+, or the first m = 0
+        // block), B (warp 8) the second (o-, or the second block); while one polls
+        // or commits, the other's MMAs keep the pipe busy. A stage is released and a
+        // group completed when both have committed. Warp A also issues the rotate-
+        // back MMAs of the previous group (operands from the epilogue) halfway
+        // through each group, in its own stream, so they are neither starved nor
+        // on the epilogue's critical path.
+        const bool wa = warp == 13;
         if (lane == 0) {
             int stage = 0;
             uint32_t ph = 0;
@@ -1032,6 +980,34 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
             long long w_t = 0, w_f = 0;
             const long long c_start = clock64();
             constexpr uint32_t ID = idesc_f16(false), IDN = idesc_f16(true);
+            // Operand descriptors of the ring stages, built once: the issue loop only
+            // adds constant offsets (the start address field counts 16-byte units,
+            // and every stage lies below 256 KB, so the additions never carry).
+            uint64_t dbase[kNS];
+#pragma unroll
+            for (int s2 = 0; s2 < kNS; ++s2) dbase[s2] = sdesc_sw64(smem_u32(ring + (size_t)s2 * kStage));
+            constexpr uint64_t kSl = kSlot >> 4, kKs = 32 >> 4;  // descriptor steps: one slot, one K=16 step
+            const uint64_t b2base = sdesc_b2(smem_u32(b2s));
+            long long m_issue = 0, m_commit = 0, m_serv = 0;
+            uint32_t a2ph = 0;
+            long long pend = -1;  // warp A: group whose rotate-back MMAs are still to be issued
+            auto rotate_back = [&]() -> bool {  // warp A, for group `pend`
+                const long long c0 = clock64();
+                if (!wait_t(a2ready, a2ph, abort_flag, P.status, w_t)) return false;
+                a2ph ^= 1;
+                tc_fence_after();
+                const int n = req_n[0];
+                const uint32_t cbt = tmem + (uint32_t)(pend & 1) * 256u;
+                for (int k = 0; k < n; ++k) {
+                    const uint32_t rq = req[k];
+                    umma_ta(cbt + (rq & 255u), cbt + ((rq >> 8) & 255u),
+                            b2base + (uint64_t)((rq >> 16) & 255u) * (kB2Bytes >> 4), idesc_n16(), (int)(rq >> 24));
+                }
+                umma_commit(d2full);
+                pend = -1;
+                m_serv += clock64() - c0;
+                return true;
+            };
             for (int t = 0; t < ntiles && ok; ++t) {
                 for (int gi = 0; gi < ng && ok; ++gi, ++gcount) {
                     const TcGroup g = P.groups[gi];
@@ -1040,41 +1016,56 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
                     if (!wait_t(tempty + slot, (use & 1) ^ 1, abort_flag, P.status, w_t)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t d0 = tmem + slot * 256, d1 = d0 + 128;
+                    const int kind = g.mu > 0 ? 2 : (g.row0b >= 0 ? 1 : 0);
+                    const int kmid = (g.klen / kKS / 2) * kKS;
                     for (int kk = 0; kk < g.klen; kk += kKS) {
+                        if (wa && kk == kmid && pend >= 0 && !rotate_back()) { ok = false; break; }
                         if (!wait_t(full + stage, ph, abort_flag, P.status, w_f)) { ok = false; break; }
                         tc_fence_after();
-                        const uint32_t sa = smem_u32(ring + (size_t)stage * kStage);
-#pragma unroll
-                        for (int ks = 0; ks < 2; ++ks) {
-                            const uint64_t a0 = sdesc_sw64(sa + ks * 32);
-                            const uint64_t a1 = sdesc_sw64(sa + kSlot + ks * 32);
-                            const uint64_t x0 = sdesc_sw64(sa + 2 * kSlot + ks * 32);
-                            const uint64_t x1 = sdesc_sw64(sa + 3 * kSlot + ks * 32);
-                            const uint32_t acc = (kk > 0 || ks > 0) ? 1u : 0u;
-                            if (g.mu > 0) {
-                                umma(d0, a0, x0, ID, acc);    // o+ += A h+
-                                umma(d1, a1, x0, ID, acc);    // o- += B h+
-                                umma(d0, a1, x1, IDN, 1u);    // o+ -= B h-
-                                umma(d1, a0, x1, ID, 1u);     // o- += A h-
-                            } else {
-                                umma(d0, a0, x0, ID, acc);
-                                if (g.row0b >= 0) umma(d1, a1, x0, ID, acc);
+                        const long long c_i0 = dbgon ? clock64() : 0;
+                        const uint64_t a0 = dbase[stage], a1 = a0 + kSl, x0 = a0 + 2 * kSl, x1 = a0 + 3 * kSl;
+                        if (kind == 2) {
+                            if (wa) {  // o+ = A h+ - B h-
+                                if (kk == 0) umma_f(d0, a0, x0, ID, 0); else umma_f(d0, a0, x0, ID, 1);
+                                umma_f(d0, a1, x1, IDN, 1);
+                                umma_f(d0, a0 + kKs, x0 + kKs, ID, 1);
+                                umma_f(d0, a1 + kKs, x1 + kKs, IDN, 1);
+                            } else {   // o- = B h+ + A h-
+                                if (kk == 0) umma_f(d1, a1, x0, ID, 0); else umma_f(d1, a1, x0, ID, 1);
+                                umma_f(d1, a0, x1, ID, 1);
+                                umma_f(d1, a1 + kKs, x0 + kKs, ID, 1);
+                                umma_f(d1, a0 + kKs, x1 + kKs, ID, 1);
                             }
+                        } else if (wa) {
+                            if (kk == 0) umma_f(d0, a0, x0, ID, 0); else umma_f(d0, a0, x0, ID, 1);
+                            umma_f(d0, a0 + kKs, x0 + kKs, ID, 1);
+                        } else if (kind == 1) {
+                            if (kk == 0) umma_f(d1, a1, x0, ID, 0); else umma_f(d1, a1, x0, ID, 1);
+                            umma_f(d1, a1 + kKs, x0 + kKs, ID, 1);
                         }
+                        const long long c_i1 = dbgon ? clock64() : 0;
                         umma_commit(empty + stage);
                         if (++stage == kNS) { stage = 0; ph ^= 1; }
+                        if (dbgon) {
+                            const long long c_i2 = clock64();
+                            m_issue += c_i1 - c_i0; m_commit += c_i2 - c_i1;
+                        }
                     }
                     if (ok) umma_commit(tfull + slot);
+                    if (wa) pend = gcount;
                 }
             }
-            if (P.dbg) {
+            if (wa && ok && pend >= 0 && !rotate_back()) ok = false;  // the last group's rotate-back
+            if (P.dbg && wa) {
                 long long* d = P.dbg + blockIdx.x * kDbgSlots;
                 d[5] = w_t; d[6] = w_f; d[7] = clock64() - c_start;
+                d[25] = m_issue; d[26] = m_commit; d[27] = m_serv;
             }
             // every issued MMA completes (bounded wait) before TMEM is released
-            umma_commit(fin);
+            uint64_t* fb = fin + (wa ? 0 : 1);
+            umma_commit(fb);
             const uint64_t t0 = gtimer();
-            while (!mbar_try(fin, 0) && gtimer() - t0 < kWaitNs) {
+            while (!mbar_try(fb, 0) && gtimer() - t0 < kWaitNs) {
             }
         }
         __syncwarp();
@@ -1184,27 +1175,75 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
             long long* d = P.dbg + blockIdx.x * kDbgSlots;
             d[23] = w_g; d[24] = clock64() - c_start;
         }
-    } else if (warp < 12) {
-        // ---------------- epilogue (warps 0-3 and 8-11) ----------------
+    } else if (warp < 4) {
+        // ---------------- epilogue (warps 0-3) ----------------
+        // Per group, the rotate-back v = D(R)^T o weighted by the softmax and summed
+        // over each node's edges runs on the tensor cores:
+        //   1. conversion: each thread owns one TMEM lane (one output row (l3, c)) of
+        //      the group's accumulators and converts its 128 edge columns to fp16
+        //      p_e o[c, e] in place (packed into the accumulator's first 64 columns);
+        //   2. per pass over up to 8 node segments of the tile, the epilogue builds
+        //      the operand blocks B2[m'][e] = D_e^{l3}[+-mu][m'] (zero outside the
+        //      node's edges) and a list of M128 N16 K16 MMAs
+        //      D2[c][m'] += sum_e A2[c][e] B2[m'][e] (A2 = the converted operand in
+        //      TMEM), one 16-column result per node; MMA warp A issues the first
+        //      pass in its stream, the epilogue issues any further pass itself;
+        //   3. drain: out[node][l3, m'][c] += D2[c][m'] (m' < 2 l3 + 1), each output
+        //      element added by one thread (lane c) in program order, so the order
+        //      of additions is fixed.
         // Every decision to stop goes through bar_and, so the 128 threads leave
         // together and no thread is left at a named barrier.
         const int r = threadIdx.x;
+        const int row = r;                               // this thread's TMEM lane
+        const int et = r;
+        const int ew = warp;                             // epilogue warp 0..3
+        const uint32_t tlane = tmem + ((uint32_t)(32 * warp) << 16);
         long long gcount = 0;
         bool ok = true;
         long long w_x = 0, w_t = 0;
         long long staged[2] = {-1, -1};  // last group index staged into each buffer (thread 0)
+        uint32_t d2ph = 0;
+        int d2_pending = 0;  // rotate-back MMAs issued by this thread whose completion was not seen
         const long long c_start = clock64();
         for (int t = 0; t < ntiles; ++t) {
             const int b = t & 1;
             const bool okx = wait_t(xready + b, (t >> 1) & 1, abort_flag, P.status, w_x);
             if (!bar_and(2, kEpiThreads, ok && okx)) { ok = false; break; }
             const __half2* Dg = P.dscr + (size_t)(blockIdx.x * 2 + b) * dglob_pairs();
-            const float* pb = pch + (size_t)b * kTileE * (C / 8);
             const int* nb = nid + b * kTileE;
-            const uint32_t* sg = segm + b * (kTileE / kChunk);
             if (r == 0) {
                 stage_group_pairs(P.groups[0], C, Dg, dstage + (gcount & 1) * S.dstride, dbar + (gcount & 1));
                 staged[gcount & 1] = gcount;
+            }
+            // node segments of the tile (its edges are the prefix with nid >= 0)
+            if (ew == 0) {
+                int f[4], c = 0;
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const int e = 4 * lane + k;
+                    f[k] = nb[e] >= 0 && (e == 0 || nb[e] != nb[e - 1]);
+                    c += f[k];
+                }
+                int incl = c;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+                    if (lane >= o) incl += v;
+                }
+                int pos = incl - c;
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const int e = 4 * lane + k;
+                    if (f[k]) { sl_start[pos] = e; sl_node[pos] = nb[e]; ++pos; }
+                }
+                // end of the last segment: the first padding edge (or 128)
+                int ne_l = 0;
+#pragma unroll
+                for (int k = 0; k < 4; ++k) ne_l += nb[4 * lane + k] >= 0;
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) ne_l += __shfl_xor_sync(0xffffffffu, ne_l, o);
+                const int ns = __shfl_sync(0xffffffffu, incl, 31);
+                if (lane == 0) { sl_count[0] = ns; sl_start[ns] = ne_l; }
             }
             for (int gi = 0; gi < ng; ++gi, ++gcount) {
                 // all threads are done with group gcount-1, so its staging buffer can be refilled
@@ -1219,29 +1258,148 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
                 const uint32_t use = (uint32_t)(gcount >> 1);
                 const bool okd = wait_t(dbar + slot, use & 1, abort_flag, P.status, w_t);
                 const bool okt = okd && wait_t(tfull + slot, use & 1, abort_flag, P.status, w_t);
-                if (okt) {
-                    const long long c_e0 = clock64();
-                    tc_fence_after();
-                    const __half2* Ds = reinterpret_cast<const __half2*>(dstage + slot * S.dstride);
-                    const int lrow = (warp & 3) * 32 + (warp >> 3) * 16;  // this warp's 16 TMEM lanes
-                    const uint32_t twarp = tmem + ((uint32_t)lrow << 16) + slot * 256;
-                    if (g.mu > 0) {
-                        const int row = g.row0 + lrow;  // rows of this warp: one l3, 16 channels
-                        epi_mma<2>(twarp, g.mu + row / C, row % C, K, C, Ds, pb, nb, sg, P.out);
+                if (!bar_and(2, kEpiThreads, okt)) {
+                    ok = false;
+                    mbar_arrive(tempty + slot);
+                    break;
+                }
+                const long long c_e0 = clock64();
+                tc_fence_after();
+                const uint32_t cb = (uint32_t)slot * 256u;
+                const bool two = g.mu > 0 || g.row0b >= 0;
+                const int rowA = g.row0 + row, rowB = g.mu > 0 ? rowA : g.row0b + row;
+                const int cA = rowA % C, cB = rowB % C;
+                const int l3A = (g.mu > 0 ? g.mu : 0) + rowA / C, l3B = (g.mu > 0 ? g.mu : 0) + rowB / C;
+                const float* pA = php + ((size_t)b * H + cA / dh) * kTileE;
+                const float* pB = php + ((size_t)b * H + cB / dh) * kTileE;
+                // 1. conversion of this thread's 128 edge columns: o -> fp16 p o, packed in place
+#pragma unroll 1
+                for (int j = 0; j < kTileE / 16; ++j) {
+                    const int e0 = 16 * j;
+                    float v[16], w[16];
+                    tmem_ld16(tlane + cb + e0, v);
+                    if (two) tmem_ld16(tlane + cb + 128 + e0, w);
+                    tmem_wait_ld();
+                    uint32_t u[8];
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) u[k] = pack_h2(v[2 * k] * pA[e0 + 2 * k], v[2 * k + 1] * pA[e0 + 2 * k + 1]);
+                    tmem_st8(tlane + cb + a2col(j), u);
+                    if (two) {
+#pragma unroll
+                        for (int k = 0; k < 8; ++k)
+                            u[k] = pack_h2(w[2 * k] * pB[e0 + 2 * k], w[2 * k + 1] * pB[e0 + 2 * k + 1]);
+                        tmem_st8(tlane + cb + 128 + a2col(j), u);
+                    }
+                }
+                tmem_wait_st();
+                // 2./3. passes over the node segments
+                const __half2* Ds = reinterpret_cast<const __half2*>(dstage + slot * S.dstride);
+                const int nseg = sl_count[0];
+                const int per = (g.mu == 0 && g.row0b >= 0) ? 4 : 8;  // segments per pass (result regions)
+                const int NPA = npair(l3A), NPB = npair(l3B);
+                const __half2* DsB = (g.mu > 0) ? Ds : Ds + kTileE * NPA;  // m = 0: second block's pairs
+                bool okp = true;
+                for (int s0 = 0; s0 < nseg; s0 += per) {
+                    const bool first_pass = s0 == 0;
+                    const int s1 = min(nseg, s0 + per);
+                    if (et == 0) {  // request list: (result column, operand column, block, accumulate)
+                        int n = 0;
+                        for (int sg = s0; sg < s1; ++sg) {
+                            const int ea = sl_start[sg], eb = sl_start[sg + 1];
+                            const int nacc = (g.mu == 0 && g.row0b < 0) ? 1 : 2;
+                            for (int a2 = 0; a2 < nacc; ++a2) {  // mu > 0: sign +/-; mu = 0: block a/b
+                                const int dcol = (g.mu == 0 && g.row0b >= 0) ? d2col((sg - s0) + 4 * a2) : d2col(sg - s0);
+                                for (int J = ea >> 4; J <= (eb - 1) >> 4; ++J) {
+                                    const bool first = (J == (ea >> 4)) && (a2 == 0 || (g.mu == 0));
+                                    req[n] = (uint32_t)dcol | ((uint32_t)(128 * a2 + a2col(J)) << 8) | ((uint32_t)n << 16) |
+                                             ((first ? 0u : 1u) << 24);
+                                    req_bp[n] = (uint32_t)sg | ((uint32_t)a2 << 8) | ((uint32_t)J << 16);
+                                    ++n;
+                                }
+                            }
+                        }
+                        req_n[0] = n;
+                    }
+                    asm volatile("bar.sync 2, %0;" ::"n"(kEpiThreads) : "memory");
+                    // operand blocks: one warp per block; lane = (row m', 8-edge half)
+                    {
+                        const int n = req_n[0];
+                        const int mp = lane & 15, kg = lane >> 4;
+                        for (int q = ew; q < n; q += kEpiThreads / 32) {
+                            const uint32_t bp = req_bp[q];
+                            const int sg = bp & 255, a2 = (bp >> 8) & 255, J = bp >> 16;
+                            const int ea = sl_start[sg], eb = sl_start[sg + 1];
+                            const int l3 = a2 == 0 ? l3A : l3B;
+                            const int NP = (g.mu > 0) ? NPA : (a2 == 0 ? NPA : NPB);
+                            const __half2* Dq = (g.mu > 0 || a2 == 0) ? Ds : DsB;
+                            const bool hi = g.mu > 0 && a2 == 1;  // sign -: the pair's high half
+                            uint32_t pk[4];
+#pragma unroll
+                            for (int i2 = 0; i2 < 4; ++i2) {
+                                float f2[2];
+#pragma unroll
+                                for (int i1 = 0; i1 < 2; ++i1) {
+                                    const int e = 16 * J + 8 * kg + 2 * i2 + i1;
+                                    float v = 0.f;
+                                    if (e >= ea && e < eb && mp < 2 * l3 + 1) {
+                                        const __half2 pr = Dq[e * NP + mp];
+                                        v = __half2float(hi ? __high2half(pr) : __low2half(pr));
+                                    }
+                                    f2[i1] = v;
+                                }
+                                pk[i2] = pack_h2(f2[0], f2[1]);
+                            }
+                            *reinterpret_cast<uint4*>(b2s + (size_t)q * kB2Bytes + 2 * b2_off(mp, 8 * kg)) =
+                                make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                        }
+                    }
+                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // blocks -> tensor core
+                    tc_fence_before();
+                    if (first_pass) {
+                        mbar_arrive(a2ready);  // MMA warp A issues this pass in its own stream
                     } else {
-                        const int ra = g.row0 + lrow, la = ra / C;
-                        epi_mma<1>(twarp, la, ra % C, K, C, Ds, pb, nb, sg, P.out);
-                        if (g.row0b >= 0) {
-                            const int rb = g.row0b + lrow;
-                            epi_mma<1>(twarp + 128, rb / C, rb % C, K, C, Ds + kTileE * npair(la), pb, nb, sg, P.out);
+                        asm volatile("bar.sync 2, %0;" ::"n"(kEpiThreads) : "memory");
+                        if (et == 0) {
+                            tc_fence_after();
+                            const int n = req_n[0];
+                            const uint32_t cbt = tmem + cb;
+                            const uint64_t b2base = sdesc_b2(smem_u32(b2s));
+                            for (int k = 0; k < n; ++k) {
+                                const uint32_t rq = req[k];
+                                umma_ta(cbt + (rq & 255u), cbt + ((rq >> 8) & 255u),
+                                        b2base + (uint64_t)((rq >> 16) & 255u) * (kB2Bytes >> 4), idesc_n16(),
+                                        (int)(rq >> 24));
+                            }
+                            umma_commit(d2full);
+                            d2_pending = 1;
+                        }
+                    }
+                    const bool okw = wait_t(d2full, d2ph, abort_flag, P.status, w_t);
+                    if (okw) d2_pending = 0;
+                    d2ph ^= 1;
+                    if (!bar_and(2, kEpiThreads, okw)) { okp = false; break; }
+                    tc_fence_after();
+                    // drain: lane c of this warp owns out[node][l3, m'][c]
+                    for (int sg = s0; sg < s1; ++sg) {
+                        const int node = sl_node[sg];
+                        const int nacc = (g.mu == 0 && g.row0b >= 0) ? 2 : 1;
+                        for (int a2 = 0; a2 < nacc; ++a2) {
+                            const int dcol = nacc == 2 ? d2col((sg - s0) + 4 * a2) : d2col(sg - s0);
+                            float v[16];
+                            tmem_ld16(tlane + cb + dcol, v);
+                            tmem_wait_ld();
+                            const int l3 = a2 == 0 ? l3A : l3B, c = a2 == 0 ? cA : cB;
+                            float* o = P.out + ((size_t)node * K + l3 * l3) * C + c;
+#pragma unroll
+                            for (int mp = 0; mp < 2 * kMaxL + 1; ++mp)
+                                if (mp < 2 * l3 + 1) atomicAdd(o + (size_t)mp * C, v[mp]);
                         }
                     }
                     tc_fence_before();
-                    if (dbgon && r == 0) dsub[8] += clock64() - c_e0;
-                } else {
-                    ok = false;
                 }
+                if (dbgon && r == 0) dsub[8] += clock64() - c_e0;
                 mbar_arrive(tempty + slot);
+                if (!okp) { ok = false; }
             }
             if (!bar_and(2, kEpiThreads, ok)) { ok = false; break; }
             mbar_arrive(xfree + b);
@@ -1249,6 +1407,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
         if (P.dbg && r == 0) {
             long long* d = P.dbg + blockIdx.x * kDbgSlots;
             d[8] = w_x; d[9] = w_t; d[10] = clock64() - c_start; d[13] = ntiles; d[22] = dsub[8];
+        }
+        // rotate-back MMAs issued but not seen to complete finish before TMEM is released
+        if (d2_pending) {
+            const uint64_t t0 = gtimer();
+            while (!mbar_try(d2full, d2ph ^ 1) && gtimer() - t0 < kWaitNs) {
+            }
         }
         // a staging copy that was issued but never waited for lands before exit
         if (r == 0) {
