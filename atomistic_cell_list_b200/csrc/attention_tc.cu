@@ -19,23 +19,20 @@
 // fills the other.
 //
 // Warp roles (512 threads, 128 registers each):
-//   0-3        epilogue (warp w: TMEM lanes 32w..32w+31): converts a group's
-//              accumulators in place to fp16 p * o (p = softmax weight of the
-//              edge and the row's head), builds per-node Wigner operand blocks
-//              and drains the rotate-back results D2 = (p o) D into out[node]
-//              (one owner thread per element: fixed order)
+//   0-3, 8-11  epilogue: tcgen05.ld 16x256b fragments of the accumulators;
+//              rotate-back p * D^l3(R)^T restricted to the group's |m| rows
+//              on mma.sync, summed over each node's edges, added to
+//              out[node] (one owner thread per element: fixed order)
 //   4-7        producer: per edge the node, frame, Wigner blocks (fp16 pairs,
 //              shared and global copies); per (edge, head) the softmax weight
 //              p = exp(a - lse) (statistics from an O(N) pre-pass); per
 //              (edge, 8 channels) the gathered, gated, rotated features,
 //              written once per tile to a per-CTA global scratch row for TMA
-//   8, 13      tcgen05.mma issue (one thread each): warp 13 the first
-//              accumulator of a group and the rotate-back MMAs (A operand in
-//              TMEM) of the previous group, warp 8 the second accumulator
 //   12         TMA loads of weight and feature tiles into a 3-stage ring
+//   13         tcgen05.mma issue (one thread), commits to the ring and TMEM
+//              barriers
 //   14-15      value gates rho(d) W_rad of a tile (mma.sync), up to two tiles
 //              ahead of the producer, into a double-buffered global scratch
-//   9-11       idle
 // Every mbarrier wait is bounded by the global timer; on expiry the kernel
 // records E2F_ERR_TIMEOUT, drains what it issued and returns.
 #include <cuda.h>
@@ -345,15 +342,18 @@ __device__ __forceinline__ void mma_16816(float* d, const uint32_t* a, const uin
 // ----------------------------------------------------------------------------
 // main kernel
 // ----------------------------------------------------------------------------
-constexpr int kTileE = 128;                   // edges of a pair tile (MMA N)
-constexpr int kHalfE = 64;                    // edges of a pair tile held by each CTA
+constexpr int kTileE = 128;
 constexpr int kKS = 32;                       // K per ring stage
-constexpr int kNS = 5;                        // ring stages
-constexpr int kWSlot = 128 * kKS * 2;         // 8 KB weight tile (128 rows of this CTA)
-constexpr int kXSlot = kHalfE * kKS * 2;      // 4 KB feature tile (this CTA's 64 edges)
-constexpr int kStage = 2 * kWSlot + 2 * kXSlot;
+constexpr int kNS = 3;                        // ring stages
+constexpr int kSlot = kTileE * kKS * 2;       // 8 KB per operand tile
+constexpr int kStage = 4 * kSlot;
 constexpr int kThreads = 512;
-constexpr int kEpiThreads = 128;
+// Warp roles (16 warps, 65536 / 512 = 128 registers per thread):
+//   0-3, 8-11  epilogue (warp w: TMEM lane quadrant w % 4, lane half w / 8)
+//   4-7        producer
+//   12         TMA, 13 MMA, 14-15 idle
+constexpr int kEpiThreads = 256;
+constexpr int kChunk = 16;                    // epilogue: edges per TMEM load
 
 // Wigner blocks of an edge in "pair" form: for each degree l and each
 // |m| = mu <= l the 2l+1 pairs (D^l[+mu][n], D^l[-mu][n]) as fp16x2, padded
@@ -370,55 +370,50 @@ __host__ __device__ constexpr int dptotal(int L) { return dpo(L + 1, 0); }  // 1
 // shared copy (producer): [edge][dptotal + 4] pairs; the 4 spare pairs move
 // consecutive edges 4 banks apart
 __host__ __device__ constexpr int dph_stride(int L) { return dptotal(L) + 4; }
-// global copy (epilogue), per CTA and tile buffer, block-major: block (l, mu)
-// holds npair(l) x the CTA's 64 edges (pair index outer, edge inner), so each
-// CTA's part of a group's slice is one bulk copy and the epilogue reads a
-// pair for 8 consecutive edges with two 16-byte loads
-__host__ __device__ constexpr size_t dglob_pairs() { return (size_t)kHalfE * dptotal(kMaxL); }
-__host__ __device__ constexpr size_t dglob_block(int l, int mu) { return (size_t)kHalfE * dpo(l, mu); }
+// global copy (epilogue), per tile buffer, block-major: block (l, mu) holds
+// 128 edges x npair(l) pairs, so a group's slice is one bulk copy
+__host__ __device__ constexpr size_t dglob_pairs() { return (size_t)kTileE * dptotal(kMaxL); }
+__host__ __device__ constexpr size_t dglob_block(int l, int mu) { return (size_t)kTileE * dpo(l, mu); }
 static_assert(npair(0) == 4 && npair(1) == 4 && npair(2) == 8 && npair(3) == 8 && npair(4) == 12, "pairs");
 static_assert(dptotal(4) == 128, "pair layout");
 
-// Bytes of Wigner pairs one group's epilogue stages in a CTA: npair(l)
-// pairs of 4 bytes per edge of the pair tile for each of the CTA's one or two
-// accumulators (their degrees may differ).
+// Bytes of Wigner pairs one group's epilogue stages: npair(l) pairs of 4
+// bytes per edge for each feature block the group covers (m = 0 groups cover
+// two 128-row blocks, possibly of different degrees).
 __host__ __device__ inline size_t stage_bytes(int L, int C) {
-    (void)C;
-    return (size_t)kTileE * 4 * 2 * npair(L);
+    size_t mx = (size_t)kTileE * 4 * npair(L);  // an |m| >= 1 group of degree L
+    const int n0 = (L + 1) * C;
+    for (int r0 = 0; r0 < n0; r0 += 256) {
+        const int la = r0 / C, lb = (r0 + 128 < n0) ? (r0 + 128) / C : -1;
+        size_t b = (size_t)kTileE * 4 * npair(la);
+        if (lb >= 0) b += (size_t)kTileE * 4 * npair(lb);
+        mx = b > mx ? b : mx;
+    }
+    return mx;
 }
-
-// Rotate-back contraction on the tensor cores (see the epilogue): per pass at
-// most kB2Blocks operand blocks of 16 rows (m') x 16 edges, fp16.
-constexpr int kB2Blocks = 24;  // per buffer; two buffers
-constexpr int kB2Bytes = 512;  // this CTA's 16 rows (m') x 16 edges of a 32-row pair operand
 
 // Shared memory layout (bytes), shared by host (size) and device (offsets).
 struct SmemLayout {
-    size_t ring, dstage, dstride, dph, php, nid, jn, rpw, rho, rrs, wga, b2, slots, req, bars, misc, dsub, total;
+    size_t ring, dstage, dstride, dph, pch, nid, jn, segm, rpw, rho, rrs, wga, bars, misc, dsub, total;
     __host__ __device__ SmemLayout(int L, int C, int H, int n_rbf) {
         size_t o = 0;
         ring = o;   o += (size_t)kNS * kStage;
         dstride = (stage_bytes(L, C) + 127) & ~size_t(127);
         dstage = o; o += 2 * dstride;
-        dph = o;    o += (size_t)kHalfE * dph_stride(L) * 4;
-        php = o;    o += 2ull * H * kTileE * 4;          // [2][H][128] softmax weight per head and pair-tile edge
-        nid = o;    o += 2ull * kTileE * 4;              // [2][128] node of each pair-tile edge
-        jn = o;     o += 2ull * kHalfE * 4;              // [2][64] neighbour of each of this CTA's edges
+        dph = o;    o += (size_t)kTileE * dph_stride(L) * 4;
+        pch = o;    o += 2ull * kTileE * (C / 8) * 4;
+        nid = o;    o += 2ull * kTileE * 4;
+        jn = o;     o += 2ull * kTileE * 4;
+        segm = o;   o += 2ull * (kTileE / kChunk) * 4;
         rpw = o;    o += (size_t)kTileE * 4;
-        rho = o;    o += (size_t)kHalfE * kTcMaxRbf * 2;
-        rrs = o;    o += (size_t)kHalfE * kTcMaxRbf * 4;
+        rho = o;    o += (size_t)kTileE * kTcMaxRbf * 2;
+        rrs = o;    o += (size_t)kTileE * kTcMaxRbf * 4;
         wga = o;    o += (size_t)kTcMaxRbf * kMaxHeads * 4;
-        o = (o + 1023) & ~size_t(1023);
-        b2 = o;     o += 2ull * kB2Blocks * kB2Bytes;     // rotate-back operand blocks, two buffers
-        slots = o;  o += (2 * kTileE + 8) * 4;            // node segments of the tile: start, node, count
-        req = o;    o += 2 * ((2 * kB2Blocks + 4) * 4) + 16;  // per buffer: MMA requests, header, block parameters; mailbox
-        o += 3 * 2 * kB2Blocks * 4 + 16;                      // first-pass lists per group kind (per tile), counts
         o = (o + 7) & ~size_t(7);
-        bars = o;   o += (2 * kNS + 20) * 8;
-        misc = o;   o += 64 + 4 * kHalfE * 4;  // TMEM base, abort flag, last slot; gate (i, j) lists
+        bars = o;   o += (2 * kNS + 17) * 8;
+        misc = o;   o += 64 + 4 * kTileE * 4;  // TMEM base, abort flag, last slot; gate (i, j) lists
         dsub = o;   o += 16 * 8;
         total = o;
-        (void)n_rbf;
     }
 };
 
@@ -459,231 +454,155 @@ __device__ __forceinline__ void tmem_ld_16x256(uint32_t taddr, uint32_t* r) {
                  : "memory");
 }
 
-// tcgen05.mma kind::f16 with the accumulate flag as an immediate (no predicate setup in the issue loop)
-__device__ __forceinline__ void umma_f(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, int accumulate) {
-    if (accumulate)
-        asm volatile("tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, 1;" ::"r"(d), "l"(a), "l"(b), "r"(idesc)
-                     : "memory");
-    else
-        asm volatile("tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, 0;" ::"r"(d), "l"(a), "l"(b), "r"(idesc)
-                     : "memory");
-}
-
 __device__ __forceinline__ uint32_t pack_h2(float a, float b) {
     __half2 h = __floats2half2_rn(a, b);
     return *reinterpret_cast<uint32_t*>(&h);
 }
 
-__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t* r) {
-    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(r[0]),
-                 "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
-                 : "memory");
-}
-__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+// Epilogue of one accumulator pair (o+ at tacc, o- at tacc + 128) or one
+// accumulator (SIGNS = 1) holding output rows (l3, channel) for the tile's
+// 128 edges, on mma.sync: per 16-edge chunk and 8 channels,
+//     acc[m'][c] += sum_e D_e[+mu][m'] y+[e][c] + D_e[-mu][m'] y-[e][c],
+//     y[e][c] = p_e^{head(c)} o[c][e],
+// i.e. the rotate-back D^T of the |m| = mu rows weighted by the softmax and
+// summed over the node's edges. A = Wigner rows (m' padded to 16, built from
+// the staged fp16 pairs), B = p * o straight from tcgen05.ld.16x256b (whose
+// thread layout is the mma B/D fragment layout), D = fp32 accumulators.
+// Node sums go to out with fire-and-forget reductions at segment ends: one
+// thread owns each (node, l3, m', c) element, so the additions happen in
+// program order. The warp covers 16 TMEM lanes (channels cbase..cbase+15);
+// the two warps of a lane quadrant take one half each.
+template <int SIGNS>
+__device__ __noinline__ void epi_mma(uint32_t tacc, int l3, int cbase, int K, int C,
+                                     const __half2* __restrict__ Ds, const float* __restrict__ pch,
+                                     const int* __restrict__ nb, const uint32_t* __restrict__ segm,
+                                     float* __restrict__ out) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
+    const int W3 = 2 * l3 + 1, NP = npair(l3), C8 = C / 8;
+    float acc[2][4];  // [n-tile lo/hi][fragment]
+#pragma unroll
+    for (int b2 = 0; b2 < 2; ++b2)
+#pragma unroll
+        for (int r = 0; r < 4; ++r) acc[b2][r] = 0.f;
+    int cur = -1;
+    const float* pc = pch + cbase / 8;  // 8-channel groups cbase/8 (lh = 0) and +1 (lh = 1)
 
-// Rotate-back operand block: 16 rows (m') x 16 K (edges) fp16, no swizzle,
-// K-major core matrices (8 rows x 16 bytes) 128 bytes apart along K and 256
-// bytes apart along rows. Element (m', k) in halves:
-__device__ __forceinline__ int b2_off(int mp, int k) { return ((mp >> 3) * 2 + (k >> 3)) * 64 + (mp & 7) * 8 + (k & 7); }
-__device__ __forceinline__ uint64_t sdesc_b2(uint32_t saddr) {
-    uint64_t d = 0;
-    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
-    d |= (uint64_t)(128u >> 4) << 16;   // leading byte offset: next core matrix along K
-    d |= (uint64_t)(256u >> 4) << 32;   // stride byte offset: next 8-row group
-    d |= (uint64_t)1u << 46;            // descriptor version (sm_100)
-    return d;                           // swizzle: none
-}
-// kind::f16, D fp32, A and B fp16, K-major, M = 256 (a CTA pair), N = n, optional negation of A
-__host__ __device__ constexpr uint32_t idesc_pair(int n, bool neg_a) {
-    return (1u << 4) | ((neg_a ? 1u : 0u) << 13) | ((uint32_t)(n >> 3) << 17) | ((256u >> 4) << 24);
-}
+    auto flush = [&]() {
+        if (cur < 0) return;
+#pragma unroll
+        for (int lh = 0; lh < 2; ++lh)
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                const int mp = g + ((r >> 1) << 3);
+                if (mp < W3) {
+                    const int c = cbase + 8 * lh + 2 * q + (r & 1);
+                    atomicAdd(out + ((size_t)cur * K + l3 * l3 + mp) * C + c, acc[lh][r]);
+                }
+                acc[lh][r] = 0.f;
+            }
+    };
 
-__device__ __forceinline__ void umma_ta(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc, int accumulate) {
-    if (accumulate)
-        asm volatile("tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, 1;" ::"r"(d), "r"(a_tmem), "l"(b),
-                     "r"(idesc)
-                     : "memory");
-    else
-        asm volatile("tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, 0;" ::"r"(d), "r"(a_tmem), "l"(b),
-                     "r"(idesc)
-                     : "memory");
-}
-
-// TMEM column (within an accumulator's 128) of the fp16 operand of edges
-// 16J..16J+15 after the in-place conversion (two fp16 per 32-bit column).
-__device__ __forceinline__ int a2col(int J) { return 8 * J; }
-// Rotate-back result regions (32 columns each, N of the pair MMA) inside a
-// group's 256 columns: the halves of the two accumulators that the conversion
-// has freed. In region k, CTA r's results are columns 16r..16r+15.
-__device__ __forceinline__ int d2col(int k) { return 64 + 32 * (k & 1) + 128 * (k >> 1); }
-
-// Wigner slice a CTA's accumulator needs: block (l3, mu) for the 128 edges of
-// the pair tile, the first 64 from the even CTA's global copy and the rest
-// from the odd CTA's (Dg0, Dg1). Queued on `bar` into `dst`; returns bytes.
-__device__ __forceinline__ uint32_t stage_block(int l3, int mu, const __half2* Dg0, const __half2* Dg1, uint8_t* dst,
-                                                uint64_t* bar) {
-    const uint32_t half = (uint32_t)kHalfE * npair(l3) * 4;
-    bulk_load(dst, Dg0 + dglob_block(l3, mu), half, bar);
-    bulk_load(dst + half, Dg1 + dglob_block(l3, mu), half, bar);
-    return 2 * half;
-}
-
-
-// Degree, channel and validity of this CTA's rows of accumulator a (a2 = 0) or b
-// (a2 = 1, m = 0 groups) of group g for TMEM lane `row`: rows r0 + 128 rank + row of
-// the group's block (o+/o- share the rows when mu > 0).
-__device__ __forceinline__ void epi_rows(const TcGroup& g, int a2, int rank, int row, int L, int C, int& l3, int& c,
-                                         bool& valid) {
-    const int nrow = g.mu > 0 ? (L + 1 - g.mu) * C : (L + 1) * C;
-    const int r0 = (a2 == 0 || g.mu > 0) ? g.row0 : g.row0b;
-    const int rr = r0 + 128 * rank;
-    valid = r0 >= 0 && rr < nrow;
-    const int rc = valid ? rr + row : 0;
-    l3 = (g.mu > 0 ? g.mu : 0) + (valid ? rr / C : 0);
-    c = rc % C;
-}
-
-// Shared state of the epilogue's rotate-back passes (pointers into shared memory).
-struct EpiShared {
-    const int* sl_start;   // [segments + 1] first edge of each node segment, then the end
-    uint32_t* req0;        // per buffer: requests [kB2Blocks], header [4], block parameters [kB2Blocks]
-    uint8_t* b2s;          // operand blocks, two buffers
-    const uint8_t* dstage; // staged Wigner slices, two buffers of dstride bytes
-    size_t dstride;
-};
-__device__ __forceinline__ uint32_t* epi_req(const EpiShared& E, int q) { return E.req0 + q * (2 * kB2Blocks + 4); }
-__device__ __forceinline__ int* epi_reqh(const EpiShared& E, int q) {
-    return reinterpret_cast<int*>(E.req0 + q * (2 * kB2Blocks + 4) + kB2Blocks);
-}
-__device__ __forceinline__ uint32_t* epi_reqbp(const EpiShared& E, int q) {
-    return E.req0 + q * (2 * kB2Blocks + 4) + kB2Blocks + 4;
-}
-
-// Request list of a rotate-back pass over segments [s0, s1) for a group kind: 0 =
-// one m = 0 block (one accumulator), 1 = two m = 0 blocks (a, b), 2 = |m| >= 1
-// (signs +, -). Entry: (result column, operand column, block, accumulate); block
-// parameters: (segment, accumulator, 16-edge step). Returns the entry count.
-__device__ __forceinline__ int epi_build_list(const int* sl_start, int kind, int s0, int s1, uint32_t* rl, uint32_t* bpl) {
-    int n = 0;
-    const int nacc = kind == 0 ? 1 : 2;
-    for (int sg = s0; sg < s1; ++sg) {
-        const int ea = sl_start[sg], eb = sl_start[sg + 1];
-        for (int a2 = 0; a2 < nacc; ++a2) {
-            const int dcol = kind == 1 ? d2col((sg - s0) + 2 * a2) : d2col(sg - s0);
-            for (int J = ea >> 4; J <= (eb - 1) >> 4; ++J) {
-                const bool first = (J == (ea >> 4)) && (a2 == 0 || kind != 2);
-                rl[n] = (uint32_t)dcol | ((uint32_t)(128 * a2 + a2col(J)) << 8) | ((uint32_t)n << 16) |
-                        ((first ? 0u : 1u) << 24);
-                bpl[n] = (uint32_t)sg | ((uint32_t)a2 << 8) | ((uint32_t)J << 16);
-                ++n;
+#pragma unroll 1
+    for (int ch = 0; ch < kTileE / 16; ++ch) {
+        const int e0 = ch * 16;
+        // o values: [sign][edge half][4]: (c_lo,e), (c_lo,e+1), (c_hi,e), (c_hi,e+1)
+        uint32_t ov[SIGNS][2][4];
+#pragma unroll
+        for (int s2 = 0; s2 < SIGNS; ++s2)
+#pragma unroll
+            for (int eh = 0; eh < 2; ++eh) tmem_ld_16x256(tacc + s2 * 128 + e0 + 8 * eh, ov[s2][eh]);
+        // this thread's four edges: e0 + 2q, +1, e0 + 8 + 2q, +1
+        const int ea = e0 + 2 * q, eb = e0 + 8 + 2 * q;
+        // Wigner A fragments per sign: rows m' = g (a0, a2) and g + 8 (a1, a3)
+        uint32_t af[SIGNS][4];
+        {
+            const bool r0 = g < W3, r1 = g + 8 < W3;
+            const __half2 z = __float2half2_rn(0.f);
+            const __half2 p00 = r0 ? Ds[ea * NP + g] : z, p01 = r0 ? Ds[(ea + 1) * NP + g] : z;
+            const __half2 p10 = r1 ? Ds[ea * NP + g + 8] : z, p11 = r1 ? Ds[(ea + 1) * NP + g + 8] : z;
+            const __half2 p20 = r0 ? Ds[eb * NP + g] : z, p21 = r0 ? Ds[(eb + 1) * NP + g] : z;
+            const __half2 p30 = r1 ? Ds[eb * NP + g + 8] : z, p31 = r1 ? Ds[(eb + 1) * NP + g + 8] : z;
+            const __half2 lo[4] = {__lows2half2(p00, p01), __lows2half2(p10, p11), __lows2half2(p20, p21),
+                                   __lows2half2(p30, p31)};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) af[0][k] = *reinterpret_cast<const uint32_t*>(&lo[k]);
+            if (SIGNS == 2) {
+                const __half2 hi[4] = {__highs2half2(p00, p01), __highs2half2(p10, p11), __highs2half2(p20, p21),
+                                       __highs2half2(p30, p31)};
+#pragma unroll
+                for (int k = 0; k < 4; ++k) af[SIGNS - 1][k] = *reinterpret_cast<const uint32_t*>(&hi[k]);
             }
         }
-    }
-    return n;
-}
-
-// This CTA's operand blocks for a rotate-back pass of group gg (global group count
-// gc2) from a request list (rl, bpl, n entries) into buffer gc2 & 1, and the
-// buffer's header. Called by all epilogue threads; et = thread index, ew = warp.
-// A warp takes blocks ew, ew + 4, ...: all their loads are issued before any is
-// used.
-constexpr int kBlkPerWarp = (kB2Blocks + kEpiThreads / 32 - 1) / (kEpiThreads / 32);
-__device__ __forceinline__ void epi_prep_pass(const EpiShared& E, const TcGroup& gg, long long gc2, const uint32_t* rl,
-                                              const uint32_t* bpl, int n, int rank, int L, int C, int et, int ew,
-                                              int lane, long long* dt) {
-    const long long t0 = dt ? clock64() : 0;
-    const int q = (int)(gc2 & 1);
-    int l3a, ca, l3b, cb2;
-    bool va, vb;
-    epi_rows(gg, 0, rank, 0, L, C, l3a, ca, va);
-    epi_rows(gg, 1, rank, 0, L, C, l3b, cb2, vb);
-    if (gg.mu > 0) { l3b = l3a; vb = va; }
-    const bool tb = gg.mu == 0 && gg.row0b >= 0;
-    if (et == 0) {
-        epi_reqh(E, q)[0] = n;
-        epi_reqh(E, q)[1] = q;  // TMEM slot of the group
-        reinterpret_cast<const uint32_t**>(epi_reqh(E, q) + 2)[0] = rl;  // the list warp A issues
-    }
-    const long long t1 = dt ? clock64() : 0;
-    const uint8_t* dsl = E.dstage + q * E.dstride;
-    const int npa = npair(l3a);
-    const int mp = lane & 15, kg = lane >> 4;
-    const bool hi_sign = gg.mu > 0;
-    long long tl = 0;
-    for (int i0 = 0; i0 < kBlkPerWarp; i0 += 3) {  // three blocks in flight at a time
-        uint4 pr[3][2];
-        int eaa[3], ebb[3], e0a[3];
-        bool hia[3];
+        // softmax weights of the four edges for the two 8-channel groups
+        const float2 w0 = *reinterpret_cast<const float2*>(pc + ea * C8);
+        const float2 w1 = *reinterpret_cast<const float2*>(pc + (ea + 1) * C8);
+        const float2 w2 = *reinterpret_cast<const float2*>(pc + eb * C8);
+        const float2 w3 = *reinterpret_cast<const float2*>(pc + (eb + 1) * C8);
+        const float pw[2][4] = {{w0.x, w1.x, w2.x, w3.x}, {w0.y, w1.y, w2.y, w3.y}};
+        tmem_wait_ld();
+        // segments of this chunk: bit k = edge e0 + k starts a node
+        uint32_t bits = segm[ch];
+        int lo = 0;
+        if (bits & 1u) {
+            flush();
+            cur = nb[e0];
+        }
+        bits &= ~1u;
+        while (true) {
+            const int hi = bits ? __ffs(bits) - 1 : 16;
+            // edge masks of this thread's four edges for [lo, hi)
+            const float m0 = (2 * q >= lo && 2 * q < hi) ? 1.f : 0.f;
+            const float m1 = (2 * q + 1 >= lo && 2 * q + 1 < hi) ? 1.f : 0.f;
+            const float m2 = (8 + 2 * q >= lo && 8 + 2 * q < hi) ? 1.f : 0.f;
+            const float m3 = (9 + 2 * q >= lo && 9 + 2 * q < hi) ? 1.f : 0.f;
 #pragma unroll
-        for (int i = 0; i < 3; ++i) {
-            const int k = ew + (i0 + i) * (kEpiThreads / 32);
-            pr[i][0] = make_uint4(0, 0, 0, 0);
-            pr[i][1] = make_uint4(0, 0, 0, 0);
-            eaa[i] = 0; ebb[i] = 0; e0a[i] = 0; hia[i] = false;
-            if (k < n) {
-                const uint32_t bp = bpl[k];
-                const int sg = bp & 255, a2 = (bp >> 8) & 255, J = bp >> 16;
-                eaa[i] = E.sl_start[sg];
-                ebb[i] = E.sl_start[sg + 1];
-                const int l3 = a2 == 0 ? l3a : l3b;
-                const bool vv = a2 == 0 ? va : vb;
-                const int NP = npair(l3);
-                const __half2* Dq = reinterpret_cast<const __half2*>(dsl) + ((tb && a2 == 1) ? kTileE * npa : 0);
-                hia[i] = hi_sign && a2 == 1;  // sign -: the pair's high half
-                const int e0 = 16 * J + 8 * kg;  // this lane's 8 edges (one half of the pair tile)
-                e0a[i] = e0;
-                if (vv && mp < 2 * l3 + 1) {
-                    const uint4* src = reinterpret_cast<const uint4*>(Dq + ((e0 >> 6) * NP + mp) * kHalfE + (e0 & 63));
-                    pr[i][0] = src[0];
-                    pr[i][1] = src[1];
+            for (int lh = 0; lh < 2; ++lh) {
+                const float* pwv = pw[lh];
+#pragma unroll
+                for (int s2 = 0; s2 < SIGNS; ++s2) {
+                    const uint32_t* va = ov[s2][0];
+                    const uint32_t* vb = ov[s2][1];
+                    uint32_t bf[2];
+                    bf[0] = pack_h2(pwv[0] * m0 * __uint_as_float(va[2 * lh]),
+                                    pwv[1] * m1 * __uint_as_float(va[2 * lh + 1]));
+                    bf[1] = pack_h2(pwv[2] * m2 * __uint_as_float(vb[2 * lh]),
+                                    pwv[3] * m3 * __uint_as_float(vb[2 * lh + 1]));
+                    mma_16816(acc[lh], af[s2], bf);
                 }
             }
+            if (hi == 16) break;
+            flush();
+            cur = nb[e0 + hi];
+            lo = hi;
+            bits &= bits - 1;
         }
-        if (dt) tl -= clock64();
-#pragma unroll
-        for (int i = 0; i < 3; ++i) {
-            const int k = ew + (i0 + i) * (kEpiThreads / 32);
-            if (k < n) {
-                const __half2* ph = reinterpret_cast<const __half2*>(pr[i]);
-                uint32_t pk[4];
-#pragma unroll
-                for (int i2 = 0; i2 < 4; ++i2) {
-                    float f2[2];
-#pragma unroll
-                    for (int i1 = 0; i1 < 2; ++i1) {
-                        const int e = e0a[i] + 2 * i2 + i1;
-                        const __half2 pv = ph[2 * i2 + i1];
-                        f2[i1] = (e >= eaa[i] && e < ebb[i]) ? __half2float(hia[i] ? __high2half(pv) : __low2half(pv)) : 0.f;
-                    }
-                    pk[i2] = pack_h2(f2[0], f2[1]);
-                }
-                *reinterpret_cast<uint4*>(E.b2s + (size_t)q * kB2Blocks * kB2Bytes + (size_t)k * kB2Bytes +
-                                          2 * b2_off(mp, 8 * kg)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-            }
-        }
-        if (dt) tl += clock64();
     }
-    const long long t2 = dt ? clock64() - tl : 0;  // (loads and stores are timed together below)
-    const long long t3 = dt ? clock64() : 0;
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // blocks -> tensor core
-    if (dt) {
-        const long long t4 = clock64();
-        dt[0] += t1 - t0; dt[1] += t2 - t1; dt[2] += t3 - t2; dt[3] += t4 - t3;
-    }
+    flush();
 }
 
-// 16 accumulator columns of chunk j (edges 16j..16j+15) -> fp16 p o, packed into
-// 8 columns in place (p = softmax weights of the row's head, 16 floats)
-__device__ __forceinline__ void epi_convert16(uint32_t taddr_acc, const float* v, const float* p16, int j) {
-    const float4* p4 = reinterpret_cast<const float4*>(p16);
-    uint32_t u[8];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        const float4 pa = p4[k];
-        u[2 * k] = pack_h2(v[4 * k] * pa.x, v[4 * k + 1] * pa.y);
-        u[2 * k + 1] = pack_h2(v[4 * k + 2] * pa.z, v[4 * k + 3] * pa.w);
+// Wigner slice(s) a group's epilogue needs, by block (l, mu): returns bytes
+// queued on `bar` into staging buffer `dst`.
+__device__ __forceinline__ uint32_t stage_group_pairs(const TcGroup& g, int C, const __half2* Dglob, uint8_t* dst,
+                                                      uint64_t* bar) {
+    if (g.mu > 0) {
+        const int l3 = g.mu + g.row0 / C;
+        const uint32_t bytes = (uint32_t)kTileE * npair(l3) * 4;
+        mbar_arrive_tx(bar, bytes);
+        bulk_load(dst, Dglob + dglob_block(l3, g.mu), bytes, bar);
+        return bytes;
     }
-    tmem_st8(taddr_acc + a2col(j), u);
+    const int la = g.row0 / C;
+    const uint32_t ba = (uint32_t)kTileE * npair(la) * 4;
+    uint32_t bb = 0;
+    int lb = -1;
+    if (g.row0b >= 0) {
+        lb = g.row0b / C;
+        bb = (uint32_t)kTileE * npair(lb) * 4;
+    }
+    mbar_arrive_tx(bar, ba + bb);
+    bulk_load(dst, Dglob + dglob_block(la, 0), ba, bar);
+    if (lb >= 0) bulk_load(dst + ba, Dglob + dglob_block(lb, 0), bb, bar);
+    return ba + bb;
 }
 
 template <int L>
@@ -700,70 +619,45 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
     uint8_t* ring = smem + S.ring;
     uint8_t* dstage = smem + S.dstage;
     __half2* dph = reinterpret_cast<__half2*>(smem + S.dph);
-    float* php = reinterpret_cast<float*>(smem + S.php);  // [2][H][128] softmax weight per head and edge
-    int* nid = reinterpret_cast<int*>(smem + S.nid);      // [2][128]
-    int* jn = reinterpret_cast<int*>(smem + S.jn);        // [2][64]
-    uint8_t* b2s = smem + S.b2;                                   // rotate-back operand blocks
-    int* sl_start = reinterpret_cast<int*>(smem + S.slots);       // [129] first edge of each node segment
-    int* sl_node = sl_start + kTileE + 1;                         // [128] its node
-    int* sl_count = sl_node + kTileE;                             // number of segments
-    // per buffer q: req(q)[kB2Blocks] MMA requests, reqh(q)[4] count and TMEM slot,
-    // reqbp(q)[kB2Blocks] block parameters; mailbox: buffer of the pass being handed over
-    uint32_t* req0 = reinterpret_cast<uint32_t*>(smem + S.req);
-    auto req = [=](int q) { return req0 + q * (2 * kB2Blocks + 4); };
-    auto reqh = [=](int q) { return reinterpret_cast<int*>(req0 + q * (2 * kB2Blocks + 4) + kB2Blocks); };
-    auto reqbp = [=](int q) { return req0 + q * (2 * kB2Blocks + 4) + kB2Blocks + 4; };
-    volatile int* mailbox = reinterpret_cast<volatile int*>(req0 + 2 * (2 * kB2Blocks + 4));
-    // first-pass request lists of the current tile per group kind (0: one m = 0 block, 1: two
-    // m = 0 blocks, 2: |m| >= 1): entries [kB2Blocks], block parameters [kB2Blocks]; counts
-    uint32_t* klist = req0 + 2 * (2 * kB2Blocks + 4) + 4;
-    int* klistn = reinterpret_cast<int*>(klist + 3 * 2 * kB2Blocks);
+    float* pch = reinterpret_cast<float*>(smem + S.pch);  // [2][128][C/8] softmax weight per 8 channels
+    int* nid = reinterpret_cast<int*>(smem + S.nid);
+    int* jn = reinterpret_cast<int*>(smem + S.jn);
+    uint32_t* segm = reinterpret_cast<uint32_t*>(smem + S.segm);
     int* rpw = reinterpret_cast<int*>(smem + S.rpw);
-    __half* rho = reinterpret_cast<__half*>(smem + S.rho);  // [64][16] radial basis, fp16 (gate warps)
-    float* rrs = reinterpret_cast<float*>(smem + S.rrs);    // [64][16] radial basis, fp32 (logits)
+    __half* rho = reinterpret_cast<__half*>(smem + S.rho);  // [128][16] radial basis, fp16 (gate warps)
+    float* rrs = reinterpret_cast<float*>(smem + S.rrs);    // [128][16] radial basis, fp32 (logits)
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S.bars);
-    uint64_t* full = bars;            // stage landed in both CTAs (even CTA's barrier; TMA transactions)
-    uint64_t* empty = bars + kNS;     // stage consumed (both MMA warps of the even CTA, to both CTAs)
-    uint64_t* tfull = bars + 2 * kNS; // accumulator slot complete (both MMA warps, to both CTAs)
-    uint64_t* tempty = tfull + 2;     // accumulator slot drained (even CTA's barrier; both epilogues)
-    uint64_t* xready = tempty + 2;    // tile buffer produced (both producers, to both CTAs)
-    uint64_t* xfree = xready + 2;     // tile buffer consumed (both epilogues, to both CTAs)
-    uint64_t* dbar = xfree + 2;       // epilogue Wigner staging, per buffer
-    uint64_t* fin = dbar + 2;         // [2] final commits of the two MMA warps
-    uint64_t* gfull = fin + 2;        // value gate of a tile buffer written (gate warps -> producer)
-    uint64_t* gempty = gfull + 2;     // value gate of a tile buffer consumed (producer -> gate warps)
-    uint64_t* jfull = gempty + 2;     // fused traversal: (i, j) of a tile buffer listed (gate warps -> producer)
-    uint64_t* d2full = jfull + 2;     // rotate-back MMAs of a pass complete (to both CTAs)
-    uint64_t* a2ready = d2full + 1;   // rotate-back operands of a pass ready (even CTA's barrier; both epilogues)
+    uint64_t* full = bars;
+    uint64_t* empty = bars + kNS;
+    uint64_t* tfull = bars + 2 * kNS;
+    uint64_t* tempty = tfull + 2;
+    uint64_t* xready = tempty + 2;
+    uint64_t* xfree = xready + 2;
+    uint64_t* dbar = xfree + 2;   // epilogue Wigner staging, per buffer
+    uint64_t* fin = dbar + 2;
+    uint64_t* gfull = fin + 1;    // value gate of a tile buffer written (gate warps -> producer)
+    uint64_t* gempty = gfull + 2; // value gate of a tile buffer consumed (producer -> gate warps)
+    uint64_t* jfull = gempty + 2; // fused traversal: (i, j) of a tile buffer listed (gate warps -> producer)
     uint32_t* tmem_sm = reinterpret_cast<uint32_t*>(smem + S.misc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + S.misc + 8);
     int* last_slot = reinterpret_cast<int*>(smem + S.misc + 16);  // producer: node slot of the last edge
-    int* gij = reinterpret_cast<int*>(smem + S.misc + 64);        // gate warps: [2][2][64] (i, j) per edge
+    int* gij = reinterpret_cast<int*>(smem + S.misc + 64);        // gate warps: [2][128] (i, j) per edge
     long long* dsub = reinterpret_cast<long long*>(smem + S.dsub);  // sub-step cycle sums (timers on)
     float* wga = reinterpret_cast<float*>(smem + S.wga);            // [16][H] logit-gate weights
     const bool dbgon = P.dbg != nullptr;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const uint32_t rank = cluster_rank();      // 0: issues the pair's MMAs
-    const uint32_t peer = rank ^ 1u;
-    const int pair = blockIdx.x >> 1;
-    // cluster addresses of barriers in the peer / even CTA
-    auto at_peer = [=](const void* local) { return mapa(smem_u32(local), peer); };
-    auto at_even = [=](const void* local) { return mapa(smem_u32(local), 0u); };
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kNS; ++s) { mbar_init(full + s, 1); mbar_init(empty + s, 2); }
+        for (int s = 0; s < kNS; ++s) { mbar_init(full + s, 1); mbar_init(empty + s, 1); }
         for (int b = 0; b < 2; ++b) {
-            mbar_init(tfull + b, 2);
-            mbar_init(tempty + b, 2 * kEpiThreads);
-            mbar_init(xready + b, 2 * 128);
-            mbar_init(xfree + b, 2 * kEpiThreads);
+            mbar_init(tfull + b, 1);
+            mbar_init(tempty + b, kEpiThreads);
+            mbar_init(xready + b, 128);
+            mbar_init(xfree + b, kEpiThreads);
             mbar_init(dbar + b, 1);
         }
         mbar_init(fin, 1);
-        mbar_init(fin + 1, 1);
-        mbar_init(d2full, 1);
-        mbar_init(a2ready, 2 * kEpiThreads);
         for (int b = 0; b < 2; ++b) {
             mbar_init(gfull + b, 64);
             mbar_init(gempty + b, 128);
@@ -774,19 +668,19 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == 12) {
-        tmem_alloc2(tmem_sm, 512);
-        tmem_relinquish2();
+        tmem_alloc(tmem_sm, 512);
+        tmem_relinquish();
     }
     tc_fence_before();
-    cluster_sync();  // barriers initialised and TMEM allocated in both CTAs
+    __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_sm;
 
-    const int n_begin = P.part[pair], n_end = P.part[pair + 1];
+
+    const int n_begin = P.part[blockIdx.x], n_end = P.part[blockIdx.x + 1];
     const int e_begin = P.row_ptr[n_begin], e_end = P.row_ptr[n_end];
     const int ntiles = (e_end - e_begin + kTileE - 1) / kTileE;
     const int ng = P.n_groups;
-    const int eoff = (int)rank * kHalfE;  // this CTA's edges within a pair tile
 
     if (warp >= 4 && warp < 8) {
         // ---------------- producer ----------------
@@ -795,6 +689,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
         const float inv_s = P.scale[1];
         const int CG = C / 8;
         const int Gv = (L + 1) * C;
+        const int C8 = C / 8;
         for (int t2 = p; t2 < kTcMaxRbf * H; t2 += 128) {
             const int kb = t2 / H, h = t2 % H;
             wga[t2] = kb < NR ? P.Wrad[(size_t)kb * G + Gv + h] : 0.f;
@@ -817,25 +712,23 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
         const long long c_start = clock64();
         for (int t = 0; t < ntiles; ++t) {
             const int b = t & 1;
-            // both epilogues are done with this buffer (this producer also writes the peer's copy)
-            const bool okw = (t < 2) || wait_cluster(xfree + b, ((t - 2) >> 1) & 1, abort_flag, P.status, w_free);
+            const bool okw = (t < 2) || wait_t(xfree + b, ((t - 2) >> 1) & 1, abort_flag, P.status, w_free);
             if (!bar_and(1, 128, okw)) break;
             const long long c_a = clock64();
-            const int e0 = e_begin + t * kTileE + eoff;       // this CTA's first edge
-            const int ne = max(0, min(kHalfE, e_end - e0));   // and count
-            // window of row_ptr after the node of this CTA's first edge
+            const int e0 = e_begin + t * kTileE;
+            const int ne = min(kTileE, e_end - e0);
+            // window of row_ptr after the node of the tile's first edge
             {
                 int nb0;
                 if (t == 0) {
-                    const int ef = min(e0, max(e_begin, e_end - 1));
                     int lo = n_begin, hi = n_end - 1;
                     while (lo < hi) {
                         int mid = (lo + hi + 1) >> 1;
-                        if (P.row_ptr[mid] <= ef) lo = mid; else hi = mid - 1;
+                        if (P.row_ptr[mid] <= e0) lo = mid; else hi = mid - 1;
                     }
                     nb0 = lo;
                 } else {
-                    nb0 = *last_slot;  // node slot of this CTA's last edge of the previous tile
+                    nb0 = *last_slot;  // node slot of edge e0 - 1
                 }
                 nbase = nb0;
                 const int n = nbase + 1 + p;
@@ -843,7 +736,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
             }
             asm volatile("bar.sync 1, 128;" ::: "memory");
             if (P.cells) {
-                // fused traversal: the gate warps list (atom, neighbour) of this CTA's edges in
+                // fused traversal: the gate warps list (atom, neighbour) of the tile's edges in
                 // gij[b]; they refill it only after gempty[b], i.e. after this tile's P2
                 const bool okj = wait_t(jfull + b, (t >> 1) & 1, abort_flag, P.status, w_free);
                 if (!bar_and(1, 128, okj)) break;
@@ -852,14 +745,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
             E2F_TICK(0);
             __half2* Dg = P.dscr + (size_t)(blockIdx.x * 2 + b) * dglob_pairs();
             // P1: one edge per thread: frame, Wigner pairs (fp16x2; shared copy for
-            // the rotation below, global copy for the epilogues of both CTAs)
-            if (p < kHalfE) {
+            // the rotation below, global copy for the epilogue), softmax weights
+            {
                 __half2* Dh = dph + (size_t)p * DPS;
-                const uint32_t nid_peer = at_peer(nid + b * kTileE + eoff + p);
                 if (p < ne) {
                     const int e = e0 + p;
-                    const int* gl = gij + b * 2 * kHalfE;  // fused traversal: [i x 64][j x 64]
-                    const int j = P.cells ? gl[kHalfE + p] : P.col[e];
+                    const int* gl = gij + b * 2 * kTileE;  // fused traversal: [i x 128][j x 128]
+                    const int j = P.cells ? gl[kTileE + p] : P.col[e];
                     // node slot: last n with row_ptr[n] <= e = nbase + #{k: rpw[k] <= e}
                     int i;
                     if (e < rpw[kTileE - 1]) {
@@ -877,7 +769,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
                         }
                         i = lo;
                     }
-                    if (p == ne - 1) *last_slot = i;
+                    if (p == kTileE - 1) *last_slot = i;
                     if (P.cells) i = gl[p];  // slot -> atom
                     float3 r = edge_vec(P.pos, i, j, P.box);
                     const float d = sqrtf(r.x * r.x + r.y * r.y + r.z * r.z);
@@ -894,7 +786,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
 #pragma unroll
                         for (int mu = 0; mu <= l; ++mu) {
                             uint4* sq = reinterpret_cast<uint4*>(Dh + dpo(l, mu));
-                            uint32_t* gq = reinterpret_cast<uint32_t*>(Dg + dglob_block(l, mu)) + p;
+                            uint4* gq = reinterpret_cast<uint4*>(Dg + dglob_block(l, mu) + (size_t)p * npair(l));
 #pragma unroll
                             for (int n4 = 0; n4 < npair(l); n4 += 4) {
                                 uint32_t wv[4];
@@ -904,9 +796,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
                                     const float a0 = n < w ? Dl[(l + mu) * w + n] : 0.f;
                                     const float b0 = n < w ? Dl[(l - mu) * w + n] : 0.f;
                                     wv[t4] = pack_h2(a0, b0);
-                                    gq[(size_t)n * kHalfE] = wv[t4];  // a warp writes 32 consecutive words
                                 }
-                                sq[n4 / 4] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+                                const uint4 u = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+                                sq[n4 / 4] = u;
+                                gq[n4 / 4] = u;
                             }
                         }
                     }
@@ -925,41 +818,36 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
                                      "r"((uint32_t)(KT * 2))
                                      : "memory");
                     E2F_TICK(4);
-                    nid[b * kTileE + eoff + p] = i;
-                    st_cluster_u32(nid_peer, (uint32_t)i);
-                    jn[b * kHalfE + p] = j;
+                    nid[b * kTileE + p] = i;
+                    jn[b * kTileE + p] = j;
                 } else {
                     const uint4 z = make_uint4(0, 0, 0, 0);
 #pragma unroll
                     for (int l = 0; l <= L; ++l)
 #pragma unroll
                         for (int mu = 0; mu <= l; ++mu) {
-                            uint32_t* gq = reinterpret_cast<uint32_t*>(Dg + dglob_block(l, mu)) + p;
-                            for (int n = 0; n < npair(l); ++n) gq[(size_t)n * kHalfE] = 0u;
+                            uint4* gq = reinterpret_cast<uint4*>(Dg + dglob_block(l, mu) + (size_t)p * npair(l));
+                            for (int n4 = 0; n4 < npair(l); n4 += 4) gq[n4 / 4] = z;
                         }
                     for (int a = 0; a < DPS; a += 4) *reinterpret_cast<uint4*>(Dh + a) = z;
-                    for (int h = 0; h < H; ++h) {
-                        php[(b * H + h) * kTileE + eoff + p] = 0.f;
-                        st_cluster_f32(at_peer(php + (b * H + h) * kTileE + eoff + p), 0.f);
-                    }
-                    nid[b * kTileE + eoff + p] = -1;
-                    st_cluster_u32(nid_peer, 0xffffffffu);
-                    jn[b * kHalfE + p] = 0;
+                    for (int k8 = 0; k8 < C8; ++k8) pch[(b * kTileE + p) * C8 + k8] = 0.f;
+                    nid[b * kTileE + p] = -1;
+                    jn[b * kTileE + p] = 0;
                 }
             }
             asm volatile("bar.sync 1, 128;" ::: "memory");
             E2F_TICK(6);
             // logits and softmax weights, one (edge, head) pair per thread and step: the
             // thread's head h = p % H is fixed (H divides 128), the H lanes of an edge read
-            // its key row as consecutive float4; written to both CTAs
+            // its key row as consecutive float4
             {
                 const int h = p % H, d4 = dh / 4;
                 float wh[kTcMaxRbf];
 #pragma unroll
                 for (int kb = 0; kb < kTcMaxRbf; ++kb) wh[kb] = wga[kb * H + h];
 #pragma unroll 2
-                for (int e = p / H; e < ne; e += 128 / H) {
-                    const int i = nid[b * kTileE + eoff + e], j = jn[b * kHalfE + e];
+                for (int e = p / H; e < ne; e += kTileE / H) {
+                    const int i = nid[b * kTileE + e], j = jn[b * kTileE + e];
                     const float4* rq = reinterpret_cast<const float4*>(rrs + e * kTcMaxRbf);
                     float ga = 0.f;
 #pragma unroll
@@ -982,11 +870,18 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
                     }
                     const float a = ga * dot * inv_sqrt_dh;
                     const float pw = expf(a - P.lse[(size_t)i * H + h]) * inv_s;
-                    php[(b * H + h) * kTileE + eoff + e] = pw;
-                    st_cluster_f32(at_peer(php + (b * H + h) * kTileE + eoff + e), pw);
+                    for (int k8 = h * (dh / 8); k8 < (h + 1) * (dh / 8); ++k8) pch[(b * kTileE + e) * C8 + k8] = pw;
                 }
             }
             E2F_TICK(5);
+            if (p < kTileE / kChunk) {  // segment starts per 16-edge chunk
+                uint32_t m = 0;
+                for (int q = 0; q < kChunk; ++q) {
+                    const int e = p * kChunk + q;
+                    if (e == 0 || nid[b * kTileE + e] != nid[b * kTileE + e - 1]) m |= 1u << q;
+                }
+                segm[b * (kTileE / kChunk) + p] = m;
+            }
             asm volatile("bar.sync 1, 128;" ::: "memory");
             E2F_TICK(7);
             const long long c_b = clock64();
@@ -996,9 +891,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
                 const bool okg = wait_t(gfull + b, (t >> 1) & 1, abort_flag, P.status, w_free);
                 if (!bar_and(1, 128, okg)) break;
             }
-            const __half* gs = P.gscr + ((size_t)blockIdx.x * 2 + b) * kHalfE * Gv;
-            __half* xrow0 = P.xs + ((size_t)(blockIdx.x * 2 + b) * kHalfE) * KT;
-            for (int it = p; it < kHalfE * CG; it += 128) {
+            const __half* gs = P.gscr + ((size_t)blockIdx.x * 2 + b) * kTileE * Gv;
+            __half* xrow0 = P.xs + ((size_t)(blockIdx.x * 2 + b) * kTileE) * KT;
+            for (int it = p; it < kTileE * CG; it += 128) {
                 const int e = it / CG, c0 = (it % CG) * 8;
                 __half* xrow = xrow0 + (size_t)e * KT;
                 if (e >= ne) {
@@ -1010,10 +905,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
                             *reinterpret_cast<uint4*>(xrow + kpos(l1, m, L, C) + c0) = z;
                     continue;
                 }
-                const int j = jn[b * kHalfE + e];
-                if (c0 == 0 && e + 8 < ne)  // neighbour row of the edge one round ahead
+                const int j = jn[b * kTileE + e];
+                if (c0 == 0 && e + 16 < ne)  // neighbour row of the edge two rounds ahead
                     asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(
-                                     P.x + (size_t)jn[b * kHalfE + e + 8] * KT),
+                                     P.x + (size_t)jn[b * kTileE + e + 16] * KT),
                                  "r"((uint32_t)(KT * 2))
                                  : "memory");
                 const __half2* De = dph + (size_t)e * DPS;
@@ -1066,11 +961,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
                 }
             }
             mbar_arrive(gempty + b);  // this tile's value gates have been read
-            // generic-proxy stores (features, Wigner pairs) -> visible to TMA / bulk copies; the
-            // shared-memory stores into the peer (nid, php) are released by the cluster arrive
+            // generic-proxy stores (features, Wigner pairs) -> visible to TMA / bulk copies
             asm volatile("fence.proxy.async.global;" ::: "memory");
             mbar_arrive(xready + b);
-            mbar_arrive_cluster(at_peer(xready + b));
             c_p2 += clock64() - c_b;
         }
         if (P.dbg && p == 0) {
@@ -1080,10 +973,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
         }
 #undef E2F_TICK
     } else if (warp == 12) {
-        // ---------------- TMA (both CTAs) ----------------
-        // Each CTA loads its 128 weight rows and its 64 edges of the feature tile into
-        // its own ring; every load's completion is counted on the even CTA's `full`
-        // barrier, where the even CTA expects the bytes of both.
+        // ---------------- TMA ----------------
         if (lane == 0) {
             const uint64_t pol_xs = policy_evict_last();
             int stage = 0;
@@ -1093,33 +983,26 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
             for (int s2 = 0; s2 < kNS; ++s2) pending[s2] = -1;
             long long w_x = 0, w_e = 0;
             const long long c_start = clock64();
-            (void)pol_xs;
             for (int t = 0; t < ntiles && ok; ++t) {
                 const int b = t & 1;
-                if (!wait_cluster(xready + b, (t >> 1) & 1, abort_flag, P.status, w_x)) { ok = false; break; }
-                const int rowT = (blockIdx.x * 2 + b) * kHalfE;
+                if (!wait_t(xready + b, (t >> 1) & 1, abort_flag, P.status, w_x)) { ok = false; break; }
+                const int rowT = (blockIdx.x * 2 + b) * kTileE;
                 for (int gi = 0; gi < ng && ok; ++gi) {
                     const TcGroup g = P.groups[gi];
-                    const int wr0 = g.row0 + 128 * (int)rank, wr0b = g.row0b + 128 * (int)rank;
-                    const int ntw = g.mu > 0 ? 2 : (g.row0b >= 0 ? 2 : 1);
-                    const int ntx = g.mu > 0 ? 2 : 1;
-                    const uint32_t bytes_cta = (uint32_t)(ntw * kWSlot + ntx * kXSlot);
                     for (int kk = 0; kk < g.klen; kk += kKS) {
                         if (!wait_t(empty + stage, ph ^ 1, abort_flag, P.status, w_e)) { ok = false; break; }
                         uint8_t* st = ring + (size_t)stage * kStage;
-                        const uint32_t fb = at_even(full + stage);
-                        // local barrier, local waiters: a CTA-scope arrive (a cluster-scope release
-                        // here would wait for this thread's loads in flight)
-                        if (rank == 0) mbar_arrive_tx(full + stage, 2 * bytes_cta);
+                        const int ntile = g.mu > 0 ? 4 : (g.row0b >= 0 ? 3 : 2);
+                        mbar_arrive_tx(full + stage, ntile * kSlot);
                         if (g.mu > 0) {
-                            tma_load_2d_pair(st, &T.w[g.wa], kk, wr0, fb);
-                            tma_load_2d_pair(st + kWSlot, &T.w[g.wb], kk, wr0, fb);
-                            tma_load_2d_pair(st + 2 * kWSlot, &T.xs, g.xoff0 + kk, rowT, fb);
-                            tma_load_2d_pair(st + 2 * kWSlot + kXSlot, &T.xs, g.xoff1 + kk, rowT, fb);
+                            tma_load_2d(st, &T.w[g.wa], kk, g.row0, full + stage);
+                            tma_load_2d(st + kSlot, &T.w[g.wb], kk, g.row0, full + stage);
+                            tma_load_2d_hint(st + 2 * kSlot, &T.xs, g.xoff0 + kk, rowT, full + stage, pol_xs);
+                            tma_load_2d_hint(st + 3 * kSlot, &T.xs, g.xoff1 + kk, rowT, full + stage, pol_xs);
                         } else {
-                            tma_load_2d_pair(st, &T.w[g.wa], kk, wr0, fb);
-                            if (g.row0b >= 0) tma_load_2d_pair(st + kWSlot, &T.w[g.wa], kk, wr0b, fb);
-                            tma_load_2d_pair(st + 2 * kWSlot, &T.xs, g.xoff0 + kk, rowT, fb);
+                            tma_load_2d(st, &T.w[g.wa], kk, g.row0, full + stage);
+                            if (g.row0b >= 0) tma_load_2d(st + kSlot, &T.w[g.wa], kk, g.row0b, full + stage);
+                            tma_load_2d_hint(st + 2 * kSlot, &T.xs, g.xoff0 + kk, rowT, full + stage, pol_xs);
                         }
                         pending[stage] = (int)ph;
                         if (++stage == kNS) { stage = 0; ph ^= 1; }
@@ -1130,26 +1013,17 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
                 long long* d = P.dbg + blockIdx.x * kDbgSlots;
                 d[2] = w_x; d[3] = w_e; d[4] = clock64() - c_start;
             }
-            // the loads this CTA issued complete before it can leave: the last use of each
-            // stage is released (consumed) by the MMAs only after its data landed
+            // every issued load lands (bounded wait) before the CTA can leave
             for (int s2 = 0; s2 < kNS; ++s2) {
                 if (pending[s2] < 0) continue;
                 const uint64_t t0 = gtimer();
-                while (!mbar_try(empty + s2, (uint32_t)pending[s2]) && gtimer() - t0 < kWaitNs) {
+                while (!mbar_try(full + s2, (uint32_t)pending[s2]) && gtimer() - t0 < kWaitNs) {
                 }
             }
         }
         __syncwarp();
-    } else if (rank == 0 && (warp == 13 || warp == 8)) {
-        // ---------------- MMA (even CTA; two issuing warps) ----------------
-        // One M256 x N128 x K16 instruction covers both CTAs: rows 0-127 of the group's
-        // weights and its accumulator lanes in the even CTA, rows 128-255 in the odd
-        // one; the 128 edge columns come 64 from each CTA's feature tile. The issuing
-        // thread runs in step with the tensor pipe, so two warps issue: A (warp 13) the
-        // first accumulator of each group (o+, or the first m = 0 block), B (warp 8) the
-        // second (o-, or the second block). Warp A also issues the rotate-back MMAs of
-        // the previous group halfway through each group, in its own stream.
-        const bool wa = warp == 13;
+    } else if (warp == 13) {
+        // ---------------- MMA ----------------
         if (lane == 0) {
             int stage = 0;
             uint32_t ph = 0;
@@ -1157,136 +1031,57 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
             bool ok = true;
             long long w_t = 0, w_f = 0;
             const long long c_start = clock64();
-            constexpr uint32_t ID = idesc_pair(128, false), IDN = idesc_pair(128, true), ID2 = idesc_pair(32, false);
-            // Operand descriptors of the ring stages, built once: the issue loop only
-            // adds constant offsets (the start address field counts 16-byte units,
-            // and every stage lies below 256 KB, so the additions never carry).
-            const uint64_t dbase0 = sdesc_sw64(smem_u32(ring));
-            constexpr uint64_t kWs = kWSlot >> 4, kXs = kXSlot >> 4, kKs = 32 >> 4, kSt = kStage >> 4;
-            const uint64_t b2base = sdesc_b2(smem_u32(b2s));
-            long long m_issue = 0, m_commit = 0, m_serv = 0;
-            uint32_t a2ph = 0;
-            // A rotate-back pass (its arrival on a2ready observed): the epilogues' request
-            // list, identical in both CTAs, read from this one; passes arrive in order and
-            // are issued in that order. Written as a macro, not a lambda, so that the loop
-            // counters stay in registers.
-#define E2F_ISSUE_PASS()                                                                                     \
-    do {                                                                                                    \
-        a2ph ^= 1;                                                                                          \
-        tc_fence_after();                                                                                   \
-        const int q_ = *mailbox;                                                                            \
-        const int n_ = reqh(q_)[0];                                                                         \
-        const uint32_t cbt_ = tmem + (uint32_t)reqh(q_)[1] * 256u;                                          \
-        const uint32_t* rl_ = reinterpret_cast<const uint32_t* const*>(reqh(q_) + 2)[0];                    \
-        const uint64_t bq_ = b2base + (uint64_t)q_ * (kB2Blocks * kB2Bytes >> 4);                           \
-        for (int k_ = 0; k_ < n_; ++k_) {                                                                   \
-            const uint32_t rq_ = rl_[k_];                                                                   \
-            umma2_ts(cbt_ + (rq_ & 255u), cbt_ + ((rq_ >> 8) & 255u),                                       \
-                     bq_ + (uint64_t)((rq_ >> 16) & 255u) * (kB2Bytes >> 4), ID2, (int)(rq_ >> 24));        \
-        }                                                                                                   \
-        umma2_commit_both(d2full);                                                                          \
-    } while (0)
-            // bounded wait that serves rotate-back passes arriving meanwhile; sets `ok`
-#define E2F_WAIT_S(bar_, par_, acc_)                                                                         \
-    do {                                                                                                    \
-        if (!mbar_try((bar_), (par_))) {                                                                    \
-            const long long c0_ = clock64();                                                                \
-            const uint64_t t0_ = gtimer();                                                                  \
-            while (!mbar_try((bar_), (par_))) {                                                             \
-                if (wa && mbar_test(a2ready, a2ph)) E2F_ISSUE_PASS();                                        \
-                if (*abort_flag) { ok = false; break; }                                                     \
-                if (gtimer() - t0_ > kWaitNs) {                                                             \
-                    *abort_flag = 1;                                                                        \
-                    atomicExch(P.status, (int)E2F_ERR_TIMEOUT);                                             \
-                    ok = false;                                                                             \
-                    break;                                                                                  \
-                }                                                                                           \
-            }                                                                                               \
-            (acc_) += clock64() - c0_;                                                                      \
-        }                                                                                                   \
-    } while (0)
+            constexpr uint32_t ID = idesc_f16(false), IDN = idesc_f16(true);
             for (int t = 0; t < ntiles && ok; ++t) {
                 for (int gi = 0; gi < ng && ok; ++gi, ++gcount) {
                     const TcGroup g = P.groups[gi];
                     const int slot = (int)(gcount & 1);
                     const uint32_t use = (uint32_t)(gcount >> 1);
-                    E2F_WAIT_S(tempty + slot, (use & 1) ^ 1, w_t);
-                    if (!ok) break;
+                    if (!wait_t(tempty + slot, (use & 1) ^ 1, abort_flag, P.status, w_t)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t d0 = tmem + slot * 256, d1 = d0 + 128;
-                    const int kind = g.mu > 0 ? 2 : (g.row0b >= 0 ? 1 : 0);
                     for (int kk = 0; kk < g.klen; kk += kKS) {
-                        E2F_WAIT_S(full + stage, ph, w_f);
-                        if (!ok) break;
+                        if (!wait_t(full + stage, ph, abort_flag, P.status, w_f)) { ok = false; break; }
                         tc_fence_after();
-                        const long long c_i0 = dbgon ? clock64() : 0;
-                        // stage: weights A (0), B (kWs) / second block; features x+ (2 kWs), x- (+kXs)
-                        const uint64_t a0 = dbase0 + (uint64_t)stage * kSt, a1 = a0 + kWs, x0 = a0 + 2 * kWs,
-                                       x1 = x0 + kXs;
-                        if (kind == 2) {
-                            if (wa) {  // o+ = A h+ - B h-
-                                if (kk == 0) umma2_ss(d0, a0, x0, ID, 0); else umma2_ss(d0, a0, x0, ID, 1);
-                                umma2_ss(d0, a1, x1, IDN, 1);
-                                umma2_ss(d0, a0 + kKs, x0 + kKs, ID, 1);
-                                umma2_ss(d0, a1 + kKs, x1 + kKs, IDN, 1);
-                            } else {   // o- = B h+ + A h-
-                                if (kk == 0) umma2_ss(d1, a1, x0, ID, 0); else umma2_ss(d1, a1, x0, ID, 1);
-                                umma2_ss(d1, a0, x1, ID, 1);
-                                umma2_ss(d1, a1 + kKs, x0 + kKs, ID, 1);
-                                umma2_ss(d1, a0 + kKs, x1 + kKs, ID, 1);
+                        const uint32_t sa = smem_u32(ring + (size_t)stage * kStage);
+#pragma unroll
+                        for (int ks = 0; ks < 2; ++ks) {
+                            const uint64_t a0 = sdesc_sw64(sa + ks * 32);
+                            const uint64_t a1 = sdesc_sw64(sa + kSlot + ks * 32);
+                            const uint64_t x0 = sdesc_sw64(sa + 2 * kSlot + ks * 32);
+                            const uint64_t x1 = sdesc_sw64(sa + 3 * kSlot + ks * 32);
+                            const uint32_t acc = (kk > 0 || ks > 0) ? 1u : 0u;
+                            if (g.mu > 0) {
+                                umma(d0, a0, x0, ID, acc);    // o+ += A h+
+                                umma(d1, a1, x0, ID, acc);    // o- += B h+
+                                umma(d0, a1, x1, IDN, 1u);    // o+ -= B h-
+                                umma(d1, a0, x1, ID, 1u);     // o- += A h-
+                            } else {
+                                umma(d0, a0, x0, ID, acc);
+                                if (g.row0b >= 0) umma(d1, a1, x0, ID, acc);
                             }
-                        } else if (wa) {
-                            if (kk == 0) umma2_ss(d0, a0, x0, ID, 0); else umma2_ss(d0, a0, x0, ID, 1);
-                            umma2_ss(d0, a0 + kKs, x0 + kKs, ID, 1);
-                        } else if (kind == 1) {
-                            if (kk == 0) umma2_ss(d1, a1, x0, ID, 0); else umma2_ss(d1, a1, x0, ID, 1);
-                            umma2_ss(d1, a1 + kKs, x0 + kKs, ID, 1);
                         }
-                        const long long c_i1 = dbgon ? clock64() : 0;
-                        umma2_commit_both(empty + stage);
+                        umma_commit(empty + stage);
                         if (++stage == kNS) { stage = 0; ph ^= 1; }
-                        if (dbgon) {
-                            const long long c_i2 = clock64();
-                            m_issue += c_i1 - c_i0; m_commit += c_i2 - c_i1;
-                        }
-                        // a rotate-back pass of the previous group, if its operands are ready
-                        // (while this warp polls, the other warp's MMAs keep the pipe busy)
-                        if (wa && mbar_test(a2ready, a2ph)) {
-                            const long long c_s0 = dbgon ? clock64() : 0;
-                            E2F_ISSUE_PASS();
-                            if (dbgon) m_serv += clock64() - c_s0;
-                        }
                     }
-                    if (ok) umma2_commit_both(tfull + slot);
+                    if (ok) umma_commit(tfull + slot);
                 }
             }
-            // further passes of the last groups: serve them until both slots are released
-            if (wa) {
-                for (int s2 = 0; s2 < 2 && ok; ++s2) {
-                    const long long nuse = (gcount + 1 - s2) / 2;  // uses of slot s2
-                    if (nuse > 0) E2F_WAIT_S(tempty + s2, (uint32_t)((nuse & 1) ^ 1), w_t);
-                }
-            }
-#undef E2F_WAIT_S
-#undef E2F_ISSUE_PASS
-            if (P.dbg && wa) {
+            if (P.dbg) {
                 long long* d = P.dbg + blockIdx.x * kDbgSlots;
                 d[5] = w_t; d[6] = w_f; d[7] = clock64() - c_start;
-                d[25] = m_issue; d[26] = m_commit; d[27] = m_serv;
             }
             // every issued MMA completes (bounded wait) before TMEM is released
-            uint64_t* fb = fin + (wa ? 0 : 1);
-            umma2_commit_both(fb);
+            umma_commit(fin);
             const uint64_t t0 = gtimer();
-            while (!mbar_try(fb, 0) && gtimer() - t0 < kWaitNs) {
+            while (!mbar_try(fin, 0) && gtimer() - t0 < kWaitNs) {
             }
         }
         __syncwarp();
     } else if (warp >= 14) {
         // ---------------- value gate (warps 14-15), up to two tiles ahead ----------------
-        // g[e][n] = rho(d_e) . W_rad[:, n] for this CTA's 64 edges of a tile and
-        // n < (L+1)C, into a per-CTA global buffer per tile parity that the
-        // producer's rotation reads.
+        // g[e][n] = rho(d_e) . W_rad[:, n] for the tile's 128 edges and n < (L+1)C, into a
+        // per-CTA global buffer per tile parity that the producer's rotation reads.
         const int gp = threadIdx.x - 448, gw = warp - 14, g8 = lane >> 2, t4 = lane & 3;
         const int Gv = (L + 1) * C;
         long long w_g = 0;
@@ -1295,9 +1090,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
             const int b = t & 1;
             const bool okw = (t < 2) || wait_t(gempty + b, ((t - 2) >> 1) & 1, abort_flag, P.status, w_g);
             if (!bar_and(3, 64, okw)) break;
-            const int e0 = e_begin + t * kTileE + eoff;
-            const int ne = max(0, min(kHalfE, e_end - e0));
-            int* gi = gij + b * 2 * kHalfE;
+            const int e0 = e_begin + t * kTileE;
+            const int ne = min(kTileE, e_end - e0);
+            int* gi = gij + b * 2 * kTileE;
             if (P.cells) {  // fused traversal: (atom, neighbour) of each edge from the cell lists
                 auto slot_of = [&](int e) {
                     int lo = n_begin, hi = n_end - 1;
@@ -1307,34 +1102,31 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
                     }
                     return lo;
                 };
-                if (ne > 0) {
-                    const int s_first = slot_of(e0), s_last = slot_of(e0 + ne - 1);
-                    for (int sl = s_first + (warp - 14); sl <= s_last; sl += 2) {
-                        const int base = P.row_ptr[sl], ia = P.cv.sidx[sl];
-                        warp_neighbors(
-                            P.cv, P.cv.spos[sl], ia,
-                            [&](int k, int j) {
-                                const int e = base + k;
-                                if (e >= e0 && e < e0 + ne) {
-                                    gi[e - e0] = ia;
-                                    gi[kHalfE + e - e0] = j;
-                                }
-                            },
-                            0, sl);
-                    }
+                const int s_first = slot_of(e0), s_last = slot_of(e0 + ne - 1);
+                for (int sl = s_first + (warp - 14); sl <= s_last; sl += 2) {
+                    const int base = P.row_ptr[sl], ia = P.cv.sidx[sl];
+                    warp_neighbors(
+                        P.cv, P.cv.spos[sl], ia,
+                        [&](int k, int j) {
+                            const int e = base + k;
+                            if (e >= e0 && e < e0 + ne) {
+                                gi[e - e0] = ia;
+                                gi[kTileE + e - e0] = j;
+                            }
+                        },
+                        0, sl);
                 }
                 asm volatile("bar.sync 3, 64;" ::: "memory");
                 mbar_arrive(jfull + b);  // releases the lists to the producer (CTA scope)
             }
-            {  // radial basis of this CTA's edges, one per thread
-                const int k = gp;
+            for (int k = gp; k < kTileE; k += 64) {  // radial basis of the tile's edges
                 float rr[kTcMaxRbf];
                 if (k < ne) {
                     const int e = e0 + k;
                     int lo, j;
                     if (P.cells) {
                         lo = gi[k];
-                        j = gi[kHalfE + k];
+                        j = gi[kTileE + k];
                     } else {
                         j = P.col[e];
                         lo = n_begin;
@@ -1359,12 +1151,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
                 rq[1] = make_uint4(hw[4], hw[5], hw[6], hw[7]);
             }
             asm volatile("bar.sync 3, 64;" ::: "memory");
-            // one k = 16 mma.sync per 16 edges x 8 columns; warp gw takes edge blocks 2 gw, 2 gw + 1
-            __half* gs = P.gscr + ((size_t)blockIdx.x * 2 + b) * kHalfE * Gv;
-            uint32_t af[2][4];
+            // one k = 16 mma.sync per 16 edges x 8 columns; warp gw takes edge blocks 4 gw .. 4 gw + 3
+            __half* gs = P.gscr + ((size_t)blockIdx.x * 2 + b) * kTileE * Gv;
+            uint32_t af[4][4];
 #pragma unroll
-            for (int mb = 0; mb < 2; ++mb) {
-                const __half* rr0 = rho + ((2 * gw + mb) * 16 + g8) * kTcMaxRbf + 2 * t4;
+            for (int mb = 0; mb < 4; ++mb) {
+                const __half* rr0 = rho + ((4 * gw + mb) * 16 + g8) * kTcMaxRbf + 2 * t4;
                 af[mb][0] = *reinterpret_cast<const uint32_t*>(rr0);
                 af[mb][1] = *reinterpret_cast<const uint32_t*>(rr0 + 8 * kTcMaxRbf);
                 af[mb][2] = *reinterpret_cast<const uint32_t*>(rr0 + 8);
@@ -1377,10 +1169,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
                 bf[0] = __ldg(reinterpret_cast<const unsigned int*>(wb));
                 bf[1] = __ldg(reinterpret_cast<const unsigned int*>(wb + 8));
 #pragma unroll
-                for (int mb = 0; mb < 2; ++mb) {
+                for (int mb = 0; mb < 4; ++mb) {
                     float acc4[4] = {0.f, 0.f, 0.f, 0.f};
                     mma_16816(acc4, af[mb], bf);
-                    const int e = (2 * gw + mb) * 16 + g8;
+                    const int e = (4 * gw + mb) * 16 + g8;
                     *reinterpret_cast<__half2*>(gs + (size_t)e * Gv + n0 + 2 * t4) = __floats2half2_rn(acc4[0], acc4[1]);
                     *reinterpret_cast<__half2*>(gs + (size_t)(e + 8) * Gv + n0 + 2 * t4) =
                         __floats2half2_rn(acc4[2], acc4[3]);
@@ -1392,255 +1184,72 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
             long long* d = P.dbg + blockIdx.x * kDbgSlots;
             d[23] = w_g; d[24] = clock64() - c_start;
         }
-    } else if (warp < 4) {
-        // ---------------- epilogue (warps 0-3, both CTAs) ----------------
-        // Per group, the rotate-back v = D(R)^T o weighted by the softmax and summed
-        // over each node's edges runs on the tensor cores:
-        //   1. conversion: each thread owns one TMEM lane (one output row (l3, c) of
-        //      this CTA's half of the group) and converts its 128 edge columns to
-        //      fp16 p_e o[c, e] in place (packed into the accumulator's first 64 columns);
-        //   2. per pass over up to 4 node segments of the tile (2 for a two-block m = 0
-        //      group), each CTA builds 16-row operand blocks B2[m'][e] = D_e^{l3}[+-mu][m']
-        //      (zero outside the node's edges) for its own degree l3, and the even CTA's
-        //      MMA warp A issues M256 N32 K16 pair MMAs D2[c][n] += sum_e A2[c][e] B2[n][e]
-        //      (A2 = the converted operand in TMEM); for a lane of CTA r the columns
-        //      16r..16r+15 of a node's 32 are its own degree's rotate-back;
-        //   3. drain: out[node][l3, m'][c] += D2[c][16r + m'] (m' < 2 l3 + 1), each output
-        //      element added by one thread (lane c of the CTA holding row (l3, c)) in
-        //      program order, so the order of additions is fixed.
+    } else if (warp < 12) {
+        // ---------------- epilogue (warps 0-3 and 8-11) ----------------
         // Every decision to stop goes through bar_and, so the 128 threads leave
         // together and no thread is left at a named barrier.
         const int r = threadIdx.x;
-        const int row = r;                               // this thread's TMEM lane
-        const int et = r;
-        const int ew = warp;                             // epilogue warp 0..3
-        const uint32_t tlane = tmem + ((uint32_t)(32 * warp) << 16);
         long long gcount = 0;
         bool ok = true;
         long long w_x = 0, w_t = 0;
         long long staged[2] = {-1, -1};  // last group index staged into each buffer (thread 0)
-        uint32_t d2ph = 0;
         const long long c_start = clock64();
-        EpiShared E;
-        E.sl_start = sl_start;
-        E.req0 = req0;
-        E.b2s = b2s;
-        E.dstage = dstage;
-        E.dstride = S.dstride;
-        const __half2* dg_even = P.dscr + (size_t)((blockIdx.x & ~1) * 2) * dglob_pairs();
-        const __half2* dg_odd = P.dscr + (size_t)((blockIdx.x | 1) * 2) * dglob_pairs();
-        // stages the Wigner slices of a group's accumulators in this CTA (one thread)
-#define E2F_STAGE_GROUP(gg_, b_, dst_, bar_)                                                                 \
-    do {                                                                                                    \
-        const TcGroup gq_ = (gg_);                                                                          \
-        const __half2* Dg0_ = dg_even + (size_t)(b_) * dglob_pairs();                                       \
-        const __half2* Dg1_ = dg_odd + (size_t)(b_) * dglob_pairs();                                        \
-        int l3a_, ca_, l3b_, cb_;                                                                           \
-        bool va_, vb_;                                                                                      \
-        epi_rows(gq_, 0, (int)rank, 0, L, C, l3a_, ca_, va_);                                               \
-        epi_rows(gq_, 1, (int)rank, 0, L, C, l3b_, cb_, vb_);                                               \
-        const bool tb_ = gq_.mu == 0 && gq_.row0b >= 0;                                                     \
-        const uint32_t ba_ = (uint32_t)kTileE * npair(l3a_) * 4;                                            \
-        const uint32_t bb_ = tb_ ? (uint32_t)kTileE * npair(l3b_) * 4 : 0u;                                 \
-        mbar_arrive_tx((bar_), ba_ + bb_);                                                                  \
-        stage_block(l3a_, gq_.mu, Dg0_, Dg1_, (dst_), (bar_));                                              \
-        if (tb_) stage_block(l3b_, 0, Dg0_, Dg1_, (dst_) + ba_, (bar_));                                    \
-    } while (0)
         for (int t = 0; t < ntiles; ++t) {
             const int b = t & 1;
-            const bool okx = wait_cluster(xready + b, (t >> 1) & 1, abort_flag, P.status, w_x);
+            const bool okx = wait_t(xready + b, (t >> 1) & 1, abort_flag, P.status, w_x);
             if (!bar_and(2, kEpiThreads, ok && okx)) { ok = false; break; }
+            const __half2* Dg = P.dscr + (size_t)(blockIdx.x * 2 + b) * dglob_pairs();
+            const float* pb = pch + (size_t)b * kTileE * (C / 8);
             const int* nb = nid + b * kTileE;
+            const uint32_t* sg = segm + b * (kTileE / kChunk);
             if (r == 0) {
-                E2F_STAGE_GROUP(P.groups[0], b, dstage + (gcount & 1) * S.dstride, dbar + (gcount & 1));
+                stage_group_pairs(P.groups[0], C, Dg, dstage + (gcount & 1) * S.dstride, dbar + (gcount & 1));
                 staged[gcount & 1] = gcount;
             }
-            // node segments of the tile (its edges are the prefix with nid >= 0)
-            if (ew == 0) {
-                int f[4], c = 0;
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const int e = 4 * lane + k;
-                    f[k] = nb[e] >= 0 && (e == 0 || nb[e] != nb[e - 1]);
-                    c += f[k];
-                }
-                int incl = c;
-#pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    const int v = __shfl_up_sync(0xffffffffu, incl, o);
-                    if (lane >= o) incl += v;
-                }
-                int pos = incl - c;
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const int e = 4 * lane + k;
-                    if (f[k]) { sl_start[pos] = e; sl_node[pos] = nb[e]; ++pos; }
-                }
-                // end of the last segment: the first padding edge (or 128)
-                int ne_l = 0;
-#pragma unroll
-                for (int k = 0; k < 4; ++k) ne_l += nb[4 * lane + k] >= 0;
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) ne_l += __shfl_xor_sync(0xffffffffu, ne_l, o);
-                const int ns = __shfl_sync(0xffffffffu, incl, 31);
-                if (lane == 0) { sl_count[0] = ns; sl_start[ns] = ne_l; }
-                __syncwarp();
-                if (lane < 3) {  // first-pass lists per group kind, one lane each
-                    const int per = lane == 1 ? 2 : 4;
-                    uint32_t* kl = klist + lane * 2 * kB2Blocks;
-                    klistn[lane] = epi_build_list(sl_start, lane, 0, min(ns, per), kl, kl + kB2Blocks);
-                }
-            }
-            bool prepped = false;  // the current group's first pass was prepared during the previous group
             for (int gi = 0; gi < ng; ++gi, ++gcount) {
                 // all threads are done with group gcount-1, so its staging buffer can be refilled
                 if (!bar_and(2, kEpiThreads, ok)) { ok = false; break; }
                 if (r == 0 && gi + 1 < ng) {
-                    E2F_STAGE_GROUP(P.groups[gi + 1], b, dstage + ((gcount + 1) & 1) * S.dstride, dbar + ((gcount + 1) & 1));
+                    stage_group_pairs(P.groups[gi + 1], C, Dg, dstage + ((gcount + 1) & 1) * S.dstride,
+                                      dbar + ((gcount + 1) & 1));
                     staged[(gcount + 1) & 1] = gcount + 1;
                 }
                 const TcGroup g = P.groups[gi];
                 const int slot = (int)(gcount & 1);
                 const uint32_t use = (uint32_t)(gcount >> 1);
-                const long long c_e0 = clock64();
-                const uint32_t cb = (uint32_t)slot * 256u;
-                const bool two = g.mu > 0 || g.row0b >= 0;
-                int l3A, cA, l3B, cB;
-                bool vA, vB;
-                epi_rows(g, 0, (int)rank, row, L, C, l3A, cA, vA);
-                epi_rows(g, 1, (int)rank, row, L, C, l3B, cB, vB);
-                if (g.mu > 0) { l3B = l3A; cB = cA; vB = vA; }
-                const int nseg = sl_count[0];
-                const bool twob = g.mu == 0 && g.row0b >= 0;
-                const int per = twob ? 2 : 4;  // segments per pass (result regions)
-                if (!prepped) {
-                    const bool okd = wait_t(dbar + slot, use & 1, abort_flag, P.status, w_t);
-                    if (!bar_and(2, kEpiThreads, okd)) {
-                        ok = false;
-                        break;
-                    }
-                    const int kd = g.mu > 0 ? 2 : (twob ? 1 : 0);
-                    const uint32_t* kl = klist + kd * 2 * kB2Blocks;
-                    epi_prep_pass(E, g, gcount, kl, kl + kB2Blocks, klistn[kd], (int)rank, L, C, et, ew, lane,
-                                  (dbgon && r == 0) ? dsub + 12 : nullptr);
-                }
-                const long long c_e1 = clock64();
-                const bool okt = wait_t(tfull + slot, use & 1, abort_flag, P.status, w_t);
-                if (!bar_and(2, kEpiThreads, okt)) {
-                    ok = false;
-                    break;
-                }
-                tc_fence_after();
-                const float* pA = php + ((size_t)b * H + cA / dh) * kTileE;
-                const float* pB = php + ((size_t)b * H + cB / dh) * kTileE;
-                // 1. conversion of this thread's 128 edge columns: o -> fp16 p o, packed in
-                // place; the next 16 columns load while these convert
-                {
-                    const uint32_t ta = tlane + cb, tb2 = tlane + cb + 128;
-                    float va[16], wa[16], vb[16], wb[16];
-                    tmem_ld16(ta, va);
-                    if (two) tmem_ld16(tb2, wa);
-#pragma unroll 1
-                    for (int j = 0; j < kTileE / 16; j += 2) {
-                        tmem_wait_ld();  // columns of chunk j in va / wa
-                        tmem_ld16(ta + 16 * (j + 1), vb);
-                        if (two) tmem_ld16(tb2 + 16 * (j + 1), wb);
-                        epi_convert16(ta, va, pA + 16 * j, j);
-                        if (two) epi_convert16(tb2, wa, pB + 16 * j, j);
-                        tmem_wait_ld();  // chunk j + 1 in vb / wb
-                        if (j + 2 < kTileE / 16) {
-                            tmem_ld16(ta + 16 * (j + 2), va);
-                            if (two) tmem_ld16(tb2 + 16 * (j + 2), wa);
-                        }
-                        epi_convert16(ta, vb, pA + 16 * (j + 1), j + 1);
-                        if (two) epi_convert16(tb2, wb, pB + 16 * (j + 1), j + 1);
-                    }
-                }
-                tmem_wait_st();
-                const long long c_e2 = clock64();
-                // 2./3. passes over the node segments
-                bool okp = true;
-                long long c_dr = 0;
-                prepped = false;
-                for (int s0 = 0; s0 < nseg; s0 += per) {
-                    const int s1 = min(nseg, s0 + per);
-                    if (s0 > 0) {  // later passes (many nodes in the tile): list built here
-                        const int kd = g.mu > 0 ? 2 : (twob ? 1 : 0);
-                        const int q = slot;
-                        if (et == 0) epi_reqh(E, q)[0] = epi_build_list(sl_start, kd, s0, s1, epi_req(E, q), epi_reqbp(E, q));
-                        asm volatile("bar.sync 2, %0;" ::"n"(kEpiThreads) : "memory");
-                        epi_prep_pass(E, g, gcount, epi_req(E, q), epi_reqbp(E, q), epi_reqh(E, q)[0], (int)rank, L, C, et,
-                                      ew, lane, (dbgon && r == 0) ? dsub + 12 : nullptr);
-                    }
-                    tc_fence_before();
-                    if (et == 0) *mailbox = slot;
-                    asm volatile("bar.sync 2, %0;" ::"n"(kEpiThreads) : "memory");
-                    // this CTA's operands of the pass are ready: the even CTA's warp A issues it
-                    if (rank == 0) mbar_arrive(a2ready); else mbar_arrive_cluster(at_even(a2ready));
-                    const bool okw = okp && wait_t(d2full, d2ph, abort_flag, P.status, w_t);
-                    d2ph ^= 1;
-                    if (!bar_and(2, kEpiThreads, okw)) { okp = false; break; }
+                const bool okd = wait_t(dbar + slot, use & 1, abort_flag, P.status, w_t);
+                const bool okt = okd && wait_t(tfull + slot, use & 1, abort_flag, P.status, w_t);
+                if (okt) {
+                    const long long c_e0 = clock64();
                     tc_fence_after();
-                    const long long c_d0 = clock64();
-                    // drain: lane c of this warp owns out[node][l3, m'][c]
-                    for (int sg = s0; sg < s1; ++sg) {
-                        const int node = sl_node[sg];
-                        const int nacc = twob ? 2 : 1;
-                        for (int a2 = 0; a2 < nacc; ++a2) {
-                            const bool vv = a2 == 0 ? vA : vB;
-                            if (!vv) continue;  // warp-uniform: this CTA has no rows of that accumulator
-                            const int dcol = twob ? d2col((sg - s0) + 2 * a2) : d2col(sg - s0);
-                            float v[16];
-                            tmem_ld16(tlane + cb + dcol + 16 * rank, v);
-                            tmem_wait_ld();
-                            const int l3 = a2 == 0 ? l3A : l3B, c = a2 == 0 ? cA : cB;
-                            float* o = P.out + ((size_t)node * K + l3 * l3) * C + c;
-#pragma unroll
-                            for (int mp = 0; mp < 2 * kMaxL + 1; ++mp)
-                                if (mp < 2 * l3 + 1) atomicAdd(o + (size_t)mp * C, v[mp]);
+                    const __half2* Ds = reinterpret_cast<const __half2*>(dstage + slot * S.dstride);
+                    const int lrow = (warp & 3) * 32 + (warp >> 3) * 16;  // this warp's 16 TMEM lanes
+                    const uint32_t twarp = tmem + ((uint32_t)lrow << 16) + slot * 256;
+                    if (g.mu > 0) {
+                        const int row = g.row0 + lrow;  // rows of this warp: one l3, 16 channels
+                        epi_mma<2>(twarp, g.mu + row / C, row % C, K, C, Ds, pb, nb, sg, P.out);
+                    } else {
+                        const int ra = g.row0 + lrow, la = ra / C;
+                        epi_mma<1>(twarp, la, ra % C, K, C, Ds, pb, nb, sg, P.out);
+                        if (g.row0b >= 0) {
+                            const int rb = g.row0b + lrow;
+                            epi_mma<1>(twarp + 128, rb / C, rb % C, K, C, Ds + kTileE * npair(la), pb, nb, sg, P.out);
                         }
                     }
-                    c_dr += clock64() - c_d0;
                     tc_fence_before();
+                    if (dbgon && r == 0) dsub[8] += clock64() - c_e0;
+                } else {
+                    ok = false;
                 }
-                if (dbgon && r == 0) {
-                    const long long c_e3 = clock64();
-                    dsub[8] += c_e3 - c_e0;
-                    dsub[9] += c_e1 - c_e0;   // first pass prepared (if not during the previous group)
-                    dsub[10] += c_e2 - c_e1;  // accumulators awaited and converted
-                    dsub[11] += c_e3 - c_e2;  // passes: issue, completion, drains
-                }
-                if (rank == 0) mbar_arrive(tempty + slot); else mbar_arrive_cluster(at_even(tempty + slot));
-                if (!okp) { ok = false; }
-                // the next group's first pass (its pairs staged, the other buffer free), while its
-                // accumulators are still being computed
-                if (ok && gi + 1 < ng) {
-                    const bool okd2 = wait_t(dbar + (slot ^ 1), ((gcount + 1) >> 1) & 1, abort_flag, P.status, w_t);
-                    if (bar_and(2, kEpiThreads, okd2)) {
-                        const TcGroup gn = P.groups[gi + 1];
-                        const int pern = (gn.mu == 0 && gn.row0b >= 0) ? 2 : 4;
-                        const int kdn = gn.mu > 0 ? 2 : ((gn.mu == 0 && gn.row0b >= 0) ? 1 : 0);
-                        const uint32_t* kln = klist + kdn * 2 * kB2Blocks;
-                        epi_prep_pass(E, gn, gcount + 1, kln, kln + kB2Blocks, klistn[kdn], (int)rank, L, C, et, ew, lane,
-                                      (dbgon && r == 0) ? dsub + 12 : nullptr);
-                        (void)pern;
-                        prepped = true;
-                    } else {
-                        ok = false;
-                    }
-                }
+                mbar_arrive(tempty + slot);
             }
             if (!bar_and(2, kEpiThreads, ok)) { ok = false; break; }
             mbar_arrive(xfree + b);
-            mbar_arrive_cluster(at_peer(xfree + b));
         }
         if (P.dbg && r == 0) {
             long long* d = P.dbg + blockIdx.x * kDbgSlots;
             d[8] = w_x; d[9] = w_t; d[10] = clock64() - c_start; d[13] = ntiles; d[22] = dsub[8];
-            d[28] = dsub[9]; d[29] = dsub[10]; d[30] = dsub[11]; d[31] = dsub[12];
-            d[14] = dsub[13]; d[15] = dsub[14]; d[16] = dsub[15];
         }
-#undef E2F_STAGE_GROUP
         // a staging copy that was issued but never waited for lands before exit
         if (r == 0) {
             for (int s2 = 0; s2 < 2; ++s2) {
@@ -1653,10 +1262,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
     }
 
     tc_fence_before();
-    cluster_sync();  // no MMA of the pair can still touch either CTA's TMEM or shared memory
+    __syncthreads();
     if (warp == 12) {
         tc_fence_after();
-        tmem_dealloc2(tmem, 512);
+        tmem_dealloc(tmem, 512);
     }
 }
 
@@ -1683,12 +1292,12 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-bool make_map(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint32_t box_rows = 128) {
+bool make_map(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows) {
     EncodeTiledFn f = encode_fn();
     if (!f) return false;
     cuuint64_t dims[2] = {cols, rows};
     cuuint64_t strides[1] = {cols * 2};
-    cuuint32_t box[2] = {(cuuint32_t)tc::kKS, box_rows};
+    cuuint32_t box[2] = {(cuuint32_t)tc::kKS, 128};
     cuuint32_t es[2] = {1, 1};
     return f(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -1713,12 +1322,12 @@ struct TcWs {
         dbg = take(kTcDebugBytes);
         lse = take(4 * (size_t)n_atoms * H);
         part = take(4 * (size_t)(kMaxCtas + 1));
-        xs = take((size_t)kMaxCtas * 2 * tc::kHalfE * K * C * 2);
+        xs = take((size_t)kMaxCtas * 2 * tc::kTileE * K * C * 2);
         dscr = take((size_t)kMaxCtas * 2 * tc::dglob_pairs() * 4);
         x16 = take((size_t)n_atoms * K * C * 2);
         w16 = take(so2_total(L, C) * 2);
         whT = take((size_t)Gv * kTcMaxRbf * 2);
-        gscr = take((size_t)kMaxCtas * 2 * tc::kHalfE * Gv * 2);  // two tile buffers per CTA
+        gscr = take((size_t)kMaxCtas * 2 * tc::kTileE * Gv * 2);  // two tile buffers per CTA
         words = take(256);
         total = o;
     }
@@ -1743,21 +1352,9 @@ static cudaError_t launch_tc(const tc::TcParams& P, const tc::TcMaps& T, int gri
     const size_t smem = tc::SmemLayout(L, P.C, P.H, P.n_rbf).total + 1024;
     cudaError_t e = cudaFuncSetAttribute(tc::k_attn_tc<L>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    // CTA pairs: clusters of two along x, sharing tcgen05.mma.cta_group::2
-    cudaLaunchConfig_t lc = {};
-    lc.gridDim = dim3((unsigned)grid);
-    lc.blockDim = dim3(tc::kThreads);
-    lc.dynamicSmemBytes = smem;
-    lc.stream = s;
-    cudaLaunchAttribute at[1];
-    at[0].id = cudaLaunchAttributeClusterDimension;
-    at[0].val.clusterDim.x = 2;
-    at[0].val.clusterDim.y = 1;
-    at[0].val.clusterDim.z = 1;
-    lc.attrs = at;
-    lc.numAttrs = 1;
     count_launch();
-    return cudaLaunchKernelEx(&lc, tc::k_attn_tc<L>, P, T);
+    tc::k_attn_tc<L><<<grid, tc::kThreads, smem, s>>>(P, T);
+    return cudaGetLastError();
 }
 
 cudaError_t run_attention_tc(const AttnArgs& a, void* tc_ws, cudaStream_t s, const CellLists* cl) {
@@ -1772,8 +1369,7 @@ cudaError_t run_attention_tc(const AttnArgs& a, void* tc_ws, cudaStream_t s, con
         const int v = atoi(env);
         if (v > 0 && v < cap) cap = v;
     }
-    const int npairs = std::max(1, std::min(sms, cap) / 2);
-    const int grid = 2 * npairs;
+    const int grid = std::max(1, std::min(sms, cap));
     const TcWs Wl(N, L, C, H);
     char* w = static_cast<char*>(tc_ws);
     long long* dbg = reinterpret_cast<long long*>(w + Wl.dbg);
@@ -1824,7 +1420,7 @@ cudaError_t run_attention_tc(const AttnArgs& a, void* tc_ws, cudaStream_t s, con
         tc::k_softmax_stats<<<(N + 7) / 8, 256, 0, s>>>(sp);
     }
     count_launch();
-    tc::k_partition<<<(npairs + 1 + 127) / 128, 128, 0, s>>>(a.row_ptr, N, npairs, part);
+    tc::k_partition<<<(grid + 1 + 127) / 128, 128, 0, s>>>(a.row_ptr, N, grid, part);
     e = cudaMemsetAsync(a.out, 0, (size_t)N * K * C * 4, s);
     if (e != cudaSuccess) return e;
 
@@ -1843,20 +1439,19 @@ cudaError_t run_attention_tc(const AttnArgs& a, void* tc_ws, cudaStream_t s, con
             if (e != cudaSuccess) return e;
         }
     }
-    // groups of M = 256 rows (rows r0 .. r0 + 127 in the even CTA, r0 + 128 .. in the odd one):
-    // m = 0 feature blocks two at a time; then (o+, o-) per 256 features for m >= 1
+    // groups: m = 0 feature blocks in pairs; then (o+, o-) pairs per block for m >= 1
     int ng = 0;
     const int n0 = (L + 1) * C;
-    for (int r0 = 0; r0 < n0; r0 += 512) {
+    for (int r0 = 0; r0 < n0; r0 += 256) {
         tc::TcGroup g{};
-        g.mu = 0; g.row0 = r0; g.row0b = (r0 + 256 < n0) ? r0 + 256 : -1; g.klen = n0; g.xoff0 = 0; g.xoff1 = 0;
+        g.mu = 0; g.row0 = r0; g.row0b = (r0 + 128 < n0) ? r0 + 128 : -1; g.klen = n0; g.xoff0 = 0; g.xoff1 = 0;
         g.wa = 0; g.wb = 0;
         P.groups[ng++] = g;
     }
     int koff = n0;
     for (int mu = 1; mu <= a.M; ++mu) {  // |m| > M: no message (truncated layer)
         const int nm = (L + 1 - mu) * C;
-        for (int r0 = 0; r0 < nm; r0 += 256) {
+        for (int r0 = 0; r0 < nm; r0 += 128) {
             tc::TcGroup g{};
             g.mu = mu; g.row0 = r0; g.row0b = -1; g.klen = nm; g.xoff0 = koff; g.xoff1 = koff + nm;
             g.wa = 2 * mu - 1; g.wb = 2 * mu;
@@ -1874,7 +1469,7 @@ cudaError_t run_attention_tc(const AttnArgs& a, void* tc_ws, cudaStream_t s, con
         if (!make_map(&T.w[2 * mu - 1], W + so2_offset(L, C, mu, 0), nm, nm)) return cudaErrorInvalidValue;
         if (!make_map(&T.w[2 * mu], W + so2_offset(L, C, mu, 1), nm, nm)) return cudaErrorInvalidValue;
     }
-    if (!make_map(&T.xs, xs, (uint64_t)K * C, (uint64_t)grid * 2 * tc::kHalfE, tc::kHalfE)) return cudaErrorInvalidValue;
+    if (!make_map(&T.xs, xs, (uint64_t)K * C, (uint64_t)grid * 2 * tc::kTileE)) return cudaErrorInvalidValue;
 
     if (g_kernel_ev[0] && g_kernel_ev[1]) {
         e = cudaEventRecord(g_kernel_ev[0], s);

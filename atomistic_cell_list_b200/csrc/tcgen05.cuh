@@ -35,33 +35,6 @@ __device__ __forceinline__ bool mbar_try(uint64_t* b, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
-// non-blocking test of a phase (never suspends the thread)
-__device__ __forceinline__ bool mbar_test(uint64_t* b, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}\n"
-        : "=r"(ok)
-        : "r"(smem_u32(b)), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-// Same, suspending the thread for up to `ns` nanoseconds while the phase is
-// incomplete (it resumes as soon as the phase completes): waiting threads then
-// take no issue slots from the working ones.
-__device__ __forceinline__ bool mbar_try_sleep(uint64_t* b, uint32_t parity, uint32_t ns) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}\n"
-        : "=r"(ok)
-        : "r"(smem_u32(b)), "r"(parity), "r"(ns)
-        : "memory");
-    return ok != 0;
-}
-constexpr uint32_t kSuspendNs = 20000;  // per try: the bounded-wait checks still run every 20 us
 __device__ __forceinline__ uint64_t gtimer() {
     uint64_t t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -91,7 +64,7 @@ __device__ __forceinline__ bool wait(uint64_t* b, uint32_t parity, volatile int*
     if (mbar_try(b, parity)) return true;
     const uint64_t t0 = gtimer();
     while (true) {
-        if (mbar_try_sleep(b, parity, kSuspendNs)) return true;
+        if (mbar_try(b, parity)) return true;
         if (*abort_flag) return false;
         if (gtimer() - t0 > kWaitNs) {
             *abort_flag = 1;
@@ -104,7 +77,6 @@ __device__ __forceinline__ bool wait(uint64_t* b, uint32_t parity, volatile int*
 // Same, adding the cycles spent waiting to `acc` (per-role wait counters).
 __device__ __forceinline__ bool wait_t(uint64_t* b, uint32_t parity, volatile int* abort_flag, int* status,
                                        long long& acc) {
-    if (mbar_try(b, parity)) return true;
     const long long c0 = clock64();
     const bool r = wait(b, parity, abort_flag, status);
     acc += clock64() - c0;
@@ -195,151 +167,6 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
-
-}  // namespace tc
-}  // namespace e2f
-
-namespace e2f {
-namespace tc {
-
-// ---- CTA pairs (clusters of two) sharing one tcgen05.mma.cta_group::2 stream ----
-__device__ __forceinline__ uint32_t cluster_rank() {
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-    return r;
-}
-// shared::cluster address of the same shared-memory offset in CTA `rank` of the cluster
-__device__ __forceinline__ uint32_t mapa(uint32_t saddr, uint32_t rank) {
-    uint32_t r;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
-    return r;
-}
-__device__ __forceinline__ void cluster_sync() {
-    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-// arrive on an mbarrier of any CTA of the cluster (release at cluster scope)
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t caddr) {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(caddr) : "memory");
-}
-// expect `tx` bytes on a local barrier and arrive (release at cluster scope)
-__device__ __forceinline__ void mbar_arrive_tx_cluster(uint64_t* b, uint32_t tx) {
-    asm volatile("mbarrier.arrive.expect_tx.release.cluster.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(b)), "r"(tx)
-                 : "memory");
-}
-// wait with acquire at cluster scope (for phases completed by arrivals from the peer CTA)
-__device__ __forceinline__ bool mbar_try_cluster(uint64_t* b, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}\n"
-        : "=r"(ok)
-        : "r"(smem_u32(b)), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-__device__ __forceinline__ bool mbar_try_cluster_sleep(uint64_t* b, uint32_t parity, uint32_t ns) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}\n"
-        : "=r"(ok)
-        : "r"(smem_u32(b)), "r"(parity), "r"(ns)
-        : "memory");
-    return ok != 0;
-}
-// non-blocking test of a phase (no suspension), acquire at cluster scope
-__device__ __forceinline__ bool mbar_test_cluster(uint64_t* b, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.test_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}\n"
-        : "=r"(ok)
-        : "r"(smem_u32(b)), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-__device__ __forceinline__ bool wait_cluster(uint64_t* b, uint32_t parity, volatile int* abort_flag, int* status,
-                                             long long& acc) {
-    const long long c0 = clock64();
-    bool r = true;
-    if (!mbar_try_cluster(b, parity)) {
-        const uint64_t t0 = gtimer();
-        while (true) {
-            if (mbar_try_cluster_sleep(b, parity, kSuspendNs)) break;
-            if (*abort_flag) { r = false; break; }
-            if (gtimer() - t0 > kWaitNs) {
-                *abort_flag = 1;
-                atomicExch(status, (int)E2F_ERR_TIMEOUT);
-                r = false;
-                break;
-            }
-        }
-    }
-    acc += clock64() - c0;
-    return r;
-}
-__device__ __forceinline__ void st_cluster_f32(uint32_t caddr, float v) {
-    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(caddr), "f"(v) : "memory");
-}
-__device__ __forceinline__ void st_cluster_u32(uint32_t caddr, uint32_t v) {
-    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(caddr), "r"(v) : "memory");
-}
-
-// TMEM allocation shared by the two CTAs of a pair (one warp with the same
-// warp index in each CTA executes these)
-__device__ __forceinline__ void tmem_alloc2(uint32_t* dst, uint32_t ncols) {
-    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst)), "r"(ncols)
-                 : "memory");
-}
-__device__ __forceinline__ void tmem_relinquish2() {
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void tmem_dealloc2(uint32_t taddr, uint32_t ncols) {
-    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
-}
-
-// Pair MMAs (issued by one thread of the even CTA): A rows split between the
-// CTAs' shared memory (or TMEM), B columns split between their shared
-// memory, each CTA's TMEM holding its half of the rows of D.
-__device__ __forceinline__ void umma2_ss(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, int accumulate) {
-    if (accumulate)
-        asm volatile("tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, 1;" ::"r"(d), "l"(a), "l"(b), "r"(idesc)
-                     : "memory");
-    else
-        asm volatile("tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, 0;" ::"r"(d), "l"(a), "l"(b), "r"(idesc)
-                     : "memory");
-}
-__device__ __forceinline__ void umma2_ts(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc, int accumulate) {
-    if (accumulate)
-        asm volatile("tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, 1;" ::"r"(d), "r"(a_tmem), "l"(b),
-                     "r"(idesc)
-                     : "memory");
-    else
-        asm volatile("tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, 0;" ::"r"(d), "r"(a_tmem), "l"(b),
-                     "r"(idesc)
-                     : "memory");
-}
-// completion of this thread's pair MMAs arrives on the barrier at the same
-// offset in both CTAs
-__device__ __forceinline__ void umma2_commit_both(uint64_t* bar) {
-    asm volatile(
-        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
-            smem_u32(bar)),
-        "h"((uint16_t)3)
-        : "memory");
-}
-// TMA tile load into this CTA's shared memory whose completion is counted on
-// the even CTA's barrier (cluster address `bar_c`); no multicast
-__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map, int x, int y, uint32_t bar_c) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
-        "[%4];" ::"r"(smem_u32(dst)),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar_c)
-        : "memory");
-}
 
 }  // namespace tc
 }  // namespace e2f
