@@ -66,6 +66,7 @@ _SIGS = {
     "e2f_launch_count": (_i64, []),
     "e2f_attention_uses_tensor_cores": (ctypes.c_int, [ctypes.POINTER(e2f_attn_cfg)]),
     "e2f_attention_set_kernel_events": (None, [_vp, _vp]),
+    "e2f_attention_set_debug": (None, [ctypes.c_int, ctypes.c_int, ctypes.c_int]),
     "e2f_attention_debug_timers": (ctypes.c_int, [_vp, _sz, _i64, ctypes.POINTER(e2f_attn_cfg),
                                                   ctypes.POINTER(_i64), ctypes.c_int, _vp]),
 }
@@ -349,7 +350,7 @@ DEBUG_SLOTS = 32
 
 def e2f_attention_debug_timers(workspace: torch.Tensor, n_atoms: int, cfg: e2f_attn_cfg, n_ctas: int = 160,
                                stream=None):
-    """Per-CTA role cycle counters of the last tensor-core call (E2F_TC_TIMERS=1)."""
+    """Per-CTA role cycle counters of the last tensor-core call (timers on: e2f_attention_set_debug)."""
     import numpy as np
     n = DEBUG_SLOTS * n_ctas
     buf = (_i64 * n)()
@@ -363,6 +364,11 @@ def e2f_attention_set_kernel_events(start=None, stop=None):
     a = None if start is None else ctypes.c_void_p(start.cuda_event)
     b = None if stop is None else ctypes.c_void_p(stop.cuda_event)
     lib().e2f_attention_set_kernel_events(a, b)
+
+
+def e2f_attention_set_debug(max_ctas: int = 0, timers: bool = False, drop_arrive: bool = False):
+    """Debug and test controls of the tensor-core kernel (process-wide; all off restores the default)."""
+    lib().e2f_attention_set_debug(int(max_ctas), int(bool(timers)), int(bool(drop_arrive)))
 
 
 def e2f_launch_count() -> int:

@@ -277,6 +277,10 @@ extern "C" void e2f_attention_set_kernel_events(void* start_event, void* stop_ev
     set_tc_kernel_events(start_event, stop_event);
 }
 
+extern "C" void e2f_attention_set_debug(int max_ctas, int timers, int drop_arrive) {
+    set_tc_debug(max_ctas, timers, drop_arrive);
+}
+
 namespace {
 
 struct BwdWs {

@@ -90,6 +90,10 @@ struct CellLists;
 // cl != nullptr: fused traversal (a.row_ptr = per-slot offsets in cell order, a.col unused)
 cudaError_t run_attention_tc(const AttnArgs& a, void* tc_ws, cudaStream_t s, const CellLists* cl = nullptr);
 void set_tc_kernel_events(void* start, void* stop);
+// Debug and test controls of the tensor-core kernel (process-wide): max_ctas > 0
+// caps the persistent CTAs, timers != 0 records role cycle counters, drop_arrive
+// != 0 makes CTA 0 withhold one producer arrival on its first tile.
+void set_tc_debug(int max_ctas, int timers, int drop_arrive);
 cudaError_t run_edge_wigner(const float* r, int64_t n, int L, float* out, float* frames, cudaStream_t s);
 
 }  // namespace e2f

@@ -963,7 +963,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
             mbar_arrive(gempty + b);  // this tile's value gates have been read
             // generic-proxy stores (features, Wigner pairs) -> visible to TMA / bulk copies
             asm volatile("fence.proxy.async.global;" ::: "memory");
-            mbar_arrive(xready + b);
+            // (test hook: CTA 0 withholds one arrival on its first tile, so that the
+            // bounded waits on xready run out and the CTA takes its abort path)
+            if (!(P.drop_arrive && blockIdx.x == 0 && t == 0 && p == 0)) mbar_arrive(xready + b);
             c_p2 += clock64() - c_b;
         }
         if (P.dbg && p == 0) {
@@ -1340,11 +1342,19 @@ namespace {
 // caller events recorded around the main kernel (profiling aid; see
 // e2f_attention_set_kernel_events)
 cudaEvent_t g_kernel_ev[2] = {nullptr, nullptr};
+// debug and test controls (set_tc_debug)
+int g_dbg_max_ctas = 0, g_dbg_timers = 0, g_dbg_drop = 0;
 }  // namespace
 
 void set_tc_kernel_events(void* start, void* stop) {
     g_kernel_ev[0] = static_cast<cudaEvent_t>(start);
     g_kernel_ev[1] = static_cast<cudaEvent_t>(stop);
+}
+
+void set_tc_debug(int max_ctas, int timers, int drop_arrive) {
+    g_dbg_max_ctas = max_ctas;
+    g_dbg_timers = timers;
+    g_dbg_drop = drop_arrive;
 }
 
 template <int L>
@@ -1365,10 +1375,7 @@ cudaError_t run_attention_tc(const AttnArgs& a, void* tc_ws, cudaStream_t s, con
     e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
     int cap = kMaxCtas;
-    if (const char* env = getenv("E2F_TC_MAX_CTAS")) {  // launch-shape override (tests): fewer, longer CTAs
-        const int v = atoi(env);
-        if (v > 0 && v < cap) cap = v;
-    }
+    if (g_dbg_max_ctas > 0 && g_dbg_max_ctas < cap) cap = g_dbg_max_ctas;  // fewer, longer CTAs (tests)
     const int grid = std::max(1, std::min(sms, cap));
     const TcWs Wl(N, L, C, H);
     char* w = static_cast<char*>(tc_ws);
@@ -1432,13 +1439,12 @@ cudaError_t run_attention_tc(const AttnArgs& a, void* tc_ws, cudaStream_t s, con
     P.cells = cl ? 1 : 0;
     if (cl) P.cv = cl->view;
     P.dbg = nullptr;
-    if (const char* env = getenv("E2F_TC_TIMERS")) {
-        if (atoi(env) > 0) {
-            P.dbg = dbg;
-            e = cudaMemsetAsync(dbg, 0, kTcDebugBytes, s);
-            if (e != cudaSuccess) return e;
-        }
+    if (g_dbg_timers) {
+        P.dbg = dbg;
+        e = cudaMemsetAsync(dbg, 0, kTcDebugBytes, s);
+        if (e != cudaSuccess) return e;
     }
+    P.drop_arrive = g_dbg_drop ? 1 : 0;
     // groups: m = 0 feature blocks in pairs; then (o+, o-) pairs per block for m >= 1
     int ng = 0;
     const int n0 = (L + 1) * C;

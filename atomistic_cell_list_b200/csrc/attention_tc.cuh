@@ -67,6 +67,7 @@ struct TcParams {
     float* out;
     int* status;
     long long* dbg;  // per-CTA role cycle counters, or null
+    int drop_arrive; // test hook: CTA 0 withholds one producer arrival on its first tile
     int n_groups;
     TcGroup groups[kMaxGroups];
 };

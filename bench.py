@@ -48,8 +48,8 @@ def measured_peaks():
         "fallback"
 
 
-# DRAM traffic of one k_attn_tc launch on the 30000-atom workload, from the ncu
-# capture summarised in profiles/k_attn_tc_chain_water_30k.md. Valid only for
+# DRAM traffic of one k_attn_tc launch on the 30000-atom workload, from an ncu
+# capture of that kernel on that workload (dram__bytes_read/write). Valid only for
 # the kernel source it was taken on (sha256 of the files below); otherwise the
 # bench reports traffic null.
 KERNEL_TRAFFIC = {
@@ -457,7 +457,7 @@ def run_ours(args):
     roof["kernel"] = "k_attn_tc (tcgen05)" if path == "tensor" else "k_attn_simt (fp32 CUDA cores)"
     roof["ms_per_launch"] = ms_ker
     roof["units_per_launch"] = f"{E} edges x {F} SO(2) FLOP"
-    roof["traffic_note"] = ("dram read+write bytes per launch from ncu (profiles/k_attn_tc_chain_water_30k.md); "
+    roof["traffic_note"] = ("dram read+write bytes per launch from an ncu capture of k_attn_tc on this workload; "
                             "null when the kernel source differs from the profiled one")
 
     nbr_bytes = 16 * w.n_atoms + 4 * (w.n_atoms + 1) + 4 * E + 8 * w.n_atoms

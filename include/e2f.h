@@ -181,9 +181,9 @@ e2f_status e2f_build_neighbors_noalloc(const float* pos, int64_t n_atoms,
  *              aligned, contents need no initialisation. Holds the
  *              repacked weights, per-node Q/K and softmax statistics and a
  *              device status word; it must not be shared by calls in flight.
- * Launch shape: the tensor-core kernel runs one persistent CTA per SM; the
- * environment variable E2F_TC_MAX_CTAS (read at each call) caps that count,
- * which lets tests give each CTA many tiles on small systems.
+ * Launch shape: the tensor-core kernel runs one persistent CTA per SM
+ * (e2f_attention_set_debug can cap that count, which lets tests give each
+ * CTA many tiles on small systems).
  * Asynchronous: returns after enqueueing. Device-side failures (a bounded
  * wait that ran out) are recorded in the workspace status word; read it
  * with e2f_attention_status.
@@ -214,8 +214,21 @@ int e2f_attention_uses_tensor_cores(const e2f_attn_cfg* cfg);
  * for concurrent calls from several threads. */
 void e2f_attention_set_kernel_events(void* start_event, void* stop_event);
 
-/* Diagnostics of the tensor-core kernel. When the environment variable
- * E2F_TC_TIMERS=1 is set at call time, each persistent CTA records clock64
+/* Debug and test controls of the tensor-core kernel (no counterpart in the
+ * pages). One process-wide setting, read when a call is enqueued; not for
+ * concurrent calls from several threads. All zero (the default) is the
+ * product behaviour.
+ *   max_ctas     > 0: at most this many persistent CTAs (fewer, longer CTAs).
+ *   timers       != 0: record the role cycle counters (e2f_attention_debug_timers).
+ *   drop_arrive  != 0: CTA 0 withholds one producer arrival on its first tile,
+ *                so its bounded waits run out (about 2 s): the CTA records
+ *                E2F_ERR_TIMEOUT in the workspace status word, drains what it
+ *                issued and returns; the other CTAs finish normally. Used to
+ *                test the timeout path; the output of such a call is invalid. */
+void e2f_attention_set_debug(int max_ctas, int timers, int drop_arrive);
+
+/* Diagnostics of the tensor-core kernel. When timers are on
+ * (e2f_attention_set_debug), each persistent CTA records clock64
  * cycle counts of its warp roles into the workspace: per CTA 32 int64 values,
  * [0] producer wait for a free tile buffer, [1] producer total, [2] TMA wait
  * for features, [3] TMA wait for a free ring stage, [4] TMA total, [5] MMA

@@ -1,9 +1,7 @@
 """Tensor-core (tcgen05) attention against the fp64 oracle on every node of
 small systems: several 128-edge tiles per CTA (grid capped through
-E2F_TC_MAX_CTAS), nodes straddling tiles, ragged tails, isolated atoms, and
+e2f_attention_set_debug), nodes straddling tiles, ragged tails, isolated atoms, and
 the supported shapes (L = 1..4, C = 128 or 256, H = 4..16)."""
-import os
-
 import numpy as np
 import pytest
 import torch
@@ -47,17 +45,13 @@ def run_case(seed, n, side, cutoff, L, C, H, max_ctas, rel_tol=2e-2, isolate=0):
     pos_d = torch.from_numpy(pos).to(d)
     blist = None if box is None else box.tolist()
     rp, col = e2f.e2f_build_neighbors(pos_d, blist, cutoff)
-    old = os.environ.get("E2F_TC_MAX_CTAS")
-    os.environ["E2F_TC_MAX_CTAS"] = str(max_ctas)
+    e2f.e2f_attention_set_debug(max_ctas=max_ctas)
     try:
         out = e2f.e2f_onfly_attention(cfg, pos_d, blist, rp, col, to_dev_storage(x_st, "bf16").reshape(n, -1, C),
                                       torch.from_numpy(wt.Wq).to(d), torch.from_numpy(wt.Wk).to(d),
                                       torch.from_numpy(wt.Wrad).to(d), to_dev_storage(wt.Wso2, "bf16"))
     finally:
-        if old is None:
-            del os.environ["E2F_TC_MAX_CTAS"]
-        else:
-            os.environ["E2F_TC_MAX_CTAS"] = old
+        e2f.e2f_attention_set_debug()
     out = out.cpu().numpy().astype(np.float64)
     rp0, col0 = neighbors_bruteforce(pos, box, cutoff)
     np.testing.assert_array_equal(rp.cpu().numpy(), rp0)

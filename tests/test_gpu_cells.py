@@ -8,6 +8,7 @@ import torch
 import atomistic_cell_list_b200 as e2f
 import workloads as W
 from gpu_util import TOL, DeviceInputs, oracle_csr, rel_err_per_degree
+from oracle.layer import DenseLayer
 
 pytestmark = pytest.mark.gpu
 
@@ -94,6 +95,48 @@ def test_fused_traversal_open_boundaries():
     assert rel_err_per_degree(fused.cpu().numpy(), csr.cpu().numpy(), w.L) <= 1e-3
     # atoms near the faces have fewer neighbours than in the periodic box
     assert col.numel() < e2f.e2f_build_neighbors(d.pos, d.box, w.cutoff)[1].numel()
+
+
+def test_fused_traversal_open_boundaries_matches_the_oracle():
+    # the open mode has its own enumeration (hashed buckets): compare it with the oracle
+    # directly, on random nodes and on the nodes nearest the faces of the cloud
+    from oracle.neighbors import neighbors_bruteforce
+    d = DeviceInputs(3)
+    w = d.w
+    cfg = e2f.make_cfg(w.L, w.C, w.H, w.n_rbf, w.cutoff, w.dtype)
+    fused = e2f.e2f_onfly_attention_cells(cfg, d.pos, None, d.x, d.Wq, d.Wk, d.Wrad, d.Wso2)
+    rp0, col0 = neighbors_bruteforce(w.pos, None, w.cutoff)
+    p = w.pos.astype(np.float64)
+    face = np.minimum(p - p.min(axis=0), p.max(axis=0) - p).min(axis=1)
+    nodes = np.unique(np.concatenate([np.random.default_rng(12).choice(w.n_atoms, 24, replace=False),
+                                      np.argsort(face)[:12]]))
+    ref = d.oracle()(w.pos, None, rp0, col0, d.x_f64, nodes=nodes)
+    assert rel_err_per_degree(fused.cpu().numpy()[nodes].astype(np.float64), ref, w.L) <= TOL[w.dtype]
+
+
+def test_fused_traversal_dense_open_matches_the_oracle():
+    # about 300-570 neighbours per atom without a box: several tiles and statistics windows
+    # per node in the open mode, checked against the oracle on sampled nodes
+    from oracle.neighbors import neighbors_bruteforce
+    d = DeviceInputs(3)
+    w = d.w
+    n, side, rc = 4000, 17.0, 5.5
+    pos = np.random.default_rng(6).uniform(0.0, side, (n, 3)).astype(np.float32)
+    reps = -(-n // w.n_atoms)
+    x = d.x.repeat(reps, 1, 1)[:n].contiguous()
+    x_f64 = np.concatenate([d.x_f64] * reps)[:n]
+    cfg = e2f.make_cfg(w.L, w.C, w.H, w.n_rbf, rc, w.dtype)
+    fused = e2f.e2f_onfly_attention_cells(cfg, torch.from_numpy(pos).to(d.pos.device), None, x, d.Wq, d.Wk,
+                                          d.Wrad, d.Wso2)
+    rp0, col0 = neighbors_bruteforce(pos, None, rc)
+    deg = np.diff(rp0)
+    assert deg.max() > 512
+    nodes = np.unique(np.concatenate([np.random.default_rng(13).choice(n, 6, replace=False),
+                                      np.argsort(-deg, kind="stable")[:3], np.argsort(deg, kind="stable")[:3]]))
+    wt = d.weights  # the oracle layer with this case's cutoff (radial basis and envelope)
+    ref = DenseLayer(w.L, w.C, w.H, w.n_rbf, rc, wt.Wq, wt.Wk, wt.Wrad, wt.Wso2_f64)(pos, None, rp0, col0, x_f64,
+                                                                                    nodes=nodes)
+    assert rel_err_per_degree(fused.cpu().numpy()[nodes].astype(np.float64), ref, w.L) <= TOL[w.dtype]
 
 
 # ---- Verlet-skin reuse of the cell lists across MD steps ---------------------

@@ -40,7 +40,7 @@ def test_kernel_events_bracket_the_main_kernel():
     assert torch.equal(out, ref)  # recording events changes nothing
 
 
-def test_debug_timers_count_every_tile(monkeypatch):
+def test_debug_timers_count_every_tile():
     d = DeviceInputs(3)
     w = d.w
     cfg = e2f.make_cfg(w.L, w.C, w.H, w.n_rbf, w.cutoff, w.dtype)
@@ -48,8 +48,11 @@ def test_debug_timers_count_every_tile(monkeypatch):
     ws = torch.empty(e2f.e2f_attention_workspace_size(w.n_atoms, col.numel(), cfg), dtype=torch.uint8,
                      device=d.pos.device)
     ref = _call(d, cfg, rp, col, ws)
-    monkeypatch.setenv("E2F_TC_TIMERS", "1")
-    out = _call(d, cfg, rp, col, ws)
+    e2f.e2f_attention_set_debug(timers=True)
+    try:
+        out = _call(d, cfg, rp, col, ws)
+    finally:
+        e2f.e2f_attention_set_debug()
     t = e2f.e2f_attention_debug_timers(ws, w.n_atoms, cfg)
     tiles = int(t[:, 13].sum())
     # every 128-edge tile of every CTA is counted once: at least ceil(E / 128) tiles
