@@ -377,19 +377,39 @@ __host__ __device__ constexpr size_t dglob_block(int l, int mu) { return (size_t
 static_assert(npair(0) == 4 && npair(1) == 4 && npair(2) == 8 && npair(3) == 8 && npair(4) == 12, "pairs");
 static_assert(dptotal(4) == 128, "pair layout");
 
-// Bytes of Wigner pairs one group's epilogue stages: npair(l) pairs of 4
-// bytes per edge for each feature block the group covers (m = 0 groups cover
-// two 128-row blocks, possibly of different degrees).
+// Degrees of the rows of a group: its 128-row blocks (one, or two for m = 0)
+// start at rows row0 (and row0b) of the |m| section, whose rows are (l3, c)
+// with l3 from |m| (m > 0) or 0 upwards; a block holds 128 / C degrees when
+// C = 64. The range [lo, hi] is contiguous and clipped to L (rows past the
+// section are zero-filled padding).
+__host__ __device__ inline void group_l3_range(const TcGroup& g, int L, int C, int& lo, int& hi) {
+    const int base = g.mu > 0 ? g.mu : 0;
+    const int last = (g.mu == 0 && g.row0b >= 0) ? g.row0b : g.row0;
+    lo = base + g.row0 / C;
+    hi = min(L, base + (last + 127) / C);
+}
+__host__ __device__ inline int pairs_in(int lo, int hi) {
+    int n = 0;
+    for (int l = lo; l <= hi; ++l) n += npair(l);
+    return n;
+}
+
+// Bytes of Wigner pairs one group's epilogue stages: npair(l3) pairs of 4
+// bytes per edge for each degree l3 of the group's rows (largest over the
+// groups of a layer).
 __host__ __device__ inline size_t stage_bytes(int L, int C) {
-    size_t mx = (size_t)kTileE * 4 * npair(L);  // an |m| >= 1 group of degree L
-    const int n0 = (L + 1) * C;
-    for (int r0 = 0; r0 < n0; r0 += 256) {
-        const int la = r0 / C, lb = (r0 + 128 < n0) ? (r0 + 128) / C : -1;
-        size_t b = (size_t)kTileE * 4 * npair(la);
-        if (lb >= 0) b += (size_t)kTileE * 4 * npair(lb);
-        mx = b > mx ? b : mx;
+    int mx = 0;
+    for (int mu = 0; mu <= L; ++mu) {
+        const int nm = (L + 1 - mu) * C, step = mu > 0 ? 128 : 256;
+        for (int r0 = 0; r0 < nm; r0 += step) {
+            TcGroup g{};
+            g.mu = mu; g.row0 = r0; g.row0b = (mu == 0 && r0 + 128 < nm) ? r0 + 128 : -1;
+            int lo, hi;
+            group_l3_range(g, L, C, lo, hi);
+            mx = max(mx, pairs_in(lo, hi));
+        }
     }
-    return mx;
+    return (size_t)kTileE * 4 * mx;
 }
 
 // Shared memory layout (bytes), shared by host (size) and device (offsets).
@@ -582,27 +602,20 @@ __device__ __noinline__ void epi_mma(uint32_t tacc, int l3, int cbase, int K, in
 
 // Wigner slice(s) a group's epilogue needs, by block (l, mu): returns bytes
 // queued on `bar` into staging buffer `dst`.
-__device__ __forceinline__ uint32_t stage_group_pairs(const TcGroup& g, int C, const __half2* Dglob, uint8_t* dst,
-                                                      uint64_t* bar) {
-    if (g.mu > 0) {
-        const int l3 = g.mu + g.row0 / C;
+// The slices (l3, |m|) of every degree of the group's rows, in increasing l3,
+// one after another (the slice of degree l3 starts at pairs_in(lo, l3 - 1)).
+__device__ __forceinline__ uint32_t stage_group_pairs(const TcGroup& g, int L, int C, const __half2* Dglob,
+                                                      uint8_t* dst, uint64_t* bar) {
+    int lo, hi;
+    group_l3_range(g, L, C, lo, hi);
+    const uint32_t total = (uint32_t)kTileE * 4 * pairs_in(lo, hi);
+    mbar_arrive_tx(bar, total);
+    for (int l3 = lo; l3 <= hi; ++l3) {
         const uint32_t bytes = (uint32_t)kTileE * npair(l3) * 4;
-        mbar_arrive_tx(bar, bytes);
         bulk_load(dst, Dglob + dglob_block(l3, g.mu), bytes, bar);
-        return bytes;
+        dst += bytes;
     }
-    const int la = g.row0 / C;
-    const uint32_t ba = (uint32_t)kTileE * npair(la) * 4;
-    uint32_t bb = 0;
-    int lb = -1;
-    if (g.row0b >= 0) {
-        lb = g.row0b / C;
-        bb = (uint32_t)kTileE * npair(lb) * 4;
-    }
-    mbar_arrive_tx(bar, ba + bb);
-    bulk_load(dst, Dglob + dglob_block(la, 0), ba, bar);
-    if (lb >= 0) bulk_load(dst + ba, Dglob + dglob_block(lb, 0), bb, bar);
-    return ba + bb;
+    return total;
 }
 
 template <int L>
@@ -1205,14 +1218,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
             const int* nb = nid + b * kTileE;
             const uint32_t* sg = segm + b * (kTileE / kChunk);
             if (r == 0) {
-                stage_group_pairs(P.groups[0], C, Dg, dstage + (gcount & 1) * S.dstride, dbar + (gcount & 1));
+                stage_group_pairs(P.groups[0], L, C, Dg, dstage + (gcount & 1) * S.dstride, dbar + (gcount & 1));
                 staged[gcount & 1] = gcount;
             }
             for (int gi = 0; gi < ng; ++gi, ++gcount) {
                 // all threads are done with group gcount-1, so its staging buffer can be refilled
                 if (!bar_and(2, kEpiThreads, ok)) { ok = false; break; }
                 if (r == 0 && gi + 1 < ng) {
-                    stage_group_pairs(P.groups[gi + 1], C, Dg, dstage + ((gcount + 1) & 1) * S.dstride,
+                    stage_group_pairs(P.groups[gi + 1], L, C, Dg, dstage + ((gcount + 1) & 1) * S.dstride,
                                       dbar + ((gcount + 1) & 1));
                     staged[(gcount + 1) & 1] = gcount + 1;
                 }
@@ -1227,15 +1240,22 @@ __global__ void __launch_bounds__(kThreads, 1) k_attn_tc(const __grid_constant__
                     const __half2* Ds = reinterpret_cast<const __half2*>(dstage + slot * S.dstride);
                     const int lrow = (warp & 3) * 32 + (warp >> 3) * 16;  // this warp's 16 TMEM lanes
                     const uint32_t twarp = tmem + ((uint32_t)lrow << 16) + slot * 256;
+                    int lo, hi;
+                    group_l3_range(g, L, C, lo, hi);
+                    // rows of this warp: one l3, 16 channels; rows past degree L are padding
                     if (g.mu > 0) {
-                        const int row = g.row0 + lrow;  // rows of this warp: one l3, 16 channels
-                        epi_mma<2>(twarp, g.mu + row / C, row % C, K, C, Ds, pb, nb, sg, P.out);
+                        const int row = g.row0 + lrow, l3 = g.mu + row / C;
+                        if (l3 <= L)
+                            epi_mma<2>(twarp, l3, row % C, K, C, Ds + kTileE * pairs_in(lo, l3 - 1), pb, nb, sg, P.out);
                     } else {
                         const int ra = g.row0 + lrow, la = ra / C;
-                        epi_mma<1>(twarp, la, ra % C, K, C, Ds, pb, nb, sg, P.out);
+                        if (la <= L)
+                            epi_mma<1>(twarp, la, ra % C, K, C, Ds + kTileE * pairs_in(lo, la - 1), pb, nb, sg, P.out);
                         if (g.row0b >= 0) {
-                            const int rb = g.row0b + lrow;
-                            epi_mma<1>(twarp + 128, rb / C, rb % C, K, C, Ds + kTileE * npair(la), pb, nb, sg, P.out);
+                            const int rb = g.row0b + lrow, lb = rb / C;
+                            if (lb <= L)
+                                epi_mma<1>(twarp + 128, lb, rb % C, K, C, Ds + kTileE * pairs_in(lo, lb - 1), pb, nb, sg,
+                                           P.out);
                         }
                     }
                     tc_fence_before();
@@ -1309,7 +1329,7 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows) {
 }  // namespace
 
 bool tc_supported(int L, int C, int H, int n_rbf, bool bf16) {
-    return bf16 && L >= 1 && L <= kMaxL && C % 128 == 0 && C <= 256 && H <= kMaxHeads && H % 4 == 0 &&
+    return bf16 && L >= 1 && L <= kMaxL && (C % 128 == 0 || C == 64) && C <= 256 && H <= kMaxHeads && H % 4 == 0 &&
            C % H == 0 && (C / H) % 8 == 0 &&
            n_rbf <= kTcMaxRbf && tc::SmemLayout(L, C, H, n_rbf).total + 1024 <= 232448;
 }

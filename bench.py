@@ -56,7 +56,7 @@ KERNEL_TRAFFIC = {
     "sources": ["atomistic_cell_list_b200/csrc/attention_tc.cu", "atomistic_cell_list_b200/csrc/attention_tc.cuh",
                 "atomistic_cell_list_b200/csrc/common.cuh", "atomistic_cell_list_b200/csrc/cell_grid.cuh",
                 "atomistic_cell_list_b200/csrc/tcgen05.cuh"],
-    "sha256": "4c8b466ccf817451f58f192ae9c8b4a7c5decf41b270e270320e7b009d33a20c",
+    "sha256": "94a15b5a5f563af2dc088583fad46535cb12fb3126d4e1ccb3e7ac6cb5500fae",
     "dram_read_bytes": 44.43e9,
     "dram_write_bytes": 23.97e9,
 }
@@ -487,6 +487,13 @@ def run_ours(args):
                                   "note": "the library's only scratch is the caller's workspace: O(N) + O(SMs), "
                                           "no per-edge float tensor"},
             "clocks": clk.summary()}
+    if world == 1 and not args.no_extra:
+        # the other workloads (parity-test cases, not bench lines) and the backward, after the timed region
+        del dbuf, obuf, pinned, h_outs
+        line["per_config"] = {}
+        for c in (2, 3, 4, 5):
+            line["per_config"][f"cfg{c}"] = measure_config(c, dev, 3, 2, flush, peaks)
+        line["backward"] = backward_record(args.config, dev, 2, peaks)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = oracle_rate(args.config, float(os.environ.get("E2F_CPU_BUDGET_S", "15")))
     if rank == 0:
@@ -494,6 +501,132 @@ def run_ours(args):
     if world > 1:
         dist.destroy_process_group()
     return 0
+
+
+def measure_config(cfg_id, dev, steps, warmup, flush, peaks):
+    """One workload of the five: step time (neighbour build + attention, L2 flushed
+    between steps), pairs/s, SO(2) TFLOP/s and its fraction of the measured peak of
+    the path it runs on, and the peak activation memory of the attention call
+    measured with the allocator (max_memory_allocated during a call that allocates
+    its own workspace and output, minus the fp32 output), per atom."""
+    import torch
+
+    import atomistic_cell_list_b200 as e2f
+    import workloads as W
+
+    w = W.load_workload(cfg_id)
+    xs, _ = W.make_features(cfg_id, w.n_atoms, w.L, w.C, w.dtype)
+    wt = W.make_weights(cfg_id, w.L, w.C, w.H, w.n_rbf, w.dtype)
+
+    def dt(a):
+        if a.dtype == np.uint16:
+            return torch.from_numpy(a.view(np.int16).copy()).view(torch.bfloat16).to(dev)
+        return torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+
+    pos, x = dt(w.pos), dt(xs).reshape(w.n_atoms, w.K, w.C)
+    Wq, Wk, Wrad, Wso2 = dt(wt.Wq), dt(wt.Wk), dt(wt.Wrad), dt(wt.Wso2)
+    box = None if w.box is None else [float(b) for b in w.box]
+    gptr = None if w.graph_ptr is None else torch.from_numpy(w.graph_ptr).to(dev)
+    cfg = e2f.make_cfg(w.L, w.C, w.H, w.n_rbf, w.cutoff, w.dtype)
+    tc = bool(e2f.e2f_attention_uses_tensor_cores(cfg))
+    rp, col = e2f.e2f_build_neighbors(pos, box, w.cutoff, gptr)
+    E = int(col.numel())
+    col_buf = torch.empty(E + E // 8 + 1024, dtype=torch.int32, device=dev)
+    out = torch.empty((w.n_atoms, w.K, w.C), dtype=torch.float32, device=dev)
+    ws = torch.empty(e2f.e2f_attention_workspace_size(w.n_atoms, E, cfg), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        rp_, col_ = e2f.e2f_build_neighbors(pos, box, w.cutoff, gptr, col_capacity=col_buf.numel())
+        e2f.e2f_onfly_attention(cfg, pos, box, rp_, col_, x, Wq, Wk, Wrad, Wso2, out=out, workspace=ws, check=False)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    assert e2f.e2f_attention_status(ws) == 0
+    ts = []
+    for _ in range(steps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        step()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        ts.append(a.elapsed_time(b))
+    assert e2f.e2f_attention_status(ws) == 0
+    ms = statistics.mean(ts)
+    F = so2_flops_per_edge(w.L, w.C)
+    tflops = E * F / (ms * 1e-3) / 1e12
+    if tc:
+        peak, bound = float(peaks["bf16_tflops"]), "bf16 tensor (burst, whole step)"
+    else:
+        peak = 148 * 128 * 2 * float(peaks.get("sm_max_mhz", 1965.0)) * 1e6 / 1e12
+        bound = "fp32 FMA pipe (derived, whole step)"
+    # peak activation memory of one call that allocates its own workspace and output
+    del ws
+    torch.cuda.synchronize(dev)
+    torch.cuda.empty_cache()
+    torch.cuda.reset_peak_memory_stats(dev)
+    base = torch.cuda.memory_allocated(dev)
+    o2 = e2f.e2f_onfly_attention(cfg, pos, box, rp, col, x, Wq, Wk, Wrad, Wso2)
+    torch.cuda.synchronize(dev)
+    act = torch.cuda.max_memory_allocated(dev) - base - o2.numel() * 4
+    del o2
+    fixed = int(e2f.e2f_attention_workspace_size(1, 0, cfg))  # per-SM scratch and other size-independent parts
+    return {"workload": workload_desc(w)["workload"], "n_atoms": w.n_atoms, "n_pairs": E,
+            "path": "tcgen05" if tc else "fp32 CUDA cores", "ms_per_step": ms, "pairs_per_s": E / (ms * 1e-3),
+            "tflops": tflops, "frac": tflops / peak, "peak": peak, "peak_note": bound,
+            "peak_activation_bytes": int(act), "activation_mb_per_atom": act / w.n_atoms / 1e6,
+            "fixed_scratch_bytes": fixed, "activation_bytes_per_atom_beyond_fixed": (act - fixed) / w.n_atoms,
+            "csr_bytes": 4 * (w.n_atoms + 1) + 4 * E}
+
+
+def backward_record(cfg_id, dev, steps, peaks):
+    """The attention's backward (all gradients) on one workload: ms, pairs/s, and the
+    SO(2) work 3 E F_so2 (recomputed forward maps, transposed maps, weight gradient)
+    over the time, against the measured bf16 burst peak."""
+    import torch
+
+    import atomistic_cell_list_b200 as e2f
+    import workloads as W
+
+    w = W.load_workload(cfg_id)
+    xs, _ = W.make_features(cfg_id, w.n_atoms, w.L, w.C, w.dtype)
+    wt = W.make_weights(cfg_id, w.L, w.C, w.H, w.n_rbf, w.dtype)
+
+    def dt(a):
+        if a.dtype == np.uint16:
+            return torch.from_numpy(a.view(np.int16).copy()).view(torch.bfloat16).to(dev)
+        return torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+
+    pos, x = dt(w.pos), dt(xs).reshape(w.n_atoms, w.K, w.C)
+    Wq, Wk, Wrad, Wso2 = dt(wt.Wq), dt(wt.Wk), dt(wt.Wrad), dt(wt.Wso2)
+    box = None if w.box is None else [float(b) for b in w.box]
+    gptr = None if w.graph_ptr is None else torch.from_numpy(w.graph_ptr).to(dev)
+    cfg = e2f.make_cfg(w.L, w.C, w.H, w.n_rbf, w.cutoff, w.dtype)
+    rp, col = e2f.e2f_build_neighbors(pos, box, w.cutoff, gptr)
+    E = int(col.numel())
+    G = torch.randn((w.n_atoms, w.K, w.C), generator=torch.Generator().manual_seed(1)).to(dev)
+    ws = torch.empty(e2f.e2f_attention_backward_workspace_size(w.n_atoms, E, cfg), dtype=torch.uint8, device=dev)
+    outs = e2f.e2f_onfly_attention_backward(cfg, pos, box, rp, col, x, Wq, Wk, Wrad, Wso2, G, want_weights=True,
+                                            workspace=ws)
+    torch.cuda.synchronize(dev)
+    ts = []
+    for _ in range(steps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        e2f.e2f_onfly_attention_backward(cfg, pos, box, rp, col, x, Wq, Wk, Wrad, Wso2, G, want_weights=True,
+                                         workspace=ws, out=outs)
+        b.record()
+        torch.cuda.synchronize(dev)
+        ts.append(a.elapsed_time(b))
+    ms = statistics.mean(ts)
+    F = so2_flops_per_edge(w.L, w.C)
+    tflops = 3 * E * F / (ms * 1e-3) / 1e12
+    peak = float(peaks["bf16_tflops"])
+    return {"workload": workload_desc(w)["workload"], "n_pairs": E, "ms": ms, "pairs_per_s": E / (ms * 1e-3),
+            "tflops": tflops, "frac": tflops / peak, "peak": peak,
+            "units": f"{E} edges x 3 x {F} SO(2) FLOP (all gradients)", "steps": steps}
 
 
 def run_naive(args):
@@ -654,6 +787,7 @@ def main():
     ap.add_argument("--config", type=int, default=4)
     ap.add_argument("--impl", choices=["ours", "reference", "naive"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true", help="skip the per-config block and the backward record")
     ap.add_argument("--m-max", type=int, default=-1, help="SO(2) truncation order (-1: full layer)")
     ap.add_argument("--backward", action="store_true", help="time the attention's backward instead")
     args = ap.parse_args()

@@ -201,7 +201,7 @@ e2f_status e2f_onfly_attention(const e2f_attn_cfg* cfg, const float* pos,
                                void* stream);
 
 /* 1 when e2f_onfly_attention runs this shape on the tcgen05 tensor-core
- * kernel (bf16 features, L >= 1, C a multiple of 128 up to 256, H <= 16 and
+ * kernel (bf16 features, L >= 1, C = 64 or a multiple of 128 up to 256, H <= 16 and
  * a multiple of 4), 0 when it runs the fp32 CUDA-core kernel. */
 int e2f_attention_uses_tensor_cores(const e2f_attn_cfg* cfg);
 

@@ -95,7 +95,8 @@ def test_tensor_core_dispatch_rule():
     assert uses(4, 128, 8, 16, 6.0, "bf16")
     assert uses(2, 256, 16, 16, 6.0, "bf16")
     assert not uses(4, 128, 8, 16, 6.0, "f32")      # fp32 features: CUDA-core kernel
-    assert not uses(4, 64, 8, 16, 5.0, "bf16")      # C not a multiple of 128
+    assert uses(4, 64, 8, 16, 5.0, "bf16")          # C = 64: two degrees per 128-row block
+    assert not uses(4, 96, 8, 16, 5.0, "bf16")      # C neither 64 nor a multiple of 128
     assert not uses(2, 16, 1, 16, 5.0, "bf16")
     assert not uses(0, 128, 8, 16, 5.0, "bf16")
     assert not uses(4, 128, 2, 16, 5.0, "bf16")     # H not a multiple of 4

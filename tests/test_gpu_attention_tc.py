@@ -1,7 +1,7 @@
 """Tensor-core (tcgen05) attention against the fp64 oracle on every node of
 small systems: several 128-edge tiles per CTA (grid capped through
 e2f_attention_set_debug), nodes straddling tiles, ragged tails, isolated atoms, and
-the supported shapes (L = 1..4, C = 128 or 256, H = 4..16)."""
+the supported shapes (L = 1..4, C = 64, 128 or 256, H = 4..16)."""
 import numpy as np
 import pytest
 import torch
@@ -65,7 +65,8 @@ def run_case(seed, n, side, cutoff, L, C, H, max_ctas, rel_tol=2e-2, isolate=0):
 
 
 @pytest.mark.parametrize("L,C,H,max_ctas", [(4, 128, 8, 2), (4, 128, 8, 148), (3, 128, 4, 3), (2, 256, 16, 2),
-                                            (1, 128, 8, 1)])
+                                            (1, 128, 8, 1), (4, 64, 8, 2), (3, 64, 4, 3), (2, 64, 8, 1),
+                                            (1, 64, 8, 148)])
 def test_tc_matches_oracle_every_node(L, C, H, max_ctas):
     err, E = run_case(10 + L, 90, 9.6, 4.6, L, C, H, max_ctas)
     assert E > 3 * 128
