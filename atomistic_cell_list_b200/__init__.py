@@ -46,6 +46,8 @@ _SIGS = {
     "e2f_neighbors_workspace_size": (_sz, [_i64, _vp, ctypes.c_float, ctypes.c_int32]),
     "e2f_build_neighbors": (ctypes.c_int, [_vp, _i64, _vp, ctypes.c_float, _vp, ctypes.c_int32, _vp, _vp, _i64,
                                            ctypes.POINTER(_i64), _vp, _sz, _vp]),
+    "e2f_build_neighbors_rows": (ctypes.c_int, [_vp, _i64, _i64, _vp, ctypes.c_float, _vp, ctypes.c_int32, _vp, _vp,
+                                                _i64, ctypes.POINTER(_i64), _vp, _sz, _vp]),
     "e2f_build_neighbors_noalloc": (ctypes.c_int, [_vp, _i64, _vp, ctypes.c_float, _vp, ctypes.c_int32, _vp, _vp,
                                                    _i64, ctypes.POINTER(_i64), _vp]),
     "e2f_attention_workspace_size": (_sz, [_i64, _i64, ctypes.POINTER(e2f_attn_cfg)]),
@@ -134,8 +136,9 @@ def e2f_neighbors_workspace_size(n_atoms: int, box, cutoff: float, n_graphs: int
 
 
 def e2f_build_neighbors(pos: torch.Tensor, box, cutoff: float, graph_ptr: torch.Tensor | None = None,
-                        col_capacity: int | None = None, stream=None):
-    """CSR neighbour list (row_ptr int32 [N+1], col int32 [E]) by the GPU cell list."""
+                        col_capacity: int | None = None, stream=None, rows: int | None = None):
+    """CSR neighbour list (row_ptr int32 [N+1], col int32 [E]) by the GPU cell list; with
+    rows = n, only the rows of atoms 0 .. n-1 (e2f_build_neighbors_rows)."""
     _need_cuda(pos, graph_ptr)
     assert pos.dtype == torch.float32 and pos.dim() == 2 and pos.shape[1] == 3
     n = pos.shape[0]
@@ -149,9 +152,14 @@ def e2f_build_neighbors(pos: torch.Tensor, box, cutoff: float, graph_ptr: torch.
     for _ in range(2):
         col = torch.empty(max(cap, 1), dtype=torch.int32, device=dev)
         npairs = ctypes.c_int64(0)
-        code = lib().e2f_build_neighbors(_ptr(pos), n, b, float(cutoff), _ptr(graph_ptr), n_graphs,
-                                         _ptr(row_ptr), _ptr(col), cap, ctypes.byref(npairs), _ptr(ws), ws_bytes,
-                                         _stream(stream))
+        if rows is None:
+            code = lib().e2f_build_neighbors(_ptr(pos), n, b, float(cutoff), _ptr(graph_ptr), n_graphs,
+                                             _ptr(row_ptr), _ptr(col), cap, ctypes.byref(npairs), _ptr(ws),
+                                             ws_bytes, _stream(stream))
+        else:
+            code = lib().e2f_build_neighbors_rows(_ptr(pos), n, int(rows), b, float(cutoff), _ptr(graph_ptr),
+                                                  n_graphs, _ptr(row_ptr), _ptr(col), cap, ctypes.byref(npairs),
+                                                  _ptr(ws), ws_bytes, _stream(stream))
         if code == 3:  # capacity: grow to the exact size and retry
             cap = int(npairs.value)
             continue

@@ -80,7 +80,7 @@ __global__ void k_scatter(const float* __restrict__ pos, int n, const int32_t* g
 // row ascending at col[row_ptr[i] ...].
 template <int MODE>
 __global__ void __launch_bounds__(32 * kWarpsPerBlock)
-k_pairs(const float* __restrict__ pos, int n, const int32_t* gp, int n_graphs, Grid g, float rc2,
+k_pairs(const float* __restrict__ pos, int n, int nq, const int32_t* gp, int n_graphs, Grid g, float rc2,
         const uint32_t* __restrict__ start, const float4* __restrict__ sorted_pos,
         const int32_t* __restrict__ sorted_idx, int32_t* deg, const int32_t* __restrict__ row_ptr,
         int32_t* col) {
@@ -88,6 +88,10 @@ k_pairs(const float* __restrict__ pos, int n, const int32_t* gp, int n_graphs, G
     const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
     const int i = blockIdx.x * kWarpsPerBlock + wib;
     if (i >= n) return;
+    if (i >= nq) {  // not a query row: an empty row (its atom is still a candidate neighbour)
+        if (MODE == 0 && lane == 0) deg[i] = 0;
+        return;
+    }
     const int gid = graph_id(gp, n_graphs, i);
     const float4 me = make_float4(pos[3 * i], pos[3 * i + 1], pos[3 * i + 2], __int_as_float(gid));
     int row0 = 0, rlen = 0;
@@ -323,14 +327,15 @@ extern "C" size_t e2f_neighbors_workspace_size(int64_t n_atoms, const float* box
     return carve(nullptr, n_atoms, g.n_buckets).bytes;
 }
 
-extern "C" e2f_status e2f_build_neighbors(const float* pos, int64_t n_atoms, const float* box_host,
-                                          float cutoff, const int32_t* graph_ptr, int32_t n_graphs,
-                                          int32_t* row_ptr, int32_t* col, int64_t col_capacity,
-                                          int64_t* n_pairs_host, void* workspace, size_t ws_bytes,
-                                          void* stream_) {
+namespace e2f {
+namespace {
+e2f_status build_neighbors(const float* pos, int64_t n_atoms, int64_t n_rows, const float* box_host, float cutoff,
+                           const int32_t* graph_ptr, int32_t n_graphs, int32_t* row_ptr, int32_t* col,
+                           int64_t col_capacity, int64_t* n_pairs_host, void* workspace, size_t ws_bytes,
+                           void* stream_) {
     cudaStream_t stream = static_cast<cudaStream_t>(stream_);
     if (!n_pairs_host || !row_ptr || n_atoms < 0 || n_atoms > INT32_MAX - 1 || !(cutoff > 0.f) ||
-        !std::isfinite(cutoff) || col_capacity < 0)
+        !std::isfinite(cutoff) || col_capacity < 0 || n_rows < 0 || n_rows > n_atoms)
         return E2F_ERR_INVALID_ARG;
     if (n_atoms > 0 && (!pos || !workspace)) return E2F_ERR_INVALID_ARG;
     if (graph_ptr && n_graphs < 1) return E2F_ERR_INVALID_ARG;
@@ -370,7 +375,7 @@ extern "C" e2f_status e2f_build_neighbors(const float* pos, int64_t n_atoms, con
                                        w.sorted_idx);
     const int wb = (n + kWarpsPerBlock - 1) / kWarpsPerBlock;
     count_launch();
-    k_pairs<0><<<wb, 32 * kWarpsPerBlock, 0, stream>>>(pos, n, graph_ptr, ng, g, rc2, w.count,
+    k_pairs<0><<<wb, 32 * kWarpsPerBlock, 0, stream>>>(pos, n, (int)n_rows, graph_ptr, ng, g, rc2, w.count,
                                                        w.sorted_pos, w.sorted_idx, w.deg, nullptr, nullptr);
     E2F_CUDA_TRY(cudaMemsetAsync(w.deg + n, 0, sizeof(int32_t), stream));
     E2F_CUDA_TRY(exclusive_scan_u32(reinterpret_cast<uint32_t*>(w.deg), reinterpret_cast<uint32_t*>(row_ptr),
@@ -387,9 +392,29 @@ extern "C" e2f_status e2f_build_neighbors(const float* pos, int64_t n_atoms, con
     if (E > col_capacity) return E2F_ERR_CAPACITY;
     if (E > 0) {
         count_launch();
-        k_pairs<1><<<wb, 32 * kWarpsPerBlock, 0, stream>>>(pos, n, graph_ptr, ng, g, rc2, w.count,
+        k_pairs<1><<<wb, 32 * kWarpsPerBlock, 0, stream>>>(pos, n, (int)n_rows, graph_ptr, ng, g, rc2, w.count,
                                                            w.sorted_pos, w.sorted_idx, nullptr, row_ptr, col);
         E2F_CUDA_TRY(cudaGetLastError());
     }
     return E2F_OK;
+}
+}  // namespace
+}  // namespace e2f
+
+extern "C" e2f_status e2f_build_neighbors(const float* pos, int64_t n_atoms, const float* box_host,
+                                          float cutoff, const int32_t* graph_ptr, int32_t n_graphs,
+                                          int32_t* row_ptr, int32_t* col, int64_t col_capacity,
+                                          int64_t* n_pairs_host, void* workspace, size_t ws_bytes,
+                                          void* stream) {
+    return e2f::build_neighbors(pos, n_atoms, n_atoms, box_host, cutoff, graph_ptr, n_graphs, row_ptr, col,
+                                col_capacity, n_pairs_host, workspace, ws_bytes, stream);
+}
+
+extern "C" e2f_status e2f_build_neighbors_rows(const float* pos, int64_t n_atoms, int64_t n_rows,
+                                               const float* box_host, float cutoff, const int32_t* graph_ptr,
+                                               int32_t n_graphs, int32_t* row_ptr, int32_t* col,
+                                               int64_t col_capacity, int64_t* n_pairs_host, void* workspace,
+                                               size_t ws_bytes, void* stream) {
+    return e2f::build_neighbors(pos, n_atoms, n_rows, box_host, cutoff, graph_ptr, n_graphs, row_ptr, col,
+                                col_capacity, n_pairs_host, workspace, ws_bytes, stream);
 }

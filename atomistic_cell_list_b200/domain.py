@@ -92,6 +92,22 @@ class SlabDecomposition:
                 req.wait()
         return torch.cat([x_owned] + [bufs[p] for p in sorted(bufs)], dim=0)
 
+    # -- one step --------------------------------------------------------
+    def step(self, plan, x_owned: torch.Tensor, layer, marks=None):
+        """One layer step of this rank: the halo exchange, then layer(x_local) on the
+        local atoms (owned then halo rows); returns what the layer returns (the owned
+        rows). marks, if given, is called with "start", "exchanged" and "done", so
+        that a caller can time the exchange and the local layer apart."""
+        if marks:
+            marks("start")
+        x_local = self.exchange(plan, x_owned)
+        if marks:
+            marks("exchanged")
+        out = layer(x_local)
+        if marks:
+            marks("done")
+        return out
+
     # -- the layer on this rank's atoms -----------------------------------
     def attention(self, cfg, pos: np.ndarray, x_owned: torch.Tensor, Wq, Wk, Wrad, Wso2, plan=None):
         """out rows of this rank's owned atoms (plan["owned"] order), computed
@@ -100,18 +116,22 @@ class SlabDecomposition:
         x_local = self.exchange(plan, x_owned)
         return self.local_attention(cfg, pos, plan, x_local, Wq, Wk, Wrad, Wso2)
 
-    def local_attention(self, cfg, pos: np.ndarray, plan, x_local: torch.Tensor, Wq, Wk, Wrad, Wso2):
-        """The layer on the local atoms (owned then halo rows of x_local):
-        neighbour list of the local set with the halo rows emptied, then the
-        attention; returns the owned rows."""
+    def local_positions(self, pos: np.ndarray, plan, device) -> torch.Tensor:
+        """Positions of the local atoms (owned then halo), on the device."""
+        return torch.as_tensor(np.asarray(pos, np.float32)[plan["local"]], device=device)
+
+    def local_attention(self, cfg, pos, plan, x_local: torch.Tensor, Wq, Wk, Wrad, Wso2):
+        """The layer on the local atoms (owned then halo rows of x_local): the
+        neighbour rows of the owned atoms only (halo atoms are candidates, their
+        own rows are not searched), then the attention; returns the owned rows.
+        pos: all positions (numpy), or the local positions already on the device."""
         import atomistic_cell_list_b200 as e2f
-        dev = x_local.device
-        p_local = torch.as_tensor(np.asarray(pos, np.float32)[plan["local"]], device=dev)
+        p_local = pos if isinstance(pos, torch.Tensor) else self.local_positions(pos, plan, x_local.device)
         box = [float(b) for b in self.box]
-        rp, col = e2f.e2f_build_neighbors(p_local, box, float(cfg.cutoff))
-        rp, col = owned_rows(rp, col, plan["owned"].size)
+        n_owned = plan["owned"].size
+        rp, col = e2f.e2f_build_neighbors(p_local, box, float(cfg.cutoff), rows=n_owned)
         out = e2f.e2f_onfly_attention(cfg, p_local, box, rp, col, x_local, Wq, Wk, Wrad, Wso2)
-        return out[:plan["owned"].size]
+        return out[:n_owned]
 
 
 def owned_rows(row_ptr: torch.Tensor, col: torch.Tensor, n_owned: int):

@@ -536,25 +536,28 @@ def measure_config(cfg_id, dev, steps, warmup, flush, peaks):
     ws = torch.empty(e2f.e2f_attention_workspace_size(w.n_atoms, E, cfg), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    def step():
+    def step(mid=None):
         rp_, col_ = e2f.e2f_build_neighbors(pos, box, w.cutoff, gptr, col_capacity=col_buf.numel())
+        if mid is not None:
+            mid.record(stream)
         e2f.e2f_onfly_attention(cfg, pos, box, rp_, col_, x, Wq, Wk, Wrad, Wso2, out=out, workspace=ws, check=False)
 
     for _ in range(warmup):
         step()
     torch.cuda.synchronize(dev)
     assert e2f.e2f_attention_status(ws) == 0
-    ts = []
+    ts, tn = [], []
     for _ in range(steps):
         flush.zero_()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a, m, b = (torch.cuda.Event(enable_timing=True) for _ in range(3))
         a.record(stream)
-        step()
+        step(m)
         b.record(stream)
         torch.cuda.synchronize(dev)
         ts.append(a.elapsed_time(b))
+        tn.append(a.elapsed_time(m))
     assert e2f.e2f_attention_status(ws) == 0
-    ms = statistics.mean(ts)
+    ms, ms_n = statistics.mean(ts), statistics.mean(tn)
     F = so2_flops_per_edge(w.L, w.C)
     tflops = E * F / (ms * 1e-3) / 1e12
     if tc:
@@ -575,6 +578,8 @@ def measure_config(cfg_id, dev, steps, warmup, flush, peaks):
     fixed = int(e2f.e2f_attention_workspace_size(1, 0, cfg))  # per-SM scratch and other size-independent parts
     return {"workload": workload_desc(w)["workload"], "n_atoms": w.n_atoms, "n_pairs": E,
             "path": "tcgen05" if tc else "fp32 CUDA cores", "ms_per_step": ms, "pairs_per_s": E / (ms * 1e-3),
+            "ms_neighbors": ms_n, "neighbor_pairs_per_s": E / (ms_n * 1e-3),
+            "attention_pairs_per_s": E / ((ms - ms_n) * 1e-3),
             "tflops": tflops, "frac": tflops / peak, "peak": peak, "peak_note": bound,
             "peak_activation_bytes": int(act), "activation_mb_per_atom": act / w.n_atoms / 1e6,
             "fixed_scratch_bytes": fixed, "activation_bytes_per_atom_beyond_fixed": (act - fixed) / w.n_atoms,
@@ -627,6 +632,101 @@ def backward_record(cfg_id, dev, steps, peaks):
     return {"workload": workload_desc(w)["workload"], "n_pairs": E, "ms": ms, "pairs_per_s": E / (ms * 1e-3),
             "tflops": tflops, "frac": tflops / peak, "peak": peak,
             "units": f"{E} edges x 3 x {F} SO(2) FLOP (all gradients)", "steps": steps}
+
+
+def run_slab(args):
+    """One system over the ranks (--decompose slab): each rank owns a slab of the
+    periodic box, receives its halo rows from the two neighbouring slabs by NCCL
+    point-to-point (batch_isend_irecv), searches the neighbours of its owned atoms
+    and runs the layer on them. The halo exchange and the local layer (neighbour
+    rows + attention) are timed apart with CUDA events; every figure is the maximum
+    over ranks. The total work is one system whatever the rank count (strong
+    scaling); value = all ranks' pairs / the slowest rank's step time."""
+    import torch
+    import torch.distributed as dist
+
+    import atomistic_cell_list_b200 as e2f
+    import workloads as W
+    from atomistic_cell_list_b200.domain import SlabDecomposition
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
+    w = W.load_workload(args.config)
+    if w.box is None or w.graph_ptr is not None:
+        raise SystemExit("--decompose slab needs one periodic system")
+    xs, _ = W.make_features(args.config, w.n_atoms, w.L, w.C, w.dtype)
+    wt = W.make_weights(args.config, w.L, w.C, w.H, w.n_rbf, w.dtype)
+
+    def dt(a):
+        if a.dtype == np.uint16:
+            return torch.from_numpy(a.view(np.int16).copy()).view(torch.bfloat16).to(dev)
+        return torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+
+    x_all = torch.from_numpy(xs.view(np.int16).copy()).view(torch.bfloat16) if xs.dtype == np.uint16 \
+        else torch.from_numpy(np.ascontiguousarray(xs))
+    x_all = x_all.reshape(w.n_atoms, w.K, w.C)
+    Wq, Wk, Wrad, Wso2 = dt(wt.Wq), dt(wt.Wk), dt(wt.Wrad), dt(wt.Wso2)
+    cfg = e2f.make_cfg(w.L, w.C, w.H, w.n_rbf, w.cutoff, w.dtype)
+    dec = SlabDecomposition(w.box, w.cutoff, world, rank)
+    plan = dec.plan(w.pos)
+    x_owned = x_all[torch.as_tensor(plan["owned"])].to(dev)
+    p_local = dec.local_positions(w.pos, plan, dev)
+    stream = torch.cuda.current_stream(dev)
+    n_edges = [0]
+
+    def layer(x_local):
+        box = [float(b) for b in dec.box]
+        rp, col = e2f.e2f_build_neighbors(p_local, box, float(cfg.cutoff), rows=plan["owned"].size)
+        n_edges[0] = int(col.numel())
+        return e2f.e2f_onfly_attention(cfg, p_local, box, rp, col, x_local, Wq, Wk, Wrad, Wso2, check=False)
+
+    for _ in range(args.warmup):
+        dec.step(plan, x_owned, layer)
+    torch.cuda.synchronize(dev)
+    evs = []
+
+    def marks(name):
+        e_ = torch.cuda.Event(enable_timing=True)
+        e_.record(stream)
+        evs[-1][name] = e_
+
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    for _ in range(args.steps):
+        evs.append({})
+        dec.step(plan, x_owned, layer, marks=marks)
+    torch.cuda.synchronize(dev)
+    t_x = sum(e["start"].elapsed_time(e["exchanged"]) for e in evs)
+    t_l = sum(e["exchanged"].elapsed_time(e["done"]) for e in evs)
+    t_s = sum(e["start"].elapsed_time(e["done"]) for e in evs)
+    tot = torch.tensor([t_s, t_x, t_l], dtype=torch.float64, device=dev)
+    edges = torch.tensor([n_edges[0], plan["owned"].size, plan["local"].size - plan["owned"].size],
+                         dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(tot, op=dist.ReduceOp.MAX)
+        dist.all_reduce(edges, op=dist.ReduceOp.SUM)
+    ms_step, ms_x, ms_l = (float(v) / args.steps for v in tot)
+    E = int(edges[0])
+    line = {"metric": METRIC, "value": E / (ms_step * 1e-3), "unit": "pairs/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "strong", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+            "config": {**workload_desc(w), "n_pairs": E, "parallelism": f"slab x{world}"},
+            "decompose": "slab", "ms_halo_exchange": ms_x, "ms_local_layer": ms_l,
+            "halo_atoms": int(edges[2]), "owned_atoms": int(edges[1]),
+            "note": "one system over the ranks: NCCL point-to-point halo exchange, then the neighbour rows of "
+                    "the owned atoms and the attention on owned + halo atoms; times are the maximum over ranks"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
 
 
 def run_naive(args):
@@ -790,6 +890,8 @@ def main():
     ap.add_argument("--no-extra", action="store_true", help="skip the per-config block and the backward record")
     ap.add_argument("--m-max", type=int, default=-1, help="SO(2) truncation order (-1: full layer)")
     ap.add_argument("--backward", action="store_true", help="time the attention's backward instead")
+    ap.add_argument("--decompose", choices=["replicas", "slab"], default="replicas",
+                    help="slab: one system over the ranks with a halo exchange (default: independent replicas)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -799,6 +901,8 @@ def main():
         return run_reference(args)
     if args.impl == "naive":
         return run_naive(args)
+    if args.decompose == "slab":
+        return run_slab(args)
     return run_ours(args)
 
 

@@ -109,6 +109,24 @@ e2f_status e2f_build_neighbors(const float* pos, int64_t n_atoms,
                                void* workspace, size_t ws_bytes,
                                void* stream);
 
+/* The same list for the destination rows 0 .. n_rows-1 only: rows n_rows ..
+ * N-1 are empty (row_ptr constant there), while every atom remains a
+ * candidate neighbour of the query rows. The node-centric layer needs, for
+ * each destination node, only its own neighbours (gist.science Technical
+ * Summary 2.2, Eq. 6), so a rank of a spatial decomposition that holds its
+ * owned atoms first and their halo after needs the rows of its owned atoms
+ * only; searching the halo atoms' rows would be wasted work. Arguments,
+ * outputs, checks and synchronisation as for e2f_build_neighbors;
+ * 0 <= n_rows <= n_atoms (E2F_ERR_INVALID_ARG otherwise). The rows
+ * 0 .. n_rows-1 equal those of e2f_build_neighbors on the same atoms. */
+e2f_status e2f_build_neighbors_rows(const float* pos, int64_t n_atoms,
+                                    int64_t n_rows, const float* box_host,
+                                    float cutoff, const int32_t* graph_ptr,
+                                    int32_t n_graphs, int32_t* row_ptr,
+                                    int32_t* col, int64_t col_capacity,
+                                    int64_t* n_pairs_host, void* workspace,
+                                    size_t ws_bytes, void* stream);
+
 /* ------------------------------------------------------------------------
  * Neighbour list without a caller workspace. The pages have no counterpart
  * of this call: it exists for callers that cannot allocate device memory

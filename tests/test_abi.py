@@ -81,6 +81,9 @@ def test_neighbor_argument_checks():
     assert f(vp(16), 4, None, 5.0, None, 1, vp(16), vp(16), 10, ctypes.byref(n), vp(128), 1 << 20, None) == 4
     assert f(vp(16), 4, None, 5.0, vp(16), 0, vp(16), vp(16), 10, ctypes.byref(n), vp(256), 1 << 20, None) == 1
     assert f(vp(16), 4, None, 5.0, None, 1, vp(16), vp(16), 10, ctypes.byref(n), vp(256), 16, None) == 1
+    g = e2f.lib().e2f_build_neighbors_rows  # query rows outside 0 .. n_atoms
+    assert g(vp(16), 4, 5, None, 5.0, None, 1, vp(16), vp(16), 10, ctypes.byref(n), vp(256), 1 << 20, None) == 1
+    assert g(vp(16), 4, -1, None, 5.0, None, 1, vp(16), vp(16), 10, ctypes.byref(n), vp(256), 1 << 20, None) == 1
 
 
 def test_wigner_entry_checks():

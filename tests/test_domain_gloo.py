@@ -45,9 +45,14 @@ def _rank(rank, world, port, q):
         pos, x, layer = system()
         dec = SlabDecomposition(BOX, RC, world, rank, axis=0)
         plan = dec.plan(pos)
-        x_local = dec.exchange(plan, torch.as_tensor(x[plan["owned"]]))
-        assert np.array_equal(x_local.numpy(), x[plan["local"]])  # the halo rows arrived
-        out = local_oracle(dec, plan, pos, x_local.numpy(), layer)
+        seen_marks = []
+
+        def local_layer(x_local):  # the oracle stands in for the GPU layer (as in the bench's slab mode)
+            assert np.array_equal(x_local.numpy(), x[plan["local"]])  # the halo rows arrived
+            return local_oracle(dec, plan, pos, x_local.numpy(), layer)
+
+        out = dec.step(plan, torch.as_tensor(x[plan["owned"]]), local_layer, marks=seen_marks.append)
+        assert seen_marks == ["start", "exchanged", "done"]
         q.put((rank, plan["owned"], out, {p: v.size for p, v in plan["send"].items()}))
     finally:
         dist.destroy_process_group()

@@ -100,3 +100,19 @@ def test_dense_rows_beyond_the_shared_memory_sort():
     rp0, col0 = neighbors_bruteforce(pos_np, None, 5.0)
     np.testing.assert_array_equal(rp.cpu().numpy(), rp0)
     np.testing.assert_array_equal(col.cpu().numpy(), col0)
+
+
+@pytest.mark.parametrize("cfg", [2, 3])
+def test_query_rows_equal_the_full_list_restricted(cfg):
+    # rows of atoms 0 .. n_rows-1 only: those rows as in the full list (bit-exact, as the
+    # oracle's), every later row empty; all atoms stay candidates
+    d = DeviceInputs(cfg)
+    rp0, col0 = oracle_csr(cfg)
+    n = d.w.n_atoms
+    for n_rows in (0, 1, n // 3, n):
+        rp, col = e2f.e2f_build_neighbors(d.pos, d.box, d.w.cutoff, d.graph_ptr, rows=n_rows)
+        rp, col = rp.cpu().numpy(), col.cpu().numpy()
+        end = rp0[n_rows]
+        np.testing.assert_array_equal(rp[:n_rows + 1], rp0[:n_rows + 1])
+        assert (rp[n_rows:] == end).all()
+        np.testing.assert_array_equal(col, col0[:end])
