@@ -481,17 +481,13 @@ __device__ __forceinline__ uint32_t pack_h2(float a, float b) {
 
 // Epilogue of one accumulator pair (o+ at tacc, o- at tacc + 128) or one
 // accumulator (SIGNS = 1) holding output rows (l3, channel) for the tile's
-// 128 edges, on mma.sync: per 16-edge chunk,
-//     acc[c][m'] += sum_e y+[c][e] D_e[+mu][m'] + y-[c][e] D_e[-mu][m'],
-//     y[c][e] = p_e^{head(c)} o[c][e],
+// 128 edges, on mma.sync: per 16-edge chunk and 8 channels,
+//     acc[m'][c] += sum_e D_e[+mu][m'] y+[e][c] + D_e[-mu][m'] y-[e][c],
+//     y[e][c] = p_e^{head(c)} o[c][e],
 // i.e. the rotate-back D^T of the |m| = mu rows weighted by the softmax and
-// summed over the node's edges. A = y for the warp's 16 channels straight
-// from tcgen05.ld.16x256b (whose thread layout is the m16n8k16 A fragment
-// layout: lanes g, g + 8, edge columns 2q, 2q + 1 and 8 more), B = the Wigner
-// rows m' (N = 8; a second n-tile only when 2 l3 + 1 > 8), built from the
-// staged fp16 pairs, D = fp32 accumulators [channel][m']. Putting the
-// channels on M leaves no M rows idle whatever l3 is, so degrees l3 <= 3
-// take one MMA per chunk and sign instead of two.
+// summed over the node's edges. A = Wigner rows (m' padded to 16, built from
+// the staged fp16 pairs), B = p * o straight from tcgen05.ld.16x256b (whose
+// thread layout is the mma B/D fragment layout), D = fp32 accumulators.
 // Node sums go to out with fire-and-forget reductions at segment ends: one
 // thread owns each (node, l3, m', c) element, so the additions happen in
 // program order. The warp covers 16 TMEM lanes (channels cbase..cbase+15);
@@ -503,73 +499,67 @@ __device__ __noinline__ void epi_mma(uint32_t tacc, int l3, int cbase, int K, in
                                      float* __restrict__ out) {
     const int lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
     const int W3 = 2 * l3 + 1, NP = npair(l3), C8 = C / 8;
-    const bool two = W3 > 8;  // a second n-tile of m' (l3 = 4)
-    float acc[2][4];  // [n-tile][fragment]: (c = g, m' = 2q, 2q+1), (c = g + 8, m' = 2q, 2q+1)
+    float acc[2][4];  // [n-tile lo/hi][fragment]
 #pragma unroll
     for (int b2 = 0; b2 < 2; ++b2)
 #pragma unroll
         for (int r = 0; r < 4; ++r) acc[b2][r] = 0.f;
     int cur = -1;
-    const float* pc = pch + cbase / 8;  // 8-channel groups cbase/8 (rows g) and +1 (rows g + 8)
+    const float* pc = pch + cbase / 8;  // 8-channel groups cbase/8 (lh = 0) and +1 (lh = 1)
 
     auto flush = [&]() {
         if (cur < 0) return;
 #pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
+        for (int lh = 0; lh < 2; ++lh)
 #pragma unroll
             for (int r = 0; r < 4; ++r) {
-                const int mp = 8 * nt + 2 * q + (r & 1);
+                const int mp = g + ((r >> 1) << 3);
                 if (mp < W3) {
-                    const int c = cbase + g + 8 * (r >> 1);
-                    atomicAdd(out + ((size_t)cur * K + l3 * l3 + mp) * C + c, acc[nt][r]);
+                    const int c = cbase + 8 * lh + 2 * q + (r & 1);
+                    atomicAdd(out + ((size_t)cur * K + l3 * l3 + mp) * C + c, acc[lh][r]);
                 }
-                acc[nt][r] = 0.f;
+                acc[lh][r] = 0.f;
             }
     };
 
-    // the staged Wigner fragments and softmax weights of a chunk: shared-memory loads,
-    // issued one chunk ahead so that their latency (long beside the tensor core's
-    // operand reads) overlaps the previous chunk's work
-    auto load_chunk = [&](int ch2, uint32_t (&bf)[SIGNS][2][2], float (&pw)[2][4]) {
-        const int ea = ch2 * 16 + 2 * q, eb = ch2 * 16 + 8 + 2 * q;
-        const bool r0 = g < W3, r1 = two && g + 8 < W3;
-        const __half2 z = __float2half2_rn(0.f);
-        const __half2 p00 = r0 ? Ds[ea * NP + g] : z, p01 = r0 ? Ds[(ea + 1) * NP + g] : z;
-        const __half2 p20 = r0 ? Ds[eb * NP + g] : z, p21 = r0 ? Ds[(eb + 1) * NP + g] : z;
-        const __half2 p10 = r1 ? Ds[ea * NP + g + 8] : z, p11 = r1 ? Ds[(ea + 1) * NP + g + 8] : z;
-        const __half2 p30 = r1 ? Ds[eb * NP + g + 8] : z, p31 = r1 ? Ds[(eb + 1) * NP + g + 8] : z;
-        const __half2 lo[4] = {__lows2half2(p00, p01), __lows2half2(p20, p21), __lows2half2(p10, p11),
-                               __lows2half2(p30, p31)};
+#pragma unroll 1
+    for (int ch = 0; ch < kTileE / 16; ++ch) {
+        const int e0 = ch * 16;
+        // o values: [sign][edge half][4]: (c_lo,e), (c_lo,e+1), (c_hi,e), (c_hi,e+1)
+        uint32_t ov[SIGNS][2][4];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) bf[0][k >> 1][k & 1] = *reinterpret_cast<const uint32_t*>(&lo[k]);
-        if (SIGNS == 2) {
-            const __half2 hi[4] = {__highs2half2(p00, p01), __highs2half2(p20, p21), __highs2half2(p10, p11),
-                                   __highs2half2(p30, p31)};
+        for (int s2 = 0; s2 < SIGNS; ++s2)
 #pragma unroll
-            for (int k = 0; k < 4; ++k) bf[SIGNS - 1][k >> 1][k & 1] = *reinterpret_cast<const uint32_t*>(&hi[k]);
+            for (int eh = 0; eh < 2; ++eh) tmem_ld_16x256(tacc + s2 * 128 + e0 + 8 * eh, ov[s2][eh]);
+        // this thread's four edges: e0 + 2q, +1, e0 + 8 + 2q, +1
+        const int ea = e0 + 2 * q, eb = e0 + 8 + 2 * q;
+        // Wigner A fragments per sign: rows m' = g (a0, a2) and g + 8 (a1, a3)
+        uint32_t af[SIGNS][4];
+        {
+            const bool r0 = g < W3, r1 = g + 8 < W3;
+            const __half2 z = __float2half2_rn(0.f);
+            const __half2 p00 = r0 ? Ds[ea * NP + g] : z, p01 = r0 ? Ds[(ea + 1) * NP + g] : z;
+            const __half2 p10 = r1 ? Ds[ea * NP + g + 8] : z, p11 = r1 ? Ds[(ea + 1) * NP + g + 8] : z;
+            const __half2 p20 = r0 ? Ds[eb * NP + g] : z, p21 = r0 ? Ds[(eb + 1) * NP + g] : z;
+            const __half2 p30 = r1 ? Ds[eb * NP + g + 8] : z, p31 = r1 ? Ds[(eb + 1) * NP + g + 8] : z;
+            const __half2 lo[4] = {__lows2half2(p00, p01), __lows2half2(p10, p11), __lows2half2(p20, p21),
+                                   __lows2half2(p30, p31)};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) af[0][k] = *reinterpret_cast<const uint32_t*>(&lo[k]);
+            if (SIGNS == 2) {
+                const __half2 hi[4] = {__highs2half2(p00, p01), __highs2half2(p10, p11), __highs2half2(p20, p21),
+                                       __highs2half2(p30, p31)};
+#pragma unroll
+                for (int k = 0; k < 4; ++k) af[SIGNS - 1][k] = *reinterpret_cast<const uint32_t*>(&hi[k]);
+            }
         }
+        // softmax weights of the four edges for the two 8-channel groups
         const float2 w0 = *reinterpret_cast<const float2*>(pc + ea * C8);
         const float2 w1 = *reinterpret_cast<const float2*>(pc + (ea + 1) * C8);
         const float2 w2 = *reinterpret_cast<const float2*>(pc + eb * C8);
         const float2 w3 = *reinterpret_cast<const float2*>(pc + (eb + 1) * C8);
-        pw[0][0] = w0.x; pw[0][1] = w1.x; pw[0][2] = w2.x; pw[0][3] = w3.x;
-        pw[1][0] = w0.y; pw[1][1] = w1.y; pw[1][2] = w2.y; pw[1][3] = w3.y;
-    };
-    uint32_t bfr[SIGNS][2][2], bfn[SIGNS][2][2];
-    float pw[2][4], pwn[2][4];
-    // o values: [sign][edge half][4]: (c_lo,e), (c_lo,e+1), (c_hi,e), (c_hi,e+1)
-    uint32_t ov[SIGNS][2][4];
-    load_chunk(0, bfr, pw);
-#pragma unroll
-    for (int s2 = 0; s2 < SIGNS; ++s2)
-#pragma unroll
-        for (int eh = 0; eh < 2; ++eh) tmem_ld_16x256(tacc + s2 * 128 + 8 * eh, ov[s2][eh]);
-    tmem_wait_ld();
-#pragma unroll 1
-    for (int ch = 0; ch < kTileE / 16; ++ch) {
-        const int e0 = ch * 16;
-        const bool more = ch + 1 < kTileE / 16;
-        if (more) load_chunk(ch + 1, bfn, pwn);
+        const float pw[2][4] = {{w0.x, w1.x, w2.x, w3.x}, {w0.y, w1.y, w2.y, w3.y}};
+        tmem_wait_ld();
         // segments of this chunk: bit k = edge e0 + k starts a node
         uint32_t bits = segm[ch];
         int lo = 0;
@@ -586,36 +576,25 @@ __device__ __noinline__ void epi_mma(uint32_t tacc, int l3, int cbase, int K, in
             const float m2 = (8 + 2 * q >= lo && 8 + 2 * q < hi) ? 1.f : 0.f;
             const float m3 = (9 + 2 * q >= lo && 9 + 2 * q < hi) ? 1.f : 0.f;
 #pragma unroll
-            for (int s2 = 0; s2 < SIGNS; ++s2) {
-                const uint32_t* va = ov[s2][0];
-                const uint32_t* vb = ov[s2][1];
-                // A fragment: rows g (channel group 0) and g + 8 (group 1), edges 2q.. and 8 + 2q..
-                uint32_t af[4];
-                af[0] = pack_h2(pw[0][0] * m0 * __uint_as_float(va[0]), pw[0][1] * m1 * __uint_as_float(va[1]));
-                af[1] = pack_h2(pw[1][0] * m0 * __uint_as_float(va[2]), pw[1][1] * m1 * __uint_as_float(va[3]));
-                af[2] = pack_h2(pw[0][2] * m2 * __uint_as_float(vb[0]), pw[0][3] * m3 * __uint_as_float(vb[1]));
-                af[3] = pack_h2(pw[1][2] * m2 * __uint_as_float(vb[2]), pw[1][3] * m3 * __uint_as_float(vb[3]));
-                mma_16816(acc[0], af, bfr[s2][0]);
-                if (two) mma_16816(acc[1], af, bfr[s2][1]);
+            for (int lh = 0; lh < 2; ++lh) {
+                const float* pwv = pw[lh];
+#pragma unroll
+                for (int s2 = 0; s2 < SIGNS; ++s2) {
+                    const uint32_t* va = ov[s2][0];
+                    const uint32_t* vb = ov[s2][1];
+                    uint32_t bf[2];
+                    bf[0] = pack_h2(pwv[0] * m0 * __uint_as_float(va[2 * lh]),
+                                    pwv[1] * m1 * __uint_as_float(va[2 * lh + 1]));
+                    bf[1] = pack_h2(pwv[2] * m2 * __uint_as_float(vb[2 * lh]),
+                                    pwv[3] * m3 * __uint_as_float(vb[2 * lh + 1]));
+                    mma_16816(acc[lh], af[s2], bf);
+                }
             }
             if (hi == 16) break;
             flush();
             cur = nb[e0 + hi];
             lo = hi;
             bits &= bits - 1;
-        }
-        if (more) {
-#pragma unroll
-            for (int s2 = 0; s2 < SIGNS; ++s2)
-#pragma unroll
-                for (int eh = 0; eh < 2; ++eh) tmem_ld_16x256(tacc + s2 * 128 + e0 + 16 + 8 * eh, ov[s2][eh]);
-#pragma unroll
-            for (int s2 = 0; s2 < SIGNS; ++s2)
-#pragma unroll
-                for (int k = 0; k < 4; ++k) bfr[s2][k >> 1][k & 1] = bfn[s2][k >> 1][k & 1];
-#pragma unroll
-            for (int k = 0; k < 8; ++k) pw[k >> 2][k & 3] = pwn[k >> 2][k & 3];
-            tmem_wait_ld();
         }
     }
     flush();
