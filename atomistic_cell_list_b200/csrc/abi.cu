@@ -284,7 +284,7 @@ extern "C" void e2f_attention_set_debug(int max_ctas, int timers, int drop_arriv
 namespace {
 
 struct BwdWs {
-    size_t o_status, o_q, o_k, o_wt, o_lse, o_gq, o_gk, o_beta, o_part, o_w16, bytes;
+    size_t o_status, o_q, o_k, o_wt, o_lse, o_gq, o_gk, o_beta, o_part, o_w16, o_ops, bytes;
 };
 
 BwdWs bwd_layout(int64_t n_atoms, int64_t n_pairs, const e2f_attn_cfg& c) {
@@ -299,8 +299,10 @@ BwdWs bwd_layout(int64_t n_atoms, int64_t n_pairs, const e2f_attn_cfg& c) {
     w.o_gq = take(4 * (size_t)n_atoms * c.C);
     w.o_gk = take(4 * (size_t)n_atoms * c.C);
     w.o_beta = take(4 * (size_t)n_pairs * c.H);
-    w.o_part = take(bwd_partial_bytes(c.L, c.C, effective_mmax(c.L, c.m_max)));
-    w.o_w16 = c.feat_dtype == E2F_BF16 ? take(4 * so2_total(c.L, c.C, effective_mmax(c.L, c.m_max))) : 0;
+    const bool bf = c.feat_dtype == E2F_BF16;
+    w.o_part = bf ? 0 : take(bwd_partial_bytes(c.L, c.C, effective_mmax(c.L, c.m_max)));
+    w.o_w16 = bf ? take(4 * so2_total(c.L, c.C, effective_mmax(c.L, c.m_max))) : 0;
+    w.o_ops = bf ? take(bwd_ops_bytes(n_pairs, c.L, c.C)) : 0;
     w.bytes = o;
     return w;
 }
@@ -324,6 +326,7 @@ extern "C" e2f_status e2f_onfly_attention_backward(const e2f_attn_cfg* cfg, cons
     e2f_status st = check_cfg(cfg);
     if (st != E2F_OK) return st;
     if (!bwd_supported(cfg->L, cfg->C, cfg->H, cfg->n_rbf)) return E2F_ERR_UNSUPPORTED;
+    if (cfg->feat_dtype == E2F_BF16 && cfg->H > 32) return E2F_ERR_UNSUPPORTED;  // weight-gradient operand build
     if (n_atoms < 0 || n_atoms > INT32_MAX || n_pairs < 0 || n_pairs > INT32_MAX) return E2F_ERR_INVALID_ARG;
     if (n_atoms == 0) return E2F_OK;
     if (!pos || !row_ptr || (n_pairs > 0 && !col) || !x || !W_q || !W_k || !W_rad || !W_so2 || !grad_out ||
@@ -367,8 +370,9 @@ extern "C" e2f_status e2f_onfly_attention_backward(const e2f_attn_cfg* cfg, cons
     b.gk = reinterpret_cast<float*>(ws + L.o_gk);
     b.gpos = grad_pos; b.gx = grad_x; b.gWq = grad_W_q; b.gWk = grad_W_k; b.gWrad = grad_W_rad;
     b.gWso2 = grad_W_so2;
-    b.gWpart = reinterpret_cast<float*>(ws + L.o_part);
+    b.gWpart = cfg->feat_dtype == E2F_BF16 ? nullptr : reinterpret_cast<float*>(ws + L.o_part);
     b.w16 = cfg->feat_dtype == E2F_BF16 ? ws + L.o_w16 : nullptr;
+    b.ops = cfg->feat_dtype == E2F_BF16 ? ws + L.o_ops : nullptr;
     b.status = reinterpret_cast<int*>(ws + L.o_status);
     E2F_CUDA_TRY(cudaMemsetAsync(b.status, 0, sizeof(int), stream));
     E2F_CUDA_TRY(run_attention_bwd(b, stream));

@@ -81,10 +81,13 @@ struct BwdArgs {
     float* gWso2;
     float* gWpart;  // bwd_partial_bytes(L, C, M) of scratch for gWso2
     void* w16;      // bf16 storage: 4 so2_total(L, C, M) bytes for fp16 copies of W_so2
+    void* ops;      // bf16 storage: bwd_ops_bytes(...) of scratch for the weight-gradient operands
     int* status;    // device status word (cleared by the caller)
 };
 bool bwd_supported(int L, int C, int H, int n_rbf);
 size_t bwd_partial_bytes(int L, int C, int M);
+// bf16 storage: the per-chunk operand rows of the SO(2) weight gradient
+size_t bwd_ops_bytes(int64_t n_pairs, int L, int C);
 cudaError_t run_attention_bwd(const BwdArgs& b, cudaStream_t s);
 struct CellLists;
 // cl != nullptr: fused traversal (a.row_ptr = per-slot offsets in cell order, a.col unused)

@@ -32,7 +32,13 @@
 #include <cuda_fp16.h>
 #include <stdint.h>
 
+#include <cuda.h>
+#include <cublas_v2.h>
+#include <dlfcn.h>
+
 #include <algorithm>
+#include <map>
+#include <mutex>
 #include <type_traits>
 
 #include "attention.cuh"
@@ -1496,9 +1502,279 @@ cudaError_t launch_dw(const BwdParams& P, int n_tiles, size_t smem, cudaStream_t
 }
 
 
+
+// ---------------------------------------------------------------------------
+// SO(2) weight gradient for bf16 storage as GEMMs over the edges. Per chunk of
+// edges, k_bwd_ops writes each edge's two operand rows in fp16:
+//   X[e][col(l1, m) + c] = g_v(d_e)[l1, c] sum_n D_e^{l1}[l1 + m][n] x_j[l1, n][c]
+//       (the rotated, gated neighbour features the maps act on),
+//   Y[e][col(l3, m) + c] = alpha_e^{head(c)} sum_n D_e^{l3}[l3 + m][n] G_i[l3, n][c]
+//       (the softmax-weighted upstream gradient in the edge frame, dLoss/dY),
+// for m = 0 and m = +-mu (mu <= M), in the packed order of the SO(2) blocks:
+// block mu holds the +mu rows (l - mu) C + c, then the -mu rows (ops_col).
+// The gradient of block mu is then
+//   dA(mu) = sum_e Y+ X+^T + Y- X-^T,   dB(mu) = sum_e Y- X+^T - Y+ X-^T
+// (dA(0) = sum_e Y0 X0^T): plain GEMMs over the chunk's edges (K = edges),
+// which cuBLAS runs with fp32 accumulation into the output, chunk after chunk
+// (a fixed order, so the result is deterministic). Each operand is built once
+// per edge instead of once per weight tile.
+constexpr int kOpsChunk = 32768;  // edges per chunk
+constexpr int kOpsE = 32;         // edges per CTA of k_bwd_ops
+constexpr int kOpsNt = 256;
+constexpr int kOpsMaxH = 32;
+
+__host__ __device__ inline int ops_col(int l, int m, int L, int C) {
+    const int mu = m < 0 ? -m : m;
+    if (mu == 0) return l * C;
+    int off = (L + 1) * C;
+    for (int k = 1; k < mu; ++k) off += 2 * (L + 1 - k) * C;
+    const int nm = (L + 1 - mu) * C;
+    return off + (m > 0 ? 0 : nm) + (l - mu) * C;
+}
+
+template <int L>
+__global__ void __launch_bounds__(kOpsNt, 2) k_bwd_ops(BwdParams P, int e0, int ne, __half* __restrict__ Xo,
+                                                      __half* __restrict__ Yo) {
+    constexpr int K = n_sh(L), WS = wig_size(L);
+    const int C = P.C, H = P.H, dh = C / H, nr = P.n_rbf, M = P.M;
+    const int Gv = (L + 1) * C, G = Gv + H;
+    const size_t KC = (size_t)K * C;
+    const __nv_bfloat16* __restrict__ x = static_cast<const __nv_bfloat16*>(P.x);
+    __shared__ float Ds[kOpsE][WS];
+    __shared__ float rho[kOpsE][kURbf];
+    __shared__ float alpha[kOpsE][kOpsMaxH];
+    __shared__ int ei[kOpsE], ej[kOpsE];
+    const int tid = threadIdx.x;
+    const int eb = blockIdx.x * kOpsE;  // first edge of this CTA within the chunk
+    const int nb = min(kOpsE, ne - eb);
+    if (tid < nb) {
+        const int e = e0 + eb + tid;
+        int lo = 0, hi = P.n_atoms - 1;  // node: last n with row_ptr[n] <= e
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (P.row_ptr[mid] <= e) lo = mid; else hi = mid - 1;
+        }
+        const int i = lo, j = P.col[e];
+        const float3 r = edge_vec(P.pos, i, j, P.box);
+        const float d = sqrtf(r.x * r.x + r.y * r.y + r.z * r.z);
+        float R[3][3];
+        edge_frame(r.x / d, r.y / d, r.z / d, R);
+        float D[WS];
+        wigner_blocks<L>(R, D);
+        for (int k2 = 0; k2 < WS; ++k2) Ds[tid][k2] = D[k2];
+        float rr[kURbf];
+        rbf_all<kURbf>(d, P.cutoff, nr, rr);
+        for (int kb = 0; kb < kURbf; ++kb) rho[tid][kb] = rr[kb];
+        const float inv = rsqrtf((float)dh);
+        for (int h = 0; h < H; ++h) {
+            float ga = 0.f;
+            for (int kb = 0; kb < nr; ++kb) ga = fmaf(rr[kb], P.Wrad[(size_t)kb * G + Gv + h], ga);
+            const float* qi = P.q + (size_t)i * C + h * dh;
+            const float* kj = P.k + (size_t)j * C + h * dh;
+            float dot = 0.f;
+            for (int c = 0; c < dh; ++c) dot = fmaf(qi[c], kj[c], dot);
+            alpha[tid][h] = expf(ga * dot * inv - P.lse[(size_t)i * H + h]);
+        }
+        ei[tid] = i;
+        ej[tid] = j;
+    }
+    __syncthreads();
+    const int CG = C / 8;
+    for (int it = tid; it < nb * CG; it += kOpsNt) {
+        const int el = it / CG, c0 = (it % CG) * 8;
+        const int i = ei[el], j = ej[el];
+        __half* xrow = Xo + (size_t)(eb + el) * KC;
+        __half* yrow = Yo + (size_t)(eb + el) * KC;
+        float al[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) al[q] = alpha[el][(c0 + q) / dh];
+#pragma unroll
+        for (int l = 0; l <= L; ++l) {
+            constexpr int kW = 2 * L + 1;
+            const int w = 2 * l + 1;
+            const float* Dl = &Ds[el][wig_off(l)];
+            // value gate of the 8 channels of degree l
+            float gv[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) gv[q] = 0.f;
+            for (int kb = 0; kb < nr; ++kb) {
+                const float rk = rho[el][kb];
+                const float* wr = P.Wrad + (size_t)kb * G + l * C + c0;  // rows of (L+1)C + H: no vector alignment
+#pragma unroll
+                for (int q = 0; q < 8; ++q) gv[q] = fmaf(rk, __ldg(wr + q), gv[q]);
+            }
+            // X: rows (l, n) of x_j for these channels, rotated and gated
+            {
+                float xv[kW][8];
+#pragma unroll
+                for (int n = 0; n < kW; ++n) {
+                    if (n < w) {
+                        const uint4 u = *reinterpret_cast<const uint4*>(x + ((size_t)j * K + l * l + n) * C + c0);
+                        const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            const float2 f = __bfloat1622float2(b2[q]);
+                            xv[n][2 * q] = f.x;
+                            xv[n][2 * q + 1] = f.y;
+                        }
+                    }
+                }
+#pragma unroll
+                for (int mu = 0; mu <= L; ++mu) {
+                    if (mu > l || mu > M) continue;
+#pragma unroll
+                    for (int sg = 0; sg < 2; ++sg) {
+                        if (mu == 0 && sg == 1) continue;
+                        const int m = sg == 0 ? mu : -mu;
+                        const float* Dr = Dl + (l + m) * w;  // D^l[l + m][n]
+                        float o[8];
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) o[q] = 0.f;
+#pragma unroll
+                        for (int n = 0; n < kW; ++n) {
+                            if (n < w) {
+                                const float dv = Dr[n];
+#pragma unroll
+                                for (int q = 0; q < 8; ++q) o[q] = fmaf(dv, xv[n][q], o[q]);
+                            }
+                        }
+                        __align__(16) __half hx[8];
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) hx[q] = __float2half_rn(gv[q] * o[q]);
+                        *reinterpret_cast<uint4*>(xrow + ops_col(l, m, L, C) + c0) = *reinterpret_cast<const uint4*>(hx);
+                    }
+                }
+            }
+            // Y: rows (l, n) of G_i for these channels, rotated and weighted by the softmax
+            {
+                float gg[kW][8];
+#pragma unroll
+                for (int n = 0; n < kW; ++n) {
+                    if (n < w) {
+                        const float4* gp = reinterpret_cast<const float4*>(P.G + ((size_t)i * K + l * l + n) * C + c0);
+                        const float4 ga = gp[0], gb = gp[1];
+                        gg[n][0] = ga.x; gg[n][1] = ga.y; gg[n][2] = ga.z; gg[n][3] = ga.w;
+                        gg[n][4] = gb.x; gg[n][5] = gb.y; gg[n][6] = gb.z; gg[n][7] = gb.w;
+                    }
+                }
+#pragma unroll
+                for (int mu = 0; mu <= L; ++mu) {
+                    if (mu > l || mu > M) continue;
+#pragma unroll
+                    for (int sg = 0; sg < 2; ++sg) {
+                        if (mu == 0 && sg == 1) continue;
+                        const int m = sg == 0 ? mu : -mu;
+                        const float* Dr = Dl + (l + m) * w;
+                        float o[8];
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) o[q] = 0.f;
+#pragma unroll
+                        for (int n = 0; n < kW; ++n) {
+                            if (n < w) {
+                                const float dv = Dr[n];
+#pragma unroll
+                                for (int q = 0; q < 8; ++q) o[q] = fmaf(dv, gg[n][q], o[q]);
+                            }
+                        }
+                        __align__(16) __half hy[8];
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) hy[q] = __float2half_rn(al[q] * o[q]);
+                        *reinterpret_cast<uint4*>(yrow + ops_col(l, m, L, C) + c0) = *reinterpret_cast<const uint4*>(hy);
+                    }
+                }
+            }
+        }
+    }
+}
+
+template <int L>
+cudaError_t launch_ops(const BwdParams& P, int e0, int ne, __half* Xo, __half* Yo, cudaStream_t s) {
+    count_launch();
+    k_bwd_ops<L><<<(ne + kOpsE - 1) / kOpsE, kOpsNt, 0, s>>>(P, e0, ne, Xo, Yo);
+    return cudaGetLastError();
+}
+
+// cuBLAS, loaded at run time (the library links no BLAS; the host process
+// normally has it loaded already). One handle per CUDA context, found by the
+// context's unique id, so a handle is never used in another context.
+struct CublasRt {
+    decltype(&cublasCreate_v2) create = nullptr;
+    decltype(&cublasSetStream_v2) set_stream = nullptr;
+    cublasStatus_t (*gemm)(cublasHandle_t, cublasOperation_t, cublasOperation_t, int, int, int, const void*,
+                           const void*, cudaDataType, int, const void*, cudaDataType, int, const void*, void*,
+                           cudaDataType, int, cublasComputeType_t, cublasGemmAlgo_t) = nullptr;
+    bool ok = false;
+};
+CublasRt& cublas_rt() {
+    static CublasRt rt;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        const char* names[] = {"libcublas.so.12", "/usr/local/cuda/lib64/libcublas.so.12", "libcublas.so"};
+        void* h = nullptr;
+        for (const char* n : names) {
+            h = dlopen(n, RTLD_NOW | RTLD_GLOBAL);
+            if (h) break;
+        }
+        if (!h) return;
+        rt.create = reinterpret_cast<decltype(rt.create)>(dlsym(h, "cublasCreate_v2"));
+        rt.set_stream = reinterpret_cast<decltype(rt.set_stream)>(dlsym(h, "cublasSetStream_v2"));
+        rt.gemm = reinterpret_cast<decltype(rt.gemm)>(dlsym(h, "cublasGemmEx"));
+        rt.ok = rt.create && rt.set_stream && rt.gemm;
+    });
+    return rt;
+}
+cublasHandle_t cublas_handle() {
+    CublasRt& rt = cublas_rt();
+    if (!rt.ok) return nullptr;
+    // driver entry points through the runtime (the library does not link the driver)
+    using GetCurrentFn = CUresult (*)(CUcontext*);
+    using GetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+    static GetCurrentFn get_current = nullptr;
+    static GetIdFn get_id = nullptr;
+    if (!get_current || !get_id) {
+        void* p1 = nullptr;
+        void* p2 = nullptr;
+        cudaDriverEntryPointQueryResult q1, q2;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p1, cudaEnableDefault, &q1) != cudaSuccess ||
+            q1 != cudaDriverEntryPointSuccess ||
+            cudaGetDriverEntryPoint("cuCtxGetId", &p2, cudaEnableDefault, &q2) != cudaSuccess ||
+            q2 != cudaDriverEntryPointSuccess)
+            return nullptr;
+        get_current = reinterpret_cast<GetCurrentFn>(p1);
+        get_id = reinterpret_cast<GetIdFn>(p2);
+    }
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (get_current(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS) return nullptr;
+    static std::mutex mu;
+    static std::map<unsigned long long, cublasHandle_t> handles;
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = handles.find(id);
+    if (it != handles.end()) return it->second;
+    cublasHandle_t h = nullptr;
+    if (rt.create(&h) != CUBLAS_STATUS_SUCCESS) return nullptr;
+    handles[id] = h;
+    return h;
+}
+
+// out (nm x nm, row-major [f][k]) += alpha sum_e Y[e][f] X[e][k] over ne edges; X, Y point at
+// the block's columns of rows of KC halves
+cublasStatus_t gemm_edges(cublasHandle_t h, int nm, int ne, size_t KC, const __half* X, const __half* Y,
+                          float alpha, float* out) {
+    const float beta = 1.f;
+    // column-major view: out^T (k x f) = X^T (k x e) * Y (e x f)
+    return cublas_rt().gemm(h, CUBLAS_OP_N, CUBLAS_OP_T, nm, nm, ne, &alpha, X, CUDA_R_16F, (int)KC, Y, CUDA_R_16F,
+                            (int)KC, &beta, out, CUDA_R_32F, nm, CUBLAS_COMPUTE_32F, CUBLAS_GEMM_DEFAULT);
+}
+
 }  // namespace bwd
 
 size_t bwd_partial_bytes(int L, int C, int M) { return 4 * bwd::dw_part_floats(L, C, M); }
+
+size_t bwd_ops_bytes(int64_t n_pairs, int L, int C) {
+    const int64_t ec = std::min<int64_t>(std::max<int64_t>(n_pairs, 1), bwd::kOpsChunk);
+    return 2 * (size_t)ec * (size_t)n_sh(L) * C * 2;
+}
 
 bool bwd_supported(int L, int C, int H, int n_rbf) {
     if (L < 0 || L > kMaxL || bwd::kNt % H != 0 || bwd::kNodeNt % H != 0) return false;
@@ -1570,7 +1846,45 @@ cudaError_t run_attention_bwd(const BwdArgs& b, cudaStream_t s) {
     count_launch();
     k_bwd_x0<<<(N * C + 255) / 256, 256, 0, s>>>(N, K, C, a.Wq, a.Wk, b.gq, b.gk, b.gx);
     E2F_CUDA_TRY_E(cudaGetLastError());
-    if (b.gWso2 && a.n_pairs > 0) {
+    if (b.gWso2 && a.n_pairs > 0 && a.bf16) {
+        // operand rows per chunk of edges, then the block GEMMs over the chunk (cuBLAS)
+        if (C % 8 != 0 || H > kOpsMaxH || a.n_rbf > kURbf || !b.ops) return cudaErrorInvalidValue;
+        cublasHandle_t h = cublas_handle();
+        if (!h) return cudaErrorNotSupported;
+        if (cublas_rt().set_stream(h, s) != CUBLAS_STATUS_SUCCESS) return cudaErrorNotSupported;
+        E2F_CUDA_TRY_E(cudaMemsetAsync(b.gWso2, 0, 4 * so2_total(L, C, a.M), s));
+        const size_t KC = (size_t)K * C;
+        __half* Xo = static_cast<__half*>(b.ops);
+        __half* Yo = Xo + (size_t)std::min<int64_t>(a.n_pairs, kOpsChunk) * KC;
+        for (int64_t c0 = 0; c0 < a.n_pairs; c0 += kOpsChunk) {
+            const int nc = (int)std::min<int64_t>(kOpsChunk, a.n_pairs - c0);
+            switch (L) {
+                case 0: e = launch_ops<0>(P, (int)c0, nc, Xo, Yo, s); break;
+                case 1: e = launch_ops<1>(P, (int)c0, nc, Xo, Yo, s); break;
+                case 2: e = launch_ops<2>(P, (int)c0, nc, Xo, Yo, s); break;
+                case 3: e = launch_ops<3>(P, (int)c0, nc, Xo, Yo, s); break;
+                case 4: e = launch_ops<4>(P, (int)c0, nc, Xo, Yo, s); break;
+                default: return cudaErrorInvalidValue;
+            }
+            if (e != cudaSuccess) return e;
+            for (int mu = 0; mu <= a.M; ++mu) {
+                const int nm = (L + 1 - mu) * C;
+                float* dA = b.gWso2 + so2_offset(L, C, mu, 0);
+                const int cp = ops_col(mu, mu, L, C), cm = ops_col(mu, -mu, L, C);
+                cublasStatus_t cs;
+                if (mu == 0) {
+                    cs = gemm_edges(h, nm, nc, KC, Xo + cp, Yo + cp, 1.f, dA);
+                } else {
+                    float* dB = b.gWso2 + so2_offset(L, C, mu, 1);
+                    cs = gemm_edges(h, nm, nc, KC, Xo + cp, Yo + cp, 1.f, dA);  // Y+ X+^T
+                    if (cs == CUBLAS_STATUS_SUCCESS) cs = gemm_edges(h, nm, nc, KC, Xo + cm, Yo + cm, 1.f, dA);
+                    if (cs == CUBLAS_STATUS_SUCCESS) cs = gemm_edges(h, nm, nc, KC, Xo + cp, Yo + cm, 1.f, dB);
+                    if (cs == CUBLAS_STATUS_SUCCESS) cs = gemm_edges(h, nm, nc, KC, Xo + cm, Yo + cp, -1.f, dB);
+                }
+                if (cs != CUBLAS_STATUS_SUCCESS) return cudaErrorUnknown;
+            }
+        }
+    } else if (b.gWso2 && a.n_pairs > 0) {
         const int nt = P.dw_tiles * kDwSplit;
         const size_t dsm = a.bf16 ? dw_umma_smem_bytes(H, a.n_rbf) : dw_smem_bytes(H, a.n_rbf);
 #define E2F_BWD_DW(LL)                                                                                         \

@@ -369,21 +369,30 @@ e2f_status e2f_onfly_attention_cells_skin(const e2f_attn_cfg* cfg,
  *               NULL (not computed).
  *   grad_W_rad  device, float [n_rbf, (L+1)C + H], written.
  *   grad_W_so2  device, float, packed like W_so2 (truncation included),
- *               written; NULL skips it (its kernel is the costliest part:
- *               a sweep over all edges per 64 x 64 tile of the SO(2) blocks).
+ *               written; NULL skips it. With fp32 storage its kernel sweeps
+ *               all edges per 64 x 64 tile of the SO(2) blocks. With bf16
+ *               storage each edge's two operand rows (the rotated, gated
+ *               features and the softmax-weighted rotated upstream
+ *               gradient) are built once per chunk of 32,768 edges in the
+ *               workspace, and each block's gradient is a GEMM over the
+ *               chunk's edges, run by cuBLAS (loaded at run time; absent
+ *               cuBLAS gives E2F_ERR_CUDA).
  *   workspace   device, >= e2f_attention_backward_workspace_size(...)
  *               bytes, 256-byte aligned. Its status word (a bounded
  *               device-side wait that ran out: E2F_ERR_TIMEOUT) is read
  *               with e2f_attention_status, as for the forward.
  * Arithmetic: with fp32 storage, fp32 on CUDA cores throughout. With bf16
- * storage, the SO(2) maps, their transposes and the SO(2) weight-gradient
- * contraction run on tensor cores (mma.sync) with fp16 operands and fp32
- * accumulation (about 3e-4 relative error against an exact evaluation);
+ * storage, the SO(2) maps and their transposes run on tensor cores
+ * (mma.sync), and the SO(2) weight-gradient GEMMs on cuBLAS; all take fp16
+ * operands with fp32 accumulation (about 3e-4 relative error against an
+ * exact evaluation);
  * the rest stays fp32. Gradients that sum over edges use fp32 atomics, so
  * their last bits may differ between runs; grad_W_so2, grad_W_q and
- * grad_W_k are deterministic. Shapes: those of e2f_onfly_attention with H dividing 256
- * and the kernels' shared memory within 227 KB (L = 4 allows C <= 128);
- * otherwise E2F_ERR_UNSUPPORTED. Asynchronous.
+ * grad_W_k are deterministic (the weight-gradient GEMMs run chunk after
+ * chunk into the output). Shapes: those of e2f_onfly_attention with H
+ * dividing 256 (at most 32 heads with bf16 storage) and the kernels' shared
+ * memory within 227 KB (L = 4 allows C <= 128); otherwise
+ * E2F_ERR_UNSUPPORTED. Asynchronous.
  * ---------------------------------------------------------------------- */
 size_t e2f_attention_backward_workspace_size(int64_t n_atoms, int64_t n_pairs,
                                              const e2f_attn_cfg* cfg);
