@@ -1,7 +1,8 @@
 // Backward of the on-the-fly equivariant attention. fp32 CUDA cores; with
-// bf16 storage the SO(2) maps, their transposes and the weight-gradient
-// contraction run on tensor cores (m16n8k16 mma.sync, fp16 operands, fp32
-// accumulation).
+// bf16 storage the SO(2) maps and their transposes run on tensor cores
+// (m16n8k16 mma.sync, fp16 operands, fp32 accumulation), and the SO(2)
+// weight gradient is a GEMM over edges on operand rows built once per edge
+// chunk (cuBLAS, fp16 operands, fp32 accumulation).
 //
 // The pages' conservative variant takes forces as the negative gradient of
 // the energy with respect to the positions (E2Former-V2, gist.science
@@ -10,14 +11,15 @@
 // this file computes dLoss / d(pos, x, W_q, W_k, W_rad, W_so2) in the same
 // recompute style as the forward: per-edge quantities (frame, Wigner blocks,
 // gates, rotated features, SO(2) outputs) are rebuilt on chip and never
-// stored per edge; the only O(E) scratch is one scalar per edge and head.
+// stored per edge, except for one scalar per edge and head and, with bf16
+// storage, the weight gradient's operand rows of one chunk of edges.
 //
 // Per edge e = (i <- j) with alpha = softmax weight, X~ = D(g_v . x_j),
 // Y = F(X~) (the SO(2) maps), v = D^T Y, out_i = sum_e alpha v:
 //   beta^h   = sum_{c in h} <D G_i, Y>                 (= <G_i, v> per head)
 //   dY       = alpha D G_i,   dX~ = F^T(dY)
 //   dx_j    += g_v . D^T dX~,  dg_v = sum_m x_j . D^T dX~
-//   dW_so2   = sum_e dY (x) X~   (A and B blocks; a separate tile kernel)
+//   dW_so2   = sum_e dY (x) X~   (A and B blocks; a tile kernel, or GEMMs over edges)
 //   da^h     = alpha^h (beta^h - delta_i^h),  delta_i^h = sum_e alpha beta
 //   logits a = g_a <q_i, k_j>/sqrt(d): dq_i, dk_j, dg_a
 //   gates    [g_v | g_a] = rho(d) W_rad: dW_rad, dd through rho'(d)
@@ -1045,363 +1047,7 @@ __global__ void __launch_bounds__(kNt, 2) k_bwd_dw(BwdParams P) {
     }
 }
 
-// ---------------------------------------------------------------------------
-// dW_so2 on tcgen05 (bf16 storage): one 128 x 256 tile (rows x columns) of one
-// |m| block per CTA, both the A and B gradients accumulated in TMEM (2 x 256
-// fp32 columns), over one of kDwSplit edge ranges. Per sub-chunk of 32 edges
-// the threads rebuild the fp16 operands (dY rows, X~ columns; as in k_bwd_dw)
-// into one of two shared buffers in the canonical no-swizzle K-major layout
-// (core matrices of 8 rows x 16 bytes, 128 bytes apart along K and 512 bytes
-// apart along rows), and one thread issues M128 N256 K16 MMAs:
-//   dA += Y+ X+^T + Y- X-^T,   dB += Y- X+^T - Y+ X-^T   (K = edges)
-// committing to the buffer's mbarrier, which the threads wait on (bounded)
-// before refilling it.
-// ---------------------------------------------------------------------------
-constexpr int kUR = 128, kUC = 256, kUE = 32, kUChunk = 128;
-constexpr int kURow = 12;   // a Wigner row (2l+1 <= 9 entries) padded to three float4
-constexpr int kUDr = 120;   // floats per edge: rows (l+m), (l-m) for l = m..L, padded
-constexpr int kURbf = 32;   // radial basis per edge, padded (n_rbf <= 32)
-
-// padded Wigner rows of one edge: (l+m) and (l-m) for l = m..L, kURow floats each
-__device__ __forceinline__ int drow_off_p(int m, int l, int s) {
-    const int nrow = (m == 0) ? 1 : 2;
-    return ((l - m) * nrow + s) * kURow;
-}
-
-int n_dw_tiles_umma(int L, int C, int M) {
-    int n = 0;
-    for (int m = 0; m <= M; ++m) {
-        const int nm = (L + 1 - m) * C;
-        n += ((nm + kUR - 1) / kUR) * ((nm + kUC - 1) / kUC);
-    }
-    return n;
-}
-
-size_t dw_umma_smem_bytes(int H, int n_rbf) {
-    (void)n_rbf;
-    return 4 * ((size_t)kUChunk * kUDr + (size_t)kUChunk * kURbf + (size_t)kUChunk * H + 2 * kUChunk) +
-           2 * 2 * 2 * (size_t)(kUR + kUC) * kUE  // [buffer][sign] fp16 operands
-           + 64;                                  // mbarriers, TMEM address, abort flag
-}
-
-// element (row r, k) of a rows x 32 K-major fp16 operand in core-matrix order
-__device__ __forceinline__ int core_off(int r, int k) { return ((r >> 3) * 4 + (k >> 3)) * 64 + (r & 7) * 8 + (k & 7); }
-
-__device__ __forceinline__ uint64_t sdesc_none(uint32_t saddr) {
-    uint64_t d = 0;
-    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
-    d |= (uint64_t)(128u >> 4) << 16;   // leading byte offset: next core matrix along K
-    d |= (uint64_t)(512u >> 4) << 32;   // stride byte offset: next 8-row group
-    d |= (uint64_t)1u << 46;            // descriptor version (sm_100)
-    return d;                           // swizzle: none
-}
-
-// kind::f16: D fp32, A and B fp16, both K-major, M = 128, N = 256, optional negation of A
-__host__ __device__ constexpr uint32_t idesc_m128n256(bool neg_a) {
-    return (1u << 4) | ((neg_a ? 1u : 0u) << 13) | ((256u >> 3) << 17) | ((128u >> 4) << 24);
-}
-
-template <int L>
-__global__ void __launch_bounds__(kNt, 1) k_bwd_dw_umma(BwdParams P) {
-    using namespace tc;
-    constexpr int K = n_sh(L);
-    constexpr int WS = wig_size(L);
-    const int C = P.C, H = P.H, dh = C / H, nr = P.n_rbf;
-    const int Gv = (L + 1) * C, G = Gv + H;
-    const __nv_bfloat16* __restrict__ x = static_cast<const __nv_bfloat16*>(P.x);
-    const int split = blockIdx.x / P.dw_tiles;
-    int m = 0, nm = (L + 1) * C, b = blockIdx.x % P.dw_tiles;
-    int sr = (nm + kUR - 1) / kUR, sc = (nm + kUC - 1) / kUC;
-    while (b >= sr * sc && m < P.M) {
-        b -= sr * sc;
-        ++m;
-        nm = (L + 1 - m) * C;
-        sr = (nm + kUR - 1) / kUR;
-        sc = (nm + kUC - 1) / kUC;
-    }
-    const int r0 = (b / sc) * kUR, k0 = (b % sc) * kUC;
-    const int nrow = (m == 0) ? 1 : 2;
-
-    extern __shared__ __align__(1024) float sm[];
-    float* drow = sm;                          // [chunk][kUDr] padded Wigner rows
-    float* rho = drow + kUChunk * kUDr;        // [chunk][kURbf] radial basis, zero-padded
-    float* alpha = rho + kUChunk * kURbf;      // [chunk][H]
-    int* ei = reinterpret_cast<int*>(alpha + kUChunk * H);
-    int* ej = ei + kUChunk;
-    __half* ops = reinterpret_cast<__half*>(ej + kUChunk);
-    // Ys(buf, sign): kUR x kUE halves; Xs(buf, sign): kUC x kUE halves
-    auto Ys = [&](int bf, int sg) { return ops + (size_t)(bf * 2 + sg) * kUR * kUE; };
-    auto Xs = [&](int bf, int sg) { return ops + (size_t)4 * kUR * kUE + (size_t)(bf * 2 + sg) * kUC * kUE; };
-    uint64_t* bars = reinterpret_cast<uint64_t*>(ops + (size_t)4 * (kUR + kUC) * kUE);  // [2] buffers, [2] final
-    uint32_t* tmem_sm = reinterpret_cast<uint32_t*>(bars + 3);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 4);
-
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const float inv = rsqrtf((float)dh);
-    if (tid == 0) {
-        mbar_init(bars + 0, 1);
-        mbar_init(bars + 1, 1);
-        mbar_init(bars + 2, 1);
-        *abort_flag = 0;
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    }
-    if (warp == 0) {
-        tmem_alloc(tmem_sm, 512);
-        tmem_relinquish();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = *tmem_sm;
-
-    // operand roles: dY row y_q (both signs) over half of the sub-chunk's edges (y_half);
-    // X~ column x_q (both signs) over all of them. The signs share their loads of G_i
-    // and x_j, the softmax weight and the value gate.
-    const int y_q = tid % kUR, y_half = tid / kUR, ry = r0 + y_q;
-    const bool y_ok = ry < nm;
-    const int y_l = m + (y_ok ? ry / C : 0), y_c = y_ok ? ry % C : 0;
-    const int y_g = y_l * y_l * C + y_c, y_w = 2 * y_l + 1;
-    const int y_d0 = y_ok ? drow_off_p(m, y_l, 0) : 0, y_d1 = (y_ok && m > 0) ? drow_off_p(m, y_l, 1) : 0;
-    const int y_h = y_c / dh;
-    const int x_q = tid, kxx = k0 + x_q;
-    const bool x_ok = kxx < nm;
-    const int x_l = m + (x_ok ? kxx / C : 0), x_c = x_ok ? kxx % C : 0;
-    const int x_g = x_l * x_l * C + x_c, x_w = 2 * x_l + 1;
-    const int x_d0 = x_ok ? drow_off_p(m, x_l, 0) : 0, x_d1 = (x_ok && m > 0) ? drow_off_p(m, x_l, 1) : 0;
-    float wreg[kURbf];  // this column's W_rad entries (value gate), zero beyond n_rbf
-#pragma unroll
-    for (int kb = 0; kb < kURbf; ++kb)
-        wreg[kb] = (x_ok && kb < nr) ? P.Wrad[(size_t)kb * G + x_l * C + x_c] : 0.f;
-    static_assert(2 * kUR == kNt && kUC == kNt && kUE % 16 == 0, "operand roles");
-
-    const int e_lo = (int)((long long)P.n_pairs * split / kDwSplit);
-    const int e_hi = (int)((long long)P.n_pairs * (split + 1) / kDwSplit);
-    int u = 0;           // sub-chunks issued
-    bool ok = true;
-    for (int c0 = e_lo; c0 < e_hi && ok; c0 += kUChunk) {
-        const int nc = min(kUChunk, e_hi - c0);
-        __syncthreads();
-        if (tid < nc) {
-            const int e = c0 + tid;
-            int lo = 0, hi = P.n_atoms - 1;
-            while (lo < hi) {
-                const int mid = (lo + hi + 1) >> 1;
-                if (P.row_ptr[mid] <= e) lo = mid; else hi = mid - 1;
-            }
-            const int i = lo, j = P.col[e];
-            ei[tid] = i;
-            ej[tid] = j;
-            const float3 r = edge_vec(P.pos, i, j, P.box);
-            const float d = sqrtf(r.x * r.x + r.y * r.y + r.z * r.z);
-            float R[3][3];
-            edge_frame(r.x / d, r.y / d, r.z / d, R);
-            float D[WS];
-            wigner_blocks<L>(R, D);
-            float* dr = drow + tid * kUDr;
-            for (int l = m; l <= L; ++l) {
-                const int w = 2 * l + 1;
-                for (int s2 = 0; s2 < nrow; ++s2) {
-                    const int row = s2 == 0 ? l + m : l - m;
-                    float* o = dr + drow_off_p(m, l, s2);
-                    for (int n = 0; n < kURow; ++n) o[n] = (n < w) ? D[wig_off(l) + row * w + n] : 0.f;
-                }
-            }
-            for (int kb = 0; kb < kURbf; ++kb) rho[tid * kURbf + kb] = (kb < nr) ? rbf(d, kb, P.cutoff, nr) : 0.f;
-            for (int h = 0; h < H; ++h) {
-                float ga = 0.f;
-                for (int kb = 0; kb < nr; ++kb) ga = fmaf(rho[tid * kURbf + kb], P.Wrad[(size_t)kb * G + Gv + h], ga);
-                const float* qi = P.q + (size_t)i * C + h * dh;
-                const float* kj = P.k + (size_t)j * C + h * dh;
-                float dot = 0.f;
-                for (int c = 0; c < dh; ++c) dot = fmaf(qi[c], kj[c], dot);
-                alpha[tid * H + h] = expf(ga * dot * inv - P.lse[(size_t)i * H + h]);
-            }
-        }
-        __syncthreads();
-        for (int s0 = 0; s0 < nc; s0 += kUE, ++u) {
-            const int ns = min(kUE, nc - s0);
-            const int bf = u & 1;
-            // the MMAs that read this buffer two sub-chunks ago have completed
-            bool mine = true;
-            if (u >= 2) {
-                const uint32_t par = (uint32_t)(((u >> 1) & 1) ^ 1);
-                if (!mbar_try(bars + bf, par)) {
-                    const uint64_t t0 = gtimer();
-                    while (!mbar_try(bars + bf, par)) {
-                        if (*abort_flag) { mine = false; break; }
-                        if (gtimer() - t0 > kWaitNs) {
-                            *abort_flag = 1;
-                            atomicExch(P.status, (int)E2F_ERR_TIMEOUT);
-                            mine = false;
-                            break;
-                        }
-                    }
-                }
-            }
-            if (!__syncthreads_and(mine)) { ok = false; break; }
-            // dY row of this thread, both signs, edges 16 y_half .. 16 y_half + 15
-            {
-                int cached = -1;
-                float gr[2 * L + 1];
-#pragma unroll
-                for (int n = 0; n < 2 * L + 1; ++n) gr[n] = 0.f;
-                for (int kg = 2 * y_half; kg < 2 * y_half + 2; ++kg) {
-                    __half hp[8], hm[8];
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        const int e = kg * 8 + q;
-                        float vp = 0.f, vm = 0.f;
-                        if (e < ns && y_ok) {
-                            const int el = s0 + e, node = ei[el];
-                            if (node != cached) {
-                                const float* gi = P.G + (size_t)node * K * C + y_g;
-#pragma unroll
-                                for (int n = 0; n < 2 * L + 1; ++n) gr[n] = (n < y_w) ? gi[(size_t)n * C] : 0.f;
-                                cached = node;
-                            }
-                            float d0[kURow], d1[kURow];
-                            const float4* r0v = reinterpret_cast<const float4*>(drow + el * kUDr + y_d0);
-                            const float4* r1v = reinterpret_cast<const float4*>(drow + el * kUDr + y_d1);
-#pragma unroll
-                            for (int v4 = 0; v4 < kURow / 4; ++v4) {
-                                *reinterpret_cast<float4*>(d0 + 4 * v4) = r0v[v4];
-                                *reinterpret_cast<float4*>(d1 + 4 * v4) = r1v[v4];
-                            }
-                            float ap = 0.f, am = 0.f;
-#pragma unroll
-                            for (int n = 0; n < 2 * L + 1; ++n) {
-                                ap = fmaf(d0[n], gr[n], ap);
-                                am = fmaf(d1[n], gr[n], am);
-                            }
-                            const float al = alpha[el * H + y_h];
-                            vp = al * ap;
-                            vm = al * am;
-                        }
-                        hp[q] = __float2half_rn(vp);
-                        hm[q] = __float2half_rn(vm);
-                    }
-                    *reinterpret_cast<uint4*>(Ys(bf, 0) + core_off(y_q, kg * 8)) = *reinterpret_cast<const uint4*>(hp);
-                    if (nrow == 2)
-                        *reinterpret_cast<uint4*>(Ys(bf, 1) + core_off(y_q, kg * 8)) = *reinterpret_cast<const uint4*>(hm);
-                }
-            }
-            // X~ column of this thread, both signs, all edges of the sub-chunk
-            for (int kg = 0; kg < kUE / 8; ++kg) {
-                __half hp[8], hm[8];
-#pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    const int e = kg * 8 + q;
-                    float vp = 0.f, vm = 0.f;
-                    if (e < ns && x_ok) {
-                        const int el = s0 + e;
-                        const size_t xb = (size_t)ej[el] * K * C + x_g;
-                        float xr[2 * L + 1];
-#pragma unroll
-                        for (int n = 0; n < 2 * L + 1; ++n)
-                            xr[n] = (n < x_w) ? __bfloat162float(x[xb + (size_t)n * C]) : 0.f;
-                        float d0[kURow], d1[kURow];
-                        const float4* r0v = reinterpret_cast<const float4*>(drow + el * kUDr + x_d0);
-                        const float4* r1v = reinterpret_cast<const float4*>(drow + el * kUDr + x_d1);
-#pragma unroll
-                        for (int v4 = 0; v4 < kURow / 4; ++v4) {
-                            *reinterpret_cast<float4*>(d0 + 4 * v4) = r0v[v4];
-                            *reinterpret_cast<float4*>(d1 + 4 * v4) = r1v[v4];
-                        }
-                        float ap = 0.f, am = 0.f;
-#pragma unroll
-                        for (int n = 0; n < 2 * L + 1; ++n) {
-                            ap = fmaf(d0[n], xr[n], ap);
-                            am = fmaf(d1[n], xr[n], am);
-                        }
-                        const float4* rv = reinterpret_cast<const float4*>(rho + el * kURbf);
-                        float gv = 0.f;
-#pragma unroll
-                        for (int v4 = 0; v4 < kURbf / 4; ++v4) {
-                            const float4 q4 = rv[v4];
-                            gv = fmaf(q4.x, wreg[4 * v4 + 0], gv);
-                            gv = fmaf(q4.y, wreg[4 * v4 + 1], gv);
-                            gv = fmaf(q4.z, wreg[4 * v4 + 2], gv);
-                            gv = fmaf(q4.w, wreg[4 * v4 + 3], gv);
-                        }
-                        vp = gv * ap;
-                        vm = gv * am;
-                    }
-                    hp[q] = __float2half_rn(vp);
-                    hm[q] = __float2half_rn(vm);
-                }
-                *reinterpret_cast<uint4*>(Xs(bf, 0) + core_off(x_q, kg * 8)) = *reinterpret_cast<const uint4*>(hp);
-                if (nrow == 2)
-                    *reinterpret_cast<uint4*>(Xs(bf, 1) + core_off(x_q, kg * 8)) = *reinterpret_cast<const uint4*>(hm);
-            }
-            // make the generic-proxy stores visible to the tensor cores, then issue
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            __syncthreads();
-            if (tid == 0) {
-                tc_fence_after();
-                constexpr uint32_t ID = idesc_m128n256(false), IDN = idesc_m128n256(true);
-#pragma unroll
-                for (int ks = 0; ks < kUE / 16; ++ks) {
-                    const uint32_t kb = (uint32_t)ks * 256u;  // two core matrices along K
-                    const uint64_t yp = sdesc_none(smem_u32(Ys(bf, 0)) + kb), xp = sdesc_none(smem_u32(Xs(bf, 0)) + kb);
-                    const uint32_t first = (u == 0 && ks == 0) ? 0u : 1u;
-                    umma(tmem, yp, xp, ID, first);
-                    if (nrow == 2) {
-                        const uint64_t ym = sdesc_none(smem_u32(Ys(bf, 1)) + kb), xm = sdesc_none(smem_u32(Xs(bf, 1)) + kb);
-                        umma(tmem, ym, xm, ID, 1u);
-                        umma(tmem + 256, ym, xp, ID, first);
-                        umma(tmem + 256, yp, xm, IDN, 1u);
-                    }
-                }
-                umma_commit(bars + bf);
-            }
-        }
-    }
-    // drain: every issued MMA completes (bounded) before TMEM is read and released
-    if (tid == 0 && u > 0) umma_commit(bars + 2);
-    bool fin = true;
-    if (u > 0) {
-        const uint64_t t0 = gtimer();
-        while (!mbar_try(bars + 2, 0)) {
-            if (gtimer() - t0 > kWaitNs) {
-                atomicExch(P.status, (int)E2F_ERR_TIMEOUT);
-                fin = false;
-                break;
-            }
-        }
-    }
-    fin = __syncthreads_and(fin && ok);
-    tc_fence_after();
-    const size_t oa = so2_offset(L, C, m, 0), ob = so2_offset(L, C, m, 1);
-    float* dst = P.gWpart + (size_t)split * so2_total(L, C, P.M);
-    {
-        const int q4 = warp & 3, half = warp >> 2;  // TMEM lanes 32 q4.. (rows), columns 128 half..
-        const int r = r0 + 32 * q4 + lane;
-        for (int acc = 0; acc < nrow; ++acc) {
-            for (int c32 = 0; c32 < 4; ++c32) {
-                const int col = 128 * half + 32 * c32;
-                float v[32];
-                if (fin && u > 0) {
-                    tmem_ld32(tmem + ((uint32_t)(32 * q4) << 16) + (uint32_t)(256 * acc + col), v);
-                    tmem_wait_ld();
-                } else {
-#pragma unroll
-                    for (int q = 0; q < 32; ++q) v[q] = 0.f;
-                }
-                if (r < nm) {
-                    float* out = dst + (acc == 0 ? oa : ob) + (size_t)r * nm;
-#pragma unroll
-                    for (int q = 0; q < 32; ++q) {
-                        const int kx = k0 + col + q;
-                        if (kx < nm) out[kx] = v[q];
-                    }
-                }
-            }
-        }
-    }
-    tc_fence_before();
-    __syncthreads();
-    if (warp == 0) tmem_dealloc(tmem, 512);
-}
+constexpr int kURbf = 32;  // radial basis per edge, padded (n_rbf <= 32)
 
 // Position of element (r, k) of an n x n block (n a multiple of 16) in fragment
 // order: 16 x 16 tiles row-major, and within a tile the 8 halves that lane
@@ -1483,15 +1129,6 @@ cudaError_t launch_node(const BwdParams& P, size_t smem, int grid, cudaStream_t 
     return cudaGetLastError();
 }
 
-template <int L>
-cudaError_t launch_dw_umma(const BwdParams& P, int n_tiles, size_t smem, cudaStream_t s) {
-    cudaError_t e = cudaFuncSetAttribute(k_bwd_dw_umma<L>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    count_launch();
-    k_bwd_dw_umma<L><<<n_tiles, kNt, smem, s>>>(P);
-    return cudaGetLastError();
-}
-
 template <int L, typename T>
 cudaError_t launch_dw(const BwdParams& P, int n_tiles, size_t smem, cudaStream_t s) {
     cudaError_t e = cudaFuncSetAttribute(k_bwd_dw<L, T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -1518,7 +1155,7 @@ cudaError_t launch_dw(const BwdParams& P, int n_tiles, size_t smem, cudaStream_t
 // which cuBLAS runs with fp32 accumulation into the output, chunk after chunk
 // (a fixed order, so the result is deterministic). Each operand is built once
 // per edge instead of once per weight tile.
-constexpr int kOpsChunk = 32768;  // edges per chunk
+constexpr int kOpsChunk = 131072;  // edges per chunk
 constexpr int kOpsE = 32;         // edges per CTA of k_bwd_ops
 constexpr int kOpsNt = 256;
 constexpr int kOpsMaxH = 32;
@@ -1779,7 +1416,7 @@ size_t bwd_ops_bytes(int64_t n_pairs, int L, int C) {
 bool bwd_supported(int L, int C, int H, int n_rbf) {
     if (L < 0 || L > kMaxL || bwd::kNt % H != 0 || bwd::kNodeNt % H != 0) return false;
     return bwd::node_smem_floats(L, C, H, n_rbf, true) * 4 <= 227 * 1024 &&
-           bwd::dw_smem_bytes(H, n_rbf) <= 227 * 1024 && bwd::dw_umma_smem_bytes(H, n_rbf) <= 227 * 1024;
+           bwd::dw_smem_bytes(H, n_rbf) <= 227 * 1024;
 }
 
 cudaError_t run_attention_bwd(const BwdArgs& b, cudaStream_t s) {
@@ -1802,7 +1439,7 @@ cudaError_t run_attention_bwd(const BwdArgs& b, cudaStream_t s) {
     P.lse = b.lse; P.beta = b.beta; P.gq = b.gq; P.gk = b.gk; P.gpos = b.gpos; P.gx = b.gx; P.gWrad = b.gWrad;
     P.gW = b.gWso2;
     P.gWpart = b.gWpart;
-    P.dw_tiles = a.bf16 ? n_dw_tiles_umma(L, C, a.M) : n_dw_tiles(L, C, a.M);
+    P.dw_tiles = n_dw_tiles(L, C, a.M);
     P.status = b.status;
 
     int dev = 0, n_sm = 148;
@@ -1886,10 +1523,10 @@ cudaError_t run_attention_bwd(const BwdArgs& b, cudaStream_t s) {
         }
     } else if (b.gWso2 && a.n_pairs > 0) {
         const int nt = P.dw_tiles * kDwSplit;
-        const size_t dsm = a.bf16 ? dw_umma_smem_bytes(H, a.n_rbf) : dw_smem_bytes(H, a.n_rbf);
+        const size_t dsm = dw_smem_bytes(H, a.n_rbf);
 #define E2F_BWD_DW(LL)                                                                                         \
     case LL:                                                                                                   \
-        e = a.bf16 ? launch_dw_umma<LL>(P, nt, dsm, s) : launch_dw<LL, float>(P, nt, dsm, s);               \
+        e = launch_dw<LL, float>(P, nt, dsm, s);                                                           \
         break;
         switch (L) {
             E2F_BWD_DW(0)

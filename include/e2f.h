@@ -373,7 +373,7 @@ e2f_status e2f_onfly_attention_cells_skin(const e2f_attn_cfg* cfg,
  *               all edges per 64 x 64 tile of the SO(2) blocks. With bf16
  *               storage each edge's two operand rows (the rotated, gated
  *               features and the softmax-weighted rotated upstream
- *               gradient) are built once per chunk of 32,768 edges in the
+ *               gradient) are built once per chunk of 131,072 edges in the
  *               workspace, and each block's gradient is a GEMM over the
  *               chunk's edges, run by cuBLAS (loaded at run time; absent
  *               cuBLAS gives E2F_ERR_CUDA).

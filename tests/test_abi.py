@@ -120,12 +120,12 @@ def test_backward_workspace_and_argument_checks():
     bf = e2f.make_cfg(4, 128, 8, 16, 6.0, "bf16")
     f32 = e2f.make_cfg(4, 128, 8, 16, 6.0, "f32")
     # an edge adds one float per head; with bf16 storage it also adds its two fp16 operand rows of the
-    # weight gradient ((L+1)^2 C halves each), up to a chunk of 32768 edges, beyond which only the floats grow
+    # weight gradient ((L+1)^2 C halves each), up to a chunk of 131072 edges, beyond which only the floats grow
     ws = e2f.e2f_attention_backward_workspace_size
     assert ws(100, 1000, bf) > 0 and ws(100, 1000, f32) > 0
     assert ws(100, 2000, f32) - ws(100, 1000, f32) >= 4 * 8 * 1000
     assert ws(100, 2000, bf) - ws(100, 1000, bf) >= 4 * 8 * 1000 + 2 * 2 * 25 * 128 * 1000
-    assert ws(100, 200000, bf) - ws(100, 100000, bf) < 4 * 8 * 100000 + 4096
+    assert ws(100, 400000, bf) - ws(100, 200000, bf) < 4 * 8 * 200000 + 4096
     assert e2f.e2f_attention_backward_workspace_size(100, 1000, e2f.make_cfg(5, 128, 8, 16, 6.0, "bf16")) == 0
     cfg = e2f.make_cfg(2, 16, 1, 16, 5.0, "f32")
     assert _bwd(cfg, gout=None) == 1
