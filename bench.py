@@ -807,9 +807,10 @@ def run_naive(args):
 def run_backward(args):
     """The attention's backward (e2f_onfly_attention_backward) on the bench workload: all
     gradients (positions, features, every weight), and positions + features + W_rad only
-    (what forces need). With bf16 storage the contractions run on tensor cores (mma.sync);
-    the per-edge rebuild of their operands (rotations, gates) on the FP32 pipe bounds the
-    kernels, so the roofline reported is the FP32 FMA pipe's."""
+    (what forces need). With bf16 storage the maps run on tensor cores (mma.sync) and the
+    SO(2) weight gradient as GEMMs over edge chunks (cuBLAS); the node kernel's per-edge
+    CUDA-core work (rotations, gates, reductions) bounds the call, so the roofline reported
+    is the FP32 FMA pipe's."""
     import torch
 
     import atomistic_cell_list_b200 as e2f
