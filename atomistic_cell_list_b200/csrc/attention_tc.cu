@@ -75,6 +75,41 @@ __host__ __device__ constexpr uint32_t idesc_f16(bool neg_a) {
 // ----------------------------------------------------------------------------
 // pre-passes
 // ----------------------------------------------------------------------------
+// Logit a = g_a <q_i, k_j> / sqrt(dh) of edge (i, j) for this lane's head.
+__device__ __forceinline__ float stats_logit(const StatsParams& P, int i, int j, const float* wcol,
+                                             const float4* q4, int d4, int h, int dh, float inv) {
+    const float3 r = edge_vec(P.pos, i, j, P.box);
+    const float d = sqrtf(r.x * r.x + r.y * r.y + r.z * r.z);
+    float rr[kTcMaxRbf];
+    rbf_all<kTcMaxRbf>(d, P.cutoff, P.n_rbf, rr);
+    float ga = 0.f;
+#pragma unroll
+    for (int kb = 0; kb < kTcMaxRbf; ++kb) ga = fmaf(rr[kb], wcol[kb], ga);
+    const float4* k4 = reinterpret_cast<const float4*>(P.k + (size_t)j * P.C + h * dh);
+    float dot = 0.f;
+    for (int c4 = 0; c4 < d4; ++c4) {
+        const float4 qa = __ldg(q4 + c4), kv = __ldg(k4 + c4);
+        dot = fmaf(qa.x, kv.x, dot);
+        dot = fmaf(qa.y, kv.y, dot);
+        dot = fmaf(qa.z, kv.z, dot);
+        dot = fmaf(qa.w, kv.w, dot);
+    }
+    return ga * dot * inv;
+}
+// Logits of a lane are evaluated kStatsB at a time, independently (so that their
+// gathers overlap), and merged into the running (max, sum) once per batch.
+constexpr int kStatsB = 4;
+__device__ __forceinline__ void stats_merge(const float (&a)[kStatsB], float& m, float& s) {
+    float mb = m;
+#pragma unroll
+    for (int u = 0; u < kStatsB; ++u) mb = fmaxf(mb, a[u]);
+    if (mb == -INFINITY) return;  // no edge yet
+    float sb = (m == -INFINITY) ? 0.f : s * expf(m - mb);
+#pragma unroll
+    for (int u = 0; u < kStatsB; ++u) sb += (a[u] == -INFINITY) ? 0.f : expf(a[u] - mb);
+    m = mb;
+    s = sb;
+}
 // Softmax statistics per node and head, lse = m + log(sum exp(a - m)), by an
 // online max/sum over the node's edges. One warp per node; lane = (edge slot
 // es, head h) with 32 / H edge slots, so a head's q and logit-gate column
@@ -95,28 +130,14 @@ __global__ void __launch_bounds__(256) k_softmax_stats(StatsParams P) {
     const int d4 = dh / 4;
     float m = -INFINITY, s = 0.f;
     const int e0 = P.row_ptr[i], e1 = P.row_ptr[i + 1];
-    for (int e = e0 + es; e < e1; e += EP) {
-        const int j = P.col[e];
-        const float3 r = edge_vec(P.pos, i, j, P.box);
-        const float d = sqrtf(r.x * r.x + r.y * r.y + r.z * r.z);
-        float rr[kTcMaxRbf];
-        rbf_all<kTcMaxRbf>(d, P.cutoff, P.n_rbf, rr);
-        float ga = 0.f;
+    for (int eb = e0 + es; eb < e1; eb += EP * kStatsB) {
+        float a[kStatsB];
 #pragma unroll
-        for (int kb = 0; kb < kTcMaxRbf; ++kb) ga = fmaf(rr[kb], wcol[kb], ga);
-        const float4* k4 = reinterpret_cast<const float4*>(P.k + (size_t)j * C + h * dh);
-        float dot = 0.f;
-        for (int c4 = 0; c4 < d4; ++c4) {
-            const float4 qa = __ldg(q4 + c4), kv = __ldg(k4 + c4);
-            dot = fmaf(qa.x, kv.x, dot);
-            dot = fmaf(qa.y, kv.y, dot);
-            dot = fmaf(qa.z, kv.z, dot);
-            dot = fmaf(qa.w, kv.w, dot);
+        for (int u = 0; u < kStatsB; ++u) {
+            const int e = eb + u * EP;
+            a[u] = e < e1 ? stats_logit(P, i, P.col[e], wcol, q4, d4, h, dh, inv) : -INFINITY;
         }
-        const float a = ga * dot * inv;
-        const float mn = fmaxf(m, a);
-        s = s * expf(m - mn) + expf(a - mn);
-        m = mn;
+        stats_merge(a, m, s);
     }
     // combine the edge slots of each head
     for (int o = H; o < 32; o <<= 1) {
@@ -163,28 +184,14 @@ __global__ void __launch_bounds__(256) k_softmax_stats_cells(StatsParams P, Cell
             0, s);
         __syncwarp();
         const int n_here = min(cnt - w0, kStatsCap);
-        for (int k = es; k < n_here; k += EP) {
-            const int j = jb[k];
-            const float3 r = edge_vec(P.pos, i, j, P.box);
-            const float d = sqrtf(r.x * r.x + r.y * r.y + r.z * r.z);
-            float rr[kTcMaxRbf];
-            rbf_all<kTcMaxRbf>(d, P.cutoff, P.n_rbf, rr);
-            float ga = 0.f;
+        for (int kb0 = es; kb0 < n_here; kb0 += EP * kStatsB) {
+            float a[kStatsB];
 #pragma unroll
-            for (int kb = 0; kb < kTcMaxRbf; ++kb) ga = fmaf(rr[kb], wcol[kb], ga);
-            const float4* k4 = reinterpret_cast<const float4*>(P.k + (size_t)j * C + h * dh);
-            float dot = 0.f;
-            for (int c4 = 0; c4 < d4; ++c4) {
-                const float4 qa = __ldg(q4 + c4), kv = __ldg(k4 + c4);
-                dot = fmaf(qa.x, kv.x, dot);
-                dot = fmaf(qa.y, kv.y, dot);
-                dot = fmaf(qa.z, kv.z, dot);
-                dot = fmaf(qa.w, kv.w, dot);
+            for (int u = 0; u < kStatsB; ++u) {
+                const int k = kb0 + u * EP;
+                a[u] = k < n_here ? stats_logit(P, i, jb[k], wcol, q4, d4, h, dh, inv) : -INFINITY;
             }
-            const float a = ga * dot * inv;
-            const float mn = fmaxf(m, a);
-            sum = sum * expf(m - mn) + expf(a - mn);
-            m = mn;
+            stats_merge(a, m, sum);
         }
         __syncwarp();
         if (cnt <= w0 + kStatsCap) break;
@@ -222,35 +229,60 @@ __global__ void k_partition(const int32_t* row_ptr, int n_atoms, int n_ctas, int
     part[k] = lo;
 }
 
-// Q/K projection, 32 nodes per CTA, weights staged in shared memory in blocks
-// of 64 output channels.
-constexpr int kQkRows = 64;
+// Q/K projection (Eq. 6): q = W_q x[l=0], k = W_k x[l=0], as one [N x C] x [C x 2C]
+// product on the FP32 pipe. A CTA computes 64 nodes x 64 outputs (outputs
+// o < C are q, the rest k); K = C runs in chunks of 32 through shared memory:
+// the features node-major (row stride 33: conflict-free stores of coalesced
+// reads), the weights k-major (a thread reads its 4 outputs of a k step as one
+// float4). Each of the 256 threads accumulates a 4 x 4 block.
+constexpr int kQkM = 64, kQkN = 64, kQkK = 32;
 __global__ void __launch_bounds__(256) k_qk_tiled(const __nv_bfloat16* __restrict__ x, int n_atoms, int K, int C,
                                                    const float* __restrict__ Wq, const float* __restrict__ Wk,
                                                    float* q, float* k) {
-    extern __shared__ float sm[];
-    float* xs = sm;                // [32][C]
-    float* ws = xs + 32 * C;       // [kQkRows][C+1]
-    const int n0 = blockIdx.x * 32;
-    for (int t = threadIdx.x; t < 32 * C; t += blockDim.x) {
-        const int a = t / C, c = t % C;
-        xs[t] = (n0 + a < n_atoms) ? __bfloat162float(x[(size_t)(n0 + a) * K * C + c]) : 0.f;
-    }
-    for (int which = 0; which < 2; ++which) {
-        const float* W = which ? Wk : Wq;
-        float* dst = which ? k : q;
-        for (int r0 = 0; r0 < C; r0 += kQkRows) {
-            const int nr = min(kQkRows, C - r0);
-            __syncthreads();
-            for (int t = threadIdx.x; t < nr * C; t += blockDim.x)
-                ws[(t / C) * (C + 1) + t % C] = W[(size_t)(r0 + t / C) * C + t % C];
-            __syncthreads();
-            for (int t = threadIdx.x; t < 32 * nr; t += blockDim.x) {
-                const int a = t / nr, c = t % nr;
-                float s = 0.f;
-                for (int c2 = 0; c2 < C; ++c2) s = fmaf(ws[c * (C + 1) + c2], xs[a * C + c2], s);
-                if (n0 + a < n_atoms) dst[(size_t)(n0 + a) * C + r0 + c] = s;
+    __shared__ float xs[kQkM][kQkK + 1];
+    __shared__ __align__(16) float ws[kQkK][kQkN];
+    const int tid = threadIdx.x, tx = tid % 16, ty = tid / 16;
+    const int n0 = blockIdx.x * kQkM, o0 = blockIdx.y * kQkN;
+    float acc[4][4];
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) acc[a][b] = 0.f;
+    for (int c0 = 0; c0 < C; c0 += kQkK) {
+        __syncthreads();
+        for (int t = tid; t < kQkM * kQkK; t += 256) {
+            const int a = t / kQkK, kk = t % kQkK;  // consecutive threads: consecutive channels of a node
+            const int n = n0 + a;
+            xs[a][kk] = n < n_atoms ? __bfloat162float(x[(size_t)n * K * C + c0 + kk]) : 0.f;
+        }
+        for (int t = tid; t < kQkN * kQkK; t += 256) {
+            const int o = t % kQkN, kk = t / kQkN;  // consecutive threads: consecutive outputs
+            const int og = o0 + o;
+            const float* W = og < C ? Wq + (size_t)og * C : Wk + (size_t)(og - C) * C;
+            ws[kk][o] = og < 2 * C ? W[c0 + kk] : 0.f;
+        }
+        __syncthreads();
+#pragma unroll 8
+        for (int kk = 0; kk < kQkK; ++kk) {
+            const float4 wb = *reinterpret_cast<const float4*>(&ws[kk][4 * tx]);
+            const float wv[4] = {wb.x, wb.y, wb.z, wb.w};
+#pragma unroll
+            for (int a = 0; a < 4; ++a) {
+                const float xv = xs[4 * ty + a][kk];
+#pragma unroll
+                for (int b = 0; b < 4; ++b) acc[a][b] = fmaf(xv, wv[b], acc[a][b]);
             }
+        }
+    }
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+        const int n = n0 + 4 * ty + a;
+        if (n >= n_atoms) continue;
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+            const int og = o0 + 4 * tx + b;
+            if (og < C) q[(size_t)n * C + og] = acc[a][b];
+            else if (og < 2 * C) k[(size_t)n * C + og - C] = acc[a][b];
         }
     }
 }
@@ -1428,12 +1460,9 @@ cudaError_t run_attention_tc(const AttnArgs& a, void* tc_ws, cudaStream_t s, con
     tc::k_wrad_t<<<(Gv * kTcMaxRbf + 255) / 256, 256, 0, s>>>(a.Wrad, a.n_rbf, G, Gv, whT);
 
     // pre-passes: Q/K, softmax statistics, partition, zeroed output
-    const size_t qk_smem = (32 * C + tc::kQkRows * (C + 1)) * 4;
-    e = cudaFuncSetAttribute(tc::k_qk_tiled, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)qk_smem);
-    if (e != cudaSuccess) return e;
     count_launch();
-    tc::k_qk_tiled<<<(N + 31) / 32, 256, qk_smem, s>>>(static_cast<const __nv_bfloat16*>(a.x), N, K, C, a.Wq, a.Wk,
-                                                       a.q, a.k);
+    tc::k_qk_tiled<<<dim3((N + tc::kQkM - 1) / tc::kQkM, (2 * C + tc::kQkN - 1) / tc::kQkN), 256, 0, s>>>(
+        static_cast<const __nv_bfloat16*>(a.x), N, K, C, a.Wq, a.Wk, a.q, a.k);
     StatsParams sp{};
     sp.n_atoms = N; sp.C = C; sp.H = H; sp.n_rbf = a.n_rbf; sp.G = (L + 1) * C + H; sp.cutoff = a.cutoff;
     sp.box = a.box; sp.pos = a.pos; sp.row_ptr = a.row_ptr; sp.col = a.col; sp.q = a.q; sp.k = a.k;
