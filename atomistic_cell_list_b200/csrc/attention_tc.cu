@@ -75,41 +75,6 @@ __host__ __device__ constexpr uint32_t idesc_f16(bool neg_a) {
 // ----------------------------------------------------------------------------
 // pre-passes
 // ----------------------------------------------------------------------------
-// Logit a = g_a <q_i, k_j> / sqrt(dh) of edge (i, j) for this lane's head.
-__device__ __forceinline__ float stats_logit(const StatsParams& P, int i, int j, const float* wcol,
-                                             const float4* q4, int d4, int h, int dh, float inv) {
-    const float3 r = edge_vec(P.pos, i, j, P.box);
-    const float d = sqrtf(r.x * r.x + r.y * r.y + r.z * r.z);
-    float rr[kTcMaxRbf];
-    rbf_all<kTcMaxRbf>(d, P.cutoff, P.n_rbf, rr);
-    float ga = 0.f;
-#pragma unroll
-    for (int kb = 0; kb < kTcMaxRbf; ++kb) ga = fmaf(rr[kb], wcol[kb], ga);
-    const float4* k4 = reinterpret_cast<const float4*>(P.k + (size_t)j * P.C + h * dh);
-    float dot = 0.f;
-    for (int c4 = 0; c4 < d4; ++c4) {
-        const float4 qa = __ldg(q4 + c4), kv = __ldg(k4 + c4);
-        dot = fmaf(qa.x, kv.x, dot);
-        dot = fmaf(qa.y, kv.y, dot);
-        dot = fmaf(qa.z, kv.z, dot);
-        dot = fmaf(qa.w, kv.w, dot);
-    }
-    return ga * dot * inv;
-}
-// Logits of a lane are evaluated kStatsB at a time, independently (so that their
-// gathers overlap), and merged into the running (max, sum) once per batch.
-constexpr int kStatsB = 4;
-__device__ __forceinline__ void stats_merge(const float (&a)[kStatsB], float& m, float& s) {
-    float mb = m;
-#pragma unroll
-    for (int u = 0; u < kStatsB; ++u) mb = fmaxf(mb, a[u]);
-    if (mb == -INFINITY) return;  // no edge yet
-    float sb = (m == -INFINITY) ? 0.f : s * expf(m - mb);
-#pragma unroll
-    for (int u = 0; u < kStatsB; ++u) sb += (a[u] == -INFINITY) ? 0.f : expf(a[u] - mb);
-    m = mb;
-    s = sb;
-}
 // Softmax statistics per node and head, lse = m + log(sum exp(a - m)), by an
 // online max/sum over the node's edges. One warp per node; lane = (edge slot
 // es, head h) with 32 / H edge slots, so a head's q and logit-gate column
@@ -130,14 +95,28 @@ __global__ void __launch_bounds__(256) k_softmax_stats(StatsParams P) {
     const int d4 = dh / 4;
     float m = -INFINITY, s = 0.f;
     const int e0 = P.row_ptr[i], e1 = P.row_ptr[i + 1];
-    for (int eb = e0 + es; eb < e1; eb += EP * kStatsB) {
-        float a[kStatsB];
+    for (int e = e0 + es; e < e1; e += EP) {
+        const int j = P.col[e];
+        const float3 r = edge_vec(P.pos, i, j, P.box);
+        const float d = sqrtf(r.x * r.x + r.y * r.y + r.z * r.z);
+        float rr[kTcMaxRbf];
+        rbf_all<kTcMaxRbf>(d, P.cutoff, P.n_rbf, rr);
+        float ga = 0.f;
 #pragma unroll
-        for (int u = 0; u < kStatsB; ++u) {
-            const int e = eb + u * EP;
-            a[u] = e < e1 ? stats_logit(P, i, P.col[e], wcol, q4, d4, h, dh, inv) : -INFINITY;
+        for (int kb = 0; kb < kTcMaxRbf; ++kb) ga = fmaf(rr[kb], wcol[kb], ga);
+        const float4* k4 = reinterpret_cast<const float4*>(P.k + (size_t)j * C + h * dh);
+        float dot = 0.f;
+        for (int c4 = 0; c4 < d4; ++c4) {
+            const float4 qa = __ldg(q4 + c4), kv = __ldg(k4 + c4);
+            dot = fmaf(qa.x, kv.x, dot);
+            dot = fmaf(qa.y, kv.y, dot);
+            dot = fmaf(qa.z, kv.z, dot);
+            dot = fmaf(qa.w, kv.w, dot);
         }
-        stats_merge(a, m, s);
+        const float a = ga * dot * inv;
+        const float mn = fmaxf(m, a);
+        s = s * expf(m - mn) + expf(a - mn);
+        m = mn;
     }
     // combine the edge slots of each head
     for (int o = H; o < 32; o <<= 1) {
@@ -184,14 +163,28 @@ __global__ void __launch_bounds__(256) k_softmax_stats_cells(StatsParams P, Cell
             0, s);
         __syncwarp();
         const int n_here = min(cnt - w0, kStatsCap);
-        for (int kb0 = es; kb0 < n_here; kb0 += EP * kStatsB) {
-            float a[kStatsB];
+        for (int k = es; k < n_here; k += EP) {
+            const int j = jb[k];
+            const float3 r = edge_vec(P.pos, i, j, P.box);
+            const float d = sqrtf(r.x * r.x + r.y * r.y + r.z * r.z);
+            float rr[kTcMaxRbf];
+            rbf_all<kTcMaxRbf>(d, P.cutoff, P.n_rbf, rr);
+            float ga = 0.f;
 #pragma unroll
-            for (int u = 0; u < kStatsB; ++u) {
-                const int k = kb0 + u * EP;
-                a[u] = k < n_here ? stats_logit(P, i, jb[k], wcol, q4, d4, h, dh, inv) : -INFINITY;
+            for (int kb = 0; kb < kTcMaxRbf; ++kb) ga = fmaf(rr[kb], wcol[kb], ga);
+            const float4* k4 = reinterpret_cast<const float4*>(P.k + (size_t)j * C + h * dh);
+            float dot = 0.f;
+            for (int c4 = 0; c4 < d4; ++c4) {
+                const float4 qa = __ldg(q4 + c4), kv = __ldg(k4 + c4);
+                dot = fmaf(qa.x, kv.x, dot);
+                dot = fmaf(qa.y, kv.y, dot);
+                dot = fmaf(qa.z, kv.z, dot);
+                dot = fmaf(qa.w, kv.w, dot);
             }
-            stats_merge(a, m, sum);
+            const float a = ga * dot * inv;
+            const float mn = fmaxf(m, a);
+            sum = sum * expf(m - mn) + expf(a - mn);
+            m = mn;
         }
         __syncwarp();
         if (cnt <= w0 + kStatsCap) break;
