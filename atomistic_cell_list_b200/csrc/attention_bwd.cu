@@ -1333,7 +1333,10 @@ cudaError_t launch_ops(const BwdParams& P, int e0, int ne, __half* Xo, __half* Y
 
 // cuBLAS, loaded at run time (the library links no BLAS; the host process
 // normally has it loaded already). One handle per CUDA context, found by the
-// context's unique id, so a handle is never used in another context.
+// context's unique id, so a handle is never used in another context. Handles
+// live until the process ends (a destroyed context's entry is never found
+// again); the stream is set on the handle per call, so concurrent calls on
+// one context from several host threads must be serialised by the caller.
 struct CublasRt {
     decltype(&cublasCreate_v2) create = nullptr;
     decltype(&cublasSetStream_v2) set_stream = nullptr;

@@ -376,7 +376,9 @@ e2f_status e2f_onfly_attention_cells_skin(const e2f_attn_cfg* cfg,
  *               gradient) are built once per chunk of 131,072 edges in the
  *               workspace, and each block's gradient is a GEMM over the
  *               chunk's edges, run by cuBLAS (loaded at run time; absent
- *               cuBLAS gives E2F_ERR_CUDA).
+ *               cuBLAS gives E2F_ERR_CUDA). One cuBLAS handle serves each
+ *               CUDA context, so calls from several host threads at once
+ *               on one context must be serialised by the caller.
  *   workspace   device, >= e2f_attention_backward_workspace_size(...)
  *               bytes, 256-byte aligned. Its status word (a bounded
  *               device-side wait that ran out: E2F_ERR_TIMEOUT) is read
