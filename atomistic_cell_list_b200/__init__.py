@@ -38,6 +38,11 @@ class e2f_attn_cfg(ctypes.Structure):
                 ("cutoff", ctypes.c_float), ("feat_dtype", ctypes.c_int), ("m_max", ctypes.c_int)]
 
 
+class e2f_sixj_cfg(ctypes.Structure):
+    _fields_ = [("L", ctypes.c_int), ("Lf", ctypes.c_int), ("C", ctypes.c_int), ("H", ctypes.c_int),
+                ("n_rbf", ctypes.c_int), ("cutoff", ctypes.c_float)]
+
+
 _lib = None
 _vp, _i64, _sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t
 
@@ -71,6 +76,10 @@ _SIGS = {
     "e2f_attention_set_debug": (None, [ctypes.c_int, ctypes.c_int, ctypes.c_int]),
     "e2f_attention_debug_timers": (ctypes.c_int, [_vp, _sz, _i64, ctypes.POINTER(e2f_attn_cfg),
                                                   ctypes.POINTER(_i64), ctypes.c_int, _vp]),
+    "e2f_sixj_n_paths": (ctypes.c_int, [ctypes.c_int, ctypes.c_int]),
+    "e2f_sixj_workspace_size": (_sz, [_i64, ctypes.POINTER(e2f_sixj_cfg)]),
+    "e2f_sixj_attention": (ctypes.c_int, [ctypes.POINTER(e2f_sixj_cfg), _vp, _i64, _vp, ctypes.c_int32, _vp, _vp,
+                                          _i64, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
 }
 
 
@@ -381,6 +390,39 @@ def e2f_attention_set_debug(max_ctas: int = 0, timers: bool = False, drop_arrive
 
 def e2f_launch_count() -> int:
     return int(lib().e2f_launch_count())
+
+
+def make_sixj_cfg(L: int, Lf: int, C: int, H: int, n_rbf: int, cutoff: float) -> e2f_sixj_cfg:
+    return e2f_sixj_cfg(int(L), int(Lf), int(C), int(H), int(n_rbf), float(cutoff))
+
+
+def e2f_sixj_n_paths(L: int, Lf: int) -> int:
+    return int(lib().e2f_sixj_n_paths(int(L), int(Lf)))
+
+
+def e2f_sixj_workspace_size(n_atoms: int, cfg: e2f_sixj_cfg) -> int:
+    return int(lib().e2f_sixj_workspace_size(int(n_atoms), ctypes.byref(cfg)))
+
+
+def e2f_sixj_attention(cfg: e2f_sixj_cfg, pos, row_ptr, col, x, W_q, W_k, W_rad, w_path,
+                       graph_ptr: torch.Tensor | None = None, out: torch.Tensor | None = None,
+                       workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """out[N, (L+1)^2, C] fp32 = the Wigner-6j node-level convolution layer (see include/e2f.h)."""
+    _need_cuda(pos, row_ptr, col, x, W_q, W_k, W_rad, w_path, graph_ptr, out, workspace)
+    n = pos.shape[0]
+    if out is None:
+        out = torch.empty((n, (cfg.L + 1) ** 2, cfg.C), dtype=torch.float32, device=pos.device)
+    ws_bytes = e2f_sixj_workspace_size(n, cfg)
+    if ws_bytes == 0:
+        raise E2FError(2, "e2f_sixj_workspace_size")
+    if workspace is None or workspace.numel() < ws_bytes:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=pos.device)
+    n_graphs = 0 if graph_ptr is None else graph_ptr.numel() - 1
+    code = lib().e2f_sixj_attention(ctypes.byref(cfg), _ptr(pos), n, _ptr(graph_ptr), n_graphs, _ptr(row_ptr),
+                                    _ptr(col), col.numel(), _ptr(x), _ptr(W_q), _ptr(W_k), _ptr(W_rad),
+                                    _ptr(w_path), _ptr(out), _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(code, "e2f_sixj_attention")
+    return out
 
 
 # short aliases

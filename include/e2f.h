@@ -432,6 +432,83 @@ e2f_status e2f_edge_wigner_blocks(const float* r, int64_t n_edges, int L,
  * devices, all entry points); lets a caller count launches in a region. */
 int64_t e2f_launch_count(void);
 
+/* ------------------------------------------------------------------------
+ * Wigner-6j node-level convolution: the E2Former attention variant whose
+ * edge tensor product is moved onto the nodes (fugumt abstract page: EAAS
+ * starts from this convolution, which takes the work from O(|E|) to O(|V|);
+ * gist.science Technical Summary 3: EAAS joins Wigner-6j re-coupling with the
+ * SO(2) alignment). The pages print no formula. The layer computed here,
+ * open boundaries, r_ij = x_j - x_i:
+ *   S^l_m(r) = sqrt(4 pi/(2l+1)) |r|^l Y_lm(r/|r|)    regular solid harmonics
+ *              in the real basis of the main layer (S^0 = 1, S^1 = (y, z, x))
+ *   v_ij[l3,m3,c] = sum over paths (l1,l2,l3) of w_path[p][c]
+ *              sum_{m1,m2} Q^{l1l2l3}[m1,m2,m3] x_j[l1,m1,c] S^l2_m2(r_ij)
+ *   a_ij^h   = g_a^h <q_i^h, k_j^h> / sqrt(C/H),  g_a = rho(|r_ij|) W_rad,
+ *              rho and q, k as for e2f_onfly_attention
+ *   out_i[l,m,c] = sum_j softmax_j(a_ij^{h(c)}) v_ij[l,m,c]; 0 if N(i) is empty
+ * Q^{l1l2l3} is the real coupling tensor: with the unitary U_l taking the
+ * complex harmonics (Condon-Shortley phase) to the real ones (none),
+ *   Q[m1,m2,m3] = part of sum U3[m3,mu3] conj(U1[m1,mu1]) conj(U2[m2,mu2])
+ *                 <l1 mu1 l2 mu2 | l3 mu3>,
+ * the real part when l1+l2+l3 is even, the imaginary part when it is odd.
+ * Paths, packed in this order: l1 = 0..L, then l3 = 0..L, then
+ * l2 = |l1-l3| .. min(l1+l3, Lf); e2f_sixj_n_paths gives their count.
+ *
+ * The library never forms an edge tensor product: it expands S^l2(r_ij)
+ * around each graph's mean position o (addition theorem of solid
+ * harmonics), forms [x_j (x) S^lam(x_j - o)]^k per node, sums those with the
+ * softmax weights over the edges, and re-couples with S^mu(o - x_i) per node
+ * through the 6j symbols. The expansion's terms grow as (graph radius /
+ * neighbour distance)^Lf while their sum does not, so the node products,
+ * their sums and the tables are held in fp64 (inputs, logits and output are
+ * fp32). The cost per atom grows with the graph's spread, not its size: the
+ * layer is meant for molecules, not for extended systems (which also have no
+ * single origin under periodic images).
+ *
+ *   cfg        host; L (0..4), Lf (0..2L, highest l2), C (1..256), H
+ *              (1..32, divides C), n_rbf (2..32), cutoff > 0.
+ *   pos        device, float [N*3]; open boundaries.
+ *   graph_ptr  device, int32 [n_graphs+1] as for e2f_build_neighbors, or
+ *              NULL (one graph). Every CSR pair must join two atoms of one
+ *              graph (as e2f_build_neighbors lists them).
+ *   row_ptr, col  device CSR, rows in atom order, col entries in [0, N).
+ *   x          device, float [N, (L+1)^2, C].
+ *   W_q, W_k   device, float [C, C] row-major (as for e2f_onfly_attention).
+ *   W_rad      device, float [n_rbf, H] row-major: g_a = rho W_rad.
+ *   w_path     device, float [n_paths, C].
+ *   out        device, float [N, (L+1)^2, C], written.
+ *   workspace  device, >= e2f_sixj_workspace_size(...) bytes, 256-byte
+ *              aligned (0 from the size query means the shape is not
+ *              supported). Holds the coupling tables and, per atom, the node
+ *              products and their sums: 16 Z C + 8 C + 24 bytes, Z the number
+ *              of node product components that reach the output (895 at
+ *              L = 4, Lf = 8; 454 at L = 4, Lf = 4).
+ * Errors: E2F_ERR_INVALID_ARG (null pointer, negative size, workspace too
+ * small), E2F_ERR_UNSUPPORTED (shape outside the limits), E2F_ERR_ALIGNMENT,
+ * E2F_ERR_CUDA. The coupling tables are built on the host the first time a
+ * (L, Lf) is used and kept for the process. Asynchronous.
+ * ---------------------------------------------------------------------- */
+typedef struct {
+    int L;
+    int Lf;
+    int C;
+    int H;
+    int n_rbf;
+    float cutoff;
+} e2f_sixj_cfg;
+
+int e2f_sixj_n_paths(int L, int Lf);
+
+size_t e2f_sixj_workspace_size(int64_t n_atoms, const e2f_sixj_cfg* cfg);
+
+e2f_status e2f_sixj_attention(const e2f_sixj_cfg* cfg, const float* pos, int64_t n_atoms,
+                              const int32_t* graph_ptr, int32_t n_graphs,
+                              const int32_t* row_ptr, const int32_t* col,
+                              int64_t n_pairs, const float* x, const float* W_q,
+                              const float* W_k, const float* W_rad,
+                              const float* w_path, float* out, void* workspace,
+                              size_t ws_bytes, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

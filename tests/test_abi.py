@@ -168,3 +168,30 @@ def test_fused_traversal_argument_checks():
     assert fs(*sargs(1.0, 0)) == 1              # reuse of a workspace no rebuild was recorded for
     assert fs(*sargs(-0.5, 1)) == 1             # negative skin
     assert fs(*sargs(float("nan"), 1)) == 1
+
+
+def test_sixj_host_queries_and_argument_checks():
+    from oracle.sixj import sixj_paths
+    for L in range(5):
+        for Lf in range(2 * L + 1):
+            assert e2f.e2f_sixj_n_paths(L, Lf) == len(sixj_paths(L, Lf))
+    assert e2f.e2f_sixj_n_paths(2, 5) == -1 and e2f.e2f_sixj_n_paths(5, 2) == -1
+    ok = e2f.make_sixj_cfg(4, 8, 64, 8, 16, 5.0)
+    assert e2f.e2f_sixj_workspace_size(10000, ok) > 16 * 895 * 64 * 10000
+    for bad in [e2f.make_sixj_cfg(2, 5, 16, 1, 16, 5.0), e2f.make_sixj_cfg(5, 2, 16, 1, 16, 5.0),
+                e2f.make_sixj_cfg(2, 2, 16, 3, 16, 5.0), e2f.make_sixj_cfg(2, 2, 512, 1, 16, 5.0),
+                e2f.make_sixj_cfg(2, 2, 16, 1, 1, 5.0), e2f.make_sixj_cfg(2, 2, 16, 1, 16, 0.0)]:
+        assert e2f.e2f_sixj_workspace_size(10, bad) == 0
+    cfg = e2f.make_sixj_cfg(2, 4, 16, 1, 16, 5.0)
+    need = e2f.e2f_sixj_workspace_size(4, cfg)
+    v = lambda p: None if p is None else ctypes.c_void_p(p)
+
+    def call(pos=16, n=4, gp=None, ng=0, rp=16, col=16, npairs=4, ws=256, wsb=need):
+        return e2f.lib().e2f_sixj_attention(ctypes.byref(cfg), v(pos), n, v(gp), ng, v(rp), v(col), npairs, v(16),
+                                            v(16), v(16), v(16), v(16), v(16), v(ws), wsb, None)
+    assert call(pos=None) == 1
+    assert call(npairs=-1) == 1
+    assert call(gp=16, ng=0) == 1
+    assert call(ws=128) == 4
+    assert call(wsb=need - 1) == 1
+    assert call(n=0) == 0

@@ -153,3 +153,40 @@ def test_catches_radial_basis_without_envelope_or_with_wrong_width(monkeypatch):
         monkeypatch.setattr(layer_mod, "radial_basis", bad)
         monkeypatch.setattr(T, "radial_basis", bad)
         _fails(T.test_radial_basis_special_points)
+
+
+# --- the Wigner-6j node-level convolution oracle (oracle/sixj.py) ---
+
+def test_catches_sign_flipped_odd_couplings_in_the_6j_layer(monkeypatch):
+    import oracle.sixj as sixj_mod
+    import test_oracle_sixj as X
+    good = sixj_mod.real_cg
+    monkeypatch.setattr(sixj_mod, "real_cg", lambda a, b, c: -good(a, b, c) if (a + b + c) % 2 else good(a, b, c))
+    X.test_sixj_layer_rotation_equivariance_and_translation_invariance()  # still equivariant ...
+    _fails(X.test_sixj_layer_equals_a_node_split_evaluation)             # ... but not the same layer
+
+
+def test_catches_condon_shortley_phase_in_solid_harmonics(monkeypatch):
+    import oracle.sixj as sixj_mod
+    import test_oracle_sixj as X
+    good = sixj_mod.real_sh
+
+    def with_phase(lmax, v):
+        Y = good(lmax, v).copy()
+        for l in range(lmax + 1):
+            for m in range(1, l + 1, 2):
+                Y[..., l * l + l + m] *= -1
+                Y[..., l * l + l - m] *= -1
+        return Y
+    monkeypatch.setattr(sixj_mod, "real_sh", with_phase)
+    _fails(X.test_solid_harmonics_closed_forms_l_le_2)
+
+
+def test_catches_a_wrong_triangle_coefficient_in_the_6j_symbol(monkeypatch):
+    from fractions import Fraction
+    from math import factorial as f
+
+    import oracle.sixj as sixj_mod
+    import test_oracle_sixj as X
+    monkeypatch.setattr(sixj_mod, "_delta", lambda a, b, c: Fraction(f(a + b - c) * f(a - b + c) * f(-a + b + c)))
+    _fails(X.test_6j_matches_sympy)

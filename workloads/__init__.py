@@ -373,3 +373,15 @@ def make_weights(cfg_id: int, L: int, C: int, H: int, n_rbf: int, dtype: str,
     n = sum(so2_block_sizes(L, C))
     W, Wf = round_to_dtype(rng.normal(size=n) * s, dtype)
     return Weights(Wq, Wk, Wrad, W, Wf)
+
+
+def make_sixj_weights(seed: int, C: int, H: int, n_rbf: int, n_paths: int):
+    """Weights of the Wigner-6j node-level convolution layer, float32:
+    W_q, W_k [C, C], W_rad [n_rbf, H] (logit gates), w_path [n_paths, C]."""
+    rng = np.random.default_rng(4000 + seed)
+    s = 1.0 / math.sqrt(C)
+    Wq = (rng.normal(size=(C, C)) * s).astype(np.float32)
+    Wk = (rng.normal(size=(C, C)) * s).astype(np.float32)
+    Wrad = rng.normal(size=(n_rbf, H)).astype(np.float32)
+    w_path = (rng.normal(size=(n_paths, C)) * 0.3).astype(np.float32)
+    return Wq, Wk, Wrad, w_path
