@@ -494,6 +494,10 @@ def run_ours(args):
         for c in (2, 3, 4, 5):
             line["per_config"][f"cfg{c}"] = measure_config(c, dev, 3, 2, flush, peaks)
         line["backward"] = backward_record(args.config, dev, 2, peaks)
+        try:
+            line["sixj"] = sixj_record(dev, 3)
+        except Exception as err:  # a record of a variant, never a reason to lose the bench line
+            line["sixj"] = {"error": f"{type(err).__name__}: {err}"}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = oracle_rate(args.config, float(os.environ.get("E2F_CPU_BUDGET_S", "15")))
     if rank == 0:
@@ -632,6 +636,48 @@ def backward_record(cfg_id, dev, steps, peaks):
     return {"workload": workload_desc(w)["workload"], "n_pairs": E, "ms": ms, "pairs_per_s": E / (ms * 1e-3),
             "tflops": tflops, "frac": tflops / peak, "peak": peak,
             "units": f"{E} edges x 3 x {F} SO(2) FLOP (all gradients)", "steps": steps}
+
+
+def sixj_record(dev, steps):
+    """The Wigner-6j node-level convolution variant (e2f_sixj_attention) on the
+    batch of 256 molecule graphs, L = 4, Lf = 4, C = 64, H = 8, fp32 features:
+    ms per call with inputs resident, pairs/s, and the workspace it needs."""
+    import torch
+
+    import atomistic_cell_list_b200 as e2f
+    import workloads as W
+
+    w = W.load_workload(2)
+    L, Lf, C, H, n_rbf = 4, 4, 64, 8, 16
+    n = w.n_atoms
+    xs, _ = W.make_features(100, n, L, C, "f32")
+    Wq, Wk, Wrad, wp = W.make_sixj_weights(0, C, H, n_rbf, e2f.e2f_sixj_n_paths(L, Lf))
+
+    def dt(a):
+        return torch.from_numpy(np.ascontiguousarray(a, np.float32)).to(dev)
+
+    pos, gp = dt(w.pos), torch.from_numpy(w.graph_ptr).to(dev)
+    rp, col = e2f.e2f_build_neighbors(pos, None, w.cutoff, gp)
+    cfg = e2f.make_sixj_cfg(L, Lf, C, H, n_rbf, w.cutoff)
+    ws = torch.empty(e2f.e2f_sixj_workspace_size(n, cfg), dtype=torch.uint8, device=dev)
+    args = (cfg, pos, rp, col, dt(xs).reshape(n, (L + 1) ** 2, C), dt(Wq), dt(Wk), dt(Wrad), dt(wp))
+    out = e2f.e2f_sixj_attention(*args, graph_ptr=gp, workspace=ws)
+    torch.cuda.synchronize(dev)
+    ts = []
+    for _ in range(steps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        e2f.e2f_sixj_attention(*args, graph_ptr=gp, workspace=ws, out=out)
+        b.record()
+        torch.cuda.synchronize(dev)
+        ts.append(a.elapsed_time(b))
+    ms = statistics.mean(ts)
+    E = int(col.numel())
+    rec = {"workload": "256 molecule graphs, 20-60 atoms", "n_atoms": n, "n_pairs": E, "L": L, "Lf": Lf, "C": C,
+           "H": H, "ms": ms, "pairs_per_s": E / (ms * 1e-3), "workspace_bytes": int(ws.numel()), "steps": steps}
+    del ws, out
+    torch.cuda.empty_cache()
+    return rec
 
 
 def run_slab(args):
