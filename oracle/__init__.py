@@ -26,4 +26,6 @@ Modules:
   neighbors  the exact fp32 cutoff predicate, brute force and KD-tree search
   grad       the same layer in plain PyTorch fp64, differentiated by autograd
              (gradients for the backward pass)
+  sixj       the Wigner-6j node-level convolution variant, edge by edge, and
+             Racah's 6j formula (for the pins)
 """
