@@ -486,7 +486,10 @@ int64_t e2f_launch_count(void);
  * Errors: E2F_ERR_INVALID_ARG (null pointer, negative size, workspace too
  * small), E2F_ERR_UNSUPPORTED (shape outside the limits), E2F_ERR_ALIGNMENT,
  * E2F_ERR_CUDA. The coupling tables are built on the host the first time a
- * (L, Lf) is used and kept for the process. Asynchronous.
+ * (L, Lf) is used and kept for the process; every call copies them from
+ * that pageable host memory into the workspace on `stream` (the driver
+ * stages such a copy before the call returns), so the call cannot be
+ * captured into a CUDA graph. Otherwise asynchronous.
  * ---------------------------------------------------------------------- */
 typedef struct {
     int L;
