@@ -190,3 +190,24 @@ def test_catches_a_wrong_triangle_coefficient_in_the_6j_symbol(monkeypatch):
     import test_oracle_sixj as X
     monkeypatch.setattr(sixj_mod, "_delta", lambda a, b, c: Fraction(f(a + b - c) * f(a - b + c) * f(-a + b + c)))
     _fails(X.test_6j_matches_sympy)
+
+
+def test_catches_interleaved_heads_in_the_6j_layer(monkeypatch):
+    # channel c must take the softmax of head c // (C/H); a plausible slip
+    # assigns head c % H instead
+    import oracle.sixj as sixj_mod
+    import test_oracle_sixj as X
+
+    real_repeat = np.repeat
+
+    class _NP:
+        def __getattr__(self, name):
+            return getattr(np, name)
+
+        @staticmethod
+        def repeat(a, r, axis=None):
+            if axis == 1:
+                return np.tile(a, (1, r))
+            return real_repeat(a, r, axis=axis)
+    monkeypatch.setattr(sixj_mod, "np", _NP())
+    _fails(X.test_sixj_layer_equals_a_node_split_evaluation)
